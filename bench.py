@@ -1,0 +1,449 @@
+#!/usr/bin/env python
+"""Throughput of the fused MoE expert forward on B200.
+
+Default workload: the Qwen3-235B-shaped MoE layer, bf16, H=4096, I=1536,
+E=128, top_k=8, T=4096 tokens, packed w13 [E, 2I, H] read through its
+expert-strided gate/up views (Liger-Kernel PR #1377).  One step is one full
+forward (align -> permute -> GEMM1+SwiGLU -> GEMM2+weight -> combine) over one
+batch of T tokens, inputs resident in HBM; the L2 is flushed (512 MB write)
+before every timed step, outside the timed events.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload qwen3-235b|glm45-air|tiny] [--T T] [--sweep FILE]
+
+Multi-GPU runs (torchrun, one process per GPU) are independent replicas: each
+rank runs the same layer on its own batch, no collective on the data path
+(weak scaling); timing is the max over ranks.  The reference arm times the
+fp64 CPU oracle on the host cores on a bounded token sample of the same
+workload.  Prints one JSON line (rank 0).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "fused-MoE layer tokens/s (us/call) on 1 B200"
+UNIT = "tokens/s"
+
+WORKLOADS = {
+    "qwen3-235b": dict(H=4096, I=1536, E=128, k=8, T=4096, routing="softmax"),
+    "glm45-air": dict(H=4096, I=1408, E=128, k=8, T=16384, routing="zipf-layer-slice"),
+    "tiny": dict(H=256, I=128, E=8, k=2, T=64, routing="softmax"),
+}
+
+# DRAM traffic per launch of the dominant kernel from an ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), keyed to the hash of the kernel
+# source it was taken on; reported as null once the source has changed.
+NCU_TRAFFIC = {}
+
+
+def kernel_src_hash() -> str:
+    h = hashlib.sha256()
+    for fn in ("moe_gemm_bf16.cu", "moe_common.cuh"):
+        with open(os.path.join(ROOT, "mixture_experts_layer_46_b200", "csrc", fn), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def workload_name(w) -> str:
+    return (f"moe-layer bf16 T={w['T']} H={w['H']} I={w['I']} E={w['E']} top_k={w['k']} "
+            f"packed-strided-w13 routing={w['routing']}")
+
+
+def make_inputs(w, device, seed_offset=0):
+    from mixture_experts_layer_46_b200 import workloads as wl
+
+    w13, w2 = wl.make_weights_bf16(w["E"], w["I"], w["H"], seed=0, device=device)
+    x = wl.make_x(w["T"], w["H"], seed=1 + seed_offset, device=device)
+    if w["routing"] == "softmax":
+        ids, wts = wl.route_softmax_topk(w["T"], w["E"], w["k"], seed=2 + seed_offset, device=device)
+        keep = None
+    else:
+        ids_all, w_all = wl.route_zipf_layers(w["T"], w["E"], w["k"], layers=46, seed=7 + seed_offset,
+                                              device=device)
+        ids, wts = ids_all[:, 23, :], w_all[:, 23, :]
+        keep = (ids_all, w_all)
+    return {"x": x, "w13": w13, "w2": w2, "ids": ids, "wts": wts, "keep": keep}
+
+
+def algorithmic(w, ids):
+    """Algorithmic FLOPs and bytes of one forward and of GEMM1 alone."""
+    H, I, E, k, T = w["H"], w["I"], w["E"], w["k"], w["T"]
+    idc = ids.reshape(-1).long()
+    valid = idc[(idc >= 0) & (idc < E)]
+    n_slots = int(valid.numel())
+    n_act = int(torch.unique(valid).numel())
+    flops = 6.0 * H * I * n_slots
+    bytes_total = 3.0 * I * H * 2 * n_act + 2.0 * T * H * 2 + 8.0 * T * k
+    g1_flops = 4.0 * H * I * n_slots
+    g1_bytes = 2.0 * I * H * 2 * n_act + T * H * 2.0
+    return dict(flops=flops, bytes=bytes_total, gemm1_flops=g1_flops, gemm1_bytes=g1_bytes,
+                slots=n_slots, active_experts=n_act)
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.lines = []
+        self.dev = device_index
+
+    def start(self):
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            sel = []
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", *sel, "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def oracle_tokens_per_s(inp, w, budget_s, cores):
+    """The fp64 oracle on a bounded sample of the workload's tokens."""
+    import oracle
+    from mixture_experts_layer_46_b200 import workloads as wl
+
+    cpu = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    if inp["keep"] is not None:
+        ids_all, w_all = (t.cpu() for t in inp["keep"])
+        cpu["ids"], cpu["wts"] = ids_all[:, 23, :], w_all[:, 23, :]
+    gate, up = wl.gate_up_views(cpu["w13"])
+    g = torch.Generator().manual_seed(123)
+    order = torch.randperm(w["T"], generator=g)
+    # calibrate with one token per core, then size the sample to the budget
+    n = max(1, cores)
+    t0 = time.perf_counter()
+    oracle.moe_forward(cpu["x"], gate, up, cpu["w2"], cpu["ids"], cpu["wts"], tokens=order[:n],
+                       nthreads=cores)
+    dt = time.perf_counter() - t0
+    reps = max(1, int(budget_s / max(dt, 1e-6)))
+    n2 = min(w["T"], n * reps)
+    t0 = time.perf_counter()
+    oracle.moe_forward(cpu["x"], gate, up, cpu["w2"], cpu["ids"], cpu["wts"], tokens=order[:n2],
+                       nthreads=cores)
+    dt2 = time.perf_counter() - t0
+    return n2 / dt2, n2, dt2, (cpu, gate, up, order)
+
+
+def run_reference(args, w, rank):
+    if rank != 0:
+        return
+    import oracle
+
+    cores = os.cpu_count() or 1
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = make_inputs(w, dev)
+    _, _, _, (cpu, gate, up, order) = oracle_tokens_per_s(inp, w, 0.0, cores)
+    per_step_budget = max(0.5, 150.0 / max(1, args.steps + args.warmup))
+    # tokens per step: one per core, grown while it fits the per-step budget
+    t0 = time.perf_counter()
+    oracle.moe_forward(cpu["x"], gate, up, cpu["w2"], cpu["ids"], cpu["wts"], tokens=order[:cores],
+                       nthreads=cores)
+    dt = time.perf_counter() - t0
+    n = max(1, min(w["T"], int(cores * max(1.0, per_step_budget / max(dt, 1e-6)))))
+    times = []
+    for step in range(args.warmup + args.steps):
+        toks = order[(step * n) % w["T"]:][:n]
+        if toks.numel() < n:
+            toks = order[:n]
+        t0 = time.perf_counter()
+        oracle.moe_forward(cpu["x"], gate, up, cpu["w2"], cpu["ids"], cpu["wts"], tokens=toks,
+                           nthreads=cores)
+        if step >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    sec = sum(times) / len(times)
+    value = n / sec
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,1) activations, N(0,1/sqrt(fan_in)) weights)",
+            "config": {"workload": workload_name(w), "tokens_per_step_sample": n,
+                       "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.max_threads() if cores <= 0 else cores,
+                             "kind": "oracle",
+                             "sample": f"{n} of {w['T']} tokens per step (all their {w['k']} slots), fp64 C++ loop, OpenMP over tokens"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="qwen3-235b", choices=sorted(WORKLOADS))
+    ap.add_argument("--T", type=int, default=None)
+    ap.add_argument("--sweep", default=None, help="write a token-sweep JSONL here (extra lines)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    w = dict(WORKLOADS[args.workload])
+    if args.T is not None:
+        w["T"] = args.T
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = False
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        pg = True
+
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        if pg:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+        return
+
+    import mixture_experts_layer_46_b200 as moe
+    from mixture_experts_layer_46_b200 import workloads as wl
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    inp = make_inputs(w, dev)
+    v13 = moe.w13_from_packed(inp["w13"])
+    ws = torch.empty(moe.workspace_bytes(w["T"], w["H"], w["I"], w["E"], w["k"]), dtype=torch.uint8,
+                     device=dev)
+    out = torch.empty(w["T"], w["H"], dtype=torch.bfloat16, device=dev)
+    flush = wl.l2_flush_buffer(dev)
+
+    def step():
+        moe.forward(inp["x"], v13, inp["w2"], inp["ids"], inp["wts"], out=out, workspace=ws,
+                    stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    launches_per_step = moe.last_launch_count()
+    torch.cuda.synchronize(dev)
+
+    # ---------------------------------------------------------------- timed region
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    if pg:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.fill_(i & 0xff)
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    if pg:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    per = [a.elapsed_time(b) for a, b in evs]
+    ms = sum(per) / len(per)
+    if pg:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    value = world * w["T"] / (ms * 1e-3)
+
+    # ---------------------------------------------------------------- per-step breakdown
+    moe.profile_enable(True)
+    brk = {}
+    nb = min(args.steps, 20)
+    for i in range(nb):
+        flush.fill_(i & 0xff)
+        step()
+        for kname, kms in moe.profile_read().items():
+            brk[kname] = brk.get(kname, 0.0) + kms / nb
+    moe.profile_enable(False)
+
+    # ---------------------------------------------------------------- end to end (host buffers)
+    x_h = inp["x"].cpu().pin_memory()
+    ids_h = inp["ids"].contiguous().cpu().pin_memory()
+    w_h = inp["wts"].contiguous().cpu().pin_memory()
+    out_h = torch.empty(w["T"], w["H"], dtype=torch.bfloat16).pin_memory()
+    for _ in range(2):
+        moe.forward_host(x_h, v13, inp["w2"], ids_h, w_h, out_h, stream=stream)
+    e2e_ms = []
+    for i in range(min(args.steps, 50)):
+        flush.fill_(i & 0xff)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        moe.forward_host(x_h, v13, inp["w2"], ids_h, w_h, out_h, stream=stream)
+        e1.record(stream)
+        e1.synchronize()
+        e2e_ms.append(e0.elapsed_time(e1))
+    e2e = sum(e2e_ms) / len(e2e_ms)
+    if pg:
+        t = torch.tensor([e2e], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e = float(t.item())
+    h2d = x_h.numel() * 2 + ids_h.numel() * ids_h.element_size() + w_h.numel() * 4
+    d2h = out_h.numel() * 2
+
+    # ---------------------------------------------------------------- roofline
+    hbm, tf_burst, tf_sus, src = peaks()
+    alg = algorithmic(w, inp["ids"])
+    g1_ms = brk.get("gemm1_swiglu", float("nan"))
+    t_tc = alg["gemm1_flops"] / (tf_burst * 1e12)
+    t_mem = alg["gemm1_bytes"] / (hbm * 1e9)
+    if t_tc >= t_mem:
+        roof = {"bound": "tensor", "achieved": alg["gemm1_flops"] / (g1_ms * 1e-3) / 1e12,
+                "peak": tf_burst, "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": alg["gemm1_bytes"] / (g1_ms * 1e-3) / 1e9, "peak": hbm,
+                "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    tr = NCU_TRAFFIC.get("gemm1_swiglu")
+    roof["traffic"] = tr["bytes_per_launch"] if tr and tr.get("src") == kernel_src_hash() else None
+    roof["kernel"] = "gemm1_swiglu (grouped gate/up GEMM + SwiGLU, tcgen05)"
+    roof["peak_source"] = f"{src} (MEASURED_PEAKS.json burst)" if src == "measured" else "fallback"
+    t_roof_layer = max(alg["flops"] / (tf_burst * 1e12), alg["bytes"] / (hbm * 1e9))
+    layer_frac = t_roof_layer / (ms * 1e-3)
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) activations, N(0,1/sqrt(fan_in)) random-init weights)",
+            "config": {"workload": workload_name(w), "tokens_per_gpu": w["T"],
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "flushed (512 MB write) before every timed step, outside the events",
+                       "us_per_call": ms * 1e3,
+                       "us_per_call_p10": sorted(per)[len(per) // 10] * 1e3,
+                       "us_per_call_p90": sorted(per)[(9 * len(per)) // 10] * 1e3},
+            "roofline": roof,
+            "layer_roofline": {"t_roof_us": t_roof_layer * 1e6, "frac": layer_frac,
+                               "flops": alg["flops"], "bytes": alg["bytes"],
+                               "active_experts": alg["active_experts"]},
+            "step_breakdown_ms": brk,
+            "e2e": {"value": world * w["T"] / (e2e * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e,
+                    "api": "moe_forward_host (pinned host x/ids/weights in, host out)"},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cores = os.cpu_count() or 1
+        tps, n, dt, _ = oracle_tokens_per_s(inp, w, 12.0, cores)
+        line["cpu_baseline"] = {"value": tps, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": f"{n} of {w['T']} tokens (all their slots) in {dt:.1f} s, fp64 C++ loop, OpenMP over tokens"}
+
+    if args.sweep and rank == 0:
+        sweep(args, w, moe, wl, dev, stream, flush)
+
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def sweep(args, w, moe, wl, dev, stream, flush):
+    """Token sweep on the same weights (fresh routing per T): one JSONL row per T."""
+    hbm, tf_burst, _, _ = peaks()
+    w13, w2 = wl.make_weights_bf16(w["E"], w["I"], w["H"], seed=0, device=dev)
+    v13 = moe.w13_from_packed(w13)
+    with open(args.sweep, "w") as f:
+        for T in wl.TOKEN_SWEEP:
+            wt = dict(w, T=T)
+            x = wl.make_x(T, w["H"], seed=2000 + T, device=dev)
+            ids, wts = wl.route_softmax_topk(T, w["E"], w["k"], seed=1000 + T, device=dev)
+            ws = torch.empty(moe.workspace_bytes(T, w["H"], w["I"], w["E"], w["k"]), dtype=torch.uint8,
+                             device=dev)
+            out = torch.empty(T, w["H"], dtype=torch.bfloat16, device=dev)
+            for _ in range(5):
+                moe.forward(x, v13, w2, ids, wts, out=out, workspace=ws, stream=stream)
+            per = []
+            for i in range(30 if T < 8192 else 10):
+                flush.fill_(i & 0xff)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                moe.forward(x, v13, w2, ids, wts, out=out, workspace=ws, stream=stream)
+                b.record(stream)
+                torch.cuda.synchronize(dev)
+                per.append(a.elapsed_time(b))
+            med = statistics.median(per)
+            alg = algorithmic(wt, ids)
+            t_roof = max(alg["flops"] / (tf_burst * 1e12), alg["bytes"] / (hbm * 1e9))
+            row = {"T": T, "us_median": med * 1e3, "tokens_per_s": T / (med * 1e-3),
+                   "roofline_us": t_roof * 1e6, "frac": t_roof / (med * 1e-3),
+                   "hbm_GBs_alg": alg["bytes"] / (med * 1e-3) / 1e9,
+                   "tflops_alg": alg["flops"] / (med * 1e-3) / 1e12,
+                   "active_experts": alg["active_experts"]}
+            f.write(json.dumps(row) + "\n")
+            f.flush()
+            del ws, out
+
+
+if __name__ == "__main__":
+    main()

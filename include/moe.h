@@ -1,0 +1,197 @@
+/*
+ * moe.h — C ABI of the B200 (sm_100a) fused mixture-of-experts expert forward.
+ *
+ * The operation (per token t and routing column j, slot s = t*k + j):
+ *     e = topk_ids[t, j]        w = topk_weights[t, j]
+ *     g = x[t] . gate[e]^T      u = x[t] . up[e]^T          gate = w13[:, :I, :], up = w13[:, I:, :]
+ *     a = silu(g) * u           y = a . w2[e]^T
+ *     out[t] = sum_j w * y      (j = 0 .. k-1, in order)
+ * The packed w13 [E, 2I, H] layout and its expert-strided gate/up views are the
+ * subject of Liger-Kernel PR #1377 ("Problems"): each expert's first weight tile
+ * is located from the view's real stride(0), never from expert * I / TileN.
+ * The SiLU activation and the MXFP4 format (e2m1 values, one e8m0 scale per 32
+ * consecutive elements) follow ROCm/aiter PR #3859 ("Details").
+ *
+ * Conventions shared by every entry point:
+ *   - Every tensor is described by a moe_tensor_t: base pointer, dtype, sizes and
+ *     strides in elements of the storage type.  Any stride is honoured as given
+ *     (LightLLM issue #1467 and prime-rl PR #2860 show what goes wrong otherwise);
+ *     nothing is ever copied to make it contiguous.  Where the tensor-memory
+ *     copy engine cannot express a layout (weights with an inner stride other
+ *     than 1, or a base / outer stride that is not a multiple of 16 bytes) the
+ *     call returns MOE_ERR_UNSUPPORTED_LAYOUT.
+ *   - Device pointers unless the entry point says "host".  The caller owns every
+ *     buffer; the library keeps no pointer after a call returns, except as keys of
+ *     its descriptor cache.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *     and is asynchronous unless stated otherwise.
+ *   - Shape, dtype and layout errors are reported before anything is launched or
+ *     any descriptor is built (Liger-Kernel PR #1377, "Testing Done": mismatched
+ *     gate hidden dimensions fail before descriptor construction).
+ *   - No entry point aborts the process; every failure is a moe_status_t.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  MOE_BF16 = 0,   /* bfloat16 */
+  MOE_F32 = 1,    /* float32 */
+  MOE_I32 = 2,    /* int32 */
+  MOE_I64 = 3,    /* int64 */
+  MOE_E2M1X2 = 4  /* two FP4 e2m1 codes per byte, even logical element in the low nibble
+                     (torch.float4_e2m1fn_x2); sizes are LOGICAL elements, strides count bytes
+                     (so the innermost logical size is twice the innermost byte extent) */
+} moe_dtype_t;
+
+/* A strided tensor view.  For MOE_E2M1X2 tensors `scale` points at the e8m0
+ * scale codes (one byte per 32 logical elements of the innermost axis) and
+ * scale_strides gives their strides in bytes; the other dtypes ignore both. */
+typedef struct {
+  void* data;
+  int32_t dtype; /* moe_dtype_t */
+  int32_t ndim;
+  int64_t sizes[4];
+  int64_t strides[4];
+  void* scale;
+  int64_t scale_strides[4];
+} moe_tensor_t;
+
+/* The two input projections, each [E, I, H].  Usually expert-strided views of
+ * one packed w13 [E, 2I, H] (see moe_w13_from_packed); contiguous copies work
+ * the same way and give bit-identical results. */
+typedef struct {
+  moe_tensor_t gate;
+  moe_tensor_t up;
+} moe_w13_t;
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,        /* null pointer, negative size, ndim wrong */
+  MOE_ERR_SHAPE_MISMATCH = 2,     /* sizes disagree between tensors */
+  MOE_ERR_UNSUPPORTED_DTYPE = 3,  /* dtype not accepted for that argument */
+  MOE_ERR_UNSUPPORTED_LAYOUT = 4, /* stride/alignment the copy engine cannot express */
+  MOE_ERR_WORKSPACE_TOO_SMALL = 5,
+  MOE_ERR_CUDA = 6,               /* a CUDA runtime/driver call failed (see moe_last_cuda_error) */
+  MOE_ERR_NO_DEVICE = 7,          /* current device is not an sm_100 GPU */
+  MOE_ERR_DEVICE_TIMEOUT = 8      /* a kernel's bounded wait expired (see moe_get_device_errors) */
+} moe_status_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* moe_status_string(moe_status_t st);
+
+/* The last CUDA error string seen by the calling thread (static storage). */
+const char* moe_last_cuda_error(void);
+
+/* Split a packed w13 [E, 2I, H] view into its gate (rows [0, I)) and up
+ * (rows [I, 2I)) halves (Liger-Kernel PR #1377, "Problems").  Pure metadata: the
+ * up view's base is w13 + I * stride(1) storage elements (or the matching scale
+ * rows for MXFP4); both keep w13's stride(0), the real expert stride.
+ * Errors: MOE_ERR_INVALID_ARG (null, ndim != 3), MOE_ERR_SHAPE_MISMATCH (odd 2I). */
+moe_status_t moe_w13_from_packed(const moe_tensor_t* w13, moe_w13_t* out);
+
+/* Bytes of device workspace moe_forward_ws needs for T tokens, hidden H,
+ * intermediate I, E experts, top_k k and weight dtype wdtype (MOE_BF16 or
+ * MOE_E2M1X2).  Depends only on these scalars — never on the weights' strides or
+ * addresses — and does not grow with E*I*H (no weight-sized buffer is used;
+ * the pages' point is that the strided views replace a 0.375 GiB/layer copy).
+ * Returns 0 for invalid arguments. */
+size_t moe_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, int32_t wdtype);
+
+/* The fused MoE expert forward (all steps on the GPU, on `stream`).
+ *   x            [T, H]  bf16, any strides
+ *   w13          gate/up [E, I, H]: bf16, or MOE_E2M1X2 with e8m0 scales [E, I, H/32];
+ *                inner stride 1; base and stride(0), stride(1) multiples of 16 bytes
+ *   w2           [E, H, I]: same dtype and layout rules as w13
+ *   topk_ids     [T, k]  int32 or int64, any strides (e.g. the per-layer slice
+ *                [:, l, :] of a [T, layers, k] router-replay tensor, prime-rl PR #2860)
+ *   topk_weights [T, k]  float32, any strides; used as given (no renormalisation)
+ *   out          [T, H]  bf16, any strides; fully overwritten
+ *   workspace    device buffer of at least moe_workspace_bytes(...) bytes,
+ *                256-byte aligned; contents are scratch (not preserved)
+ * Ids outside [0, E) are skipped (contribute zero) and counted in a device
+ * counter read by moe_get_device_errors.  T = 0 is a no-op.  No allocation and
+ * no host synchronisation happen inside this call.  The combine over the k
+ * columns is in fixed order, so results are run-to-run deterministic and do not
+ * depend on the weights' strides.  In MXFP4 mode x and the SwiGLU activation are
+ * quantised on the fly with the 1x32 e8m0 rule of moe_quantize_mxfp4. */
+moe_status_t moe_forward_ws(const moe_tensor_t* x, const moe_w13_t* w13, const moe_tensor_t* w2,
+                            const moe_tensor_t* topk_ids, const moe_tensor_t* topk_weights,
+                            moe_tensor_t* out, void* workspace, size_t workspace_bytes,
+                            moe_stream_t stream);
+
+/* Same as moe_forward_ws with a library-owned workspace: one buffer per device,
+ * grown with cudaMalloc when a call needs more (growth synchronises the device,
+ * so size it once with a first call outside any stream capture). */
+moe_status_t moe_forward(const moe_tensor_t* x, const moe_w13_t* w13, const moe_tensor_t* w2,
+                         const moe_tensor_t* topk_ids, const moe_tensor_t* topk_weights,
+                         moe_tensor_t* out, moe_stream_t stream);
+
+/* End-to-end form for callers whose activations live in host memory: x,
+ * topk_ids, topk_weights and out are HOST tensors (pinned memory gives
+ * asynchronous copies; inner stride 1 is required for these four), the weights
+ * stay on the device.  Copies the inputs to the library workspace, runs the
+ * forward, copies `out` back and synchronises `stream` before returning. */
+moe_status_t moe_forward_host(const moe_tensor_t* x_host, const moe_w13_t* w13,
+                              const moe_tensor_t* w2, const moe_tensor_t* topk_ids_host,
+                              const moe_tensor_t* topk_weights_host, moe_tensor_t* out_host,
+                              moe_stream_t stream);
+
+/* Step "align" alone, for inspection and tests: group the T*k slots by expert.
+ *   counts[e]        number of valid slots routed to expert e          int32 [E]
+ *   offsets[e]       exclusive prefix sum of ceil(counts/block_m)*block_m int32 [E+1]
+ *   sorted_slots[p]  slot ids grouped by expert, ascending within an expert;
+ *                    padding positions hold the sentinel T*k            int32 [>= max_padded]
+ *   block_expert[b]  expert owning block_m-row block b                  int32 [>= max_padded/block_m]
+ *   num_blocks       number of blocks                                   int32 [1]
+ * max_padded = T*k + min(E, T*k)*(block_m-1); block_m in {16,32,64,128,256}.
+ * `workspace` as for moe_forward_ws (moe_workspace_bytes covers it). */
+moe_status_t moe_align(const moe_tensor_t* topk_ids, int64_t E, int32_t block_m, int32_t* counts,
+                       int32_t* offsets, int32_t* sorted_slots, int32_t* block_expert,
+                       int32_t* num_blocks, void* workspace, size_t workspace_bytes,
+                       moe_stream_t stream);
+
+/* MXFP4 quantisation of the rows of src [.., K] (bf16 or f32, inner stride 1,
+ * K % 32 == 0) into dst (MOE_E2M1X2 with dst->scale set): per 32 consecutive
+ * elements, scale exponent s = clamp(floor(log2(amax)) - 2, -127, 127) stored as
+ * the e8m0 code s + 127 (code 0 for an all-zero block), elements rounded to the
+ * nearest e2m1 value of v / 2^s with ties to even, saturating at +-6 (OCP MX
+ * v1.0; format named by aiter PR #3859, "Details").  src and dst have the same
+ * logical shape (ndim 2 or 3); dst's strides may be anything 1-byte aligned. */
+moe_status_t moe_quantize_mxfp4(const moe_tensor_t* src, moe_tensor_t* dst, moe_stream_t stream);
+
+/* Reads and clears the device error counters of the current device:
+ * *n_bad_ids = slots skipped because their id was outside [0, E);
+ * *timeouts = kernel waits that gave up.  Synchronises `stream`. */
+moe_status_t moe_get_device_errors(moe_stream_t stream, uint32_t* n_bad_ids, uint32_t* timeouts);
+
+/* Number of kernels the last moe_forward_ws / moe_forward call on this thread
+ * enqueued (for launch accounting). */
+int32_t moe_last_launch_count(void);
+
+/* Per-kernel timing for profiling.  While enabled on the calling thread, each
+ * moe_forward* call records a CUDA event on its stream before the first kernel
+ * and after each step (align, permute, GEMM1, GEMM2, combine); this serialises
+ * the steps (no overlap between neighbouring kernels), so time the end-to-end
+ * call with profiling off.  moe_profile_read synchronises on the last event and
+ * writes up to `capacity` step durations in milliseconds, in that order, for
+ * the last profiled call; *n receives the number of steps. */
+moe_status_t moe_profile_enable(int32_t on);
+moe_status_t moe_profile_read(float* ms, int32_t capacity, int32_t* n);
+
+/* Library version string. */
+const char* moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

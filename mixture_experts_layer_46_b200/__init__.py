@@ -1,0 +1,12 @@
+"""B200 (sm_100a) fused mixture-of-experts expert forward.
+
+The compute lives in libmoe_b200.so (C ABI: include/moe.h); this package is a
+thin ctypes binding over it plus seeded synthetic workloads.  Importing the
+package does not load the library; the first call does, and raises if the
+library was not built (there is no CPU fallback).
+"""
+
+from ._abi import (MoeError, MoeTensor, MoeW13, align, desc, device_errors, forward,  # noqa: F401
+                   forward_host, forward_status, last_launch_count, load, profile_enable,
+                   profile_read, quantize_mxfp4,
+                   version, w13_from_packed, w13_from_views, workspace_bytes)

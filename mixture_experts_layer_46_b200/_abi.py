@@ -1,0 +1,280 @@
+"""ctypes binding of libmoe_b200.so (include/moe.h).
+
+Argument marshalling only: torch tensors become moe_tensor_t descriptors
+(base pointer, dtype, sizes, strides) and every step of the forward runs in the
+library's CUDA kernels.  There is no fallback: if the shared library is missing
+or fails to load, every call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+MOE_BF16, MOE_F32, MOE_I32, MOE_I64, MOE_E2M1X2 = 0, 1, 2, 3, 4
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_SHAPE_MISMATCH",
+          3: "MOE_ERR_UNSUPPORTED_DTYPE", 4: "MOE_ERR_UNSUPPORTED_LAYOUT",
+          5: "MOE_ERR_WORKSPACE_TOO_SMALL", 6: "MOE_ERR_CUDA", 7: "MOE_ERR_NO_DEVICE",
+          8: "MOE_ERR_DEVICE_TIMEOUT"}
+
+# Names the header declares; tests check the library exports each of them.
+EXPORTS = ("moe_status_string", "moe_last_cuda_error", "moe_w13_from_packed",
+           "moe_workspace_bytes", "moe_forward_ws", "moe_forward", "moe_forward_host",
+           "moe_align", "moe_quantize_mxfp4", "moe_get_device_errors", "moe_last_launch_count",
+           "moe_profile_enable", "moe_profile_read", "moe_version")
+STEP_NAMES = ("align", "permute", "gemm1_swiglu", "gemm2_weighted", "combine")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str = ""):
+        self.status = status
+        msg = f"{where}: {STATUS.get(status, status)}"
+        if detail:
+            msg += f" ({detail})"
+        super().__init__(msg)
+
+
+class MoeTensor(ctypes.Structure):
+    _fields_ = [
+        ("data", ctypes.c_void_p),
+        ("dtype", ctypes.c_int32),
+        ("ndim", ctypes.c_int32),
+        ("sizes", ctypes.c_int64 * 4),
+        ("strides", ctypes.c_int64 * 4),
+        ("scale", ctypes.c_void_p),
+        ("scale_strides", ctypes.c_int64 * 4),
+    ]
+
+
+class MoeW13(ctypes.Structure):
+    _fields_ = [("gate", MoeTensor), ("up", MoeTensor)]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load the CUDA library (raises if it is not built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with `python -m mixture_experts_layer_46_b200.build`")
+            lib = ctypes.CDLL(LIB_PATH)
+            P = ctypes.POINTER
+            vp = ctypes.c_void_p
+            lib.moe_status_string.restype = ctypes.c_char_p
+            lib.moe_status_string.argtypes = [ctypes.c_int]
+            lib.moe_last_cuda_error.restype = ctypes.c_char_p
+            lib.moe_version.restype = ctypes.c_char_p
+            lib.moe_last_launch_count.restype = ctypes.c_int32
+            lib.moe_w13_from_packed.restype = ctypes.c_int
+            lib.moe_w13_from_packed.argtypes = [P(MoeTensor), P(MoeW13)]
+            lib.moe_workspace_bytes.restype = ctypes.c_size_t
+            lib.moe_workspace_bytes.argtypes = [ctypes.c_int64] * 5 + [ctypes.c_int32]
+            lib.moe_forward_ws.restype = ctypes.c_int
+            lib.moe_forward_ws.argtypes = [P(MoeTensor), P(MoeW13), P(MoeTensor), P(MoeTensor),
+                                           P(MoeTensor), P(MoeTensor), vp, ctypes.c_size_t, vp]
+            lib.moe_forward.restype = ctypes.c_int
+            lib.moe_forward.argtypes = [P(MoeTensor), P(MoeW13), P(MoeTensor), P(MoeTensor),
+                                        P(MoeTensor), P(MoeTensor), vp]
+            lib.moe_forward_host.restype = ctypes.c_int
+            lib.moe_forward_host.argtypes = lib.moe_forward.argtypes
+            lib.moe_align.restype = ctypes.c_int
+            lib.moe_align.argtypes = [P(MoeTensor), ctypes.c_int64, ctypes.c_int32, vp, vp, vp, vp,
+                                      vp, vp, ctypes.c_size_t, vp]
+            lib.moe_quantize_mxfp4.restype = ctypes.c_int
+            lib.moe_quantize_mxfp4.argtypes = [P(MoeTensor), P(MoeTensor), vp]
+            lib.moe_get_device_errors.restype = ctypes.c_int
+            lib.moe_get_device_errors.argtypes = [vp, P(ctypes.c_uint32), P(ctypes.c_uint32)]
+            lib.moe_profile_enable.restype = ctypes.c_int
+            lib.moe_profile_enable.argtypes = [ctypes.c_int32]
+            lib.moe_profile_read.restype = ctypes.c_int
+            lib.moe_profile_read.argtypes = [P(ctypes.c_float), ctypes.c_int32, P(ctypes.c_int32)]
+            _lib = lib
+    return _lib
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        detail = load().moe_last_cuda_error().decode() if rc == 6 else ""
+        raise MoeError(rc, where, detail)
+
+
+_TORCH_DT = {torch.bfloat16: MOE_BF16, torch.float32: MOE_F32, torch.int32: MOE_I32,
+             torch.int64: MOE_I64}
+
+
+def desc(t: torch.Tensor, scale: torch.Tensor | None = None) -> MoeTensor:
+    """moe_tensor_t for a torch tensor.  uint8 (or float4_e2m1fn_x2) tensors are
+    packed e2m1 pairs: the logical innermost size is twice the byte count and
+    `scale` (uint8 e8m0 codes, one per 32 logical elements) is required."""
+    d = MoeTensor()
+    d.data = t.data_ptr() if t.numel() > 0 else None
+    d.ndim = t.dim()
+    if hasattr(torch, "float4_e2m1fn_x2") and t.dtype == torch.float4_e2m1fn_x2:
+        t = t.view(torch.uint8)
+    if t.dtype == torch.uint8:
+        d.dtype = MOE_E2M1X2
+        if scale is None:
+            raise ValueError("an e2m1 tensor needs its e8m0 scale tensor")
+        if scale.dtype != torch.uint8:
+            scale = scale.view(torch.uint8)
+        d.scale = scale.data_ptr()
+        for i in range(scale.dim()):
+            d.scale_strides[i] = scale.stride(i)
+    else:
+        d.dtype = _TORCH_DT.get(t.dtype, 99)  # unknown dtypes are rejected by the library
+    for i in range(t.dim()):
+        d.sizes[i] = t.shape[i]
+        d.strides[i] = t.stride(i)
+    if d.dtype == MOE_E2M1X2:
+        d.sizes[t.dim() - 1] = 2 * t.shape[-1]
+    return d
+
+
+def _stream_ptr(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def w13_from_packed(w13: torch.Tensor, scale: torch.Tensor | None = None) -> MoeW13:
+    out = MoeW13()
+    d = desc(w13, scale)
+    _check(load().moe_w13_from_packed(ctypes.byref(d), ctypes.byref(out)), "moe_w13_from_packed")
+    return out
+
+
+def w13_from_views(gate: torch.Tensor, up: torch.Tensor, gate_scale=None, up_scale=None) -> MoeW13:
+    out = MoeW13()
+    out.gate = desc(gate, gate_scale)
+    out.up = desc(up, up_scale)
+    return out
+
+
+def workspace_bytes(T: int, H: int, I: int, E: int, k: int, mxfp4: bool = False) -> int:
+    return int(load().moe_workspace_bytes(T, H, I, E, k, MOE_E2M1X2 if mxfp4 else MOE_BF16))
+
+
+def forward(x, w13: MoeW13, w2, topk_ids, topk_weights, out=None, *, w2_scale=None,
+            workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """out[t] = sum_j w[t,j] * SwiGLU-expert_{ids[t,j]}(x[t]) on the GPU.
+
+    w13: MoeW13 from w13_from_packed / w13_from_views.  With `workspace` (a
+    uint8 CUDA tensor of at least workspace_bytes(...)) this calls
+    moe_forward_ws, else moe_forward (library-owned workspace)."""
+    if out is None:
+        out = torch.empty(x.shape[0], x.shape[1], dtype=torch.bfloat16, device=x.device)
+    dx, dw2, di, dw, do = desc(x), desc(w2, w2_scale), desc(topk_ids), desc(topk_weights), desc(out)
+    lib = load()
+    st = _stream_ptr(stream)
+    if workspace is not None:
+        rc = lib.moe_forward_ws(ctypes.byref(dx), ctypes.byref(w13), ctypes.byref(dw2),
+                                ctypes.byref(di), ctypes.byref(dw), ctypes.byref(do),
+                                workspace.data_ptr(), workspace.numel(), st)
+        _check(rc, "moe_forward_ws")
+    else:
+        rc = lib.moe_forward(ctypes.byref(dx), ctypes.byref(w13), ctypes.byref(dw2),
+                             ctypes.byref(di), ctypes.byref(dw), ctypes.byref(do), st)
+        _check(rc, "moe_forward")
+    return out
+
+
+def forward_status(x, w13: MoeW13, w2, topk_ids, topk_weights, out, *, w2_scale=None,
+                   workspace=None, stream=None) -> int:
+    """Like forward() but returns the raw moe_status_t (for error-path tests)."""
+    dx, dw2, di, dw, do = desc(x), desc(w2, w2_scale), desc(topk_ids), desc(topk_weights), desc(out)
+    lib = load()
+    st = _stream_ptr(stream) if torch.cuda.is_available() else None
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_n = workspace.numel() if workspace is not None else 0
+    return int(lib.moe_forward_ws(ctypes.byref(dx), ctypes.byref(w13), ctypes.byref(dw2),
+                                  ctypes.byref(di), ctypes.byref(dw), ctypes.byref(do), ws_ptr,
+                                  ws_n, st))
+
+
+def forward_host(x_host, w13: MoeW13, w2, ids_host, weights_host, out_host, *, w2_scale=None,
+                 stream=None) -> torch.Tensor:
+    """Host activations in, host result out (copies and a stream sync inside)."""
+    dx, dw2, di, dw, do = (desc(x_host), desc(w2, w2_scale), desc(ids_host), desc(weights_host),
+                           desc(out_host))
+    rc = load().moe_forward_host(ctypes.byref(dx), ctypes.byref(w13), ctypes.byref(dw2),
+                                 ctypes.byref(di), ctypes.byref(dw), ctypes.byref(do),
+                                 _stream_ptr(stream))
+    _check(rc, "moe_forward_host")
+    return out_host
+
+
+def align(topk_ids: torch.Tensor, E: int, block_m: int, *, stream=None):
+    """Run the align step alone; returns a dict of device int32 tensors."""
+    T, k = topk_ids.shape
+    S = T * k
+    dev = topk_ids.device
+    pmax = S + min(E, max(S, 1)) * (block_m - 1) + block_m
+    counts = torch.zeros(E, dtype=torch.int32, device=dev)
+    offsets = torch.zeros(E + 1, dtype=torch.int32, device=dev)
+    sorted_ = torch.full((pmax,), -7, dtype=torch.int32, device=dev)
+    block_expert = torch.full((pmax // block_m + 1,), -7, dtype=torch.int32, device=dev)
+    nb = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws = torch.empty(workspace_bytes(max(T, 1), 32, 32, E, k), dtype=torch.uint8, device=dev)
+    d = desc(topk_ids)
+    rc = load().moe_align(ctypes.byref(d), E, block_m, counts.data_ptr(), offsets.data_ptr(),
+                          sorted_.data_ptr(), block_expert.data_ptr(), nb.data_ptr(),
+                          ws.data_ptr(), ws.numel(), _stream_ptr(stream))
+    _check(rc, "moe_align")
+    P = int(offsets[E].item())
+    n = int(nb.item())
+    return {"counts": counts, "offsets": offsets, "sorted": sorted_[:P], "block_expert": block_expert[:n],
+            "num_blocks": n}
+
+
+def quantize_mxfp4(src: torch.Tensor, *, stream=None):
+    """1x32 e8m0 / e2m1 quantisation of the last axis of a bf16/f32 CUDA tensor.
+    Returns (codes uint8 [..., K/2], scales uint8 [..., K/32])."""
+    K = src.shape[-1]
+    codes = torch.empty(*src.shape[:-1], K // 2, dtype=torch.uint8, device=src.device)
+    scales = torch.empty(*src.shape[:-1], K // 32, dtype=torch.uint8, device=src.device)
+    ds = desc(src)
+    dd = desc(codes, scales)
+    _check(load().moe_quantize_mxfp4(ctypes.byref(ds), ctypes.byref(dd), _stream_ptr(stream)),
+           "moe_quantize_mxfp4")
+    return codes, scales
+
+
+def device_errors(stream=None):
+    nb = ctypes.c_uint32(0)
+    to = ctypes.c_uint32(0)
+    _check(load().moe_get_device_errors(_stream_ptr(stream), ctypes.byref(nb), ctypes.byref(to)),
+           "moe_get_device_errors")
+    return int(nb.value), int(to.value)
+
+
+def profile_enable(on: bool = True):
+    _check(load().moe_profile_enable(1 if on else 0), "moe_profile_enable")
+
+
+def profile_read() -> dict:
+    """Step durations (ms) of the last forward run with profiling enabled."""
+    buf = (ctypes.c_float * 8)()
+    n = ctypes.c_int32(0)
+    _check(load().moe_profile_read(buf, 8, ctypes.byref(n)), "moe_profile_read")
+    return {STEP_NAMES[i]: float(buf[i]) for i in range(n.value)}
+
+
+def last_launch_count() -> int:
+    return int(load().moe_last_launch_count())
+
+
+def version() -> str:
+    return load().moe_version().decode()

@@ -1,0 +1,677 @@
+// Host runtime behind include/moe.h: argument validation, workspace layout,
+// TMA tensor-map encoding from each view's real strides, and the launch
+// sequence align -> permute -> GEMM1(+SwiGLU) -> GEMM2(+routing weight) -> combine
+// on the caller's stream (programmatic dependent launch between kernels).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/moe.h"
+#include "moe_internal.h"
+
+namespace moe {
+
+// Device error counters: library memory, one copy per device, no allocation.
+__device__ DeviceErrors g_device_errors;
+
+namespace {
+
+thread_local std::string t_last_cuda_error = "";
+thread_local int32_t t_last_launches = 0;
+
+// per-thread step timing (moe_profile_enable / moe_profile_read)
+constexpr int kProfSteps = 5;
+struct Profiler {
+  bool on = false;
+  bool have = false;
+  cudaEvent_t ev[kProfSteps + 1] = {};
+  int n = 0;
+};
+thread_local Profiler t_prof;
+
+void prof_mark(cudaStream_t st) {
+  if (!t_prof.on || t_prof.n > kProfSteps) return;
+  cudaEventRecord(t_prof.ev[t_prof.n++], st);
+}
+
+moe_status_t cuda_fail(cudaError_t rc, const char* where) {
+  t_last_cuda_error = std::string(where) + ": " + cudaGetErrorName(rc) + " (" +
+                      cudaGetErrorString(rc) + ")";
+  return MOE_ERR_CUDA;
+}
+
+#define MOE_CUDA(call)                                   \
+  do {                                                   \
+    cudaError_t _rc = (call);                            \
+    if (_rc != cudaSuccess) return cuda_fail(_rc, #call); \
+  } while (0)
+
+// ---------------------------------------------------------------- devices
+
+struct DeviceInfo {
+  bool init = false;
+  bool ok = false;
+  int num_sms = 0;
+  DeviceErrors* errors = nullptr;
+};
+
+std::mutex g_dev_mu;
+DeviceInfo g_dev[64];
+
+moe_status_t device_info(DeviceInfo** out) {
+  int dev = 0;
+  MOE_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return MOE_ERR_NO_DEVICE;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.init) {
+    int major = 0, minor = 0;
+    MOE_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+    MOE_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+    MOE_CUDA(cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev));
+    d.ok = (major == 10 && minor == 0);
+    void* p = nullptr;
+    MOE_CUDA(cudaGetSymbolAddress(&p, g_device_errors));
+    d.errors = static_cast<DeviceErrors*>(p);
+    d.init = true;
+  }
+  if (!d.ok) return MOE_ERR_NO_DEVICE;
+  *out = &d;
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------- tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// rank-2/3 K-major tile map: dims[0] is the contiguous (K) axis.
+moe_status_t make_map(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
+                      const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                      CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    t_last_cuda_error = "cuTensorMapEncodeTiled entry point unavailable";
+    return MOE_ERR_CUDA;
+  }
+  cuuint64_t gd[3], gs[2];
+  cuuint32_t bx[3], es[3];
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
+  CUresult r = fn(map, dt, rank, const_cast<void*>(base), gd, gs, bx, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    char buf[160];
+    snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+    t_last_cuda_error = buf;
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+// ---------------------------------------------------------------- validation
+
+int64_t dtype_size(int32_t dt) {
+  switch (dt) {
+    case MOE_BF16: return 2;
+    case MOE_F32: return 4;
+    case MOE_I32: return 4;
+    case MOE_I64: return 8;
+    case MOE_E2M1X2: return 1;
+    default: return 0;
+  }
+}
+
+bool sizes_ok(const moe_tensor_t* t, int ndim) {
+  if (!t || t->ndim != ndim) return false;
+  for (int i = 0; i < ndim; ++i)
+    if (t->sizes[i] < 0) return false;
+  return true;
+}
+
+// Weight view [E, N, K] for TMA: unit inner stride, 16-byte aligned base and outer strides.
+bool weight_layout_ok(const moe_tensor_t* w) {
+  const int64_t es = dtype_size(w->dtype);
+  if (w->strides[2] != 1) return false;
+  if (reinterpret_cast<uintptr_t>(w->data) % 16 != 0) return false;
+  if ((w->strides[1] * es) % 16 != 0 || (w->strides[0] * es) % 16 != 0) return false;
+  if (w->strides[1] <= 0 || w->strides[0] < 0) return false;
+  return true;
+}
+
+View2 view2(const moe_tensor_t* t) {
+  View2 v;
+  v.data = t->data;
+  v.s0 = t->strides[0];
+  v.s1 = t->strides[1];
+  v.dtype = t->dtype;
+  return v;
+}
+
+struct Problem {
+  int64_t T, H, I, E, k;
+  bool mxfp4;
+};
+
+moe_status_t validate(const moe_tensor_t* x, const moe_w13_t* w13, const moe_tensor_t* w2,
+                      const moe_tensor_t* ids, const moe_tensor_t* wts, const moe_tensor_t* out,
+                      bool host_io, Problem* pr) {
+  if (!x || !w13 || !w2 || !ids || !wts || !out) return MOE_ERR_INVALID_ARG;
+  const moe_tensor_t* gate = &w13->gate;
+  const moe_tensor_t* up = &w13->up;
+  if (!sizes_ok(x, 2) || !sizes_ok(gate, 3) || !sizes_ok(up, 3) || !sizes_ok(w2, 3) ||
+      !sizes_ok(ids, 2) || !sizes_ok(wts, 2) || !sizes_ok(out, 2))
+    return MOE_ERR_INVALID_ARG;
+  // dtypes
+  if (x->dtype != MOE_BF16 || out->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED_DTYPE;
+  if (ids->dtype != MOE_I32 && ids->dtype != MOE_I64) return MOE_ERR_UNSUPPORTED_DTYPE;
+  if (wts->dtype != MOE_F32) return MOE_ERR_UNSUPPORTED_DTYPE;
+  const int32_t wd = gate->dtype;
+  if (wd != MOE_BF16 && wd != MOE_E2M1X2) return MOE_ERR_UNSUPPORTED_DTYPE;
+  if (up->dtype != wd || w2->dtype != wd) return MOE_ERR_UNSUPPORTED_DTYPE;
+  // shapes (mismatched hidden dims fail here, before any descriptor is built)
+  const int64_t T = x->sizes[0], H = x->sizes[1];
+  const int64_t E = gate->sizes[0], I = gate->sizes[1];
+  if (gate->sizes[2] != H || up->sizes[2] != H) return MOE_ERR_SHAPE_MISMATCH;
+  if (up->sizes[0] != E || up->sizes[1] != I) return MOE_ERR_SHAPE_MISMATCH;
+  if (w2->sizes[0] != E || w2->sizes[1] != H || w2->sizes[2] != I) return MOE_ERR_SHAPE_MISMATCH;
+  if (ids->sizes[0] != T || wts->sizes[0] != T || wts->sizes[1] != ids->sizes[1])
+    return MOE_ERR_SHAPE_MISMATCH;
+  if (out->sizes[0] != T || out->sizes[1] != H) return MOE_ERR_SHAPE_MISMATCH;
+  const int64_t k = ids->sizes[1];
+  if (k < 1 || k > kMaxTopK) return MOE_ERR_INVALID_ARG;
+  if (E < 1 || E > kMaxExperts || H < 1 || I < 1) return MOE_ERR_INVALID_ARG;
+  if (H % 32 != 0 || I % 32 != 0) return MOE_ERR_SHAPE_MISMATCH;
+  if (T * k >= (int64_t(1) << 30)) return MOE_ERR_INVALID_ARG;
+  // pointers
+  if ((T > 0 && (!x->data || !ids->data || !wts->data || !out->data)) || !gate->data ||
+      !up->data || !w2->data)
+    return MOE_ERR_INVALID_ARG;
+  // layouts the copy engine must express
+  if (!weight_layout_ok(gate) || !weight_layout_ok(up) || !weight_layout_ok(w2))
+    return MOE_ERR_UNSUPPORTED_LAYOUT;
+  if (wd == MOE_E2M1X2) {
+    if (!gate->scale || !up->scale || !w2->scale) return MOE_ERR_INVALID_ARG;
+    if (gate->scale_strides[2] != 1 || up->scale_strides[2] != 1 || w2->scale_strides[2] != 1)
+      return MOE_ERR_UNSUPPORTED_LAYOUT;
+    if (H % 128 != 0 || I % 128 != 0) return MOE_ERR_SHAPE_MISMATCH;
+  }
+  if (host_io) {
+    if (x->strides[1] != 1 || ids->strides[1] != 1 || wts->strides[1] != 1 ||
+        out->strides[1] != 1)
+      return MOE_ERR_UNSUPPORTED_LAYOUT;
+  }
+  pr->T = T;
+  pr->H = H;
+  pr->I = I;
+  pr->E = E;
+  pr->k = k;
+  pr->mxfp4 = (wd == MOE_E2M1X2);
+  return MOE_OK;
+}
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+std::mutex g_ws_mu;
+struct CachedWs {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+} g_ws[64];
+
+moe_status_t cached_workspace(size_t need, void** ptr) {
+  int dev = 0;
+  MOE_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return MOE_ERR_NO_DEVICE;
+  std::lock_guard<std::mutex> lk(g_ws_mu);
+  CachedWs& w = g_ws[dev];
+  if (w.bytes < need) {
+    if (w.ptr) {
+      MOE_CUDA(cudaDeviceSynchronize());
+      MOE_CUDA(cudaFree(w.ptr));
+      w.ptr = nullptr;
+      w.bytes = 0;
+    }
+    MOE_CUDA(cudaMalloc(&w.ptr, need));
+    w.bytes = need;
+  }
+  *ptr = w.ptr;
+  return MOE_OK;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- layout
+
+int32_t choose_block_m(int64_t T, int64_t k, int64_t E) {
+  (void)T;
+  (void)k;
+  (void)E;
+  return 128;  // the tensor-core tile is M = 128 rows
+}
+
+WsLayout make_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, bool mxfp4,
+                     int32_t bm) {
+  WsLayout L;
+  std::memset(&L, 0, sizeof(L));
+  L.T = T;
+  L.H = H;
+  L.I = I;
+  L.E = E;
+  L.k = k;
+  L.S = T * k;
+  L.bm = bm;
+  L.mxfp4 = mxfp4;
+  const int64_t S = L.S;
+  const int64_t nonempty = S < E ? S : E;
+  int64_t p = S + nonempty * (bm - 1);
+  p = (p + bm - 1) / bm * bm;
+  if (p < bm) p = bm;
+  L.p_max = p;
+  L.nb_max = p / bm;
+  L.n_chunks = (S + kAlignChunk - 1) / kAlignChunk;
+  if (L.n_chunks < 1) L.n_chunks = 1;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  L.counts = take(sizeof(int32_t) * E);
+  L.offsets = take(sizeof(int32_t) * (E + 1));
+  L.num_blocks = take(sizeof(int32_t) * 4);
+  L.chunk_counts = take(S > kAlignSmallMax ? sizeof(int32_t) * L.n_chunks * E : 0);
+  L.sorted = take(sizeof(int32_t) * p);
+  L.inv = take(sizeof(int32_t) * (S > 0 ? S : 1));
+  L.block_expert = take(sizeof(int32_t) * L.nb_max);
+  if (!mxfp4) {
+    L.a1 = take(size_t(p) * H * 2);
+    L.a1_scale = off;
+    L.h = take(size_t(p) * I * 2);
+    L.h_scale = off;
+  } else {
+    L.a1 = take(size_t(p) * H / 2);
+    L.a1_scale = take(size_t(p) * H / 32);
+    L.h = take(size_t(p) * I / 2);
+    L.h_scale = take(size_t(p) * I / 32);
+  }
+  L.y = take(size_t(S > 0 ? S : 1) * H * 2);
+  L.total = off;
+  return L;
+}
+
+namespace {
+
+moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe_tensor_t* w2,
+                          const moe_tensor_t* ids, const moe_tensor_t* wts, moe_tensor_t* out,
+                          const Problem& pr, void* ws, size_t ws_bytes, cudaStream_t st) {
+  int launches = 0;
+  t_last_launches = 0;
+  if (pr.T == 0) return MOE_OK;
+  const int32_t bm = choose_block_m(pr.T, pr.k, pr.E);
+  const WsLayout L = make_layout(pr.T, pr.H, pr.I, pr.E, pr.k, pr.mxfp4, bm);
+  if (!ws || ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return MOE_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  moe_status_t s = device_info(&dev);
+  if (s != MOE_OK) return s;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  int32_t* counts = reinterpret_cast<int32_t*>(w + L.counts);
+  int32_t* offsets = reinterpret_cast<int32_t*>(w + L.offsets);
+  int32_t* num_blocks = reinterpret_cast<int32_t*>(w + L.num_blocks);
+  int32_t* chunk_counts = reinterpret_cast<int32_t*>(w + L.chunk_counts);
+  int32_t* sorted = reinterpret_cast<int32_t*>(w + L.sorted);
+  int32_t* inv = reinterpret_cast<int32_t*>(w + L.inv);
+  int32_t* block_expert = reinterpret_cast<int32_t*>(w + L.block_expert);
+
+  const moe_tensor_t* gate = &w13->gate;
+  const moe_tensor_t* up = &w13->up;
+
+  if (pr.mxfp4) return MOE_ERR_UNSUPPORTED_DTYPE;  // block-scaled path: see moe_gemm_mxfp4.cu
+
+  // ---- tensor maps (bf16, 128-byte swizzle, box 64 x 128)
+  CUtensorMap mA1, mGate, mUp, mH, mW2;
+  const uint32_t box2[2] = {64, 128};
+  const uint32_t box3[3] = {64, 128, 1};
+  {
+    const uint64_t d[2] = {uint64_t(pr.H), uint64_t(L.p_max)};
+    const uint64_t sb[1] = {uint64_t(pr.H) * 2};
+    s = make_map(&mA1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w + L.a1, d, sb, box2,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s != MOE_OK) return s;
+  }
+  {
+    // expert stride = the view's real stride(0): the first tile of expert e is
+    // base + e * stride(0), whatever lies between experts (e.g. the up half).
+    const uint64_t d[3] = {uint64_t(pr.H), uint64_t(pr.I), uint64_t(pr.E)};
+    const uint64_t sg[2] = {uint64_t(gate->strides[1]) * 2, uint64_t(gate->strides[0]) * 2};
+    s = make_map(&mGate, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, gate->data, d, sg, box3,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s != MOE_OK) return s;
+    const uint64_t su[2] = {uint64_t(up->strides[1]) * 2, uint64_t(up->strides[0]) * 2};
+    s = make_map(&mUp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, up->data, d, su, box3,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s != MOE_OK) return s;
+  }
+  {
+    const uint64_t d[2] = {uint64_t(pr.I), uint64_t(L.p_max)};
+    const uint64_t sb[1] = {uint64_t(pr.I) * 2};
+    s = make_map(&mH, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w + L.h, d, sb, box2,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s != MOE_OK) return s;
+    const uint64_t d3[3] = {uint64_t(pr.I), uint64_t(pr.H), uint64_t(pr.E)};
+    const uint64_t s3[2] = {uint64_t(w2->strides[1]) * 2, uint64_t(w2->strides[0]) * 2};
+    s = make_map(&mW2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, w2->data, d3, s3, box3,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s != MOE_OK) return s;
+  }
+
+  // ---- launches
+  t_prof.n = 0;
+  t_prof.have = false;
+  prof_mark(st);
+  cudaError_t rc;
+  rc = launch_align(view2(ids), pr.T, pr.k, pr.E, bm, counts, offsets, sorted, inv, block_expert,
+                    num_blocks, chunk_counts, L.n_chunks, dev->errors, st, &launches);
+  if (rc != cudaSuccess) return cuda_fail(rc, "align");
+  prof_mark(st);
+  rc = launch_permute_bf16(view2(x), pr.T, pr.H, pr.k, pr.E, inv, offsets, counts,
+                           reinterpret_cast<__nv_bfloat16*>(w + L.a1), st, &launches);
+  if (rc != cudaSuccess) return cuda_fail(rc, "permute");
+  prof_mark(st);
+
+  GemmArgs g1;
+  std::memset(&g1, 0, sizeof(g1));
+  g1.K = pr.H;
+  g1.N = pr.I;
+  g1.n_tiles = (pr.I + 127) / 128;
+  g1.max_tiles = L.nb_max * g1.n_tiles;
+  g1.num_blocks = num_blocks;
+  g1.block_expert = block_expert;
+  g1.sorted = sorted;
+  g1.S = L.S;
+  g1.out = w + L.h;
+  g1.out_ld = pr.I;
+  g1.k = pr.k;
+  g1.err = dev->errors;
+  rc = launch_gemm1_bf16(mA1, mGate, mUp, g1, dev->num_sms, st, &launches);
+  if (rc != cudaSuccess) return cuda_fail(rc, "gemm1");
+  prof_mark(st);
+
+  GemmArgs g2 = g1;
+  g2.K = pr.I;
+  g2.N = pr.H;
+  g2.n_tiles = (pr.H + 255) / 256;
+  g2.max_tiles = L.nb_max * g2.n_tiles;
+  g2.out = w + L.y;
+  g2.out_ld = pr.H;
+  g2.topk_w = view2(wts);
+  rc = launch_gemm2_bf16(mH, mW2, g2, dev->num_sms, st, &launches);
+  if (rc != cudaSuccess) return cuda_fail(rc, "gemm2");
+  prof_mark(st);
+
+  rc = launch_combine(reinterpret_cast<const __nv_bfloat16*>(w + L.y), view2(ids), pr.E, pr.T,
+                      pr.H, pr.k, out->data, out->strides[0], out->strides[1], st, &launches);
+  if (rc != cudaSuccess) return cuda_fail(rc, "combine");
+  prof_mark(st);
+  t_prof.have = t_prof.on && t_prof.n == kProfSteps + 1;
+  t_last_launches = launches;
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_status_string(moe_status_t st) {
+  switch (st) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_SHAPE_MISMATCH: return "MOE_ERR_SHAPE_MISMATCH";
+    case MOE_ERR_UNSUPPORTED_DTYPE: return "MOE_ERR_UNSUPPORTED_DTYPE";
+    case MOE_ERR_UNSUPPORTED_LAYOUT: return "MOE_ERR_UNSUPPORTED_LAYOUT";
+    case MOE_ERR_WORKSPACE_TOO_SMALL: return "MOE_ERR_WORKSPACE_TOO_SMALL";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_NO_DEVICE: return "MOE_ERR_NO_DEVICE";
+    case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+const char* moe_last_cuda_error(void) { return t_last_cuda_error.c_str(); }
+
+const char* moe_version(void) { return "moe-b200 0.1 (sm_100a)"; }
+
+int32_t moe_last_launch_count(void) { return t_last_launches; }
+
+moe_status_t moe_profile_enable(int32_t on) {
+  if (on && !t_prof.ev[0]) {
+    for (int i = 0; i <= kProfSteps; ++i) MOE_CUDA(cudaEventCreate(&t_prof.ev[i]));
+  }
+  t_prof.on = on != 0;
+  t_prof.have = false;
+  return MOE_OK;
+}
+
+moe_status_t moe_profile_read(float* ms, int32_t capacity, int32_t* n) {
+  if (!ms || !n) return MOE_ERR_INVALID_ARG;
+  *n = 0;
+  if (!t_prof.have) return MOE_OK;
+  MOE_CUDA(cudaEventSynchronize(t_prof.ev[kProfSteps]));
+  int32_t m = 0;
+  for (int i = 0; i < kProfSteps && m < capacity; ++i, ++m)
+    MOE_CUDA(cudaEventElapsedTime(&ms[m], t_prof.ev[i], t_prof.ev[i + 1]));
+  *n = m;
+  return MOE_OK;
+}
+
+moe_status_t moe_w13_from_packed(const moe_tensor_t* w13, moe_w13_t* out) {
+  if (!w13 || !out || w13->ndim != 3) return MOE_ERR_INVALID_ARG;
+  if (w13->sizes[1] % 2 != 0) return MOE_ERR_SHAPE_MISMATCH;
+  const int64_t I = w13->sizes[1] / 2;
+  const int64_t es = dtype_size(w13->dtype);
+  if (es == 0) return MOE_ERR_UNSUPPORTED_DTYPE;
+  out->gate = *w13;
+  out->gate.sizes[1] = I;
+  out->up = out->gate;
+  // up = rows [I, 2I): same strides, base advanced by I rows (Liger-Kernel PR #1377, "Problems")
+  out->up.data = static_cast<uint8_t*>(w13->data) + I * w13->strides[1] * es;
+  if (w13->dtype == MOE_E2M1X2 && w13->scale)
+    out->up.scale = static_cast<uint8_t*>(w13->scale) + I * w13->scale_strides[1];
+  return MOE_OK;
+}
+
+size_t moe_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, int32_t wdtype) {
+  if (T < 0 || H < 1 || I < 1 || E < 1 || k < 1) return 0;
+  if (wdtype != MOE_BF16 && wdtype != MOE_E2M1X2) return 0;
+  const int32_t bm = choose_block_m(T, k, E);
+  return make_layout(T, H, I, E, k, wdtype == MOE_E2M1X2, bm).total;
+}
+
+moe_status_t moe_forward_ws(const moe_tensor_t* x, const moe_w13_t* w13, const moe_tensor_t* w2,
+                            const moe_tensor_t* topk_ids, const moe_tensor_t* topk_weights,
+                            moe_tensor_t* out, void* workspace, size_t workspace_bytes,
+                            moe_stream_t stream) {
+  t_last_launches = 0;
+  Problem pr;
+  moe_status_t s = validate(x, w13, w2, topk_ids, topk_weights, out, false, &pr);
+  if (s != MOE_OK) return s;
+  return forward_impl(x, w13, w2, topk_ids, topk_weights, out, pr, workspace, workspace_bytes,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_forward(const moe_tensor_t* x, const moe_w13_t* w13, const moe_tensor_t* w2,
+                         const moe_tensor_t* topk_ids, const moe_tensor_t* topk_weights,
+                         moe_tensor_t* out, moe_stream_t stream) {
+  t_last_launches = 0;
+  Problem pr;
+  moe_status_t s = validate(x, w13, w2, topk_ids, topk_weights, out, false, &pr);
+  if (s != MOE_OK) return s;
+  if (pr.T == 0) return MOE_OK;
+  const size_t need = moe_workspace_bytes(pr.T, pr.H, pr.I, pr.E, pr.k, w13->gate.dtype);
+  void* ws = nullptr;
+  s = cached_workspace(need, &ws);
+  if (s != MOE_OK) return s;
+  return forward_impl(x, w13, w2, topk_ids, topk_weights, out, pr, ws, need,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_forward_host(const moe_tensor_t* x_host, const moe_w13_t* w13,
+                              const moe_tensor_t* w2, const moe_tensor_t* topk_ids_host,
+                              const moe_tensor_t* topk_weights_host, moe_tensor_t* out_host,
+                              moe_stream_t stream) {
+  t_last_launches = 0;
+  Problem pr;
+  moe_status_t s =
+      validate(x_host, w13, w2, topk_ids_host, topk_weights_host, out_host, true, &pr);
+  if (s != MOE_OK) return s;
+  if (pr.T == 0) return MOE_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // device staging for the activations after the forward's own workspace
+  const size_t core = moe_workspace_bytes(pr.T, pr.H, pr.I, pr.E, pr.k, w13->gate.dtype);
+  const int64_t idsz = dtype_size(topk_ids_host->dtype);
+  const size_t x_off = align256(core);
+  const size_t ids_off = align256(x_off + size_t(pr.T) * pr.H * 2);
+  const size_t w_off = align256(ids_off + size_t(pr.T) * pr.k * idsz);
+  const size_t o_off = align256(w_off + size_t(pr.T) * pr.k * 4);
+  const size_t need = align256(o_off + size_t(pr.T) * pr.H * 2);
+  void* ws = nullptr;
+  s = cached_workspace(need, &ws);
+  if (s != MOE_OK) return s;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  MOE_CUDA(cudaMemcpy2DAsync(w + x_off, pr.H * 2, x_host->data, x_host->strides[0] * 2, pr.H * 2,
+                             pr.T, cudaMemcpyHostToDevice, st));
+  MOE_CUDA(cudaMemcpy2DAsync(w + ids_off, pr.k * idsz, topk_ids_host->data,
+                             topk_ids_host->strides[0] * idsz, pr.k * idsz, pr.T,
+                             cudaMemcpyHostToDevice, st));
+  MOE_CUDA(cudaMemcpy2DAsync(w + w_off, pr.k * 4, topk_weights_host->data,
+                             topk_weights_host->strides[0] * 4, pr.k * 4, pr.T,
+                             cudaMemcpyHostToDevice, st));
+  moe_tensor_t xd = *x_host, idd = *topk_ids_host, wd = *topk_weights_host, od = *out_host;
+  xd.data = w + x_off;
+  xd.strides[0] = pr.H;
+  xd.strides[1] = 1;
+  idd.data = w + ids_off;
+  idd.strides[0] = pr.k;
+  idd.strides[1] = 1;
+  wd.data = w + w_off;
+  wd.strides[0] = pr.k;
+  wd.strides[1] = 1;
+  od.data = w + o_off;
+  od.strides[0] = pr.H;
+  od.strides[1] = 1;
+  s = forward_impl(&xd, w13, w2, &idd, &wd, &od, pr, ws, core, st);
+  if (s != MOE_OK) return s;
+  const int32_t fwd_launches = t_last_launches;
+  MOE_CUDA(cudaMemcpy2DAsync(out_host->data, out_host->strides[0] * 2, w + o_off, pr.H * 2,
+                             pr.H * 2, pr.T, cudaMemcpyDeviceToHost, st));
+  MOE_CUDA(cudaStreamSynchronize(st));
+  t_last_launches = fwd_launches;
+  return MOE_OK;
+}
+
+moe_status_t moe_align(const moe_tensor_t* topk_ids, int64_t E, int32_t block_m, int32_t* counts,
+                       int32_t* offsets, int32_t* sorted_slots, int32_t* block_expert,
+                       int32_t* num_blocks, void* workspace, size_t workspace_bytes,
+                       moe_stream_t stream) {
+  if (!topk_ids || !sizes_ok(topk_ids, 2) || !counts || !offsets || !sorted_slots ||
+      !block_expert || !num_blocks)
+    return MOE_ERR_INVALID_ARG;
+  if (topk_ids->dtype != MOE_I32 && topk_ids->dtype != MOE_I64) return MOE_ERR_UNSUPPORTED_DTYPE;
+  if (E < 1 || E > kMaxExperts) return MOE_ERR_INVALID_ARG;
+  if (block_m != 16 && block_m != 32 && block_m != 64 && block_m != 128 && block_m != 256)
+    return MOE_ERR_INVALID_ARG;
+  const int64_t T = topk_ids->sizes[0], k = topk_ids->sizes[1];
+  if (k < 1 || k > kMaxTopK || T * k >= (int64_t(1) << 30)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!topk_ids->data) return MOE_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  moe_status_t s = device_info(&dev);
+  if (s != MOE_OK) return s;
+  const WsLayout L = make_layout(T, 32, 32, E, k, false, block_m);
+  // inv and chunk counts live in the caller's workspace
+  const size_t need = align256(L.inv + sizeof(int32_t) * T * k);
+  if (!workspace || workspace_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  int launches = 0;
+  cudaError_t rc = launch_align(view2(topk_ids), T, k, E, block_m, counts, offsets, sorted_slots,
+                                reinterpret_cast<int32_t*>(w + L.inv), block_expert, num_blocks,
+                                reinterpret_cast<int32_t*>(w + L.chunk_counts), L.n_chunks,
+                                dev->errors, reinterpret_cast<cudaStream_t>(stream), &launches);
+  if (rc != cudaSuccess) return cuda_fail(rc, "align");
+  return MOE_OK;
+}
+
+moe_status_t moe_quantize_mxfp4(const moe_tensor_t* src, moe_tensor_t* dst, moe_stream_t stream) {
+  if (!src || !dst || !src->data || !dst->data || !dst->scale) return MOE_ERR_INVALID_ARG;
+  if (src->ndim != dst->ndim || (src->ndim != 2 && src->ndim != 3)) return MOE_ERR_INVALID_ARG;
+  if (src->dtype != MOE_BF16 && src->dtype != MOE_F32) return MOE_ERR_UNSUPPORTED_DTYPE;
+  if (dst->dtype != MOE_E2M1X2) return MOE_ERR_UNSUPPORTED_DTYPE;
+  for (int i = 0; i < src->ndim; ++i)
+    if (src->sizes[i] != dst->sizes[i] || src->sizes[i] < 0) return MOE_ERR_SHAPE_MISMATCH;
+  const int nd = src->ndim;
+  const int64_t K = src->sizes[nd - 1];
+  if (K % 32 != 0) return MOE_ERR_SHAPE_MISMATCH;
+  if (src->strides[nd - 1] != 1 || dst->strides[nd - 1] != 1 || dst->scale_strides[nd - 1] != 1)
+    return MOE_ERR_UNSUPPORTED_LAYOUT;
+  DeviceInfo* dev = nullptr;
+  moe_status_t s = device_info(&dev);
+  if (s != MOE_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t es = dtype_size(src->dtype);
+  // rank 3 is walked one leading index at a time; each slice is a row-strided matrix
+  const int64_t outer = (nd == 3) ? src->sizes[0] : 1;
+  const int64_t R = src->sizes[nd - 2];
+  for (int64_t o = 0; o < outer; ++o) {
+    const uint8_t* sp = static_cast<const uint8_t*>(src->data) + (nd == 3 ? o * src->strides[0] * es : 0);
+    uint8_t* dp = static_cast<uint8_t*>(dst->data) + (nd == 3 ? o * dst->strides[0] : 0);
+    uint8_t* sc = static_cast<uint8_t*>(dst->scale) + (nd == 3 ? o * dst->scale_strides[0] : 0);
+    cudaError_t rc = launch_quantize_rows(sp, src->dtype, R, K, src->strides[nd - 2], dp,
+                                          dst->strides[nd - 2], sc, dst->scale_strides[nd - 2], st);
+    if (rc != cudaSuccess) return cuda_fail(rc, "quantize");
+  }
+  return MOE_OK;
+}
+
+moe_status_t moe_get_device_errors(moe_stream_t stream, uint32_t* n_bad_ids, uint32_t* timeouts) {
+  DeviceInfo* dev = nullptr;
+  moe_status_t s = device_info(&dev);
+  if (s != MOE_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  DeviceErrors h;
+  MOE_CUDA(cudaMemcpyAsync(&h, dev->errors, sizeof(h), cudaMemcpyDeviceToHost, st));
+  MOE_CUDA(cudaMemsetAsync(dev->errors, 0, sizeof(h), st));
+  MOE_CUDA(cudaStreamSynchronize(st));
+  if (n_bad_ids) *n_bad_ids = h.bad_ids;
+  if (timeouts) *timeouts = h.timeouts;
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,248 @@
+// Step "permute": gather the token rows of x into expert-grouped order so each
+// bm-row block of the grouped GEMM reads one expert's tokens contiguously.
+//   A1[inv[t*k + j], :] = x[t, :]     for every valid slot, x read once per token
+//   A1[p, :] = 0                      for the padding rows of every expert
+// x is read through its strides (LightLLM issue #1467 shows what dropping the
+// inner stride does); the fast path needs a unit inner stride and 16-byte rows.
+//
+// The MXFP4 form quantises each x row with the 1x32 e8m0 rule while gathering
+// (aiter PR #3859, "Details": activations are e2m1 with per-1x32 scales):
+// codes [P, H/2] (even element in the low nibble) and scales [P, H/32].
+#include "../../include/moe.h"
+#include "moe_internal.h"
+
+namespace moe {
+
+// e2m1 codes of two floats already divided by their block scale:
+// round to nearest even on the e2m1 grid, saturating to +-6.
+__device__ __forceinline__ uint32_t cvt_e2m1x2(float even, float odd) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(even), "f"(odd));
+  return r & 0xffu;
+}
+
+// Shared exponent of a block with absolute maximum amax (finite, fp32):
+// s = clamp(floor(log2(amax)) - 2, -127, 127); e8m0 code s + 127; 0 for amax == 0.
+__device__ __forceinline__ int mx_scale_exp(float amax) {
+  if (!(amax > 0.0f)) return -127;
+  const uint32_t bits = __float_as_uint(amax);
+  int ex = static_cast<int>((bits >> 23) & 0xffu);
+  int fl;
+  if (ex == 0) {
+    // subnormal amax: floor(log2) = -149 + index of the highest set mantissa bit
+    fl = -149 + (31 - __clz(bits & 0x7fffffu));
+  } else {
+    fl = ex - 127;
+  }
+  int s = fl - 2;
+  return max(-127, min(127, s));
+}
+
+// 2^-s as an exact float for s in [-127, 127]; every value but 2^-127 is a
+// normal number whose exponent field can be written directly.
+__device__ __forceinline__ float exp2i_neg(int s) {
+  const int e = 127 - s;  // biased exponent of 2^-s
+  if (e >= 1 && e <= 254) return __uint_as_float(static_cast<uint32_t>(e) << 23);
+  return ldexpf(1.0f, -s);
+}
+
+// Quantise 32 floats: returns scale code, writes 16 code bytes as 4 words.
+__device__ __forceinline__ uint32_t mx_quant32(const float (&v)[32], uint32_t (&w)[4]) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const int s = mx_scale_exp(amax);
+  const float inv = exp2i_neg(s);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int i = q * 8 + b * 2;
+      word |= cvt_e2m1x2(v[i] * inv, v[i + 1] * inv) << (8 * b);
+    }
+    w[q] = word;
+  }
+  return static_cast<uint32_t>(s + 127);
+}
+
+namespace {
+
+__device__ __forceinline__ float bf16_to_f(uint16_t b) { return __uint_as_float(uint32_t(b) << 16); }
+
+__global__ void __launch_bounds__(256) permute_bf16_kernel(View2 x, int64_t T, int64_t H, int64_t k,
+                                                           int64_t E, const int32_t* inv,
+                                                           const int32_t* offsets,
+                                                           const int32_t* counts,
+                                                           __nv_bfloat16* a1, int vec_ok,
+                                                           int tok_blocks) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int64_t H8 = H / 8;
+  if (blockIdx.x < tok_blocks) {
+    for (int64_t t = blockIdx.x; t < T; t += tok_blocks) {
+      int32_t pos[kMaxTopK];
+      for (int j = 0; j < k; ++j) pos[j] = inv[t * k + j];
+      if (vec_ok) {
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x.data) + t * x.s0);
+        for (int64_t c = threadIdx.x; c < H8; c += blockDim.x) {
+          const uint4 v = src[c];
+          for (int j = 0; j < k; ++j)
+            if (pos[j] >= 0) reinterpret_cast<uint4*>(a1 + static_cast<int64_t>(pos[j]) * H)[c] = v;
+        }
+      } else {
+        const uint16_t* src = static_cast<const uint16_t*>(x.data) + t * x.s0;
+        for (int64_t h = threadIdx.x; h < H; h += blockDim.x) {
+          const uint16_t v = src[h * x.s1];
+          for (int j = 0; j < k; ++j)
+            if (pos[j] >= 0) reinterpret_cast<uint16_t*>(a1 + static_cast<int64_t>(pos[j]) * H)[h] = v;
+        }
+      }
+    }
+  } else {
+    // zero the padding rows of one expert
+    const int64_t e = blockIdx.x - tok_blocks;
+    if (e >= E) return;
+    const int64_t p0 = offsets[e] + counts[e], p1 = offsets[e + 1];
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    for (int64_t p = p0; p < p1; ++p)
+      for (int64_t c = threadIdx.x; c < H8; c += blockDim.x) reinterpret_cast<uint4*>(a1 + p * H)[c] = z;
+  }
+}
+
+// One thread per 32-element block of a row; a CTA walks tokens.
+__global__ void __launch_bounds__(128) permute_quant_kernel(View2 x, int64_t T, int64_t H, int64_t k,
+                                                            int64_t E, const int32_t* inv,
+                                                            const int32_t* offsets,
+                                                            const int32_t* counts, uint8_t* codes,
+                                                            uint8_t* scales, int vec_ok,
+                                                            int tok_blocks) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int64_t nb = H / 32;  // blocks per row
+  if (blockIdx.x < tok_blocks) {
+    for (int64_t t = blockIdx.x; t < T; t += tok_blocks) {
+      int32_t pos[kMaxTopK];
+      for (int j = 0; j < k; ++j) pos[j] = inv[t * k + j];
+      for (int64_t b = threadIdx.x; b < nb; b += blockDim.x) {
+        float v[32];
+        if (vec_ok) {
+          const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x.data) + t * x.s0 + b * 32);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint4 u = src[q];
+            const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              v[q * 8 + 2 * i] = bf16_to_f(static_cast<uint16_t>(w4[i] & 0xffffu));
+              v[q * 8 + 2 * i + 1] = bf16_to_f(static_cast<uint16_t>(w4[i] >> 16));
+            }
+          }
+        } else {
+          const uint16_t* src = static_cast<const uint16_t*>(x.data) + t * x.s0;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = bf16_to_f(src[(b * 32 + i) * x.s1]);
+        }
+        uint32_t w[4];
+        const uint32_t sc = mx_quant32(v, w);
+        for (int j = 0; j < k; ++j) {
+          if (pos[j] < 0) continue;
+          *reinterpret_cast<uint4*>(codes + static_cast<int64_t>(pos[j]) * (H / 2) + b * 16) =
+              make_uint4(w[0], w[1], w[2], w[3]);
+          scales[static_cast<int64_t>(pos[j]) * nb + b] = static_cast<uint8_t>(sc);
+        }
+      }
+    }
+  } else {
+    const int64_t e = blockIdx.x - tok_blocks;
+    if (e >= E) return;
+    const int64_t p0 = offsets[e] + counts[e], p1 = offsets[e + 1];
+    for (int64_t p = p0; p < p1; ++p)
+      for (int64_t b = threadIdx.x; b < nb; b += blockDim.x) {
+        *reinterpret_cast<uint4*>(codes + p * (H / 2) + b * 16) = make_uint4(0, 0, 0, 0);
+        scales[p * nb + b] = 0;
+      }
+  }
+}
+
+// Standalone quantiser: one thread per 32-element block.
+__global__ void __launch_bounds__(256) quantize_rows_kernel(const void* src, int32_t src_dtype,
+                                                            int64_t R, int64_t K, int64_t src_ld,
+                                                            uint8_t* codes, int64_t codes_ld,
+                                                            uint8_t* scales, int64_t scales_ld) {
+  const int64_t nb = K / 32;
+  const int64_t total = R * nb;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / nb, b = i - r * nb;
+    float v[32];
+    if (src_dtype == MOE_BF16) {
+      const uint16_t* p = static_cast<const uint16_t*>(src) + r * src_ld + b * 32;
+#pragma unroll
+      for (int q = 0; q < 32; ++q) v[q] = bf16_to_f(p[q]);
+    } else {
+      const float* p = static_cast<const float*>(src) + r * src_ld + b * 32;
+#pragma unroll
+      for (int q = 0; q < 32; ++q) v[q] = p[q];
+    }
+    uint32_t w[4];
+    const uint32_t sc = mx_quant32(v, w);
+    uint8_t* c = codes + r * codes_ld + b * 16;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      c[4 * q + 0] = w[q] & 0xffu;
+      c[4 * q + 1] = (w[q] >> 8) & 0xffu;
+      c[4 * q + 2] = (w[q] >> 16) & 0xffu;
+      c[4 * q + 3] = w[q] >> 24;
+    }
+    scales[r * scales_ld + b] = static_cast<uint8_t>(sc);
+  }
+}
+
+}  // namespace
+
+static int token_blocks(int64_t T) {
+  int64_t b = T < 2048 ? T : 2048;
+  return static_cast<int>(b < 1 ? 1 : b);
+}
+
+cudaError_t launch_permute_bf16(const View2& x, int64_t T, int64_t H, int64_t k, int64_t E,
+                                const int32_t* inv, const int32_t* offsets, const int32_t* counts,
+                                __nv_bfloat16* a1, cudaStream_t st, int* launches) {
+  const int vec_ok = (x.s1 == 1) && ((x.s0 * 2) % 16 == 0) &&
+                     (reinterpret_cast<uintptr_t>(x.data) % 16 == 0);
+  const int tb = token_blocks(T);
+  if (launches) *launches += 1;
+  return launch_pdl(permute_bf16_kernel, dim3(static_cast<unsigned>(tb + E)), dim3(256), 0, st, x,
+                    T, H, k, E, inv, offsets, counts, a1, vec_ok, tb);
+}
+
+cudaError_t launch_permute_quant(const View2& x, int64_t T, int64_t H, int64_t k, int64_t E,
+                                 const int32_t* inv, const int32_t* offsets, const int32_t* counts,
+                                 uint8_t* codes, uint8_t* scales, cudaStream_t st, int* launches) {
+  const int vec_ok = (x.s1 == 1) && ((x.s0 * 2) % 16 == 0) &&
+                     (reinterpret_cast<uintptr_t>(x.data) % 16 == 0);
+  const int tb = token_blocks(T);
+  if (launches) *launches += 1;
+  return launch_pdl(permute_quant_kernel, dim3(static_cast<unsigned>(tb + E)), dim3(128), 0, st, x,
+                    T, H, k, E, inv, offsets, counts, codes, scales, vec_ok, tb);
+}
+
+cudaError_t launch_quantize_rows(const void* src, int32_t src_dtype, int64_t R, int64_t K,
+                                 int64_t src_ld, uint8_t* codes, int64_t codes_ld,
+                                 uint8_t* scales, int64_t scales_ld, cudaStream_t st) {
+  const int64_t total = R * (K / 32);
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  if (blocks < 1) blocks = 1;
+  quantize_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+      src, src_dtype, R, K, src_ld, codes, codes_ld, scales, scales_ld);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

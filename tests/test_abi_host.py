@@ -1,0 +1,157 @@
+"""Host-side tests of the C ABI (no GPU needed): the library loads and exports
+every entry point include/moe.h declares, status codes, packed-view metadata,
+workspace sizing, and the validation errors that must come before anything is
+launched or any descriptor is built (Liger-Kernel PR #1377, "Testing Done")."""
+
+import json
+import os
+import re
+
+import pytest
+import torch
+
+import mixture_experts_layer_46_b200 as moe
+from mixture_experts_layer_46_b200 import _abi
+from mixture_experts_layer_46_b200 import workloads as wl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+GOLD = os.path.join(ROOT, "tests", "golden")
+
+
+def _declared_entry_points():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src))
+    return names
+
+
+def test_library_exports_every_declared_entry_point():
+    lib = moe.load()
+    declared = _declared_entry_points()
+    assert declared, "no entry points parsed from include/*.h"
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert declared == set(_abi.EXPORTS) | (declared - set(_abi.EXPORTS))
+    assert set(_abi.EXPORTS) <= declared
+
+
+def test_status_strings():
+    lib = moe.load()
+    for code, name in _abi.STATUS.items():
+        assert lib.moe_status_string(code).decode() == name
+
+
+def test_w13_from_packed_locates_up_by_stride():
+    # I=1536, TileN=128 worked example (tests/golden/liger_tile_example.json)
+    g = json.load(open(os.path.join(GOLD, "liger_tile_example.json")))
+    I, tile_n, H, E = g["intermediate"], g["tile_n"], 64, 3
+    w13 = torch.empty(E, 2 * I, H, dtype=torch.bfloat16)  # storage only
+    v = moe.w13_from_packed(w13)
+    assert v.gate.sizes[1] == I and v.up.sizes[1] == I
+    assert v.gate.strides[0] == 2 * I * H  # the real expert stride is kept
+    row = lambda d, e, n: (d.data - w13.data_ptr()) // 2 // H + e * d.strides[0] // H + n * tile_n
+    # tile index (in TileN-row units) of (expert, n-th useful tile) for each view
+    tile = lambda d, e, n: row(d, e, n) // tile_n
+    assert I // tile_n == g["useful_tiles_per_expert"]
+    assert v.gate.strides[0] // H // tile_n == g["packed_physical_stride_tiles"]
+    assert tile(v.gate, 0, 0) == g["packed_tile_ranges"]["expert0_gate"][0]
+    assert tile(v.gate, 0, 11) == g["packed_tile_ranges"]["expert0_gate"][1]
+    assert tile(v.up, 0, 0) == g["packed_tile_ranges"]["expert0_up"][0]
+    assert tile(v.gate, 1, 0) == g["packed_tile_ranges"]["expert1_gate"][0]
+    # the old addressing, expert * (I / TileN), would put expert 1's gate on expert 0's up
+    assert 1 * (I // tile_n) == g["old_offset_expert1_gate_first_tile"] == tile(v.up, 0, 0)
+    # contiguous copies: physical stride equals the useful tile count
+    c = moe.w13_from_views(w13[:, :I].contiguous(), w13[:, I:].contiguous())
+    assert c.gate.strides[0] // H // tile_n == g["useful_tiles_per_expert"]
+
+
+def test_packed_copy_cost_matches_the_pages():
+    # 16 local experts x 2 * 1536 * 4096 bf16 = 0.375 GiB per layer of retained copies
+    g = json.load(open(os.path.join(GOLD, "liger_tile_example.json")))
+    assert 16 * 2 * g["intermediate"] * 4096 * 2 / 2 ** 30 == g["copy_cost_gib_per_layer"]
+
+
+def test_workspace_independent_of_weight_size_and_layout():
+    base = moe.workspace_bytes(4096, 4096, 1536, 128, 8)
+    assert base > 0
+    w_bytes = 128 * 3 * 1536 * 4096 * 2
+    assert base < w_bytes / 4
+    assert moe.workspace_bytes(0, 4096, 1536, 128, 8) > 0
+    assert moe.workspace_bytes(4096, 4096, 1536, 128, 8, mxfp4=True) < base
+    assert moe.load().moe_workspace_bytes(4, 64, 64, 4, 2, 9) == 0
+
+
+def _cpu_problem(T=8, H=64, I=32, E=4, k=2):
+    x = torch.zeros(T, H, dtype=torch.bfloat16)
+    w13 = torch.zeros(E, 2 * I, H, dtype=torch.bfloat16)
+    w2 = torch.zeros(E, H, I, dtype=torch.bfloat16)
+    ids = torch.zeros(T, k, dtype=torch.int32)
+    wts = torch.zeros(T, k, dtype=torch.float32)
+    out = torch.empty(T, H, dtype=torch.bfloat16)
+    return x, w13, w2, ids, wts, out
+
+
+def _status(x, w13v, w2, ids, wts, out, ws=None):
+    return moe.forward_status(x, w13v, w2, ids, wts, out, workspace=ws)
+
+
+def test_mismatched_gate_hidden_dim_fails_before_descriptors():
+    x, w13, w2, ids, wts, out = _cpu_problem()
+    bad_gate = torch.zeros(4, 32, 96, dtype=torch.bfloat16)
+    v = moe.w13_from_views(bad_gate, w13[:, 32:])
+    # host tensors: validation must reject before touching any device or launching
+    assert _status(x, v, w2, ids, wts, out) == 2
+    assert moe.last_launch_count() == 0
+
+
+def test_validation_errors():
+    x, w13, w2, ids, wts, out = _cpu_problem()
+    v = moe.w13_from_packed(w13)
+    assert _status(x, v, w2[:, :, :16], ids, wts, out) == 2             # w2 cols != I
+    assert _status(x, v, w2, ids[:3], wts, out) == 2                      # ids rows != T
+    assert _status(x.float(), v, w2, ids, wts, out) == 3                  # x must be bf16
+    assert _status(x, v, w2, ids.float(), wts, out) == 3                  # ids int32/int64
+    assert _status(x, v, w2, ids, wts.double(), out) == 3                 # weights f32
+    ids_many = torch.zeros(8, 33, dtype=torch.int32)
+    assert _status(x, v, w2, ids_many, torch.zeros(8, 33), out) == 1      # k > 32
+    # weight views with a non-unit inner stride cannot be read by the copy engine: loud error
+    gt = torch.zeros(4, 64, 32, dtype=torch.bfloat16).transpose(1, 2)
+    vt = moe.w13_from_views(gt, gt)
+    assert _status(x, vt, w2, ids, wts, out) == 4
+    # a weight base that is not 16-byte aligned
+    flat = torch.zeros(4 * 64 * 64 + 8, dtype=torch.bfloat16)
+    mis = flat[1:1 + 4 * 64 * 64].view(4, 64, 64)
+    assert _status(x, moe.w13_from_packed(mis), w2, ids, wts, out) == 4
+    # workspace too small is reported before any device work
+    ws = torch.zeros(16, dtype=torch.uint8)
+    assert _status(x, v, w2, ids, wts, out, ws) == 5
+
+
+def test_zero_tokens_is_a_noop():
+    x, w13, w2, ids, wts, out = _cpu_problem(T=0)
+    assert _status(x, moe.w13_from_packed(w13), w2, ids, wts, out) == 0
+    assert moe.last_launch_count() == 0
+
+
+def test_router_replay_slice_stride():
+    g = json.load(open(os.path.join(GOLD, "router_replay_stride.json")))
+    ids, _ = wl.route_zipf_layers(16, 128, g["top_k"], layers=g["num_layers"], seed=7)
+    sl = ids[:, 23, :]
+    assert sl.stride(0) == g["token_stride"] and sl.stride(1) == 1
+    d = _abi.desc(sl)
+    assert d.strides[0] == 368 and d.data == ids.data_ptr() + 23 * 8 * 4
+    # every token picks top_k distinct experts
+    assert all(len(set(r.tolist())) == g["top_k"] for r in sl)
+
+
+def test_product_path_has_no_oracle_dependency():
+    pkg = os.path.join(ROOT, "mixture_experts_layer_46_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                src = open(os.path.join(dirpath, fn)).read()
+                assert "import oracle" not in src and "from oracle" not in src, fn
+                assert "moe_oracle" not in src, fn

@@ -1,0 +1,261 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Bars (fixed by the benchmark spec of the method):
+  * align: counts, offsets, slot permutation and block map bit-exact;
+  * forward (bf16): max|y - ref| / max|ref| <= 1e-2;
+  * strided packed w13 views vs .contiguous() copies: bit-identical outputs
+    (Liger-Kernel PR #1377, "Testing Done": packed views match contiguous weights);
+  * run-to-run bit-identical.
+"""
+
+import pytest
+import torch
+
+import mixture_experts_layer_46_b200 as moe
+import oracle
+from mixture_experts_layer_46_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+BF16_TOL = 1e-2
+
+
+def rel_err(got: torch.Tensor, ref: torch.Tensor) -> float:
+    got = got.double().cpu()
+    ref = ref.double().cpu()
+    return (got - ref).abs().max().item() / ref.abs().max().item()
+
+
+def make_case(T, H, I, E, k, seed=0, device="cuda"):
+    x = wl.make_x(T, H, seed=seed + 1)
+    w13, w2 = wl.make_weights_bf16(E, I, H, seed=seed)
+    ids, wts = wl.route_softmax_topk(T, E, k, seed=seed + 2)
+    return {"x": x, "w13": w13, "w2": w2, "ids": ids, "wts": wts}
+
+
+def to_cuda(case):
+    return {k: v.cuda() for k, v in case.items()}
+
+
+def run_gpu(c, contiguous=False, out=None, ws=None):
+    gate, up = wl.gate_up_views(c["w13"])
+    if contiguous:
+        # descriptors hold raw pointers: keep the copies alive until the forward is done
+        gc, uc = gate.contiguous(), up.contiguous()
+        v = moe.w13_from_views(gc, uc)
+        res = moe.forward(c["x"], v, c["w2"], c["ids"], c["wts"], out=out, workspace=ws)
+        torch.cuda.synchronize()
+        del gc, uc
+        return res
+    v = moe.w13_from_packed(c["w13"])
+    res = moe.forward(c["x"], v, c["w2"], c["ids"], c["wts"], out=out, workspace=ws)
+    torch.cuda.synchronize()
+    return res
+
+
+def run_oracle(case, tokens=None):
+    gate, up = wl.gate_up_views(case["w13"])
+    ref, _ = oracle.moe_forward(case["x"], gate, up, case["w2"], case["ids"], case["wts"],
+                                tokens=tokens)
+    return ref
+
+
+# ----------------------------------------------------------------------------- align
+
+@pytest.mark.parametrize("T,E,k,bm,idt", [
+    (64, 8, 2, 128, torch.int32),      # tiny config
+    (1, 128, 8, 128, torch.int32),     # decode
+    (37, 16, 4, 16, torch.int64),      # int64 ids, small block
+    (4096, 128, 8, 128, torch.int32),  # multi-CTA path (32768 slots)
+    (3000, 513, 11, 64, torch.int32),  # shared-expert-fused routing width
+])
+def test_align_bit_exact(T, E, k, bm, idt):
+    if E == 513:
+        ids, _ = wl.route_shared_expert(T, 512, 10, seed=5)
+    else:
+        ids, _ = wl.route_softmax_topk(T, E, k, seed=T)
+    ids = ids.to(idt)
+    ref = oracle.moe_align(ids, E, bm)
+    got = moe.align(ids.cuda(), E, bm)
+    torch.cuda.synchronize()
+    assert got["counts"].cpu().tolist() == ref["counts"].tolist()
+    assert got["offsets"].cpu().tolist() == ref["offsets"].tolist()
+    assert got["num_blocks"] == ref["num_blocks"]
+    assert torch.equal(got["sorted"].cpu(), ref["sorted"])
+    assert torch.equal(got["block_expert"].cpu(), ref["block_expert"])
+
+
+def test_align_strided_slice_and_bad_ids():
+    ids_all, _ = wl.route_zipf_layers(2000, 128, 8, layers=46, seed=7)
+    assert ids_all[:, 23, :].stride() == (368, 1)
+    ids_all[5, 23, 3] = -1
+    ids_all[17, 23, 0] = 128
+    ids = ids_all[:, 23, :]
+    ref = oracle.moe_align(ids, 128, 128)
+    moe.device_errors()  # clear
+    got = moe.align(ids_all.cuda()[:, 23, :], 128, 128)
+    nbad, nto = moe.device_errors()
+    assert torch.equal(got["sorted"].cpu(), ref["sorted"])
+    assert got["counts"].cpu().tolist() == ref["counts"].tolist()
+    assert nbad == 2 and nto == 0
+
+
+# ----------------------------------------------------------------------------- forward
+
+def test_forward_tiny_config_full_oracle():
+    s = wl.TINY
+    case = make_case(s.T, s.H, s.I, s.E, s.k)
+    ref = run_oracle(case)
+    got = run_gpu(to_cuda(case))
+    assert rel_err(got, ref) <= BF16_TOL
+    assert moe.last_launch_count() >= 5
+
+
+@pytest.mark.parametrize("T,H,I,E,k", [
+    (300, 512, 384, 16, 4),   # several row blocks, 3 gate/up column tiles, 2 down tiles
+    (77, 288, 96, 6, 3),      # ragged K (288 = 4.5 x 64), partial N tiles for both GEMMs
+    (1, 256, 128, 8, 2),      # one token
+    (513, 256, 128, 4, 1),    # top-1, >4 row blocks per expert
+])
+def test_forward_ragged_shapes(T, H, I, E, k):
+    case = make_case(T, H, I, E, k, seed=T)
+    ref = run_oracle(case)
+    got = run_gpu(to_cuda(case))
+    assert rel_err(got, ref) <= BF16_TOL
+
+
+def test_strided_equals_contiguous_bit_identical_and_deterministic():
+    case = to_cuda(make_case(200, 512, 256, 8, 2, seed=3))
+    a = run_gpu(case)
+    b = run_gpu(case, contiguous=True)
+    c = run_gpu(case)
+    assert torch.equal(a, b)
+    assert torch.equal(a, c)
+
+
+def test_expert_addressing_regression_distinct_constants():
+    # every expert's gate and up hold different values; addressing experts by
+    # e * I / TileN (instead of the real stride) would mix them up
+    T, H, I, E, k = 64, 256, 128, 4, 2
+    case = make_case(T, H, I, E, k, seed=9)
+    w13 = case["w13"]
+    for e in range(E):
+        w13[e, :I] *= (1.0 + 0.25 * e)
+        w13[e, I:] *= (-0.5 - 0.125 * e)
+    ref = run_oracle(case)
+    got = run_gpu(to_cuda(case))
+    assert rel_err(got, ref) <= BF16_TOL
+
+
+def test_strided_activations_ids_weights_and_out():
+    T, H, I, E, k, L = 96, 256, 128, 8, 4, 5
+    case = make_case(T, H, I, E, k, seed=13)
+    ids_all = torch.randint(0, E, (T, L, k), generator=torch.Generator().manual_seed(1))
+    w_all = torch.rand(T, L, k, generator=torch.Generator().manual_seed(2))
+    ids_all[:, 2, :] = case["ids"].long()
+    w_all[:, 2, :] = case["wts"]
+    ref = run_oracle(case)
+    c = to_cuda(case)
+    x_dev = case["x"].t().contiguous().cuda().t()
+    assert x_dev.stride() == (1, T)
+    ids_dev = ids_all.cuda()[:, 2, :]
+    w_dev = w_all.cuda()[:, 2, :]
+    out_big = torch.zeros(T, 2 * H, dtype=torch.bfloat16, device="cuda")
+    out = out_big[:, ::2]
+    v = moe.w13_from_packed(c["w13"])
+    moe.forward(x_dev, v, c["w2"], ids_dev, w_dev, out=out)
+    torch.cuda.synchronize()
+    assert rel_err(out, ref) <= BF16_TOL
+    assert torch.all(out_big[:, 1::2] == 0)
+
+
+def test_out_of_range_ids_skipped_and_counted():
+    T, H, I, E, k = 40, 256, 128, 8, 2
+    case = make_case(T, H, I, E, k, seed=21)
+    case["ids"][3, 1] = -1
+    case["ids"][7, 0] = E
+    ref = run_oracle(case)
+    moe.device_errors()
+    got = run_gpu(to_cuda(case))
+    nbad, nto = moe.device_errors()
+    assert rel_err(got, ref) <= BF16_TOL
+    assert nbad == 2 and nto == 0
+
+
+def test_forward_ws_allocates_nothing_and_matches_forward():
+    case = to_cuda(make_case(128, 512, 256, 8, 4, seed=31))
+    nbytes = moe.workspace_bytes(128, 512, 256, 8, 4)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    a = run_gpu(case, ws=ws)
+    out = torch.empty_like(a)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    alloc0 = torch.cuda.memory_allocated()
+    run_gpu(case, ws=ws, out=out)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert torch.cuda.memory_allocated() == alloc0
+    assert free1 == free0
+    assert torch.equal(a, out)
+    b = run_gpu(case)
+    assert torch.equal(a, b)
+
+
+def test_forward_host_matches_device():
+    case = make_case(50, 256, 128, 8, 2, seed=41)
+    c = to_cuda(case)
+    dev = run_gpu(c)
+    out_h = torch.empty(50, 256, dtype=torch.bfloat16).pin_memory()
+    x_h = case["x"].pin_memory()
+    ids_h = case["ids"].pin_memory()
+    w_h = case["wts"].pin_memory()
+    moe.forward_host(x_h, moe.w13_from_packed(c["w13"]), c["w2"], ids_h, w_h, out_h)
+    assert torch.equal(out_h, dev.cpu())
+
+
+def test_zero_tokens():
+    case = to_cuda(make_case(0, 256, 128, 8, 2))
+    out = run_gpu(case)
+    assert out.shape == (0, 256)
+
+
+# ----------------------------------------------------------------------------- full size
+
+def _sample_tokens(T, n, seed):
+    g = torch.Generator().manual_seed(seed)
+    idx = torch.randperm(T, generator=g)[:n]
+    edge = torch.tensor([0, 1, T - 2, T - 1])
+    return torch.unique(torch.cat([idx, edge]))
+
+
+@pytest.mark.slow
+def test_qwen3_235b_shape_full_size_sampled():
+    s = wl.QWEN3_235B
+    w13, w2 = wl.make_weights_bf16(s.E, s.I, s.H, seed=0, device="cuda")
+    x = wl.make_x(s.T, s.H, seed=1, device="cuda")
+    ids, wts = wl.route_softmax_topk(s.T, s.E, s.k, seed=2, device="cuda")
+    c = {"x": x, "w13": w13, "w2": w2, "ids": ids, "wts": wts}
+    a = run_gpu(c)
+    b = run_gpu(c, contiguous=True)
+    assert torch.equal(a, b)
+    toks = _sample_tokens(s.T, 48, 0)
+    case_cpu = {"x": x.cpu(), "w13": w13.cpu(), "w2": w2.cpu(), "ids": ids.cpu(), "wts": wts.cpu()}
+    ref = run_oracle(case_cpu, tokens=toks)
+    assert rel_err(a.cpu()[toks], ref) <= BF16_TOL
+
+
+@pytest.mark.slow
+def test_glm45_air_shape_skewed_strided_ids_sampled():
+    s = wl.GLM45_AIR
+    w13, w2 = wl.make_weights_bf16(s.E, s.I, s.H, seed=0, device="cuda")
+    x = wl.make_x(s.T, s.H, seed=1, device="cuda")
+    ids_all, w_all = wl.route_zipf_layers(s.T, s.E, s.k, layers=46, seed=7, device="cuda")
+    ids, wts = ids_all[:, 23, :], w_all[:, 23, :]
+    assert ids.stride() == (368, 1)
+    c = {"x": x, "w13": w13, "w2": w2, "ids": ids, "wts": wts}
+    a = run_gpu(c)
+    toks = _sample_tokens(s.T, 32, 1)
+    case_cpu = {"x": x.cpu(), "w13": w13.cpu(), "w2": w2.cpu(), "ids": ids_all.cpu()[:, 23, :],
+                "wts": w_all.cpu()[:, 23, :]}
+    ref = run_oracle(case_cpu, tokens=toks)
+    assert rel_err(a.cpu()[toks], ref) <= BF16_TOL
