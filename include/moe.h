@@ -159,6 +159,26 @@ moe_status_t moe_align(const moe_tensor_t* topk_ids, int64_t E, int32_t block_m,
                        int32_t* num_blocks, void* workspace, size_t workspace_bytes,
                        moe_stream_t stream);
 
+/* moe_align without a workspace argument and without any allocation.  The
+ * pages have no counterpart to this entry point; it exists for callers that
+ * cannot allocate device memory at all — for instance a plugin running inside
+ * a serving engine that has already split the GPU's memory between its own
+ * pools, or a component whose host framework only hands it the input and
+ * output tensors — and so can neither call cudaMalloc nor pass a workspace.
+ * Arguments and outputs are those of moe_align.  The scratch lives in a fixed
+ * 5 MiB array inside the library (held on every GPU that loads it until the
+ * process exits), which limits the problem to T*k <= 1,048,576 slots; larger
+ * problems return MOE_ERR_WORKSPACE_TOO_SMALL and nothing is launched.
+ * The first call on each device looks up that array's device address (a
+ * one-time host-side query); make that first call before any stream capture.
+ * All calls share the array and it keeps the previous call's contents (the
+ * kernels rewrite everything they read).  Calls whose GPU work overlaps, e.g.
+ * on two unordered streams, race on it.  Out-of-range ids are skipped but not
+ * counted in the device error word. */
+moe_status_t moe_align_noalloc(const moe_tensor_t* topk_ids, int64_t E, int32_t block_m,
+                               int32_t* counts, int32_t* offsets, int32_t* sorted_slots,
+                               int32_t* block_expert, int32_t* num_blocks, moe_stream_t stream);
+
 /* MXFP4 quantisation of the rows of src [.., K] (bf16 or f32, inner stride 1,
  * K % 32 == 0) into dst (MOE_E2M1X2 with dst->scale set): per 32 consecutive
  * elements, scale exponent s = clamp(floor(log2(amax)) - 2, -127, 127) stored as

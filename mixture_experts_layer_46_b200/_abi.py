@@ -27,7 +27,7 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_SHAPE_MISMATCH",
 EXPORTS = ("moe_status_string", "moe_last_cuda_error", "moe_w13_from_packed",
            "moe_workspace_bytes", "moe_forward_ws", "moe_forward", "moe_forward_host",
            "moe_align", "moe_quantize_mxfp4", "moe_get_device_errors", "moe_last_launch_count",
-           "moe_profile_enable", "moe_profile_read", "moe_version")
+           "moe_profile_enable", "moe_profile_read", "moe_version", "moe_align_noalloc")
 STEP_NAMES = ("align", "permute", "gemm1_swiglu", "gemm2_weighted", "combine")
 
 
@@ -95,6 +95,9 @@ def load() -> ctypes.CDLL:
             lib.moe_quantize_mxfp4.argtypes = [P(MoeTensor), P(MoeTensor), vp]
             lib.moe_get_device_errors.restype = ctypes.c_int
             lib.moe_get_device_errors.argtypes = [vp, P(ctypes.c_uint32), P(ctypes.c_uint32)]
+            lib.moe_align_noalloc.restype = ctypes.c_int
+            lib.moe_align_noalloc.argtypes = [P(MoeTensor), ctypes.c_int64, ctypes.c_int32, vp, vp,
+                                              vp, vp, vp, vp]
             lib.moe_profile_enable.restype = ctypes.c_int
             lib.moe_profile_enable.argtypes = [ctypes.c_int32]
             lib.moe_profile_read.restype = ctypes.c_int

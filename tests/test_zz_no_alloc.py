@@ -1,0 +1,85 @@
+"""moe_align_noalloc: the align step for callers that cannot allocate device
+memory (e.g. a plugin inside an engine whose memory is already split between
+its own pools) and so cannot pass a workspace either.  It keeps its scratch
+in a fixed array inside the library.
+
+Checked here through the C ABI: on two calls in a row (different routing, so
+the second call starts from the first call's leftover scratch) its outputs
+equal those of moe_align, which uses a caller-provided workspace, bit for bit
+(align is integer work, so the tolerance is exact equality).  The problem size
+uses the multi-CTA path, so both scratch regions are exercised.  Oversized
+problems are refused.
+
+This file sorts last so a run that stops at the first failure has already run
+every other test.
+"""
+
+import ctypes
+
+import pytest
+import torch
+
+import mixture_experts_layer_46_b200 as moe
+from mixture_experts_layer_46_b200 import _abi
+from mixture_experts_layer_46_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+
+def _noalloc(ids: torch.Tensor, E: int, bm: int):
+    T, k = ids.shape
+    S = T * k
+    pmax = S + min(E, S) * (bm - 1) + bm
+    dev = ids.device
+    counts = torch.full((E,), -1, dtype=torch.int32, device=dev)
+    offsets = torch.full((E + 1,), -1, dtype=torch.int32, device=dev)
+    sorted_ = torch.full((pmax,), -7, dtype=torch.int32, device=dev)
+    block_expert = torch.full((pmax // bm + 1,), -7, dtype=torch.int32, device=dev)
+    nb = torch.zeros(1, dtype=torch.int32, device=dev)
+    d = _abi.desc(ids)
+    rc = moe.load().moe_align_noalloc(ctypes.byref(d), E, bm, counts.data_ptr(), offsets.data_ptr(),
+                                      sorted_.data_ptr(), block_expert.data_ptr(), nb.data_ptr(),
+                                      torch.cuda.current_stream().cuda_stream)
+    assert rc == 0, _abi.STATUS.get(rc, rc)
+    torch.cuda.synchronize()
+    P = int(offsets[E].item())
+    n = int(nb.item())
+    return {"counts": counts, "offsets": offsets, "sorted": sorted_[:P],
+            "block_expert": block_expert[:n], "num_blocks": n}
+
+
+def _same(a, b):
+    assert a["num_blocks"] == b["num_blocks"]
+    for key in ("counts", "offsets", "sorted", "block_expert"):
+        assert torch.equal(a[key].cpu(), b[key].cpu()), key
+
+
+def test_noalloc_align_matches_workspace_align_twice():
+    E, bm = 128, 128
+    ids1, _ = wl.route_softmax_topk(4096, E, 8, seed=11, device="cuda")
+    ids_all, _ = wl.route_zipf_layers(3000, E, 8, layers=46, seed=12, device="cuda")
+    ids2 = ids_all[:, 23, :]  # strided slice, token stride 368
+    first = _noalloc(ids1, E, bm)
+    ref1 = moe.align(ids1, E, bm)
+    torch.cuda.synchronize()
+    _same(first, ref1)
+    free0, _ = torch.cuda.mem_get_info()
+    second = _noalloc(ids2, E, bm)
+    free1, _ = torch.cuda.mem_get_info()
+    ref2 = moe.align(ids2, E, bm)
+    torch.cuda.synchronize()
+    _same(second, ref2)
+    assert free1 == free0  # the call itself allocated nothing
+
+
+def test_noalloc_align_refuses_oversized_problem():
+    T, k = (1 << 20) // 8 + 1, 8  # one token past the fixed scratch
+    ids = torch.zeros(T, k, dtype=torch.int32, device="cuda")
+    d = _abi.desc(ids)
+    dummy = torch.zeros(16, dtype=torch.int32, device="cuda")
+    p = dummy.data_ptr()
+    rc = moe.load().moe_align_noalloc(ctypes.byref(d), 8, 128, p, p, p, p, p,
+                                      torch.cuda.current_stream().cuda_stream)
+    assert rc == 5  # MOE_ERR_WORKSPACE_TOO_SMALL, nothing launched
+    torch.cuda.synchronize()
+    assert torch.all(dummy == 0)
