@@ -43,12 +43,20 @@ WORKLOADS = {
     "qwen3-235b": dict(H=4096, I=1536, E=128, k=8, T=4096, routing="softmax"),
     "glm45-air": dict(H=4096, I=1408, E=128, k=8, T=16384, routing="zipf-layer-slice"),
     "tiny": dict(H=256, I=128, E=8, k=2, T=64, routing="softmax"),
+    "qwen35-tp2-mxfp4": dict(H=4096, I=512, E=512, k=10, T=4096, routing="softmax", mxfp4=True),
+    "qwen35-tp2-mxfp4-shared": dict(H=4096, I=512, E=513, k=11, T=4096, routing="shared",
+                                    mxfp4=True),
 }
 
 # DRAM traffic per launch of the dominant kernel from an ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed to the hash of the kernel
 # source it was taken on; reported as null once the source has changed.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # profiles/grouped_gemm_bf16_qwen3shape_E32_T1024.md: 988.6 MB read + 27.7 MB written on
+    # the E=32, T=1024 case, scaled x4 (experts) to the E=128, T=4096 launch
+    "gemm1_swiglu": {"bytes_per_launch": 4.0 * (988.558080e6 + 27.661568e6), "src": "5c4c0d592bfeac3f",
+                     "workload": "qwen3-235b T=4096"},
+}
 
 
 def kernel_src_hash() -> str:
@@ -69,24 +77,52 @@ def peaks():
 
 
 def workload_name(w) -> str:
-    return (f"moe-layer bf16 T={w['T']} H={w['H']} I={w['I']} E={w['E']} top_k={w['k']} "
+    dt = "mxfp4 (e2m1 + e8m0 per 1x32)" if w.get("mxfp4") else "bf16"
+    return (f"moe-layer {dt} T={w['T']} H={w['H']} I={w['I']} E={w['E']} top_k={w['k']} "
             f"packed-strided-w13 routing={w['routing']}")
+
+
+def make_mx_weights(w, device):
+    """MXFP4 weights: fp32 N(0, 1/sqrt(fan_in)) drawn expert by expert and quantised
+    with the library's 1x32 quantiser (the bench times the forward, not this)."""
+    import mixture_experts_layer_46_b200 as moe
+    from mixture_experts_layer_46_b200 import workloads as wl
+
+    E, I, H = w["E"], w["I"], w["H"]
+    c13 = torch.empty(E, 2 * I, H // 2, dtype=torch.uint8, device=device)
+    s13 = torch.empty(E, 2 * I, H // 32, dtype=torch.uint8, device=device)
+    c2 = torch.empty(E, H, I // 2, dtype=torch.uint8, device=device)
+    s2 = torch.empty(E, H, I // 32, dtype=torch.uint8, device=device)
+    for e, w13e, w2e in wl.iter_weights_fp32(E, I, H, seed=0, device=device):
+        c13[e], s13[e] = moe.quantize_mxfp4(w13e)
+        c2[e], s2[e] = moe.quantize_mxfp4(w2e)
+    return c13, s13, c2, s2
 
 
 def make_inputs(w, device, seed_offset=0):
     from mixture_experts_layer_46_b200 import workloads as wl
 
-    w13, w2 = wl.make_weights_bf16(w["E"], w["I"], w["H"], seed=0, device=device)
+    if w.get("mxfp4"):
+        c13, s13, c2, s2 = make_mx_weights(w, device)
+        w13, w2 = c13, c2
+        scales = (s13, s2)
+    else:
+        w13, w2 = wl.make_weights_bf16(w["E"], w["I"], w["H"], seed=0, device=device)
+        scales = None
     x = wl.make_x(w["T"], w["H"], seed=1 + seed_offset, device=device)
     if w["routing"] == "softmax":
         ids, wts = wl.route_softmax_topk(w["T"], w["E"], w["k"], seed=2 + seed_offset, device=device)
+        keep = None
+    elif w["routing"] == "shared":
+        ids, wts = wl.route_shared_expert(w["T"], w["E"] - 1, w["k"] - 1, seed=2 + seed_offset,
+                                          device=device)
         keep = None
     else:
         ids_all, w_all = wl.route_zipf_layers(w["T"], w["E"], w["k"], layers=46, seed=7 + seed_offset,
                                               device=device)
         ids, wts = ids_all[:, 23, :], w_all[:, 23, :]
         keep = (ids_all, w_all)
-    return {"x": x, "w13": w13, "w2": w2, "ids": ids, "wts": wts, "keep": keep}
+    return {"x": x, "w13": w13, "w2": w2, "ids": ids, "wts": wts, "keep": keep, "scales": scales}
 
 
 def algorithmic(w, ids):
@@ -96,10 +132,12 @@ def algorithmic(w, ids):
     valid = idc[(idc >= 0) & (idc < E)]
     n_slots = int(valid.numel())
     n_act = int(torch.unique(valid).numel())
+    wbytes = (0.5 + 1.0 / 32.0) if w.get("mxfp4") else 2.0   # per weight element
     flops = 6.0 * H * I * n_slots
-    bytes_total = 3.0 * I * H * 2 * n_act + 2.0 * T * H * 2 + 8.0 * T * k
+    bytes_total = 3.0 * I * H * wbytes * n_act + 2.0 * T * H * 2 + 8.0 * T * k
     g1_flops = 4.0 * H * I * n_slots
-    g1_bytes = 2.0 * I * H * 2 * n_act + T * H * 2.0
+    abytes = (0.5 + 1.0 / 32.0) if w.get("mxfp4") else 2.0
+    g1_bytes = 2.0 * I * H * wbytes * n_act + T * H * abytes
     return dict(flops=flops, bytes=bytes_total, gemm1_flops=g1_flops, gemm1_bytes=g1_bytes,
                 slots=n_slots, active_experts=n_act)
 
@@ -162,47 +200,60 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def oracle_tokens_per_s(inp, w, budget_s, cores):
-    """The fp64 oracle on a bounded sample of the workload's tokens."""
+def oracle_runner(inp, w):
+    """A closure that runs the fp64 oracle on a list of token indices of the workload."""
     import oracle
     from mixture_experts_layer_46_b200 import workloads as wl
 
-    cpu = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    cpu = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()
+           if k != "scales"}
     if inp["keep"] is not None:
         ids_all, w_all = (t.cpu() for t in inp["keep"])
         cpu["ids"], cpu["wts"] = ids_all[:, 23, :], w_all[:, 23, :]
     gate, up = wl.gate_up_views(cpu["w13"])
+    scales = None
+    if w.get("mxfp4"):
+        s13, s2 = (t.cpu() for t in inp["scales"])
+        sg, su = wl.gate_up_views(s13)
+        scales = (sg, su, s2)
+
+    def run(tokens, nthreads):
+        oracle.moe_forward(cpu["x"], gate, up, cpu["w2"], cpu["ids"], cpu["wts"], scales=scales,
+                           tokens=tokens, nthreads=nthreads)
+
+    return run
+
+
+def oracle_tokens_per_s(inp, w, budget_s, cores):
+    """The fp64 oracle on a bounded sample of the workload's tokens."""
+    run = oracle_runner(inp, w)
     g = torch.Generator().manual_seed(123)
     order = torch.randperm(w["T"], generator=g)
     # calibrate with one token per core, then size the sample to the budget
     n = max(1, cores)
     t0 = time.perf_counter()
-    oracle.moe_forward(cpu["x"], gate, up, cpu["w2"], cpu["ids"], cpu["wts"], tokens=order[:n],
-                       nthreads=cores)
+    run(order[:n], cores)
     dt = time.perf_counter() - t0
     reps = max(1, int(budget_s / max(dt, 1e-6)))
     n2 = min(w["T"], n * reps)
     t0 = time.perf_counter()
-    oracle.moe_forward(cpu["x"], gate, up, cpu["w2"], cpu["ids"], cpu["wts"], tokens=order[:n2],
-                       nthreads=cores)
+    run(order[:n2], cores)
     dt2 = time.perf_counter() - t0
-    return n2 / dt2, n2, dt2, (cpu, gate, up, order)
+    return n2 / dt2, n2, dt2
 
 
 def run_reference(args, w, rank):
     if rank != 0:
         return
-    import oracle
-
     cores = os.cpu_count() or 1
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = make_inputs(w, dev)
-    _, _, _, (cpu, gate, up, order) = oracle_tokens_per_s(inp, w, 0.0, cores)
+    run = oracle_runner(inp, w)
+    order = torch.randperm(w["T"], generator=torch.Generator().manual_seed(123))
     per_step_budget = max(0.5, 150.0 / max(1, args.steps + args.warmup))
     # tokens per step: one per core, grown while it fits the per-step budget
     t0 = time.perf_counter()
-    oracle.moe_forward(cpu["x"], gate, up, cpu["w2"], cpu["ids"], cpu["wts"], tokens=order[:cores],
-                       nthreads=cores)
+    run(order[:cores], cores)
     dt = time.perf_counter() - t0
     n = max(1, min(w["T"], int(cores * max(1.0, per_step_budget / max(dt, 1e-6)))))
     times = []
@@ -211,8 +262,7 @@ def run_reference(args, w, rank):
         if toks.numel() < n:
             toks = order[:n]
         t0 = time.perf_counter()
-        oracle.moe_forward(cpu["x"], gate, up, cpu["w2"], cpu["ids"], cpu["wts"], tokens=toks,
-                           nthreads=cores)
+        run(toks, cores)
         if step >= args.warmup:
             times.append(time.perf_counter() - t0)
     sec = sum(times) / len(times)
@@ -223,8 +273,7 @@ def run_reference(args, w, rank):
             "data": "synthetic (seeded N(0,1) activations, N(0,1/sqrt(fan_in)) weights)",
             "config": {"workload": workload_name(w), "tokens_per_step_sample": n,
                        "l2": "n/a (CPU)"},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.max_threads() if cores <= 0 else cores,
-                             "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": f"{n} of {w['T']} tokens per step (all their {w['k']} slots), fp64 C++ loop, OpenMP over tokens"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -238,6 +287,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="qwen3-235b", choices=sorted(WORKLOADS))
     ap.add_argument("--T", type=int, default=None)
+    ap.add_argument("--E", type=int, default=None, help="override the expert count (profiling)")
     ap.add_argument("--sweep", default=None, help="write a token-sweep JSONL here (extra lines)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -246,6 +296,8 @@ def main():
     w = dict(WORKLOADS[args.workload])
     if args.T is not None:
         w["T"] = args.T
+    if args.E is not None:
+        w["E"] = args.E
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -276,15 +328,17 @@ def main():
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
     inp = make_inputs(w, dev)
-    v13 = moe.w13_from_packed(inp["w13"])
-    ws = torch.empty(moe.workspace_bytes(w["T"], w["H"], w["I"], w["E"], w["k"]), dtype=torch.uint8,
-                     device=dev)
+    mx = bool(w.get("mxfp4"))
+    s13, s2 = inp["scales"] if mx else (None, None)
+    v13 = moe.w13_from_packed(inp["w13"], s13)
+    ws = torch.empty(moe.workspace_bytes(w["T"], w["H"], w["I"], w["E"], w["k"], mxfp4=mx),
+                     dtype=torch.uint8, device=dev)
     out = torch.empty(w["T"], w["H"], dtype=torch.bfloat16, device=dev)
     flush = wl.l2_flush_buffer(dev)
 
     def step():
         moe.forward(inp["x"], v13, inp["w2"], inp["ids"], inp["wts"], out=out, workspace=ws,
-                    stream=stream)
+                    stream=stream, w2_scale=s2)
 
     for _ in range(args.warmup):
         step()
@@ -333,13 +387,13 @@ def main():
     w_h = inp["wts"].contiguous().cpu().pin_memory()
     out_h = torch.empty(w["T"], w["H"], dtype=torch.bfloat16).pin_memory()
     for _ in range(2):
-        moe.forward_host(x_h, v13, inp["w2"], ids_h, w_h, out_h, stream=stream)
+        moe.forward_host(x_h, v13, inp["w2"], ids_h, w_h, out_h, stream=stream, w2_scale=s2)
     e2e_ms = []
     for i in range(min(args.steps, 50)):
         flush.fill_(i & 0xff)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        moe.forward_host(x_h, v13, inp["w2"], ids_h, w_h, out_h, stream=stream)
+        moe.forward_host(x_h, v13, inp["w2"], ids_h, w_h, out_h, stream=stream, w2_scale=s2)
         e1.record(stream)
         e1.synchronize()
         e2e_ms.append(e0.elapsed_time(e1))
@@ -353,6 +407,9 @@ def main():
 
     # ---------------------------------------------------------------- roofline
     hbm, tf_burst, tf_sus, src = peaks()
+    if mx:
+        # FP4 dense peak = measured bf16 x the nominal 9 / 2.25 PFLOP/s ratio (assumed)
+        tf_burst = tf_burst * 4.0
     alg = algorithmic(w, inp["ids"])
     g1_ms = brk.get("gemm1_swiglu", float("nan"))
     t_tc = alg["gemm1_flops"] / (tf_burst * 1e12)
@@ -365,15 +422,20 @@ def main():
                 "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     tr = NCU_TRAFFIC.get("gemm1_swiglu")
-    roof["traffic"] = tr["bytes_per_launch"] if tr and tr.get("src") == kernel_src_hash() else None
-    roof["kernel"] = "gemm1_swiglu (grouped gate/up GEMM + SwiGLU, tcgen05)"
-    roof["peak_source"] = f"{src} (MEASURED_PEAKS.json burst)" if src == "measured" else "fallback"
+    same_case = (args.workload == "qwen3-235b" and w["T"] == 4096 and w["E"] == 128)
+    roof["traffic"] = (tr["bytes_per_launch"] if tr and same_case and tr.get("src") == kernel_src_hash()
+                       else None)
+    roof["kernel"] = ("gemm1_swiglu (grouped gate/up GEMM + SwiGLU, tcgen05 "
+                      + ("kind::mxf4 block-scaled)" if mx else "kind::f16)"))
+    roof["peak_source"] = (f"{src} (MEASURED_PEAKS.json burst)" if src == "measured" else "fallback")
+    if mx and roof["bound"] == "tensor":
+        roof["peak_source"] += " x4 nominal FP4/bf16 ratio (FP4 peak not measured)"
     t_roof_layer = max(alg["flops"] / (tf_burst * 1e12), alg["bytes"] / (hbm * 1e9))
     layer_frac = t_roof_layer / (ms * 1e-3)
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16",
+            "vs_baseline": None, "dtype": "e2m1/e8m0 (fp32 accumulate)" if mx else "bf16",
             "data": "synthetic (seeded N(0,1) activations, N(0,1/sqrt(fan_in)) random-init weights)",
             "config": {"workload": workload_name(w), "tokens_per_gpu": w["T"],
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
@@ -394,7 +456,7 @@ def main():
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cores = os.cpu_count() or 1
-        tps, n, dt, _ = oracle_tokens_per_s(inp, w, 12.0, cores)
+        tps, n, dt = oracle_tokens_per_s(inp, w, 12.0, cores)
         line["cpu_baseline"] = {"value": tps, "unit": UNIT, "cores": cores, "kind": "oracle",
                                 "sample": f"{n} of {w['T']} tokens (all their slots) in {dt:.1f} s, fp64 C++ loop, OpenMP over tokens"}
 

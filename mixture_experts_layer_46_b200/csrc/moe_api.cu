@@ -217,9 +217,14 @@ moe_status_t validate(const moe_tensor_t* x, const moe_w13_t* w13, const moe_ten
     return MOE_ERR_UNSUPPORTED_LAYOUT;
   if (wd == MOE_E2M1X2) {
     if (!gate->scale || !up->scale || !w2->scale) return MOE_ERR_INVALID_ARG;
-    if (gate->scale_strides[2] != 1 || up->scale_strides[2] != 1 || w2->scale_strides[2] != 1)
-      return MOE_ERR_UNSUPPORTED_LAYOUT;
-    if (H % 128 != 0 || I % 128 != 0) return MOE_ERR_SHAPE_MISMATCH;
+    // scales are read 8 blocks (8 bytes) at a time per row and k-step
+    for (const moe_tensor_t* t : {gate, up, w2}) {
+      if (t->scale_strides[2] != 1 || t->scale_strides[1] % 8 != 0 ||
+          t->scale_strides[0] % 8 != 0 || reinterpret_cast<uintptr_t>(t->scale) % 8 != 0)
+        return MOE_ERR_UNSUPPORTED_LAYOUT;
+    }
+    // k-steps of 256 elements; GEMM1 column tiles of 64, GEMM2 column tiles of 128
+    if (H % 256 != 0 || I % 256 != 0) return MOE_ERR_SHAPE_MISMATCH;
   }
   if (host_io) {
     if (x->strides[1] != 1 || ids->strides[1] != 1 || wts->strides[1] != 1 ||
@@ -326,6 +331,108 @@ WsLayout make_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, bool
 
 namespace {
 
+// MXFP4: align -> permute+quantise -> block-scaled GEMM1 (+SwiGLU, requantise)
+// -> block-scaled GEMM2 (+routing weight) -> combine.
+moe_status_t forward_mxfp4(const moe_tensor_t* x, const moe_w13_t* w13, const moe_tensor_t* w2,
+                           const moe_tensor_t* ids, const moe_tensor_t* wts, moe_tensor_t* out,
+                           const Problem& pr, const WsLayout& L, uint8_t* w, DeviceInfo* dev,
+                           cudaStream_t st) {
+  int launches = 0;
+  int32_t* counts = reinterpret_cast<int32_t*>(w + L.counts);
+  int32_t* offsets = reinterpret_cast<int32_t*>(w + L.offsets);
+  int32_t* num_blocks = reinterpret_cast<int32_t*>(w + L.num_blocks);
+  int32_t* chunk_counts = reinterpret_cast<int32_t*>(w + L.chunk_counts);
+  int32_t* sorted = reinterpret_cast<int32_t*>(w + L.sorted);
+  int32_t* inv = reinterpret_cast<int32_t*>(w + L.inv);
+  int32_t* block_expert = reinterpret_cast<int32_t*>(w + L.block_expert);
+  const moe_tensor_t* gate = &w13->gate;
+  const moe_tensor_t* up = &w13->up;
+  moe_status_t s;
+  CUtensorMap mA1, mGate, mUp, mH, mW2;
+  const uint32_t box2[2] = {128, 128};
+  const uint32_t box3[3] = {128, 64, 1};
+  {
+    const uint64_t d[2] = {uint64_t(pr.H / 2), uint64_t(L.p_max)};
+    const uint64_t sb[1] = {uint64_t(pr.H / 2)};
+    s = make_map(&mA1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w + L.a1, d, sb, box2,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s != MOE_OK) return s;
+    // packed e2m1 views: strides are bytes; the expert stride is the view's real stride(0)
+    const uint64_t d3[3] = {uint64_t(pr.H / 2), uint64_t(pr.I), uint64_t(pr.E)};
+    const uint64_t sg[2] = {uint64_t(gate->strides[1]), uint64_t(gate->strides[0])};
+    s = make_map(&mGate, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, gate->data, d3, sg, box3,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s != MOE_OK) return s;
+    const uint64_t su[2] = {uint64_t(up->strides[1]), uint64_t(up->strides[0])};
+    s = make_map(&mUp, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, up->data, d3, su, box3,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s != MOE_OK) return s;
+    const uint64_t dh[2] = {uint64_t(pr.I / 2), uint64_t(L.p_max)};
+    const uint64_t sh[1] = {uint64_t(pr.I / 2)};
+    s = make_map(&mH, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w + L.h, dh, sh, box2,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s != MOE_OK) return s;
+    const uint64_t dw[3] = {uint64_t(pr.I / 2), uint64_t(pr.H), uint64_t(pr.E)};
+    const uint64_t sw[2] = {uint64_t(w2->strides[1]), uint64_t(w2->strides[0])};
+    s = make_map(&mW2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w2->data, dw, sw, box3,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s != MOE_OK) return s;
+  }
+  t_prof.n = 0;
+  t_prof.have = false;
+  prof_mark(st);
+  cudaError_t rc = launch_align(view2(ids), pr.T, pr.k, pr.E, L.bm, counts, offsets, sorted, inv,
+                                block_expert, num_blocks, chunk_counts, L.n_chunks, dev->errors,
+                                st, &launches);
+  if (rc != cudaSuccess) return cuda_fail(rc, "align");
+  prof_mark(st);
+  rc = launch_permute_quant(view2(x), pr.T, pr.H, pr.k, pr.E, inv, offsets, counts, w + L.a1,
+                            w + L.a1_scale, st, &launches);
+  if (rc != cudaSuccess) return cuda_fail(rc, "permute_quant");
+  prof_mark(st);
+  GemmArgs g1;
+  std::memset(&g1, 0, sizeof(g1));
+  g1.K = pr.H;
+  g1.N = pr.I;
+  g1.n_tiles = pr.I / 64;
+  g1.max_tiles = L.nb_max * g1.n_tiles;
+  g1.num_blocks = num_blocks;
+  g1.block_expert = block_expert;
+  g1.sorted = sorted;
+  g1.S = L.S;
+  g1.out = w + L.h;
+  g1.out_ld = pr.I / 2;
+  g1.k = pr.k;
+  g1.err = dev->errors;
+  rc = launch_gemm1_mxfp4(mA1, w + L.a1_scale, pr.H / 32, mGate,
+                          static_cast<const uint8_t*>(gate->scale), gate->scale_strides[0],
+                          gate->scale_strides[1], mUp, static_cast<const uint8_t*>(up->scale),
+                          up->scale_strides[0], up->scale_strides[1], w + L.h_scale, pr.I / 32,
+                          g1, dev->num_sms, st, &launches);
+  if (rc != cudaSuccess) return cuda_fail(rc, "gemm1_mxfp4");
+  prof_mark(st);
+  GemmArgs g2 = g1;
+  g2.K = pr.I;
+  g2.N = pr.H;
+  g2.n_tiles = pr.H / 128;
+  g2.max_tiles = L.nb_max * g2.n_tiles;
+  g2.out = w + L.y;
+  g2.out_ld = pr.H;
+  g2.topk_w = view2(wts);
+  rc = launch_gemm2_mxfp4(mH, w + L.h_scale, pr.I / 32, mW2, static_cast<const uint8_t*>(w2->scale),
+                          w2->scale_strides[0], w2->scale_strides[1], g2, dev->num_sms, st,
+                          &launches);
+  if (rc != cudaSuccess) return cuda_fail(rc, "gemm2_mxfp4");
+  prof_mark(st);
+  rc = launch_combine(reinterpret_cast<const __nv_bfloat16*>(w + L.y), view2(ids), pr.E, pr.T,
+                      pr.H, pr.k, out->data, out->strides[0], out->strides[1], st, &launches);
+  if (rc != cudaSuccess) return cuda_fail(rc, "combine");
+  prof_mark(st);
+  t_prof.have = t_prof.on && t_prof.n == kProfSteps + 1;
+  t_last_launches = launches;
+  return MOE_OK;
+}
+
 moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe_tensor_t* w2,
                           const moe_tensor_t* ids, const moe_tensor_t* wts, moe_tensor_t* out,
                           const Problem& pr, void* ws, size_t ws_bytes, cudaStream_t st) {
@@ -351,7 +458,7 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   const moe_tensor_t* gate = &w13->gate;
   const moe_tensor_t* up = &w13->up;
 
-  if (pr.mxfp4) return MOE_ERR_UNSUPPORTED_DTYPE;  // block-scaled path: see moe_gemm_mxfp4.cu
+  if (pr.mxfp4) return forward_mxfp4(x, w13, w2, ids, wts, out, pr, L, w, dev, st);
 
   // ---- tensor maps (bf16, 128-byte swizzle, box 64 x 128)
   CUtensorMap mA1, mGate, mUp, mH, mW2;

@@ -209,6 +209,56 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          ((uint32_t)(M >> 4) << 24);
 }
 
+// ---------------------------------------------------------------- block-scaled (MXFP4)
+
+// D[tmem] (+)= (A * SFA) x (B * SFB)^T, kind::mxf4: packed e2m1 A/B read from
+// shared memory (K = 64 per instruction), one e8m0 scale per 32 elements of K
+// read from tensor memory.  sfa/sfb carry the scale byte offset in bits 30-31.
+__device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Instruction descriptor for kind::mxf4 with e8m0 scales, both operands
+// K-major e2m1.  Bits: B scale byte id [4,6), A format [7,10) (1 = e2m1),
+// B format [10,13) (1 = e2m1), N >> 3 at [17,23), scale format bit 23
+// (1 = e8m0), M >> 4 at [24,29), A scale byte id [29,31), bit 31 = 0 (K = 64).
+__host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N, uint32_t a_sf_id, uint32_t b_sf_id) {
+  return (b_sf_id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | (1u << 23) |
+         ((uint32_t)(M >> 4) << 24) | (a_sf_id << 29);
+}
+
+// Copy 32 rows x 16 bytes from shared memory into TMEM lanes 0..31 of every
+// 32-lane sub-partition (four copies), 4 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t src_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc)
+               : "memory");
+}
+
+// Shared-memory descriptor of an unswizzled K-major block whose rows are 16 bytes
+// apart (8-row core matrices of 128 contiguous bytes, stride-dimension offset
+// 128 bytes).  Used as the source of tcgen05.cp.
+__device__ __forceinline__ uint64_t plain_rows16_desc(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)(16u >> 4) << 16;
+  d |= (uint64_t)(128u >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  return d;
+}
+
+// Make this thread's generic-proxy shared-memory writes visible to the async
+// proxy (TMA, tensor cores) once ordered by a barrier.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- misc
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

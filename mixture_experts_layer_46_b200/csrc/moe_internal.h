@@ -84,13 +84,18 @@ cudaError_t launch_gemm1_bf16(const CUtensorMap& a, const CUtensorMap& gate, con
 cudaError_t launch_gemm2_bf16(const CUtensorMap& a, const CUtensorMap& w2, const GemmArgs& g,
                               int num_sms, cudaStream_t st, int* launches);
 
-cudaError_t launch_gemm1_mxfp4(const CUtensorMap& a, const CUtensorMap& a_sf,
-                               const CUtensorMap& gate, const CUtensorMap& gate_sf,
-                               const CUtensorMap& up, const CUtensorMap& up_sf, const GemmArgs& g,
-                               int num_sms, cudaStream_t st, int* launches);
-cudaError_t launch_gemm2_mxfp4(const CUtensorMap& a, const CUtensorMap& a_sf,
-                               const CUtensorMap& w2, const CUtensorMap& w2_sf,
+// MXFP4 (e2m1 codes + e8m0 scales): A codes through TMA maps, scales read
+// through their own pointers/strides (bytes).  GEMM1 writes h codes to g.out and
+// h scales to h_sf; GEMM2 writes y like the bf16 GEMM2.
+cudaError_t launch_gemm1_mxfp4(const CUtensorMap& a, const uint8_t* a_sf, int64_t a_sf_ld,
+                               const CUtensorMap& gate, const uint8_t* gate_sf, int64_t gs0,
+                               int64_t gs1, const CUtensorMap& up, const uint8_t* up_sf,
+                               int64_t us0, int64_t us1, uint8_t* h_sf, int64_t h_sf_ld,
                                const GemmArgs& g, int num_sms, cudaStream_t st, int* launches);
+cudaError_t launch_gemm2_mxfp4(const CUtensorMap& a, const uint8_t* a_sf, int64_t a_sf_ld,
+                               const CUtensorMap& w2, const uint8_t* w2_sf, int64_t ws0,
+                               int64_t ws1, const GemmArgs& g, int num_sms, cudaStream_t st,
+                               int* launches);
 
 // standalone MXFP4 quantiser for rows of a [R, K] bf16/f32 matrix (unit inner stride)
 cudaError_t launch_quantize_rows(const void* src, int32_t src_dtype, int64_t R, int64_t K,

@@ -79,6 +79,16 @@ def make_weights_bf16(E: int, I: int, H: int, seed: int = 0, device="cpu"):
     return w13, w2
 
 
+def iter_weights_fp32(E: int, I: int, H: int, seed: int = 0, device="cpu"):
+    """Expert by expert: (e, w13_e [2I, H] fp32, w2_e [H, I] fp32), std 1/sqrt(fan_in).
+    For MXFP4 layers, whose fp32 weights are quantised once and never held whole."""
+    g = _gen(seed, device)
+    for e in range(E):
+        w13 = torch.randn(2 * I, H, generator=g, device=device).mul_(1.0 / math.sqrt(H))
+        w2 = torch.randn(H, I, generator=g, device=device).mul_(1.0 / math.sqrt(I))
+        yield e, w13, w2
+
+
 def gate_up_views(w13: torch.Tensor):
     """gate = w13[:, :I, :], up = w13[:, I:, :]: strided views, no copy
     (Liger-Kernel PR #1377, "Problems")."""

@@ -178,6 +178,9 @@ double oracle_e2m1_value(uint32_t code) { return e2m1_value(code & 15u); }
 int oracle_mxfp4_quantize(const float* src, int64_t R, int64_t K, int64_t rs, uint8_t* codes,
                           uint8_t* scales) {
   if (K % 32 != 0) return 1;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
   for (int64_t r = 0; r < R; ++r) {
     for (int64_t b = 0; b < K / 32; ++b) {
       double v[32];

@@ -1,0 +1,160 @@
+"""GPU parity of the MXFP4 path (aiter PR #3859, "Details": e2m1 weights and
+activations with per-1x32 e8m0 scales) against the fp64 oracle.
+
+Bars: the quantiser is bit-exact (codes and scales) against the oracle's; the
+forward is within max|y - ref| / max|ref| <= 6e-2 (the oracle quantises the
+SwiGLU activation from fp64, the GPU from fp32, so a few codes near rounding
+boundaries may differ); strided packed views vs contiguous copies are
+bit-identical on the GPU.
+"""
+
+import pytest
+import torch
+
+import mixture_experts_layer_46_b200 as moe
+import oracle
+from mixture_experts_layer_46_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+MX_TOL = 6e-2
+
+
+def rel_err(got, ref):
+    got = got.double().cpu()
+    ref = ref.double().cpu()
+    return (got - ref).abs().max().item() / ref.abs().max().item()
+
+
+def _special_rows(K):
+    """Rows exercising ties, saturation, zeros, tiny blocks and negative zeros."""
+    rows = []
+    base = torch.tensor([6.0, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 7.0, -0.2, -0.25, -3.5, 0.0, -0.0,
+                         4.0, 0.5] * 2)
+    rows.append(base)
+    rows.append(base * 2.0 ** -20)
+    rows.append(torch.zeros(32))
+    rows.append(-base * 3.0)
+    rows.append(torch.full((32,), 1e-30))
+    r = torch.cat(rows)
+    reps = (K * 8 + r.numel() - 1) // r.numel()
+    return r.repeat(reps)[:K * 8].reshape(8, K)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_quantize_bit_exact(dtype):
+    g = torch.Generator().manual_seed(3)
+    K = 512
+    src = torch.randn(64, K, generator=g) * torch.logspace(-6, 6, 64)[:, None]
+    src = torch.cat([src, _special_rows(K)]).to(dtype)
+    ref_c, ref_s = oracle.mxfp4_quantize(src.float())
+    got_c, got_s = moe.quantize_mxfp4(src.cuda())
+    torch.cuda.synchronize()
+    assert torch.equal(got_s.cpu(), ref_s)
+    assert torch.equal(got_c.cpu(), ref_c)
+
+
+def test_quantize_3d_strided_destination():
+    g = torch.Generator().manual_seed(4)
+    src = torch.randn(3, 40, 256, generator=g)
+    ref_c, ref_s = oracle.mxfp4_quantize(src.reshape(-1, 256))
+    codes_big = torch.zeros(3, 48, 128, dtype=torch.uint8, device="cuda")
+    scales_big = torch.zeros(3, 48, 16, dtype=torch.uint8, device="cuda")
+    codes, scales = codes_big[:, 4:44], scales_big[:, 4:44, :8]  # padded rows and row stride
+    d_src = moe.desc(src.cuda())
+    d_dst = moe.desc(codes, scales)
+    import ctypes
+    rc = moe.load().moe_quantize_mxfp4(ctypes.byref(d_src), ctypes.byref(d_dst),
+                                       torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert torch.equal(codes.cpu().reshape(-1, 128), ref_c)
+    assert torch.equal(scales.cpu().reshape(-1, 8), ref_s)
+    assert torch.all(codes_big[:, :4] == 0) and torch.all(scales_big[:, 44:] == 0)
+    assert torch.all(scales_big[:, :, 8:] == 0)
+
+
+def make_mx_case(T, H, I, E, k, seed=0, shared=False):
+    x = wl.make_x(T, H, seed=seed + 1)
+    c13 = torch.empty(E, 2 * I, H // 2, dtype=torch.uint8)
+    s13 = torch.empty(E, 2 * I, H // 32, dtype=torch.uint8)
+    c2 = torch.empty(E, H, I // 2, dtype=torch.uint8)
+    s2 = torch.empty(E, H, I // 32, dtype=torch.uint8)
+    for e, w13e, w2e in wl.iter_weights_fp32(E, I, H, seed=seed):
+        c13[e], s13[e] = oracle.mxfp4_quantize(w13e)
+        c2[e], s2[e] = oracle.mxfp4_quantize(w2e)
+    if shared:
+        ids, wts = wl.route_shared_expert(T, E - 1, k - 1, seed=seed + 2)
+    else:
+        ids, wts = wl.route_softmax_topk(T, E, k, seed=seed + 2)
+    return {"x": x, "c13": c13, "s13": s13, "c2": c2, "s2": s2, "ids": ids, "wts": wts}
+
+
+def mx_oracle(case, tokens=None):
+    I = case["c13"].shape[1] // 2
+    ref, _ = oracle.moe_forward(case["x"], case["c13"][:, :I], case["c13"][:, I:], case["c2"],
+                                case["ids"], case["wts"],
+                                scales=(case["s13"][:, :I], case["s13"][:, I:], case["s2"]),
+                                tokens=tokens)
+    return ref
+
+
+def mx_gpu(c, contiguous=False):
+    I = c["c13"].shape[1] // 2
+    if contiguous:
+        keep = [c["c13"][:, :I].contiguous(), c["c13"][:, I:].contiguous(),
+                c["s13"][:, :I].contiguous(), c["s13"][:, I:].contiguous()]
+        v = moe.w13_from_views(keep[0], keep[1], keep[2], keep[3])
+    else:
+        keep = []
+        v = moe.w13_from_packed(c["c13"], c["s13"])
+    out = moe.forward(c["x"], v, c["c2"], c["ids"], c["wts"], w2_scale=c["s2"])
+    torch.cuda.synchronize()
+    del keep
+    return out
+
+
+def cuda_case(case):
+    return {k: v.cuda() for k, v in case.items()}
+
+
+@pytest.mark.parametrize("T,H,I,E,k", [
+    (64, 256, 256, 8, 2),
+    (200, 512, 512, 16, 4),
+    (1, 256, 256, 4, 2),
+])
+def test_mxfp4_forward_matches_oracle(T, H, I, E, k):
+    case = make_mx_case(T, H, I, E, k, seed=T)
+    ref = mx_oracle(case)
+    got = mx_gpu(cuda_case(case))
+    assert rel_err(got, ref) <= MX_TOL
+
+
+def test_mxfp4_strided_equals_contiguous_and_deterministic():
+    c = cuda_case(make_mx_case(150, 512, 256, 8, 4, seed=5))
+    a = mx_gpu(c)
+    b = mx_gpu(c, contiguous=True)
+    d = mx_gpu(c)
+    assert torch.equal(a, b)
+    assert torch.equal(a, d)
+
+
+def test_mxfp4_shared_expert_fused_routing():
+    # E = 32 routed + 1 shared, top_k = 4 + 1, the 513/11 convention at reduced size
+    case = make_mx_case(96, 512, 256, 33, 5, seed=7, shared=True)
+    assert torch.all(case["ids"][:, 4] == 32)
+    ref = mx_oracle(case)
+    got = mx_gpu(cuda_case(case))
+    assert rel_err(got, ref) <= MX_TOL
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("shared", [False, True])
+def test_qwen35_tp2_mxfp4_full_size_sampled(shared):
+    s = wl.QWEN35_TP2_MXFP4_SHARED if shared else wl.QWEN35_TP2_MXFP4
+    case = make_mx_case(s.T, s.H, s.I, s.E, s.k, seed=0, shared=shared)
+    got = mx_gpu(cuda_case(case))
+    g = torch.Generator().manual_seed(11)
+    toks = torch.unique(torch.cat([torch.randperm(s.T, generator=g)[:24], torch.tensor([0, s.T - 1])]))
+    ref = mx_oracle(case, tokens=toks)
+    assert rel_err(got.cpu()[toks], ref) <= MX_TOL
