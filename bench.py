@@ -51,17 +51,12 @@ WORKLOADS = {
 # DRAM traffic per launch of the dominant kernel from an ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed to the hash of the kernel
 # source it was taken on; reported as null once the source has changed.
-NCU_TRAFFIC = {
-    # profiles/grouped_gemm_bf16_qwen3shape_E32_T1024.md: 988.6 MB read + 27.7 MB written on
-    # the E=32, T=1024 case, scaled x4 (experts) to the E=128, T=4096 launch
-    "gemm1_swiglu": {"bytes_per_launch": 4.0 * (988.558080e6 + 27.661568e6), "src": "5c4c0d592bfeac3f",
-                     "workload": "qwen3-235b T=4096"},
-}
+NCU_TRAFFIC = {}
 
 
 def kernel_src_hash() -> str:
     h = hashlib.sha256()
-    for fn in ("moe_gemm_bf16.cu", "moe_common.cuh"):
+    for fn in ("moe_gemm_ws.cu", "moe_common.cuh"):
         with open(os.path.join(ROOT, "mixture_experts_layer_46_b200", "csrc", fn), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -495,13 +490,22 @@ def sweep(args, w, moe, wl, dev, stream, flush):
                 torch.cuda.synchronize(dev)
                 per.append(a.elapsed_time(b))
             med = statistics.median(per)
+            moe.profile_enable(True)
+            brk = {}
+            for i in range(5):
+                flush.fill_(i & 0xff)
+                moe.forward(x, v13, w2, ids, wts, out=out, workspace=ws, stream=stream)
+                for kname, kms in moe.profile_read().items():
+                    brk[kname] = brk.get(kname, 0.0) + kms * 1e3 / 5
+            moe.profile_enable(False)
             alg = algorithmic(wt, ids)
             t_roof = max(alg["flops"] / (tf_burst * 1e12), alg["bytes"] / (hbm * 1e9))
             row = {"T": T, "us_median": med * 1e3, "tokens_per_s": T / (med * 1e-3),
                    "roofline_us": t_roof * 1e6, "frac": t_roof / (med * 1e-3),
                    "hbm_GBs_alg": alg["bytes"] / (med * 1e-3) / 1e9,
                    "tflops_alg": alg["flops"] / (med * 1e-3) / 1e12,
-                   "active_experts": alg["active_experts"]}
+                   "active_experts": alg["active_experts"],
+                   "step_us": {k: round(v, 1) for k, v in brk.items()}}
             f.write(json.dumps(row) + "\n")
             f.flush()
             del ws, out

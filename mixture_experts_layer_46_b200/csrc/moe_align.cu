@@ -83,59 +83,74 @@ __device__ void block_scatter(const View2& ids, int64_t k, int64_t E, int64_t s0
   }
 }
 
-// From per-expert counts (shared), write counts, offsets, num_blocks,
-// block_expert and the sentinel padding of sorted.  offs (shared, E+1 ints)
-// receives the offsets for the caller's later use.
-__device__ void block_finalize(const int* cnt, int64_t E, int32_t bm, int32_t S, int* offs,
-                               int32_t* counts, int32_t* offsets, int32_t* sorted,
-                               int32_t* block_expert, int32_t* num_blocks) {
+// Block-wide exclusive scan over experts of v(e) (each thread owns a
+// contiguous run of experts).  out[e] receives the prefix, out[E] the total;
+// every thread gets the total back.
+template <class F>
+__device__ int block_scan_experts(int64_t E, F v, int* out) {
   __shared__ int warp_sums[32];
   __shared__ int total_sh;
-  // exclusive scan of padded counts: each thread owns a contiguous run of experts
   const int per = static_cast<int>((E + blockDim.x - 1) / blockDim.x);
   const int e0 = threadIdx.x * per;
   int local = 0;
-  for (int i = 0; i < per; ++i) {
-    const int e = e0 + i;
-    if (e < E) local += (cnt[e] + bm - 1) / bm * bm;
-  }
-  // block-wide exclusive scan of `local`
+  for (int i = 0; i < per; ++i)
+    if (e0 + i < E) local += v(e0 + i);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int incl = local;
   for (int d = 1; d < 32; d <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, d);
-    if (lane >= d) incl += v;
+    const int u = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += u;
   }
+  __syncthreads();  // warp_sums may still be read by a previous call
   if (lane == 31) warp_sums[warp] = incl;
   __syncthreads();
   if (warp == 0) {
     const int nw = (blockDim.x + 31) / 32;
-    int v = lane < nw ? warp_sums[lane] : 0;
+    int x = lane < nw ? warp_sums[lane] : 0;
     for (int d = 1; d < 32; d <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, v, d);
-      if (lane >= d) v += u;
+      const int u = __shfl_up_sync(0xffffffffu, x, d);
+      if (lane >= d) x += u;
     }
-    if (lane < nw) warp_sums[lane] = v;  // inclusive warp totals
-    if (lane == nw - 1) total_sh = v;
+    if (lane < nw) warp_sums[lane] = x;
+    if (lane == nw - 1) total_sh = x;
   }
   __syncthreads();
   int run = incl - local + (warp > 0 ? warp_sums[warp - 1] : 0);
   for (int i = 0; i < per; ++i) {
-    const int e = e0 + i;
-    if (e < E) {
-      offs[e] = run;
-      offsets[e] = run;
-      counts[e] = cnt[e];
-      run += (cnt[e] + bm - 1) / bm * bm;
+    if (e0 + i < E) {
+      out[e0 + i] = run;
+      run += v(e0 + i);
     }
   }
-  if (threadIdx.x == 0) {
-    offs[E] = total_sh;
-    offsets[E] = total_sh;
-    *num_blocks = total_sh / bm;
-  }
+  if (threadIdx.x == 0) out[E] = total_sh;
   __syncthreads();
-  const int nb = total_sh / bm;
+  return total_sh;
+}
+
+// Outputs of align beyond sorted/offsets: the token-tile list consumed by the
+// weight-stationary GEMMs (tiles of up to tile_max rows, never crossing an
+// expert), written when tile_max > 0.
+struct TileOut {
+  int32_t tile_max;
+  int32_t* tile_row;     // first padded row of the tile
+  int32_t* tile_rows;    // rows in the tile (multiple of bm)
+  int32_t* tile_expert;
+  int32_t* num_tiles;
+};
+
+// From per-expert counts (shared), write counts, offsets, num_blocks,
+// block_expert, the sentinel padding of sorted and the tile list.  offs
+// (shared, E+1 ints) receives the offsets; tsc (shared, E+1 ints) is scratch.
+__device__ void block_finalize(const int* cnt, int64_t E, int32_t bm, int32_t S, int* offs, int* tsc,
+                               int32_t* counts, int32_t* offsets, int32_t* sorted,
+                               int32_t* block_expert, int32_t* num_blocks, const TileOut& to) {
+  const int total = block_scan_experts(E, [&](int e) { return (cnt[e] + bm - 1) / bm * bm; }, offs);
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+    offsets[e] = offs[e];
+    if (e < E) counts[e] = cnt[e];
+  }
+  if (threadIdx.x == 0) *num_blocks = total / bm;
+  const int nb = total / bm;
   for (int b = threadIdx.x; b < nb; b += blockDim.x) {
     // last expert whose offset is <= b*bm (empty experts share offsets with the next one)
     int lo = 0, hi = static_cast<int>(E);  // answer in [lo, hi)
@@ -148,16 +163,32 @@ __device__ void block_finalize(const int* cnt, int64_t E, int32_t bm, int32_t S,
   }
   for (int e = threadIdx.x; e < E; e += blockDim.x)
     for (int p = offs[e] + cnt[e]; p < offs[e + 1]; ++p) sorted[p] = S;
+  if (to.tile_max > 0) {
+    const int tm = to.tile_max;
+    const int nt = block_scan_experts(
+        E, [&](int e) { return (offs[e + 1] - offs[e] + tm - 1) / tm; }, tsc);
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      const int rows = offs[e + 1] - offs[e];
+      for (int j = 0, t = tsc[e]; j * tm < rows; ++j, ++t) {
+        to.tile_row[t] = offs[e] + j * tm;
+        to.tile_rows[t] = min(tm, rows - j * tm);
+        to.tile_expert[t] = e;
+      }
+    }
+    if (threadIdx.x == 0) *to.num_tiles = nt;
+  }
 }
 
 __global__ void __launch_bounds__(kThreads) align_small_kernel(
     View2 ids, int64_t T, int64_t k, int64_t E, int32_t bm, int32_t* counts, int32_t* offsets,
-    int32_t* sorted, int32_t* inv, int32_t* block_expert, int32_t* num_blocks, DeviceErrors* err) {
+    int32_t* sorted, int32_t* inv, int32_t* block_expert, int32_t* num_blocks, TileOut to,
+    DeviceErrors* err) {
   extern __shared__ int sm[];
   int* hist = sm;                       // [E]
   int* offs = hist + E;                 // [E + 1]
   int* base = offs + E + 1;             // [E]
   int* warp_cnt = base + E;             // [kWarps * E]
+  int* tsc = warp_cnt + kWarps * E;     // [E + 1]
   __shared__ int bad_sh;
   pdl_wait();
   const int64_t S = T * k;
@@ -170,8 +201,8 @@ __global__ void __launch_bounds__(kThreads) align_small_kernel(
   const int bad = block_hist(ids, k, E, 0, S, hist);
   if (bad) atomicAdd(&bad_sh, bad);
   __syncthreads();
-  block_finalize(hist, E, bm, static_cast<int32_t>(S), offs, counts, offsets, sorted, block_expert,
-                 num_blocks);
+  block_finalize(hist, E, bm, static_cast<int32_t>(S), offs, tsc, counts, offsets, sorted,
+                 block_expert, num_blocks, to);
   for (int e = threadIdx.x; e < E; e += blockDim.x) base[e] = offs[e];
   __syncthreads();
   block_scatter(ids, k, E, 0, S, base, warp_cnt, sorted, inv);
@@ -204,10 +235,11 @@ __global__ void __launch_bounds__(1024) align_scan_kernel(int64_t T, int64_t k, 
                                                           int32_t* chunk_counts, int32_t* counts,
                                                           int32_t* offsets, int32_t* sorted,
                                                           int32_t* block_expert,
-                                                          int32_t* num_blocks) {
+                                                          int32_t* num_blocks, TileOut to) {
   extern __shared__ int sm[];
-  int* cnt = sm;         // [E]
-  int* offs = cnt + E;   // [E + 1]
+  int* cnt = sm;              // [E]
+  int* offs = cnt + E;        // [E + 1]
+  int* tsc = offs + E + 1;    // [E + 1]
   pdl_wait();
   // per expert: exclusive prefix over chunks (in place), total count
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -220,8 +252,8 @@ __global__ void __launch_bounds__(1024) align_scan_kernel(int64_t T, int64_t k, 
     cnt[e] = run;
   }
   __syncthreads();
-  block_finalize(cnt, E, bm, static_cast<int32_t>(T * k), offs, counts, offsets, sorted,
-                 block_expert, num_blocks);
+  block_finalize(cnt, E, bm, static_cast<int32_t>(T * k), offs, tsc, counts, offsets, sorted,
+                 block_expert, num_blocks, to);
   pdl_launch_dependents();
 }
 
@@ -250,19 +282,26 @@ __global__ void __launch_bounds__(kThreads) align_scatter_kernel(View2 ids, int6
 cudaError_t launch_align(const View2& ids, int64_t T, int64_t k, int64_t E, int32_t bm,
                          int32_t* counts, int32_t* offsets, int32_t* sorted, int32_t* inv,
                          int32_t* block_expert, int32_t* num_blocks, int32_t* chunk_counts,
-                         int64_t n_chunks, DeviceErrors* err, cudaStream_t st, int* launches) {
+                         int64_t n_chunks, DeviceErrors* err, cudaStream_t st, int* launches,
+                         const AlignTiles* tiles) {
+  TileOut to;
+  to.tile_max = tiles ? tiles->tile_max : 0;
+  to.tile_row = tiles ? tiles->tile_row : nullptr;
+  to.tile_rows = tiles ? tiles->tile_rows : nullptr;
+  to.tile_expert = tiles ? tiles->tile_expert : nullptr;
+  to.num_tiles = tiles ? tiles->num_tiles : nullptr;
   if (E > kMaxExperts) return cudaErrorInvalidValue;
   const int64_t S = T * k;
   cudaError_t rc;
   if (S <= kAlignSmallMax) {
-    const size_t smem = sizeof(int) * (E * (kWarps + 3) + 1);
+    const size_t smem = sizeof(int) * (E * (kWarps + 4) + 2);
     if (smem > 48 * 1024) {
       rc = cudaFuncSetAttribute(align_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)smem);
       if (rc != cudaSuccess) return rc;
     }
     rc = launch_pdl(align_small_kernel, dim3(1), dim3(kThreads), smem, st, ids, T, k, E, bm,
-                    counts, offsets, sorted, inv, block_expert, num_blocks, err);
+                    counts, offsets, sorted, inv, block_expert, num_blocks, to, err);
     if (launches) *launches += 1;
     return rc;
   }
@@ -270,9 +309,9 @@ cudaError_t launch_align(const View2& ids, int64_t T, int64_t k, int64_t E, int3
   rc = launch_pdl(align_count_kernel, dim3((unsigned)n_chunks), dim3(kThreads), smem_count, st,
                   ids, T, k, E, chunk_counts, err);
   if (rc != cudaSuccess) return rc;
-  const size_t smem_scan = sizeof(int) * (2 * E + 1);
+  const size_t smem_scan = sizeof(int) * (3 * E + 2);
   rc = launch_pdl(align_scan_kernel, dim3(1), dim3(1024), smem_scan, st, T, k, E, bm, n_chunks,
-                  chunk_counts, counts, offsets, sorted, block_expert, num_blocks);
+                  chunk_counts, counts, offsets, sorted, block_expert, num_blocks, to);
   if (rc != cudaSuccess) return rc;
   const size_t smem_sc = sizeof(int) * E * (kWarps + 1);
   if (smem_sc > 48 * 1024) {

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -272,15 +273,30 @@ moe_status_t cached_workspace(size_t need, void** ptr) {
 
 // ---------------------------------------------------------------- layout
 
-int32_t choose_block_m(int64_t T, int64_t k, int64_t E) {
-  (void)T;
-  (void)k;
-  (void)E;
-  return 128;  // the tensor-core tile is M = 128 rows
+void choose_tiling(int64_t T, int64_t k, int64_t E, bool mxfp4, int32_t* bm, int32_t* tile_max) {
+  if (mxfp4) {
+    // block-scaled weight-stationary kernels: token tiles of up to 32 or 96 rows
+    // (96 keeps both accumulator buffers and the per-stage scales inside TMEM)
+    *bm = 32;
+    const int64_t avg = E > 0 ? (T * k) / E : 0;
+    *tile_max = avg <= 8 ? 32 : 96;
+    return;
+  }
+  // weight-stationary bf16 kernels: tokens are the MMA's N side in 32-row
+  // granules, in tiles of up to 32 rows while experts average <= 8 slots
+  // (decode: 6-stage ring, more weight bytes in flight) and up to 128 rows
+  // beyond (double-buffered accumulators).  MOE_TILE=32|128 overrides (tuning).
+  *bm = 32;
+  const int64_t avg = E > 0 ? (T * k) / E : 0;
+  *tile_max = avg <= 8 ? 32 : 128;
+  if (const char* env = getenv("MOE_TILE")) {
+    const int v = atoi(env);
+    if (v == 32 || v == 128) *tile_max = v;
+  }
 }
 
 WsLayout make_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, bool mxfp4,
-                     int32_t bm) {
+                     int32_t bm, int32_t tile_max) {
   WsLayout L;
   std::memset(&L, 0, sizeof(L));
   L.T = T;
@@ -290,6 +306,7 @@ WsLayout make_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, bool
   L.k = k;
   L.S = T * k;
   L.bm = bm;
+  L.tile_max = tile_max;
   L.mxfp4 = mxfp4;
   const int64_t S = L.S;
   const int64_t nonempty = S < E ? S : E;
@@ -298,6 +315,7 @@ WsLayout make_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, bool
   if (p < bm) p = bm;
   L.p_max = p;
   L.nb_max = p / bm;
+  L.t_max = tile_max > 0 ? p / tile_max + nonempty + 1 : 0;
   L.n_chunks = (S + kAlignChunk - 1) / kAlignChunk;
   if (L.n_chunks < 1) L.n_chunks = 1;
   size_t off = 0;
@@ -313,6 +331,9 @@ WsLayout make_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, bool
   L.sorted = take(sizeof(int32_t) * p);
   L.inv = take(sizeof(int32_t) * (S > 0 ? S : 1));
   L.block_expert = take(sizeof(int32_t) * L.nb_max);
+  L.tile_row = take(sizeof(int32_t) * L.t_max);
+  L.tile_rows = take(sizeof(int32_t) * L.t_max);
+  L.tile_expert = take(sizeof(int32_t) * L.t_max);
   if (!mxfp4) {
     L.a1 = take(size_t(p) * H * 2);
     L.a1_scale = off;
@@ -349,79 +370,100 @@ moe_status_t forward_mxfp4(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   const moe_tensor_t* up = &w13->up;
   moe_status_t s;
   CUtensorMap mA1, mGate, mUp, mH, mW2;
-  const uint32_t box2[2] = {128, 128};
-  const uint32_t box3[3] = {128, 64, 1};
+  const uint32_t boxt[2] = {128, 32};
+  const uint32_t boxw[3] = {128, 128, 1};
   {
     const uint64_t d[2] = {uint64_t(pr.H / 2), uint64_t(L.p_max)};
     const uint64_t sb[1] = {uint64_t(pr.H / 2)};
-    s = make_map(&mA1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w + L.a1, d, sb, box2,
+    s = make_map(&mA1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w + L.a1, d, sb, boxt,
                  CU_TENSOR_MAP_SWIZZLE_128B);
     if (s != MOE_OK) return s;
     // packed e2m1 views: strides are bytes; the expert stride is the view's real stride(0)
     const uint64_t d3[3] = {uint64_t(pr.H / 2), uint64_t(pr.I), uint64_t(pr.E)};
     const uint64_t sg[2] = {uint64_t(gate->strides[1]), uint64_t(gate->strides[0])};
-    s = make_map(&mGate, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, gate->data, d3, sg, box3,
+    s = make_map(&mGate, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, gate->data, d3, sg, boxw,
                  CU_TENSOR_MAP_SWIZZLE_128B);
     if (s != MOE_OK) return s;
     const uint64_t su[2] = {uint64_t(up->strides[1]), uint64_t(up->strides[0])};
-    s = make_map(&mUp, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, up->data, d3, su, box3,
+    s = make_map(&mUp, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, up->data, d3, su, boxw,
                  CU_TENSOR_MAP_SWIZZLE_128B);
     if (s != MOE_OK) return s;
     const uint64_t dh[2] = {uint64_t(pr.I / 2), uint64_t(L.p_max)};
     const uint64_t sh[1] = {uint64_t(pr.I / 2)};
-    s = make_map(&mH, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w + L.h, dh, sh, box2,
+    s = make_map(&mH, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w + L.h, dh, sh, boxt,
                  CU_TENSOR_MAP_SWIZZLE_128B);
     if (s != MOE_OK) return s;
     const uint64_t dw[3] = {uint64_t(pr.I / 2), uint64_t(pr.H), uint64_t(pr.E)};
     const uint64_t sw[2] = {uint64_t(w2->strides[1]), uint64_t(w2->strides[0])};
-    s = make_map(&mW2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w2->data, dw, sw, box3,
+    s = make_map(&mW2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w2->data, dw, sw, boxw,
                  CU_TENSOR_MAP_SWIZZLE_128B);
     if (s != MOE_OK) return s;
   }
+  AlignTiles tiles;
+  tiles.tile_max = L.tile_max;
+  tiles.tile_row = reinterpret_cast<int32_t*>(w + L.tile_row);
+  tiles.tile_rows = reinterpret_cast<int32_t*>(w + L.tile_rows);
+  tiles.tile_expert = reinterpret_cast<int32_t*>(w + L.tile_expert);
+  tiles.num_tiles = num_blocks + 1;
   t_prof.n = 0;
   t_prof.have = false;
   prof_mark(st);
   cudaError_t rc = launch_align(view2(ids), pr.T, pr.k, pr.E, L.bm, counts, offsets, sorted, inv,
                                 block_expert, num_blocks, chunk_counts, L.n_chunks, dev->errors,
-                                st, &launches);
+                                st, &launches, &tiles);
   if (rc != cudaSuccess) return cuda_fail(rc, "align");
   prof_mark(st);
   rc = launch_permute_quant(view2(x), pr.T, pr.H, pr.k, pr.E, inv, offsets, counts, w + L.a1,
                             w + L.a1_scale, st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "permute_quant");
   prof_mark(st);
-  GemmArgs g1;
+  WsGemmMx g1;
   std::memset(&g1, 0, sizeof(g1));
   g1.K = pr.H;
   g1.N = pr.I;
-  g1.n_tiles = pr.I / 64;
-  g1.max_tiles = L.nb_max * g1.n_tiles;
-  g1.num_blocks = num_blocks;
-  g1.block_expert = block_expert;
+  g1.n_wt = pr.I / 128;
+  g1.max_tiles = L.t_max;
+  g1.num_tiles = tiles.num_tiles;
+  g1.tile_row = tiles.tile_row;
+  g1.tile_rows = tiles.tile_rows;
+  g1.tile_expert = tiles.tile_expert;
   g1.sorted = sorted;
   g1.S = L.S;
   g1.out = w + L.h;
   g1.out_ld = pr.I / 2;
+  g1.out_sf = w + L.h_scale;
+  g1.out_sf_ld = pr.I / 32;
   g1.k = pr.k;
+  g1.x_sf = w + L.a1_scale;
+  g1.x_sf_ld = pr.H / 32;
+  g1.w0_sf = static_cast<const uint8_t*>(gate->scale);
+  g1.w0_s0 = gate->scale_strides[0];
+  g1.w0_s1 = gate->scale_strides[1];
+  g1.w1_sf = static_cast<const uint8_t*>(up->scale);
+  g1.w1_s0 = up->scale_strides[0];
+  g1.w1_s1 = up->scale_strides[1];
   g1.err = dev->errors;
-  rc = launch_gemm1_mxfp4(mA1, w + L.a1_scale, pr.H / 32, mGate,
-                          static_cast<const uint8_t*>(gate->scale), gate->scale_strides[0],
-                          gate->scale_strides[1], mUp, static_cast<const uint8_t*>(up->scale),
-                          up->scale_strides[0], up->scale_strides[1], w + L.h_scale, pr.I / 32,
-                          g1, dev->num_sms, st, &launches);
+  rc = launch_gemm_ws_mxfp4(0, L.tile_max, mGate, mUp, mA1, g1, dev->num_sms, st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm1_mxfp4");
   prof_mark(st);
-  GemmArgs g2 = g1;
+  WsGemmMx g2 = g1;
   g2.K = pr.I;
   g2.N = pr.H;
-  g2.n_tiles = pr.H / 128;
-  g2.max_tiles = L.nb_max * g2.n_tiles;
+  g2.n_wt = pr.H / 256;
   g2.out = w + L.y;
   g2.out_ld = pr.H;
+  g2.out_sf = nullptr;
+  g2.out_sf_ld = 0;
   g2.topk_w = view2(wts);
-  rc = launch_gemm2_mxfp4(mH, w + L.h_scale, pr.I / 32, mW2, static_cast<const uint8_t*>(w2->scale),
-                          w2->scale_strides[0], w2->scale_strides[1], g2, dev->num_sms, st,
-                          &launches);
+  g2.x_sf = w + L.h_scale;
+  g2.x_sf_ld = pr.I / 32;
+  g2.w0_sf = static_cast<const uint8_t*>(w2->scale);
+  g2.w0_s0 = w2->scale_strides[0];
+  g2.w0_s1 = w2->scale_strides[1];
+  g2.w1_sf = g2.w0_sf;
+  g2.w1_s0 = g2.w0_s0;
+  g2.w1_s1 = g2.w0_s1;
+  rc = launch_gemm_ws_mxfp4(1, L.tile_max, mW2, mW2, mH, g2, dev->num_sms, st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm2_mxfp4");
   prof_mark(st);
   rc = launch_combine(reinterpret_cast<const __nv_bfloat16*>(w + L.y), view2(ids), pr.E, pr.T,
@@ -439,8 +481,9 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   int launches = 0;
   t_last_launches = 0;
   if (pr.T == 0) return MOE_OK;
-  const int32_t bm = choose_block_m(pr.T, pr.k, pr.E);
-  const WsLayout L = make_layout(pr.T, pr.H, pr.I, pr.E, pr.k, pr.mxfp4, bm);
+  int32_t bm = 0, tile_max = 0;
+  choose_tiling(pr.T, pr.k, pr.E, pr.mxfp4, &bm, &tile_max);
+  const WsLayout L = make_layout(pr.T, pr.H, pr.I, pr.E, pr.k, pr.mxfp4, bm, tile_max);
   if (!ws || ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
   if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return MOE_ERR_INVALID_ARG;
   DeviceInfo* dev = nullptr;
@@ -460,14 +503,15 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
 
   if (pr.mxfp4) return forward_mxfp4(x, w13, w2, ids, wts, out, pr, L, w, dev, st);
 
-  // ---- tensor maps (bf16, 128-byte swizzle, box 64 x 128)
+  // ---- tensor maps (bf16, 128-byte swizzle): weights in [64 x 128] boxes,
+  // gathered token rows in [64 x 32] boxes
   CUtensorMap mA1, mGate, mUp, mH, mW2;
-  const uint32_t box2[2] = {64, 128};
-  const uint32_t box3[3] = {64, 128, 1};
+  const uint32_t boxw[3] = {64, 128, 1};
+  const uint32_t boxt[2] = {64, 32};
   {
     const uint64_t d[2] = {uint64_t(pr.H), uint64_t(L.p_max)};
     const uint64_t sb[1] = {uint64_t(pr.H) * 2};
-    s = make_map(&mA1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w + L.a1, d, sb, box2,
+    s = make_map(&mA1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w + L.a1, d, sb, boxt,
                  CU_TENSOR_MAP_SWIZZLE_128B);
     if (s != MOE_OK) return s;
   }
@@ -476,34 +520,40 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
     // base + e * stride(0), whatever lies between experts (e.g. the up half).
     const uint64_t d[3] = {uint64_t(pr.H), uint64_t(pr.I), uint64_t(pr.E)};
     const uint64_t sg[2] = {uint64_t(gate->strides[1]) * 2, uint64_t(gate->strides[0]) * 2};
-    s = make_map(&mGate, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, gate->data, d, sg, box3,
+    s = make_map(&mGate, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, gate->data, d, sg, boxw,
                  CU_TENSOR_MAP_SWIZZLE_128B);
     if (s != MOE_OK) return s;
     const uint64_t su[2] = {uint64_t(up->strides[1]) * 2, uint64_t(up->strides[0]) * 2};
-    s = make_map(&mUp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, up->data, d, su, box3,
+    s = make_map(&mUp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, up->data, d, su, boxw,
                  CU_TENSOR_MAP_SWIZZLE_128B);
     if (s != MOE_OK) return s;
   }
   {
     const uint64_t d[2] = {uint64_t(pr.I), uint64_t(L.p_max)};
     const uint64_t sb[1] = {uint64_t(pr.I) * 2};
-    s = make_map(&mH, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w + L.h, d, sb, box2,
+    s = make_map(&mH, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w + L.h, d, sb, boxt,
                  CU_TENSOR_MAP_SWIZZLE_128B);
     if (s != MOE_OK) return s;
     const uint64_t d3[3] = {uint64_t(pr.I), uint64_t(pr.H), uint64_t(pr.E)};
     const uint64_t s3[2] = {uint64_t(w2->strides[1]) * 2, uint64_t(w2->strides[0]) * 2};
-    s = make_map(&mW2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, w2->data, d3, s3, box3,
+    s = make_map(&mW2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, w2->data, d3, s3, boxw,
                  CU_TENSOR_MAP_SWIZZLE_128B);
     if (s != MOE_OK) return s;
   }
 
   // ---- launches
+  AlignTiles tiles;
+  tiles.tile_max = L.tile_max;
+  tiles.tile_row = reinterpret_cast<int32_t*>(w + L.tile_row);
+  tiles.tile_rows = reinterpret_cast<int32_t*>(w + L.tile_rows);
+  tiles.tile_expert = reinterpret_cast<int32_t*>(w + L.tile_expert);
+  tiles.num_tiles = num_blocks + 1;
   t_prof.n = 0;
   t_prof.have = false;
   prof_mark(st);
   cudaError_t rc;
   rc = launch_align(view2(ids), pr.T, pr.k, pr.E, bm, counts, offsets, sorted, inv, block_expert,
-                    num_blocks, chunk_counts, L.n_chunks, dev->errors, st, &launches);
+                    num_blocks, chunk_counts, L.n_chunks, dev->errors, st, &launches, &tiles);
   if (rc != cudaSuccess) return cuda_fail(rc, "align");
   prof_mark(st);
   rc = launch_permute_bf16(view2(x), pr.T, pr.H, pr.k, pr.E, inv, offsets, counts,
@@ -511,33 +561,34 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   if (rc != cudaSuccess) return cuda_fail(rc, "permute");
   prof_mark(st);
 
-  GemmArgs g1;
+  WsGemm g1;
   std::memset(&g1, 0, sizeof(g1));
   g1.K = pr.H;
   g1.N = pr.I;
-  g1.n_tiles = (pr.I + 127) / 128;
-  g1.max_tiles = L.nb_max * g1.n_tiles;
-  g1.num_blocks = num_blocks;
-  g1.block_expert = block_expert;
+  g1.n_wt = (pr.I + 127) / 128;
+  g1.max_tiles = L.t_max;
+  g1.num_tiles = tiles.num_tiles;
+  g1.tile_row = tiles.tile_row;
+  g1.tile_rows = tiles.tile_rows;
+  g1.tile_expert = tiles.tile_expert;
   g1.sorted = sorted;
   g1.S = L.S;
   g1.out = w + L.h;
   g1.out_ld = pr.I;
   g1.k = pr.k;
   g1.err = dev->errors;
-  rc = launch_gemm1_bf16(mA1, mGate, mUp, g1, dev->num_sms, st, &launches);
+  rc = launch_gemm_ws_bf16(0, L.tile_max, mGate, mUp, mA1, g1, dev->num_sms, st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm1");
   prof_mark(st);
 
-  GemmArgs g2 = g1;
+  WsGemm g2 = g1;
   g2.K = pr.I;
   g2.N = pr.H;
-  g2.n_tiles = (pr.H + 255) / 256;
-  g2.max_tiles = L.nb_max * g2.n_tiles;
+  g2.n_wt = (pr.H + 255) / 256;
   g2.out = w + L.y;
   g2.out_ld = pr.H;
   g2.topk_w = view2(wts);
-  rc = launch_gemm2_bf16(mH, mW2, g2, dev->num_sms, st, &launches);
+  rc = launch_gemm_ws_bf16(1, L.tile_max, mW2, mW2, mH, g2, dev->num_sms, st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm2");
   prof_mark(st);
 
@@ -618,8 +669,9 @@ moe_status_t moe_w13_from_packed(const moe_tensor_t* w13, moe_w13_t* out) {
 size_t moe_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, int32_t wdtype) {
   if (T < 0 || H < 1 || I < 1 || E < 1 || k < 1) return 0;
   if (wdtype != MOE_BF16 && wdtype != MOE_E2M1X2) return 0;
-  const int32_t bm = choose_block_m(T, k, E);
-  return make_layout(T, H, I, E, k, wdtype == MOE_E2M1X2, bm).total;
+  int32_t bm = 0, tile_max = 0;
+  choose_tiling(T, k, E, wdtype == MOE_E2M1X2, &bm, &tile_max);
+  return make_layout(T, H, I, E, k, wdtype == MOE_E2M1X2, bm, tile_max).total;
 }
 
 moe_status_t moe_forward_ws(const moe_tensor_t* x, const moe_w13_t* w13, const moe_tensor_t* w2,
@@ -722,7 +774,7 @@ moe_status_t moe_align(const moe_tensor_t* topk_ids, int64_t E, int32_t block_m,
   DeviceInfo* dev = nullptr;
   moe_status_t s = device_info(&dev);
   if (s != MOE_OK) return s;
-  const WsLayout L = make_layout(T, 32, 32, E, k, false, block_m);
+  const WsLayout L = make_layout(T, 32, 32, E, k, false, block_m, 0);
   // inv and chunk counts live in the caller's workspace
   const size_t need = align256(L.inv + sizeof(int32_t) * T * k);
   if (!workspace || workspace_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;

@@ -1,26 +1,29 @@
-// Block-scaled MXFP4 grouped expert GEMMs (tcgen05.mma kind::mxf4, sm_100a).
+// Weight-stationary block-scaled MXFP4 grouped expert GEMMs
+// (tcgen05.mma kind::mxf4.block_scale, sm_100a).
 //
 // Operands are packed e2m1 codes (two per byte) with one e8m0 scale per 32
 // consecutive elements of the contraction axis (aiter PR #3859, "Details":
-// float4_e2m1fn_x2 weights and activations, QuantType.per_1x32):
-//   GEMM1: A1 codes [P, H/2] x gate/up codes [E, I, H/2] -> G, U (fp32 in TMEM)
-//          h = silu(G) * U quantised per 1x32 along I -> codes [P, I/2], scales [P, I/32]
-//   GEMM2: h codes x w2 codes [E, H, I/2] -> Y; y[slot] = bf16(w_slot * Y[row])
-// Expert addressing is the same as the bf16 kernels: 3-D TMA maps whose expert
-// stride is each view's real stride(0) (Liger-Kernel PR #1377, "Problems").
+// float4_e2m1fn_x2 weights and activations, QuantType.per_1x32).  As in the
+// bf16 kernels the weights are the MMA's M side (two 128-row tiles per work
+// item) and one expert's token tile (up to 32 or 96 rows) is the N side:
+//   GEMM1: acc0 = gate_tile . X^T, acc1 = up_tile . X^T (fp32 in TMEM);
+//          h = silu(acc0) * acc1, requantised per 1x32 along I -> codes [P, I/2], scales [P, I/32]
+//   GEMM2: acc0/acc1 = two 128-row w2 slices . H^T; y[slot, o] = bf16(w_slot * acc)
+// Expert addressing: 3-D TMA maps whose expert stride is each view's real
+// stride(0) (Liger-Kernel PR #1377, "Problems").
 //
 // Kernel shape: one persistent CTA per SM, 7 warps.
-//   warp 0    TMA producer: A [128 rows x 128 B] + two B boxes [64 rows x 128 B]
-//             per k-step (256 elements of K), 6-stage ring, 128-byte swizzle
+//   warp 0    TMA producer: two weight boxes [128 rows x 128 B] + the token tile
+//             in 32-row boxes per k-step (256 elements of K), 128-byte swizzle
 //   warp 1    TMEM allocator, MMA issuer: per stage copies the stage's scales
 //             from shared memory to TMEM (tcgen05.cp 32x128b.warpx4) and issues
-//             4 x tcgen05.mma.kind::mxf4.block_scale (M=128, N=128, K=64)
+//             2 x 4 x tcgen05.mma.kind::mxf4.block_scale (M=128, N=tile, K=64)
 //   warp 2    scale producer: reads the stage's e8m0 scales through their strides
 //             and writes them in the 128-row x 4-block atom the tensor core reads:
-//             byte (m % 32) * 16 + (m / 32) * 4 + block
-//   warps 3-6 epilogue (one accumulator row per thread)
-// TMEM: two 128-column accumulators, then 16 scale columns per stage
-// (A: 2 atoms x 4 columns, B: 2 atoms x 4 columns).
+//             byte (row % 32) * 16 + (row / 32) * 4 + block
+//   warps 3-6 epilogue (one weight row per thread)
+// TMEM: kBufs accumulator buffers of 2 x kNmax columns, then 24 scale columns
+// per stage (two weight tiles and the token tile, each 2 atoms x 4 columns).
 #include "../../include/moe.h"
 #include "moe_internal.h"
 #include "moe_mx.cuh"
@@ -28,26 +31,55 @@
 namespace moe {
 namespace {
 
-constexpr int kBM = 128;
+constexpr int kWRows = 128;
 constexpr int kRowBytes = 128;                 // packed bytes per row per stage (256 elements)
-constexpr int kBoxRows = 64;                   // rows per B TMA box
-constexpr int kUmmaN = 128;
+constexpr int kTokBox = 32;
 constexpr int kUmmaKBytes = 32;                // 64 e2m1 elements per instruction
-constexpr int kStages = 6;
-constexpr int kABytes = kBM * kRowBytes;       // 16 KiB
-constexpr int kBBytes = kUmmaN * kRowBytes;    // 16 KiB
 constexpr int kAtomBytes = 512;                // 128 rows x 4 scale blocks
-constexpr int kSfABytes = 2 * kAtomBytes;      // 8 blocks of 32 per stage
-constexpr int kSfBBytes = 2 * kAtomBytes;
-constexpr int kStageBytes = kABytes + kBBytes + kSfABytes + kSfBBytes;  // 34 KiB
+constexpr int kSfBytes = 2 * kAtomBytes;       // 8 blocks of 32 per stage
 constexpr int kEpiWarps = 4;
 constexpr int kStagingBytes = 32 * 64;
-constexpr int kAccCols = 128;
-constexpr int kSfColsPerStage = 16;
+constexpr int kSfColsPerStage = 24;
 constexpr int kTmemCols = 512;
 constexpr int kThreads = 224;
-constexpr size_t kSmemBytes = 1024 + size_t(kStages) * kStageBytes + kEpiWarps * kStagingBytes +
-                              (2 * kStages + 5) * 8 + 16;
+
+template <int kNmax, int kStages>
+struct Cfg {
+  static constexpr int kWBytes = kWRows * kRowBytes;                 // 16 KiB
+  static constexpr int kTokBytes = kNmax * kRowBytes;
+  // [W0][W1][X][SF W0][SF W1][SF X]; 1024-byte aligned stage size
+  static constexpr int kRaw = 2 * kWBytes + kTokBytes + 3 * kSfBytes;
+  static constexpr int kStageBytes = (kRaw + 1023) / 1024 * 1024;
+  static constexpr int kBufCols = 2 * kNmax;
+  static constexpr int kBufs = (2 * kBufCols + kStages * kSfColsPerStage <= kTmemCols) ? 2 : 1;
+  static constexpr int kSfCol0 = kBufs * kBufCols;
+  static_assert(kSfCol0 + kStages * kSfColsPerStage <= kTmemCols, "TMEM budget");
+  static constexpr size_t kSmem = 1024 + size_t(kStages) * kStageBytes +
+                                  kEpiWarps * kStagingBytes + (2 * kStages + 5) * 8 + 16;
+};
+
+struct MxArgs {
+  int64_t K, N, n_wt;
+  const int32_t* num_tiles;
+  const int32_t* tile_row;
+  const int32_t* tile_rows;
+  const int32_t* tile_expert;
+  const int32_t* sorted;
+  int64_t S;
+  void* out;             // GEMM1: h codes [P, I/2]; GEMM2: y [S, H] bf16
+  int64_t out_ld;        // bytes (codes) or elements (y)
+  uint8_t* out_sf;       // GEMM1: h scales [P, I/32]
+  int64_t out_sf_ld;
+  View2 topk_w;
+  int64_t k;
+  const uint8_t* x_sf;   // token scales [P, K/32]
+  int64_t x_sf_ld;
+  const uint8_t* w0_sf;  // weight scales [E, rows, K/32] (byte strides)
+  int64_t w0_s0, w0_s1;
+  const uint8_t* w1_sf;
+  int64_t w1_s0, w1_s1;
+  DeviceErrors* err;
+};
 
 struct Smem {
   uint8_t* stages;
@@ -60,11 +92,13 @@ struct Smem {
   uint32_t* tmem_slot;
 };
 
+template <int kNmax, int kStages>
 __device__ __forceinline__ Smem carve(uint8_t* raw) {
+  using C = Cfg<kNmax, kStages>;
   Smem s;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
   s.stages = base;
-  s.staging = base + kStages * kStageBytes;
+  s.staging = base + kStages * C::kStageBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(s.staging + kEpiWarps * kStagingBytes);
   s.full = bars;
   s.empty = bars + kStages;
@@ -75,46 +109,37 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   return s;
 }
 
-__device__ __forceinline__ uint32_t stg_off(int r, int part) {
-  return static_cast<uint32_t>(r * 64 + ((part ^ ((r >> 1) & 3)) << 4));
-}
-
-struct MxArgs {
-  const uint8_t* a_sf;   // [P, K/32] activation scales (row stride a_sf_ld bytes)
-  int64_t a_sf_ld;
-  const uint8_t* b0_sf;  // GEMM1: gate scales; GEMM2: w2 scales ([E, N, K/32], strides in bytes)
-  int64_t b0_s0, b0_s1;
-  const uint8_t* b1_sf;  // GEMM1: up scales
-  int64_t b1_s0, b1_s1;
-  uint8_t* h_sf;         // GEMM1 output scales [P, I/32]
-  int64_t h_sf_ld;
-};
-
 __device__ __forceinline__ uint2 ld_u2(const uint8_t* p) {
   return *reinterpret_cast<const uint2*>(p);
 }
 
-template <int kMode>
+__device__ __forceinline__ void st_v4(uint32_t addr, const uint32_t (&v)[4]) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v[0]), "r"(v[1]),
+               "r"(v[2]), "r"(v[3])
+               : "memory");
+}
+
+template <int kMode, int kNmax, int kStages>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_mxfp4_kernel(const __grid_constant__ CUtensorMap tmA,
-                              const __grid_constant__ CUtensorMap tmB0,
-                              const __grid_constant__ CUtensorMap tmB1, const GemmArgs g,
-                              const MxArgs mx) {
+    gemm_ws_mxfp4_kernel(const __grid_constant__ CUtensorMap tmW0,
+                         const __grid_constant__ CUtensorMap tmW1,
+                         const __grid_constant__ CUtensorMap tmX, const MxArgs g) {
+  using C = Cfg<kNmax, kStages>;
   extern __shared__ uint8_t smem_raw[];
-  const Smem sm = carve(smem_raw);
+  const Smem sm = carve<kNmax, kStages>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB0);
-    if (kMode == 0) tma_prefetch_desc(&tmB1);
+    tma_prefetch_desc(&tmW0);
+    if (kMode == 0) tma_prefetch_desc(&tmW1);
+    tma_prefetch_desc(&tmX);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.full[s], 2);  // TMA producer (with bytes) + scale producer
       mbar_init(&sm.empty[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&sm.tfull[a], 1);
-      mbar_init(&sm.tempty[a], kEpiWarps);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.tfull[b], 1);
+      mbar_init(&sm.tempty[b], kEpiWarps);
     }
     mbar_init(sm.drain, 1);
     fence_barrier_init();
@@ -129,8 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *sm.tmem_slot;
 
   pdl_wait();
-  const int64_t num_blocks = *g.num_blocks;
-  const int64_t total = num_blocks * g.n_tiles;
+  const int64_t total = static_cast<int64_t>(*g.num_tiles) * g.n_wt;
   const int num_k = static_cast<int>(g.K / 256);  // K % 256 == 0 (validated)
 
   if (warp == 0) {
@@ -141,20 +165,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s < kStages; ++s) last_phase[s] = -1;
       const uint64_t pol = l2_policy_evict_last();
       bool ok = true;
-      for (int64_t tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        const int64_t m = tile / g.n_tiles, n = tile - m * g.n_tiles;
-        const int32_t e = g.block_expert[m];
-        const int32_t row0 = static_cast<int32_t>(kMode == 0 ? n * kBoxRows : n * kUmmaN);
-        const int32_t row1 = kMode == 0 ? row0 : row0 + kBoxRows;
+      for (int64_t item = blockIdx.x; item < total && ok; item += gridDim.x) {
+        const int64_t t = item / g.n_wt, wt = item - t * g.n_wt;
+        const int32_t e = g.tile_expert[t], row0 = g.tile_row[t], rows = g.tile_rows[t];
+        const int32_t w0 = static_cast<int32_t>(kMode == 0 ? wt * kWRows : wt * 2 * kWRows);
+        const int32_t w1 = kMode == 0 ? w0 : w0 + kWRows;
+        const int nbox = rows / kTokBox;
+        const uint32_t bytes = 2 * C::kWBytes + nbox * kTokBox * kRowBytes;
         for (int kb = 0; kb < num_k; ++kb) {
           if (!mbar_wait(&sm.empty[stage], phase ^ 1u, g.err)) { ok = false; break; }
-          uint8_t* sa = sm.stages + stage * kStageBytes;
-          uint8_t* sb = sa + kABytes;
-          mbar_arrive_expect_tx(&sm.full[stage], kABytes + kBBytes);
-          tma_load_2d(sa, &tmA, &sm.full[stage], kb * kRowBytes, static_cast<int32_t>(m * kBM), pol);
-          tma_load_3d(sb, &tmB0, &sm.full[stage], kb * kRowBytes, row0, e, pol);
-          tma_load_3d(sb + kBoxRows * kRowBytes, kMode == 0 ? &tmB1 : &tmB0, &sm.full[stage],
-                      kb * kRowBytes, row1, e, pol);
+          uint8_t* sw0 = sm.stages + stage * C::kStageBytes;
+          uint8_t* sw1 = sw0 + C::kWBytes;
+          uint8_t* sx = sw1 + C::kWBytes;
+          mbar_arrive_expect_tx(&sm.full[stage], bytes);
+          tma_load_3d(sw0, &tmW0, &sm.full[stage], kb * kRowBytes, w0, e, pol);
+          tma_load_3d(sw1, kMode == 0 ? &tmW1 : &tmW0, &sm.full[stage], kb * kRowBytes, w1, e, pol);
+          for (int b = 0; b < nbox; ++b)
+            tma_load_2d(sx + b * kTokBox * kRowBytes, &tmX, &sm.full[stage], kb * kRowBytes,
+                        row0 + b * kTokBox, pol);
           last_phase[stage] = static_cast<int8_t>(phase);
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
@@ -167,88 +195,83 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 2) {
     // ------------------------------------------------------------ scale producer
     uint32_t stage = 0, phase = 0;
-    for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      const int64_t m = tile / g.n_tiles, n = tile - m * g.n_tiles;
-      const int32_t e = g.block_expert[m];
-      bool ok = true;
+    bool ok = true;
+    for (int64_t item = blockIdx.x; item < total && ok; item += gridDim.x) {
+      const int64_t t = item / g.n_wt, wt = item - t * g.n_wt;
+      const int32_t e = g.tile_expert[t], row0 = g.tile_row[t], rows = g.tile_rows[t];
+      const int64_t w0 = kMode == 0 ? wt * kWRows : wt * 2 * kWRows;
+      const int64_t w1 = kMode == 0 ? w0 : w0 + kWRows;
       for (int kb = 0; kb < num_k; ++kb) {
         if (!mbar_wait(&sm.empty[stage], phase ^ 1u, g.err)) { ok = false; break; }
-        uint8_t* sfa = sm.stages + stage * kStageBytes + kABytes + kBBytes;
-        uint8_t* sfb = sfa + kSfABytes;
-        uint32_t alo[4], ahi[4], blo[4], bhi[4];
+        uint8_t* sf = sm.stages + stage * C::kStageBytes + 2 * C::kWBytes + C::kTokBytes;
+        uint32_t a_lo[4], a_hi[4], b_lo[4], b_hi[4], x_lo[4], x_hi[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const int r = lane + 32 * j;
-          const uint2 va = ld_u2(mx.a_sf + (m * kBM + r) * mx.a_sf_ld + kb * 8);
-          alo[j] = va.x;
-          ahi[j] = va.y;
-          const uint8_t* pb;
-          if (kMode == 0) {
-            pb = (r < kBoxRows)
-                     ? mx.b0_sf + e * mx.b0_s0 + (n * kBoxRows + r) * mx.b0_s1
-                     : mx.b1_sf + e * mx.b1_s0 + (n * kBoxRows + (r - kBoxRows)) * mx.b1_s1;
-          } else {
-            pb = mx.b0_sf + e * mx.b0_s0 + (n * kUmmaN + r) * mx.b0_s1;
-          }
-          const uint2 vb = ld_u2(pb + kb * 8);
-          blo[j] = vb.x;
-          bhi[j] = vb.y;
+          const int64_t r = lane + 32 * j;  // row inside the tile (atom row = lane, column = j)
+          // rows outside the weight matrix or the token tile read as scale 0
+          uint2 v0 = make_uint2(0, 0), v1 = make_uint2(0, 0), vx = make_uint2(0, 0);
+          if (w0 + r < g.N) v0 = ld_u2(g.w0_sf + e * g.w0_s0 + (w0 + r) * g.w0_s1 + kb * 8);
+          if (w1 + r < g.N) v1 = ld_u2(g.w1_sf + e * g.w1_s0 + (w1 + r) * g.w1_s1 + kb * 8);
+          if (r < rows) vx = ld_u2(g.x_sf + (row0 + r) * g.x_sf_ld + kb * 8);
+          a_lo[j] = v0.x; a_hi[j] = v0.y;
+          b_lo[j] = v1.x; b_hi[j] = v1.y;
+          x_lo[j] = vx.x; x_hi[j] = vx.y;
         }
-        const uint32_t a_s = smem_u32(sfa) + 16 * lane, b_s = smem_u32(sfb) + 16 * lane;
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a_s), "r"(alo[0]), "r"(alo[1]),
-                     "r"(alo[2]), "r"(alo[3]) : "memory");
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a_s + kAtomBytes), "r"(ahi[0]),
-                     "r"(ahi[1]), "r"(ahi[2]), "r"(ahi[3]) : "memory");
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(b_s), "r"(blo[0]), "r"(blo[1]),
-                     "r"(blo[2]), "r"(blo[3]) : "memory");
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(b_s + kAtomBytes), "r"(bhi[0]),
-                     "r"(bhi[1]), "r"(bhi[2]), "r"(bhi[3]) : "memory");
+        const uint32_t s0 = smem_u32(sf) + 16 * lane;
+        st_v4(s0, a_lo);
+        st_v4(s0 + kAtomBytes, a_hi);
+        st_v4(s0 + kSfBytes, b_lo);
+        st_v4(s0 + kSfBytes + kAtomBytes, b_hi);
+        st_v4(s0 + 2 * kSfBytes, x_lo);
+        st_v4(s0 + 2 * kSfBytes + kAtomBytes, x_hi);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.full[stage]);
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
       }
-      if (!ok) break;
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (elect_one()) {
-      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+      uint32_t stage = 0, phase = 0, buf = 0, acc_phase = 0;
       bool ok = true, issued = false;
-      for (int64_t tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        if (!mbar_wait(&sm.tempty[acc], acc_phase ^ 1u, g.err)) { ok = false; break; }
+      for (int64_t item = blockIdx.x; item < total && ok; item += gridDim.x) {
+        const int64_t t = item / g.n_wt;
+        const int32_t rows = g.tile_rows[t];
+        if (!mbar_wait(&sm.tempty[buf], acc_phase ^ 1u, g.err)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d = tmem_base + acc * kAccCols;
+        const uint32_t acc0 = tmem_base + buf * C::kBufCols, acc1 = acc0 + kNmax;
         for (int kb = 0; kb < num_k; ++kb) {
           if (!mbar_wait(&sm.full[stage], phase, g.err)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(sm.stages + stage * kStageBytes);
-          const uint32_t b_addr = a_addr + kABytes;
-          const uint32_t sfa_smem = b_addr + kBBytes;
-          const uint32_t sfb_smem = sfa_smem + kSfABytes;
-          const uint32_t sfa_t = tmem_base + 2 * kAccCols + stage * kSfColsPerStage;
-          const uint32_t sfb_t = sfa_t + 8;
-          tmem_cp_32x128b_x4(sfa_t, plain_rows16_desc(sfa_smem));
-          tmem_cp_32x128b_x4(sfa_t + 4, plain_rows16_desc(sfa_smem + kAtomBytes));
-          tmem_cp_32x128b_x4(sfb_t, plain_rows16_desc(sfb_smem));
-          tmem_cp_32x128b_x4(sfb_t + 4, plain_rows16_desc(sfb_smem + kAtomBytes));
+          const uint32_t w0_addr = smem_u32(sm.stages + stage * C::kStageBytes);
+          const uint32_t w1_addr = w0_addr + C::kWBytes;
+          const uint32_t x_addr = w1_addr + C::kWBytes;
+          const uint32_t sf_smem = x_addr + C::kTokBytes;
+          const uint32_t sf_t = tmem_base + C::kSfCol0 + stage * kSfColsPerStage;
+          // scales of W0 -> cols [0, 8), W1 -> [8, 16), X -> [16, 24); 4 columns per atom
+#pragma unroll
+          for (int q = 0; q < 6; ++q)
+            tmem_cp_32x128b_x4(sf_t + 4 * q, plain_rows16_desc(sf_smem + kAtomBytes * q));
 #pragma unroll
           for (int kk = 0; kk < kRowBytes / kUmmaKBytes; ++kk) {
             const uint32_t atom = kk >> 1, sfid = 2u * (kk & 1);
-            const uint32_t idesc = idesc_mxf4(kBM, kUmmaN, sfid, sfid);
-            mma_mxf4(d, sw128_kmajor_desc(a_addr + kk * kUmmaKBytes),
-                     sw128_kmajor_desc(b_addr + kk * kUmmaKBytes), idesc,
-                     (sfa_t + 4 * atom) | (sfid << 30), (sfb_t + 4 * atom) | (sfid << 30),
-                     (kb > 0 || kk > 0) ? 1u : 0u);
+            const uint32_t idesc = idesc_mxf4(kWRows, rows, sfid, sfid);
+            const uint64_t xd = sw128_kmajor_desc(x_addr + kk * kUmmaKBytes);
+            const uint32_t sfx = (sf_t + 16 + 4 * atom) | (sfid << 30);
+            const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+            mma_mxf4(acc0, sw128_kmajor_desc(w0_addr + kk * kUmmaKBytes), xd, idesc,
+                     (sf_t + 4 * atom) | (sfid << 30), sfx, acc);
+            mma_mxf4(acc1, sw128_kmajor_desc(w1_addr + kk * kUmmaKBytes), xd, idesc,
+                     (sf_t + 8 + 4 * atom) | (sfid << 30), sfx, acc);
           }
           issued = true;
           mma_commit(&sm.empty[stage]);
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        mma_commit(&sm.tfull[acc]);
-        acc ^= 1u;
-        if (acc == 0) acc_phase ^= 1u;
+        mma_commit(&sm.tfull[buf]);
+        if (++buf == C::kBufs) { buf = 0; acc_phase ^= 1u; }
       }
       if (!ok && issued) {
         mma_commit(sm.drain);
@@ -258,82 +281,98 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int quad = warp & 3;
-    const int row_in_tile = quad * 32 + lane;
     uint8_t* stg = sm.staging + (warp - 3) * kStagingBytes;
     const uint32_t stg_s = smem_u32(stg);
-    uint32_t acc = 0, acc_phase = 0;
-    for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      const int64_t m = tile / g.n_tiles, n = tile - m * g.n_tiles;
-      int32_t slot = 0;
-      float wgt = 0.0f;
-      if (kMode == 1) {
-        slot = g.sorted[m * kBM + row_in_tile];
-        if (slot < g.S) {
-          const int64_t t = slot / g.k, j = slot - t * g.k;
-          wgt = static_cast<const float*>(g.topk_w.data)[t * g.topk_w.s0 + j * g.topk_w.s1];
-        }
-      }
-      if (!mbar_wait(&sm.tfull[acc], acc_phase, g.err)) break;
+    uint32_t buf = 0, acc_phase = 0;
+    for (int64_t item = blockIdx.x; item < total; item += gridDim.x) {
+      const int64_t t = item / g.n_wt, wt = item - t * g.n_wt;
+      const int32_t row0 = g.tile_row[t], rows = g.tile_rows[t];
+      if (!mbar_wait(&sm.tfull[buf], acc_phase, g.err)) break;
       tc_fence_after();
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * kAccCols;
+      const uint32_t lane_base = (static_cast<uint32_t>(quad * 32) << 16) + buf * C::kBufCols;
       if (kMode == 0) {
-        // 64 intermediate columns per tile: two 1x32 blocks, quantised in registers
-        const int64_t p = m * kBM + row_in_tile;
+        // this warp's 32 weight rows = one 1x32 block of I for every token
+        const int64_t i0 = wt * kWRows + quad * 32;
 #pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < rows / 32; ++c) {
           uint32_t gv[32], uv[32];
-          tmem_ld32(tbase + c * 32, gv);
-          tmem_ld32(tbase + kBoxRows + c * 32, uv);
+          tmem_ld32(tmem_base + lane_base + c * 32, gv);
+          tmem_ld32(tmem_base + lane_base + kNmax + c * 32, uv);
           tmem_wait_ld();
-          float hv[32];
+          uint32_t my_sc = 0;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) hv[i] = silu_mul(__uint_as_float(gv[i]), __uint_as_float(uv[i]));
-          uint32_t w[4];
-          const uint32_t sc = mx_quant32(hv, w);
-          const int64_t col = n * kBoxRows + c * 32;  // intermediate index of the block start
-          *reinterpret_cast<uint4*>(static_cast<uint8_t*>(g.out) + p * g.out_ld + col / 2) =
-              make_uint4(w[0], w[1], w[2], w[3]);
-          mx.h_sf[p * mx.h_sf_ld + col / 32] = static_cast<uint8_t>(sc);
+          for (int j = 0; j < 32; ++j) {
+            const float h = silu_mul(__uint_as_float(gv[j]), __uint_as_float(uv[j]));
+            float amax = fabsf(h);
+#pragma unroll
+            for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
+            const int sexp = mx_scale_exp(amax);
+            const float q = h * exp2i_neg(sexp);
+            const float qn = __shfl_xor_sync(0xffffffffu, q, 1);
+            if ((lane & 1) == 0) {
+              const uint32_t byte = cvt_e2m1x2(q, qn);
+              asm volatile("st.shared.b8 [%0], %1;" ::"r"(stg_s + j * 16 + (lane >> 1)), "r"(byte)
+                           : "memory");
+            }
+            if (lane == j) my_sc = static_cast<uint32_t>(sexp + 127);
+          }
+          __syncwarp();
+          // lane j stores token j's 16 code bytes and its scale
+          uint4 v;
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                       : "r"(stg_s + lane * 16));
+          if (i0 < g.N) {
+            const int64_t p = row0 + c * 32 + lane;
+            *reinterpret_cast<uint4*>(static_cast<uint8_t*>(g.out) + p * g.out_ld + i0 / 2) = v;
+            g.out_sf[p * g.out_sf_ld + i0 / 32] = static_cast<uint8_t>(my_sc);
+          }
+          __syncwarp();
         }
       } else {
 #pragma unroll 1
-        for (int c = 0; c < kUmmaN / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tbase + c * 32, v);
-          tmem_wait_ld();
-          uint32_t packed[16];
+        for (int a = 0; a < 2; ++a) {
+          const int64_t col0 = wt * 2 * kWRows + a * kWRows + quad * 32;
+          const bool col_ok = col0 < g.N;
+#pragma unroll 1
+          for (int c = 0; c < rows / 32; ++c) {
+            int32_t my_slot = g.sorted[row0 + c * 32 + lane];
+            float my_w = 0.0f;
+            if (my_slot < g.S) {
+              const int64_t tt = my_slot / g.k, jj = my_slot - tt * g.k;
+              my_w = static_cast<const float*>(g.topk_w.data)[tt * g.topk_w.s0 + jj * g.topk_w.s1];
+            }
+            uint32_t v0[32];
+            tmem_ld32(tmem_base + lane_base + a * kNmax + c * 32, v0);
+            tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            packed[i] = pack_bf16x2(wgt * __uint_as_float(v[2 * i]), wgt * __uint_as_float(v[2 * i + 1]));
+            for (int j = 0; j < 32; ++j) {
+              const float y = __shfl_sync(0xffffffffu, my_w, j) * __uint_as_float(v0[j]);
+              const __nv_bfloat16 yb = __float2bfloat16_rn(y);
+              asm volatile("st.shared.b16 [%0], %1;" ::"r"(stg_s + j * 64 + lane * 2),
+                           "h"(*reinterpret_cast<const uint16_t*>(&yb)) : "memory");
+            }
+            __syncwarp();
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stg_s + stg_off(lane, q)),
-                         "r"(packed[4 * q]), "r"(packed[4 * q + 1]), "r"(packed[4 * q + 2]),
-                         "r"(packed[4 * q + 3])
-                         : "memory");
+            for (int q = 0; q < 4; ++q) {
+              const int idx = q * 32 + lane;
+              const int j = idx >> 2, part = idx & 3;
+              uint4 v;
+              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                           : "r"(stg_s + j * 64 + part * 16));
+              const int32_t s_j = __shfl_sync(0xffffffffu, my_slot, j);
+              if (col_ok && s_j < g.S)
+                *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + static_cast<int64_t>(s_j) * g.out_ld + col0 + part * 8) = v;
+            }
+            __syncwarp();
           }
-          __syncwarp();
-          const int64_t col0 = n * kUmmaN + c * 32;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int idx = q * 32 + lane;
-            const int r = idx >> 2, part = idx & 3;
-            uint4 vv;
-            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(vv.x), "=r"(vv.y), "=r"(vv.z), "=r"(vv.w)
-                         : "r"(stg_s + stg_off(r, part)));
-            const int32_t s_r = __shfl_sync(0xffffffffu, slot, r);
-            if (col0 < g.N && s_r < g.S)
-              *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + static_cast<int64_t>(s_r) * g.out_ld + col0 + part * 8) = vv;
-          }
-          __syncwarp();
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.tempty[acc]);
-      acc ^= 1u;
-      if (acc == 0) acc_phase ^= 1u;
+      if (lane == 0) mbar_arrive(&sm.tempty[buf]);
+      if (++buf == C::kBufs) { buf = 0; acc_phase ^= 1u; }
     }
   }
 
@@ -345,65 +384,68 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int kMode>
-cudaError_t launch_mx(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                      const GemmArgs& g, const MxArgs& mx, int num_sms, cudaStream_t st) {
+template <int kMode, int kNmax, int kStages>
+cudaError_t launch_mx(const CUtensorMap& w0, const CUtensorMap& w1, const CUtensorMap& x,
+                      const MxArgs& g, int64_t max_items, int num_sms, cudaStream_t st) {
+  using C = Cfg<kNmax, kStages>;
   static unsigned long long configured = 0;
   int dev = 0;
   cudaError_t rc = cudaGetDevice(&dev);
   if (rc != cudaSuccess) return rc;
   if (dev >= 64 || !(configured & (1ull << dev))) {
-    rc = cudaFuncSetAttribute(grouped_gemm_mxfp4_kernel<kMode>,
+    rc = cudaFuncSetAttribute(gemm_ws_mxfp4_kernel<kMode, kNmax, kStages>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(kSmemBytes));
+                              static_cast<int>(C::kSmem));
     if (rc != cudaSuccess) return rc;
     if (dev < 64) configured |= 1ull << dev;
   }
-  int64_t grid = g.max_tiles < num_sms ? g.max_tiles : num_sms;
+  int64_t grid = max_items < num_sms ? max_items : num_sms;
   if (grid < 1) grid = 1;
-  return launch_pdl(grouped_gemm_mxfp4_kernel<kMode>, dim3(static_cast<unsigned>(grid)),
-                    dim3(kThreads), kSmemBytes, st, a, b0, b1, g, mx);
+  return launch_pdl(gemm_ws_mxfp4_kernel<kMode, kNmax, kStages>, dim3(static_cast<unsigned>(grid)),
+                    dim3(kThreads), C::kSmem, st, w0, w1, x, g);
 }
 
 }  // namespace
 
-cudaError_t launch_gemm1_mxfp4(const CUtensorMap& a, const uint8_t* a_sf, int64_t a_sf_ld,
-                               const CUtensorMap& gate, const uint8_t* gate_sf, int64_t gs0,
-                               int64_t gs1, const CUtensorMap& up, const uint8_t* up_sf,
-                               int64_t us0, int64_t us1, uint8_t* h_sf, int64_t h_sf_ld,
-                               const GemmArgs& g, int num_sms, cudaStream_t st, int* launches) {
-  MxArgs mx;
-  mx.a_sf = a_sf;
-  mx.a_sf_ld = a_sf_ld;
-  mx.b0_sf = gate_sf;
-  mx.b0_s0 = gs0;
-  mx.b0_s1 = gs1;
-  mx.b1_sf = up_sf;
-  mx.b1_s0 = us0;
-  mx.b1_s1 = us1;
-  mx.h_sf = h_sf;
-  mx.h_sf_ld = h_sf_ld;
+cudaError_t launch_gemm_ws_mxfp4(int mode, int tile_max, const CUtensorMap& w0,
+                                 const CUtensorMap& w1, const CUtensorMap& x, const WsGemmMx& p,
+                                 int num_sms, cudaStream_t st, int* launches) {
+  MxArgs g;
+  g.K = p.K;
+  g.N = p.N;
+  g.n_wt = p.n_wt;
+  g.num_tiles = p.num_tiles;
+  g.tile_row = p.tile_row;
+  g.tile_rows = p.tile_rows;
+  g.tile_expert = p.tile_expert;
+  g.sorted = p.sorted;
+  g.S = p.S;
+  g.out = p.out;
+  g.out_ld = p.out_ld;
+  g.out_sf = p.out_sf;
+  g.out_sf_ld = p.out_sf_ld;
+  g.topk_w = p.topk_w;
+  g.k = p.k;
+  g.x_sf = p.x_sf;
+  g.x_sf_ld = p.x_sf_ld;
+  g.w0_sf = p.w0_sf;
+  g.w0_s0 = p.w0_s0;
+  g.w0_s1 = p.w0_s1;
+  g.w1_sf = p.w1_sf;
+  g.w1_s0 = p.w1_s0;
+  g.w1_s1 = p.w1_s1;
+  g.err = p.err;
   if (launches) *launches += 1;
-  return launch_mx<0>(a, gate, up, g, mx, num_sms, st);
-}
-
-cudaError_t launch_gemm2_mxfp4(const CUtensorMap& a, const uint8_t* a_sf, int64_t a_sf_ld,
-                               const CUtensorMap& w2, const uint8_t* w2_sf, int64_t ws0,
-                               int64_t ws1, const GemmArgs& g, int num_sms, cudaStream_t st,
-                               int* launches) {
-  MxArgs mx;
-  mx.a_sf = a_sf;
-  mx.a_sf_ld = a_sf_ld;
-  mx.b0_sf = w2_sf;
-  mx.b0_s0 = ws0;
-  mx.b0_s1 = ws1;
-  mx.b1_sf = w2_sf;
-  mx.b1_s0 = ws0;
-  mx.b1_s1 = ws1;
-  mx.h_sf = nullptr;
-  mx.h_sf_ld = 0;
-  if (launches) *launches += 1;
-  return launch_mx<1>(a, w2, w2, g, mx, num_sms, st);
+  const int64_t max_items = p.max_tiles * p.n_wt;
+  if (tile_max == 96) {
+    if (mode == 0) return launch_mx<0, 96, 4>(w0, w1, x, g, max_items, num_sms, st);
+    return launch_mx<1, 96, 4>(w0, w1, x, g, max_items, num_sms, st);
+  }
+  if (tile_max == 32) {
+    if (mode == 0) return launch_mx<0, 32, 5>(w0, w1, x, g, max_items, num_sms, st);
+    return launch_mx<1, 32, 5>(w0, w1, x, g, max_items, num_sms, st);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace moe

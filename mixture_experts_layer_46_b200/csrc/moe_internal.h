@@ -21,12 +21,15 @@ struct View2 {
 // boundary.  Sizes depend only on (T, H, I, E, k, weight dtype).
 struct WsLayout {
   int64_t T, H, I, E, k, S;
-  int32_t bm;         // block_m: rows per expert block (the MMA tile M)
+  int32_t bm;         // block_m: padding granule of each expert's rows
+  int32_t tile_max;   // token-tile rows of the weight-stationary GEMMs (0: unused)
+  int64_t t_max;      // upper bound of the token-tile count
   int64_t n_chunks;   // align chunks
   int64_t p_max;      // upper bound of padded slot count
   int64_t nb_max;     // upper bound of the block count
   bool mxfp4;
   size_t counts, offsets, num_blocks, chunk_counts, sorted, inv, block_expert;
+  size_t tile_row, tile_rows, tile_expert;
   size_t a1, a1_scale, h, h_scale, y;
   size_t total;
 };
@@ -36,16 +39,29 @@ constexpr int kMaxExperts = 1024;       // experts per layer
 constexpr int kAlignChunk = 4096;        // slots per CTA in the multi-CTA align
 constexpr int kAlignSmallMax = 8192;     // single-CTA align up to this many slots
 
-int32_t choose_block_m(int64_t T, int64_t k, int64_t E);
-WsLayout make_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, bool mxfp4, int32_t bm);
+// Padding granule and token-tile size for a problem (depend only on T, k, E, dtype).
+void choose_tiling(int64_t T, int64_t k, int64_t E, bool mxfp4, int32_t* bm, int32_t* tile_max);
+WsLayout make_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, bool mxfp4, int32_t bm,
+                     int32_t tile_max);
 
 // ---- launchers (return cudaError_t of the launch) ----------------------------
 
-// align: ids -> counts, offsets, sorted, block_expert, num_blocks
+// Token-tile list for the weight-stationary GEMMs: tiles of up to tile_max
+// padded rows that never cross an expert boundary.
+struct AlignTiles {
+  int32_t tile_max;
+  int32_t* tile_row;
+  int32_t* tile_rows;
+  int32_t* tile_expert;
+  int32_t* num_tiles;
+};
+
+// align: ids -> counts, offsets, sorted, block_expert, num_blocks (+ tile list)
 cudaError_t launch_align(const View2& ids, int64_t T, int64_t k, int64_t E, int32_t bm,
                          int32_t* counts, int32_t* offsets, int32_t* sorted, int32_t* inv,
                          int32_t* block_expert, int32_t* num_blocks, int32_t* chunk_counts,
-                         int64_t n_chunks, DeviceErrors* err, cudaStream_t st, int* launches);
+                         int64_t n_chunks, DeviceErrors* err, cudaStream_t st, int* launches,
+                         const AlignTiles* tiles = nullptr);
 
 // permute: A1[inv[t*k+j], :] = x[t, :] (x read once per token), padding rows zeroed
 cudaError_t launch_permute_bf16(const View2& x, int64_t T, int64_t H, int64_t k, int64_t E,
@@ -79,23 +95,56 @@ struct GemmArgs {
   DeviceErrors* err;
 };
 
-cudaError_t launch_gemm1_bf16(const CUtensorMap& a, const CUtensorMap& gate, const CUtensorMap& up,
-                              const GemmArgs& g, int num_sms, cudaStream_t st, int* launches);
-cudaError_t launch_gemm2_bf16(const CUtensorMap& a, const CUtensorMap& w2, const GemmArgs& g,
-                              int num_sms, cudaStream_t st, int* launches);
 
-// MXFP4 (e2m1 codes + e8m0 scales): A codes through TMA maps, scales read
-// through their own pointers/strides (bytes).  GEMM1 writes h codes to g.out and
-// h scales to h_sf; GEMM2 writes y like the bf16 GEMM2.
-cudaError_t launch_gemm1_mxfp4(const CUtensorMap& a, const uint8_t* a_sf, int64_t a_sf_ld,
-                               const CUtensorMap& gate, const uint8_t* gate_sf, int64_t gs0,
-                               int64_t gs1, const CUtensorMap& up, const uint8_t* up_sf,
-                               int64_t us0, int64_t us1, uint8_t* h_sf, int64_t h_sf_ld,
-                               const GemmArgs& g, int num_sms, cudaStream_t st, int* launches);
-cudaError_t launch_gemm2_mxfp4(const CUtensorMap& a, const uint8_t* a_sf, int64_t a_sf_ld,
-                               const CUtensorMap& w2, const uint8_t* w2_sf, int64_t ws0,
-                               int64_t ws1, const GemmArgs& g, int num_sms, cudaStream_t st,
-                               int* launches);
+// Weight-stationary ("swap AB") bf16 GEMMs over the token-tile list of align.
+struct WsGemm {
+  int64_t K, N, n_wt, max_tiles;
+  const int32_t* num_tiles;
+  const int32_t* tile_row;
+  const int32_t* tile_rows;
+  const int32_t* tile_expert;
+  const int32_t* sorted;
+  int64_t S;
+  void* out;
+  int64_t out_ld;
+  View2 topk_w;
+  int64_t k;
+  DeviceErrors* err;
+};
+// mode 0: GEMM1 (gate/up + SwiGLU -> h), mode 1: GEMM2 (down + routing weight -> y)
+// tile_max: 128 (4-stage ring) or 32 (6-stage ring)
+cudaError_t launch_gemm_ws_bf16(int mode, int tile_max, const CUtensorMap& w0,
+                                const CUtensorMap& w1, const CUtensorMap& x, const WsGemm& p,
+                                int num_sms, cudaStream_t st, int* launches);
+
+// Weight-stationary block-scaled MXFP4 GEMMs over the token-tile list of align.
+// Codes through the TMA maps; scales through their own pointers (byte strides).
+struct WsGemmMx {
+  int64_t K, N, n_wt, max_tiles;
+  const int32_t* num_tiles;
+  const int32_t* tile_row;
+  const int32_t* tile_rows;
+  const int32_t* tile_expert;
+  const int32_t* sorted;
+  int64_t S;
+  void* out;              // GEMM1: h codes; GEMM2: y bf16
+  int64_t out_ld;
+  uint8_t* out_sf;        // GEMM1: h scales
+  int64_t out_sf_ld;
+  View2 topk_w;
+  int64_t k;
+  const uint8_t* x_sf;    // token scales [P, K/32]
+  int64_t x_sf_ld;
+  const uint8_t* w0_sf;   // GEMM1: gate scales; GEMM2: w2 scales
+  int64_t w0_s0, w0_s1;
+  const uint8_t* w1_sf;   // GEMM1: up scales; GEMM2: w2 scales
+  int64_t w1_s0, w1_s1;
+  DeviceErrors* err;
+};
+// tile_max: 96 (4-stage ring) or 32 (5-stage ring)
+cudaError_t launch_gemm_ws_mxfp4(int mode, int tile_max, const CUtensorMap& w0,
+                                 const CUtensorMap& w1, const CUtensorMap& x, const WsGemmMx& p,
+                                 int num_sms, cudaStream_t st, int* launches);
 
 // standalone MXFP4 quantiser for rows of a [R, K] bf16/f32 matrix (unit inner stride)
 cudaError_t launch_quantize_rows(const void* src, int32_t src_dtype, int64_t R, int64_t K,
