@@ -18,8 +18,9 @@
 //   warp 1    TMEM allocator, MMA issuer: per stage copies the stage's scales
 //             from shared memory to TMEM (tcgen05.cp 32x128b.warpx4) and issues
 //             2 x 4 x tcgen05.mma.kind::mxf4.block_scale (M=128, N=tile, K=64)
-//   warp 2    scale producer: reads the stage's e8m0 scales through their strides
-//             and writes them in the 128-row x 4-block atom the tensor core reads:
+//   warp 2    scale producer: reads the next stage's e8m0 scales through their
+//             strides (loads in flight while it waits for the slot) and writes
+//             them in the 128-row x 4-block atom the tensor core reads:
 //             byte (row % 32) * 16 + (row / 32) * 4 + block
 //   warps 3-6 epilogue (one weight row per thread)
 // TMEM: kBufs accumulator buffers of 2 x kNmax columns, then 24 scale columns
@@ -38,10 +39,12 @@ constexpr int kUmmaKBytes = 32;                // 64 e2m1 elements per instructi
 constexpr int kAtomBytes = 512;                // 128 rows x 4 scale blocks
 constexpr int kSfBytes = 2 * kAtomBytes;       // 8 blocks of 32 per stage
 constexpr int kEpiWarps = 4;
+constexpr int kSfWarps = 1;                    // scale producers, taking k-steps in turn
+constexpr int kFirstEpiWarp = 2 + kSfWarps;
 constexpr int kStagingBytes = 32 * 64;
 constexpr int kSfColsPerStage = 24;
 constexpr int kTmemCols = 512;
-constexpr int kThreads = 224;
+constexpr int kThreads = 32 * (kFirstEpiWarp + kEpiWarps);
 
 template <int kNmax, int kStages>
 struct Cfg {
@@ -192,18 +195,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (last_phase[s] >= 0) mbar_wait(&sm.full[s], static_cast<uint32_t>(last_phase[s]), g.err);
       }
     }
-  } else if (warp == 2) {
-    // ------------------------------------------------------------ scale producer
-    uint32_t stage = 0, phase = 0;
+  } else if (warp >= 2 && warp < kFirstEpiWarp) {
+    // ------------------------------------------------------------ scale producers
+    const uint32_t sfw = static_cast<uint32_t>(warp - 2);
+    uint32_t gstep = 0;  // k-steps issued so far by the CTA (all items)
     bool ok = true;
     for (int64_t item = blockIdx.x; item < total && ok; item += gridDim.x) {
       const int64_t t = item / g.n_wt, wt = item - t * g.n_wt;
       const int32_t e = g.tile_expert[t], row0 = g.tile_row[t], rows = g.tile_rows[t];
       const int64_t w0 = kMode == 0 ? wt * kWRows : wt * 2 * kWRows;
       const int64_t w1 = kMode == 0 ? w0 : w0 + kWRows;
-      for (int kb = 0; kb < num_k; ++kb) {
-        if (!mbar_wait(&sm.empty[stage], phase ^ 1u, g.err)) { ok = false; break; }
-        uint8_t* sf = sm.stages + stage * C::kStageBytes + 2 * C::kWBytes + C::kTokBytes;
+      for (int kb = 0; kb < num_k; ++kb, ++gstep) {
+        if (gstep % kSfWarps != sfw) continue;
+        const uint32_t stage = gstep % kStages;
+        const uint32_t phase = (gstep / kStages) & 1u;
         uint32_t a_lo[4], a_hi[4], b_lo[4], b_hi[4], x_lo[4], x_hi[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -217,6 +222,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           b_lo[j] = v1.x; b_hi[j] = v1.y;
           x_lo[j] = vx.x; x_hi[j] = vx.y;
         }
+        // the loads above are in flight while this warp waits for the slot
+        if (!mbar_wait(&sm.empty[stage], phase ^ 1u, g.err)) { ok = false; break; }
+        uint8_t* sf = sm.stages + stage * C::kStageBytes + 2 * C::kWBytes + C::kTokBytes;
         const uint32_t s0 = smem_u32(sf) + 16 * lane;
         st_v4(s0, a_lo);
         st_v4(s0 + kAtomBytes, a_hi);
@@ -227,7 +235,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.full[stage]);
-        if (++stage == kStages) { stage = 0; phase ^= 1u; }
       }
     }
   } else if (warp == 1) {
@@ -281,12 +288,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int quad = warp & 3;
-    uint8_t* stg = sm.staging + (warp - 3) * kStagingBytes;
+    uint8_t* stg = sm.staging + (warp - kFirstEpiWarp) * kStagingBytes;
     const uint32_t stg_s = smem_u32(stg);
     uint32_t buf = 0, acc_phase = 0;
     for (int64_t item = blockIdx.x; item < total; item += gridDim.x) {
       const int64_t t = item / g.n_wt, wt = item - t * g.n_wt;
       const int32_t row0 = g.tile_row[t], rows = g.tile_rows[t];
+      // GEMM2: slots and routing weights of the tile's tokens (lane j of chunk c
+      // holds token c*32 + j), fetched while the accumulator is still being built
+      int32_t slot_r[kNmax / 32];
+      float w_r[kNmax / 32];
+      if (kMode == 1) {
+#pragma unroll
+        for (int c = 0; c < kNmax / 32; ++c)
+          slot_r[c] = (c * 32 < rows) ? g.sorted[row0 + c * 32 + lane] : static_cast<int32_t>(g.S);
+#pragma unroll
+        for (int c = 0; c < kNmax / 32; ++c) {
+          w_r[c] = 0.0f;
+          if (slot_r[c] < g.S) {
+            const int64_t tt = slot_r[c] / g.k, jj = slot_r[c] - tt * g.k;
+            w_r[c] = static_cast<const float*>(g.topk_w.data)[tt * g.topk_w.s0 + jj * g.topk_w.s1];
+          }
+        }
+      }
       if (!mbar_wait(&sm.tfull[buf], acc_phase, g.err)) break;
       tc_fence_after();
       const uint32_t lane_base = (static_cast<uint32_t>(quad * 32) << 16) + buf * C::kBufCols;
@@ -334,14 +358,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int a = 0; a < 2; ++a) {
           const int64_t col0 = wt * 2 * kWRows + a * kWRows + quad * 32;
           const bool col_ok = col0 < g.N;
-#pragma unroll 1
-          for (int c = 0; c < rows / 32; ++c) {
-            int32_t my_slot = g.sorted[row0 + c * 32 + lane];
-            float my_w = 0.0f;
-            if (my_slot < g.S) {
-              const int64_t tt = my_slot / g.k, jj = my_slot - tt * g.k;
-              my_w = static_cast<const float*>(g.topk_w.data)[tt * g.topk_w.s0 + jj * g.topk_w.s1];
-            }
+#pragma unroll
+          for (int c = 0; c < kNmax / 32; ++c) {
+            if (c * 32 >= rows) break;
+            const int32_t my_slot = slot_r[c];
+            const float my_w = w_r[c];
             uint32_t v0[32];
             tmem_ld32(tmem_base + lane_base + a * kNmax + c * 32, v0);
             tmem_wait_ld();

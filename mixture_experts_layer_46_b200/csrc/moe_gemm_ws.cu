@@ -219,6 +219,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int64_t item = blockIdx.x; item < total; item += gridDim.x) {
       const int64_t t = item / g.n_wt, wt = item - t * g.n_wt;
       const int32_t row0 = g.tile_row[t], rows = g.tile_rows[t];
+      // GEMM2: slots and routing weights of the tile's tokens (lane j of chunk c
+      // holds token c*32 + j), fetched while the accumulator is still being built
+      int32_t slot_r[kNmax / 32];
+      float w_r[kNmax / 32];
+      if (kMode == 1) {
+#pragma unroll
+        for (int c = 0; c < kNmax / 32; ++c)
+          slot_r[c] = (c * 32 < rows) ? g.sorted[row0 + c * 32 + lane] : static_cast<int32_t>(g.S);
+#pragma unroll
+        for (int c = 0; c < kNmax / 32; ++c) {
+          w_r[c] = 0.0f;
+          if (slot_r[c] < g.S) {
+            const int64_t tt = slot_r[c] / g.k, jj = slot_r[c] - tt * g.k;
+            w_r[c] = static_cast<const float*>(g.topk_w.data)[tt * g.topk_w.s0 + jj * g.topk_w.s1];
+          }
+        }
+      }
       if (!mbar_wait(&sm.tfull[buf], acc_phase, g.err)) break;
       tc_fence_after();
       const uint32_t lane_base = (static_cast<uint32_t>(quad * 32) << 16) + buf * C::kBufCols;
@@ -229,18 +246,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t col0 = (kMode == 0) ? wt * kWRows + quad * 32
                                           : wt * 2 * kWRows + a * kWRows + quad * 32;
         const bool col_ok = col0 < g.N;
-#pragma unroll 1
-        for (int c = 0; c < rows / 32; ++c) {
-          // GEMM2: lane j holds the slot and routing weight of token c*32 + j
-          int32_t my_slot = 0;
-          float my_w = 0.0f;
-          if (kMode == 1) {
-            my_slot = g.sorted[row0 + c * 32 + lane];
-            if (my_slot < g.S) {
-              const int64_t tt = my_slot / g.k, jj = my_slot - tt * g.k;
-              my_w = static_cast<const float*>(g.topk_w.data)[tt * g.topk_w.s0 + jj * g.topk_w.s1];
-            }
-          }
+#pragma unroll
+        for (int c = 0; c < kNmax / 32; ++c) {
+          if (c * 32 >= rows) break;
+          const int32_t my_slot = (kMode == 1) ? slot_r[c] : 0;
+          const float my_w = (kMode == 1) ? w_r[c] : 0.0f;
           uint32_t v0[32];
           tmem_ld32(tmem_base + lane_base + a * kNmax + c * 32, v0);
           if (kMode == 0) {
