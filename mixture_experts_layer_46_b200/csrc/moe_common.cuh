@@ -253,6 +253,20 @@ __device__ __forceinline__ uint64_t plain_rows16_desc(uint32_t smem_addr) {
   return d;
 }
 
+// 4-byte asynchronous global->shared copy; src_bytes = 0 writes zeros instead.
+__device__ __forceinline__ void cp_async_4(uint32_t dst_smem, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst_smem), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+
+// Arrive on an mbarrier once this thread's earlier cp.async copies have landed.
+// The pending count is raised now and lowered on completion (no arrival of its
+// own): pair it with a regular arrive.
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // Make this thread's generic-proxy shared-memory writes visible to the async
 // proxy (TMA, tensor cores) once ordered by a barrier.
 __device__ __forceinline__ void fence_proxy_async_smem() {

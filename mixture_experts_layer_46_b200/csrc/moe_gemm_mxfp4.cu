@@ -12,17 +12,18 @@
 // Expert addressing: 3-D TMA maps whose expert stride is each view's real
 // stride(0) (Liger-Kernel PR #1377, "Problems").
 //
-// Kernel shape: one persistent CTA per SM, 7 warps.
+// Kernel shape: one persistent CTA per SM, 11 warps.
 //   warp 0    TMA producer: two weight boxes [128 rows x 128 B] + the token tile
 //             in 32-row boxes per k-step (256 elements of K), 128-byte swizzle
 //   warp 1    TMEM allocator, MMA issuer: per stage copies the stage's scales
 //             from shared memory to TMEM (tcgen05.cp 32x128b.warpx4) and issues
 //             2 x 4 x tcgen05.mma.kind::mxf4.block_scale (M=128, N=tile, K=64)
-//   warp 2    scale producer: reads the next stage's e8m0 scales through their
-//             strides (loads in flight while it waits for the slot) and writes
-//             them in the 128-row x 4-block atom the tensor core reads:
-//             byte (row % 32) * 16 + (row / 32) * 4 + block
-//   warps 3-6 epilogue (one weight row per thread)
+//   warp 2    scale producer: copies the stage's e8m0 scales through their
+//             strides with 4-byte cp.async straight into the 128-row x 4-block
+//             atom the tensor core reads: byte (row % 32) * 16 + (row / 32) * 4
+//             + block; the stage barrier completes when the copies land
+//   warps 3-10 epilogue: two warps per 32-lane TMEM quadrant (one weight row
+//             per thread), each taking every other 32-token chunk
 // TMEM: kBufs accumulator buffers of 2 x kNmax columns, then 24 scale columns
 // per stage (two weight tiles and the token tile, each 2 atoms x 4 columns).
 #include "../../include/moe.h"
@@ -38,8 +39,8 @@ constexpr int kTokBox = 32;
 constexpr int kUmmaKBytes = 32;                // 64 e2m1 elements per instruction
 constexpr int kAtomBytes = 512;                // 128 rows x 4 scale blocks
 constexpr int kSfBytes = 2 * kAtomBytes;       // 8 blocks of 32 per stage
-constexpr int kEpiWarps = 4;
-constexpr int kSfWarps = 1;                    // scale producers, taking k-steps in turn
+constexpr int kEpiWarps = 8;                   // two per TMEM lane quadrant, alternating chunks
+constexpr int kSfWarps = 1;                    // scale producer warps
 constexpr int kFirstEpiWarp = 2 + kSfWarps;
 constexpr int kStagingBytes = 32 * 64;
 constexpr int kSfColsPerStage = 24;
@@ -112,16 +113,6 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   return s;
 }
 
-__device__ __forceinline__ uint2 ld_u2(const uint8_t* p) {
-  return *reinterpret_cast<const uint2*>(p);
-}
-
-__device__ __forceinline__ void st_v4(uint32_t addr, const uint32_t (&v)[4]) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v[0]), "r"(v[1]),
-               "r"(v[2]), "r"(v[3])
-               : "memory");
-}
-
 template <int kMode, int kNmax, int kStages>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_ws_mxfp4_kernel(const __grid_constant__ CUtensorMap tmW0,
@@ -137,7 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (kMode == 0) tma_prefetch_desc(&tmW1);
     tma_prefetch_desc(&tmX);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sm.full[s], 2);  // TMA producer (with bytes) + scale producer
+      mbar_init(&sm.full[s], 1 + 32);  // TMA producer (with bytes) + 32 scale-producer lanes
       mbar_init(&sm.empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -196,45 +187,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp >= 2 && warp < kFirstEpiWarp) {
-    // ------------------------------------------------------------ scale producers
-    const uint32_t sfw = static_cast<uint32_t>(warp - 2);
-    uint32_t gstep = 0;  // k-steps issued so far by the CTA (all items)
+    // ------------------------------------------------------------ scale producer
+    // Asynchronous 4-byte copies place every scale word directly at its atom
+    // position; the stage's full barrier completes only once they have landed,
+    // so this warp never waits for load latency and runs ahead like the TMA warp.
+    uint32_t stage = 0, phase = 0;
     bool ok = true;
     for (int64_t item = blockIdx.x; item < total && ok; item += gridDim.x) {
       const int64_t t = item / g.n_wt, wt = item - t * g.n_wt;
       const int32_t e = g.tile_expert[t], row0 = g.tile_row[t], rows = g.tile_rows[t];
       const int64_t w0 = kMode == 0 ? wt * kWRows : wt * 2 * kWRows;
       const int64_t w1 = kMode == 0 ? w0 : w0 + kWRows;
-      for (int kb = 0; kb < num_k; ++kb, ++gstep) {
-        if (gstep % kSfWarps != sfw) continue;
-        const uint32_t stage = gstep % kStages;
-        const uint32_t phase = (gstep / kStages) & 1u;
-        uint32_t a_lo[4], a_hi[4], b_lo[4], b_hi[4], x_lo[4], x_hi[4];
+      for (int kb = 0; kb < num_k; ++kb) {
+        if (!mbar_wait(&sm.empty[stage], phase ^ 1u, g.err)) { ok = false; break; }
+        const uint32_t sf = smem_u32(sm.stages + stage * C::kStageBytes + 2 * C::kWBytes + C::kTokBytes);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const int64_t r = lane + 32 * j;  // row inside the tile (atom row = lane, column = j)
-          // rows outside the weight matrix or the token tile read as scale 0
-          uint2 v0 = make_uint2(0, 0), v1 = make_uint2(0, 0), vx = make_uint2(0, 0);
-          if (w0 + r < g.N) v0 = ld_u2(g.w0_sf + e * g.w0_s0 + (w0 + r) * g.w0_s1 + kb * 8);
-          if (w1 + r < g.N) v1 = ld_u2(g.w1_sf + e * g.w1_s0 + (w1 + r) * g.w1_s1 + kb * 8);
-          if (r < rows) vx = ld_u2(g.x_sf + (row0 + r) * g.x_sf_ld + kb * 8);
-          a_lo[j] = v0.x; a_hi[j] = v0.y;
-          b_lo[j] = v1.x; b_hi[j] = v1.y;
-          x_lo[j] = vx.x; x_hi[j] = vx.y;
+          const int64_t r = lane + 32 * j;  // row inside the tile: atom row = lane, column = j
+          const uint32_t dst = sf + 16 * lane + 4 * j;
+          // rows outside the weight matrix or the token tile are zero-filled
+          const uint8_t* p0 = g.w0_sf + e * g.w0_s0 + (w0 + r) * g.w0_s1 + kb * 8;
+          const uint8_t* p1 = g.w1_sf + e * g.w1_s0 + (w1 + r) * g.w1_s1 + kb * 8;
+          const uint8_t* px = g.x_sf + (row0 + r) * g.x_sf_ld + kb * 8;
+          const uint32_t n0 = (w0 + r < g.N) ? 4u : 0u;
+          const uint32_t n1 = (w1 + r < g.N) ? 4u : 0u;
+          const uint32_t nx = (r < rows) ? 4u : 0u;
+          cp_async_4(dst, n0 ? p0 : g.w0_sf, n0);
+          cp_async_4(dst + kAtomBytes, n0 ? p0 + 4 : g.w0_sf, n0);
+          cp_async_4(dst + kSfBytes, n1 ? p1 : g.w1_sf, n1);
+          cp_async_4(dst + kSfBytes + kAtomBytes, n1 ? p1 + 4 : g.w1_sf, n1);
+          cp_async_4(dst + 2 * kSfBytes, nx ? px : g.x_sf, nx);
+          cp_async_4(dst + 2 * kSfBytes + kAtomBytes, nx ? px + 4 : g.x_sf, nx);
         }
-        // the loads above are in flight while this warp waits for the slot
-        if (!mbar_wait(&sm.empty[stage], phase ^ 1u, g.err)) { ok = false; break; }
-        uint8_t* sf = sm.stages + stage * C::kStageBytes + 2 * C::kWBytes + C::kTokBytes;
-        const uint32_t s0 = smem_u32(sf) + 16 * lane;
-        st_v4(s0, a_lo);
-        st_v4(s0 + kAtomBytes, a_hi);
-        st_v4(s0 + kSfBytes, b_lo);
-        st_v4(s0 + kSfBytes + kAtomBytes, b_hi);
-        st_v4(s0 + 2 * kSfBytes, x_lo);
-        st_v4(s0 + 2 * kSfBytes + kAtomBytes, x_hi);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.full[stage]);
+        cp_async_mbar_arrive(&sm.full[stage]);
+        mbar_arrive(&sm.full[stage]);
+        if (++stage == kStages) { stage = 0; phase ^= 1u; }
       }
     }
   } else if (warp == 1) {
@@ -251,6 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < num_k; ++kb) {
           if (!mbar_wait(&sm.full[stage], phase, g.err)) { ok = false; break; }
           tc_fence_after();
+          fence_proxy_async_smem();  // scales were written by cp.async, read by tcgen05.cp
           const uint32_t w0_addr = smem_u32(sm.stages + stage * C::kStageBytes);
           const uint32_t w1_addr = w0_addr + C::kWBytes;
           const uint32_t x_addr = w1_addr + C::kWBytes;
@@ -288,6 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int quad = warp & 3;
+    const int half = (warp - kFirstEpiWarp) >> 2;  // which of the quadrant's two warps
     uint8_t* stg = sm.staging + (warp - kFirstEpiWarp) * kStagingBytes;
     const uint32_t stg_s = smem_u32(stg);
     uint32_t buf = 0, acc_phase = 0;
@@ -318,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // this warp's 32 weight rows = one 1x32 block of I for every token
         const int64_t i0 = wt * kWRows + quad * 32;
 #pragma unroll 1
-        for (int c = 0; c < rows / 32; ++c) {
+        for (int c = half; c < rows / 32; c += 2) {
           uint32_t gv[32], uv[32];
           tmem_ld32(tmem_base + lane_base + c * 32, gv);
           tmem_ld32(tmem_base + lane_base + kNmax + c * 32, uv);
@@ -327,9 +316,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const float h = silu_mul(__uint_as_float(gv[j]), __uint_as_float(uv[j]));
-            float amax = fabsf(h);
-#pragma unroll
-            for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
+            // |h| as bits orders like its value: one warp reduction gives the block amax
+            const float amax = __uint_as_float(
+                __reduce_max_sync(0xffffffffu, __float_as_uint(h) & 0x7fffffffu));
             const int sexp = mx_scale_exp(amax);
             const float q = h * exp2i_neg(sexp);
             const float qn = __shfl_xor_sync(0xffffffffu, q, 1);
@@ -354,21 +343,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
         }
       } else {
-#pragma unroll 1
-        for (int a = 0; a < 2; ++a) {
-          const int64_t col0 = wt * 2 * kWRows + a * kWRows + quad * 32;
-          const bool col_ok = col0 < g.N;
+        // both accumulators of a 32-token chunk are loaded together (one wait)
+        // and share the chunk's routing weights
 #pragma unroll
-          for (int c = 0; c < kNmax / 32; ++c) {
-            if (c * 32 >= rows) break;
-            const int32_t my_slot = slot_r[c];
-            const float my_w = w_r[c];
-            uint32_t v0[32];
-            tmem_ld32(tmem_base + lane_base + a * kNmax + c * 32, v0);
-            tmem_wait_ld();
+        for (int c = 0; c < kNmax / 32; ++c) {
+          if (c * 32 >= rows) break;
+          if ((c & 1) != half) continue;
+          const int32_t my_slot = slot_r[c];
+          const float my_w = w_r[c];
+          uint32_t v0[32], v1[32];
+          tmem_ld32(tmem_base + lane_base + c * 32, v0);
+          tmem_ld32(tmem_base + lane_base + kNmax + c * 32, v1);
+          float wj[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) wj[j] = __shfl_sync(0xffffffffu, my_w, j);
+          tmem_wait_ld();
+#pragma unroll
+          for (int a = 0; a < 2; ++a) {
+            const int64_t col0 = wt * 2 * kWRows + a * kWRows + quad * 32;
+            const bool col_ok = col0 < g.N;
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-              const float y = __shfl_sync(0xffffffffu, my_w, j) * __uint_as_float(v0[j]);
+              const float y = wj[j] * __uint_as_float(a == 0 ? v0[j] : v1[j]);
               const __nv_bfloat16 yb = __float2bfloat16_rn(y);
               asm volatile("st.shared.b16 [%0], %1;" ::"r"(stg_s + j * 64 + lane * 2),
                            "h"(*reinterpret_cast<const uint16_t*>(&yb)) : "memory");
