@@ -345,7 +345,7 @@ WsLayout make_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, bool
     L.h = take(size_t(p) * I / 2);
     L.h_scale = take(size_t(p) * I / 32);
   }
-  L.y = take(size_t(S > 0 ? S : 1) * H * 2);
+  L.y = take(size_t(p) * H * 2);
   L.total = off;
   return L;
 }
@@ -466,8 +466,8 @@ moe_status_t forward_mxfp4(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   rc = launch_gemm_ws_mxfp4(1, L.tile_max, mW2, mW2, mH, g2, dev->num_sms, st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm2_mxfp4");
   prof_mark(st);
-  rc = launch_combine(reinterpret_cast<const __nv_bfloat16*>(w + L.y), view2(ids), pr.E, pr.T,
-                      pr.H, pr.k, out->data, out->strides[0], out->strides[1], st, &launches);
+  rc = launch_combine(reinterpret_cast<const __nv_bfloat16*>(w + L.y), inv, pr.T, pr.H, pr.k,
+                      out->data, out->strides[0], out->strides[1], st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "combine");
   prof_mark(st);
   t_prof.have = t_prof.on && t_prof.n == kProfSteps + 1;
@@ -592,8 +592,8 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm2");
   prof_mark(st);
 
-  rc = launch_combine(reinterpret_cast<const __nv_bfloat16*>(w + L.y), view2(ids), pr.E, pr.T,
-                      pr.H, pr.k, out->data, out->strides[0], out->strides[1], st, &launches);
+  rc = launch_combine(reinterpret_cast<const __nv_bfloat16*>(w + L.y), inv, pr.T, pr.H, pr.k,
+                      out->data, out->strides[0], out->strides[1], st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "combine");
   prof_mark(st);
   t_prof.have = t_prof.on && t_prof.n == kProfSteps + 1;

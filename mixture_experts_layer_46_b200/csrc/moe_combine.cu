@@ -1,5 +1,6 @@
-// Step "combine": out[t, :] = sum_{j = 0..k-1} y[t*k + j, :] over the valid
-// slots of token t, accumulated in fp32 in fixed j order and rounded once to
+// Step "combine": out[t, :] = sum_{j = 0..k-1} y[inv[t*k + j], :] over the
+// valid slots of token t (inv = the slot's row in expert-grouped order, -1 for
+// a skipped slot), accumulated in fp32 in fixed j order and rounded once to
 // bf16.  The routing weight is already folded into y by the down-projection
 // epilogue.  No atomics, so the result is identical run to run and does not
 // depend on how the slots were grouped.  out is written through its strides.
@@ -8,12 +9,6 @@
 
 namespace moe {
 namespace {
-
-__device__ __forceinline__ int64_t read_id2(const View2& v, int64_t t, int64_t j) {
-  const int64_t off = t * v.s0 + j * v.s1;
-  if (v.dtype == MOE_I64) return static_cast<const int64_t*>(v.data)[off];
-  return static_cast<int64_t>(static_cast<const int32_t*>(v.data)[off]);
-}
 
 __device__ __forceinline__ void acc_bf16x8(float (&a)[8], const uint4& v) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -25,31 +20,23 @@ __device__ __forceinline__ void acc_bf16x8(float (&a)[8], const uint4& v) {
 }
 
 __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __restrict__ y,
-                                                      View2 ids, int64_t E, int64_t T, int64_t H,
-                                                      int64_t k, __nv_bfloat16* out, int64_t os0,
-                                                      int64_t os1, int vec_out) {
-  __shared__ uint32_t valid_mask;
+                                                      const int32_t* __restrict__ inv, int64_t T,
+                                                      int64_t H, int64_t k, __nv_bfloat16* out,
+                                                      int64_t os0, int64_t os1, int vec_out) {
+  __shared__ int32_t rows_sh[kMaxTopK];
   pdl_wait();
   pdl_launch_dependents();
   const int64_t H8 = H / 8;
   for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
     __syncthreads();
-    if (threadIdx.x < 32) {
-      bool ok = false;
-      if (threadIdx.x < k) {
-        const int64_t e = read_id2(ids, t, threadIdx.x);
-        ok = (e >= 0 && e < E);
-      }
-      const uint32_t m = __ballot_sync(0xffffffffu, ok);
-      if (threadIdx.x == 0) valid_mask = m;
-    }
+    if (threadIdx.x < k) rows_sh[threadIdx.x] = inv[t * k + threadIdx.x];
     __syncthreads();
-    const uint32_t vm = valid_mask;
-    const __nv_bfloat16* yt = y + t * k * H;
     for (int64_t c = threadIdx.x; c < H8; c += blockDim.x) {
       float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      for (int j = 0; j < k; ++j)
-        if (vm & (1u << j)) acc_bf16x8(a, reinterpret_cast<const uint4*>(yt + j * H)[c]);
+      for (int j = 0; j < k; ++j) {
+        const int32_t r = rows_sh[j];
+        if (r >= 0) acc_bf16x8(a, reinterpret_cast<const uint4*>(y + static_cast<int64_t>(r) * H)[c]);
+      }
       if (vec_out) {
         uint4 o;
         o.x = pack_bf16x2(a[0], a[1]);
@@ -67,16 +54,16 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
 
 }  // namespace
 
-cudaError_t launch_combine(const __nv_bfloat16* y, const View2& ids, int64_t E, int64_t T,
-                           int64_t H, int64_t k, void* out, int64_t os0, int64_t os1,
-                           cudaStream_t st, int* launches) {
+cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* inv, int64_t T, int64_t H,
+                           int64_t k, void* out, int64_t os0, int64_t os1, cudaStream_t st,
+                           int* launches) {
   const int vec_out = (os1 == 1) && ((os0 * 2) % 16 == 0) &&
                       (reinterpret_cast<uintptr_t>(out) % 16 == 0);
   int64_t blocks = T < 148 * 16 ? T : 148 * 16;
   if (blocks < 1) blocks = 1;
   if (launches) *launches += 1;
-  return launch_pdl(combine_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, y, ids,
-                    E, T, H, k, static_cast<__nv_bfloat16*>(out), os0, os1, vec_out);
+  return launch_pdl(combine_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, y, inv,
+                    T, H, k, static_cast<__nv_bfloat16*>(out), os0, os1, vec_out);
 }
 
 }  // namespace moe

@@ -380,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                            : "r"(stg_s + j * 64 + part * 16));
               const int32_t s_j = __shfl_sync(0xffffffffu, my_slot, j);
               if (col_ok && s_j < g.S)
-                *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + static_cast<int64_t>(s_j) * g.out_ld + col0 + part * 8) = v;
+                *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + (row0 + c * 32 + j) * g.out_ld + col0 + part * 8) = v;
             }
             __syncwarp();
           }

@@ -291,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + p * g.out_ld + col0 + part * 8) = v;
             } else {
               if (s_j < g.S)
-                *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + static_cast<int64_t>(s_j) * g.out_ld + col0 + part * 8) = v;
+                *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + (row0 + c * 32 + j) * g.out_ld + col0 + part * 8) = v;
             }
           }
           __syncwarp();

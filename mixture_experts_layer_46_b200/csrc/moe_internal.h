@@ -73,10 +73,10 @@ cudaError_t launch_permute_quant(const View2& x, int64_t T, int64_t H, int64_t k
                                  const int32_t* inv, const int32_t* offsets, const int32_t* counts,
                                  uint8_t* codes, uint8_t* scales, cudaStream_t st, int* launches);
 
-// combine: out[t, :] = sum_j y[t*k + j, :] over valid slots (fixed j order)
-cudaError_t launch_combine(const __nv_bfloat16* y, const View2& ids, int64_t E, int64_t T,
-                           int64_t H, int64_t k, void* out, int64_t os0, int64_t os1,
-                           cudaStream_t st, int* launches);
+// combine: out[t, :] = sum_j y[inv[t*k + j], :] over valid slots (fixed j order)
+cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* inv, int64_t T, int64_t H,
+                           int64_t k, void* out, int64_t os0, int64_t os1, cudaStream_t st,
+                           int* launches);
 
 struct GemmArgs {
   int64_t K;            // contraction length
