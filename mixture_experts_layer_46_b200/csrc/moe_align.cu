@@ -128,8 +128,8 @@ __device__ int block_scan_experts(int64_t E, F v, int* out) {
 }
 
 // Outputs of align beyond sorted/offsets: the token-tile list consumed by the
-// weight-stationary GEMMs (tiles of up to tile_max rows, never crossing an
-// expert), written when tile_max > 0.
+// weight-stationary GEMMs (tiles of at most tile_max rows, balanced within an
+// expert, never crossing one), written when tile_max > 0.
 struct TileOut {
   int32_t tile_max;
   int32_t* tile_row;     // first padded row of the tile
@@ -167,12 +167,21 @@ __device__ void block_finalize(const int* cnt, int64_t E, int32_t bm, int32_t S,
     const int tm = to.tile_max;
     const int nt = block_scan_experts(
         E, [&](int e) { return (offs[e + 1] - offs[e] + tm - 1) / tm; }, tsc);
+    // an expert's rows are split into its n tiles as evenly as the bm granule
+    // allows (e.g. 288 rows with tm = 256 -> 160 + 128, not 256 + 32), so no
+    // work item streams a whole weight tile for a handful of tokens
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
       const int rows = offs[e + 1] - offs[e];
-      for (int j = 0, t = tsc[e]; j * tm < rows; ++j, ++t) {
-        to.tile_row[t] = offs[e] + j * tm;
-        to.tile_rows[t] = min(tm, rows - j * tm);
-        to.tile_expert[t] = e;
+      const int n = (rows + tm - 1) / tm;
+      if (n == 0) continue;
+      const int units = rows / bm;  // rows is a multiple of bm
+      int start = offs[e];
+      for (int j = 0; j < n; ++j) {
+        const int u = units / n + (j < units % n ? 1 : 0);
+        to.tile_row[tsc[e] + j] = start;
+        to.tile_rows[tsc[e] + j] = u * bm;
+        to.tile_expert[tsc[e] + j] = e;
+        start += u * bm;
       }
     }
     if (threadIdx.x == 0) *to.num_tiles = nt;

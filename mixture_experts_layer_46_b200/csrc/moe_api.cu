@@ -285,13 +285,13 @@ void choose_tiling(int64_t T, int64_t k, int64_t E, bool mxfp4, int32_t* bm, int
   // weight-stationary bf16 kernels: tokens are the MMA's N side in 32-row
   // granules, in tiles of up to 32 rows while experts average <= 8 slots
   // (decode: 6-stage ring, more weight bytes in flight) and up to 128 rows
-  // beyond (double-buffered accumulators).  MOE_TILE=32|128 overrides (tuning).
+  // beyond (double-buffered accumulators).  MOE_TILE overrides (tuning).
   *bm = 32;
   const int64_t avg = E > 0 ? (T * k) / E : 0;
   *tile_max = avg <= 8 ? 32 : 128;
   if (const char* env = getenv("MOE_TILE")) {
     const int v = atoi(env);
-    if (v == 32 || v == 128) *tile_max = v;
+    if (v == 32 || v == 128 || v == 256) *tile_max = v;
   }
 }
 
@@ -506,8 +506,16 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   // ---- tensor maps (bf16, 128-byte swizzle): weights in [64 x 128] boxes,
   // gathered token rows in [64 x 32] boxes
   CUtensorMap mA1, mGate, mUp, mH, mW2;
+  // 128-row token tiles run on CTA pairs once experts average >= 32 slots (the
+  // pair moves a sixth fewer shared-memory bytes per FLOP and keeps 5 stages in
+  // flight); MOE_PAIR=0|1 and MOE_WPOLICY=1 (weights evict-first in L2) are
+  // tuning overrides
+  bool pair = (L.tile_max >= 128) && (pr.T * pr.k >= 32 * pr.E);
+  if (const char* env = getenv("MOE_PAIR")) pair = (L.tile_max >= 128) && atoi(env) != 0;
+  if (L.tile_max == 256) pair = true;  // 256-row tiles exist only on CTA pairs
+  const int32_t wpolicy = getenv("MOE_WPOLICY") ? atoi(getenv("MOE_WPOLICY")) : 0;
   const uint32_t boxw[3] = {64, 128, 1};
-  const uint32_t boxt[2] = {64, 32};
+  const uint32_t boxt[2] = {64, pair ? 16u : 32u};
   {
     const uint64_t d[2] = {uint64_t(pr.H), uint64_t(L.p_max)};
     const uint64_t sb[1] = {uint64_t(pr.H) * 2};
@@ -565,7 +573,7 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   std::memset(&g1, 0, sizeof(g1));
   g1.K = pr.H;
   g1.N = pr.I;
-  g1.n_wt = (pr.I + 127) / 128;
+  g1.n_wt = pair ? (pr.I + 255) / 256 : (pr.I + 127) / 128;
   g1.max_tiles = L.t_max;
   g1.num_tiles = tiles.num_tiles;
   g1.tile_row = tiles.tile_row;
@@ -577,18 +585,21 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   g1.out_ld = pr.I;
   g1.k = pr.k;
   g1.err = dev->errors;
-  rc = launch_gemm_ws_bf16(0, L.tile_max, mGate, mUp, mA1, g1, dev->num_sms, st, &launches);
+  g1.weights_evict_first = wpolicy;
+  rc = pair ? launch_gemm_ws_pair_bf16(0, L.tile_max, mGate, mUp, mA1, g1, dev->num_sms, st, &launches)
+            : launch_gemm_ws_bf16(0, L.tile_max, mGate, mUp, mA1, g1, dev->num_sms, st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm1");
   prof_mark(st);
 
   WsGemm g2 = g1;
   g2.K = pr.I;
   g2.N = pr.H;
-  g2.n_wt = (pr.H + 255) / 256;
+  g2.n_wt = pair ? (pr.H + 511) / 512 : (pr.H + 255) / 256;
   g2.out = w + L.y;
   g2.out_ld = pr.H;
   g2.topk_w = view2(wts);
-  rc = launch_gemm_ws_bf16(1, L.tile_max, mW2, mW2, mH, g2, dev->num_sms, st, &launches);
+  rc = pair ? launch_gemm_ws_pair_bf16(1, L.tile_max, mW2, mW2, mH, g2, dev->num_sms, st, &launches)
+            : launch_gemm_ws_bf16(1, L.tile_max, mW2, mW2, mH, g2, dev->num_sms, st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm2");
   prof_mark(st);
 

@@ -280,8 +280,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// silu(g) * u = g / (1 + e^-g) * u with the fast exponential and division
+// intrinsics (both within a few ulp of fp32, far inside the 1e-2 bound).
 __device__ __forceinline__ float silu_mul(float g, float u) {
-  return g / (1.0f + __expf(-g)) * u;
+  return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
 // Programmatic dependent launch: let the next kernel in the stream start its

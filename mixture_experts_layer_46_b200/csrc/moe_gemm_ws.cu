@@ -67,6 +67,7 @@ struct WsArgs {
   int64_t out_ld;
   View2 topk_w;
   int64_t k;
+  int32_t weights_evict_first;
   DeviceErrors* err;
 };
 
@@ -144,6 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int8_t last_phase[kStages];
       for (int s = 0; s < kStages; ++s) last_phase[s] = -1;
       const uint64_t pol = l2_policy_evict_last();
+      const uint64_t wpol = g.weights_evict_first ? l2_policy_evict_first() : pol;
       bool ok = true;
       for (int64_t item = blockIdx.x; item < total && ok; item += gridDim.x) {
         const int64_t t = item / g.n_wt, wt = item - t * g.n_wt;
@@ -158,8 +160,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* sw1 = sw0 + C::kWBytes;
           uint8_t* sx = sw1 + C::kWBytes;
           mbar_arrive_expect_tx(&sm.full[stage], bytes);
-          tma_load_3d(sw0, &tmW0, &sm.full[stage], kb * kBK, w0, e, pol);
-          tma_load_3d(sw1, kMode == 0 ? &tmW1 : &tmW0, &sm.full[stage], kb * kBK, w1, e, pol);
+          tma_load_3d(sw0, &tmW0, &sm.full[stage], kb * kBK, w0, e, wpol);
+          tma_load_3d(sw1, kMode == 0 ? &tmW1 : &tmW0, &sm.full[stage], kb * kBK, w1, e, wpol);
           for (int b = 0; b < nbox; ++b)
             tma_load_2d(sx + b * kTokBox * kBK * 2, &tmX, &sm.full[stage], kb * kBK,
                         row0 + b * kTokBox, pol);
@@ -353,6 +355,7 @@ cudaError_t launch_gemm_ws_bf16(int mode, int tile_max, const CUtensorMap& w0,
   g.topk_w = p.topk_w;
   g.k = p.k;
   g.err = p.err;
+  g.weights_evict_first = p.weights_evict_first;
   if (launches) *launches += 1;
   const int64_t max_items = p.max_tiles * p.n_wt;
   if (tile_max == 128) {

@@ -109,6 +109,7 @@ struct WsGemm {
   int64_t out_ld;
   View2 topk_w;
   int64_t k;
+  int32_t weights_evict_first;  // L2 policy of the weight loads (tokens: evict-last)
   DeviceErrors* err;
 };
 // mode 0: GEMM1 (gate/up + SwiGLU -> h), mode 1: GEMM2 (down + routing weight -> y)
@@ -116,6 +117,12 @@ struct WsGemm {
 cudaError_t launch_gemm_ws_bf16(int mode, int tile_max, const CUtensorMap& w0,
                                 const CUtensorMap& w1, const CUtensorMap& x, const WsGemm& p,
                                 int num_sms, cudaStream_t st, int* launches);
+
+// The same GEMMs on CTA pairs (cluster of 2, tcgen05 cta_group::2): M = 256
+// weight rows split over the pair, token tiles of up to 256 rows (tile_max 256).
+cudaError_t launch_gemm_ws_pair_bf16(int mode, int tile_max, const CUtensorMap& w0,
+                                     const CUtensorMap& w1, const CUtensorMap& x, const WsGemm& p,
+                                     int num_sms, cudaStream_t st, int* launches);
 
 // Weight-stationary block-scaled MXFP4 GEMMs over the token-tile list of align.
 // Codes through the TMA maps; scales through their own pointers (byte strides).

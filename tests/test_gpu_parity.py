@@ -259,3 +259,23 @@ def test_glm45_air_shape_skewed_strided_ids_sampled():
                 "wts": w_all.cpu()[:, 23, :]}
     ref = run_oracle(case_cpu, tokens=toks)
     assert rel_err(a.cpu()[toks], ref) <= BF16_TOL
+
+
+@pytest.mark.parametrize("T,H,I,E,k", [
+    (300, 512, 384, 4, 2),     # 150 slots per expert: several 32-row granules, partial tiles
+    (600, 512, 640, 3, 2),     # 400 slots per expert: >1 token tile of 256 rows, N tail of I
+    (77, 288, 96, 6, 3),       # ragged K and output columns
+])
+def test_token_tile_configs_agree_and_match_oracle(T, H, I, E, k, monkeypatch):
+    # the token-tile size (32 / 128 rows on one CTA, 256 rows on a CTA pair) is a
+    # performance choice: every configuration must give the same bits
+    case = make_case(T, H, I, E, k, seed=T + 5)
+    ref = run_oracle(case)
+    c = to_cuda(case)
+    outs = {}
+    for tile in ("32", "128", "256"):
+        monkeypatch.setenv("MOE_TILE", tile)
+        outs[tile] = run_gpu(c)
+        assert rel_err(outs[tile], ref) <= BF16_TOL, tile
+    assert torch.equal(outs["32"], outs["128"])
+    assert torch.equal(outs["128"], outs["256"])
