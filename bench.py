@@ -51,12 +51,18 @@ WORKLOADS = {
 # DRAM traffic per launch of the dominant kernel from an ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed to the hash of the kernel
 # source it was taken on; reported as null once the source has changed.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # profiles/gemm_ws_pair_bf16_qwen3shape_E32_T1024.md: 983.0 MB read + 25.7 MB written on
+    # the E=32, T=1024 case (~256 slots per expert), scaled x4 (experts and tokens) to the
+    # E=128, T=4096 launch of the pair kernel
+    "gemm1_swiglu": {"bytes_per_launch": 4.0 * (982.952448e6 + 25.723648e6), "src": "0aac259f23670b9d",
+                     "workload": "qwen3-235b T=4096"},
+}
 
 
 def kernel_src_hash() -> str:
     h = hashlib.sha256()
-    for fn in ("moe_gemm_ws.cu", "moe_common.cuh"):
+    for fn in ("moe_gemm_ws2.cu", "moe_common.cuh"):
         with open(os.path.join(ROOT, "mixture_experts_layer_46_b200", "csrc", fn), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -420,8 +426,8 @@ def main():
     same_case = (args.workload == "qwen3-235b" and w["T"] == 4096 and w["E"] == 128)
     roof["traffic"] = (tr["bytes_per_launch"] if tr and same_case and tr.get("src") == kernel_src_hash()
                        else None)
-    roof["kernel"] = ("gemm1_swiglu (grouped gate/up GEMM + SwiGLU, tcgen05 "
-                      + ("kind::mxf4 block-scaled)" if mx else "kind::f16)"))
+    roof["kernel"] = ("gemm1_swiglu (weight-stationary grouped gate/up GEMM + SwiGLU, tcgen05 "
+                      + ("kind::mxf4 block-scaled)" if mx else "kind::f16, CTA pairs at this size)"))
     roof["peak_source"] = (f"{src} (MEASURED_PEAKS.json burst)" if src == "measured" else "fallback")
     if mx and roof["bound"] == "tensor":
         roof["peak_source"] += " x4 nominal FP4/bf16 ratio (FP4 peak not measured)"
