@@ -426,8 +426,10 @@ def main():
     same_case = (args.workload == "qwen3-235b" and w["T"] == 4096 and w["E"] == 128)
     roof["traffic"] = (tr["bytes_per_launch"] if tr and same_case and tr.get("src") == kernel_src_hash()
                        else None)
+    pair = (not mx) and (w["T"] * w["k"] >= 32 * w["E"])
     roof["kernel"] = ("gemm1_swiglu (weight-stationary grouped gate/up GEMM + SwiGLU, tcgen05 "
-                      + ("kind::mxf4 block-scaled)" if mx else "kind::f16, CTA pairs at this size)"))
+                      + ("kind::mxf4 block-scaled)" if mx else
+                         ("kind::f16 on CTA pairs)" if pair else "kind::f16)")))
     roof["peak_source"] = (f"{src} (MEASURED_PEAKS.json burst)" if src == "measured" else "fallback")
     if mx and roof["bound"] == "tensor":
         roof["peak_source"] += " x4 nominal FP4/bf16 ratio (FP4 peak not measured)"
