@@ -13,73 +13,102 @@
 // counted.  The order inside an expert is stable so results are reproducible.
 //
 // Small problems run in one CTA; larger ones in three kernels: per-chunk
-// histograms, one scan CTA, per-chunk stable scatter.
+// histograms and in-chunk ranks, one scan CTA, an element-wise scatter.  Ranks
+// come from warps walking contiguous runs of slots, 32 at a time, with a
+// ballot-built mask of the lanes sharing an expert, so a CTA needs only two
+// block-wide barriers.
 #include "../../include/moe.h"
 #include "moe_internal.h"
 
 namespace moe {
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
+constexpr int kSmallGroups = kAlignSmallMax / kThreads;  // 32-slot groups per warp, one CTA
+constexpr int kChunkGroups = kAlignChunk / kThreads;     // 32-slot groups per warp, per chunk
+static_assert(kAlignSmallMax % kThreads == 0 && kAlignChunk % kThreads == 0, "align tiling");
 
 __device__ __forceinline__ int64_t read_id(const View2& v, int64_t s, int64_t k) {
-  const int64_t t = s / k, j = s - t * k;
+  // slot counts are far below 2^31 (validated), so 32-bit division suffices
+  const int64_t t = static_cast<int32_t>(s) / static_cast<int32_t>(k), j = s - t * k;
   const int64_t off = t * v.s0 + j * v.s1;
   if (v.dtype == MOE_I64) return static_cast<const int64_t*>(v.data)[off];
   return static_cast<int64_t>(static_cast<const int32_t*>(v.data)[off]);
 }
 
-// Histogram of the slots [s0, s1) into hist (shared, zeroed by the caller).
-// Returns this thread's count of invalid ids.
-__device__ int block_hist(const View2& ids, int64_t k, int64_t E, int64_t s0, int64_t s1,
-                          int* hist) {
+// Lanes of the warp holding the same value v in [0, 2^nbits): one ballot per
+// bit, each lane keeping the lanes that agree with it on that bit.  The same
+// mask match.any returns, at a fraction of its cost for nbits <= 11.
+__device__ __forceinline__ unsigned same_value_lanes(unsigned v, int nbits) {
+  unsigned peers = 0xffffffffu;
+  for (int b = 0; b < nbits; ++b) {
+    const unsigned bit = (v >> b) & 1u;
+    const unsigned bal = __ballot_sync(0xffffffffu, bit);
+    peers &= bit ? bal : ~bal;
+  }
+  return peers;
+}
+
+// Stable ranks of the slots [s_begin, s_end) inside one CTA.  Warp w owns the
+// contiguous run of per_warp slots starting at s_begin + w * per_warp (per_warp
+// a multiple of 32, at most kG * 32) and walks it in 32-slot groups: lanes of a
+// group that share an expert find each other (same_value_lanes), and the warp's
+// running count of that expert (wcnt[w * E + e], zero on entry) gives the
+// group's base.  On return e_reg[g] is the expert of the lane's slot in group g
+// (-1: invalid or past the end), r_reg[g] its rank among the warp's slots of
+// that expert, and wcnt holds the per-warp totals.  Returns the lane's count of
+// ids outside [0, E).
+template <int kG>
+__device__ int warp_rank_slots(const View2& ids, int64_t k, int64_t E, int64_t s_begin,
+                               int64_t s_end, int per_warp, int* wcnt, int (&e_reg)[kG],
+                               int (&r_reg)[kG]) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  const int64_t base = s_begin + static_cast<int64_t>(warp) * per_warp;
   int bad = 0;
-  for (int64_t s = s0 + threadIdx.x; s < s1; s += blockDim.x) {
-    const int64_t e = read_id(ids, s, k);
-    if (e >= 0 && e < E)
-      atomicAdd(&hist[e], 1);
-    else
-      ++bad;
+#pragma unroll
+  for (int g = 0; g < kG; ++g) {  // all loads first: one memory round trip
+    const int64_t s = base + g * 32 + lane;
+    int e = -1;
+    if (g * 32 < per_warp && s < s_end) {
+      const int64_t v = read_id(ids, s, k);
+      if (v >= 0 && v < E)
+        e = static_cast<int>(v);
+      else
+        ++bad;
+    }
+    e_reg[g] = e;
+  }
+  int* mine = wcnt + warp * E;
+  const int nbits = 32 - __clz(static_cast<int>(E));  // e + 1 lies in [0, E]
+#pragma unroll
+  for (int g = 0; g < kG; ++g) {
+    r_reg[g] = 0;
+    if (g * 32 < per_warp) {  // uniform over the warp
+      const int e = e_reg[g];
+      const unsigned peers = same_value_lanes(static_cast<unsigned>(e + 1), nbits);
+      const int c = e >= 0 ? mine[e] : 0;
+      __syncwarp();
+      if (e >= 0 && lane == __ffs(peers) - 1) mine[e] = c + __popc(peers);
+      __syncwarp();
+      r_reg[g] = c + __popc(peers & lt_mask);
+    }
   }
   return bad;
 }
 
-// Stable scatter of slots [s0, s1): slot s of expert e goes to
-// sorted[base[e] + (number of earlier slots of e in [s0, s))].  base[] lives in
-// shared memory and is advanced as slots are placed; warp_cnt is a
-// [kWarps][E] shared array that must be all zero on entry (and is left zero).
-__device__ void block_scatter(const View2& ids, int64_t k, int64_t E, int64_t s0, int64_t s1,
-                              int* base, int* warp_cnt, int32_t* sorted, int32_t* inv) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const unsigned lt_mask = (1u << lane) - 1u;
-  for (int64_t c0 = s0; c0 < s1; c0 += blockDim.x) {
-    const int64_t s = c0 + threadIdx.x;
-    int e = -1;
-    if (s < s1) {
-      const int64_t v = read_id(ids, s, k);
-      if (v >= 0 && v < E) e = static_cast<int>(v);
+// Per expert: exclusive prefix of the per-warp counts over warps (in place) and
+// the CTA total in hist[e].
+__device__ void warp_prefix(int64_t E, int* wcnt, int* hist) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+    for (int w = 0; w < kWarps; ++w) {
+      const int v = wcnt[w * E + e];
+      wcnt[w * E + e] = run;
+      run += v;
     }
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    const int leader = __ffs(peers) - 1;
-    const int rank = __popc(peers & lt_mask);
-    if (e >= 0 && lane == leader) warp_cnt[warp * E + e] = __popc(peers);
-    __syncthreads();
-    if (e >= 0) {
-      int before = 0;
-      for (int w = 0; w < warp; ++w) before += warp_cnt[w * E + e];
-      const int pos = base[e] + before + rank;
-      sorted[pos] = static_cast<int32_t>(s);
-      inv[s] = pos;
-    } else if (s < s1) {
-      inv[s] = -1;
-    }
-    __syncthreads();
-    if (e >= 0 && lane == leader) {
-      atomicAdd(&base[e], __popc(peers));
-      warp_cnt[warp * E + e] = 0;
-    }
-    __syncthreads();
+    hist[e] = run;
   }
 }
 
@@ -193,52 +222,84 @@ __global__ void __launch_bounds__(kThreads) align_small_kernel(
     int32_t* sorted, int32_t* inv, int32_t* block_expert, int32_t* num_blocks, TileOut to,
     DeviceErrors* err) {
   extern __shared__ int sm[];
-  int* hist = sm;                       // [E]
-  int* offs = hist + E;                 // [E + 1]
-  int* base = offs + E + 1;             // [E]
-  int* warp_cnt = base + E;             // [kWarps * E]
-  int* tsc = warp_cnt + kWarps * E;     // [E + 1]
+  int* wcnt = sm;                    // [kWarps * E]
+  int* hist = wcnt + kWarps * E;     // [E]
+  int* offs = hist + E;              // [E + 1]
+  int* tsc = offs + E + 1;           // [E + 1]
   __shared__ int bad_sh;
   pdl_wait();
   const int64_t S = T * k;
-  for (int i = threadIdx.x; i < E * (kWarps + 1); i += blockDim.x) {
-    if (i < E) hist[i] = 0;
-    else warp_cnt[i - E] = 0;
-  }
+  for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) wcnt[i] = 0;
   if (threadIdx.x == 0) bad_sh = 0;
   __syncthreads();
-  const int bad = block_hist(ids, k, E, 0, S, hist);
+  const int per_warp = static_cast<int>((S + kThreads - 1) / kThreads) * 32;
+  int e_reg[kSmallGroups], r_reg[kSmallGroups];
+  const int bad = warp_rank_slots<kSmallGroups>(ids, k, E, 0, S, per_warp, wcnt, e_reg, r_reg);
   if (bad) atomicAdd(&bad_sh, bad);
+  __syncthreads();
+  warp_prefix(E, wcnt, hist);
   __syncthreads();
   block_finalize(hist, E, bm, static_cast<int32_t>(S), offs, tsc, counts, offsets, sorted,
                  block_expert, num_blocks, to);
-  for (int e = threadIdx.x; e < E; e += blockDim.x) base[e] = offs[e];
-  __syncthreads();
-  block_scatter(ids, k, E, 0, S, base, warp_cnt, sorted, inv);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t base = static_cast<int64_t>(warp) * per_warp;
+#pragma unroll
+  for (int g = 0; g < kSmallGroups; ++g) {
+    const int64_t s = base + g * 32 + lane;
+    if (g * 32 >= per_warp || s >= S) continue;
+    const int e = e_reg[g];
+    if (e >= 0) {
+      const int pos = offs[e] + wcnt[warp * E + e] + r_reg[g];
+      sorted[pos] = static_cast<int32_t>(s);
+      inv[s] = pos;
+    } else {
+      inv[s] = -1;
+    }
+  }
   if (threadIdx.x == 0 && bad_sh && err) atomicAdd(&err->bad_ids, static_cast<unsigned>(bad_sh));
   pdl_launch_dependents();
 }
 
+// Multi-CTA path, kernel 1: per chunk of kAlignChunk slots, the per-expert
+// histogram (chunk_counts[c * E + e]) and each slot's stable rank inside its
+// chunk and expert, parked in inv[s] (-1 for a skipped slot).
 __global__ void __launch_bounds__(kThreads) align_count_kernel(View2 ids, int64_t T, int64_t k,
                                                                int64_t E, int32_t* chunk_counts,
-                                                               DeviceErrors* err) {
-  extern __shared__ int hist[];
+                                                               int32_t* inv, DeviceErrors* err) {
+  extern __shared__ int sm[];
+  int* wcnt = sm;                 // [kWarps * E]
+  int* hist = wcnt + kWarps * E;  // [E]
   __shared__ int bad_sh;
   pdl_wait();
+  pdl_launch_dependents();
   const int64_t S = T * k;
-  for (int i = threadIdx.x; i < E; i += blockDim.x) hist[i] = 0;
+  for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) wcnt[i] = 0;
   if (threadIdx.x == 0) bad_sh = 0;
   __syncthreads();
   const int64_t s0 = static_cast<int64_t>(blockIdx.x) * kAlignChunk;
   const int64_t s1 = min(S, s0 + kAlignChunk);
-  const int bad = block_hist(ids, k, E, s0, s1, hist);
+  constexpr int per_warp = kChunkGroups * 32;
+  int e_reg[kChunkGroups], r_reg[kChunkGroups];
+  const int bad = warp_rank_slots<kChunkGroups>(ids, k, E, s0, s1, per_warp, wcnt, e_reg, r_reg);
   if (bad) atomicAdd(&bad_sh, bad);
   __syncthreads();
+  warp_prefix(E, wcnt, hist);
+  __syncthreads();
   for (int i = threadIdx.x; i < E; i += blockDim.x) chunk_counts[blockIdx.x * E + i] = hist[i];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t base = s0 + static_cast<int64_t>(warp) * per_warp;
+#pragma unroll
+  for (int g = 0; g < kChunkGroups; ++g) {
+    const int64_t s = base + g * 32 + lane;
+    if (s >= s1) continue;
+    const int e = e_reg[g];
+    inv[s] = e >= 0 ? wcnt[warp * E + e] + r_reg[g] : -1;
+  }
   if (threadIdx.x == 0 && bad_sh && err) atomicAdd(&err->bad_ids, static_cast<unsigned>(bad_sh));
-  pdl_launch_dependents();
 }
 
+// Kernel 2 (one CTA): per expert, exclusive prefix of the chunk histograms
+// over chunks (in place), then the counts, offsets, padding and tile list.
 __global__ void __launch_bounds__(1024) align_scan_kernel(int64_t T, int64_t k, int64_t E,
                                                           int32_t bm, int64_t n_chunks,
                                                           int32_t* chunk_counts, int32_t* counts,
@@ -250,40 +311,47 @@ __global__ void __launch_bounds__(1024) align_scan_kernel(int64_t T, int64_t k, 
   int* offs = cnt + E;        // [E + 1]
   int* tsc = offs + E + 1;    // [E + 1]
   pdl_wait();
-  // per expert: exclusive prefix over chunks (in place), total count
+  pdl_launch_dependents();
+  constexpr int kBatch = 8;  // independent loads in flight per thread
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int run = 0;
-    for (int64_t c = 0; c < n_chunks; ++c) {
-      const int v = chunk_counts[c * E + e];
-      chunk_counts[c * E + e] = run;
-      run += v;
+    for (int64_t c0 = 0; c0 < n_chunks; c0 += kBatch) {
+      int v[kBatch];
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i)
+        v[i] = c0 + i < n_chunks ? chunk_counts[(c0 + i) * E + e] : 0;
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        if (c0 + i < n_chunks) chunk_counts[(c0 + i) * E + e] = run;
+        run += v[i];
+      }
     }
     cnt[e] = run;
   }
   __syncthreads();
   block_finalize(cnt, E, bm, static_cast<int32_t>(T * k), offs, tsc, counts, offsets, sorted,
                  block_expert, num_blocks, to);
-  pdl_launch_dependents();
 }
 
-__global__ void __launch_bounds__(kThreads) align_scatter_kernel(View2 ids, int64_t T, int64_t k,
-                                                                 int64_t E,
-                                                                 const int32_t* chunk_counts,
-                                                                 const int32_t* offsets,
-                                                                 int32_t* sorted, int32_t* inv) {
-  extern __shared__ int sm[];
-  int* base = sm;            // [E]
-  int* warp_cnt = base + E;  // [kWarps * E]
+// Kernel 3: every slot independently: position = offset of its expert + the
+// expert's slots in earlier chunks + its rank inside the chunk.
+__global__ void __launch_bounds__(256) align_scatter_kernel(View2 ids, int64_t T, int64_t k,
+                                                            int64_t E,
+                                                            const int32_t* chunk_counts,
+                                                            const int32_t* offsets,
+                                                            int32_t* sorted, int32_t* inv) {
   pdl_wait();
-  const int64_t S = T * k;
-  for (int i = threadIdx.x; i < E; i += blockDim.x)
-    base[i] = offsets[i] + chunk_counts[blockIdx.x * E + i];
-  for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) warp_cnt[i] = 0;
-  __syncthreads();
-  const int64_t s0 = static_cast<int64_t>(blockIdx.x) * kAlignChunk;
-  const int64_t s1 = min(S, s0 + kAlignChunk);
-  block_scatter(ids, k, E, s0, s1, base, warp_cnt, sorted, inv);
   pdl_launch_dependents();
+  const int64_t S = T * k;
+  for (int64_t s = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; s < S;
+       s += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int32_t r = inv[s];
+    if (r < 0) continue;
+    const int e = static_cast<int>(read_id(ids, s, k));
+    const int pos = offsets[e] + chunk_counts[(s / kAlignChunk) * E + e] + r;
+    sorted[pos] = static_cast<int32_t>(s);
+    inv[s] = pos;
+  }
 }
 
 }  // namespace
@@ -303,7 +371,7 @@ cudaError_t launch_align(const View2& ids, int64_t T, int64_t k, int64_t E, int3
   const int64_t S = T * k;
   cudaError_t rc;
   if (S <= kAlignSmallMax) {
-    const size_t smem = sizeof(int) * (E * (kWarps + 4) + 2);
+    const size_t smem = sizeof(int) * (E * (kWarps + 3) + 2);
     if (smem > 48 * 1024) {
       rc = cudaFuncSetAttribute(align_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)smem);
@@ -314,22 +382,23 @@ cudaError_t launch_align(const View2& ids, int64_t T, int64_t k, int64_t E, int3
     if (launches) *launches += 1;
     return rc;
   }
-  const size_t smem_count = sizeof(int) * E;
+  const size_t smem_count = sizeof(int) * E * (kWarps + 1);
+  if (smem_count > 48 * 1024) {
+    rc = cudaFuncSetAttribute(align_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)smem_count);
+    if (rc != cudaSuccess) return rc;
+  }
   rc = launch_pdl(align_count_kernel, dim3((unsigned)n_chunks), dim3(kThreads), smem_count, st,
-                  ids, T, k, E, chunk_counts, err);
+                  ids, T, k, E, chunk_counts, inv, err);
   if (rc != cudaSuccess) return rc;
   const size_t smem_scan = sizeof(int) * (3 * E + 2);
   rc = launch_pdl(align_scan_kernel, dim3(1), dim3(1024), smem_scan, st, T, k, E, bm, n_chunks,
                   chunk_counts, counts, offsets, sorted, block_expert, num_blocks, to);
   if (rc != cudaSuccess) return rc;
-  const size_t smem_sc = sizeof(int) * E * (kWarps + 1);
-  if (smem_sc > 48 * 1024) {
-    rc = cudaFuncSetAttribute(align_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)smem_sc);
-    if (rc != cudaSuccess) return rc;
-  }
-  rc = launch_pdl(align_scatter_kernel, dim3((unsigned)n_chunks), dim3(kThreads), smem_sc, st, ids,
-                  T, k, E, chunk_counts, offsets, sorted, inv);
+  int64_t sc_blocks = (S + 255) / 256;
+  if (sc_blocks > 148 * 8) sc_blocks = 148 * 8;
+  rc = launch_pdl(align_scatter_kernel, dim3((unsigned)sc_blocks), dim3(256), 0, st, ids, T, k, E,
+                  chunk_counts, offsets, sorted, inv);
   if (launches) *launches += 3;
   return rc;
 }

@@ -37,7 +37,7 @@ struct WsLayout {
 constexpr int kMaxTopK = 32;            // routing columns per token
 constexpr int kMaxExperts = 1024;       // experts per layer
 constexpr int kAlignChunk = 4096;        // slots per CTA in the multi-CTA align
-constexpr int kAlignSmallMax = 8192;     // single-CTA align up to this many slots
+constexpr int kAlignSmallMax = 16384;    // single-CTA align up to this many slots
 
 // Padding granule and token-tile size for a problem (depend only on T, k, E, dtype).
 void choose_tiling(int64_t T, int64_t k, int64_t E, bool mxfp4, int32_t* bm, int32_t* tile_max);

@@ -19,31 +19,47 @@ namespace {
 __device__ __forceinline__ float bf16_to_f(uint16_t b) { return __uint_as_float(uint32_t(b) << 16); }
 
 __global__ void __launch_bounds__(256) permute_bf16_kernel(View2 x, int64_t T, int64_t H, int64_t k,
-                                                           int64_t E, const int32_t* inv,
+                                                           int64_t E, const int32_t* __restrict__ inv,
                                                            const int32_t* offsets,
                                                            const int32_t* counts,
-                                                           __nv_bfloat16* a1, int vec_ok,
+                                                           __nv_bfloat16* __restrict__ a1, int vec_ok,
                                                            int tok_blocks) {
   pdl_wait();
   pdl_launch_dependents();
   const int64_t H8 = H / 8;
   if (blockIdx.x < tok_blocks) {
     for (int64_t t = blockIdx.x; t < T; t += tok_blocks) {
-      int32_t pos[kMaxTopK];
-      for (int j = 0; j < k; ++j) pos[j] = inv[t * k + j];
+      const int32_t* pos = inv + t * k;
       if (vec_ok) {
-        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x.data) + t * x.s0);
-        for (int64_t c = threadIdx.x; c < H8; c += blockDim.x) {
-          const uint4 v = src[c];
-          for (int j = 0; j < k; ++j)
-            if (pos[j] >= 0) reinterpret_cast<uint4*>(a1 + static_cast<int64_t>(pos[j]) * H)[c] = v;
+        // up to four 16-byte chunks of the row loaded before any store
+        const uint4* __restrict__ src =
+            reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x.data) + t * x.s0);
+        for (int64_t c0 = threadIdx.x; c0 < H8; c0 += 4 * blockDim.x) {
+          uint4 v[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int64_t c = c0 + i * blockDim.x;
+            if (c < H8) v[i] = __ldg(src + c);
+          }
+          for (int j = 0; j < k; ++j) {
+            const int32_t p = __ldg(pos + j);
+            if (p < 0) continue;
+            uint4* dst = reinterpret_cast<uint4*>(a1 + static_cast<int64_t>(p) * H);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int64_t c = c0 + i * blockDim.x;
+              if (c < H8) dst[c] = v[i];
+            }
+          }
         }
       } else {
         const uint16_t* src = static_cast<const uint16_t*>(x.data) + t * x.s0;
         for (int64_t h = threadIdx.x; h < H; h += blockDim.x) {
           const uint16_t v = src[h * x.s1];
-          for (int j = 0; j < k; ++j)
-            if (pos[j] >= 0) reinterpret_cast<uint16_t*>(a1 + static_cast<int64_t>(pos[j]) * H)[h] = v;
+          for (int j = 0; j < k; ++j) {
+            const int32_t p = __ldg(pos + j);
+            if (p >= 0) reinterpret_cast<uint16_t*>(a1 + static_cast<int64_t>(p) * H)[h] = v;
+          }
         }
       }
     }
