@@ -504,7 +504,7 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   if (pr.mxfp4) return forward_mxfp4(x, w13, w2, ids, wts, out, pr, L, w, dev, st);
 
   // ---- tensor maps (bf16, 128-byte swizzle): weights in [64 x 128] boxes,
-  // gathered token rows in [64 x 32] boxes
+  // expert-grouped token rows in one box per CTA and token tile
   CUtensorMap mA1, mGate, mUp, mH, mW2;
   // 128-row token tiles run on CTA pairs once experts average >= 32 slots (the
   // pair moves a sixth fewer shared-memory bytes per FLOP and keeps 5 stages in
@@ -515,7 +515,12 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   if (L.tile_max == 256) pair = true;  // 256-row tiles exist only on CTA pairs
   const int32_t wpolicy = getenv("MOE_WPOLICY") ? atoi(getenv("MOE_WPOLICY")) : 0;
   const uint32_t boxw[3] = {64, 128, 1};
-  const uint32_t boxt[2] = {64, pair ? 16u : 32u};
+  // one TMA box covers a CTA's share of a token tile (fewer copy operations per
+  // stage); MOE_TOKBOX=0 selects 16-row (pair) / 32-row boxes (tuning)
+  uint32_t tok_box = pair ? static_cast<uint32_t>(L.tile_max / 2) : static_cast<uint32_t>(L.tile_max);
+  if (const char* env = getenv("MOE_TOKBOX"))
+    if (atoi(env) == 0) tok_box = pair ? 16u : 32u;
+  const uint32_t boxt[2] = {64, tok_box};
   {
     const uint64_t d[2] = {uint64_t(pr.H), uint64_t(L.p_max)};
     const uint64_t sb[1] = {uint64_t(pr.H) * 2};
@@ -586,6 +591,7 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   g1.k = pr.k;
   g1.err = dev->errors;
   g1.weights_evict_first = wpolicy;
+  g1.tok_box = static_cast<int32_t>(tok_box);
   rc = pair ? launch_gemm_ws_pair_bf16(0, L.tile_max, mGate, mUp, mA1, g1, dev->num_sms, st, &launches)
             : launch_gemm_ws_bf16(0, L.tile_max, mGate, mUp, mA1, g1, dev->num_sms, st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm1");

@@ -32,7 +32,6 @@ namespace {
 
 constexpr int kWRows = 128;                  // rows per weight tile (MMA M)
 constexpr int kBK = 64;                      // bf16 elements per 128-byte row
-constexpr int kTokBox = 32;                  // token rows per TMA box
 constexpr int kUmmaK = 16;
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 192;
@@ -68,6 +67,7 @@ struct WsArgs {
   View2 topk_w;
   int64_t k;
   int32_t weights_evict_first;
+  int32_t tok_box;  // token rows per TMA box (the map's box height)
   DeviceErrors* err;
 };
 
@@ -152,8 +152,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int32_t e = g.tile_expert[t], row0 = g.tile_row[t], rows = g.tile_rows[t];
         const int32_t w0 = static_cast<int32_t>(kMode == 0 ? wt * kWRows : wt * 2 * kWRows);
         const int32_t w1 = kMode == 0 ? w0 : w0 + kWRows;
-        const int nbox = rows / kTokBox;
-        const uint32_t bytes = 2 * C::kWBytes + nbox * kTokBox * kBK * 2;
+        // whole boxes: a box may run past the tile (rows the MMA's N excludes)
+        const int nbox = (rows + g.tok_box - 1) / g.tok_box;
+        const uint32_t bytes = 2 * C::kWBytes + nbox * g.tok_box * kBK * 2;
         for (int kb = 0; kb < num_k; ++kb) {
           if (!mbar_wait(&sm.empty[stage], phase ^ 1u, g.err)) { ok = false; break; }
           uint8_t* sw0 = sm.stages + stage * C::kStageBytes;
@@ -163,8 +164,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d(sw0, &tmW0, &sm.full[stage], kb * kBK, w0, e, wpol);
           tma_load_3d(sw1, kMode == 0 ? &tmW1 : &tmW0, &sm.full[stage], kb * kBK, w1, e, wpol);
           for (int b = 0; b < nbox; ++b)
-            tma_load_2d(sx + b * kTokBox * kBK * 2, &tmX, &sm.full[stage], kb * kBK,
-                        row0 + b * kTokBox, pol);
+            tma_load_2d(sx + b * g.tok_box * kBK * 2, &tmX, &sm.full[stage], kb * kBK,
+                        row0 + b * g.tok_box, pol);
           last_phase[stage] = static_cast<int8_t>(phase);
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
@@ -356,6 +357,7 @@ cudaError_t launch_gemm_ws_bf16(int mode, int tile_max, const CUtensorMap& w0,
   g.k = p.k;
   g.err = p.err;
   g.weights_evict_first = p.weights_evict_first;
+  g.tok_box = p.tok_box;
   if (launches) *launches += 1;
   const int64_t max_items = p.max_tiles * p.n_wt;
   if (tile_max == 128) {

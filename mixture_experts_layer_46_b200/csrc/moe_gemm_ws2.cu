@@ -32,7 +32,6 @@ namespace {
 
 constexpr int kWRows = 128;                  // weight rows per CTA per weight tile
 constexpr int kBK = 64;
-constexpr int kTokBox = 16;                  // token rows per TMA box
 constexpr int kUmmaK = 16;
 constexpr int kEpiWarps = 8;                 // two per TMEM lane quadrant
 constexpr int kThreads = 32 * (2 + kEpiWarps);
@@ -67,6 +66,7 @@ struct Args {
   View2 topk_w;
   int64_t k;
   int32_t weights_evict_first;
+  int32_t tok_box;  // token rows per TMA box (the map's box height)
   DeviceErrors* err;
 };
 
@@ -206,8 +206,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int32_t w1 = kMode == 0 ? w0 : w0 + 2 * kWRows;
         const int32_t half = rows / 2;
         const int32_t my_row0 = row0 + static_cast<int32_t>(rank) * half;
-        const int nbox = half / kTokBox;
-        const uint32_t bytes_pair = 2 * (2 * kWBytes + half * kBK * 2);
+        // whole boxes: a box may run past this CTA's half (rows the MMA's N excludes)
+        const int nbox = (half + g.tok_box - 1) / g.tok_box;
+        const uint32_t bytes_pair = 2 * (2 * kWBytes + nbox * g.tok_box * kBK * 2);
         for (int kb = 0; kb < num_k; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, g.err)) { ok = false; break; }
           uint8_t* sw0 = stages + stage * kStageBytes;
@@ -218,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d_pair(sw0, &tmW0, fb, kb * kBK, w0, e, wpol);
           tma_load_3d_pair(sw1, kMode == 0 ? &tmW1 : &tmW0, fb, kb * kBK, w1, e, wpol);
           for (int b = 0; b < nbox; ++b)
-            tma_load_2d_pair(sx + b * kTokBox * kBK * 2, &tmX, fb, kb * kBK, my_row0 + b * kTokBox, pol);
+            tma_load_2d_pair(sx + b * g.tok_box * kBK * 2, &tmX, fb, kb * kBK, my_row0 + b * g.tok_box, pol);
           last_phase[stage] = static_cast<int8_t>(phase);
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
@@ -419,6 +420,7 @@ cudaError_t launch_gemm_ws_pair_bf16(int mode, int tile_max, const CUtensorMap& 
   g.k = p.k;
   g.err = p.err;
   g.weights_evict_first = p.weights_evict_first;
+  g.tok_box = p.tok_box;
   if (launches) *launches += 1;
   const int64_t max_items = p.max_tiles * p.n_wt;
   if (tile_max == 256) {

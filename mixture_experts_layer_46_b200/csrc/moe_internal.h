@@ -37,7 +37,7 @@ struct WsLayout {
 constexpr int kMaxTopK = 32;            // routing columns per token
 constexpr int kMaxExperts = 1024;       // experts per layer
 constexpr int kAlignChunk = 4096;        // slots per CTA in the multi-CTA align
-constexpr int kAlignSmallMax = 16384;    // single-CTA align up to this many slots
+constexpr int kAlignSmallMax = 4096;     // single-CTA align up to this many slots
 
 // Padding granule and token-tile size for a problem (depend only on T, k, E, dtype).
 void choose_tiling(int64_t T, int64_t k, int64_t E, bool mxfp4, int32_t* bm, int32_t* tile_max);
@@ -110,6 +110,7 @@ struct WsGemm {
   View2 topk_w;
   int64_t k;
   int32_t weights_evict_first;  // L2 policy of the weight loads (tokens: evict-last)
+  int32_t tok_box;              // rows per token-tile TMA box of the x map (tile rows per CTA: one box)
   DeviceErrors* err;
 };
 // mode 0: GEMM1 (gate/up + SwiGLU -> h), mode 1: GEMM2 (down + routing weight -> y)
@@ -153,10 +154,11 @@ cudaError_t launch_gemm_ws_mxfp4(int mode, int tile_max, const CUtensorMap& w0,
                                  const CUtensorMap& w1, const CUtensorMap& x, const WsGemmMx& p,
                                  int num_sms, cudaStream_t st, int* launches);
 
-// standalone MXFP4 quantiser for rows of a [R, K] bf16/f32 matrix (unit inner stride)
+// MXFP4 quantiser for rows of a [R, K] bf16/f32 matrix (unit inner stride)
 cudaError_t launch_quantize_rows(const void* src, int32_t src_dtype, int64_t R, int64_t K,
                                  int64_t src_ld, uint8_t* codes, int64_t codes_ld,
-                                 uint8_t* scales, int64_t scales_ld, cudaStream_t st);
+                                 uint8_t* scales, int64_t scales_ld, cudaStream_t st,
+                                 int* launches = nullptr);
 
 // launch helper: PDL attribute on every kernel of the forward
 template <typename Kern, typename... Args>

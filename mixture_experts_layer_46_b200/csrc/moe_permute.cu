@@ -129,11 +129,15 @@ __global__ void __launch_bounds__(128) permute_quant_kernel(View2 x, int64_t T, 
   }
 }
 
-// Standalone quantiser: one thread per 32-element block.
+// Row quantiser: one thread per 32-element block (weights, offline); 16-byte
+// accesses when the rows allow them.
 __global__ void __launch_bounds__(256) quantize_rows_kernel(const void* src, int32_t src_dtype,
                                                             int64_t R, int64_t K, int64_t src_ld,
                                                             uint8_t* codes, int64_t codes_ld,
-                                                            uint8_t* scales, int64_t scales_ld) {
+                                                            uint8_t* scales, int64_t scales_ld,
+                                                            int vec_ok) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int64_t nb = K / 32;
   const int64_t total = R * nb;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
@@ -142,8 +146,21 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const void* src, int
     float v[32];
     if (src_dtype == MOE_BF16) {
       const uint16_t* p = static_cast<const uint16_t*>(src) + r * src_ld + b * 32;
+      if (vec_ok) {
 #pragma unroll
-      for (int q = 0; q < 32; ++q) v[q] = bf16_to_f(p[q]);
+        for (int q = 0; q < 4; ++q) {
+          const uint4 u = __ldg(reinterpret_cast<const uint4*>(p) + q);
+          const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            v[q * 8 + 2 * h] = bf16_to_f(static_cast<uint16_t>(w4[h] & 0xffffu));
+            v[q * 8 + 2 * h + 1] = bf16_to_f(static_cast<uint16_t>(w4[h] >> 16));
+          }
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 32; ++q) v[q] = bf16_to_f(p[q]);
+      }
     } else {
       const float* p = static_cast<const float*>(src) + r * src_ld + b * 32;
 #pragma unroll
@@ -152,12 +169,16 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const void* src, int
     uint32_t w[4];
     const uint32_t sc = mx_quant32(v, w);
     uint8_t* c = codes + r * codes_ld + b * 16;
+    if (vec_ok) {
+      *reinterpret_cast<uint4*>(c) = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      c[4 * q + 0] = w[q] & 0xffu;
-      c[4 * q + 1] = (w[q] >> 8) & 0xffu;
-      c[4 * q + 2] = (w[q] >> 16) & 0xffu;
-      c[4 * q + 3] = w[q] >> 24;
+      for (int q = 0; q < 4; ++q) {
+        c[4 * q + 0] = w[q] & 0xffu;
+        c[4 * q + 1] = (w[q] >> 8) & 0xffu;
+        c[4 * q + 2] = (w[q] >> 16) & 0xffu;
+        c[4 * q + 3] = w[q] >> 24;
+      }
     }
     scales[r * scales_ld + b] = static_cast<uint8_t>(sc);
   }
@@ -194,14 +215,19 @@ cudaError_t launch_permute_quant(const View2& x, int64_t T, int64_t H, int64_t k
 
 cudaError_t launch_quantize_rows(const void* src, int32_t src_dtype, int64_t R, int64_t K,
                                  int64_t src_ld, uint8_t* codes, int64_t codes_ld,
-                                 uint8_t* scales, int64_t scales_ld, cudaStream_t st) {
+                                 uint8_t* scales, int64_t scales_ld, cudaStream_t st,
+                                 int* launches) {
   const int64_t total = R * (K / 32);
   int64_t blocks = (total + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
   if (blocks < 1) blocks = 1;
-  quantize_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-      src, src_dtype, R, K, src_ld, codes, codes_ld, scales, scales_ld);
-  return cudaGetLastError();
+  // 16-byte source and code accesses when every block starts on a 16-byte boundary
+  const int vec_ok = src_dtype == MOE_BF16 && (src_ld * 2) % 16 == 0 &&
+                     reinterpret_cast<uintptr_t>(src) % 16 == 0 && codes_ld % 16 == 0 &&
+                     reinterpret_cast<uintptr_t>(codes) % 16 == 0;
+  if (launches) *launches += 1;
+  return launch_pdl(quantize_rows_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st,
+                    src, src_dtype, R, K, src_ld, codes, codes_ld, scales, scales_ld, vec_ok);
 }
 
 }  // namespace moe

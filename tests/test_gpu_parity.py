@@ -68,8 +68,9 @@ def run_oracle(case, tokens=None):
     (37, 16, 4, 16, torch.int64),      # int64 ids, small block
     (4096, 128, 8, 128, torch.int32),  # multi-CTA path (32768 slots)
     (3000, 513, 11, 64, torch.int32),  # shared-expert-fused routing width
-    (2000, 128, 8, 32, torch.int32),   # largest single-CTA size class (16000 slots)
-    (700, 1024, 8, 32, torch.int32),   # widest expert count, one CTA
+    (512, 128, 8, 32, torch.int32),    # largest single-CTA size class (4096 slots)
+    (2000, 128, 8, 32, torch.int32),   # multi-CTA, ragged last chunk (16000 slots)
+    (400, 1024, 8, 32, torch.int32),   # widest expert count, one CTA
     (5000, 1024, 8, 32, torch.int64),  # widest expert count, multi-CTA
 ])
 def test_align_bit_exact(T, E, k, bm, idt):
