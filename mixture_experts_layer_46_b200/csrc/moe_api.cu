@@ -413,8 +413,8 @@ moe_status_t forward_mxfp4(const moe_tensor_t* x, const moe_w13_t* w13, const mo
                                 st, &launches, &tiles);
   if (rc != cudaSuccess) return cuda_fail(rc, "align");
   prof_mark(st);
-  rc = launch_permute_quant(view2(x), pr.T, pr.H, pr.k, pr.E, inv, offsets, counts, w + L.a1,
-                            w + L.a1_scale, st, &launches);
+  rc = launch_permute_quant(view2(x), pr.T, pr.H, pr.k, inv, w + L.a1, w + L.a1_scale, st,
+                            &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "permute_quant");
   prof_mark(st);
   WsGemmMx g1;
@@ -569,7 +569,7 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
                     num_blocks, chunk_counts, L.n_chunks, dev->errors, st, &launches, &tiles);
   if (rc != cudaSuccess) return cuda_fail(rc, "align");
   prof_mark(st);
-  rc = launch_permute_bf16(view2(x), pr.T, pr.H, pr.k, pr.E, inv, offsets, counts,
+  rc = launch_permute_bf16(view2(x), pr.T, pr.H, pr.k, inv,
                            reinterpret_cast<__nv_bfloat16*>(w + L.a1), st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "permute");
   prof_mark(st);

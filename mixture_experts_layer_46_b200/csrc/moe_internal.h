@@ -63,15 +63,15 @@ cudaError_t launch_align(const View2& ids, int64_t T, int64_t k, int64_t E, int3
                          int64_t n_chunks, DeviceErrors* err, cudaStream_t st, int* launches,
                          const AlignTiles* tiles = nullptr);
 
-// permute: A1[inv[t*k+j], :] = x[t, :] (x read once per token), padding rows zeroed
-cudaError_t launch_permute_bf16(const View2& x, int64_t T, int64_t H, int64_t k, int64_t E,
-                                const int32_t* inv, const int32_t* offsets, const int32_t* counts,
-                                __nv_bfloat16* a1, cudaStream_t st, int* launches);
+// permute: A1[inv[t*k+j], :] = x[t, :] (x read once per token); padding rows untouched
+cudaError_t launch_permute_bf16(const View2& x, int64_t T, int64_t H, int64_t k,
+                                const int32_t* inv, __nv_bfloat16* a1, cudaStream_t st,
+                                int* launches);
 
 // permute + MXFP4 quantisation of x rows (codes [P, H/2], scales [P, H/32])
-cudaError_t launch_permute_quant(const View2& x, int64_t T, int64_t H, int64_t k, int64_t E,
-                                 const int32_t* inv, const int32_t* offsets, const int32_t* counts,
-                                 uint8_t* codes, uint8_t* scales, cudaStream_t st, int* launches);
+cudaError_t launch_permute_quant(const View2& x, int64_t T, int64_t H, int64_t k,
+                                 const int32_t* inv, uint8_t* codes, uint8_t* scales,
+                                 cudaStream_t st, int* launches);
 
 // combine: out[t, :] = sum_j y[inv[t*k + j], :] over valid slots (fixed j order)
 cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* inv, int64_t T, int64_t H,

@@ -1,7 +1,9 @@
 // Step "permute": gather the token rows of x into expert-grouped order so each
 // bm-row block of the grouped GEMM reads one expert's tokens contiguously.
 //   A1[inv[t*k + j], :] = x[t, :]     for every valid slot, x read once per token
-//   A1[p, :] = 0                      for the padding rows of every expert
+// Padding rows are left as they are: a token tile's padding rows only feed MMA
+// output columns (tokens) that no later step reads, and every output column
+// depends on its own B row alone, so their contents cannot reach a result.
 // x is read through its strides (LightLLM issue #1467 shows what dropping the
 // inner stride does); the fast path needs a unit inner stride and 16-byte rows.
 //
@@ -19,16 +21,13 @@ namespace {
 __device__ __forceinline__ float bf16_to_f(uint16_t b) { return __uint_as_float(uint32_t(b) << 16); }
 
 __global__ void __launch_bounds__(256) permute_bf16_kernel(View2 x, int64_t T, int64_t H, int64_t k,
-                                                           int64_t E, const int32_t* __restrict__ inv,
-                                                           const int32_t* offsets,
-                                                           const int32_t* counts,
-                                                           __nv_bfloat16* __restrict__ a1, int vec_ok,
-                                                           int tok_blocks) {
+                                                           const int32_t* __restrict__ inv,
+                                                           __nv_bfloat16* __restrict__ a1, int vec_ok) {
   pdl_wait();
   pdl_launch_dependents();
   const int64_t H8 = H / 8;
-  if (blockIdx.x < tok_blocks) {
-    for (int64_t t = blockIdx.x; t < T; t += tok_blocks) {
+  {
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
       const int32_t* pos = inv + t * k;
       if (vec_ok) {
         // up to four 16-byte chunks of the row loaded before any store
@@ -63,29 +62,18 @@ __global__ void __launch_bounds__(256) permute_bf16_kernel(View2 x, int64_t T, i
         }
       }
     }
-  } else {
-    // zero the padding rows of one expert
-    const int64_t e = blockIdx.x - tok_blocks;
-    if (e >= E) return;
-    const int64_t p0 = offsets[e] + counts[e], p1 = offsets[e + 1];
-    const uint4 z = make_uint4(0, 0, 0, 0);
-    for (int64_t p = p0; p < p1; ++p)
-      for (int64_t c = threadIdx.x; c < H8; c += blockDim.x) reinterpret_cast<uint4*>(a1 + p * H)[c] = z;
   }
 }
 
 // One thread per 32-element block of a row; a CTA walks tokens.
 __global__ void __launch_bounds__(128) permute_quant_kernel(View2 x, int64_t T, int64_t H, int64_t k,
-                                                            int64_t E, const int32_t* inv,
-                                                            const int32_t* offsets,
-                                                            const int32_t* counts, uint8_t* codes,
-                                                            uint8_t* scales, int vec_ok,
-                                                            int tok_blocks) {
+                                                            const int32_t* inv, uint8_t* codes,
+                                                            uint8_t* scales, int vec_ok) {
   pdl_wait();
   pdl_launch_dependents();
   const int64_t nb = H / 32;  // blocks per row
-  if (blockIdx.x < tok_blocks) {
-    for (int64_t t = blockIdx.x; t < T; t += tok_blocks) {
+  {
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
       int32_t pos[kMaxTopK];
       for (int j = 0; j < k; ++j) pos[j] = inv[t * k + j];
       for (int64_t b = threadIdx.x; b < nb; b += blockDim.x) {
@@ -117,15 +105,6 @@ __global__ void __launch_bounds__(128) permute_quant_kernel(View2 x, int64_t T, 
         }
       }
     }
-  } else {
-    const int64_t e = blockIdx.x - tok_blocks;
-    if (e >= E) return;
-    const int64_t p0 = offsets[e] + counts[e], p1 = offsets[e + 1];
-    for (int64_t p = p0; p < p1; ++p)
-      for (int64_t b = threadIdx.x; b < nb; b += blockDim.x) {
-        *reinterpret_cast<uint4*>(codes + p * (H / 2) + b * 16) = make_uint4(0, 0, 0, 0);
-        scales[p * nb + b] = 0;
-      }
   }
 }
 
@@ -191,26 +170,24 @@ static int token_blocks(int64_t T) {
   return static_cast<int>(b < 1 ? 1 : b);
 }
 
-cudaError_t launch_permute_bf16(const View2& x, int64_t T, int64_t H, int64_t k, int64_t E,
-                                const int32_t* inv, const int32_t* offsets, const int32_t* counts,
-                                __nv_bfloat16* a1, cudaStream_t st, int* launches) {
+cudaError_t launch_permute_bf16(const View2& x, int64_t T, int64_t H, int64_t k,
+                                const int32_t* inv, __nv_bfloat16* a1, cudaStream_t st,
+                                int* launches) {
   const int vec_ok = (x.s1 == 1) && ((x.s0 * 2) % 16 == 0) &&
                      (reinterpret_cast<uintptr_t>(x.data) % 16 == 0);
-  const int tb = token_blocks(T);
   if (launches) *launches += 1;
-  return launch_pdl(permute_bf16_kernel, dim3(static_cast<unsigned>(tb + E)), dim3(256), 0, st, x,
-                    T, H, k, E, inv, offsets, counts, a1, vec_ok, tb);
+  return launch_pdl(permute_bf16_kernel, dim3(static_cast<unsigned>(token_blocks(T))), dim3(256), 0,
+                    st, x, T, H, k, inv, a1, vec_ok);
 }
 
-cudaError_t launch_permute_quant(const View2& x, int64_t T, int64_t H, int64_t k, int64_t E,
-                                 const int32_t* inv, const int32_t* offsets, const int32_t* counts,
-                                 uint8_t* codes, uint8_t* scales, cudaStream_t st, int* launches) {
+cudaError_t launch_permute_quant(const View2& x, int64_t T, int64_t H, int64_t k,
+                                 const int32_t* inv, uint8_t* codes, uint8_t* scales,
+                                 cudaStream_t st, int* launches) {
   const int vec_ok = (x.s1 == 1) && ((x.s0 * 2) % 16 == 0) &&
                      (reinterpret_cast<uintptr_t>(x.data) % 16 == 0);
-  const int tb = token_blocks(T);
   if (launches) *launches += 1;
-  return launch_pdl(permute_quant_kernel, dim3(static_cast<unsigned>(tb + E)), dim3(128), 0, st, x,
-                    T, H, k, E, inv, offsets, counts, codes, scales, vec_ok, tb);
+  return launch_pdl(permute_quant_kernel, dim3(static_cast<unsigned>(token_blocks(T))), dim3(128), 0,
+                    st, x, T, H, k, inv, codes, scales, vec_ok);
 }
 
 cudaError_t launch_quantize_rows(const void* src, int32_t src_dtype, int64_t R, int64_t K,

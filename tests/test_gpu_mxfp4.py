@@ -139,6 +139,23 @@ def test_mxfp4_strided_equals_contiguous_and_deterministic():
     assert torch.equal(a, d)
 
 
+def test_mxfp4_stale_workspace_contents_never_reach_the_output():
+    # 0xFF scale bytes are NaN in e8m0: padding rows holding them must not matter
+    T, H, I, E, k = 45, 512, 256, 6, 3
+    case = make_mx_case(T, H, I, E, k, seed=23)
+    ref = mx_oracle(case)
+    c = cuda_case(case)
+    n = moe.workspace_bytes(T, H, I, E, k, mxfp4=True)
+    outs = []
+    for fill in (0x00, 0xFF):
+        ws = torch.full((n,), fill, dtype=torch.uint8, device="cuda")
+        v = moe.w13_from_packed(c["c13"], c["s13"])
+        outs.append(moe.forward(c["x"], v, c["c2"], c["ids"], c["wts"], w2_scale=c["s2"], workspace=ws))
+        torch.cuda.synchronize()
+    assert torch.equal(outs[0], outs[1])
+    assert rel_err(outs[0], ref) <= MX_TOL
+
+
 def test_mxfp4_shared_expert_fused_routing():
     # E = 32 routed + 1 shared, top_k = 4 + 1, the 513/11 convention at reduced size
     case = make_mx_case(96, 512, 256, 33, 5, seed=7, shared=True)

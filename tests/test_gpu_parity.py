@@ -217,6 +217,25 @@ def test_forward_host_matches_device():
     assert torch.equal(out_h, dev.cpu())
 
 
+@pytest.mark.parametrize("T,H,I,E,k", [
+    (37, 288, 96, 6, 3),       # one-CTA kernels, padded 32-row granules
+    (300, 512, 384, 4, 2),     # CTA pairs
+])
+def test_stale_workspace_contents_never_reach_the_output(T, H, I, E, k):
+    # padding rows of the expert-grouped buffers are never written; a workspace
+    # full of NaN bit patterns must give the same bits as a zeroed one
+    case = make_case(T, H, I, E, k, seed=T + 17)
+    ref = run_oracle(case)
+    c = to_cuda(case)
+    n = moe.workspace_bytes(T, H, I, E, k)
+    ws0 = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    wsn = torch.full((n,), 0xFF, dtype=torch.uint8, device="cuda")
+    a = run_gpu(c, ws=ws0)
+    b = run_gpu(c, ws=wsn)
+    assert torch.equal(a, b)
+    assert rel_err(a, ref) <= BF16_TOL
+
+
 def test_zero_tokens():
     case = to_cuda(make_case(0, 256, 128, 8, 2))
     out = run_gpu(case)
