@@ -156,15 +156,18 @@ __device__ int block_scan_experts(int64_t E, F v, int* out) {
   return total_sh;
 }
 
-// Outputs of align beyond sorted/offsets: the token-tile list consumed by the
-// weight-stationary GEMMs (tiles of at most tile_max rows, balanced within an
-// expert, never crossing one), written when tile_max > 0.
-struct TileOut {
+// Outputs of align beyond sorted/offsets: up to two token-tile lists consumed
+// by the weight-stationary GEMMs (tiles of at most tile_max rows, balanced
+// within an expert, never crossing one), each written when its tile_max > 0.
+struct TileList {
   int32_t tile_max;
   int32_t* tile_row;     // first padded row of the tile
   int32_t* tile_rows;    // rows in the tile (multiple of bm)
   int32_t* tile_expert;
   int32_t* num_tiles;
+};
+struct TileOut {
+  TileList list[2];
 };
 
 // From per-expert counts (shared), write counts, offsets, num_blocks,
@@ -192,8 +195,10 @@ __device__ void block_finalize(const int* cnt, int64_t E, int32_t bm, int32_t S,
   }
   for (int e = threadIdx.x; e < E; e += blockDim.x)
     for (int p = offs[e] + cnt[e]; p < offs[e + 1]; ++p) sorted[p] = S;
-  if (to.tile_max > 0) {
-    const int tm = to.tile_max;
+  for (int li = 0; li < 2; ++li) {
+    const TileList& tl = to.list[li];
+    if (tl.tile_max <= 0) continue;
+    const int tm = tl.tile_max;
     const int nt = block_scan_experts(
         E, [&](int e) { return (offs[e + 1] - offs[e] + tm - 1) / tm; }, tsc);
     // an expert's rows are split into its n tiles as evenly as the bm granule
@@ -207,13 +212,13 @@ __device__ void block_finalize(const int* cnt, int64_t E, int32_t bm, int32_t S,
       int start = offs[e];
       for (int j = 0; j < n; ++j) {
         const int u = units / n + (j < units % n ? 1 : 0);
-        to.tile_row[tsc[e] + j] = start;
-        to.tile_rows[tsc[e] + j] = u * bm;
-        to.tile_expert[tsc[e] + j] = e;
+        tl.tile_row[tsc[e] + j] = start;
+        tl.tile_rows[tsc[e] + j] = u * bm;
+        tl.tile_expert[tsc[e] + j] = e;
         start += u * bm;
       }
     }
-    if (threadIdx.x == 0) *to.num_tiles = nt;
+    if (threadIdx.x == 0) *tl.num_tiles = nt;
   }
 }
 
@@ -362,11 +367,14 @@ cudaError_t launch_align(const View2& ids, int64_t T, int64_t k, int64_t E, int3
                          int64_t n_chunks, DeviceErrors* err, cudaStream_t st, int* launches,
                          const AlignTiles* tiles) {
   TileOut to;
-  to.tile_max = tiles ? tiles->tile_max : 0;
-  to.tile_row = tiles ? tiles->tile_row : nullptr;
-  to.tile_rows = tiles ? tiles->tile_rows : nullptr;
-  to.tile_expert = tiles ? tiles->tile_expert : nullptr;
-  to.num_tiles = tiles ? tiles->num_tiles : nullptr;
+  for (int li = 0; li < 2; ++li) {
+    TileList& tl = to.list[li];
+    tl.tile_max = tiles ? tiles->list[li].tile_max : 0;
+    tl.tile_row = tiles ? tiles->list[li].tile_row : nullptr;
+    tl.tile_rows = tiles ? tiles->list[li].tile_rows : nullptr;
+    tl.tile_expert = tiles ? tiles->list[li].tile_expert : nullptr;
+    tl.num_tiles = tiles ? tiles->list[li].num_tiles : nullptr;
+  }
   if (E > kMaxExperts) return cudaErrorInvalidValue;
   const int64_t S = T * k;
   cudaError_t rc;

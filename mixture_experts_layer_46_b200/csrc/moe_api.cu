@@ -316,6 +316,8 @@ WsLayout make_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, bool
   L.p_max = p;
   L.nb_max = p / bm;
   L.t_max = tile_max > 0 ? p / tile_max + nonempty + 1 : 0;
+  // 256-row tiles for the single-slice GEMM2 on CTA pairs (bf16, 128-row tiles)
+  L.t_max2 = (!mxfp4 && tile_max == 128) ? p / 256 + nonempty + 1 : 0;
   L.n_chunks = (S + kAlignChunk - 1) / kAlignChunk;
   if (L.n_chunks < 1) L.n_chunks = 1;
   size_t off = 0;
@@ -334,6 +336,9 @@ WsLayout make_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, bool
   L.tile_row = take(sizeof(int32_t) * L.t_max);
   L.tile_rows = take(sizeof(int32_t) * L.t_max);
   L.tile_expert = take(sizeof(int32_t) * L.t_max);
+  L.tile_row2 = take(sizeof(int32_t) * L.t_max2);
+  L.tile_rows2 = take(sizeof(int32_t) * L.t_max2);
+  L.tile_expert2 = take(sizeof(int32_t) * L.t_max2);
   if (!mxfp4) {
     L.a1 = take(size_t(p) * H * 2);
     L.a1_scale = off;
@@ -400,11 +405,12 @@ moe_status_t forward_mxfp4(const moe_tensor_t* x, const moe_w13_t* w13, const mo
     if (s != MOE_OK) return s;
   }
   AlignTiles tiles;
-  tiles.tile_max = L.tile_max;
-  tiles.tile_row = reinterpret_cast<int32_t*>(w + L.tile_row);
-  tiles.tile_rows = reinterpret_cast<int32_t*>(w + L.tile_rows);
-  tiles.tile_expert = reinterpret_cast<int32_t*>(w + L.tile_expert);
-  tiles.num_tiles = num_blocks + 1;
+  std::memset(&tiles, 0, sizeof(tiles));
+  tiles.list[0].tile_max = L.tile_max;
+  tiles.list[0].tile_row = reinterpret_cast<int32_t*>(w + L.tile_row);
+  tiles.list[0].tile_rows = reinterpret_cast<int32_t*>(w + L.tile_rows);
+  tiles.list[0].tile_expert = reinterpret_cast<int32_t*>(w + L.tile_expert);
+  tiles.list[0].num_tiles = num_blocks + 1;
   t_prof.n = 0;
   t_prof.have = false;
   prof_mark(st);
@@ -423,10 +429,10 @@ moe_status_t forward_mxfp4(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   g1.N = pr.I;
   g1.n_wt = pr.I / 128;
   g1.max_tiles = L.t_max;
-  g1.num_tiles = tiles.num_tiles;
-  g1.tile_row = tiles.tile_row;
-  g1.tile_rows = tiles.tile_rows;
-  g1.tile_expert = tiles.tile_expert;
+  g1.num_tiles = tiles.list[0].num_tiles;
+  g1.tile_row = tiles.list[0].tile_row;
+  g1.tile_rows = tiles.list[0].tile_rows;
+  g1.tile_expert = tiles.list[0].tile_expert;
   g1.sorted = sorted;
   g1.S = L.S;
   g1.out = w + L.h;
@@ -521,6 +527,13 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   if (const char* env = getenv("MOE_TOKBOX"))
     if (atoi(env) == 0) tok_box = pair ? 16u : 32u;
   const uint32_t boxt[2] = {64, tok_box};
+  // GEMM2 on CTA pairs: one 256-row w2 slice per work item over 256-row token
+  // tiles (align's second list), which keeps two accumulator buffers in TMEM
+  // and stages 32 KiB per k-block.  MOE_G2=1 selects two 256-row slices over
+  // the 128-row tiles (tuning).
+  bool g2_single = pair && L.tile_max == 128 && L.t_max2 > 0;
+  if (const char* env = getenv("MOE_G2")) g2_single = g2_single && atoi(env) != 1;
+  const uint32_t boxt2[2] = {64, g2_single ? 128u : tok_box};
   {
     const uint64_t d[2] = {uint64_t(pr.H), uint64_t(L.p_max)};
     const uint64_t sb[1] = {uint64_t(pr.H) * 2};
@@ -544,7 +557,7 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   {
     const uint64_t d[2] = {uint64_t(pr.I), uint64_t(L.p_max)};
     const uint64_t sb[1] = {uint64_t(pr.I) * 2};
-    s = make_map(&mH, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w + L.h, d, sb, boxt,
+    s = make_map(&mH, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w + L.h, d, sb, boxt2,
                  CU_TENSOR_MAP_SWIZZLE_128B);
     if (s != MOE_OK) return s;
     const uint64_t d3[3] = {uint64_t(pr.I), uint64_t(pr.H), uint64_t(pr.E)};
@@ -556,11 +569,19 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
 
   // ---- launches
   AlignTiles tiles;
-  tiles.tile_max = L.tile_max;
-  tiles.tile_row = reinterpret_cast<int32_t*>(w + L.tile_row);
-  tiles.tile_rows = reinterpret_cast<int32_t*>(w + L.tile_rows);
-  tiles.tile_expert = reinterpret_cast<int32_t*>(w + L.tile_expert);
-  tiles.num_tiles = num_blocks + 1;
+  std::memset(&tiles, 0, sizeof(tiles));
+  tiles.list[0].tile_max = L.tile_max;
+  tiles.list[0].tile_row = reinterpret_cast<int32_t*>(w + L.tile_row);
+  tiles.list[0].tile_rows = reinterpret_cast<int32_t*>(w + L.tile_rows);
+  tiles.list[0].tile_expert = reinterpret_cast<int32_t*>(w + L.tile_expert);
+  tiles.list[0].num_tiles = num_blocks + 1;
+  if (g2_single) {
+    tiles.list[1].tile_max = 256;
+    tiles.list[1].tile_row = reinterpret_cast<int32_t*>(w + L.tile_row2);
+    tiles.list[1].tile_rows = reinterpret_cast<int32_t*>(w + L.tile_rows2);
+    tiles.list[1].tile_expert = reinterpret_cast<int32_t*>(w + L.tile_expert2);
+    tiles.list[1].num_tiles = num_blocks + 2;
+  }
   t_prof.n = 0;
   t_prof.have = false;
   prof_mark(st);
@@ -580,10 +601,10 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   g1.N = pr.I;
   g1.n_wt = pair ? (pr.I + 255) / 256 : (pr.I + 127) / 128;
   g1.max_tiles = L.t_max;
-  g1.num_tiles = tiles.num_tiles;
-  g1.tile_row = tiles.tile_row;
-  g1.tile_rows = tiles.tile_rows;
-  g1.tile_expert = tiles.tile_expert;
+  g1.num_tiles = tiles.list[0].num_tiles;
+  g1.tile_row = tiles.list[0].tile_row;
+  g1.tile_rows = tiles.list[0].tile_rows;
+  g1.tile_expert = tiles.list[0].tile_expert;
   g1.sorted = sorted;
   g1.S = L.S;
   g1.out = w + L.h;
@@ -601,10 +622,20 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   g2.K = pr.I;
   g2.N = pr.H;
   g2.n_wt = pair ? (pr.H + 511) / 512 : (pr.H + 255) / 256;
+  if (g2_single) {
+    g2.n_wt = (pr.H + 255) / 256;
+    g2.max_tiles = L.t_max2;
+    g2.num_tiles = tiles.list[1].num_tiles;
+    g2.tile_row = tiles.list[1].tile_row;
+    g2.tile_rows = tiles.list[1].tile_rows;
+    g2.tile_expert = tiles.list[1].tile_expert;
+    g2.tok_box = 128;
+  }
   g2.out = w + L.y;
   g2.out_ld = pr.H;
   g2.topk_w = view2(wts);
-  rc = pair ? launch_gemm_ws_pair_bf16(1, L.tile_max, mW2, mW2, mH, g2, dev->num_sms, st, &launches)
+  rc = g2_single ? launch_gemm_ws_pair_bf16(2, 256, mW2, mW2, mH, g2, dev->num_sms, st, &launches)
+     : pair      ? launch_gemm_ws_pair_bf16(1, L.tile_max, mW2, mW2, mH, g2, dev->num_sms, st, &launches)
             : launch_gemm_ws_bf16(1, L.tile_max, mW2, mW2, mH, g2, dev->num_sms, st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm2");
   prof_mark(st);

@@ -13,6 +13,8 @@
 //          h[token, i] = bf16(silu(acc0) * acc1)
 //   GEMM2: W0 = w2 rows [512 w, 512 w + 256), W1 = [512 w + 256, 512 w + 512);
 //          y[token row, o] = bf16(w_slot * acc)
+//   GEMM2, one slice (mode 2): W0 = w2 rows [256 w, 256 w + 256) only, so a
+//          256-row token tile still fits two accumulator buffers in TMEM
 //
 // Pair protocol (cluster of 2, rank 0 leads):
 //   * both producers wait on their own `empty` slot, load their halves with
@@ -39,15 +41,19 @@ constexpr int kTmemCols = 512;
 constexpr int kWBytes = kWRows * kBK * 2;    // 16 KiB
 constexpr int kStagingBytes = 32 * 64;
 
-// kNmax token rows per tile (per pair, each CTA loads half); an accumulator
-// buffer is acc0 [0, kNmax) + acc1 [kNmax, 2 kNmax) columns, two buffers when
-// they fit (kNmax <= 128) so the epilogue overlaps the next item's mainloop.
-template <int kNmax>
+// kNmax token rows per tile (per pair, each CTA loads half).  Modes 0 and 1
+// stage two weight tiles per k-block and accumulate into acc0 [0, kNmax) +
+// acc1 [kNmax, 2 kNmax); mode 2 stages one and accumulates into acc0 only.
+// Two accumulator buffers when they fit, so the epilogue overlaps the next
+// item's mainloop; as many stages as about 208 KiB of shared memory holds.
+template <int kMode, int kNmax>
 struct PairCfg {
+  static constexpr int kTiles = kMode == 2 ? 1 : 2;
   static constexpr int kXBytes = (kNmax / 2) * kBK * 2;
-  static constexpr int kStageBytes = 2 * kWBytes + kXBytes;
-  static constexpr int kStages = kNmax >= 256 ? 4 : 5;
-  static constexpr int kBufCols = 2 * kNmax;
+  static constexpr int kStageBytes = kTiles * kWBytes + kXBytes;
+  static constexpr int kStagesFit = (208 * 1024) / kStageBytes;
+  static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
+  static constexpr int kBufCols = kTiles * kNmax;
   static constexpr int kBufs = kTmemCols / kBufCols >= 2 ? 2 : 1;
   static constexpr size_t kSmem = 1024 + size_t(kStages) * kStageBytes +
                                   kEpiWarps * kStagingBytes + (2 * kStages + 5) * 8 + 16;
@@ -142,7 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemm_ws_pair_kernel(const __grid_constant__ CUtensorMap tmW0,
                         const __grid_constant__ CUtensorMap tmW1,
                         const __grid_constant__ CUtensorMap tmX, const Args g) {
-  using C = PairCfg<kNmax>;
+  using C = PairCfg<kMode, kNmax>;
   constexpr int kStages = C::kStages;
   constexpr int kStageBytes = C::kStageBytes;
   extern __shared__ uint8_t smem_raw[];
@@ -202,22 +208,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int64_t item = pair; item < total && ok; item += n_pairs) {
         const int64_t t = item / g.n_wt, wt = item - t * g.n_wt;
         const int32_t e = g.tile_expert[t], row0 = g.tile_row[t], rows = g.tile_rows[t];
-        const int32_t w0 = static_cast<int32_t>((kMode == 0 ? wt * 2 * kWRows : wt * 4 * kWRows) + rank * kWRows);
-        const int32_t w1 = kMode == 0 ? w0 : w0 + 2 * kWRows;
+        // weight rows of this CTA: GEMM1 gate/up rows 256 wt + 128 rank; GEMM2 w2
+        // rows 512 wt + 128 rank (+ 256 for the second slice); single-slice
+        // GEMM2 w2 rows 256 wt + 128 rank
+        const int32_t w0 = static_cast<int32_t>((kMode == 1 ? wt * 4 * kWRows : wt * 2 * kWRows) + rank * kWRows);
+        const int32_t w1 = kMode == 1 ? w0 + 2 * kWRows : w0;
         const int32_t half = rows / 2;
         const int32_t my_row0 = row0 + static_cast<int32_t>(rank) * half;
         // whole boxes: a box may run past this CTA's half (rows the MMA's N excludes)
         const int nbox = (half + g.tok_box - 1) / g.tok_box;
-        const uint32_t bytes_pair = 2 * (2 * kWBytes + nbox * g.tok_box * kBK * 2);
+        const uint32_t bytes_pair = 2 * (C::kTiles * kWBytes + nbox * g.tok_box * kBK * 2);
         for (int kb = 0; kb < num_k; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, g.err)) { ok = false; break; }
           uint8_t* sw0 = stages + stage * kStageBytes;
           uint8_t* sw1 = sw0 + kWBytes;
-          uint8_t* sx = sw1 + kWBytes;
+          uint8_t* sx = sw0 + C::kTiles * kWBytes;
           if (leader) mbar_arrive_expect_tx(&full[stage], bytes_pair);
           const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
           tma_load_3d_pair(sw0, &tmW0, fb, kb * kBK, w0, e, wpol);
-          tma_load_3d_pair(sw1, kMode == 0 ? &tmW1 : &tmW0, fb, kb * kBK, w1, e, wpol);
+          if (C::kTiles == 2)
+            tma_load_3d_pair(sw1, kMode == 0 ? &tmW1 : &tmW0, fb, kb * kBK, w1, e, wpol);
           for (int b = 0; b < nbox; ++b)
             tma_load_2d_pair(sx + b * g.tok_box * kBK * 2, &tmX, fb, kb * kBK, my_row0 + b * g.tok_box, pol);
           last_phase[stage] = static_cast<int8_t>(phase);
@@ -246,13 +256,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t w0_addr = smem_u32(stages + stage * kStageBytes);
           const uint32_t w1_addr = w0_addr + kWBytes;
-          const uint32_t x_addr = w1_addr + kWBytes;
+          const uint32_t x_addr = w0_addr + C::kTiles * kWBytes;
 #pragma unroll
           for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
             const uint64_t xd = sw128_kmajor_desc(x_addr + kk * kUmmaK * 2);
             const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
             mma_bf16_pair(acc0, sw128_kmajor_desc(w0_addr + kk * kUmmaK * 2), xd, idesc, acc);
-            mma_bf16_pair(acc1, sw128_kmajor_desc(w1_addr + kk * kUmmaK * 2), xd, idesc, acc);
+            if (C::kTiles == 2)
+              mma_bf16_pair(acc1, sw128_kmajor_desc(w1_addr + kk * kUmmaK * 2), xd, idesc, acc);
           }
           issued = true;
           commit_pair(&empty[stage], 0x3);
@@ -283,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // and routing weights while the accumulator is being built
       int32_t slot_r[kNmax / 64];
       float w_r[kNmax / 64];
-      if (kMode == 1) {
+      if (kMode >= 1) {
 #pragma unroll
         for (int i = 0; i < kNmax / 64; ++i) {
           const int c = half + 2 * i;
@@ -307,19 +318,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (c * 32 >= rows) break;
         uint32_t v0[32], v1[32];
         tmem_ld32(tmem_base + lane_base + c * 32, v0);
-        tmem_ld32(tmem_base + lane_base + kNmax + c * 32, v1);
+        if (C::kTiles == 2) tmem_ld32(tmem_base + lane_base + kNmax + c * 32, v1);
         float wj[32];
-        if (kMode == 1) {
+        if (kMode >= 1) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) wj[j] = __shfl_sync(0xffffffffu, w_r[i], j);
         }
         tmem_wait_ld();
-        constexpr int kOuts = (kMode == 0) ? 1 : 2;
+        constexpr int kOuts = (kMode == 1) ? 2 : 1;
 #pragma unroll
         for (int a = 0; a < kOuts; ++a) {
-          const int64_t col0 = (kMode == 0)
-                                   ? wt * 2 * kWRows + rank * kWRows + quad * 32
-                                   : wt * 4 * kWRows + a * 2 * kWRows + rank * kWRows + quad * 32;
+          const int64_t col0 = (kMode == 1)
+                                   ? wt * 4 * kWRows + a * 2 * kWRows + rank * kWRows + quad * 32
+                                   : wt * 2 * kWRows + rank * kWRows + quad * 32;
           const bool col_ok = col0 < g.N;
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
@@ -341,9 +352,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                          : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                          : "r"(stg_s + j * 64 + part * 16));
-            const int32_t s_j = (kMode == 1) ? __shfl_sync(0xffffffffu, slot_r[i], j) : 0;
+            const int32_t s_j = (kMode >= 1) ? __shfl_sync(0xffffffffu, slot_r[i], j) : 0;
             if (!col_ok) continue;
-            if (kMode == 1 && s_j >= g.S) continue;
+            if (kMode >= 1 && s_j >= g.S) continue;
             const int64_t p = row0 + c * 32 + j;
             *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + p * g.out_ld + col0 + part * 8) = v;
           }
@@ -369,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int kMode, int kNmax>
 cudaError_t launch_pair(const CUtensorMap& w0, const CUtensorMap& w1, const CUtensorMap& x,
                         const Args& g, int64_t max_items, int num_sms, cudaStream_t st) {
-  using C = PairCfg<kNmax>;
+  using C = PairCfg<kMode, kNmax>;
   static unsigned long long configured = 0;
   int dev = 0;
   cudaError_t rc = cudaGetDevice(&dev);
@@ -425,10 +436,12 @@ cudaError_t launch_gemm_ws_pair_bf16(int mode, int tile_max, const CUtensorMap& 
   const int64_t max_items = p.max_tiles * p.n_wt;
   if (tile_max == 256) {
     if (mode == 0) return launch_pair<0, 256>(w0, w1, x, g, max_items, num_sms, st);
+    if (mode == 2) return launch_pair<2, 256>(w0, w1, x, g, max_items, num_sms, st);
     return launch_pair<1, 256>(w0, w1, x, g, max_items, num_sms, st);
   }
   if (tile_max == 128) {
     if (mode == 0) return launch_pair<0, 128>(w0, w1, x, g, max_items, num_sms, st);
+    if (mode == 2) return launch_pair<2, 128>(w0, w1, x, g, max_items, num_sms, st);
     return launch_pair<1, 128>(w0, w1, x, g, max_items, num_sms, st);
   }
   return cudaErrorInvalidValue;

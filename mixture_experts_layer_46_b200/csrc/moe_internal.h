@@ -24,12 +24,14 @@ struct WsLayout {
   int32_t bm;         // block_m: padding granule of each expert's rows
   int32_t tile_max;   // token-tile rows of the weight-stationary GEMMs (0: unused)
   int64_t t_max;      // upper bound of the token-tile count
+  int64_t t_max2;     // the same for the second (256-row) tile list, 0 when absent
   int64_t n_chunks;   // align chunks
   int64_t p_max;      // upper bound of padded slot count
   int64_t nb_max;     // upper bound of the block count
   bool mxfp4;
   size_t counts, offsets, num_blocks, chunk_counts, sorted, inv, block_expert;
   size_t tile_row, tile_rows, tile_expert;
+  size_t tile_row2, tile_rows2, tile_expert2;
   size_t a1, a1_scale, h, h_scale, y;
   size_t total;
 };
@@ -48,12 +50,15 @@ WsLayout make_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, bool
 
 // Token-tile list for the weight-stationary GEMMs: tiles of up to tile_max
 // padded rows that never cross an expert boundary.
-struct AlignTiles {
-  int32_t tile_max;
+struct AlignTileList {
+  int32_t tile_max;  // 0: not produced
   int32_t* tile_row;
   int32_t* tile_rows;
   int32_t* tile_expert;
   int32_t* num_tiles;
+};
+struct AlignTiles {
+  AlignTileList list[2];  // [0]: the GEMMs' tiles, [1]: 256-row tiles for single-slice GEMM2
 };
 
 // align: ids -> counts, offsets, sorted, block_expert, num_blocks (+ tile list)

@@ -296,9 +296,14 @@ def test_token_tile_configs_agree_and_match_oracle(T, H, I, E, k, monkeypatch):
     ref = run_oracle(case)
     c = to_cuda(case)
     outs = {}
-    for tile in ("32", "128", "256"):
-        monkeypatch.setenv("MOE_TILE", tile)
+    for tile in ("32", "128", "256", "128/two-slice"):
+        # "128": on CTA pairs GEMM2 takes one 256-row w2 slice per 256-row token
+        # tile; "128/two-slice": two slices per 128-row token tile
+        monkeypatch.setenv("MOE_TILE", tile.split("/")[0])
+        if "/" in tile:
+            monkeypatch.setenv("MOE_G2", "1")
         outs[tile] = run_gpu(c)
         assert rel_err(outs[tile], ref) <= BF16_TOL, tile
     assert torch.equal(outs["32"], outs["128"])
     assert torch.equal(outs["128"], outs["256"])
+    assert torch.equal(outs["128"], outs["128/two-slice"])
