@@ -476,24 +476,36 @@ def main():
 def sweep(args, w, moe, wl, dev, stream, flush):
     """Token sweep on the same weights (fresh routing per T): one JSONL row per T."""
     hbm, tf_burst, _, _ = peaks()
-    w13, w2 = wl.make_weights_bf16(w["E"], w["I"], w["H"], seed=0, device=dev)
-    v13 = moe.w13_from_packed(w13)
+    mx = bool(w.get("mxfp4"))
+    if mx:
+        tf_burst = tf_burst * 4.0  # FP4 dense peak: measured bf16 x the nominal 4x ratio (assumed)
+        c13, s13, w2, s2 = make_mx_weights(w, dev)
+        v13 = moe.w13_from_packed(c13, s13)
+        tokens = wl.MXFP4_TOKEN_SWEEP
+    else:
+        w13, w2 = wl.make_weights_bf16(w["E"], w["I"], w["H"], seed=0, device=dev)
+        v13 = moe.w13_from_packed(w13)
+        s2 = None
+        tokens = wl.TOKEN_SWEEP
     with open(args.sweep, "w") as f:
-        for T in wl.TOKEN_SWEEP:
+        for T in tokens:
             wt = dict(w, T=T)
             x = wl.make_x(T, w["H"], seed=2000 + T, device=dev)
-            ids, wts = wl.route_softmax_topk(T, w["E"], w["k"], seed=1000 + T, device=dev)
-            ws = torch.empty(moe.workspace_bytes(T, w["H"], w["I"], w["E"], w["k"]), dtype=torch.uint8,
-                             device=dev)
+            if w["routing"] == "shared":
+                ids, wts = wl.route_shared_expert(T, w["E"] - 1, w["k"] - 1, seed=1000 + T, device=dev)
+            else:
+                ids, wts = wl.route_softmax_topk(T, w["E"], w["k"], seed=1000 + T, device=dev)
+            ws = torch.empty(moe.workspace_bytes(T, w["H"], w["I"], w["E"], w["k"], mxfp4=mx),
+                             dtype=torch.uint8, device=dev)
             out = torch.empty(T, w["H"], dtype=torch.bfloat16, device=dev)
             for _ in range(5):
-                moe.forward(x, v13, w2, ids, wts, out=out, workspace=ws, stream=stream)
+                moe.forward(x, v13, w2, ids, wts, out=out, workspace=ws, stream=stream, w2_scale=s2)
             per = []
-            for i in range(30 if T < 8192 else 10):
+            for i in range(30 if T < 8192 else 10 if T <= 16384 else 5):
                 flush.fill_(i & 0xff)
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record(stream)
-                moe.forward(x, v13, w2, ids, wts, out=out, workspace=ws, stream=stream)
+                moe.forward(x, v13, w2, ids, wts, out=out, workspace=ws, stream=stream, w2_scale=s2)
                 b.record(stream)
                 torch.cuda.synchronize(dev)
                 per.append(a.elapsed_time(b))
@@ -502,7 +514,7 @@ def sweep(args, w, moe, wl, dev, stream, flush):
             brk = {}
             for i in range(5):
                 flush.fill_(i & 0xff)
-                moe.forward(x, v13, w2, ids, wts, out=out, workspace=ws, stream=stream)
+                moe.forward(x, v13, w2, ids, wts, out=out, workspace=ws, stream=stream, w2_scale=s2)
                 for kname, kms in moe.profile_read().items():
                     brk[kname] = brk.get(kname, 0.0) + kms * 1e3 / 5
             moe.profile_enable(False)

@@ -45,6 +45,7 @@ GLM45_AIR = MoEShape(T=16384, H=4096, I=1408, E=128, k=8)
 QWEN35_TP2_MXFP4 = MoEShape(T=4096, H=4096, I=512, E=512, k=10)
 QWEN35_TP2_MXFP4_SHARED = MoEShape(T=4096, H=4096, I=512, E=513, k=11)
 TOKEN_SWEEP = (1, 2, 4, 8, 16, 32, 64, 128, 256, 512, 1023, 1024, 2048, 4096, 4097, 8192, 16384)
+MXFP4_TOKEN_SWEEP = (1, 16, 256, 4096, 32768)
 
 
 def _gen(seed: int, device) -> torch.Generator:
