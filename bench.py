@@ -52,10 +52,10 @@ WORKLOADS = {
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed to the hash of the kernel
 # source it was taken on; reported as null once the source has changed.
 NCU_TRAFFIC = {
-    # profiles/gemm_ws_pair_bf16_qwen3shape_E32_T1024.md: 983.0 MB read + 25.7 MB written on
+    # profiles/gemm_ws_pair_bf16_qwen3shape_E32_T1024.md: 984.1 MB read + 26.3 MB written on
     # the E=32, T=1024 case (~256 slots per expert), scaled x4 (experts and tokens) to the
     # E=128, T=4096 launch of the pair kernel
-    "gemm1_swiglu": {"bytes_per_launch": 4.0 * (982.952448e6 + 25.723648e6), "src": "0aac259f23670b9d",
+    "gemm1_swiglu": {"bytes_per_launch": 4.0 * (984.125952e6 + 26.287104e6), "src": "0abdc5a1383c3f9e",
                      "workload": "qwen3-235b T=4096"},
 }
 
