@@ -316,8 +316,10 @@ WsLayout make_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, bool
   L.p_max = p;
   L.nb_max = p / bm;
   L.t_max = tile_max > 0 ? p / tile_max + nonempty + 1 : 0;
-  // 256-row tiles for the single-slice GEMM2 on CTA pairs (bf16, 128-row tiles)
-  L.t_max2 = (!mxfp4 && tile_max == 128) ? p / 256 + nonempty + 1 : 0;
+  // second token-tile list: 256-row tiles for the single-slice GEMM2 on CTA
+  // pairs (bf16 with 128-row tiles)
+  L.tile_max2 = (!mxfp4 && tile_max == 128) ? 256 : 0;
+  L.t_max2 = L.tile_max2 > 0 ? p / L.tile_max2 + nonempty + 1 : 0;
   L.n_chunks = (S + kAlignChunk - 1) / kAlignChunk;
   if (L.n_chunks < 1) L.n_chunks = 1;
   size_t off = 0;

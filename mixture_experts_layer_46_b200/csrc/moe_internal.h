@@ -24,7 +24,8 @@ struct WsLayout {
   int32_t bm;         // block_m: padding granule of each expert's rows
   int32_t tile_max;   // token-tile rows of the weight-stationary GEMMs (0: unused)
   int64_t t_max;      // upper bound of the token-tile count
-  int64_t t_max2;     // the same for the second (256-row) tile list, 0 when absent
+  int32_t tile_max2;  // rows of the second token-tile list (bf16 pairs: 256; 0: none)
+  int64_t t_max2;     // upper bound of its tile count
   int64_t n_chunks;   // align chunks
   int64_t p_max;      // upper bound of padded slot count
   int64_t nb_max;     // upper bound of the block count
@@ -58,7 +59,7 @@ struct AlignTileList {
   int32_t* num_tiles;
 };
 struct AlignTiles {
-  AlignTileList list[2];  // [0]: the GEMMs' tiles, [1]: 256-row tiles for single-slice GEMM2
+  AlignTileList list[2];  // [0]: the GEMMs' tiles, [1]: 256-row tiles for the pair GEMM2
 };
 
 // align: ids -> counts, offsets, sorted, block_expert, num_blocks (+ tile list)
