@@ -353,6 +353,7 @@ WsLayout make_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, bool
     L.h_scale = take(size_t(p) * I / 32);
   }
   L.y = take(size_t(p) * H * 2);
+  L.w_row = take(mxfp4 ? sizeof(float) * size_t(p) : 0);
   L.total = off;
   return L;
 }
@@ -421,8 +422,8 @@ moe_status_t forward_mxfp4(const moe_tensor_t* x, const moe_w13_t* w13, const mo
                                 st, &launches, &tiles);
   if (rc != cudaSuccess) return cuda_fail(rc, "align");
   prof_mark(st);
-  rc = launch_permute_quant(view2(x), pr.T, pr.H, pr.k, inv, w + L.a1, w + L.a1_scale, st,
-                            &launches);
+  rc = launch_permute_quant(view2(x), pr.T, pr.H, pr.k, inv, w + L.a1, w + L.a1_scale, view2(wts),
+                            reinterpret_cast<float*>(w + L.w_row), st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "permute_quant");
   prof_mark(st);
   WsGemmMx g1;
@@ -471,6 +472,7 @@ moe_status_t forward_mxfp4(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   g2.w1_sf = g2.w0_sf;
   g2.w1_s0 = g2.w0_s0;
   g2.w1_s1 = g2.w0_s1;
+  g2.w_row = reinterpret_cast<const float*>(w + L.w_row);
   rc = launch_gemm_ws_mxfp4(1, L.tile_max, mW2, mW2, mH, g2, dev->num_sms, st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm2_mxfp4");
   prof_mark(st);

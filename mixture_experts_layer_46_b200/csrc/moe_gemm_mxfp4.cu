@@ -82,6 +82,7 @@ struct MxArgs {
   int64_t w0_s0, w0_s1;
   const uint8_t* w1_sf;
   int64_t w1_s0, w1_s1;
+  const float* w_row;    // GEMM2: routing weight per grouped row (valid rows)
   DeviceErrors* err;
 };
 
@@ -280,25 +281,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* stg = sm.staging + (warp - kFirstEpiWarp) * kStagingBytes;
     const uint32_t stg_s = smem_u32(stg);
     uint32_t buf = 0, acc_phase = 0;
+    // GEMM2: slot ids and routing weights of a tile's tokens (lane j of chunk c
+    // holds token c*32 + j), two independent loads per chunk (the weight comes
+    // from the grouped-row copy permute wrote), issued one work item ahead so
+    // their latency hides behind the previous item's epilogue
+    int32_t slot_r[kNmax / 32], slot_n[kNmax / 32];
+    float w_r[kNmax / 32], w_n[kNmax / 32];
+    auto fetch_rows = [&](int64_t it, int32_t (&sl)[kNmax / 32], float (&wv)[kNmax / 32]) {
+      if (kMode != 1 || it >= total) return;
+      const int64_t tt = it / g.n_wt;
+      const int32_t r0 = g.tile_row[tt], nr = g.tile_rows[tt];
+#pragma unroll
+      for (int c = 0; c < kNmax / 32; ++c) {
+        const bool in = c * 32 < nr;
+        sl[c] = in ? g.sorted[r0 + c * 32 + lane] : static_cast<int32_t>(g.S);
+        wv[c] = in ? g.w_row[r0 + c * 32 + lane] : 0.0f;
+      }
+    };
+    fetch_rows(blockIdx.x, slot_n, w_n);
     for (int64_t item = blockIdx.x; item < total; item += gridDim.x) {
       const int64_t t = item / g.n_wt, wt = item - t * g.n_wt;
       const int32_t row0 = g.tile_row[t], rows = g.tile_rows[t];
-      // GEMM2: slots and routing weights of the tile's tokens (lane j of chunk c
-      // holds token c*32 + j), fetched while the accumulator is still being built
-      int32_t slot_r[kNmax / 32];
-      float w_r[kNmax / 32];
       if (kMode == 1) {
 #pragma unroll
-        for (int c = 0; c < kNmax / 32; ++c)
-          slot_r[c] = (c * 32 < rows) ? g.sorted[row0 + c * 32 + lane] : static_cast<int32_t>(g.S);
-#pragma unroll
         for (int c = 0; c < kNmax / 32; ++c) {
-          w_r[c] = 0.0f;
-          if (slot_r[c] < g.S) {
-            const int64_t tt = slot_r[c] / g.k, jj = slot_r[c] - tt * g.k;
-            w_r[c] = static_cast<const float*>(g.topk_w.data)[tt * g.topk_w.s0 + jj * g.topk_w.s1];
-          }
+          slot_r[c] = slot_n[c];
+          w_r[c] = slot_n[c] < g.S ? w_n[c] : 0.0f;
         }
+        fetch_rows(item + gridDim.x, slot_n, w_n);
       }
       if (!mbar_wait(&sm.tfull[buf], acc_phase, g.err)) break;
       tc_fence_after();
@@ -451,6 +461,7 @@ cudaError_t launch_gemm_ws_mxfp4(int mode, int tile_max, const CUtensorMap& w0,
   g.w1_sf = p.w1_sf;
   g.w1_s0 = p.w1_s0;
   g.w1_s1 = p.w1_s1;
+  g.w_row = p.w_row;
   g.err = p.err;
   if (launches) *launches += 1;
   const int64_t max_items = p.max_tiles * p.n_wt;

@@ -34,6 +34,7 @@ struct WsLayout {
   size_t tile_row, tile_rows, tile_expert;
   size_t tile_row2, tile_rows2, tile_expert2;
   size_t a1, a1_scale, h, h_scale, y;
+  size_t w_row;       // MXFP4: routing weight per grouped row (written by permute)
   size_t total;
 };
 
@@ -74,10 +75,12 @@ cudaError_t launch_permute_bf16(const View2& x, int64_t T, int64_t H, int64_t k,
                                 const int32_t* inv, __nv_bfloat16* a1, cudaStream_t st,
                                 int* launches);
 
-// permute + MXFP4 quantisation of x rows (codes [P, H/2], scales [P, H/32])
+// permute + MXFP4 quantisation of x rows (codes [P, H/2], scales [P, H/32]);
+// also w_row[p] = routing weight of the slot at grouped row p (valid rows only)
 cudaError_t launch_permute_quant(const View2& x, int64_t T, int64_t H, int64_t k,
                                  const int32_t* inv, uint8_t* codes, uint8_t* scales,
-                                 cudaStream_t st, int* launches);
+                                 const View2& topk_w, float* w_row, cudaStream_t st,
+                                 int* launches);
 
 // combine: out[t, :] = sum_j y[inv[t*k + j], :] over valid slots (fixed j order)
 cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* inv, int64_t T, int64_t H,
@@ -153,6 +156,7 @@ struct WsGemmMx {
   int64_t w0_s0, w0_s1;
   const uint8_t* w1_sf;   // GEMM1: up scales; GEMM2: w2 scales
   int64_t w1_s0, w1_s1;
+  const float* w_row;     // GEMM2: routing weight per grouped row
   DeviceErrors* err;
 };
 // tile_max: 96 (4-stage ring) or 32 (5-stage ring)

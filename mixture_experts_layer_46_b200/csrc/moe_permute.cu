@@ -68,7 +68,8 @@ __global__ void __launch_bounds__(256) permute_bf16_kernel(View2 x, int64_t T, i
 // One thread per 32-element block of a row; a CTA walks tokens.
 __global__ void __launch_bounds__(128) permute_quant_kernel(View2 x, int64_t T, int64_t H, int64_t k,
                                                             const int32_t* inv, uint8_t* codes,
-                                                            uint8_t* scales, int vec_ok) {
+                                                            uint8_t* scales, View2 topk_w,
+                                                            float* w_row, int vec_ok) {
   pdl_wait();
   pdl_launch_dependents();
   const int64_t nb = H / 32;  // blocks per row
@@ -76,6 +77,10 @@ __global__ void __launch_bounds__(128) permute_quant_kernel(View2 x, int64_t T, 
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
       int32_t pos[kMaxTopK];
       for (int j = 0; j < k; ++j) pos[j] = inv[t * k + j];
+      // routing weight of each slot at its grouped row, for the down projection's epilogue
+      if (threadIdx.x < k && pos[threadIdx.x] >= 0)
+        w_row[pos[threadIdx.x]] =
+            static_cast<const float*>(topk_w.data)[t * topk_w.s0 + threadIdx.x * topk_w.s1];
       for (int64_t b = threadIdx.x; b < nb; b += blockDim.x) {
         float v[32];
         if (vec_ok) {
@@ -182,12 +187,13 @@ cudaError_t launch_permute_bf16(const View2& x, int64_t T, int64_t H, int64_t k,
 
 cudaError_t launch_permute_quant(const View2& x, int64_t T, int64_t H, int64_t k,
                                  const int32_t* inv, uint8_t* codes, uint8_t* scales,
-                                 cudaStream_t st, int* launches) {
+                                 const View2& topk_w, float* w_row, cudaStream_t st,
+                                 int* launches) {
   const int vec_ok = (x.s1 == 1) && ((x.s0 * 2) % 16 == 0) &&
                      (reinterpret_cast<uintptr_t>(x.data) % 16 == 0);
   if (launches) *launches += 1;
   return launch_pdl(permute_quant_kernel, dim3(static_cast<unsigned>(token_blocks(T))), dim3(128), 0,
-                    st, x, T, H, k, inv, codes, scales, vec_ok);
+                    st, x, T, H, k, inv, codes, scales, topk_w, w_row, vec_ok);
 }
 
 cudaError_t launch_quantize_rows(const void* src, int32_t src_dtype, int64_t R, int64_t K,
