@@ -52,17 +52,17 @@ WORKLOADS = {
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed to the hash of the kernel
 # source it was taken on; reported as null once the source has changed.
 NCU_TRAFFIC = {
-    # profiles/gemm_ws_pair_bf16_qwen3shape_E32_T1024.md: 984.1 MB read + 26.3 MB written on
-    # the E=32, T=1024 case (~256 slots per expert), scaled x4 (experts and tokens) to the
-    # E=128, T=4096 launch of the pair kernel
-    "gemm1_swiglu": {"bytes_per_launch": 4.0 * (984.125952e6 + 26.287104e6), "src": "0abdc5a1383c3f9e",
+    # profiles/gemm_ws_pair_bf16_qwen3shape_E32_T1024.md: 941.1 MB read + 26.4 MB written by
+    # GEMM1 (256-row token tiles) on the E=32, T=1024 case (~256 slots per expert), scaled x4
+    # (experts and tokens) to the E=128, T=4096 launch; keyed to the kernel and host sources
+    "gemm1_swiglu": {"bytes_per_launch": 4.0 * (941.06368e6 + 26.39104e6), "src": "51397945960f1598",
                      "workload": "qwen3-235b T=4096"},
 }
 
 
 def kernel_src_hash() -> str:
     h = hashlib.sha256()
-    for fn in ("moe_gemm_ws2.cu", "moe_common.cuh"):
+    for fn in ("moe_gemm_ws2.cu", "moe_common.cuh", "moe_api.cu"):
         with open(os.path.join(ROOT, "mixture_experts_layer_46_b200", "csrc", fn), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]

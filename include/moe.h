@@ -22,7 +22,9 @@
  *     call returns MOE_ERR_UNSUPPORTED_LAYOUT.
  *   - Device pointers unless the entry point says "host".  The caller owns every
  *     buffer; the library keeps no pointer after a call returns, except as keys of
- *     its descriptor cache.
+ *     its cache of encoded TMA descriptors (it never dereferences a cached
+ *     address; an entry is reused only for the same address, type, sizes,
+ *     strides and tile shape, whose encoding is then identical).
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream)
  *     and is asynchronous unless stated otherwise.
  *   - Shape, dtype and layout errors are reported before anything is launched or

@@ -10,6 +10,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <unordered_map>
 
 #include "../../include/moe.h"
 #include "moe_internal.h"
@@ -107,9 +108,53 @@ EncodeTiledFn encode_fn() {
 }
 
 // rank-2/3 K-major tile map: dims[0] is the contiguous (K) axis.
+// Encoded maps are cached by everything the encoding depends on (base
+// address, type, rank, sizes, strides, box, swizzle), so repeated calls on the
+// same weights and workspace skip the host-side encoding.  The cache holds
+// only keys and map bytes, never dereferences a cached address, and is cleared
+// when it reaches kMapCacheMax entries.
+struct MapKey {
+  uintptr_t base;
+  int32_t dt, rank, swz;
+  uint64_t dims[3], strides[2];
+  uint32_t box[3];
+  bool operator==(const MapKey& o) const { return std::memcmp(this, &o, sizeof(MapKey)) == 0; }
+};
+struct MapKeyHash {
+  size_t operator()(const MapKey& k) const {
+    // FNV-1a over the key bytes
+    const unsigned char* p = reinterpret_cast<const unsigned char*>(&k);
+    uint64_t h = 1469598103934665603ull;
+    for (size_t i = 0; i < sizeof(MapKey); ++i) h = (h ^ p[i]) * 1099511628211ull;
+    return static_cast<size_t>(h);
+  }
+};
+constexpr size_t kMapCacheMax = 256;
+std::mutex g_map_mu;
+std::unordered_map<MapKey, CUtensorMap, MapKeyHash> g_maps;
+
 moe_status_t make_map(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
                       const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
                       CUtensorMapSwizzle swz) {
+  MapKey key;
+  std::memset(&key, 0, sizeof(key));  // padding bytes take part in the comparison
+  key.base = reinterpret_cast<uintptr_t>(base);
+  key.dt = static_cast<int32_t>(dt);
+  key.rank = rank;
+  key.swz = static_cast<int32_t>(swz);
+  for (int i = 0; i < rank; ++i) {
+    key.dims[i] = dims[i];
+    key.box[i] = box[i];
+  }
+  for (int i = 0; i < rank - 1; ++i) key.strides[i] = strides_bytes[i];
+  {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    auto it = g_maps.find(key);
+    if (it != g_maps.end()) {
+      *map = it->second;
+      return MOE_OK;
+    }
+  }
   EncodeTiledFn fn = encode_fn();
   if (!fn) {
     t_last_cuda_error = "cuTensorMapEncodeTiled entry point unavailable";
@@ -132,6 +177,9 @@ moe_status_t make_map(CUtensorMap* map, CUtensorMapDataType dt, int rank, const 
     t_last_cuda_error = buf;
     return MOE_ERR_CUDA;
   }
+  std::lock_guard<std::mutex> lk(g_map_mu);
+  if (g_maps.size() >= kMapCacheMax) g_maps.clear();
+  g_maps.emplace(key, *map);
   return MOE_OK;
 }
 
@@ -538,10 +586,19 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   bool g2_single = pair && L.tile_max == 128 && L.t_max2 > 0;
   if (const char* env = getenv("MOE_G2")) g2_single = g2_single && atoi(env) != 1;
   const uint32_t boxt2[2] = {64, g2_single ? 128u : tok_box};
+  // GEMM1 over the same 256-row tiles (one accumulator buffer of 2 x 256
+  // columns, so its epilogue is not overlapped) while experts average 96..399
+  // slots: the halved weight re-reads outweigh the exposed epilogue there
+  // (measured 6-20 % faster at T = 2048..6144 for the Qwen3 shape, neutral at
+  // 4096, mixed at 8192).  MOE_G1_256=0|1 overrides (tuning).
+  const int64_t avg_slots = pr.E > 0 ? (pr.T * pr.k) / pr.E : 0;
+  bool g1_256 = g2_single && avg_slots >= 96 && avg_slots < 400;
+  if (const char* env = getenv("MOE_G1_256")) g1_256 = g2_single && atoi(env) == 1;
+  const uint32_t boxt1[2] = {64, g1_256 ? 128u : tok_box};
   {
     const uint64_t d[2] = {uint64_t(pr.H), uint64_t(L.p_max)};
     const uint64_t sb[1] = {uint64_t(pr.H) * 2};
-    s = make_map(&mA1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w + L.a1, d, sb, boxt,
+    s = make_map(&mA1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w + L.a1, d, sb, boxt1,
                  CU_TENSOR_MAP_SWIZZLE_128B);
     if (s != MOE_OK) return s;
   }
@@ -617,7 +674,15 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   g1.err = dev->errors;
   g1.weights_evict_first = wpolicy;
   g1.tok_box = static_cast<int32_t>(tok_box);
-  rc = pair ? launch_gemm_ws_pair_bf16(0, L.tile_max, mGate, mUp, mA1, g1, dev->num_sms, st, &launches)
+  if (g1_256) {
+    g1.max_tiles = L.t_max2;
+    g1.num_tiles = tiles.list[1].num_tiles;
+    g1.tile_row = tiles.list[1].tile_row;
+    g1.tile_rows = tiles.list[1].tile_rows;
+    g1.tile_expert = tiles.list[1].tile_expert;
+    g1.tok_box = 128;
+  }
+  rc = pair ? launch_gemm_ws_pair_bf16(0, g1_256 ? 256 : L.tile_max, mGate, mUp, mA1, g1, dev->num_sms, st, &launches)
             : launch_gemm_ws_bf16(0, L.tile_max, mGate, mUp, mA1, g1, dev->num_sms, st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm1");
   prof_mark(st);
