@@ -87,24 +87,6 @@ cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* inv, int64_t T
                            int64_t k, void* out, int64_t os0, int64_t os1, cudaStream_t st,
                            int* launches);
 
-struct GemmArgs {
-  int64_t K;            // contraction length
-  int64_t N;            // output columns (I for GEMM1, H for GEMM2)
-  int64_t n_tiles;      // output column tiles
-  int64_t max_tiles;    // upper bound of (blocks x n_tiles)
-  const int32_t* num_blocks;
-  const int32_t* block_expert;
-  const int32_t* sorted;
-  int64_t S;            // sentinel / number of slots
-  void* out;            // GEMM1: h [P, I] (bf16 or e2m1 codes); GEMM2: y [S, H] bf16
-  uint8_t* out_scale;   // GEMM1 MXFP4: h scales [P, I/32]
-  int64_t out_ld;       // row stride of out in elements (bytes for codes)
-  View2 topk_w;         // GEMM2: routing weights [T, k] f32
-  int64_t k;            // top_k (GEMM2: slot -> (t, j))
-  DeviceErrors* err;
-};
-
-
 // Weight-stationary ("swap AB") bf16 GEMMs over the token-tile list of align.
 struct WsGemm {
   int64_t K, N, n_wt, max_tiles;

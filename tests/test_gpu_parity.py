@@ -296,14 +296,21 @@ def test_token_tile_configs_agree_and_match_oracle(T, H, I, E, k, monkeypatch):
     ref = run_oracle(case)
     c = to_cuda(case)
     outs = {}
-    for tile in ("32", "128", "256", "128/two-slice"):
+    for tile in ("32", "128", "256", "128/two-slice", "128/gemm1-128"):
         # "128": on CTA pairs GEMM2 takes one 256-row w2 slice per 256-row token
-        # tile; "128/two-slice": two slices per 128-row token tile
+        # tile (and GEMM1 the same tiles where experts average 96..399 slots);
+        # "128/two-slice": two slices per 128-row token tile; "128/gemm1-128":
+        # GEMM1 on the 128-row tiles with two accumulator buffers
+        monkeypatch.delenv("MOE_G2", raising=False)
+        monkeypatch.delenv("MOE_G1_256", raising=False)
         monkeypatch.setenv("MOE_TILE", tile.split("/")[0])
-        if "/" in tile:
+        if tile.endswith("two-slice"):
             monkeypatch.setenv("MOE_G2", "1")
+        if tile.endswith("gemm1-128"):
+            monkeypatch.setenv("MOE_G1_256", "0")
         outs[tile] = run_gpu(c)
         assert rel_err(outs[tile], ref) <= BF16_TOL, tile
     assert torch.equal(outs["32"], outs["128"])
     assert torch.equal(outs["128"], outs["256"])
     assert torch.equal(outs["128"], outs["128/two-slice"])
+    assert torch.equal(outs["128"], outs["128/gemm1-128"])
