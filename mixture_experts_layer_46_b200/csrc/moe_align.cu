@@ -232,6 +232,9 @@ __global__ void __launch_bounds__(kThreads) align_small_kernel(
   int* offs = hist + E;              // [E + 1]
   int* tsc = offs + E + 1;           // [E + 1]
   __shared__ int bad_sh;
+  // permute and, through it, the GEMM may be scheduled at once: both wait for
+  // this kernel before reading what it writes
+  pdl_launch_dependents();
   pdl_wait();
   const int64_t S = T * k;
   for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) wcnt[i] = 0;
@@ -262,7 +265,6 @@ __global__ void __launch_bounds__(kThreads) align_small_kernel(
     }
   }
   if (threadIdx.x == 0 && bad_sh && err) atomicAdd(&err->bad_ids, static_cast<unsigned>(bad_sh));
-  pdl_launch_dependents();
 }
 
 // Multi-CTA path, kernel 1: per chunk of kAlignChunk slots, the per-expert
@@ -359,6 +361,140 @@ __global__ void __launch_bounds__(256) align_scatter_kernel(View2 ids, int64_t T
   }
 }
 
+// Decode batches (at most 32 slots, one CTA per token): align and the bf16
+// permute in one kernel.  Warp 0 of every CTA groups the slots by expert with
+// match/ballot instead of a histogram over all E experts: for a slot routed
+// to expert e, its row is the padded rows of the routed experts below e plus
+// its rank among the earlier slots of e.  CTA 0 writes align's outputs (the
+// same values as the general kernels); every CTA copies its token's x row to
+// the token's rows of a1.
+constexpr int kTinyThreads = 256;
+
+__global__ void __launch_bounds__(kTinyThreads) align_permute_tiny_kernel(
+    View2 ids, int64_t T, int64_t k, int64_t E, int32_t bm, int32_t* counts, int32_t* offsets,
+    int32_t* sorted, int32_t* inv, int32_t* block_expert, int32_t* num_blocks, TileOut to,
+    DeviceErrors* err, View2 x, int64_t H, __nv_bfloat16* a1, int vec_ok) {
+  __shared__ int d_e[33], d_cnt[32], d_off[33], pos_sh[32];
+  __shared__ int nd_sh;
+  pdl_launch_dependents();
+  pdl_wait();
+  const int S = static_cast<int>(T * k);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const bool writer = blockIdx.x == 0;
+  if (warp == 0) {
+    int64_t id = -1;
+    if (lane < S) id = read_id(ids, lane, k);
+    const bool valid = lane < S && id >= 0 && id < E;
+    const int key = valid ? static_cast<int>(id) : -1 - lane;  // skipped slots: distinct keys
+    const unsigned same = __match_any_sync(0xffffffffu, key);
+    const bool first = valid && (__ffs(same) - 1 == lane);
+    const unsigned firsts = __ballot_sync(0xffffffffu, first);
+    const unsigned bad = __ballot_sync(0xffffffffu, lane < S && !valid);
+    int r = 0;  // routed experts below this slot's
+    for (int j = 0; j < 32; ++j) {
+      const int o = __shfl_sync(0xffffffffu, key, j);
+      r += (((firsts >> j) & 1u) != 0u && o < key) ? 1 : 0;
+    }
+    const int nd = __popc(firsts);
+    if (first) {
+      d_e[r] = key;
+      d_cnt[r] = __popc(same);
+    }
+    __syncwarp();
+    // lane r < nd: padded rows of the r-th routed expert, scanned across lanes
+    const int pr = lane < nd ? (d_cnt[lane] + bm - 1) / bm * bm : 0;
+    int incl = pr;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane < nd) d_off[lane] = incl - pr;
+    const int total_rows = __shfl_sync(0xffffffffu, incl, 31);
+    if (lane == 0) {
+      d_off[nd] = total_rows;
+      d_e[nd] = static_cast<int>(E);
+      nd_sh = nd;
+    }
+    __syncwarp();
+    pos_sh[lane] = valid ? d_off[r] + __popc(same & ((1u << lane) - 1u)) : -1;
+    __syncwarp();
+    if (writer && lane < S) {
+      inv[lane] = pos_sh[lane];
+      if (valid) sorted[pos_sh[lane]] = lane;
+    }
+    if (writer && lane == 0 && bad && err) atomicAdd(&err->bad_ids, static_cast<unsigned>(__popc(bad)));
+    if (writer) {
+      // token-tile lists: lane r < nd holds the r-th routed expert's tiles
+      for (int li = 0; li < 2; ++li) {
+        const TileList& tl = to.list[li];
+        if (tl.tile_max <= 0) continue;
+        const int n = pr > 0 ? (pr + tl.tile_max - 1) / tl.tile_max : 0;
+        int tincl = n;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, tincl, o);
+          if (lane >= o) tincl += v;
+        }
+        const int units = pr / bm;
+        int start = lane < nd ? d_off[lane] : 0;
+        for (int j = 0; j < n; ++j) {
+          const int u = units / n + (j < units % n ? 1 : 0);
+          tl.tile_row[tincl - n + j] = start;
+          tl.tile_rows[tincl - n + j] = u * bm;
+          tl.tile_expert[tincl - n + j] = d_e[lane];
+          start += u * bm;
+        }
+        const int ntiles = __shfl_sync(0xffffffffu, tincl, 31);
+        if (lane == 0) *tl.num_tiles = ntiles;
+      }
+    }
+  }
+  __syncthreads();
+  const int nd = nd_sh;
+  if (writer) {
+    const int total = d_off[nd];
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+      int below = 0, c = 0;
+      for (int r = 0; r < nd; ++r) {
+        below += d_e[r] < e ? 1 : 0;
+        if (d_e[r] == e) c = d_cnt[r];
+      }
+      offsets[e] = d_off[below];
+      if (e < E) counts[e] = c;
+    }
+    if (threadIdx.x == 0) *num_blocks = total / bm;
+    for (int p = threadIdx.x; p < total; p += blockDim.x) {
+      int r = 0;
+      while (r + 1 < nd && d_off[r + 1] <= p) ++r;
+      if (p - d_off[r] >= d_cnt[r]) sorted[p] = S;
+      if (p % bm == 0) block_expert[p / bm] = d_e[r];
+    }
+  }
+  // this CTA's token: its x row to the rows of its valid slots
+  const int64_t t = blockIdx.x;
+  const int64_t H8 = H / 8;
+  if (vec_ok) {
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x.data) + t * x.s0);
+    for (int64_t c = threadIdx.x; c < H8; c += blockDim.x) {
+      const uint4 v = __ldg(src + c);
+      for (int j = 0; j < k; ++j) {
+        const int p = pos_sh[t * k + j];
+        if (p >= 0) reinterpret_cast<uint4*>(a1 + static_cast<int64_t>(p) * H)[c] = v;
+      }
+    }
+  } else {
+    const uint16_t* src = static_cast<const uint16_t*>(x.data) + t * x.s0;
+    for (int64_t h = threadIdx.x; h < H; h += blockDim.x) {
+      const uint16_t v = src[h * x.s1];
+      for (int j = 0; j < k; ++j) {
+        const int p = pos_sh[t * k + j];
+        if (p >= 0) reinterpret_cast<uint16_t*>(a1 + static_cast<int64_t>(p) * H)[h] = v;
+      }
+    }
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_align(const View2& ids, int64_t T, int64_t k, int64_t E, int32_t bm,
@@ -409,6 +545,29 @@ cudaError_t launch_align(const View2& ids, int64_t T, int64_t k, int64_t E, int3
                   chunk_counts, offsets, sorted, inv);
   if (launches) *launches += 3;
   return rc;
+}
+
+cudaError_t launch_align_permute_tiny(const View2& ids, int64_t T, int64_t k, int64_t E, int32_t bm,
+                                      int32_t* counts, int32_t* offsets, int32_t* sorted,
+                                      int32_t* inv, int32_t* block_expert, int32_t* num_blocks,
+                                      DeviceErrors* err, const AlignTiles* tiles, const View2& x,
+                                      int64_t H, __nv_bfloat16* a1, cudaStream_t st, int* launches) {
+  if (T * k > 32 || T * k < 1) return cudaErrorInvalidValue;
+  TileOut to;
+  for (int li = 0; li < 2; ++li) {
+    TileList& tl = to.list[li];
+    tl.tile_max = tiles ? tiles->list[li].tile_max : 0;
+    tl.tile_row = tiles ? tiles->list[li].tile_row : nullptr;
+    tl.tile_rows = tiles ? tiles->list[li].tile_rows : nullptr;
+    tl.tile_expert = tiles ? tiles->list[li].tile_expert : nullptr;
+    tl.num_tiles = tiles ? tiles->list[li].num_tiles : nullptr;
+  }
+  const int vec_ok = (x.s1 == 1) && ((x.s0 * 2) % 16 == 0) &&
+                     (reinterpret_cast<uintptr_t>(x.data) % 16 == 0);
+  if (launches) *launches += 1;
+  return launch_pdl(align_permute_tiny_kernel, dim3(static_cast<unsigned>(T)), dim3(kTinyThreads), 0,
+                    st, ids, T, k, E, bm, counts, offsets, sorted, inv, block_expert, num_blocks, to,
+                    err, x, H, a1, vec_ok);
 }
 
 }  // namespace moe

@@ -647,13 +647,24 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   t_prof.have = false;
   prof_mark(st);
   cudaError_t rc;
-  rc = launch_align(view2(ids), pr.T, pr.k, pr.E, bm, counts, offsets, sorted, inv, block_expert,
-                    num_blocks, chunk_counts, L.n_chunks, dev->errors, st, &launches, &tiles);
-  if (rc != cudaSuccess) return cuda_fail(rc, "align");
-  prof_mark(st);
-  rc = launch_permute_bf16(view2(x), pr.T, pr.H, pr.k, inv,
-                           reinterpret_cast<__nv_bfloat16*>(w + L.a1), st, &launches);
-  if (rc != cudaSuccess) return cuda_fail(rc, "permute");
+  // decode sizes (at most 32 slots): align and permute in one launch
+  // (MOE_TINY=0 keeps the two kernels, tuning)
+  const bool tiny = L.S <= 32 && !(getenv("MOE_TINY") && atoi(getenv("MOE_TINY")) == 0);
+  if (tiny) {
+    rc = launch_align_permute_tiny(view2(ids), pr.T, pr.k, pr.E, bm, counts, offsets, sorted, inv,
+                                   block_expert, num_blocks, dev->errors, &tiles, view2(x), pr.H,
+                                   reinterpret_cast<__nv_bfloat16*>(w + L.a1), st, &launches);
+    if (rc != cudaSuccess) return cuda_fail(rc, "align_permute");
+    prof_mark(st);
+  } else {
+    rc = launch_align(view2(ids), pr.T, pr.k, pr.E, bm, counts, offsets, sorted, inv, block_expert,
+                      num_blocks, chunk_counts, L.n_chunks, dev->errors, st, &launches, &tiles);
+    if (rc != cudaSuccess) return cuda_fail(rc, "align");
+    prof_mark(st);
+    rc = launch_permute_bf16(view2(x), pr.T, pr.H, pr.k, inv,
+                             reinterpret_cast<__nv_bfloat16*>(w + L.a1), st, &launches);
+    if (rc != cudaSuccess) return cuda_fail(rc, "permute");
+  }
   prof_mark(st);
 
   WsGemm g1;
@@ -674,6 +685,13 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   g1.err = dev->errors;
   g1.weights_evict_first = wpolicy;
   g1.tok_box = static_cast<int32_t>(tok_box);
+  // decode sizes: GEMM1 finds its experts from the routing ids and requests
+  // weights while align and permute run (MOE_PREFETCH=0: off, tuning)
+  if (!pair && L.tile_max == 32 && L.S <= 32 && !(getenv("MOE_PREFETCH") && atoi(getenv("MOE_PREFETCH")) == 0)) {
+    g1.pre_ids = view2(ids);
+    g1.pre_E = static_cast<int32_t>(pr.E);
+    g1.pre_S = static_cast<int32_t>(L.S);
+  }
   if (g1_256) {
     g1.max_tiles = L.t_max2;
     g1.num_tiles = tiles.list[1].num_tiles;
@@ -688,6 +706,7 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   prof_mark(st);
 
   WsGemm g2 = g1;
+  g2.pre_S = 0;
   g2.K = pr.I;
   g2.N = pr.H;
   g2.n_wt = pair ? (pr.H + 511) / 512 : (pr.H + 255) / 256;

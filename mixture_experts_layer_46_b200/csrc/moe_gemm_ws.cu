@@ -68,8 +68,37 @@ struct WsArgs {
   int64_t k;
   int32_t weights_evict_first;
   int32_t tok_box;  // token rows per TMA box (the map's box height)
+  View2 pre_ids;     // GEMM1, at most 32 slots: routing ids (pre_S = 0: not used)
+  int32_t pre_E, pre_S;
   DeviceErrors* err;
 };
+
+// Decode batches (at most 32 routing slots on 32-row tiles) have one tile per
+// routed expert, in ascending expert order, so the expert of work item `item`
+// follows from the routing ids alone.  Whole warp; returns -1 past the items.
+__device__ __forceinline__ int first_expert_from_ids(const WsArgs& g, int64_t item, int lane) {
+  int64_t id = -1;
+  if (lane < g.pre_S) {
+    const int64_t t = lane / g.k, j = lane - t * g.k;
+    const int64_t off = t * g.pre_ids.s0 + j * g.pre_ids.s1;
+    id = g.pre_ids.dtype == MOE_I64 ? static_cast<const int64_t*>(g.pre_ids.data)[off]
+                                    : static_cast<const int32_t*>(g.pre_ids.data)[off];
+  }
+  const bool valid = id >= 0 && id < g.pre_E;
+  const int key = valid ? static_cast<int>(id) : -1 - lane;  // invalid slots: distinct keys
+  const unsigned same = __match_any_sync(0xffffffffu, key);
+  const bool first = valid && (__ffs(same) - 1 == lane);
+  const unsigned firsts = __ballot_sync(0xffffffffu, first);
+  int rank = 0;  // routed experts below this lane's
+  for (int j = 0; j < 32; ++j) {
+    const int other = __shfl_sync(0xffffffffu, key, j);
+    rank += (((firsts >> j) & 1u) != 0u && other < key) ? 1 : 0;
+  }
+  const int64_t tile = item / g.n_wt;
+  if (tile >= __popc(firsts)) return -1;
+  const unsigned who = __ballot_sync(0xffffffffu, first && rank == tile);
+  return __shfl_sync(0xffffffffu, key, __ffs(who) - 1);
+}
 
 template <int kStages>
 struct Smem {
@@ -134,9 +163,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *sm.tmem_slot;
 
+  const int num_k = static_cast<int>((g.K + kBK - 1) / kBK);
+  // GEMM1 at decode sizes: request the first weight stages of this CTA's first
+  // work item before waiting for align and permute (their token boxes follow
+  // after the wait, on the same stage barriers)
+  int npre = 0;
+  if (kMode == 0 && kNmax == 32 && g.pre_S > 0 && warp == 0) {
+    const int e = first_expert_from_ids(g, blockIdx.x, lane);
+    if (e >= 0) {
+      npre = num_k < kStages ? num_k : kStages;
+      if (lane == 0) {
+        const int64_t wt = blockIdx.x % g.n_wt;
+        const uint64_t wpol = g.weights_evict_first ? l2_policy_evict_first() : l2_policy_evict_last();
+        for (int kb = 0; kb < npre; ++kb) {
+          uint8_t* sw0 = sm.stages + kb * C::kStageBytes;
+          mbar_expect_tx(&sm.full[kb], 2 * C::kWBytes);
+          tma_load_3d(sw0, &tmW0, &sm.full[kb], kb * kBK, static_cast<int32_t>(wt * kWRows), e, wpol);
+          tma_load_3d(sw0 + C::kWBytes, &tmW1, &sm.full[kb], kb * kBK, static_cast<int32_t>(wt * kWRows), e, wpol);
+        }
+      }
+    }
+  }
   pdl_wait();
   const int64_t total = static_cast<int64_t>(*g.num_tiles) * g.n_wt;
-  const int num_k = static_cast<int>((g.K + kBK - 1) / kBK);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -146,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s < kStages; ++s) last_phase[s] = -1;
       const uint64_t pol = l2_policy_evict_last();
       const uint64_t wpol = g.weights_evict_first ? l2_policy_evict_first() : pol;
-      bool ok = true;
+      bool ok = true, pre_done = false;
       for (int64_t item = blockIdx.x; item < total && ok; item += gridDim.x) {
         const int64_t t = item / g.n_wt, wt = item - t * g.n_wt;
         const int32_t e = g.tile_expert[t], row0 = g.tile_row[t], rows = g.tile_rows[t];
@@ -160,9 +209,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* sw0 = sm.stages + stage * C::kStageBytes;
           uint8_t* sw1 = sw0 + C::kWBytes;
           uint8_t* sx = sw1 + C::kWBytes;
-          mbar_arrive_expect_tx(&sm.full[stage], bytes);
-          tma_load_3d(sw0, &tmW0, &sm.full[stage], kb * kBK, w0, e, wpol);
-          tma_load_3d(sw1, kMode == 0 ? &tmW1 : &tmW0, &sm.full[stage], kb * kBK, w1, e, wpol);
+          if (item == blockIdx.x && kb < npre) {
+            // weights already requested before the PDL wait
+            mbar_arrive_expect_tx(&sm.full[stage], bytes - 2 * C::kWBytes);
+            pre_done = true;
+          } else {
+            mbar_arrive_expect_tx(&sm.full[stage], bytes);
+            tma_load_3d(sw0, &tmW0, &sm.full[stage], kb * kBK, w0, e, wpol);
+            tma_load_3d(sw1, kMode == 0 ? &tmW1 : &tmW0, &sm.full[stage], kb * kBK, w1, e, wpol);
+          }
           for (int b = 0; b < nbox; ++b)
             tma_load_2d(sx + b * g.tok_box * kBK * 2, &tmX, &sm.full[stage], kb * kBK,
                         row0 + b * g.tok_box, pol);
@@ -173,6 +228,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) {
         for (int s = 0; s < kStages; ++s)
           if (last_phase[s] >= 0) mbar_wait(&sm.full[s], static_cast<uint32_t>(last_phase[s]), g.err);
+      }
+      if (npre > 0 && !pre_done) {
+        // prefetched stages nobody consumed: let their copies land before exit
+        for (int kb = 0; kb < npre; ++kb) {
+          mbar_arrive(&sm.full[kb]);
+          mbar_wait(&sm.full[kb], 0, g.err);
+        }
       }
     }
   } else if (warp == 1) {
@@ -358,6 +420,9 @@ cudaError_t launch_gemm_ws_bf16(int mode, int tile_max, const CUtensorMap& w0,
   g.err = p.err;
   g.weights_evict_first = p.weights_evict_first;
   g.tok_box = p.tok_box;
+  g.pre_ids = p.pre_ids;
+  g.pre_E = p.pre_E;
+  g.pre_S = (mode == 0 && tile_max == 32 && p.pre_S <= 32) ? p.pre_S : 0;
   if (launches) *launches += 1;
   const int64_t max_items = p.max_tiles * p.n_wt;
   if (tile_max == 128) {

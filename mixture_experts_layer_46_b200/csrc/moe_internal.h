@@ -63,6 +63,13 @@ struct AlignTiles {
   AlignTileList list[2];  // [0]: the GEMMs' tiles, [1]: 256-row tiles for the pair GEMM2
 };
 
+// align and the bf16 permute in one launch, for 1..32 routing slots (decode)
+cudaError_t launch_align_permute_tiny(const View2& ids, int64_t T, int64_t k, int64_t E, int32_t bm,
+                                      int32_t* counts, int32_t* offsets, int32_t* sorted,
+                                      int32_t* inv, int32_t* block_expert, int32_t* num_blocks,
+                                      DeviceErrors* err, const AlignTiles* tiles, const View2& x,
+                                      int64_t H, __nv_bfloat16* a1, cudaStream_t st, int* launches);
+
 // align: ids -> counts, offsets, sorted, block_expert, num_blocks (+ tile list)
 cudaError_t launch_align(const View2& ids, int64_t T, int64_t k, int64_t E, int32_t bm,
                          int32_t* counts, int32_t* offsets, int32_t* sorted, int32_t* inv,
@@ -102,6 +109,10 @@ struct WsGemm {
   int64_t k;
   int32_t weights_evict_first;  // L2 policy of the weight loads (tokens: evict-last)
   int32_t tok_box;              // rows per token-tile TMA box of the x map (tile rows per CTA: one box)
+  // GEMM1 on 32-row tiles with at most 32 routing slots: the routing ids, from
+  // which each CTA finds its first expert before align has finished (pre_S = 0: off)
+  View2 pre_ids;
+  int32_t pre_E, pre_S;
   DeviceErrors* err;
 };
 // mode 0: GEMM1 (gate/up + SwiGLU -> h), mode 1: GEMM2 (down + routing weight -> y)

@@ -23,8 +23,10 @@ __device__ __forceinline__ float bf16_to_f(uint16_t b) { return __uint_as_float(
 __global__ void __launch_bounds__(256) permute_bf16_kernel(View2 x, int64_t T, int64_t H, int64_t k,
                                                            const int32_t* __restrict__ inv,
                                                            __nv_bfloat16* __restrict__ a1, int vec_ok) {
-  pdl_wait();
+  // dependents may start before align is done (the GEMM requests weights
+  // meanwhile); everything here still waits for align
   pdl_launch_dependents();
+  pdl_wait();
   const int64_t H8 = H / 8;
   {
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {

@@ -314,3 +314,63 @@ def test_token_tile_configs_agree_and_match_oracle(T, H, I, E, k, monkeypatch):
     assert torch.equal(outs["128"], outs["256"])
     assert torch.equal(outs["128"], outs["128/two-slice"])
     assert torch.equal(outs["128"], outs["128/gemm1-128"])
+
+
+@pytest.mark.parametrize("T,k,idt", [(1, 8, torch.int32), (4, 8, torch.int64), (3, 10, torch.int32)])
+def test_decode_weight_prefetch_matches_oracle_and_unprefetched(T, k, idt, monkeypatch):
+    # at most 32 slots: GEMM1 finds its experts from the routing ids and requests
+    # weights before align has run; results must not depend on it
+    H, I, E = 512, 384, 16
+    case = make_case(T, H, I, E, k, seed=T + 97)
+    case["ids"] = case["ids"].to(idt)
+    case["ids"][0, 1] = E            # skipped slot
+    case["ids"][T - 1, 2] = case["ids"][T - 1, 3]  # one expert twice for a token
+    ref = run_oracle(case)
+    c = to_cuda(case)
+    moe.device_errors()
+    outs = {}
+    for pre in ("1", "0"):
+        monkeypatch.setenv("MOE_PREFETCH", pre)
+        outs[pre] = run_gpu(c)
+    nbad, nto = moe.device_errors()
+    assert nbad == 2 and nto == 0
+    assert torch.equal(outs["1"], outs["0"])
+    assert rel_err(outs["1"], ref) <= BF16_TOL
+
+
+@pytest.mark.parametrize("T,k,idt,tile,strided", [
+    (1, 8, torch.int32, None, False),      # decode
+    (4, 8, torch.int64, None, False),      # 32 slots, the largest one-launch batch
+    (3, 10, torch.int32, None, True),      # strided x and ids
+    (2, 8, torch.int32, "128", False),     # 128-row token tiles
+    (3, 11, torch.int32, None, False),     # 33 slots: align + permute kernels either way
+])
+def test_decode_align_permute_one_launch_matches_two(T, k, idt, tile, strided, monkeypatch):
+    # at most 32 routing slots: align and permute run as one launch that groups
+    # the slots with warp ballots; it must give the general kernels' bits
+    H, I, E = 512, 384, 24
+    case = make_case(T, H, I, E, k, seed=T + 131)
+    case["ids"] = case["ids"].to(idt)
+    case["ids"][0, 1] = -1                          # skipped slot
+    case["ids"][T - 1, 2] = case["ids"][T - 1, 3]   # one expert twice for a token
+    ref = run_oracle(case)
+    c = to_cuda(case)
+    if strided:
+        c["x"] = case["x"].t().contiguous().cuda().t()
+        big = torch.zeros(T, 3, k, dtype=idt, device="cuda")
+        big[:, 1, :] = c["ids"]
+        c["ids"] = big[:, 1, :]
+    if tile:
+        monkeypatch.setenv("MOE_TILE", tile)
+    moe.device_errors()
+    outs, launches = {}, {}
+    for tiny in ("1", "0"):
+        monkeypatch.setenv("MOE_TINY", tiny)
+        outs[tiny] = run_gpu(c)
+        launches[tiny] = moe.last_launch_count()
+    nbad, nto = moe.device_errors()
+    assert nbad == 2 and nto == 0
+    assert torch.equal(outs["1"], outs["0"])
+    assert rel_err(outs["1"], ref) <= BF16_TOL
+    assert launches["0"] == 5
+    assert launches["1"] == (4 if T * k <= 32 else 5)
