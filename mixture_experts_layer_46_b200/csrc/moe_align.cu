@@ -19,6 +19,7 @@
 // block-wide barriers.
 #include "../../include/moe.h"
 #include "moe_internal.h"
+#include "moe_mx.cuh"
 
 namespace moe {
 namespace {
@@ -361,19 +362,22 @@ __global__ void __launch_bounds__(256) align_scatter_kernel(View2 ids, int64_t T
   }
 }
 
-// Decode batches (at most 32 slots, one CTA per token): align and the bf16
-// permute in one kernel.  Warp 0 of every CTA groups the slots by expert with
+// Decode batches (at most 32 slots, one CTA per token): align and permute in
+// one kernel.  Warp 0 of every CTA groups the slots by expert with
 // match/ballot instead of a histogram over all E experts: for a slot routed
 // to expert e, its row is the padded rows of the routed experts below e plus
 // its rank among the earlier slots of e.  CTA 0 writes align's outputs (the
 // same values as the general kernels); every CTA copies its token's x row to
-// the token's rows of a1.
+// the token's rows of a1 (kQuant: quantised to MXFP4 once, codes and scales
+// written to each row, with the slot's routing weight in w_row, as permute_quant).
 constexpr int kTinyThreads = 256;
 
+template <bool kQuant>
 __global__ void __launch_bounds__(kTinyThreads) align_permute_tiny_kernel(
     View2 ids, int64_t T, int64_t k, int64_t E, int32_t bm, int32_t* counts, int32_t* offsets,
     int32_t* sorted, int32_t* inv, int32_t* block_expert, int32_t* num_blocks, TileOut to,
-    DeviceErrors* err, View2 x, int64_t H, __nv_bfloat16* a1, int vec_ok) {
+    DeviceErrors* err, View2 x, int64_t H, void* a1, uint8_t* a1_scales, View2 topk_w,
+    float* w_row, int vec_ok) {
   __shared__ int d_e[33], d_cnt[32], d_off[33], pos_sh[32];
   __shared__ int nd_sh;
   pdl_launch_dependents();
@@ -473,6 +477,44 @@ __global__ void __launch_bounds__(kTinyThreads) align_permute_tiny_kernel(
   }
   // this CTA's token: its x row to the rows of its valid slots
   const int64_t t = blockIdx.x;
+  if (kQuant) {
+    if (threadIdx.x < k && pos_sh[t * k + threadIdx.x] >= 0)
+      w_row[pos_sh[t * k + threadIdx.x]] =
+          static_cast<const float*>(topk_w.data)[t * topk_w.s0 + threadIdx.x * topk_w.s1];
+    const int64_t nb = H / 32;
+    uint8_t* codes = static_cast<uint8_t*>(a1);
+    for (int64_t b = threadIdx.x; b < nb; b += blockDim.x) {
+      float v[32];
+      if (vec_ok) {
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x.data) + t * x.s0 + b * 32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 u = __ldg(src + q);
+          const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            v[q * 8 + 2 * i] = __uint_as_float((w4[i] & 0xffffu) << 16);
+            v[q * 8 + 2 * i + 1] = __uint_as_float(w4[i] & 0xffff0000u);
+          }
+        }
+      } else {
+        const uint16_t* src = static_cast<const uint16_t*>(x.data) + t * x.s0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(static_cast<uint32_t>(src[(b * 32 + i) * x.s1]) << 16);
+      }
+      uint32_t wq[4];
+      const uint32_t sc = mx_quant32(v, wq);
+      for (int j = 0; j < k; ++j) {
+        const int p = pos_sh[t * k + j];
+        if (p < 0) continue;
+        *reinterpret_cast<uint4*>(codes + static_cast<int64_t>(p) * (H / 2) + b * 16) =
+            make_uint4(wq[0], wq[1], wq[2], wq[3]);
+        a1_scales[static_cast<int64_t>(p) * nb + b] = static_cast<uint8_t>(sc);
+      }
+    }
+    return;
+  }
+  __nv_bfloat16* a1b = static_cast<__nv_bfloat16*>(a1);
   const int64_t H8 = H / 8;
   if (vec_ok) {
     const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x.data) + t * x.s0);
@@ -480,7 +522,7 @@ __global__ void __launch_bounds__(kTinyThreads) align_permute_tiny_kernel(
       const uint4 v = __ldg(src + c);
       for (int j = 0; j < k; ++j) {
         const int p = pos_sh[t * k + j];
-        if (p >= 0) reinterpret_cast<uint4*>(a1 + static_cast<int64_t>(p) * H)[c] = v;
+        if (p >= 0) reinterpret_cast<uint4*>(a1b + static_cast<int64_t>(p) * H)[c] = v;
       }
     }
   } else {
@@ -489,7 +531,7 @@ __global__ void __launch_bounds__(kTinyThreads) align_permute_tiny_kernel(
       const uint16_t v = src[h * x.s1];
       for (int j = 0; j < k; ++j) {
         const int p = pos_sh[t * k + j];
-        if (p >= 0) reinterpret_cast<uint16_t*>(a1 + static_cast<int64_t>(p) * H)[h] = v;
+        if (p >= 0) reinterpret_cast<uint16_t*>(a1b + static_cast<int64_t>(p) * H)[h] = v;
       }
     }
   }
@@ -551,8 +593,11 @@ cudaError_t launch_align_permute_tiny(const View2& ids, int64_t T, int64_t k, in
                                       int32_t* counts, int32_t* offsets, int32_t* sorted,
                                       int32_t* inv, int32_t* block_expert, int32_t* num_blocks,
                                       DeviceErrors* err, const AlignTiles* tiles, const View2& x,
-                                      int64_t H, __nv_bfloat16* a1, cudaStream_t st, int* launches) {
+                                      int64_t H, void* a1, uint8_t* a1_scales, const View2* topk_w,
+                                      float* w_row, cudaStream_t st, int* launches) {
   if (T * k > 32 || T * k < 1) return cudaErrorInvalidValue;
+  const bool quant = a1_scales != nullptr;
+  if (quant && (topk_w == nullptr || w_row == nullptr || k > kMaxTopK)) return cudaErrorInvalidValue;
   TileOut to;
   for (int li = 0; li < 2; ++li) {
     TileList& tl = to.list[li];
@@ -565,9 +610,14 @@ cudaError_t launch_align_permute_tiny(const View2& ids, int64_t T, int64_t k, in
   const int vec_ok = (x.s1 == 1) && ((x.s0 * 2) % 16 == 0) &&
                      (reinterpret_cast<uintptr_t>(x.data) % 16 == 0);
   if (launches) *launches += 1;
-  return launch_pdl(align_permute_tiny_kernel, dim3(static_cast<unsigned>(T)), dim3(kTinyThreads), 0,
-                    st, ids, T, k, E, bm, counts, offsets, sorted, inv, block_expert, num_blocks, to,
-                    err, x, H, a1, vec_ok);
+  const View2 tw = topk_w ? *topk_w : View2{nullptr, 0, 0, 0};
+  if (quant)
+    return launch_pdl(align_permute_tiny_kernel<true>, dim3(static_cast<unsigned>(T)), dim3(kTinyThreads),
+                      0, st, ids, T, k, E, bm, counts, offsets, sorted, inv, block_expert, num_blocks,
+                      to, err, x, H, a1, a1_scales, tw, w_row, vec_ok);
+  return launch_pdl(align_permute_tiny_kernel<false>, dim3(static_cast<unsigned>(T)), dim3(kTinyThreads),
+                    0, st, ids, T, k, E, bm, counts, offsets, sorted, inv, block_expert, num_blocks,
+                    to, err, x, H, a1, a1_scales, tw, w_row, vec_ok);
 }
 
 }  // namespace moe

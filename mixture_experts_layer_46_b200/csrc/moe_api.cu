@@ -465,14 +465,28 @@ moe_status_t forward_mxfp4(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   t_prof.n = 0;
   t_prof.have = false;
   prof_mark(st);
-  cudaError_t rc = launch_align(view2(ids), pr.T, pr.k, pr.E, L.bm, counts, offsets, sorted, inv,
-                                block_expert, num_blocks, chunk_counts, L.n_chunks, dev->errors,
-                                st, &launches, &tiles);
-  if (rc != cudaSuccess) return cuda_fail(rc, "align");
-  prof_mark(st);
-  rc = launch_permute_quant(view2(x), pr.T, pr.H, pr.k, inv, w + L.a1, w + L.a1_scale, view2(wts),
-                            reinterpret_cast<float*>(w + L.w_row), st, &launches);
-  if (rc != cudaSuccess) return cuda_fail(rc, "permute_quant");
+  cudaError_t rc;
+  // decode sizes (at most 32 slots): align and the quantising permute in one
+  // launch (MOE_TINY=0 keeps the two kernels, tuning)
+  const bool tiny = L.S <= 32 && !(getenv("MOE_TINY") && atoi(getenv("MOE_TINY")) == 0);
+  if (tiny) {
+    const View2 tw = view2(wts);
+    rc = launch_align_permute_tiny(view2(ids), pr.T, pr.k, pr.E, L.bm, counts, offsets, sorted, inv,
+                                   block_expert, num_blocks, dev->errors, &tiles, view2(x), pr.H,
+                                   w + L.a1, w + L.a1_scale, &tw,
+                                   reinterpret_cast<float*>(w + L.w_row), st, &launches);
+    if (rc != cudaSuccess) return cuda_fail(rc, "align_permute_quant");
+    prof_mark(st);
+  } else {
+    rc = launch_align(view2(ids), pr.T, pr.k, pr.E, L.bm, counts, offsets, sorted, inv,
+                      block_expert, num_blocks, chunk_counts, L.n_chunks, dev->errors,
+                      st, &launches, &tiles);
+    if (rc != cudaSuccess) return cuda_fail(rc, "align");
+    prof_mark(st);
+    rc = launch_permute_quant(view2(x), pr.T, pr.H, pr.k, inv, w + L.a1, w + L.a1_scale, view2(wts),
+                              reinterpret_cast<float*>(w + L.w_row), st, &launches);
+    if (rc != cudaSuccess) return cuda_fail(rc, "permute_quant");
+  }
   prof_mark(st);
   WsGemmMx g1;
   std::memset(&g1, 0, sizeof(g1));
@@ -578,7 +592,6 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   uint32_t tok_box = pair ? static_cast<uint32_t>(L.tile_max / 2) : static_cast<uint32_t>(L.tile_max);
   if (const char* env = getenv("MOE_TOKBOX"))
     if (atoi(env) == 0) tok_box = pair ? 16u : 32u;
-  const uint32_t boxt[2] = {64, tok_box};
   // GEMM2 on CTA pairs: one 256-row w2 slice per work item over 256-row token
   // tiles (align's second list), which keeps two accumulator buffers in TMEM
   // and stages 32 KiB per k-block.  MOE_G2=1 selects two 256-row slices over
@@ -653,7 +666,7 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   if (tiny) {
     rc = launch_align_permute_tiny(view2(ids), pr.T, pr.k, pr.E, bm, counts, offsets, sorted, inv,
                                    block_expert, num_blocks, dev->errors, &tiles, view2(x), pr.H,
-                                   reinterpret_cast<__nv_bfloat16*>(w + L.a1), st, &launches);
+                                   w + L.a1, nullptr, nullptr, nullptr, st, &launches);
     if (rc != cudaSuccess) return cuda_fail(rc, "align_permute");
     prof_mark(st);
   } else {

@@ -63,12 +63,15 @@ struct AlignTiles {
   AlignTileList list[2];  // [0]: the GEMMs' tiles, [1]: 256-row tiles for the pair GEMM2
 };
 
-// align and the bf16 permute in one launch, for 1..32 routing slots (decode)
+// align and permute in one launch, for 1..32 routing slots (decode).  a1 is
+// bf16 rows, or MXFP4 codes when a1_scales is given (then topk_w and w_row as
+// in launch_permute_quant)
 cudaError_t launch_align_permute_tiny(const View2& ids, int64_t T, int64_t k, int64_t E, int32_t bm,
                                       int32_t* counts, int32_t* offsets, int32_t* sorted,
                                       int32_t* inv, int32_t* block_expert, int32_t* num_blocks,
                                       DeviceErrors* err, const AlignTiles* tiles, const View2& x,
-                                      int64_t H, __nv_bfloat16* a1, cudaStream_t st, int* launches);
+                                      int64_t H, void* a1, uint8_t* a1_scales, const View2* topk_w,
+                                      float* w_row, cudaStream_t st, int* launches);
 
 // align: ids -> counts, offsets, sorted, block_expert, num_blocks (+ tile list)
 cudaError_t launch_align(const View2& ids, int64_t T, int64_t k, int64_t E, int32_t bm,

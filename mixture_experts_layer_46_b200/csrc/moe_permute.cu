@@ -72,8 +72,9 @@ __global__ void __launch_bounds__(128) permute_quant_kernel(View2 x, int64_t T, 
                                                             const int32_t* inv, uint8_t* codes,
                                                             uint8_t* scales, View2 topk_w,
                                                             float* w_row, int vec_ok) {
-  pdl_wait();
+  // dependents may be scheduled at once; everything here still waits for align
   pdl_launch_dependents();
+  pdl_wait();
   const int64_t nb = H / 32;  // blocks per row
   {
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
