@@ -53,10 +53,10 @@ WORKLOADS = {
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed to the hash of the kernel
 # source it was taken on; reported as null once the source has changed.
 NCU_TRAFFIC = {
-    # profiles/gemm_ws_pair_bf16_qwen3shape_E32_T1024.md: 941.1 MB read + 26.4 MB written by
+    # profiles/gemm_ws_pair_bf16_qwen3shape_E32_T1024.md: 941.5 MB read + 27.0 MB written by
     # GEMM1 (256-row token tiles) on the E=32, T=1024 case (~256 slots per expert), scaled x4
     # (experts and tokens) to the E=128, T=4096 launch; keyed to the kernel and host sources
-    "gemm1_swiglu": {"bytes_per_launch": 4.0 * (941.06368e6 + 26.39104e6), "src": "51397945960f1598",
+    "gemm1_swiglu": {"bytes_per_launch": 4.0 * (941.518848e6 + 27.002624e6), "src": "f14ab1f4b1a712fd",
                      "workload": "qwen3-235b T=4096"},
 }
 
