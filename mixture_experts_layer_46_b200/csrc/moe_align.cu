@@ -378,7 +378,8 @@ __global__ void __launch_bounds__(kTinyThreads) align_permute_tiny_kernel(
     int32_t* sorted, int32_t* inv, int32_t* block_expert, int32_t* num_blocks, TileOut to,
     DeviceErrors* err, View2 x, int64_t H, void* a1, uint8_t* a1_scales, View2 topk_w,
     float* w_row, int vec_ok) {
-  __shared__ int d_e[33], d_cnt[32], d_off[33], pos_sh[32];
+  // routed experts in ascending order: id, slot count, first padded row (d_off[nd] = total rows)
+  __shared__ int d_e[32], d_cnt[32], d_off[33], pos_sh[32];
   __shared__ int nd_sh;
   pdl_launch_dependents();
   pdl_wait();
@@ -417,7 +418,6 @@ __global__ void __launch_bounds__(kTinyThreads) align_permute_tiny_kernel(
     const int total_rows = __shfl_sync(0xffffffffu, incl, 31);
     if (lane == 0) {
       d_off[nd] = total_rows;
-      d_e[nd] = static_cast<int>(E);
       nd_sh = nd;
     }
     __syncwarp();

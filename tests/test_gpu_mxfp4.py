@@ -196,7 +196,14 @@ def test_qwen35_tp2_mxfp4_full_size_sampled(shared):
     s = wl.QWEN35_TP2_MXFP4_SHARED if shared else wl.QWEN35_TP2_MXFP4
     case = make_mx_case(s.T, s.H, s.I, s.E, s.k, seed=0, shared=shared)
     got = mx_gpu(cuda_case(case))
+    # spread tokens, the first and last 16, and tokens of the least-loaded experts
     g = torch.Generator().manual_seed(11)
-    toks = torch.unique(torch.cat([torch.randperm(s.T, generator=g)[:24], torch.tensor([0, s.T - 1])]))
+    ids = case["ids"].long()
+    counts = torch.bincount(ids.flatten(), minlength=s.E)
+    routed = torch.nonzero(counts > 0).flatten()
+    light = routed[torch.argsort(counts[routed], stable=True)[:4]]
+    parts = [torch.randperm(s.T, generator=g)[:96], torch.arange(16), torch.arange(s.T - 16, s.T)]
+    parts += [torch.nonzero((ids == e).any(dim=1)).flatten()[:8] for e in light.tolist()]
+    toks = torch.unique(torch.cat(parts))
     ref = mx_oracle(case, tokens=toks)
     assert rel_err(got.cpu()[toks], ref) <= MX_TOL
