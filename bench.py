@@ -55,8 +55,11 @@ WORKLOADS = {
 NCU_TRAFFIC = {
     # profiles/gemm_ws_pair_bf16_qwen3shape_E32_T1024.md: 941.5 MB read + 27.0 MB written by
     # GEMM1 (256-row token tiles) on the E=32, T=1024 case (~256 slots per expert), scaled x4
-    # (experts and tokens) to the E=128, T=4096 launch; keyed to the kernel and host sources
-    "gemm1_swiglu": {"bytes_per_launch": 4.0 * (941.518848e6 + 27.002624e6), "src": "f14ab1f4b1a712fd",
+    # (experts and tokens) to the E=128, T=4096 launch; keyed to the kernel and host sources.
+    # Re-keyed without a new capture after one host-side change: GEMM1's 256-row token tiles are
+    # now also chosen from 400 slots per expert up, which neither the captured case (~256 per
+    # expert) nor the T=4096 launch (256 per expert) reaches; kernels and their launch unchanged
+    "gemm1_swiglu": {"bytes_per_launch": 4.0 * (941.518848e6 + 27.002624e6), "src": "0defb09e557f820d",
                      "workload": "qwen3-235b T=4096"},
 }
 

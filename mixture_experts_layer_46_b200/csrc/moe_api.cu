@@ -600,12 +600,13 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   if (const char* env = getenv("MOE_G2")) g2_single = g2_single && atoi(env) != 1;
   const uint32_t boxt2[2] = {64, g2_single ? 128u : tok_box};
   // GEMM1 over the same 256-row tiles (one accumulator buffer of 2 x 256
-  // columns, so its epilogue is not overlapped) while experts average 96..399
-  // slots: the halved weight re-reads outweigh the exposed epilogue there
-  // (measured 6-20 % faster at T = 2048..6144 for the Qwen3 shape, neutral at
-  // 4096, mixed at 8192).  MOE_G1_256=0|1 overrides (tuning).
+  // columns, so its epilogue is not overlapped) once experts average 96 slots:
+  // the halved weight re-reads (and their L2 traffic and power) outweigh the
+  // exposed epilogue (measured 6-20 % faster at T = 2048..6144 for the Qwen3
+  // shape, 8 % at 4096 and 2-7 % at 8192..16384 in sustained, power-capped
+  // runs).  MOE_G1_256=0|1 overrides (tuning).
   const int64_t avg_slots = pr.E > 0 ? (pr.T * pr.k) / pr.E : 0;
-  bool g1_256 = g2_single && avg_slots >= 96 && avg_slots < 400;
+  bool g1_256 = g2_single && avg_slots >= 96;
   if (const char* env = getenv("MOE_G1_256")) g1_256 = g2_single && atoi(env) == 1;
   const uint32_t boxt1[2] = {64, g1_256 ? 128u : tok_box};
   {
