@@ -284,6 +284,39 @@ def run_reference(args, w, rank):
     print(json.dumps(line), flush=True)
 
 
+def init_replicas(world: int, local: int, backend: str = "nccl") -> bool:
+    """Process group of the N independent replicas (torchrun env: RANK, WORLD_SIZE, MASTER_*):
+    NCCL on the GPUs, gloo in the CPU tests.  The short timeout turns a rank that never arrives
+    into an error on the others instead of a hang."""
+    if world <= 1:
+        return False
+    import datetime
+
+    import torch.distributed as dist
+
+    kw = {}
+    if backend == "nccl":
+        torch.cuda.set_device(local)
+        kw["device_id"] = torch.device("cuda", local)
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+    return True
+
+
+def max_over_ranks(x: float, pg: bool, device) -> float:
+    """The slowest replica's figure; every rank calls it at the same point of the run."""
+    if not pg:
+        return x
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(world: int, tokens_per_rank: int, ms: float) -> float:
+    """Whole-job tokens/s: each of the `world` replicas runs its own batch of tokens_per_rank
+    tokens, and the job takes the slowest replica's ms (weak scaling)."""
+    return world * tokens_per_rank / (ms * 1e-3)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -307,16 +340,7 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    pg = False
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-        pg = True
+    pg = init_replicas(world, local)
 
     if args.impl == "reference":
         run_reference(args, w, rank)
@@ -368,12 +392,8 @@ def main():
         torch.distributed.barrier()
     clocks = sampler.stop()
     per = [a.elapsed_time(b) for a, b in evs]
-    ms = sum(per) / len(per)
-    if pg:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    value = world * w["T"] / (ms * 1e-3)
+    ms = max_over_ranks(sum(per) / len(per), pg, dev)
+    value = replica_throughput(world, w["T"], ms)
 
     # ---------------------------------------------------------------- per-step breakdown
     moe.profile_enable(True)
@@ -402,11 +422,7 @@ def main():
         e1.record(stream)
         e1.synchronize()
         e2e_ms.append(e0.elapsed_time(e1))
-    e2e = sum(e2e_ms) / len(e2e_ms)
-    if pg:
-        t = torch.tensor([e2e], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e = float(t.item())
+    e2e = max_over_ranks(sum(e2e_ms) / len(e2e_ms), pg, dev)
     h2d = x_h.numel() * 2 + ids_h.numel() * ids_h.element_size() + w_h.numel() * 4
     d2h = out_h.numel() * 2
 
@@ -456,7 +472,7 @@ def main():
                                "flops": alg["flops"], "bytes": alg["bytes"],
                                "active_experts": alg["active_experts"]},
             "step_breakdown_ms": brk,
-            "e2e": {"value": world * w["T"] / (e2e * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "e2e": {"value": replica_throughput(world, w["T"], e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e,
                     "api": "moe_forward_host (pinned host x/ids/weights in, host out)"},
             "gpu_launches": launches_per_step * args.steps,
