@@ -196,7 +196,8 @@ moe_status_t moe_quantize_mxfp4(const moe_tensor_t* src, moe_tensor_t* dst, moe_
 moe_status_t moe_get_device_errors(moe_stream_t stream, uint32_t* n_bad_ids, uint32_t* timeouts);
 
 /* Number of kernels the last moe_forward_ws / moe_forward call on this thread
- * enqueued (for launch accounting). */
+ * enqueued (for launch accounting): 4 with at most 32 routing slots, else 5,
+ * plus 2 when align runs its multi-CTA form (more than 4096 slots). */
 int32_t moe_last_launch_count(void);
 
 /* Per-kernel timing for profiling.  While enabled on the calling thread, each
@@ -205,7 +206,9 @@ int32_t moe_last_launch_count(void);
  * the steps (no overlap between neighbouring kernels), so time the end-to-end
  * call with profiling off.  moe_profile_read synchronises on the last event and
  * writes up to `capacity` step durations in milliseconds, in that order, for
- * the last profiled call; *n receives the number of steps. */
+ * the last profiled call; *n receives the number of steps.  With at most 32
+ * routing slots align and permute are one kernel: its time is reported as
+ * align's and permute's duration is zero. */
 moe_status_t moe_profile_enable(int32_t on);
 moe_status_t moe_profile_read(float* ms, int32_t capacity, int32_t* n);
 
