@@ -87,7 +87,10 @@ typedef enum {
   MOE_ERR_DEVICE_TIMEOUT = 8      /* a kernel's bounded wait expired (see moe_get_device_errors) */
 } moe_status_t;
 
-/* Human-readable name of a status code (static string, never NULL). */
+/* Human-readable name of a status code (static string, never NULL).  Every
+ * failure is reported by name rather than silently worked around, the rule the
+ * Liger-Kernel PR #1377 discussion sets for layouts the kernel cannot read
+ * ("Testing Done": a mismatched gate hidden dimension fails loudly). */
 const char* moe_status_string(moe_status_t st);
 
 /* The last CUDA error string seen by the calling thread (static storage). */
@@ -130,9 +133,14 @@ moe_status_t moe_forward_ws(const moe_tensor_t* x, const moe_w13_t* w13, const m
                             moe_tensor_t* out, void* workspace, size_t workspace_bytes,
                             moe_stream_t stream);
 
-/* Same as moe_forward_ws with a library-owned workspace: one buffer per device,
- * grown with cudaMalloc when a call needs more (growth synchronises the device,
- * so size it once with a first call outside any stream capture). */
+/* The forward as the pages state the problem: moe_forward(x, w13, w2,
+ * topk_ids, topk_weights, out, stream), with w13 the gate/up views of the
+ * packed [E, 2I, H] tensor (Liger-Kernel PR #1377, "Problems": the fused MoE
+ * kernel reads the packed expert weights through strided views instead of a
+ * retained contiguous copy).  Arguments as for moe_forward_ws; the workspace is
+ * library-owned: one buffer per device, grown with cudaMalloc when a call needs
+ * more (growth synchronises the device, so size it once with a first call
+ * outside any stream capture). */
 moe_status_t moe_forward(const moe_tensor_t* x, const moe_w13_t* w13, const moe_tensor_t* w2,
                          const moe_tensor_t* topk_ids, const moe_tensor_t* topk_weights,
                          moe_tensor_t* out, moe_stream_t stream);
@@ -147,7 +155,10 @@ moe_status_t moe_forward_host(const moe_tensor_t* x_host, const moe_w13_t* w13,
                               const moe_tensor_t* topk_weights_host, moe_tensor_t* out_host,
                               moe_stream_t stream);
 
-/* Step "align" alone, for inspection and tests: group the T*k slots by expert.
+/* Step "align" alone, for inspection and tests: group the T*k slots by expert
+ * into block_m-row blocks, block_m being the per-token-bucket block size the
+ * aiter kernels tune (ROCm/aiter PR #3859, "Tuned MoE latency": block_m 32, 64
+ * or 128 by token count).
  *   counts[e]        number of valid slots routed to expert e          int32 [E]
  *   offsets[e]       exclusive prefix sum of ceil(counts/block_m)*block_m int32 [E+1]
  *   sorted_slots[p]  slot ids grouped by expert, ascending within an expert;
@@ -191,8 +202,13 @@ moe_status_t moe_align_noalloc(const moe_tensor_t* topk_ids, int64_t E, int32_t 
 moe_status_t moe_quantize_mxfp4(const moe_tensor_t* src, moe_tensor_t* dst, moe_stream_t stream);
 
 /* Reads and clears the device error counters of the current device:
- * *n_bad_ids = slots skipped because their id was outside [0, E);
- * *timeouts = kernel waits that gave up.  Synchronises `stream`. */
+ * *n_bad_ids = slots skipped because their id was outside [0, E) (a routing
+ * replay slice read with the wrong stride produces such ids, prime-rl PR #2860,
+ * "Problem"; they are counted instead of being read out of bounds);
+ * *timeouts = kernel waits that gave up (every wait in the kernels is bounded,
+ * so a missing arrival ends the kernel with this count instead of a hang).
+ * Synchronises `stream`.  Returns MOE_ERR_DEVICE_TIMEOUT when *timeouts > 0
+ * (both counters are still written), else MOE_OK. */
 moe_status_t moe_get_device_errors(moe_stream_t stream, uint32_t* n_bad_ids, uint32_t* timeouts);
 
 /* Number of kernels the last moe_forward_ws / moe_forward call on this thread
@@ -211,6 +227,44 @@ int32_t moe_last_launch_count(void);
  * align's and permute's duration is zero. */
 moe_status_t moe_profile_enable(int32_t on);
 moe_status_t moe_profile_read(float* ms, int32_t capacity, int32_t* n);
+
+/* ---- kernel configuration (per-shape tuning table) ----------------------
+ * Which token-tile size and GEMM variant the forward runs for a problem.  The
+ * pages keep tuned kernel choices in a table keyed by shape and token count
+ * (ROCm/aiter PR #3859, "Details": tuned configurations per shape; "Tuned MoE
+ * latency": block_m per token bucket).  A forward looks its configuration up
+ * in the table installed by moe_set_config_table, then in the table compiled
+ * into the library from the committed tuning results, then falls back to a
+ * heuristic.  Every configuration gives bit-identical results; only the speed
+ * differs.  The workspace size (moe_workspace_bytes) does not depend on it. */
+typedef struct {
+  int32_t wdtype;      /* MOE_BF16 or MOE_E2M1X2 */
+  int64_t H, I, E, k;  /* shape the entry applies to; 0 matches any value */
+  int64_t t_lo, t_hi;  /* token bucket: applies when t_lo <= T <= t_hi */
+  int32_t tile;        /* token-tile rows: 32, 128 or 256 (bf16; 256 runs on CTA pairs),
+                          32 or 96 (MXFP4) */
+  int32_t pair;        /* bf16 128-row tiles: GEMMs on CTA pairs (tcgen05 cta_group::2) */
+  int32_t g1_256;      /* bf16 pairs: GEMM1 on 256-row token tiles (needs g2_single) */
+  int32_t g2_single;   /* bf16 pairs: GEMM2 with one 256-row w2 slice per 256-row tile */
+  int32_t tiny;        /* at most 32 slots: align and permute in one launch */
+  int32_t prefetch;    /* at most 32 slots, 32-row tiles: GEMM1 requests its first weight
+                          stages before align has finished (checked against align after) */
+} moe_config_t;
+
+/* Installs a process-wide configuration table (copied; n = 0 removes it).
+ * Entries are tried in order; flags that do not apply to an entry's tile are
+ * ignored.  Errors: MOE_ERR_INVALID_ARG for a malformed entry (nothing is
+ * installed then).  Not synchronised with forwards already running on other
+ * host threads: install it before them. */
+moe_status_t moe_set_config_table(const moe_config_t* entries, int32_t n);
+
+/* The configuration a forward of this problem would use (after the rules
+ * above), in *out.  Errors: MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_DTYPE. */
+moe_status_t moe_get_config(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, int32_t wdtype,
+                            moe_config_t* out);
+
+/* Number of entries of the table compiled into the library. */
+int32_t moe_builtin_config_count(void);
 
 /* Library version string. */
 const char* moe_version(void);

@@ -6,7 +6,8 @@ package does not load the library; the first call does, and raises if the
 library was not built (there is no CPU fallback).
 """
 
-from ._abi import (MoeError, MoeTensor, MoeW13, align, desc, device_errors, forward,  # noqa: F401
-                   forward_host, forward_status, last_launch_count, load, profile_enable,
-                   profile_read, quantize_mxfp4,
-                   version, w13_from_packed, w13_from_views, workspace_bytes)
+from ._abi import (MoeConfig, MoeError, MoeTensor, MoeW13, align, builtin_config_count,  # noqa: F401
+                   config_override, desc, device_errors, forward, forward_host, forward_status,
+                   get_config, last_launch_count, load, make_config, profile_enable, profile_read,
+                   quantize_mxfp4, set_config_table, version, w13_from_packed, w13_from_views,
+                   workspace_bytes)

@@ -27,7 +27,8 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_SHAPE_MISMATCH",
 EXPORTS = ("moe_status_string", "moe_last_cuda_error", "moe_w13_from_packed",
            "moe_workspace_bytes", "moe_forward_ws", "moe_forward", "moe_forward_host",
            "moe_align", "moe_quantize_mxfp4", "moe_get_device_errors", "moe_last_launch_count",
-           "moe_profile_enable", "moe_profile_read", "moe_version", "moe_align_noalloc")
+           "moe_profile_enable", "moe_profile_read", "moe_version", "moe_align_noalloc",
+           "moe_set_config_table", "moe_get_config", "moe_builtin_config_count")
 STEP_NAMES = ("align", "permute", "gemm1_swiglu", "gemm2_weighted", "combine")
 
 
@@ -54,6 +55,21 @@ class MoeTensor(ctypes.Structure):
 
 class MoeW13(ctypes.Structure):
     _fields_ = [("gate", MoeTensor), ("up", MoeTensor)]
+
+
+class MoeConfig(ctypes.Structure):
+    """moe_config_t: the kernel configuration of one shape and token bucket."""
+    _fields_ = [("wdtype", ctypes.c_int32), ("H", ctypes.c_int64), ("I", ctypes.c_int64),
+                ("E", ctypes.c_int64), ("k", ctypes.c_int64), ("t_lo", ctypes.c_int64),
+                ("t_hi", ctypes.c_int64), ("tile", ctypes.c_int32), ("pair", ctypes.c_int32),
+                ("g1_256", ctypes.c_int32), ("g2_single", ctypes.c_int32), ("tiny", ctypes.c_int32),
+                ("prefetch", ctypes.c_int32)]
+
+    def as_dict(self) -> dict:
+        return {name: int(getattr(self, name)) for name, _ in self._fields_}
+
+
+CONFIG_FLAGS = ("tile", "pair", "g1_256", "g2_single", "tiny", "prefetch")
 
 
 _lock = threading.Lock()
@@ -98,6 +114,11 @@ def load() -> ctypes.CDLL:
             lib.moe_align_noalloc.restype = ctypes.c_int
             lib.moe_align_noalloc.argtypes = [P(MoeTensor), ctypes.c_int64, ctypes.c_int32, vp, vp,
                                               vp, vp, vp, vp]
+            lib.moe_set_config_table.restype = ctypes.c_int
+            lib.moe_set_config_table.argtypes = [P(MoeConfig), ctypes.c_int32]
+            lib.moe_get_config.restype = ctypes.c_int
+            lib.moe_get_config.argtypes = [ctypes.c_int64] * 5 + [ctypes.c_int32, P(MoeConfig)]
+            lib.moe_builtin_config_count.restype = ctypes.c_int32
             lib.moe_profile_enable.restype = ctypes.c_int
             lib.moe_profile_enable.argtypes = [ctypes.c_int32]
             lib.moe_profile_read.restype = ctypes.c_int
@@ -256,11 +277,64 @@ def quantize_mxfp4(src: torch.Tensor, *, stream=None):
 
 
 def device_errors(stream=None):
+    """(skipped out-of-range slots, kernel waits that gave up) since the last read;
+    reading clears them.  MOE_ERR_DEVICE_TIMEOUT only flags a non-zero second count."""
     nb = ctypes.c_uint32(0)
     to = ctypes.c_uint32(0)
-    _check(load().moe_get_device_errors(_stream_ptr(stream), ctypes.byref(nb), ctypes.byref(to)),
-           "moe_get_device_errors")
+    rc = load().moe_get_device_errors(_stream_ptr(stream), ctypes.byref(nb), ctypes.byref(to))
+    if rc not in (0, 8):
+        _check(rc, "moe_get_device_errors")
     return int(nb.value), int(to.value)
+
+
+def make_config(wdtype: int = MOE_BF16, H=0, I=0, E=0, k=0, t_lo=0, t_hi=1 << 40, **flags) -> MoeConfig:
+    c = MoeConfig()
+    c.wdtype, c.H, c.I, c.E, c.k, c.t_lo, c.t_hi = wdtype, H, I, E, k, t_lo, t_hi
+    for name in CONFIG_FLAGS:
+        setattr(c, name, int(flags.get(name, 0)))
+    return c
+
+
+def set_config_table(entries) -> None:
+    """Install a process-wide configuration table (a list of MoeConfig; [] removes it)."""
+    n = len(entries)
+    arr = (MoeConfig * max(n, 1))(*entries)
+    _check(load().moe_set_config_table(arr, n), "moe_set_config_table")
+
+
+def get_config(T: int, H: int, I: int, E: int, k: int, mxfp4: bool = False) -> dict:
+    """The configuration a forward of this problem uses."""
+    c = MoeConfig()
+    _check(load().moe_get_config(T, H, I, E, k, MOE_E2M1X2 if mxfp4 else MOE_BF16, ctypes.byref(c)),
+           "moe_get_config")
+    return c.as_dict()
+
+
+class config_override:
+    """Context manager: forwards of the problem (T, H, I, E, k) run the
+    configuration they would use, with the given flags changed, e.g.
+    config_override((T, H, I, E, k), tile=32) or (..., mxfp4=True, tiny=0)."""
+
+    def __init__(self, shape, mxfp4: bool = False, **flags):
+        self.shape, self.mxfp4, self.flags = tuple(shape), mxfp4, flags
+
+    def __enter__(self):
+        set_config_table([])
+        T, H, I, E, k = self.shape
+        base = get_config(T, H, I, E, k, mxfp4=self.mxfp4)
+        base.update(self.flags)
+        base.update(H=H, I=I, E=E, k=k, t_lo=T, t_hi=T)
+        wd = base.pop("wdtype")
+        set_config_table([make_config(wd, **base)])
+        return self
+
+    def __exit__(self, *exc):
+        set_config_table([])
+        return False
+
+
+def builtin_config_count() -> int:
+    return int(load().moe_builtin_config_count())
 
 
 def profile_enable(on: bool = True):

@@ -321,30 +321,13 @@ moe_status_t cached_workspace(size_t need, void** ptr) {
 
 // ---------------------------------------------------------------- layout
 
-void choose_tiling(int64_t T, int64_t k, int64_t E, bool mxfp4, int32_t* bm, int32_t* tile_max) {
-  if (mxfp4) {
-    // block-scaled weight-stationary kernels: token tiles of up to 32 or 96 rows
-    // (96 keeps both accumulator buffers and the per-stage scales inside TMEM)
-    *bm = 32;
-    const int64_t avg = E > 0 ? (T * k) / E : 0;
-    *tile_max = avg <= 8 ? 32 : 96;
-    return;
-  }
-  // weight-stationary bf16 kernels: tokens are the MMA's N side in 32-row
-  // granules, in tiles of up to 32 rows while experts average <= 8 slots
-  // (decode: 6-stage ring, more weight bytes in flight) and up to 128 rows
-  // beyond (double-buffered accumulators).  MOE_TILE overrides (tuning).
-  *bm = 32;
-  const int64_t avg = E > 0 ? (T * k) / E : 0;
-  *tile_max = avg <= 8 ? 32 : 128;
-  if (const char* env = getenv("MOE_TILE")) {
-    const int v = atoi(env);
-    if (v == 32 || v == 128 || v == 256) *tile_max = v;
-  }
-}
-
+// The workspace holds the token-tile lists of every configuration the forward
+// can choose (32-row tiles give the longest list; the second list is the
+// 256-row one of the bf16 CTA-pair GEMMs), so its size depends on the problem
+// alone and never on the configuration table.
 WsLayout make_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, bool mxfp4,
-                     int32_t bm, int32_t tile_max) {
+                     int32_t bm) {
+  const int32_t tile_max = kMinTile;
   WsLayout L;
   std::memset(&L, 0, sizeof(L));
   L.T = T;
@@ -366,7 +349,7 @@ WsLayout make_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, bool
   L.t_max = tile_max > 0 ? p / tile_max + nonempty + 1 : 0;
   // second token-tile list: 256-row tiles for the single-slice GEMM2 on CTA
   // pairs (bf16 with 128-row tiles)
-  L.tile_max2 = (!mxfp4 && tile_max == 128) ? 256 : 0;
+  L.tile_max2 = !mxfp4 ? 256 : 0;
   L.t_max2 = L.tile_max2 > 0 ? p / L.tile_max2 + nonempty + 1 : 0;
   L.n_chunks = (S + kAlignChunk - 1) / kAlignChunk;
   if (L.n_chunks < 1) L.n_chunks = 1;
@@ -412,8 +395,8 @@ namespace {
 // -> block-scaled GEMM2 (+routing weight) -> combine.
 moe_status_t forward_mxfp4(const moe_tensor_t* x, const moe_w13_t* w13, const moe_tensor_t* w2,
                            const moe_tensor_t* ids, const moe_tensor_t* wts, moe_tensor_t* out,
-                           const Problem& pr, const WsLayout& L, uint8_t* w, DeviceInfo* dev,
-                           cudaStream_t st) {
+                           const Problem& pr, const WsLayout& L, const moe_config_t& cfg,
+                           uint8_t* w, DeviceInfo* dev, cudaStream_t st) {
   int launches = 0;
   int32_t* counts = reinterpret_cast<int32_t*>(w + L.counts);
   int32_t* offsets = reinterpret_cast<int32_t*>(w + L.offsets);
@@ -457,7 +440,7 @@ moe_status_t forward_mxfp4(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   }
   AlignTiles tiles;
   std::memset(&tiles, 0, sizeof(tiles));
-  tiles.list[0].tile_max = L.tile_max;
+  tiles.list[0].tile_max = cfg.tile;
   tiles.list[0].tile_row = reinterpret_cast<int32_t*>(w + L.tile_row);
   tiles.list[0].tile_rows = reinterpret_cast<int32_t*>(w + L.tile_rows);
   tiles.list[0].tile_expert = reinterpret_cast<int32_t*>(w + L.tile_expert);
@@ -466,10 +449,8 @@ moe_status_t forward_mxfp4(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   t_prof.have = false;
   prof_mark(st);
   cudaError_t rc;
-  // decode sizes (at most 32 slots): align and the quantising permute in one
-  // launch (MOE_TINY=0 keeps the two kernels, tuning)
-  const bool tiny = L.S <= 32 && !(getenv("MOE_TINY") && atoi(getenv("MOE_TINY")) == 0);
-  if (tiny) {
+  // decode sizes (at most 32 slots): align and the quantising permute in one launch
+  if (cfg.tiny) {
     const View2 tw = view2(wts);
     rc = launch_align_permute_tiny(view2(ids), pr.T, pr.k, pr.E, L.bm, counts, offsets, sorted, inv,
                                    block_expert, num_blocks, dev->errors, &tiles, view2(x), pr.H,
@@ -514,7 +495,7 @@ moe_status_t forward_mxfp4(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   g1.w1_s0 = up->scale_strides[0];
   g1.w1_s1 = up->scale_strides[1];
   g1.err = dev->errors;
-  rc = launch_gemm_ws_mxfp4(0, L.tile_max, mGate, mUp, mA1, g1, dev->num_sms, st, &launches);
+  rc = launch_gemm_ws_mxfp4(0, cfg.tile, mGate, mUp, mA1, g1, dev->num_sms, st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm1_mxfp4");
   prof_mark(st);
   WsGemmMx g2 = g1;
@@ -535,7 +516,7 @@ moe_status_t forward_mxfp4(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   g2.w1_s0 = g2.w0_s0;
   g2.w1_s1 = g2.w0_s1;
   g2.w_row = reinterpret_cast<const float*>(w + L.w_row);
-  rc = launch_gemm_ws_mxfp4(1, L.tile_max, mW2, mW2, mH, g2, dev->num_sms, st, &launches);
+  rc = launch_gemm_ws_mxfp4(1, cfg.tile, mW2, mW2, mH, g2, dev->num_sms, st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm2_mxfp4");
   prof_mark(st);
   rc = launch_combine(reinterpret_cast<const __nv_bfloat16*>(w + L.y), inv, pr.T, pr.H, pr.k,
@@ -553,9 +534,9 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   int launches = 0;
   t_last_launches = 0;
   if (pr.T == 0) return MOE_OK;
-  int32_t bm = 0, tile_max = 0;
-  choose_tiling(pr.T, pr.k, pr.E, pr.mxfp4, &bm, &tile_max);
-  const WsLayout L = make_layout(pr.T, pr.H, pr.I, pr.E, pr.k, pr.mxfp4, bm, tile_max);
+  const int32_t bm = kBm;
+  const moe_config_t cfg = select_config(pr.T, pr.H, pr.I, pr.E, pr.k, pr.mxfp4);
+  const WsLayout L = make_layout(pr.T, pr.H, pr.I, pr.E, pr.k, pr.mxfp4, bm);
   if (!ws || ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
   if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return MOE_ERR_INVALID_ARG;
   DeviceInfo* dev = nullptr;
@@ -573,41 +554,25 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   const moe_tensor_t* gate = &w13->gate;
   const moe_tensor_t* up = &w13->up;
 
-  if (pr.mxfp4) return forward_mxfp4(x, w13, w2, ids, wts, out, pr, L, w, dev, st);
+  if (pr.mxfp4) return forward_mxfp4(x, w13, w2, ids, wts, out, pr, L, cfg, w, dev, st);
 
   // ---- tensor maps (bf16, 128-byte swizzle): weights in [64 x 128] boxes,
   // expert-grouped token rows in one box per CTA and token tile
   CUtensorMap mA1, mGate, mUp, mH, mW2;
-  // 128-row token tiles run on CTA pairs once experts average >= 32 slots (the
-  // pair moves a sixth fewer shared-memory bytes per FLOP and keeps 5 stages in
-  // flight); MOE_PAIR=0|1 and MOE_WPOLICY=1 (weights evict-first in L2) are
-  // tuning overrides
-  bool pair = (L.tile_max >= 128) && (pr.T * pr.k >= 32 * pr.E);
-  if (const char* env = getenv("MOE_PAIR")) pair = (L.tile_max >= 128) && atoi(env) != 0;
-  if (L.tile_max == 256) pair = true;  // 256-row tiles exist only on CTA pairs
-  const int32_t wpolicy = getenv("MOE_WPOLICY") ? atoi(getenv("MOE_WPOLICY")) : 0;
+  // the configuration: token-tile rows (32 / 128 on one CTA, 128 / 256 on CTA
+  // pairs, which move a sixth fewer shared-memory bytes per FLOP); GEMM2 on
+  // pairs with one 256-row w2 slice per 256-row token tile (align's second
+  // list: two accumulator buffers still fit in TMEM); GEMM1 on those 256-row
+  // tiles (halved weight re-reads against an epilogue that is not overlapped)
+  const int32_t tile = cfg.tile;
+  const bool pair = cfg.pair != 0;
+  const bool g2_single = cfg.g2_single != 0;
+  const bool g1_256 = cfg.g1_256 != 0;
+  const int32_t wpolicy = 0;
   const uint32_t boxw[3] = {64, 128, 1};
-  // one TMA box covers a CTA's share of a token tile (fewer copy operations per
-  // stage); MOE_TOKBOX=0 selects 16-row (pair) / 32-row boxes (tuning)
-  uint32_t tok_box = pair ? static_cast<uint32_t>(L.tile_max / 2) : static_cast<uint32_t>(L.tile_max);
-  if (const char* env = getenv("MOE_TOKBOX"))
-    if (atoi(env) == 0) tok_box = pair ? 16u : 32u;
-  // GEMM2 on CTA pairs: one 256-row w2 slice per work item over 256-row token
-  // tiles (align's second list), which keeps two accumulator buffers in TMEM
-  // and stages 32 KiB per k-block.  MOE_G2=1 selects two 256-row slices over
-  // the 128-row tiles (tuning).
-  bool g2_single = pair && L.tile_max == 128 && L.t_max2 > 0;
-  if (const char* env = getenv("MOE_G2")) g2_single = g2_single && atoi(env) != 1;
+  // one TMA box covers a CTA's share of a token tile
+  const uint32_t tok_box = pair ? static_cast<uint32_t>(tile / 2) : static_cast<uint32_t>(tile);
   const uint32_t boxt2[2] = {64, g2_single ? 128u : tok_box};
-  // GEMM1 over the same 256-row tiles (one accumulator buffer of 2 x 256
-  // columns, so its epilogue is not overlapped) once experts average 96 slots:
-  // the halved weight re-reads (and their L2 traffic and power) outweigh the
-  // exposed epilogue (measured 6-20 % faster at T = 2048..6144 for the Qwen3
-  // shape, 8 % at 4096 and 2-7 % at 8192..16384 in sustained, power-capped
-  // runs).  MOE_G1_256=0|1 overrides (tuning).
-  const int64_t avg_slots = pr.E > 0 ? (pr.T * pr.k) / pr.E : 0;
-  bool g1_256 = g2_single && avg_slots >= 96;
-  if (const char* env = getenv("MOE_G1_256")) g1_256 = g2_single && atoi(env) == 1;
   const uint32_t boxt1[2] = {64, g1_256 ? 128u : tok_box};
   {
     const uint64_t d[2] = {uint64_t(pr.H), uint64_t(L.p_max)};
@@ -645,7 +610,7 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   // ---- launches
   AlignTiles tiles;
   std::memset(&tiles, 0, sizeof(tiles));
-  tiles.list[0].tile_max = L.tile_max;
+  tiles.list[0].tile_max = tile;
   tiles.list[0].tile_row = reinterpret_cast<int32_t*>(w + L.tile_row);
   tiles.list[0].tile_rows = reinterpret_cast<int32_t*>(w + L.tile_rows);
   tiles.list[0].tile_expert = reinterpret_cast<int32_t*>(w + L.tile_expert);
@@ -662,9 +627,7 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   prof_mark(st);
   cudaError_t rc;
   // decode sizes (at most 32 slots): align and permute in one launch
-  // (MOE_TINY=0 keeps the two kernels, tuning)
-  const bool tiny = L.S <= 32 && !(getenv("MOE_TINY") && atoi(getenv("MOE_TINY")) == 0);
-  if (tiny) {
+  if (cfg.tiny) {
     rc = launch_align_permute_tiny(view2(ids), pr.T, pr.k, pr.E, bm, counts, offsets, sorted, inv,
                                    block_expert, num_blocks, dev->errors, &tiles, view2(x), pr.H,
                                    w + L.a1, nullptr, nullptr, nullptr, st, &launches);
@@ -700,8 +663,8 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   g1.weights_evict_first = wpolicy;
   g1.tok_box = static_cast<int32_t>(tok_box);
   // decode sizes: GEMM1 finds its experts from the routing ids and requests
-  // weights while align and permute run (MOE_PREFETCH=0: off, tuning)
-  if (!pair && L.tile_max == 32 && L.S <= 32 && !(getenv("MOE_PREFETCH") && atoi(getenv("MOE_PREFETCH")) == 0)) {
+  // weights while align and permute run
+  if (cfg.prefetch) {
     g1.pre_ids = view2(ids);
     g1.pre_E = static_cast<int32_t>(pr.E);
     g1.pre_S = static_cast<int32_t>(L.S);
@@ -714,8 +677,8 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
     g1.tile_expert = tiles.list[1].tile_expert;
     g1.tok_box = 128;
   }
-  rc = pair ? launch_gemm_ws_pair_bf16(0, g1_256 ? 256 : L.tile_max, mGate, mUp, mA1, g1, dev->num_sms, st, &launches)
-            : launch_gemm_ws_bf16(0, L.tile_max, mGate, mUp, mA1, g1, dev->num_sms, st, &launches);
+  rc = pair ? launch_gemm_ws_pair_bf16(0, g1_256 ? 256 : tile, mGate, mUp, mA1, g1, dev->num_sms, st, &launches)
+            : launch_gemm_ws_bf16(0, tile, mGate, mUp, mA1, g1, dev->num_sms, st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm1");
   prof_mark(st);
 
@@ -737,8 +700,8 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   g2.out_ld = pr.H;
   g2.topk_w = view2(wts);
   rc = g2_single ? launch_gemm_ws_pair_bf16(2, 256, mW2, mW2, mH, g2, dev->num_sms, st, &launches)
-     : pair      ? launch_gemm_ws_pair_bf16(1, L.tile_max, mW2, mW2, mH, g2, dev->num_sms, st, &launches)
-            : launch_gemm_ws_bf16(1, L.tile_max, mW2, mW2, mH, g2, dev->num_sms, st, &launches);
+     : pair      ? launch_gemm_ws_pair_bf16(1, tile, mW2, mW2, mH, g2, dev->num_sms, st, &launches)
+            : launch_gemm_ws_bf16(1, tile, mW2, mW2, mH, g2, dev->num_sms, st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm2");
   prof_mark(st);
 
@@ -819,9 +782,7 @@ moe_status_t moe_w13_from_packed(const moe_tensor_t* w13, moe_w13_t* out) {
 size_t moe_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, int32_t wdtype) {
   if (T < 0 || H < 1 || I < 1 || E < 1 || k < 1) return 0;
   if (wdtype != MOE_BF16 && wdtype != MOE_E2M1X2) return 0;
-  int32_t bm = 0, tile_max = 0;
-  choose_tiling(T, k, E, wdtype == MOE_E2M1X2, &bm, &tile_max);
-  return make_layout(T, H, I, E, k, wdtype == MOE_E2M1X2, bm, tile_max).total;
+  return make_layout(T, H, I, E, k, wdtype == MOE_E2M1X2, kBm).total;
 }
 
 moe_status_t moe_forward_ws(const moe_tensor_t* x, const moe_w13_t* w13, const moe_tensor_t* w2,
@@ -924,7 +885,7 @@ moe_status_t moe_align(const moe_tensor_t* topk_ids, int64_t E, int32_t block_m,
   DeviceInfo* dev = nullptr;
   moe_status_t s = device_info(&dev);
   if (s != MOE_OK) return s;
-  const WsLayout L = make_layout(T, 32, 32, E, k, false, block_m, 0);
+  const WsLayout L = make_layout(T, 32, 32, E, k, false, block_m);
   // inv and chunk counts live in the caller's workspace
   const size_t need = align256(L.inv + sizeof(int32_t) * T * k);
   if (!workspace || workspace_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
@@ -980,7 +941,7 @@ moe_status_t moe_get_device_errors(moe_stream_t stream, uint32_t* n_bad_ids, uin
   MOE_CUDA(cudaStreamSynchronize(st));
   if (n_bad_ids) *n_bad_ids = h.bad_ids;
   if (timeouts) *timeouts = h.timeouts;
-  return MOE_OK;
+  return h.timeouts ? MOE_ERR_DEVICE_TIMEOUT : MOE_OK;
 }
 
 }  // extern "C"

@@ -49,7 +49,7 @@ struct Cfg {
   static constexpr int kBufCols = 2 * kNmax;
   static constexpr int kBufs = kTmemCols / kBufCols >= 2 ? 2 : 1;
   static constexpr size_t kSmem = 1024 + size_t(kStages) * kStageBytes +
-                                  kEpiWarps * kStagingBytes + (2 * kStages + 2 * 2 + 1) * 8 + 16;
+                                  kEpiWarps * kStagingBytes + (3 * kStages + 2 * 2 + 1) * 8 + 16;
 };
 
 struct WsArgs {
@@ -109,6 +109,7 @@ struct Smem {
   uint64_t* tfull;
   uint64_t* tempty;
   uint64_t* drain;
+  uint64_t* pre;  // decode prefetch: the early weight copies of each stage land here
   uint32_t* tmem_slot;
 };
 
@@ -125,7 +126,8 @@ __device__ __forceinline__ Smem<kStages> carve(uint8_t* raw) {
   s.tfull = bars + 2 * kStages;
   s.tempty = s.tfull + 2;
   s.drain = s.tempty + 2;
-  s.tmem_slot = reinterpret_cast<uint32_t*>(s.drain + 1);
+  s.pre = s.drain + 1;
+  s.tmem_slot = reinterpret_cast<uint32_t*>(s.pre + kStages);
   return s;
 }
 
@@ -146,6 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], 1);
+      mbar_init(&sm.pre[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.tfull[b], 1);
@@ -165,21 +168,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int num_k = static_cast<int>((g.K + kBK - 1) / kBK);
   // GEMM1 at decode sizes: request the first weight stages of this CTA's first
-  // work item before waiting for align and permute (their token boxes follow
-  // after the wait, on the same stage barriers)
-  int npre = 0;
+  // work item before waiting for align and permute.  The expert comes from the
+  // routing ids read before the PDL wait, which may still be in flight from an
+  // earlier kernel, so the copies land on their own `pre` barriers and the
+  // producer checks the expert against align's tile list after the wait: on a
+  // match the stages are used as they are (the token boxes follow on the
+  // stages' full barriers), else the early copies are let land and the stages
+  // are loaded again from the right expert.
+  int npre = 0, pre_e = -1;
   if (kMode == 0 && kNmax == 32 && g.pre_S > 0 && warp == 0) {
     const int e = first_expert_from_ids(g, blockIdx.x, lane);
     if (e >= 0) {
       npre = num_k < kStages ? num_k : kStages;
+      pre_e = e;
       if (lane == 0) {
         const int64_t wt = blockIdx.x % g.n_wt;
         const uint64_t wpol = g.weights_evict_first ? l2_policy_evict_first() : l2_policy_evict_last();
         for (int kb = 0; kb < npre; ++kb) {
           uint8_t* sw0 = sm.stages + kb * C::kStageBytes;
-          mbar_expect_tx(&sm.full[kb], 2 * C::kWBytes);
-          tma_load_3d(sw0, &tmW0, &sm.full[kb], kb * kBK, static_cast<int32_t>(wt * kWRows), e, wpol);
-          tma_load_3d(sw0 + C::kWBytes, &tmW1, &sm.full[kb], kb * kBK, static_cast<int32_t>(wt * kWRows), e, wpol);
+          mbar_arrive_expect_tx(&sm.pre[kb], 2 * C::kWBytes);
+          tma_load_3d(sw0, &tmW0, &sm.pre[kb], kb * kBK, static_cast<int32_t>(wt * kWRows), e, wpol);
+          tma_load_3d(sw0 + C::kWBytes, &tmW1, &sm.pre[kb], kb * kBK, static_cast<int32_t>(wt * kWRows), e, wpol);
         }
       }
     }
@@ -195,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s < kStages; ++s) last_phase[s] = -1;
       const uint64_t pol = l2_policy_evict_last();
       const uint64_t wpol = g.weights_evict_first ? l2_policy_evict_first() : pol;
-      bool ok = true, pre_done = false;
+      bool ok = true, pre_waited = false;
       for (int64_t item = blockIdx.x; item < total && ok; item += gridDim.x) {
         const int64_t t = item / g.n_wt, wt = item - t * g.n_wt;
         const int32_t e = g.tile_expert[t], row0 = g.tile_row[t], rows = g.tile_rows[t];
@@ -203,16 +212,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int32_t w1 = kMode == 0 ? w0 : w0 + kWRows;
         // whole boxes: a box may run past the tile (rows the MMA's N excludes)
         const int nbox = (rows + g.tok_box - 1) / g.tok_box;
-        const uint32_t bytes = 2 * C::kWBytes + nbox * g.tok_box * kBK * 2;
+        const uint32_t tok_bytes = nbox * g.tok_box * kBK * 2;
+        const uint32_t bytes = 2 * C::kWBytes + tok_bytes;
+        // the early weight copies are this item's only if align agrees on the expert
+        const int use_pre = (item == blockIdx.x && npre > 0 && e == pre_e) ? npre : 0;
+        if (item == blockIdx.x && npre > 0 && !use_pre) {
+          for (int kb = 0; kb < npre; ++kb) mbar_wait(&sm.pre[kb], 0, g.err);
+          pre_waited = true;
+        }
         for (int kb = 0; kb < num_k; ++kb) {
           if (!mbar_wait(&sm.empty[stage], phase ^ 1u, g.err)) { ok = false; break; }
           uint8_t* sw0 = sm.stages + stage * C::kStageBytes;
           uint8_t* sw1 = sw0 + C::kWBytes;
           uint8_t* sx = sw1 + C::kWBytes;
-          if (item == blockIdx.x && kb < npre) {
-            // weights already requested before the PDL wait
-            mbar_arrive_expect_tx(&sm.full[stage], bytes - 2 * C::kWBytes);
-            pre_done = true;
+          if (kb < use_pre) {
+            // weights requested before the PDL wait: the token boxes join the
+            // stage now; the stage's arrival waits until the weights have landed
+            mbar_expect_tx(&sm.full[stage], tok_bytes);
           } else {
             mbar_arrive_expect_tx(&sm.full[stage], bytes);
             tma_load_3d(sw0, &tmW0, &sm.full[stage], kb * kBK, w0, e, wpol);
@@ -221,6 +237,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int b = 0; b < nbox; ++b)
             tma_load_2d(sx + b * g.tok_box * kBK * 2, &tmX, &sm.full[stage], kb * kBK,
                         row0 + b * g.tok_box, pol);
+          if (kb + 1 == use_pre) {
+            for (int j = 0; j < use_pre; ++j) {
+              mbar_wait(&sm.pre[j], 0, g.err);
+              mbar_arrive(&sm.full[j]);
+            }
+            pre_waited = true;
+          }
           last_phase[stage] = static_cast<int8_t>(phase);
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
@@ -229,12 +252,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < kStages; ++s)
           if (last_phase[s] >= 0) mbar_wait(&sm.full[s], static_cast<uint32_t>(last_phase[s]), g.err);
       }
-      if (npre > 0 && !pre_done) {
-        // prefetched stages nobody consumed: let their copies land before exit
-        for (int kb = 0; kb < npre; ++kb) {
-          mbar_arrive(&sm.full[kb]);
-          mbar_wait(&sm.full[kb], 0, g.err);
-        }
+      if (npre > 0 && !pre_waited) {
+        // early copies nobody consumed (no item for this CTA, or a wait gave up
+        // first): let them land before the CTA exits
+        for (int kb = 0; kb < npre; ++kb) mbar_wait(&sm.pre[kb], 0, g.err);
       }
     }
   } else if (warp == 1) {

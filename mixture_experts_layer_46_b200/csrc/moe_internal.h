@@ -6,6 +6,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "../../include/moe.h"
 #include "moe_common.cuh"
 
 namespace moe {
@@ -22,8 +23,8 @@ struct View2 {
 struct WsLayout {
   int64_t T, H, I, E, k, S;
   int32_t bm;         // block_m: padding granule of each expert's rows
-  int32_t tile_max;   // token-tile rows of the weight-stationary GEMMs (0: unused)
-  int64_t t_max;      // upper bound of the token-tile count
+  int32_t tile_max;   // smallest token-tile size the list capacity is sized for
+  int64_t t_max;      // upper bound of the token-tile count (any tile size)
   int32_t tile_max2;  // rows of the second token-tile list (bf16 pairs: 256; 0: none)
   int64_t t_max2;     // upper bound of its tile count
   int64_t n_chunks;   // align chunks
@@ -42,11 +43,16 @@ constexpr int kMaxTopK = 32;            // routing columns per token
 constexpr int kMaxExperts = 1024;       // experts per layer
 constexpr int kAlignChunk = 4096;        // slots per CTA in the multi-CTA align
 constexpr int kAlignSmallMax = 4096;     // single-CTA align up to this many slots
+constexpr int32_t kBm = 32;              // padding granule of each expert's rows (block_m)
+constexpr int32_t kMinTile = 32;         // smallest token tile of any configuration
 
-// Padding granule and token-tile size for a problem (depend only on T, k, E, dtype).
-void choose_tiling(int64_t T, int64_t k, int64_t E, bool mxfp4, int32_t* bm, int32_t* tile_max);
-WsLayout make_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, bool mxfp4, int32_t bm,
-                     int32_t tile_max);
+WsLayout make_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, bool mxfp4,
+                     int32_t bm);
+
+// The kernel configuration a forward of this problem uses: the caller's table,
+// then the built-in tuned table, then the heuristic; flags that do not apply
+// to the chosen tile are cleared.
+moe_config_t select_config(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, bool mxfp4);
 
 // ---- launchers (return cudaError_t of the launch) ----------------------------
 

@@ -155,3 +155,51 @@ def test_product_path_has_no_oracle_dependency():
                 src = open(os.path.join(dirpath, fn)).read()
                 assert "import oracle" not in src and "from oracle" not in src, fn
                 assert "moe_oracle" not in src, fn
+
+
+def test_config_table_lookup_and_fixed_workspace():
+    # the per-shape configuration table (moe_set_config_table) decides the kernels
+    # only: the workspace a caller sizes with moe_workspace_bytes never depends on it
+    shape = (4096, 4096, 1536, 128, 8)
+    base = moe.get_config(*shape)
+    ws0 = moe.workspace_bytes(*shape)
+    assert base["tile"] in (32, 128, 256)
+    e = moe.make_config(_abi.MOE_BF16, H=4096, I=1536, E=128, k=8, t_lo=4000, t_hi=5000, tile=32,
+                        tiny=1, prefetch=1)
+    other_shape = moe.make_config(_abi.MOE_BF16, H=2048, t_lo=0, t_hi=10 ** 9, tile=256)
+    try:
+        moe.set_config_table([other_shape, e])
+        got = moe.get_config(*shape)
+        assert got["tile"] == 32 and got["pair"] == 0
+        assert got["tiny"] == 0 and got["prefetch"] == 0   # 32768 slots: decode-only flags cleared
+        assert moe.get_config(5001, 4096, 1536, 128, 8)["tile"] == 128  # outside the bucket
+        assert moe.get_config(64, 2048, 1536, 128, 8)["tile"] == 256
+        assert moe.get_config(64, 2048, 1536, 128, 8)["pair"] == 1   # 256-row tiles run on pairs
+        assert moe.workspace_bytes(*shape) == ws0
+        assert moe.get_config(*shape, mxfp4=True)["tile"] in (32, 96)  # bf16 entries only
+    finally:
+        moe.set_config_table([])
+    assert moe.get_config(*shape) == base
+
+
+def test_config_table_rejects_malformed_entries():
+    bad = [moe.make_config(_abi.MOE_BF16, tile=64),            # no such tile
+           moe.make_config(_abi.MOE_E2M1X2, tile=128),         # MXFP4 tiles are 32 or 96
+           moe.make_config(_abi.MOE_BF16, tile=32, pair=2),    # flags are 0 or 1
+           moe.make_config(_abi.MOE_BF16, t_lo=10, t_hi=5, tile=32),
+           moe.make_config(7, tile=32)]
+    for b in bad:
+        with pytest.raises(moe.MoeError):
+            moe.set_config_table([b])
+    assert moe.get_config(1, 4096, 1536, 128, 8)["tile"] == 32
+
+
+def test_builtin_config_table_matches_committed_csv():
+    from mixture_experts_layer_46_b200 import build
+
+    rows = build.read_config_csv()
+    assert moe.builtin_config_count() == len(rows)
+    for r in rows:
+        T = r["t_hi"]
+        got = moe.get_config(T, r["H"], r["I"], r["E"], r["k"], mxfp4=r["wdtype"] == 4)
+        assert got["tile"] == r["tile"], r

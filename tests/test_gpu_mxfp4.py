@@ -157,7 +157,7 @@ def test_mxfp4_stale_workspace_contents_never_reach_the_output():
 
 
 @pytest.mark.parametrize("T,k,strided", [(1, 10, False), (3, 10, True), (4, 8, False), (3, 11, False)])
-def test_mxfp4_decode_align_permute_one_launch_matches_two(T, k, strided, monkeypatch):
+def test_mxfp4_decode_align_permute_one_launch_matches_two(T, k, strided):
     # at most 32 slots: align and the quantising permute run as one launch
     H, I, E = 512, 256, 24
     case = make_mx_case(T, H, I, E, k, seed=T + 29)
@@ -169,16 +169,16 @@ def test_mxfp4_decode_align_permute_one_launch_matches_two(T, k, strided, monkey
         c["x"] = case["x"].t().contiguous().cuda().t()
     moe.device_errors()
     outs, launches = {}, {}
-    for tiny in ("1", "0"):
-        monkeypatch.setenv("MOE_TINY", tiny)
-        outs[tiny] = mx_gpu(c)
-        launches[tiny] = moe.last_launch_count()
+    for tiny in (1, 0):
+        with moe.config_override((T, H, I, E, k), mxfp4=True, tiny=tiny):
+            outs[tiny] = mx_gpu(c)
+            launches[tiny] = moe.last_launch_count()
     nbad, nto = moe.device_errors()
     assert nbad == 2 and nto == 0
-    assert torch.equal(outs["1"], outs["0"])
-    assert rel_err(outs["1"], ref) <= MX_TOL
-    assert launches["0"] == 5
-    assert launches["1"] == (4 if T * k <= 32 else 5)
+    assert torch.equal(outs[1], outs[0])
+    assert rel_err(outs[1], ref) <= MX_TOL
+    assert launches[0] == 5
+    assert launches[1] == (4 if T * k <= 32 else 5)
 
 
 def test_mxfp4_shared_expert_fused_routing():

@@ -295,40 +295,41 @@ def test_glm45_air_shape_skewed_strided_ids_sampled():
     assert rel_err(a.cpu()[toks], ref) <= BF16_TOL
 
 
+TILE_VARIANTS = {
+    "32": dict(tile=32),
+    "128/one-cta": dict(tile=128, pair=0),
+    "128/pair-two-slice": dict(tile=128, pair=1, g2_single=0),
+    "128/pair-one-slice": dict(tile=128, pair=1, g2_single=1, g1_256=0),
+    "128/pair-one-slice-g1-256": dict(tile=128, pair=1, g2_single=1, g1_256=1),
+    "256": dict(tile=256),
+}
+
+
 @pytest.mark.parametrize("T,H,I,E,k", [
     (300, 512, 384, 4, 2),     # 150 slots per expert: several 32-row granules, partial tiles
     (600, 512, 640, 3, 2),     # 400 slots per expert: >1 token tile of 256 rows, N tail of I
     (77, 288, 96, 6, 3),       # ragged K and output columns
 ])
-def test_token_tile_configs_agree_and_match_oracle(T, H, I, E, k, monkeypatch):
-    # the token-tile size (32 / 128 rows on one CTA, 256 rows on a CTA pair) is a
-    # performance choice: every configuration must give the same bits
+def test_token_tile_configs_agree_and_match_oracle(T, H, I, E, k):
+    # the token-tile size (32 / 128 rows on one CTA, 128 / 256 rows on a CTA pair)
+    # and the GEMM variants are a performance choice (moe_set_config_table):
+    # every configuration must give the same bits
     case = make_case(T, H, I, E, k, seed=T + 5)
     ref = run_oracle(case)
     c = to_cuda(case)
     outs = {}
-    for tile in ("32", "128", "256", "128/two-slice", "128/gemm1-128"):
-        # "128": on CTA pairs GEMM2 takes one 256-row w2 slice per 256-row token
-        # tile (and GEMM1 the same tiles where experts average 96..399 slots);
-        # "128/two-slice": two slices per 128-row token tile; "128/gemm1-128":
-        # GEMM1 on the 128-row tiles with two accumulator buffers
-        monkeypatch.delenv("MOE_G2", raising=False)
-        monkeypatch.delenv("MOE_G1_256", raising=False)
-        monkeypatch.setenv("MOE_TILE", tile.split("/")[0])
-        if tile.endswith("two-slice"):
-            monkeypatch.setenv("MOE_G2", "1")
-        if tile.endswith("gemm1-128"):
-            monkeypatch.setenv("MOE_G1_256", "0")
-        outs[tile] = run_gpu(c)
-        assert rel_err(outs[tile], ref) <= BF16_TOL, tile
-    assert torch.equal(outs["32"], outs["128"])
-    assert torch.equal(outs["128"], outs["256"])
-    assert torch.equal(outs["128"], outs["128/two-slice"])
-    assert torch.equal(outs["128"], outs["128/gemm1-128"])
+    for name, flags in TILE_VARIANTS.items():
+        with moe.config_override((T, H, I, E, k), **flags):
+            got = moe.get_config(T, H, I, E, k)
+            assert all(got[f] == v for f, v in flags.items() if f != "pair" or flags["tile"] == 128), name
+            outs[name] = run_gpu(c)
+        assert rel_err(outs[name], ref) <= BF16_TOL, name
+    for name in TILE_VARIANTS:
+        assert torch.equal(outs["32"], outs[name]), name
 
 
 @pytest.mark.parametrize("T,k,idt", [(1, 8, torch.int32), (4, 8, torch.int64), (3, 10, torch.int32)])
-def test_decode_weight_prefetch_matches_oracle_and_unprefetched(T, k, idt, monkeypatch):
+def test_decode_weight_prefetch_matches_oracle_and_unprefetched(T, k, idt):
     # at most 32 slots: GEMM1 finds its experts from the routing ids and requests
     # weights before align has run; results must not depend on it
     H, I, E = 512, 384, 16
@@ -340,23 +341,24 @@ def test_decode_weight_prefetch_matches_oracle_and_unprefetched(T, k, idt, monke
     c = to_cuda(case)
     moe.device_errors()
     outs = {}
-    for pre in ("1", "0"):
-        monkeypatch.setenv("MOE_PREFETCH", pre)
-        outs[pre] = run_gpu(c)
+    for pre in (1, 0):
+        with moe.config_override((T, H, I, E, k), prefetch=pre):
+            assert moe.get_config(T, H, I, E, k)["prefetch"] == pre
+            outs[pre] = run_gpu(c)
     nbad, nto = moe.device_errors()
     assert nbad == 2 and nto == 0
-    assert torch.equal(outs["1"], outs["0"])
-    assert rel_err(outs["1"], ref) <= BF16_TOL
+    assert torch.equal(outs[1], outs[0])
+    assert rel_err(outs[1], ref) <= BF16_TOL
 
 
 @pytest.mark.parametrize("T,k,idt,tile,strided", [
     (1, 8, torch.int32, None, False),      # decode
     (4, 8, torch.int64, None, False),      # 32 slots, the largest one-launch batch
     (3, 10, torch.int32, None, True),      # strided x and ids
-    (2, 8, torch.int32, "128", False),     # 128-row token tiles
+    (2, 8, torch.int32, 128, False),       # 128-row token tiles
     (3, 11, torch.int32, None, False),     # 33 slots: align + permute kernels either way
 ])
-def test_decode_align_permute_one_launch_matches_two(T, k, idt, tile, strided, monkeypatch):
+def test_decode_align_permute_one_launch_matches_two(T, k, idt, tile, strided):
     # at most 32 routing slots: align and permute run as one launch that groups
     # the slots with warp ballots; it must give the general kernels' bits
     H, I, E = 512, 384, 24
@@ -371,17 +373,16 @@ def test_decode_align_permute_one_launch_matches_two(T, k, idt, tile, strided, m
         big = torch.zeros(T, 3, k, dtype=idt, device="cuda")
         big[:, 1, :] = c["ids"]
         c["ids"] = big[:, 1, :]
-    if tile:
-        monkeypatch.setenv("MOE_TILE", tile)
+    extra = {"tile": tile} if tile else {}
     moe.device_errors()
     outs, launches = {}, {}
-    for tiny in ("1", "0"):
-        monkeypatch.setenv("MOE_TINY", tiny)
-        outs[tiny] = run_gpu(c)
-        launches[tiny] = moe.last_launch_count()
+    for tiny in (1, 0):
+        with moe.config_override((T, H, I, E, k), tiny=tiny, **extra):
+            outs[tiny] = run_gpu(c)
+            launches[tiny] = moe.last_launch_count()
     nbad, nto = moe.device_errors()
     assert nbad == 2 and nto == 0
-    assert torch.equal(outs["1"], outs["0"])
-    assert rel_err(outs["1"], ref) <= BF16_TOL
-    assert launches["0"] == 5
-    assert launches["1"] == (4 if T * k <= 32 else 5)
+    assert torch.equal(outs[1], outs[0])
+    assert rel_err(outs[1], ref) <= BF16_TOL
+    assert launches[0] == 5
+    assert launches[1] == (4 if T * k <= 32 else 5)
