@@ -12,7 +12,9 @@ with ``mixture_experts_layer_46_b200`` and never imports it.
 
 Parity pins: tests/test_oracle_pins.py (brute force against a dense numpy
 formulation, the one-expert special case against a textbook SwiGLU MLP, the
-invariants, and the MXFP4 worked examples).
+invariants), tests/test_oracle_mxfp4_pins.py (the MXFP4 worked examples and
+brute-force quantiser) and tests/test_oracle_router_pins.py (the router against
+torch's softmax and sort, brute force, ties and invariants).
 """
 
 from __future__ import annotations
@@ -74,6 +76,11 @@ def _load():
             lib.oracle_moe_forward.argtypes = [P(OracleTensor)] * 6 + [
                 ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
                 ctypes.c_int]
+            lib.oracle_router_topk.restype = ctypes.c_int
+            lib.oracle_router_topk.argtypes = [P(OracleTensor), ctypes.c_int64, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+            lib.oracle_e8m0_value.restype = ctypes.c_double
+            lib.oracle_e8m0_value.argtypes = [ctypes.c_uint32]
             lib.oracle_max_threads.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -108,6 +115,26 @@ def max_threads() -> int:
 
 def e2m1_value(code: int) -> float:
     return float(_load().oracle_e2m1_value(code))
+
+
+def e8m0_value(code: int) -> float:
+    return float(_load().oracle_e8m0_value(code))
+
+
+def router_topk(logits: torch.Tensor, k: int, renormalize: bool = True, shared_expert: bool = False):
+    """fp64 router: softmax over the experts, the k most probable (lower index on
+    ties), optionally renormalised; with shared_expert one more column holding
+    expert E with weight 1.0.  Returns (ids int32 [T, kk], weights float64 [T, kk])."""
+    T, E = logits.shape
+    kk = k + (1 if shared_expert else 0)
+    ids = torch.empty(T, kk, dtype=torch.int32)
+    w = torch.empty(T, kk, dtype=torch.float64)
+    d = _desc(logits)
+    rc = _load().oracle_router_topk(ctypes.byref(d), k, 1 if renormalize else 0,
+                                    1 if shared_expert else 0, ids.data_ptr(), w.data_ptr())
+    if rc != 0:
+        raise ValueError("oracle_router_topk: need 1 <= k <= E")
+    return ids, w
 
 
 def mxfp4_quantize(src: torch.Tensor):

@@ -291,6 +291,57 @@ int oracle_moe_forward(const oracle_tensor_t* x, const oracle_tensor_t* gate,
   return 0;
 }
 
+// The router that produces the forward's routing inputs, in fp64:
+//   p = softmax(logits[t, :]) over the E experts,
+//   the k experts of largest p, in descending p (a tie goes to the lower expert index),
+//   weights = those p, divided by their sum when `renormalize` is set.
+// With `shared_expert` set the row gets one more column: expert E (the shared
+// expert, which every token uses) with weight 1.0, the fused-shared-expert
+// convention of aiter PR #3859 ("Summary": expert=513, topk=11 next to the
+// unfused expert=512, topk=10).  The ids and weights are what the forward reads
+// as topk_ids / topk_weights (prime-rl PR #2860, "Problem": the per-layer routing
+// slice a router replay feeds the MoE forward).
+//   logits [T, E] bf16/f32 (strided); ids [T, kk] int32, weights [T, kk] fp64, both
+//   contiguous, kk = k + (shared_expert ? 1 : 0).  Returns 1 on bad arguments.
+int oracle_router_topk(const oracle_tensor_t* logits, int64_t k, int renormalize,
+                       int shared_expert, int32_t* ids, double* weights) {
+  const int64_t T = logits->sizes[0], E = logits->sizes[1];
+  if (k < 1 || k > E) return 1;
+  const int64_t kk = k + (shared_expert ? 1 : 0);
+  for (int64_t t = 0; t < T; ++t) {
+    std::vector<double> l(E), p(E);
+    double mx = -INFINITY;
+    for (int64_t e = 0; e < E; ++e) {
+      l[e] = read_real2(logits, t, e);
+      mx = std::max(mx, l[e]);
+    }
+    double z = 0.0;
+    for (int64_t e = 0; e < E; ++e) {
+      p[e] = std::exp(l[e] - mx);
+      z += p[e];
+    }
+    for (int64_t e = 0; e < E; ++e) p[e] /= z;
+    std::vector<int64_t> order(E);
+    for (int64_t e = 0; e < E; ++e) order[e] = e;
+    std::stable_sort(order.begin(), order.end(),
+                     [&](int64_t a, int64_t b) { return p[a] > p[b]; });
+    double sel = 0.0;
+    for (int64_t j = 0; j < k; ++j) sel += p[order[j]];
+    for (int64_t j = 0; j < k; ++j) {
+      ids[t * kk + j] = (int32_t)order[j];
+      weights[t * kk + j] = renormalize ? p[order[j]] / sel : p[order[j]];
+    }
+    if (shared_expert) {
+      ids[t * kk + k] = (int32_t)E;
+      weights[t * kk + k] = 1.0;
+    }
+  }
+  return 0;
+}
+
+// Value of one e8m0 scale code, by the format definition.
+double oracle_e8m0_value(uint32_t code) { return e8m0_value(code & 255u); }
+
 // Threads OpenMP would use (for reporting the CPU baseline's core count).
 int oracle_max_threads(void) {
 #ifdef _OPENMP

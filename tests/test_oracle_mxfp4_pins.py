@@ -41,11 +41,12 @@ def test_e2m1_values_from_bit_fields():
 
 
 def test_e8m0_decode_matches_torch():
+    # the oracle's scale decoding against torch's own float8_e8m0fnu conversion,
+    # for every finite code (255 is NaN and never produced)
     codes = torch.arange(0, 255, dtype=torch.uint8)
     ref = codes.view(torch.float8_e8m0fnu).to(torch.float64)
-    # decode path used by the oracle: a block of 1.0s quantised under a given scale
-    # is exercised below; here pin the closed form 2^(code-127) against torch.
-    assert torch.equal(ref, torch.tensor([2.0 ** (int(c) - 127) for c in codes], dtype=torch.float64))
+    got = torch.tensor([oracle.e8m0_value(int(c)) for c in codes], dtype=torch.float64)
+    assert torch.equal(got, ref)
 
 
 def _brute_quant_block(v):
