@@ -184,6 +184,8 @@ moe_status_t moe_align(const moe_tensor_t* topk_ids, int64_t E, int32_t block_m,
  * problems return MOE_ERR_WORKSPACE_TOO_SMALL and nothing is launched.
  * The first call on each device looks up that array's device address (a
  * one-time host-side query); make that first call before any stream capture.
+ * The address is kept until the process exits, so do not call this across a
+ * cudaDeviceReset of the device.
  * All calls share the array and it keeps the previous call's contents (the
  * kernels rewrite everything they read).  Calls whose GPU work overlaps, e.g.
  * on two unordered streams, race on it.  Out-of-range ids are skipped but not
@@ -191,6 +193,31 @@ moe_status_t moe_align(const moe_tensor_t* topk_ids, int64_t E, int32_t block_m,
 moe_status_t moe_align_noalloc(const moe_tensor_t* topk_ids, int64_t E, int32_t block_m,
                                int32_t* counts, int32_t* offsets, int32_t* sorted_slots,
                                int32_t* block_expert, int32_t* num_blocks, moe_stream_t stream);
+
+/* The router, the step that produces topk_ids / topk_weights for the forward.
+ * For every token t:
+ *     p = softmax(logits[t, :]) over the E experts,
+ *     topk_ids[t, 0..k-1]     = the k experts of largest p, in descending p,
+ *                               a tie going to the lower expert index,
+ *     topk_weights[t, 0..k-1] = those p, divided by their sum when renormalize = 1.
+ * shared_expert = 1 adds a column k holding expert E with weight 1.0: the
+ * fused-shared-expert routing of ROCm/aiter PR #3859 ("Summary": expert=513,
+ * topk=11 beside the unfused expert=512, topk=10), so the forward then runs
+ * with E + 1 experts and k + 1 columns.  The outputs are written through their
+ * strides, e.g. straight into the per-layer slice [:, l, :] of a
+ * [T, layers, k] routing replay tensor (prime-rl PR #2860, "Problem").
+ *   logits        [T, E] float32 or bf16, any strides; E <= 1024
+ *   topk_ids      [T, k + shared_expert] int32 or int64, any strides
+ *   topk_weights  [T, k + shared_expert] float32, any strides
+ * 1 <= k <= E and k + shared_expert <= 32.  The weights are computed in fp32
+ * with expf (within a few 1e-7 relative of the exact values); the choice of
+ * experts is exact (softmax is monotonic, so it compares the logits).  NaN
+ * logits rank below every number.  T = 0 is a no-op.  Errors:
+ * MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_DTYPE, MOE_ERR_SHAPE_MISMATCH, all
+ * before anything is launched. */
+moe_status_t moe_router_topk(const moe_tensor_t* logits, int32_t k, int32_t renormalize,
+                             int32_t shared_expert, moe_tensor_t* topk_ids,
+                             moe_tensor_t* topk_weights, moe_stream_t stream);
 
 /* MXFP4 quantisation of the rows of src [.., K] (bf16 or f32, inner stride 1,
  * K % 32 == 0) into dst (MOE_E2M1X2 with dst->scale set): per 32 consecutive
@@ -210,6 +237,45 @@ moe_status_t moe_quantize_mxfp4(const moe_tensor_t* src, moe_tensor_t* dst, moe_
  * Synchronises `stream`.  Returns MOE_ERR_DEVICE_TIMEOUT when *timeouts > 0
  * (both counters are still written), else MOE_OK. */
 moe_status_t moe_get_device_errors(moe_stream_t stream, uint32_t* n_bad_ids, uint32_t* timeouts);
+
+/* ---- inspection (tests and debugging) ------------------------------------ */
+
+/* Byte offsets, inside a moe_forward_ws workspace, of the regions a test can
+ * read back after a forward of the same problem: rows = the padded row count
+ * of the expert-grouped buffers; inv = int32 [T*k], the grouped row of each
+ * slot (-1 for a skipped slot); sorted = int32 [rows], the slot of each row;
+ * a1 = the gathered x rows (bf16 [rows, H], or MXFP4 codes [rows, H/2] with
+ * e8m0 scales at a1_scale [rows, H/32]); h = the SwiGLU activation (bf16
+ * [rows, I], or codes [rows, I/2] with scales at h_scale [rows, I/32]);
+ * y = the weighted down-projection rows (bf16 [rows, H]).  Only rows named by
+ * inv hold results; the others are padding and hold stale data. */
+typedef struct {
+  int64_t rows;
+  size_t inv, sorted, a1, a1_scale, h, h_scale, y, total;
+} moe_workspace_layout_t;
+moe_status_t moe_workspace_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k,
+                                  int32_t wdtype, moe_workspace_layout_t* out);
+
+/* Captures an intermediate of the next forwards on the calling host thread
+ * into the device buffer dst (16-byte aligned) until called again with
+ * dst = NULL.  MOE_CAPTURE_H_PREQUANT: the MXFP4 forward's SwiGLU activation
+ * in fp32 just before it is quantised, [rows, I] row-major (rows as in
+ * moe_workspace_layout); skipped when `bytes` is smaller than rows * I * 4.
+ * It lets a test apply its own quantiser to the very values the GPU
+ * quantised.  Costs one extra store per element while on. */
+enum { MOE_CAPTURE_H_PREQUANT = 1 };
+moe_status_t moe_debug_capture(int32_t what, void* dst, size_t bytes);
+
+/* Self-test of the failure path that every wait in the kernels shares: one
+ * GPU thread waits on an mbarrier that nothing arrives on and gives up after
+ * limit_us microseconds (1 .. 100000), exactly as a GEMM's bounded wait gives
+ * up on a missing copy, MMA or epilogue arrival instead of hanging the GPU.
+ * Giving up counts one timeout in the device error counters (read them with
+ * moe_get_device_errors, which then returns MOE_ERR_DEVICE_TIMEOUT) and writes
+ * *done = 2 (device int32; 1 would mean the barrier completed).  No copy or
+ * tensor-core operation is in flight when the wait gives up.  The pages have
+ * no counterpart: they state no failure handling for the kernels. */
+moe_status_t moe_selftest_bounded_wait(int32_t limit_us, int32_t* done, moe_stream_t stream);
 
 /* Number of kernels the last moe_forward_ws / moe_forward call on this thread
  * enqueued (for launch accounting): 4 with at most 32 routing slots, else 5,

@@ -9,5 +9,5 @@ library was not built (there is no CPU fallback).
 from ._abi import (MoeConfig, MoeError, MoeTensor, MoeW13, align, builtin_config_count,  # noqa: F401
                    config_override, desc, device_errors, forward, forward_host, forward_status,
                    get_config, last_launch_count, load, make_config, profile_enable, profile_read,
-                   quantize_mxfp4, set_config_table, version, w13_from_packed, w13_from_views,
-                   workspace_bytes)
+                   quantize_mxfp4, router_status, router_topk, set_config_table, version, w13_from_packed, w13_from_views,
+                   workspace_bytes, workspace_layout, debug_capture, MOE_CAPTURE_H_PREQUANT)

@@ -28,7 +28,9 @@ EXPORTS = ("moe_status_string", "moe_last_cuda_error", "moe_w13_from_packed",
            "moe_workspace_bytes", "moe_forward_ws", "moe_forward", "moe_forward_host",
            "moe_align", "moe_quantize_mxfp4", "moe_get_device_errors", "moe_last_launch_count",
            "moe_profile_enable", "moe_profile_read", "moe_version", "moe_align_noalloc",
-           "moe_set_config_table", "moe_get_config", "moe_builtin_config_count")
+           "moe_set_config_table", "moe_get_config", "moe_builtin_config_count",
+           "moe_router_topk", "moe_selftest_bounded_wait", "moe_workspace_layout",
+           "moe_debug_capture")
 STEP_NAMES = ("align", "permute", "gemm1_swiglu", "gemm2_weighted", "combine")
 
 
@@ -55,6 +57,11 @@ class MoeTensor(ctypes.Structure):
 
 class MoeW13(ctypes.Structure):
     _fields_ = [("gate", MoeTensor), ("up", MoeTensor)]
+
+
+class MoeWorkspaceLayout(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int64)] + [(n, ctypes.c_size_t) for n in (
+        "inv", "sorted", "a1", "a1_scale", "h", "h_scale", "y", "total")]
 
 
 class MoeConfig(ctypes.Structure):
@@ -119,6 +126,16 @@ def load() -> ctypes.CDLL:
             lib.moe_get_config.restype = ctypes.c_int
             lib.moe_get_config.argtypes = [ctypes.c_int64] * 5 + [ctypes.c_int32, P(MoeConfig)]
             lib.moe_builtin_config_count.restype = ctypes.c_int32
+            lib.moe_router_topk.restype = ctypes.c_int
+            lib.moe_router_topk.argtypes = [P(MoeTensor), ctypes.c_int32, ctypes.c_int32,
+                                            ctypes.c_int32, P(MoeTensor), P(MoeTensor), vp]
+            lib.moe_selftest_bounded_wait.restype = ctypes.c_int
+            lib.moe_selftest_bounded_wait.argtypes = [ctypes.c_int32, vp, vp]
+            lib.moe_workspace_layout.restype = ctypes.c_int
+            lib.moe_workspace_layout.argtypes = [ctypes.c_int64] * 5 + [ctypes.c_int32,
+                                                                        P(MoeWorkspaceLayout)]
+            lib.moe_debug_capture.restype = ctypes.c_int
+            lib.moe_debug_capture.argtypes = [ctypes.c_int32, vp, ctypes.c_size_t]
             lib.moe_profile_enable.restype = ctypes.c_int
             lib.moe_profile_enable.argtypes = [ctypes.c_int32]
             lib.moe_profile_read.restype = ctypes.c_int
@@ -263,6 +280,33 @@ def align(topk_ids: torch.Tensor, E: int, block_m: int, *, stream=None):
             "num_blocks": n}
 
 
+def router_topk(logits: torch.Tensor, k: int, *, renormalize: bool = True,
+                shared_expert: bool = False, topk_ids: torch.Tensor | None = None,
+                topk_weights: torch.Tensor | None = None, id_dtype=torch.int32, stream=None):
+    """softmax -> top-k -> renormalise on the GPU (moe_router_topk).  Writes into
+    the given (possibly strided) outputs or new [T, k + shared] tensors."""
+    T = logits.shape[0]
+    kk = k + (1 if shared_expert else 0)
+    if topk_ids is None:
+        topk_ids = torch.empty(T, kk, dtype=id_dtype, device=logits.device)
+    if topk_weights is None:
+        topk_weights = torch.empty(T, kk, dtype=torch.float32, device=logits.device)
+    dl, di, dw = desc(logits), desc(topk_ids), desc(topk_weights)
+    rc = load().moe_router_topk(ctypes.byref(dl), k, 1 if renormalize else 0,
+                                1 if shared_expert else 0, ctypes.byref(di), ctypes.byref(dw),
+                                _stream_ptr(stream))
+    _check(rc, "moe_router_topk")
+    return topk_ids, topk_weights
+
+
+def router_status(logits, k, renormalize, shared_expert, topk_ids, topk_weights) -> int:
+    """The raw moe_status_t of moe_router_topk (for argument-check tests)."""
+    dl, di, dw = desc(logits), desc(topk_ids), desc(topk_weights)
+    st = _stream_ptr(None) if torch.cuda.is_available() else None
+    return int(load().moe_router_topk(ctypes.byref(dl), k, renormalize, shared_expert,
+                                      ctypes.byref(di), ctypes.byref(dw), st))
+
+
 def quantize_mxfp4(src: torch.Tensor, *, stream=None):
     """1x32 e8m0 / e2m1 quantisation of the last axis of a bf16/f32 CUDA tensor.
     Returns (codes uint8 [..., K/2], scales uint8 [..., K/32])."""
@@ -274,6 +318,24 @@ def quantize_mxfp4(src: torch.Tensor, *, stream=None):
     _check(load().moe_quantize_mxfp4(ctypes.byref(ds), ctypes.byref(dd), _stream_ptr(stream)),
            "moe_quantize_mxfp4")
     return codes, scales
+
+
+def workspace_layout(T: int, H: int, I: int, E: int, k: int, mxfp4: bool = False) -> dict:
+    """Byte offsets of the inspectable workspace regions (moe_workspace_layout)."""
+    out = MoeWorkspaceLayout()
+    _check(load().moe_workspace_layout(T, H, I, E, k, MOE_E2M1X2 if mxfp4 else MOE_BF16,
+                                       ctypes.byref(out)), "moe_workspace_layout")
+    return {name: int(getattr(out, name)) for name, _ in out._fields_}
+
+
+MOE_CAPTURE_H_PREQUANT = 1
+
+
+def debug_capture(what: int, buf: torch.Tensor | None) -> None:
+    """Capture an intermediate of the next forwards into `buf` (None stops it)."""
+    ptr = buf.data_ptr() if buf is not None else None
+    n = buf.numel() * buf.element_size() if buf is not None else 0
+    _check(load().moe_debug_capture(what, ptr, n), "moe_debug_capture")
 
 
 def device_errors(stream=None):

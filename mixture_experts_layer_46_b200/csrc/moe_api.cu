@@ -25,6 +25,13 @@ namespace {
 thread_local std::string t_last_cuda_error = "";
 thread_local int32_t t_last_launches = 0;
 
+// inspection captures requested with moe_debug_capture (per host thread)
+struct Capture {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+thread_local Capture t_capture_h;
+
 // per-thread step timing (moe_profile_enable / moe_profile_read)
 constexpr int kProfSteps = 5;
 struct Profiler {
@@ -495,6 +502,8 @@ moe_status_t forward_mxfp4(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   g1.w1_s0 = up->scale_strides[0];
   g1.w1_s1 = up->scale_strides[1];
   g1.err = dev->errors;
+  if (t_capture_h.ptr && t_capture_h.bytes >= sizeof(float) * size_t(L.p_max) * size_t(pr.I))
+    g1.h_capture = static_cast<float*>(t_capture_h.ptr);
   rc = launch_gemm_ws_mxfp4(0, cfg.tile, mGate, mUp, mA1, g1, dev->num_sms, st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm1_mxfp4");
   prof_mark(st);
@@ -516,6 +525,7 @@ moe_status_t forward_mxfp4(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   g2.w1_s0 = g2.w0_s0;
   g2.w1_s1 = g2.w0_s1;
   g2.w_row = reinterpret_cast<const float*>(w + L.w_row);
+  g2.h_capture = nullptr;
   rc = launch_gemm_ws_mxfp4(1, cfg.tile, mW2, mW2, mH, g2, dev->num_sms, st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm2_mxfp4");
   prof_mark(st);
@@ -899,6 +909,36 @@ moe_status_t moe_align(const moe_tensor_t* topk_ids, int64_t E, int32_t block_m,
   return MOE_OK;
 }
 
+moe_status_t moe_router_topk(const moe_tensor_t* logits, int32_t k, int32_t renormalize,
+                             int32_t shared_expert, moe_tensor_t* topk_ids,
+                             moe_tensor_t* topk_weights, moe_stream_t stream) {
+  if (!sizes_ok(logits, 2) || !sizes_ok(topk_ids, 2) || !sizes_ok(topk_weights, 2))
+    return MOE_ERR_INVALID_ARG;
+  if (logits->dtype != MOE_F32 && logits->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED_DTYPE;
+  if (topk_ids->dtype != MOE_I32 && topk_ids->dtype != MOE_I64) return MOE_ERR_UNSUPPORTED_DTYPE;
+  if (topk_weights->dtype != MOE_F32) return MOE_ERR_UNSUPPORTED_DTYPE;
+  if ((renormalize != 0 && renormalize != 1) || (shared_expert != 0 && shared_expert != 1))
+    return MOE_ERR_INVALID_ARG;
+  const int64_t T = logits->sizes[0], E = logits->sizes[1];
+  const int64_t kk = int64_t(k) + shared_expert;
+  if (E < 1 || E > kMaxExperts || k < 1 || k > E || kk > kMaxTopK) return MOE_ERR_INVALID_ARG;
+  if (topk_ids->sizes[0] != T || topk_weights->sizes[0] != T || topk_ids->sizes[1] != kk ||
+      topk_weights->sizes[1] != kk)
+    return MOE_ERR_SHAPE_MISMATCH;
+  if (T == 0) return MOE_OK;
+  if (!logits->data || !topk_ids->data || !topk_weights->data) return MOE_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  moe_status_t s = device_info(&dev);
+  if (s != MOE_OK) return s;
+  int launches = 0;
+  const cudaError_t rc =
+      launch_router_topk(view2(logits), T, static_cast<int>(E), k, renormalize, shared_expert,
+                         view2(topk_ids), view2(topk_weights),
+                         reinterpret_cast<cudaStream_t>(stream), &launches);
+  if (rc != cudaSuccess) return cuda_fail(rc, "router_topk");
+  return MOE_OK;
+}
+
 moe_status_t moe_quantize_mxfp4(const moe_tensor_t* src, moe_tensor_t* dst, moe_stream_t stream) {
   if (!src || !dst || !src->data || !dst->data || !dst->scale) return MOE_ERR_INVALID_ARG;
   if (src->ndim != dst->ndim || (src->ndim != 2 && src->ndim != 3)) return MOE_ERR_INVALID_ARG;
@@ -927,6 +967,44 @@ moe_status_t moe_quantize_mxfp4(const moe_tensor_t* src, moe_tensor_t* dst, moe_
                                           dst->strides[nd - 2], sc, dst->scale_strides[nd - 2], st);
     if (rc != cudaSuccess) return cuda_fail(rc, "quantize");
   }
+  return MOE_OK;
+}
+
+moe_status_t moe_workspace_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k,
+                                  int32_t wdtype, moe_workspace_layout_t* out) {
+  if (!out || T < 0 || H < 1 || I < 1 || E < 1 || k < 1) return MOE_ERR_INVALID_ARG;
+  if (wdtype != MOE_BF16 && wdtype != MOE_E2M1X2) return MOE_ERR_UNSUPPORTED_DTYPE;
+  const bool mx = wdtype == MOE_E2M1X2;
+  const WsLayout L = make_layout(T, H, I, E, k, mx, kBm);
+  out->rows = L.p_max;
+  out->inv = L.inv;
+  out->sorted = L.sorted;
+  out->a1 = L.a1;
+  out->a1_scale = mx ? L.a1_scale : 0;
+  out->h = L.h;
+  out->h_scale = mx ? L.h_scale : 0;
+  out->y = L.y;
+  out->total = L.total;
+  return MOE_OK;
+}
+
+moe_status_t moe_debug_capture(int32_t what, void* dst, size_t bytes) {
+  if (what != MOE_CAPTURE_H_PREQUANT) return MOE_ERR_INVALID_ARG;
+  if (dst && reinterpret_cast<uintptr_t>(dst) % 16 != 0) return MOE_ERR_INVALID_ARG;
+  t_capture_h.ptr = dst;
+  t_capture_h.bytes = dst ? bytes : 0;
+  return MOE_OK;
+}
+
+moe_status_t moe_selftest_bounded_wait(int32_t limit_us, int32_t* done, moe_stream_t stream) {
+  if (limit_us < 1 || limit_us > 100000 || !done) return MOE_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  moe_status_t s = device_info(&dev);
+  if (s != MOE_OK) return s;
+  const cudaError_t rc = launch_bounded_wait_probe(static_cast<unsigned long long>(limit_us) * 1000ull,
+                                                   dev->errors, done,
+                                                   reinterpret_cast<cudaStream_t>(stream));
+  if (rc != cudaSuccess) return cuda_fail(rc, "bounded_wait_probe");
   return MOE_OK;
 }
 

@@ -80,13 +80,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after
-// kWaitLimitNs without completion: counts a timeout and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, DeviceErrors* err) {
+// limit_ns without completion: counts a timeout and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, DeviceErrors* err,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_ns() - t0 > kWaitLimitNs) {
+    if (global_ns() - t0 > limit_ns) {
       if (err) atomicAdd(&err->timeouts, 1u);
       return false;
     }

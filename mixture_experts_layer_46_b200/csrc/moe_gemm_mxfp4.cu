@@ -83,6 +83,7 @@ struct MxArgs {
   const uint8_t* w1_sf;
   int64_t w1_s0, w1_s1;
   const float* w_row;    // GEMM2: routing weight per grouped row (valid rows)
+  float* h_capture;      // GEMM1, inspection only: fp32 h before quantisation [P, N] (or null)
   DeviceErrors* err;
 };
 
@@ -326,6 +327,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const float h = silu_mul(__uint_as_float(gv[j]), __uint_as_float(uv[j]));
+            if (g.h_capture && i0 < g.N)
+              g.h_capture[(row0 + c * 32 + j) * g.N + i0 + lane] = h;
             // |h| as bits orders like its value: one warp reduction gives the block amax
             const float amax = __uint_as_float(
                 __reduce_max_sync(0xffffffffu, __float_as_uint(h) & 0x7fffffffu));
@@ -462,6 +465,7 @@ cudaError_t launch_gemm_ws_mxfp4(int mode, int tile_max, const CUtensorMap& w0,
   g.w1_s0 = p.w1_s0;
   g.w1_s1 = p.w1_s1;
   g.w_row = p.w_row;
+  g.h_capture = p.h_capture;
   g.err = p.err;
   if (launches) *launches += 1;
   const int64_t max_items = p.max_tiles * p.n_wt;

@@ -159,6 +159,7 @@ struct WsGemmMx {
   const uint8_t* w1_sf;   // GEMM1: up scales; GEMM2: w2 scales
   int64_t w1_s0, w1_s1;
   const float* w_row;     // GEMM2: routing weight per grouped row
+  float* h_capture;       // GEMM1: fp32 h before quantisation, [P, I] (inspection; null: off)
   DeviceErrors* err;
 };
 // tile_max: 96 (4-stage ring) or 32 (5-stage ring)
@@ -171,6 +172,16 @@ cudaError_t launch_quantize_rows(const void* src, int32_t src_dtype, int64_t R, 
                                  int64_t src_ld, uint8_t* codes, int64_t codes_ld,
                                  uint8_t* scales, int64_t scales_ld, cudaStream_t st,
                                  int* launches = nullptr);
+
+// router: softmax -> top-k (lower index on ties) -> optional renormalisation,
+// plus the shared-expert column; one warp per token, E <= 1024, k + shared <= 32
+cudaError_t launch_router_topk(const View2& logits, int64_t T, int E, int k, int renorm, int shared,
+                               const View2& ids, const View2& wts, cudaStream_t st, int* launches);
+
+// one thread waits on an mbarrier nobody arrives on, giving up after limit_ns:
+// *done = 2 and one timeout counted (1 would mean the barrier completed)
+cudaError_t launch_bounded_wait_probe(unsigned long long limit_ns, DeviceErrors* err,
+                                      int32_t* done, cudaStream_t st);
 
 // launch helper: PDL attribute on every kernel of the forward
 template <typename Kern, typename... Args>

@@ -45,7 +45,9 @@ ScratchAddr g_addr[64];
 
 // Device address of the scratch array on the current device.  In host code
 // the array's name is only a host-side stand-in, so the real address is looked
-// up once per device (with that device current) and cached.
+// up once per device (with that device current) and cached for the life of the
+// process: do not use this entry point across a cudaDeviceReset of that device
+// (the cached address would belong to the destroyed context).
 cudaError_t scratch_on_current_device(unsigned char** out) {
   int dev = 0;
   cudaError_t rc = cudaGetDevice(&dev);

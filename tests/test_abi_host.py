@@ -203,3 +203,21 @@ def test_builtin_config_table_matches_committed_csv():
         T = r["t_hi"]
         got = moe.get_config(T, r["H"], r["I"], r["E"], r["k"], mxfp4=r["wdtype"] == 4)
         assert got["tile"] == r["tile"], r
+
+
+def test_router_argument_errors_before_launch():
+    # refused on the host, before any device call
+    lg = torch.zeros(4, 16)
+    ids = torch.zeros(4, 2, dtype=torch.int32)
+    w = torch.zeros(4, 2)
+    assert moe.router_status(lg, 17, 1, 0, torch.zeros(4, 17, dtype=torch.int32), torch.zeros(4, 17)) == 1
+    assert moe.router_status(lg, 2, 1, 1, ids, w) == 2          # shared column missing
+    assert moe.router_status(lg, 2, 1, 0, ids.long().double(), w) == 3
+    assert moe.router_status(lg.half(), 2, 1, 0, ids, w) == 3
+    assert moe.router_status(lg, 2, 1, 0, ids, w.double()) == 3
+    assert moe.router_status(lg, 2, 2, 0, ids, w) == 1          # flags are 0 or 1
+    big = torch.zeros(2, 40)
+    assert moe.router_status(big, 32, 1, 1, torch.zeros(2, 33, dtype=torch.int32),
+                             torch.zeros(2, 33)) == 1          # more than 32 columns
+    assert moe.router_status(torch.zeros(0, 16), 2, 1, 0, torch.zeros(0, 2, dtype=torch.int32),
+                             torch.zeros(0, 2)) == 0           # no tokens: nothing to do

@@ -190,20 +190,141 @@ def test_mxfp4_shared_expert_fused_routing():
     assert rel_err(got, ref) <= MX_TOL
 
 
-@pytest.mark.slow
-@pytest.mark.parametrize("shared", [False, True])
-def test_qwen35_tp2_mxfp4_full_size_sampled(shared):
+@pytest.fixture(scope="module")
+def tp2_weights():
+    """Qwen3.5-397B TP2 MXFP4 expert weights for E = 513 (seed 0).  The weights are
+    drawn expert by expert, so the first 512 experts are exactly the E = 512 layer's."""
+    s = wl.QWEN35_TP2_MXFP4_SHARED
+    case = make_mx_case(1, s.H, s.I, s.E, s.k, seed=0, shared=True)
+    dev = {k: case[k].cuda() for k in ("c13", "s13", "c2", "s2")}
+    yield {"cpu": case, "gpu": dev}
+
+
+def _tp2_case(tp2_weights, T, shared, seed_x, seed_r):
     s = wl.QWEN35_TP2_MXFP4_SHARED if shared else wl.QWEN35_TP2_MXFP4
-    case = make_mx_case(s.T, s.H, s.I, s.E, s.k, seed=0, shared=shared)
-    got = mx_gpu(cuda_case(case))
-    # spread tokens, the first and last 16, and tokens of the least-loaded experts
-    g = torch.Generator().manual_seed(11)
-    ids = case["ids"].long()
-    counts = torch.bincount(ids.flatten(), minlength=s.E)
+    E = s.E
+    cw, gw = tp2_weights["cpu"], tp2_weights["gpu"]
+    x = wl.make_x(T, s.H, seed=seed_x)
+    if shared:
+        ids, wts = wl.route_shared_expert(T, E - 1, s.k - 1, seed=seed_r)
+    else:
+        ids, wts = wl.route_softmax_topk(T, E, s.k, seed=seed_r)
+    cpu = {"x": x, "ids": ids, "wts": wts}
+    gpu = {"x": x.cuda(), "ids": ids.cuda(), "wts": wts.cuda()}
+    for key in ("c13", "s13", "c2", "s2"):
+        cpu[key] = cw[key][:E]
+        gpu[key] = gw[key][:E]
+    return s, cpu, gpu
+
+
+def _mx_sample(T, ids, E, n, seed):
+    g = torch.Generator().manual_seed(seed)
+    ids = ids.long()
+    counts = torch.bincount(ids.flatten(), minlength=E)
     routed = torch.nonzero(counts > 0).flatten()
     light = routed[torch.argsort(counts[routed], stable=True)[:4]]
-    parts = [torch.randperm(s.T, generator=g)[:96], torch.arange(16), torch.arange(s.T - 16, s.T)]
-    parts += [torch.nonzero((ids == e).any(dim=1)).flatten()[:8] for e in light.tolist()]
-    toks = torch.unique(torch.cat(parts))
-    ref = mx_oracle(case, tokens=toks)
+    parts = [torch.randperm(T, generator=g)[:n], torch.arange(min(16, T)),
+             torch.arange(max(0, T - 16), T)]
+    parts += [torch.nonzero((ids == e).any(dim=1)).flatten()[:4] for e in light.tolist()]
+    return torch.unique(torch.cat(parts))
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("shared", [False, True])
+def test_qwen35_tp2_mxfp4_full_size_sampled(tp2_weights, shared):
+    s, cpu, gpu = _tp2_case(tp2_weights, 4096, shared, seed_x=1, seed_r=2)
+    got = mx_gpu(gpu)
+    toks = _mx_sample(s.T, cpu["ids"], s.E, 96, 11)
+    ref = mx_oracle(cpu, tokens=toks)
     assert rel_err(got.cpu()[toks], ref) <= MX_TOL
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("T", [1, 16, 32768])
+@pytest.mark.parametrize("shared", [False, True])
+def test_qwen35_tp2_mxfp4_token_sweep(tp2_weights, T, shared):
+    # the MXFP4 token buckets at full width (E = 512 / top-10 and the 513 / 11
+    # shared-expert-fused routing): T = 1 and 16 run the decode path (32-row
+    # tiles, one-launch align + quantising permute for T = 1), T = 32768 the
+    # 96-row tiles; all tokens up to 16, else a sample
+    s, cpu, gpu = _tp2_case(tp2_weights, T, shared, seed_x=2000 + T, seed_r=1000 + T)
+    got = mx_gpu(gpu)
+    toks = None if T <= 16 else _mx_sample(T, cpu["ids"], s.E, 48, T)
+    ref = mx_oracle(cpu, tokens=toks)
+    g = got.cpu() if toks is None else got.cpu()[toks]
+    assert rel_err(g, ref) <= MX_TOL
+    assert torch.isfinite(got.float()).all()
+
+
+def _ws_forward(case, T, H, I, E, k):
+    """moe_forward_ws with a caller workspace; returns (out, workspace, layout)."""
+    c = cuda_case(case)
+    n = moe.workspace_bytes(T, H, I, E, k, mxfp4=True)
+    ws = torch.full((n,), 0xAB, dtype=torch.uint8, device="cuda")
+    v = moe.w13_from_packed(c["c13"], c["s13"])
+    out = moe.forward(c["x"], v, c["c2"], c["ids"], c["wts"], w2_scale=c["s2"], workspace=ws)
+    torch.cuda.synchronize()
+    return out, ws, moe.workspace_layout(T, H, I, E, k, mxfp4=True)
+
+
+def _region(ws, off, rows, cols, dtype=torch.uint8):
+    nbytes = rows * cols * torch.tensor([], dtype=dtype).element_size()
+    return ws[off:off + nbytes].view(dtype).view(rows, cols).cpu()
+
+
+@pytest.mark.parametrize("T,H,I,E,k", [
+    (200, 512, 256, 16, 4),    # single-CTA align, quantising permute kernel
+    (3, 512, 256, 24, 10),     # at most 32 slots: align and quantising permute in one launch
+    (700, 256, 256, 8, 8),     # multi-CTA align (5600 slots)
+])
+def test_permute_quant_grouped_codes_bit_exact(T, H, I, E, k):
+    # every routed slot's grouped row holds the oracle's 1x32 codes and scales of
+    # its token's x row, at the row the oracle's align gives it (inv bit-exact)
+    case = make_mx_case(T, H, I, E, k, seed=T + 61)
+    case["ids"][0, 1] = E                          # a skipped slot
+    _, ws, L = _ws_forward(case, T, H, I, E, k)
+    S = T * k
+    inv = _region(ws, L["inv"], 1, S, torch.int32).flatten()
+    ref_al = oracle.moe_align(case["ids"], E, 32)
+    want_inv = torch.full((S,), -1, dtype=torch.int32)
+    want_inv[ref_al["sorted"][ref_al["sorted"] < S].long()] = torch.nonzero(
+        ref_al["sorted"] < S).flatten().to(torch.int32)
+    assert torch.equal(inv, want_inv)
+    rows = L["rows"]
+    codes = _region(ws, L["a1"], rows, H // 2)
+    scales = _region(ws, L["a1_scale"], rows, H // 32)
+    ref_c, ref_s = oracle.mxfp4_quantize(case["x"].float())
+    valid = inv >= 0
+    slot_tok = torch.arange(S)[valid] // k
+    assert torch.equal(codes[inv[valid].long()], ref_c[slot_tok])
+    assert torch.equal(scales[inv[valid].long()], ref_s[slot_tok])
+
+
+@pytest.mark.parametrize("T,H,I,E,k", [
+    (200, 512, 512, 16, 4),    # 96-row token tiles
+    (2, 512, 256, 24, 10),     # decode: 32-row tiles
+])
+def test_gemm1_h_requantisation_bit_exact(T, H, I, E, k):
+    # GEMM1's epilogue quantises its fp32 SwiGLU output per 1x32 block along I; the
+    # captured fp32 values quantised by the oracle must give the same codes and scales
+    case = make_mx_case(T, H, I, E, k, seed=T + 71)
+    L = moe.workspace_layout(T, H, I, E, k, mxfp4=True)
+    cap = torch.full((L["rows"], I), float("nan"), dtype=torch.float32, device="cuda")
+    moe.debug_capture(moe.MOE_CAPTURE_H_PREQUANT, cap)
+    try:
+        out, ws, L = _ws_forward(case, T, H, I, E, k)
+    finally:
+        moe.debug_capture(moe.MOE_CAPTURE_H_PREQUANT, None)
+    S = T * k
+    inv = _region(ws, L["inv"], 1, S, torch.int32).flatten()
+    rows = inv[inv >= 0].long()
+    h = cap.cpu()[rows]
+    assert torch.isfinite(h).all()
+    codes = _region(ws, L["h"], L["rows"], I // 2)[rows]
+    scales = _region(ws, L["h_scale"], L["rows"], I // 32)[rows]
+    ref_c, ref_s = oracle.mxfp4_quantize(h.contiguous())
+    assert torch.equal(scales, ref_s)
+    assert torch.equal(codes, ref_c)
+    # and the capture did not change the result
+    out2, _, _ = _ws_forward(case, T, H, I, E, k)
+    assert torch.equal(out, out2)

@@ -262,10 +262,18 @@ def _sample_tokens(T, n, seed, ids=None, E=None, per_expert=8, n_light=4):
     return torch.unique(torch.cat(parts))
 
 
-@pytest.mark.slow
-def test_qwen3_235b_shape_full_size_sampled():
+@pytest.fixture(scope="module")
+def qwen3_weights():
+    """Qwen3-235B-shaped expert weights (seed 0) on the GPU and a host copy for the oracle."""
     s = wl.QWEN3_235B
     w13, w2 = wl.make_weights_bf16(s.E, s.I, s.H, seed=0, device="cuda")
+    yield {"w13": w13, "w2": w2, "w13_cpu": w13.cpu(), "w2_cpu": w2.cpu()}
+
+
+@pytest.mark.slow
+def test_qwen3_235b_shape_full_size_sampled(qwen3_weights):
+    s = wl.QWEN3_235B
+    w13, w2 = qwen3_weights["w13"], qwen3_weights["w2"]
     x = wl.make_x(s.T, s.H, seed=1, device="cuda")
     ids, wts = wl.route_softmax_topk(s.T, s.E, s.k, seed=2, device="cuda")
     c = {"x": x, "w13": w13, "w2": w2, "ids": ids, "wts": wts}
@@ -273,9 +281,33 @@ def test_qwen3_235b_shape_full_size_sampled():
     b = run_gpu(c, contiguous=True)
     assert torch.equal(a, b)
     toks = _sample_tokens(s.T, 128, 0, ids=ids, E=s.E)
-    case_cpu = {"x": x.cpu(), "w13": w13.cpu(), "w2": w2.cpu(), "ids": ids.cpu(), "wts": wts.cpu()}
+    case_cpu = {"x": x.cpu(), "w13": qwen3_weights["w13_cpu"], "w2": qwen3_weights["w2_cpu"],
+                "ids": ids.cpu(), "wts": wts.cpu()}
     ref = run_oracle(case_cpu, tokens=toks)
     assert rel_err(a.cpu()[toks], ref) <= BF16_TOL
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("T", [1, 4, 64, 1023, 4097, 16384])
+def test_qwen3_235b_token_sweep_full_shape(qwen3_weights, T):
+    # the decode and prefill sweep on the full expert shapes (H=4096, I=1536,
+    # E=128, top-8), strided packed w13, the sweep's per-T seeds: decode sizes
+    # stream 32-row tiles on most SMs; 1023 / 4097 leave ragged last tiles and
+    # 4097 runs the multi-CTA align; 16384 runs the 256-row CTA-pair tiles.
+    # All tokens up to 64, else a sample: first and last 16, spread tokens and
+    # the least-loaded experts' tokens (their short tiles are the edge cases).
+    s = wl.QWEN3_235B
+    w13, w2 = qwen3_weights["w13"], qwen3_weights["w2"]
+    x = wl.make_x(T, s.H, seed=2000 + T, device="cuda")
+    ids, wts = wl.route_softmax_topk(T, s.E, s.k, seed=1000 + T, device="cuda")
+    a = run_gpu({"x": x, "w13": w13, "w2": w2, "ids": ids, "wts": wts})
+    toks = None if T <= 64 else _sample_tokens(T, 48, T, ids=ids, E=s.E, per_expert=4)
+    case_cpu = {"x": x.cpu(), "w13": qwen3_weights["w13_cpu"], "w2": qwen3_weights["w2_cpu"],
+                "ids": ids.cpu(), "wts": wts.cpu()}
+    ref = run_oracle(case_cpu, tokens=toks)
+    got = a.cpu() if toks is None else a.cpu()[toks]
+    assert rel_err(got, ref) <= BF16_TOL
+    assert torch.isfinite(a.float()).all()
 
 
 @pytest.mark.slow

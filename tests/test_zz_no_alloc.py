@@ -5,10 +5,11 @@ in a fixed array inside the library.
 
 Checked here through the C ABI: on two calls in a row (different routing, so
 the second call starts from the first call's leftover scratch) its outputs
-equal those of moe_align, which uses a caller-provided workspace, bit for bit
-(align is integer work, so the tolerance is exact equality).  The problem size
-uses the multi-CTA path, so both scratch regions are exercised.  Oversized
-problems are refused.
+equal, bit for bit (align is integer work, so the tolerance is exact
+equality), both those of moe_align, which uses a caller-provided workspace, and
+those of the CPU oracle's align.  The second routing holds out-of-range ids,
+which both skip.  The problem size uses the multi-CTA path, so both scratch
+regions are exercised.  Oversized problems are refused.
 
 This file sorts last so a run that stops at the first failure has already run
 every other test.
@@ -20,6 +21,7 @@ import pytest
 import torch
 
 import mixture_experts_layer_46_b200 as moe
+import oracle
 from mixture_experts_layer_46_b200 import _abi
 from mixture_experts_layer_46_b200 import workloads as wl
 
@@ -58,18 +60,30 @@ def test_noalloc_align_matches_workspace_align_twice():
     E, bm = 128, 128
     ids1, _ = wl.route_softmax_topk(4096, E, 8, seed=11, device="cuda")
     ids_all, _ = wl.route_zipf_layers(3000, E, 8, layers=46, seed=12, device="cuda")
+    ids_all[5, 23, 3] = -1      # out-of-range ids: skipped by every implementation
+    ids_all[77, 23, 0] = E
     ids2 = ids_all[:, 23, :]  # strided slice, token stride 368
     first = _noalloc(ids1, E, bm)
     ref1 = moe.align(ids1, E, bm)
     torch.cuda.synchronize()
     _same(first, ref1)
+    _same(first, oracle.moe_align(ids1.cpu(), E, bm))
+    torch.cuda.synchronize()
     free0, _ = torch.cuda.mem_get_info()
+    alloc0 = torch.cuda.memory_allocated()
     second = _noalloc(ids2, E, bm)
     free1, _ = torch.cuda.mem_get_info()
+    alloc1 = torch.cuda.memory_allocated()
     ref2 = moe.align(ids2, E, bm)
     torch.cuda.synchronize()
     _same(second, ref2)
-    assert free1 == free0  # the call itself allocated nothing
+    _same(second, oracle.moe_align(ids_all.cpu()[:, 23, :], E, bm))
+    assert int(second["counts"].sum().item()) == 3000 * 8 - 2
+    # the call itself allocated nothing: neither through torch's allocator nor on
+    # the device (device-wide free memory also moves if another process on the
+    # same GPU allocates, so this assumes the GPU is not shared meanwhile)
+    assert alloc1 == alloc0
+    assert free1 == free0
 
 
 def test_noalloc_align_refuses_oversized_problem():
