@@ -81,6 +81,25 @@ def peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+# Dense FP4 (kind::mxf4) tensor rate measured on this machine's B200s with the
+# library's MMA-rate probe (moe_measure_mma_peak: back-to-back M=128 N=128 MMAs
+# from shared memory on all 148 SMs, CUDA events, best of five launches of
+# 100000 x 4 instructions per SM), beside the same probe's bf16 rate.  The
+# MXFP4 roofline takes the measured bf16 GEMM burst peak x their ratio.
+FP4_PEAK = {"bf16_tflops": 2231.4, "mxf4_tflops": 8925.7,
+            "note": "MMA-rate probe on one B200: bf16 2231 TFLOP/s, mxf4 8926 TFLOP/s"}
+
+
+def fp4_peak(bf16_burst: float):
+    """(peak TFLOP/s, source) for kind::mxf4: the measured probe figure scaled to the
+    burst bf16 peak by the probe's own mxf4/bf16 ratio, else the nominal 4x ratio."""
+    if FP4_PEAK:
+        ratio = FP4_PEAK["mxf4_tflops"] / FP4_PEAK["bf16_tflops"]
+        return bf16_burst * ratio, (f"measured bf16 burst peak x the measured mxf4/bf16 MMA-rate "
+                                    f"ratio {ratio:.3f} ({FP4_PEAK['note']})")
+    return bf16_burst * 4.0, "measured bf16 burst peak x4 nominal FP4/bf16 ratio (FP4 peak not measured)"
+
+
 def workload_name(w) -> str:
     dt = "mxfp4 (e2m1 + e8m0 per 1x32)" if w.get("mxfp4") else "bf16"
     return (f"moe-layer {dt} T={w['T']} H={w['H']} I={w['I']} E={w['E']} top_k={w['k']} "
@@ -428,9 +447,9 @@ def main():
 
     # ---------------------------------------------------------------- roofline
     hbm, tf_burst, tf_sus, src = peaks()
+    fp4_src = None
     if mx:
-        # FP4 dense peak = measured bf16 x the nominal 9 / 2.25 PFLOP/s ratio (assumed)
-        tf_burst = tf_burst * 4.0
+        tf_burst, fp4_src = fp4_peak(tf_burst)
     alg = algorithmic(w, inp["ids"])
     g1_ms = brk.get("gemm1_swiglu", float("nan"))
     t_tc = alg["gemm1_flops"] / (tf_burst * 1e12)
@@ -452,7 +471,8 @@ def main():
                          ("kind::f16 on CTA pairs)" if pair else "kind::f16)")))
     roof["peak_source"] = (f"{src} (MEASURED_PEAKS.json burst)" if src == "measured" else "fallback")
     if mx and roof["bound"] == "tensor":
-        roof["peak_source"] += " x4 nominal FP4/bf16 ratio (FP4 peak not measured)"
+        roof["peak_source"] = fp4_src
+    roof["scope"] = "the gemm1_swiglu kernel alone; layer_roofline covers the whole forward"
     t_roof_layer = max(alg["flops"] / (tf_burst * 1e12), alg["bytes"] / (hbm * 1e9))
     layer_frac = t_roof_layer / (ms * 1e-3)
 
@@ -498,8 +518,9 @@ def sweep(args, w, moe, wl, dev, stream, flush):
     """Token sweep on the same weights (fresh routing per T): one JSONL row per T."""
     hbm, tf_burst, _, _ = peaks()
     mx = bool(w.get("mxfp4"))
+    fp4_src = None
     if mx:
-        tf_burst = tf_burst * 4.0  # FP4 dense peak: measured bf16 x the nominal 4x ratio (assumed)
+        tf_burst, fp4_src = fp4_peak(tf_burst)
         c13, s13, w2, s2 = make_mx_weights(w, dev)
         v13 = moe.w13_from_packed(c13, s13)
         tokens = wl.MXFP4_TOKEN_SWEEP
@@ -521,15 +542,20 @@ def sweep(args, w, moe, wl, dev, stream, flush):
             out = torch.empty(T, w["H"], dtype=torch.bfloat16, device=dev)
             for _ in range(5):
                 moe.forward(x, v13, w2, ids, wts, out=out, workspace=ws, stream=stream, w2_scale=s2)
-            per = []
-            for i in range(30 if T < 8192 else 10 if T <= 16384 else 5):
+            reps = 50 if T < 8192 else 20 if T <= 16384 else 10
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(reps)]
+            sampler = ClockSampler(dev.index)
+            sampler.start()
+            torch.cuda.synchronize(dev)
+            for i in range(reps):
                 wl.flush_l2(flush, i)
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(stream)
+                evs[i][0].record(stream)
                 moe.forward(x, v13, w2, ids, wts, out=out, workspace=ws, stream=stream, w2_scale=s2)
-                b.record(stream)
-                torch.cuda.synchronize(dev)
-                per.append(a.elapsed_time(b))
+                evs[i][1].record(stream)
+            torch.cuda.synchronize(dev)
+            clocks = sampler.stop()
+            per = [a.elapsed_time(b) for a, b in evs]
             med = statistics.median(per)
             moe.profile_enable(True)
             brk = {}
@@ -541,8 +567,14 @@ def sweep(args, w, moe, wl, dev, stream, flush):
             moe.profile_enable(False)
             alg = algorithmic(wt, ids)
             t_roof = max(alg["flops"] / (tf_burst * 1e12), alg["bytes"] / (hbm * 1e9))
-            row = {"T": T, "us_median": med * 1e3, "tokens_per_s": T / (med * 1e-3),
+            row = {"T": T, "workload": workload_name(wt), "us_median": med * 1e3,
+                   "us_p10": sorted(per)[len(per) // 10] * 1e3,
+                   "us_p90": sorted(per)[(9 * len(per)) // 10] * 1e3, "reps": reps,
+                   "tokens_per_s": T / (med * 1e-3),
                    "roofline_us": t_roof * 1e6, "frac": t_roof / (med * 1e-3),
+                   "bound": "tensor" if alg["flops"] / (tf_burst * 1e12) >= alg["bytes"] / (hbm * 1e9) else "hbm",
+                   "fp4_peak": fp4_src if mx else None, "clocks": clocks,
+                   "config": moe.get_config(T, w["H"], w["I"], w["E"], w["k"], mxfp4=mx),
                    "hbm_GBs_alg": alg["bytes"] / (med * 1e-3) / 1e9,
                    "tflops_alg": alg["flops"] / (med * 1e-3) / 1e12,
                    "active_experts": alg["active_experts"],

@@ -266,6 +266,17 @@ moe_status_t moe_workspace_layout(int64_t T, int64_t H, int64_t I, int64_t E, in
 enum { MOE_CAPTURE_H_PREQUANT = 1 };
 moe_status_t moe_debug_capture(int32_t what, void* dst, size_t bytes);
 
+/* Measures the dense tensor-core rate of this GPU in TFLOP/s (*tflops):
+ * every SM issues `iters` (1 .. 2^20) x 4 back-to-back tcgen05.mma (M = 128, N = 128)
+ * from operand tiles resident in shared memory, no global memory involved;
+ * kind 0 = kind::f16 (bf16 inputs, fp32 accumulate, K = 16 per instruction),
+ * kind 1 = kind::mxf4 (e2m1 inputs with e8m0 scales per 32, K = 64).  The
+ * MXFP4 roofline of the forward uses the ratio of the two rates times the
+ * measured bf16 GEMM peak, instead of a nominal ratio.  Blocking: six launches
+ * on the legacy default stream timed with CUDA events, the best of the last
+ * five.  A measurement tool; not on the forward's path. */
+moe_status_t moe_measure_mma_peak(int32_t kind, int32_t iters, double* tflops);
+
 /* Self-test of the failure path that every wait in the kernels shares: one
  * GPU thread waits on an mbarrier that nothing arrives on and gives up after
  * limit_us microseconds (1 .. 100000), exactly as a GEMM's bounded wait gives

@@ -30,7 +30,7 @@ EXPORTS = ("moe_status_string", "moe_last_cuda_error", "moe_w13_from_packed",
            "moe_profile_enable", "moe_profile_read", "moe_version", "moe_align_noalloc",
            "moe_set_config_table", "moe_get_config", "moe_builtin_config_count",
            "moe_router_topk", "moe_selftest_bounded_wait", "moe_workspace_layout",
-           "moe_debug_capture")
+           "moe_debug_capture", "moe_measure_mma_peak")
 STEP_NAMES = ("align", "permute", "gemm1_swiglu", "gemm2_weighted", "combine")
 
 
@@ -136,6 +136,9 @@ def load() -> ctypes.CDLL:
                                                                         P(MoeWorkspaceLayout)]
             lib.moe_debug_capture.restype = ctypes.c_int
             lib.moe_debug_capture.argtypes = [ctypes.c_int32, vp, ctypes.c_size_t]
+            lib.moe_measure_mma_peak.restype = ctypes.c_int
+            lib.moe_measure_mma_peak.argtypes = [ctypes.c_int32, ctypes.c_int32,
+                                                 P(ctypes.c_double)]
             lib.moe_profile_enable.restype = ctypes.c_int
             lib.moe_profile_enable.argtypes = [ctypes.c_int32]
             lib.moe_profile_read.restype = ctypes.c_int
@@ -326,6 +329,14 @@ def workspace_layout(T: int, H: int, I: int, E: int, k: int, mxfp4: bool = False
     _check(load().moe_workspace_layout(T, H, I, E, k, MOE_E2M1X2 if mxfp4 else MOE_BF16,
                                        ctypes.byref(out)), "moe_workspace_layout")
     return {name: int(getattr(out, name)) for name, _ in out._fields_}
+
+
+def measure_mma_peak(kind: str, iters: int = 100000) -> float:
+    """Dense tensor-core rate (TFLOP/s) of back-to-back MMAs: kind 'bf16' or 'mxf4'."""
+    out = ctypes.c_double(0.0)
+    _check(load().moe_measure_mma_peak({"bf16": 0, "mxf4": 1}[kind], iters, ctypes.byref(out)),
+           "moe_measure_mma_peak")
+    return float(out.value)
 
 
 MOE_CAPTURE_H_PREQUANT = 1

@@ -996,6 +996,17 @@ moe_status_t moe_debug_capture(int32_t what, void* dst, size_t bytes) {
   return MOE_OK;
 }
 
+moe_status_t moe_measure_mma_peak(int32_t kind, int32_t iters, double* tflops) {
+  if ((kind != 0 && kind != 1) || iters < 1 || iters > (1 << 20) || !tflops)
+    return MOE_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  moe_status_t s = device_info(&dev);
+  if (s != MOE_OK) return s;
+  const cudaError_t rc = measure_mma_rate(kind, iters, dev->num_sms, dev->errors, tflops);
+  if (rc != cudaSuccess) return cuda_fail(rc, "mma_rate");
+  return MOE_OK;
+}
+
 moe_status_t moe_selftest_bounded_wait(int32_t limit_us, int32_t* done, moe_stream_t stream) {
   if (limit_us < 1 || limit_us > 100000 || !done) return MOE_ERR_INVALID_ARG;
   DeviceInfo* dev = nullptr;

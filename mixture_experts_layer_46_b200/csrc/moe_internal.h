@@ -183,6 +183,10 @@ cudaError_t launch_router_topk(const View2& logits, int64_t T, int E, int k, int
 cudaError_t launch_bounded_wait_probe(unsigned long long limit_ns, DeviceErrors* err,
                                       int32_t* done, cudaStream_t st);
 
+// tensor-pipe rate of back-to-back MMAs on every SM (kind 0: bf16, 1: mxf4), TFLOP/s;
+// blocking (times six launches on the legacy stream with CUDA events, best of the last five)
+cudaError_t measure_mma_rate(int kind, int iters, int num_sms, DeviceErrors* err, double* tflops);
+
 // launch helper: PDL attribute on every kernel of the forward
 template <typename Kern, typename... Args>
 cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st,

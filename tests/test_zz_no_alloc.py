@@ -28,26 +28,40 @@ from mixture_experts_layer_46_b200 import workloads as wl
 pytestmark = pytest.mark.gpu
 
 
-def _noalloc(ids: torch.Tensor, E: int, bm: int):
+def _outputs(ids: torch.Tensor, E: int, bm: int):
+    """Output buffers of one call (the caller's own memory, allocated up front)."""
     T, k = ids.shape
     S = T * k
     pmax = S + min(E, S) * (bm - 1) + bm
     dev = ids.device
-    counts = torch.full((E,), -1, dtype=torch.int32, device=dev)
-    offsets = torch.full((E + 1,), -1, dtype=torch.int32, device=dev)
-    sorted_ = torch.full((pmax,), -7, dtype=torch.int32, device=dev)
-    block_expert = torch.full((pmax // bm + 1,), -7, dtype=torch.int32, device=dev)
-    nb = torch.zeros(1, dtype=torch.int32, device=dev)
+    return {"counts": torch.full((E,), -1, dtype=torch.int32, device=dev),
+            "offsets": torch.full((E + 1,), -1, dtype=torch.int32, device=dev),
+            "sorted": torch.full((pmax,), -7, dtype=torch.int32, device=dev),
+            "block_expert": torch.full((pmax // bm + 1,), -7, dtype=torch.int32, device=dev),
+            "nb": torch.zeros(1, dtype=torch.int32, device=dev)}
+
+
+def _call(ids: torch.Tensor, E: int, bm: int, o: dict) -> int:
     d = _abi.desc(ids)
-    rc = moe.load().moe_align_noalloc(ctypes.byref(d), E, bm, counts.data_ptr(), offsets.data_ptr(),
-                                      sorted_.data_ptr(), block_expert.data_ptr(), nb.data_ptr(),
-                                      torch.cuda.current_stream().cuda_stream)
-    assert rc == 0, _abi.STATUS.get(rc, rc)
+    return moe.load().moe_align_noalloc(ctypes.byref(d), E, bm, o["counts"].data_ptr(),
+                                        o["offsets"].data_ptr(), o["sorted"].data_ptr(),
+                                        o["block_expert"].data_ptr(), o["nb"].data_ptr(),
+                                        torch.cuda.current_stream().cuda_stream)
+
+
+def _result(o: dict, E: int):
     torch.cuda.synchronize()
-    P = int(offsets[E].item())
-    n = int(nb.item())
-    return {"counts": counts, "offsets": offsets, "sorted": sorted_[:P],
-            "block_expert": block_expert[:n], "num_blocks": n}
+    P = int(o["offsets"][E].item())
+    n = int(o["nb"].item())
+    return {"counts": o["counts"], "offsets": o["offsets"], "sorted": o["sorted"][:P],
+            "block_expert": o["block_expert"][:n], "num_blocks": n}
+
+
+def _noalloc(ids: torch.Tensor, E: int, bm: int):
+    o = _outputs(ids, E, bm)
+    rc = _call(ids, E, bm, o)
+    assert rc == 0, _abi.STATUS.get(rc, rc)
+    return _result(o, E)
 
 
 def _same(a, b):
@@ -68,12 +82,16 @@ def test_noalloc_align_matches_workspace_align_twice():
     torch.cuda.synchronize()
     _same(first, ref1)
     _same(first, oracle.moe_align(ids1.cpu(), E, bm))
+    out2 = _outputs(ids2, E, bm)
     torch.cuda.synchronize()
     free0, _ = torch.cuda.mem_get_info()
     alloc0 = torch.cuda.memory_allocated()
-    second = _noalloc(ids2, E, bm)
+    rc = _call(ids2, E, bm, out2)           # only the call itself sits between the readings
+    torch.cuda.synchronize()
     free1, _ = torch.cuda.mem_get_info()
     alloc1 = torch.cuda.memory_allocated()
+    assert rc == 0, _abi.STATUS.get(rc, rc)
+    second = _result(out2, E)
     ref2 = moe.align(ids2, E, bm)
     torch.cuda.synchronize()
     _same(second, ref2)
