@@ -190,16 +190,6 @@ def test_mxfp4_shared_expert_fused_routing():
     assert rel_err(got, ref) <= MX_TOL
 
 
-@pytest.fixture(scope="module")
-def tp2_weights():
-    """Qwen3.5-397B TP2 MXFP4 expert weights for E = 513 (seed 0).  The weights are
-    drawn expert by expert, so the first 512 experts are exactly the E = 512 layer's."""
-    s = wl.QWEN35_TP2_MXFP4_SHARED
-    case = make_mx_case(1, s.H, s.I, s.E, s.k, seed=0, shared=True)
-    dev = {k: case[k].cuda() for k in ("c13", "s13", "c2", "s2")}
-    yield {"cpu": case, "gpu": dev}
-
-
 def _tp2_case(tp2_weights, T, shared, seed_x, seed_r):
     s = wl.QWEN35_TP2_MXFP4_SHARED if shared else wl.QWEN35_TP2_MXFP4
     E = s.E

@@ -262,14 +262,6 @@ def _sample_tokens(T, n, seed, ids=None, E=None, per_expert=8, n_light=4):
     return torch.unique(torch.cat(parts))
 
 
-@pytest.fixture(scope="module")
-def qwen3_weights():
-    """Qwen3-235B-shaped expert weights (seed 0) on the GPU and a host copy for the oracle."""
-    s = wl.QWEN3_235B
-    w13, w2 = wl.make_weights_bf16(s.E, s.I, s.H, seed=0, device="cuda")
-    yield {"w13": w13, "w2": w2, "w13_cpu": w13.cpu(), "w2_cpu": w2.cpu()}
-
-
 @pytest.mark.slow
 def test_qwen3_235b_shape_full_size_sampled(qwen3_weights):
     s = wl.QWEN3_235B
