@@ -53,14 +53,8 @@ WORKLOADS = {
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed to the hash of the kernel
 # source it was taken on; reported as null once the source has changed.
 NCU_TRAFFIC = {
-    # profiles/gemm_ws_pair_bf16_qwen3shape_E32_T1024.md: 941.5 MB read + 27.0 MB written by
-    # GEMM1 (256-row token tiles) on the E=32, T=1024 case (~256 slots per expert), scaled x4
-    # (experts and tokens) to the E=128, T=4096 launch; keyed to the kernel and host sources.
-    # Re-keyed without a new capture after one host-side change: GEMM1's 256-row token tiles are
-    # now also chosen from 400 slots per expert up, which neither the captured case (~256 per
-    # expert) nor the T=4096 launch (256 per expert) reaches; kernels and their launch unchanged
-    "gemm1_swiglu": {"bytes_per_launch": 4.0 * (941.518848e6 + 27.002624e6), "src": "0defb09e557f820d",
-                     "workload": "qwen3-235b T=4096"},
+    # filled from the ncu launch of GEMM1 on the benchmarked workload (T=4096, E=128),
+    # keyed to the hash of the kernel and host sources it was captured on
 }
 
 

@@ -289,8 +289,9 @@ moe_status_t moe_measure_mma_peak(int32_t kind, int32_t iters, double* tflops);
 moe_status_t moe_selftest_bounded_wait(int32_t limit_us, int32_t* done, moe_stream_t stream);
 
 /* Number of kernels the last moe_forward_ws / moe_forward call on this thread
- * enqueued (for launch accounting): 4 with at most 32 routing slots, else 5,
- * plus 2 when align runs its multi-CTA form (more than 4096 slots). */
+ * enqueued (for launch accounting): 1 on the one-kernel decode path, 4 with at
+ * most 32 routing slots otherwise, else 5, plus 2 when align runs its
+ * multi-CTA form (more than 4096 slots). */
 int32_t moe_last_launch_count(void);
 
 /* Per-kernel timing for profiling.  While enabled on the calling thread, each
@@ -326,6 +327,11 @@ typedef struct {
   int32_t tiny;        /* at most 32 slots: align and permute in one launch */
   int32_t prefetch;    /* at most 32 slots, 32-row tiles: GEMM1 requests its first weight
                           stages before align has finished (checked against align after) */
+  int32_t fused;       /* bf16, at most 32 slots: the whole forward as one kernel (slots
+                          grouped in every CTA, token rows gathered from x, GEMM2 weights
+                          streamed across the GEMM1 hand-off, combine by the last CTA of
+                          each output tile); needs x with unit inner stride and 16-byte
+                          aligned rows and H <= 16384, else the kernels above run */
 } moe_config_t;
 
 /* Installs a process-wide configuration table (copied; n = 0 removes it).

@@ -173,6 +173,22 @@ cudaError_t launch_quantize_rows(const void* src, int32_t src_dtype, int64_t R, 
                                  uint8_t* scales, int64_t scales_ld, cudaStream_t st,
                                  int* launches = nullptr);
 
+// the whole bf16 forward as one kernel for at most 32 routing slots
+struct DecodeArgs {
+  int64_t T, H, I, E, k;
+  View2 ids, topk_w;
+  __nv_bfloat16* h_ws;  // [32, I] workspace rows (by slot)
+  __nv_bfloat16* y_ws;  // [32, H] workspace rows (by slot)
+  __nv_bfloat16* out;
+  int64_t os0, os1;
+  DeviceErrors* err;
+};
+// maps: gate/up/w2 3-D weight maps ([64 x 128] boxes), x1 = x [T, H] and h1 = h_ws [32, I]
+// with one-row [64 x 1] boxes (read by four-row gathers); grid = num_sms
+cudaError_t launch_decode_fused(const CUtensorMap& gate, const CUtensorMap& up, const CUtensorMap& w2,
+                                const CUtensorMap& x1, const CUtensorMap& h1, const DecodeArgs& p,
+                                int num_sms, cudaStream_t st, int* launches);
+
 // router: softmax -> top-k (lower index on ties) -> optional renormalisation,
 // plus the shared-expert column; one warp per token, E <= 1024, k + shared <= 32
 cudaError_t launch_router_topk(const View2& logits, int64_t T, int E, int k, int renorm, int shared,

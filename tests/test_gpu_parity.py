@@ -366,7 +366,7 @@ def test_decode_weight_prefetch_matches_oracle_and_unprefetched(T, k, idt):
     moe.device_errors()
     outs = {}
     for pre in (1, 0):
-        with moe.config_override((T, H, I, E, k), prefetch=pre):
+        with moe.config_override((T, H, I, E, k), prefetch=pre, fused=0):
             assert moe.get_config(T, H, I, E, k)["prefetch"] == pre
             outs[pre] = run_gpu(c)
     nbad, nto = moe.device_errors()
@@ -401,7 +401,7 @@ def test_decode_align_permute_one_launch_matches_two(T, k, idt, tile, strided):
     moe.device_errors()
     outs, launches = {}, {}
     for tiny in (1, 0):
-        with moe.config_override((T, H, I, E, k), tiny=tiny, **extra):
+        with moe.config_override((T, H, I, E, k), tiny=tiny, fused=0, **extra):
             outs[tiny] = run_gpu(c)
             launches[tiny] = moe.last_launch_count()
     nbad, nto = moe.device_errors()
@@ -410,3 +410,67 @@ def test_decode_align_permute_one_launch_matches_two(T, k, idt, tile, strided):
     assert rel_err(outs[1], ref) <= BF16_TOL
     assert launches[0] == 5
     assert launches[1] == (4 if T * k <= 32 else 5)
+
+
+@pytest.mark.parametrize("T,H,I,E,k,idt,case", [
+    (1, 512, 384, 24, 8, torch.int32, "plain"),
+    (4, 512, 384, 24, 8, torch.int64, "plain"),            # 32 slots, int64 ids
+    (3, 512, 384, 24, 10, torch.int32, "strided-ids"),     # ids read through a replay slice
+    (2, 288, 96, 20, 16, torch.int32, "ragged"),           # H, I off the 256/128 tiles
+    (1, 512, 384, 40, 32, torch.int32, "one-expert"),      # all 32 slots to one expert (8 gathers)
+    (2, 512, 256, 8, 4, torch.int32, "no-valid-id"),       # every id out of range: out must be zero
+])
+def test_decode_one_kernel_matches_kernels_and_oracle(T, H, I, E, k, idt, case):
+    # at most 32 slots: the whole forward as one kernel (slots grouped in every CTA,
+    # token rows gathered from x, combine by the last CTA of each output tile) must
+    # give the multi-kernel path's bits and match the oracle
+    cs = make_case(T, H, I, E, k, seed=T + k + 211)
+    ids = cs["ids"].to(idt)
+    if case in ("plain", "strided-ids", "ragged"):
+        ids[0, 1] = E                                 # a skipped slot
+        ids[T - 1, 2] = ids[T - 1, 3]                 # one expert twice for a token
+    if case == "one-expert":
+        ids[:] = 5
+    if case == "no-valid-id":
+        ids[:] = -1
+    cs["ids"] = ids
+    c = to_cuda(cs)
+    if case == "strided-ids":
+        big = torch.zeros(T, 3, k, dtype=idt, device="cuda")
+        big[:, 1, :] = c["ids"]
+        c["ids"] = big[:, 1, :]
+    moe.device_errors()
+    outs, launches = {}, {}
+    for fused in (1, 0):
+        with moe.config_override((T, H, I, E, k), fused=fused):
+            out = torch.full((T, H), 7.0, dtype=torch.bfloat16, device="cuda")  # stale contents
+            outs[fused] = run_gpu(c, out=out)
+            launches[fused] = moe.last_launch_count()
+    nbad, nto = moe.device_errors()
+    n_skip = int(((ids < 0) | (ids >= E)).sum().item())
+    assert nbad == 2 * n_skip and nto == 0
+    assert launches[1] == 1 and launches[0] == 4
+    assert torch.equal(outs[1], outs[0])
+    if case == "no-valid-id":
+        assert bool((outs[1] == 0).all())
+    else:
+        assert rel_err(outs[1], run_oracle(cs)) <= BF16_TOL
+
+
+def test_decode_one_kernel_repeated_calls_and_fallback_for_strided_x():
+    # the kernel's cross-CTA counters are reset by its last CTA: back-to-back calls
+    # (more than the counter sets in the library) keep giving the same bits; an x
+    # whose rows TMA cannot gather runs the multi-kernel path instead
+    T, H, I, E, k = 3, 512, 384, 24, 8
+    cs = make_case(T, H, I, E, k, seed=401)
+    c = to_cuda(cs)
+    first = run_gpu(c)
+    assert moe.last_launch_count() == 1
+    for _ in range(40):
+        assert torch.equal(run_gpu(c), first)
+    xs = cs["x"].t().contiguous().cuda().t()
+    c2 = dict(c, x=xs)
+    got = run_gpu(c2)
+    assert moe.last_launch_count() == 4
+    assert torch.equal(got, first)
+    assert rel_err(first, run_oracle(cs)) <= BF16_TOL

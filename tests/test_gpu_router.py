@@ -100,13 +100,17 @@ def test_router_then_forward_on_the_same_stream_decode():
         ids = torch.zeros(T, k, dtype=torch.int32, device="cuda")
         wts = torch.zeros(T, k, dtype=torch.float32, device="cuda")
         outs = {}
-        for pre in (1, 0):
-            with moe.config_override((T, H, I, E, k), prefetch=pre):
+        for name, flags in (("prefetch", dict(prefetch=1, fused=0)),
+                            ("no-prefetch", dict(prefetch=0, fused=0)),
+                            ("one-kernel", dict(fused=1))):
+            with moe.config_override((T, H, I, E, k), **flags):
                 ids.fill_(0)                     # stale routing the prefetch could see
                 moe.router_topk(logits, k, topk_ids=ids, topk_weights=wts)
-                outs[pre] = moe.forward(x, v, w2, ids, wts)
+                outs[name] = moe.forward(x, v, w2, ids, wts)
                 torch.cuda.synchronize()
-        assert torch.equal(outs[1], outs[0]), trial
+        assert torch.equal(outs["prefetch"], outs["no-prefetch"]), trial
+        assert torch.equal(outs["one-kernel"], outs["no-prefetch"]), trial
+        outs[1] = outs["prefetch"]
         if trial < 4:
             rid, rw = oracle.router_topk(logits.cpu(), k)
             gate, up = wl.gate_up_views(w13.cpu())
