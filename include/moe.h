@@ -327,11 +327,12 @@ typedef struct {
   int32_t tiny;        /* at most 32 slots: align and permute in one launch */
   int32_t prefetch;    /* at most 32 slots, 32-row tiles: GEMM1 requests its first weight
                           stages before align has finished (checked against align after) */
-  int32_t fused;       /* bf16, at most 32 slots: the whole forward as one kernel (slots
-                          grouped in every CTA, token rows gathered from x, GEMM2 weights
-                          streamed across the GEMM1 hand-off, combine by the last CTA of
-                          each output tile); needs x with unit inner stride and 16-byte
-                          aligned rows and H <= 16384, else the kernels above run */
+  int32_t fused;       /* at most 32 slots: the whole forward as one kernel (slots grouped
+                          in every CTA, token rows gathered from x (bf16) or quantised from
+                          x in the kernel (MXFP4), GEMM2 weights streamed across the GEMM1
+                          hand-off, combine by the last CTA of each output tile); bf16
+                          needs x with unit inner stride and 16-byte aligned rows; both
+                          need H <= 16384; otherwise the kernels above run */
 } moe_config_t;
 
 /* Installs a process-wide configuration table (copied; n = 0 removes it).

@@ -445,6 +445,50 @@ moe_status_t forward_mxfp4(const moe_tensor_t* x, const moe_w13_t* w13, const mo
                  CU_TENSOR_MAP_SWIZZLE_128B);
     if (s != MOE_OK) return s;
   }
+  if (cfg.fused && L.S <= 32 && pr.H <= 16384) {
+    // one kernel for decode sizes: h codes of each slot are gathered by TMA
+    CUtensorMap mHc;
+    const uint32_t box1[2] = {128, 1};
+    const uint64_t dh[2] = {uint64_t(pr.I / 2), 32};
+    const uint64_t sh[1] = {uint64_t(pr.I / 2)};
+    s = make_map(&mHc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w + L.h, dh, sh, box1,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s != MOE_OK) return s;
+    DecodeMxArgs dp;
+    dp.T = pr.T;
+    dp.H = pr.H;
+    dp.I = pr.I;
+    dp.E = pr.E;
+    dp.k = pr.k;
+    dp.ids = view2(ids);
+    dp.topk_w = view2(wts);
+    dp.x = view2(x);
+    dp.gate_sf = static_cast<const uint8_t*>(gate->scale);
+    dp.gate_s0 = gate->scale_strides[0];
+    dp.gate_s1 = gate->scale_strides[1];
+    dp.up_sf = static_cast<const uint8_t*>(up->scale);
+    dp.up_s0 = up->scale_strides[0];
+    dp.up_s1 = up->scale_strides[1];
+    dp.w2_sf = static_cast<const uint8_t*>(w2->scale);
+    dp.w2_s0 = w2->scale_strides[0];
+    dp.w2_s1 = w2->scale_strides[1];
+    dp.h_codes = w + L.h;
+    dp.h_sf = w + L.h_scale;
+    dp.y_ws = reinterpret_cast<__nv_bfloat16*>(w + L.y);
+    dp.out = static_cast<__nv_bfloat16*>(out->data);
+    dp.os0 = out->strides[0];
+    dp.os1 = out->strides[1];
+    dp.err = dev->errors;
+    t_prof.n = 0;
+    t_prof.have = false;
+    prof_mark(st);
+    const cudaError_t rc = launch_decode_fused_mx(mGate, mUp, mW2, mHc, dp, dev->num_sms, st, &launches);
+    if (rc != cudaSuccess) return cuda_fail(rc, "decode_fused_mxfp4");
+    for (int i = 0; i < kProfSteps; ++i) prof_mark(st);
+    t_prof.have = t_prof.on && t_prof.n == kProfSteps + 1;
+    t_last_launches = launches;
+    return MOE_OK;
+  }
   AlignTiles tiles;
   std::memset(&tiles, 0, sizeof(tiles));
   tiles.list[0].tile_max = cfg.tile;

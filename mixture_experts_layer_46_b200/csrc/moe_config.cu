@@ -69,6 +69,7 @@ moe_config_t heuristic(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, bo
   const int64_t S = T * k;
   const int64_t avg = E > 0 ? S / E : 0;
   c.tiny = S <= 32 ? 1 : 0;
+  c.fused = S <= 32 ? 1 : 0;
   if (mxfp4) {
     c.tile = avg <= 8 ? 32 : 96;
     return c;
@@ -78,7 +79,6 @@ moe_config_t heuristic(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, bo
   c.g2_single = c.pair;
   c.g1_256 = (c.g2_single && avg >= 96) ? 1 : 0;
   c.prefetch = (c.tile == 32 && S <= 32) ? 1 : 0;
-  c.fused = S <= 32 ? 1 : 0;
   return c;
 }
 
@@ -106,7 +106,7 @@ moe_config_t select_config(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k
   // what the kernels can run: flags that do not apply to the chosen tile are cleared
   const int64_t S = T * k;
   if (mxfp4) {
-    c.pair = c.g1_256 = c.g2_single = c.prefetch = c.fused = 0;
+    c.pair = c.g1_256 = c.g2_single = c.prefetch = 0;
   } else {
     if (c.tile == 256) c.pair = 1;  // 256-row token tiles exist only on CTA pairs
     if (c.tile == 32) c.pair = 0;

@@ -28,6 +28,7 @@
 // call slot (kDecodeSlots sets, dealt round-robin), and the last CTA to exit
 // resets them, so each launch finds them zero.
 #include <atomic>
+#include <mutex>
 
 #include "../../include/moe.h"
 #include "moe_internal.h"
@@ -52,14 +53,15 @@ constexpr int kMaxOutTiles = 64;             // H <= 16384
 constexpr size_t kSmem = 1024 + size_t(kStages) * kStageBytes + kEpiWarps * kStagingBytes +
                          (2 * kStages + 7) * 8 + 16 + 3 * 32 * 4 + 16;
 
-struct DecodeSync {
-  unsigned int g1[32];             // GEMM1 items finished, per routed expert
-  unsigned int g2[kMaxOutTiles];   // GEMM2 items finished, per 256-column output tile
-  unsigned int exit_cnt;           // CTAs finished
-  unsigned int pad[31];
-};
-constexpr int kDecodeSlots = 16;
+static_assert(sizeof(DecodeSync::g2) / sizeof(unsigned) == kMaxOutTiles, "counter sets");
+
+}  // namespace
+
+// The counter sets of the decode kernels: library memory, zero at load, left
+// zero by every launch (its last CTA resets the set it used).
 __device__ DecodeSync g_decode_sync[kDecodeSlots];
+
+namespace {
 
 struct DecArgs {
   int64_t T, H, I, E, k;
@@ -489,8 +491,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 std::atomic<unsigned> g_next_slot{0};
+std::mutex g_sync_mu;
+DecodeSync* g_sync_addr[64] = {};
 
 }  // namespace
+
+unsigned next_decode_slot() { return g_next_slot.fetch_add(1u) % kDecodeSlots; }
+
+DecodeSync* decode_sync_sets() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(g_sync_mu);
+  if (!g_sync_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_sync) != cudaSuccess) return nullptr;
+    g_sync_addr[dev] = static_cast<DecodeSync*>(p);
+  }
+  return g_sync_addr[dev];
+}
 
 cudaError_t launch_decode_fused(const CUtensorMap& gate, const CUtensorMap& up, const CUtensorMap& w2,
                                 const CUtensorMap& x1, const CUtensorMap& h1, const DecodeArgs& p,
@@ -520,7 +538,7 @@ cudaError_t launch_decode_fused(const CUtensorMap& gate, const CUtensorMap& up, 
   g.os0 = p.os0;
   g.os1 = p.os1;
   g.vec_out = (p.os1 == 1 && (p.os0 * 2) % 16 == 0 && reinterpret_cast<uintptr_t>(p.out) % 16 == 0) ? 1 : 0;
-  g.slot = static_cast<int32_t>(g_next_slot.fetch_add(1u) % kDecodeSlots);
+  g.slot = static_cast<int32_t>(next_decode_slot());
   g.err = p.err;
   if (launches) *launches += 1;
   return launch_pdl(moe_decode_fused_kernel, dim3(static_cast<unsigned>(num_sms)), dim3(kThreads), kSmem,

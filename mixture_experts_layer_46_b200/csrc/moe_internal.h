@@ -189,6 +189,42 @@ cudaError_t launch_decode_fused(const CUtensorMap& gate, const CUtensorMap& up, 
                                 const CUtensorMap& x1, const CUtensorMap& h1, const DecodeArgs& p,
                                 int num_sms, cudaStream_t st, int* launches);
 
+// Cross-CTA counters of the one-kernel decode paths: kDecodeSlots sets in
+// library memory, dealt round-robin to calls; each launch's last CTA resets its set.
+struct DecodeSync {
+  unsigned int g1[32];   // GEMM1 items finished, per routed expert
+  unsigned int g2[64];   // GEMM2 items finished, per 256-column output tile
+  unsigned int exit_cnt; // CTAs finished
+  unsigned int pad[31];
+};
+constexpr int kDecodeSlots = 16;
+unsigned next_decode_slot();
+DecodeSync* decode_sync_sets();  // device address on the current device (null on error)
+
+// the MXFP4 forward as one kernel for at most 32 routing slots
+struct DecodeMxArgs {
+  int64_t T, H, I, E, k;
+  View2 ids, topk_w, x;
+  const uint8_t* gate_sf;
+  int64_t gate_s0, gate_s1;
+  const uint8_t* up_sf;
+  int64_t up_s0, up_s1;
+  const uint8_t* w2_sf;
+  int64_t w2_s0, w2_s1;
+  uint8_t* h_codes;  // [32, I/2] workspace rows (by slot)
+  uint8_t* h_sf;     // [32, I/32]
+  __nv_bfloat16* y_ws;
+  __nv_bfloat16* out;
+  int64_t os0, os1;
+  DeviceErrors* err;
+};
+// maps: gate/up/w2 code maps ([128 B x 128] boxes), hc = h codes [32, I/2] bytes with a
+// one-row [128 x 1] box (read by four-row gathers); grid = num_sms
+cudaError_t launch_decode_fused_mx(const CUtensorMap& gate, const CUtensorMap& up,
+                                   const CUtensorMap& w2, const CUtensorMap& hc,
+                                   const DecodeMxArgs& p, int num_sms, cudaStream_t st,
+                                   int* launches);
+
 // router: softmax -> top-k (lower index on ties) -> optional renormalisation,
 // plus the shared-expert column; one warp per token, E <= 1024, k + shared <= 32
 cudaError_t launch_router_topk(const View2& logits, int64_t T, int E, int k, int renorm, int shared,

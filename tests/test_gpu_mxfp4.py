@@ -170,7 +170,7 @@ def test_mxfp4_decode_align_permute_one_launch_matches_two(T, k, strided):
     moe.device_errors()
     outs, launches = {}, {}
     for tiny in (1, 0):
-        with moe.config_override((T, H, I, E, k), mxfp4=True, tiny=tiny):
+        with moe.config_override((T, H, I, E, k), mxfp4=True, tiny=tiny, fused=0):
             outs[tiny] = mx_gpu(c)
             launches[tiny] = moe.last_launch_count()
     nbad, nto = moe.device_errors()
@@ -179,6 +179,45 @@ def test_mxfp4_decode_align_permute_one_launch_matches_two(T, k, strided):
     assert rel_err(outs[1], ref) <= MX_TOL
     assert launches[0] == 5
     assert launches[1] == (4 if T * k <= 32 else 5)
+
+
+@pytest.mark.parametrize("T,H,I,E,k,case", [
+    (1, 512, 256, 24, 10, "plain"),
+    (3, 512, 512, 24, 10, "strided-x"),       # x read through strides by the quantising warp
+    (2, 512, 256, 25, 11, "shared"),          # 24 routed + 1 shared expert, top 10 + 1
+    (1, 256, 256, 40, 32, "one-expert"),      # all 32 slots to one expert (8 gathers of h rows)
+    (2, 256, 256, 8, 4, "no-valid-id"),
+])
+def test_mxfp4_decode_one_kernel_matches_kernels_and_oracle(T, H, I, E, k, case):
+    # at most 32 slots: the MXFP4 forward as one kernel (tokens quantised in the
+    # kernel with the permute's rule, h requantised by the GEMM1 epilogue's rule)
+    # must give the multi-kernel path's bits and match the oracle
+    cs = make_mx_case(T, H, I, E, k, seed=T + k + 307, shared=(case == "shared"))
+    if case in ("plain", "strided-x"):
+        cs["ids"][0, 1] = E                           # a skipped slot
+        cs["ids"][T - 1, 2] = cs["ids"][T - 1, 3]     # one expert twice for a token
+    if case == "one-expert":
+        cs["ids"][:] = 7
+    if case == "no-valid-id":
+        cs["ids"][:] = -1
+    c = cuda_case(cs)
+    if case == "strided-x":
+        c["x"] = cs["x"].t().contiguous().cuda().t()
+    moe.device_errors()
+    outs, launches = {}, {}
+    for fused in (1, 0):
+        with moe.config_override((T, H, I, E, k), mxfp4=True, fused=fused):
+            outs[fused] = mx_gpu(c)
+            launches[fused] = moe.last_launch_count()
+    nbad, nto = moe.device_errors()
+    n_skip = int(((cs["ids"] < 0) | (cs["ids"] >= E)).sum().item())
+    assert nbad == 2 * n_skip and nto == 0
+    assert launches[1] == 1 and launches[0] == 4
+    assert torch.equal(outs[1], outs[0])
+    if case == "no-valid-id":
+        assert bool((outs[1] == 0).all())
+    else:
+        assert rel_err(outs[1], mx_oracle(cs)) <= MX_TOL
 
 
 def test_mxfp4_shared_expert_fused_routing():
