@@ -301,6 +301,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int my_slot = lane < cnt ? nth_bit(mask, lane) : -1;  // token row `lane` of the tile
       bool ready = g1;
       int pend_stage[kStages], pend_kb[kStages], npend = 0;
+      // 32 bf16 of x: block (idx % 8) of this k-step for the tile's token row idx / 8
+      auto load_x_block = [&](int idx, int kb, float (&v)[32]) {
+        const int q = idx >> 3, b = idx & 7;
+        const int64_t t = nth_bit(mask, q) / g.k;
+        const int64_t c0 = static_cast<int64_t>(kb) * 256 + b * 32;
+        if (g.vec_x) {
+          const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(g.x.data) + t * g.x.s0 + c0);
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) {
+            const uint4 w4v = __ldg(src + qq);
+            const uint32_t w4[4] = {w4v.x, w4v.y, w4v.z, w4v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              v[qq * 8 + 2 * i] = __uint_as_float((w4[i] & 0xffffu) << 16);
+              v[qq * 8 + 2 * i + 1] = __uint_as_float(w4[i] & 0xffff0000u);
+            }
+          }
+        } else {
+          const uint16_t* src = static_cast<const uint16_t*>(g.x.data) + t * g.x.s0;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            v[i] = __uint_as_float(static_cast<uint32_t>(src[(c0 + i) * g.x.s1]) << 16);
+        }
+      };
       // the h scale bytes of the tile's token rows, written by other CTAs during
       // this kernel: read from L2 (a line of L1 could hold an older copy of a
       // neighbouring slot's row) and stored into the token scale atoms
@@ -328,6 +352,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           npend = 0;
           ready = true;
         }
+        // GEMM1: this lane's first x block of the k-step is loaded before the
+        // wait for the stage, so its latency overlaps the wait
+        float v[32];
+        const bool early = g1 && lane < cnt * 8;
+        if (early) load_x_block(lane, kb, v);
         if (!mbar_wait(&empty[stage], phase ^ 1u, g.err)) { ok = false; break; }
         uint8_t* st_base = stages + stage * kStageBytes;
         const uint32_t sf = smem_u32(st_base + 2 * kWBytes + kXBytes);
@@ -353,28 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* sfx = st_base + 2 * kWBytes + kXBytes + 2 * kSfBytes;
           for (int idx = lane; idx < cnt * 8; idx += 32) {
             const int q = idx >> 3, b = idx & 7;
-            const int s = nth_bit(mask, q);
-            const int64_t t = s / g.k;
-            const int64_t c0 = static_cast<int64_t>(kb) * 256 + b * 32;
-            float v[32];
-            if (g.vec_x) {
-              const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(g.x.data) + t * g.x.s0 + c0);
-#pragma unroll
-              for (int qq = 0; qq < 4; ++qq) {
-                const uint4 w4v = __ldg(src + qq);
-                const uint32_t w4[4] = {w4v.x, w4v.y, w4v.z, w4v.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  v[qq * 8 + 2 * i] = __uint_as_float((w4[i] & 0xffffu) << 16);
-                  v[qq * 8 + 2 * i + 1] = __uint_as_float(w4[i] & 0xffff0000u);
-                }
-              }
-            } else {
-              const uint16_t* src = static_cast<const uint16_t*>(g.x.data) + t * g.x.s0;
-#pragma unroll
-              for (int i = 0; i < 32; ++i)
-                v[i] = __uint_as_float(static_cast<uint32_t>(src[(c0 + i) * g.x.s1]) << 16);
-            }
+            if (idx != lane) load_x_block(idx, kb, v);
             uint32_t wq[4];
             const uint32_t sc = mx_quant32(v, wq);
             *reinterpret_cast<uint4*>(sx + (q >> 3) * 1024 + (q & 7) * 128 + ((b ^ (q & 7)) * 16)) =

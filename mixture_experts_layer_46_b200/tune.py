@@ -56,9 +56,11 @@ def candidates(T: int, k: int, mxfp4: bool):
     tinies = (1, 0) if decode else (0,)
     out = []
     if mxfp4:
+        if decode:
+            out.append(dict(tile=32, fused=1))
         for tile in (32, 96):
             for tiny in tinies:
-                out.append(dict(tile=tile, tiny=tiny))
+                out.append(dict(tile=tile, tiny=tiny, fused=0))
         return out
     if decode:
         out.append(dict(tile=32, fused=1))
