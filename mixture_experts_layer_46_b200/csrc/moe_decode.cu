@@ -14,10 +14,11 @@
 //       per slot in the workspace; then the expert's GEMM1 counter is raised.
 //   GEMM2 item (routed expert r, 256 rows ot of H): two w2 slices, the
 //       expert's h rows as the token tile; y = w_slot * acc in bf16 per slot.
-//       Its w2 tiles are requested into L2 when the kernel starts (GEMM1's
-//       weights, read once, stream with evict-first), and its stages are
-//       filled at once: only the h rows wait for the expert's GEMM1 counter,
-//       so weights keep streaming across the GEMM1 -> GEMM2 hand-off.  Then the output tile's counter is
+//       Its weight stages are requested at once: only the h rows wait for the
+//       expert's GEMM1 counter to be complete, so weights keep streaming
+//       across the GEMM1 -> GEMM2 hand-off.  (Requesting all of GEMM2's w2
+//       tiles into L2 at kernel start was measured slower: the extra traffic
+//       slowed GEMM1's stream more than it sped up GEMM2.)  Then the output tile's counter is
 //       raised; the CTA that completes it (the last of the routed experts for
 //       those 256 columns) sums each token's k slot rows in fixed j order in
 //       fp32 and writes out[t, ot] (the same order and rounding as the combine
@@ -101,16 +102,6 @@ __device__ __forceinline__ bool wait_count(const unsigned int* p, unsigned want,
       return false;
     }
   }
-}
-
-// Requests a [64 x 128 x 1] box of a 3-D map into L2 (no shared memory written).
-__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int32_t c0, int32_t c1,
-                                                   int32_t c2, uint64_t hint) {
-  asm volatile(
-      "cp.async.bulk.prefetch.tensor.3d.L2.global.tile.L2::cache_hint [%0, {%1, %2, %3}], %4;" ::"l"(
-          reinterpret_cast<uint64_t>(map)),
-      "r"(c0), "r"(c1), "r"(c2), "l"(hint)
-      : "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async_global() {
@@ -232,19 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t stage = 0, phase = 0;
       int8_t last_phase[kStages];
       for (int s = 0; s < kStages; ++s) last_phase[s] = -1;
-      // GEMM2's w2 tiles cannot be consumed before h exists, but they can be
-      // on their way into L2 while GEMM1 streams: request them all now (kept
-      // there with evict-last) and stream GEMM1's weights, read once, evict-first
       const uint64_t pol = l2_policy_evict_last();
-      const uint64_t pol_once = l2_policy_evict_first();
-      for (int u = blockIdx.x; u < n_items; u += gridDim.x) {
-        if (u < n1) continue;
-        const int r = (u - n1) / n_wt2, wt = (u - n1) - r * n_wt2;
-        for (int kb = 0; kb < num_k2; ++kb) {
-          tma_prefetch_l2_3d(&tmW2, kb * kBK, wt * 2 * kWRows, d_e[r], pol);
-          tma_prefetch_l2_3d(&tmW2, kb * kBK, wt * 2 * kWRows + kWRows, d_e[r], pol);
-        }
-      }
       bool ok = true;
       for (int u = blockIdx.x; u < n_items && ok; u += gridDim.x) {
         const bool g1 = u < n1;
@@ -293,8 +272,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* sw1 = sw0 + kWBytes;
           if (g1) {
             mbar_arrive_expect_tx(&full[stage], 2 * kWBytes + tok_bytes);
-            tma_load_3d(sw0, &tmGate, &full[stage], kb * kBK, wt * kWRows, e, pol_once);
-            tma_load_3d(sw1, &tmUp, &full[stage], kb * kBK, wt * kWRows, e, pol_once);
+            tma_load_3d(sw0, &tmGate, &full[stage], kb * kBK, wt * kWRows, e, pol);
+            tma_load_3d(sw1, &tmUp, &full[stage], kb * kBK, wt * kWRows, e, pol);
             load_tokens(stage, kb);
           } else if (!ready) {
             mbar_expect_tx(&full[stage], 2 * kWBytes);

@@ -8,8 +8,9 @@
 //   GEMM1 item (routed expert r, 128 rows wt of I): gate/up code boxes
 //       [128 B x 128 rows] from the expert-strided views, their scales copied
 //       into the tensor cores' scale atoms, and the expert's token rows
-//       quantised straight from x into the stage (the 1x32 rule of the
-//       quantising permute, written at their 128-byte-swizzled positions);
+//       quantised from x (the 1x32 rule of the quantising permute), once per
+//       item into a shared buffer when they fit (else per k-step), and copied
+//       into each stage at their 128-byte-swizzled positions;
 //       h = silu(G) * U requantised per 1x32 along I into per-slot rows of the
 //       workspace; then the expert's GEMM1 counter is raised.
 //   GEMM2 item (routed expert r, 256 rows ot of H): two w2 slices (codes by
@@ -51,8 +52,11 @@ constexpr int kTmemCols = 256;
 static_assert(kSfCol0 + kStages * kSfColsPerStage <= kTmemCols, "TMEM budget");
 constexpr int kStagingBytes = 32 * 64;
 constexpr int kMaxOutTiles = 64;
+// a GEMM1 item's token rows, quantised once for all its k-steps (codes [cnt, H/2],
+// then scales [cnt, H/32]) when they fit; else they are quantised per k-step
+constexpr int kXbufBytes = 16 * 1024;
 constexpr size_t kSmem = 1024 + size_t(kStages) * kStageBytes + kEpiWarps * kStagingBytes +
-                         (2 * kStages + 7) * 8 + 16 + 3 * 32 * 4 + 16;
+                         kXbufBytes + (2 * kStages + 7) * 8 + 16 + 3 * 32 * 4 + 16;
 
 struct MxDecArgs {
   int64_t T, H, I, E, k;
@@ -129,7 +133,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = base;
   uint8_t* staging = base + kStages * kStageBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(staging + kEpiWarps * kStagingBytes);
+  uint8_t* xbuf = staging + kEpiWarps * kStagingBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(xbuf + kXbufBytes);
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
@@ -341,6 +346,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("st.shared.u32 [%0], %1;" ::"r"(sfx + kAtomBytes + 16 * lane), "r"(b) : "memory");
         fence_proxy_async_smem();
       };
+      // GEMM1: quantise the item's token rows once, for all its k-steps
+      const int64_t rb = g.H / 2, sbytes = g.H / 32;
+      const bool use_buf = g1 && cnt * (rb + sbytes) <= kXbufBytes;
+      __syncwarp();  // every lane is done with the previous item's buffer
+      if (use_buf) {
+        const int nb = static_cast<int>(g.H / 32);
+        for (int idx = lane; idx < cnt * nb; idx += 32) {
+          const int q = idx / nb, b = idx - q * nb;
+          float v[32];
+          load_x_block(q * 8 + (b & 7), b >> 3, v);  // row q, k-step b / 8, block b % 8
+          uint32_t wq[4];
+          const uint32_t sc = mx_quant32(v, wq);
+          *reinterpret_cast<uint4*>(xbuf + q * rb + b * 16) = make_uint4(wq[0], wq[1], wq[2], wq[3]);
+          xbuf[cnt * rb + q * sbytes + b] = static_cast<uint8_t>(sc);
+        }
+        __syncwarp();
+      }
       for (int kb = 0; kb < num_k && ok; ++kb) {
         if (!ready && npend == kStages) {
           if (!wait_count(&sync.g1[r], static_cast<unsigned>(n_wt1), g.err)) ok = false;
@@ -355,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // GEMM1: this lane's first x block of the k-step is loaded before the
         // wait for the stage, so its latency overlaps the wait
         float v[32];
-        const bool early = g1 && lane < cnt * 8;
+        const bool early = g1 && !use_buf && lane < cnt * 8;
         if (early) load_x_block(lane, kb, v);
         if (!mbar_wait(&empty[stage], phase ^ 1u, g.err)) { ok = false; break; }
         uint8_t* st_base = stages + stage * kStageBytes;
@@ -380,14 +402,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           // codes of block b of row q at 16-byte chunk b ^ (q % 8) (128-byte swizzle)
           uint8_t* sx = st_base + 2 * kWBytes;
           uint8_t* sfx = st_base + 2 * kWBytes + kXBytes + 2 * kSfBytes;
-          for (int idx = lane; idx < cnt * 8; idx += 32) {
-            const int q = idx >> 3, b = idx & 7;
-            if (idx != lane) load_x_block(idx, kb, v);
-            uint32_t wq[4];
-            const uint32_t sc = mx_quant32(v, wq);
-            *reinterpret_cast<uint4*>(sx + (q >> 3) * 1024 + (q & 7) * 128 + ((b ^ (q & 7)) * 16)) =
-                make_uint4(wq[0], wq[1], wq[2], wq[3]);
-            sfx[(b >> 2) * kAtomBytes + q * 16 + (b & 3)] = static_cast<uint8_t>(sc);
+          if (use_buf) {
+            // the k-step's 128 code bytes of each row and its 8 scale bytes, from the item's buffer
+            for (int idx = lane; idx < cnt * 8; idx += 32) {
+              const int q = idx >> 3, b = idx & 7;
+              *reinterpret_cast<uint4*>(sx + (q >> 3) * 1024 + (q & 7) * 128 + ((b ^ (q & 7)) * 16)) =
+                  *reinterpret_cast<const uint4*>(xbuf + q * rb + kb * 128 + b * 16);
+            }
+            if (lane < cnt) {
+              const uint32_t* sw = reinterpret_cast<const uint32_t*>(xbuf + cnt * rb + lane * sbytes + kb * 8);
+              *reinterpret_cast<uint32_t*>(sfx + lane * 16) = sw[0];
+              *reinterpret_cast<uint32_t*>(sfx + kAtomBytes + lane * 16) = sw[1];
+            }
+          } else {
+            for (int idx = lane; idx < cnt * 8; idx += 32) {
+              const int q = idx >> 3, b = idx & 7;
+              if (idx != lane) load_x_block(idx, kb, v);
+              uint32_t wq[4];
+              const uint32_t sc = mx_quant32(v, wq);
+              *reinterpret_cast<uint4*>(sx + (q >> 3) * 1024 + (q & 7) * 128 + ((b ^ (q & 7)) * 16)) =
+                  make_uint4(wq[0], wq[1], wq[2], wq[3]);
+              sfx[(b >> 2) * kAtomBytes + q * 16 + (b & 3)] = static_cast<uint8_t>(sc);
+            }
           }
           fence_proxy_async_smem();
           cp_async_mbar_arrive(&full[stage]);

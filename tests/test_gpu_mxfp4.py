@@ -286,13 +286,15 @@ def test_qwen35_tp2_mxfp4_token_sweep(tp2_weights, T, shared):
 
 
 def _ws_forward(case, T, H, I, E, k):
-    """moe_forward_ws with a caller workspace; returns (out, workspace, layout)."""
+    """moe_forward_ws with a caller workspace on the multi-kernel path (whose grouped
+    buffers live in the workspace); returns (out, workspace, layout)."""
     c = cuda_case(case)
     n = moe.workspace_bytes(T, H, I, E, k, mxfp4=True)
     ws = torch.full((n,), 0xAB, dtype=torch.uint8, device="cuda")
     v = moe.w13_from_packed(c["c13"], c["s13"])
-    out = moe.forward(c["x"], v, c["c2"], c["ids"], c["wts"], w2_scale=c["s2"], workspace=ws)
-    torch.cuda.synchronize()
+    with moe.config_override((T, H, I, E, k), mxfp4=True, fused=0):
+        out = moe.forward(c["x"], v, c["c2"], c["ids"], c["wts"], w2_scale=c["s2"], workspace=ws)
+        torch.cuda.synchronize()
     return out, ws, moe.workspace_layout(T, H, I, E, k, mxfp4=True)
 
 
@@ -324,6 +326,7 @@ def test_permute_quant_grouped_codes_bit_exact(T, H, I, E, k):
     scales = _region(ws, L["a1_scale"], rows, H // 32)
     ref_c, ref_s = oracle.mxfp4_quantize(case["x"].float())
     valid = inv >= 0
+    assert int(valid.sum()) == S - 1
     slot_tok = torch.arange(S)[valid] // k
     assert torch.equal(codes[inv[valid].long()], ref_c[slot_tok])
     assert torch.equal(scales[inv[valid].long()], ref_s[slot_tok])
@@ -347,6 +350,7 @@ def test_gemm1_h_requantisation_bit_exact(T, H, I, E, k):
     S = T * k
     inv = _region(ws, L["inv"], 1, S, torch.int32).flatten()
     rows = inv[inv >= 0].long()
+    assert rows.numel() == S
     h = cap.cpu()[rows]
     assert torch.isfinite(h).all()
     codes = _region(ws, L["h"], L["rows"], I // 2)[rows]
