@@ -341,6 +341,9 @@ def main():
     ap.add_argument("--E", type=int, default=None, help="override the expert count (profiling)")
     ap.add_argument("--sweep", default=None, help="write a token-sweep JSONL here (extra lines)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--config", default=None,
+                    help="override configuration flags of the timed forward, e.g. fused=1,tile=32 "
+                         "(installed with moe_set_config_table for this problem only)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -381,6 +384,10 @@ def main():
     def step():
         moe.forward(inp["x"], v13, inp["w2"], inp["ids"], inp["wts"], out=out, workspace=ws,
                     stream=stream, w2_scale=s2)
+
+    if args.config:
+        flags = {kv.split("=")[0]: int(kv.split("=")[1]) for kv in args.config.split(",")}
+        moe.config_override((w["T"], w["H"], w["I"], w["E"], w["k"]), mxfp4=mx, **flags).__enter__()
 
     for _ in range(args.warmup):
         step()
@@ -490,6 +497,7 @@ def main():
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e,
                     "api": "moe_forward_host (pinned host x/ids/weights in, host out)"},
             "gpu_launches": launches_per_step * args.steps,
+            "kernel_config": moe.get_config(w["T"], w["H"], w["I"], w["E"], w["k"], mxfp4=mx),
             "clocks": clocks}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -90,12 +90,15 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned int* p) {
   return v;
 }
 
-// Spins (bounded) until *p >= want; false on timeout (counted).
+// Spins (bounded) until *p >= want, backing off to one poll a microsecond so
+// that many waiting CTAs do not crowd the counter's L2 line; false on timeout (counted).
 __device__ __forceinline__ bool wait_count(const unsigned int* p, unsigned want, DeviceErrors* err) {
   if (ld_acquire(p) >= want) return true;
   const unsigned long long t0 = global_ns();
+  unsigned ns = 32;
   while (true) {
-    __nanosleep(64);
+    __nanosleep(ns);
+    if (ns < 1024) ns <<= 1;
     if (ld_acquire(p) >= want) return true;
     if (global_ns() - t0 > kWaitLimitNs) {
       if (err) atomicAdd(&err->timeouts, 1u);

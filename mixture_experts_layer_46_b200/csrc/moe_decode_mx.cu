@@ -90,17 +90,32 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned int* p) {
   return v;
 }
 
+// Spins (bounded) until *p >= want, backing off to one poll a microsecond so
+// that many waiting CTAs do not crowd the counter's L2 line; false on timeout (counted).
 __device__ __forceinline__ bool wait_count(const unsigned int* p, unsigned want, DeviceErrors* err) {
   if (ld_acquire(p) >= want) return true;
   const unsigned long long t0 = global_ns();
+  unsigned ns = 32;
   while (true) {
-    __nanosleep(64);
+    __nanosleep(ns);
+    if (ns < 1024) ns <<= 1;
     if (ld_acquire(p) >= want) return true;
     if (global_ns() - t0 > kWaitLimitNs) {
       if (err) atomicAdd(&err->timeouts, 1u);
       return false;
     }
   }
+}
+
+// The whole warp waits: lane 0 polls, the others follow through the warp barrier
+// (which orders lane 0's acquire before their later loads).
+__device__ __forceinline__ bool warp_wait_count(const unsigned int* p, unsigned want,
+                                                DeviceErrors* err, int lane) {
+  int ok = 1;
+  if (lane == 0) ok = wait_count(p, want, err) ? 1 : 0;
+  __syncwarp();
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  return ok != 0;
 }
 
 __device__ __forceinline__ void fence_proxy_async_global() {
@@ -365,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int kb = 0; kb < num_k && ok; ++kb) {
         if (!ready && npend == kStages) {
-          if (!wait_count(&sync.g1[r], static_cast<unsigned>(n_wt1), g.err)) ok = false;
+          if (!warp_wait_count(&sync.g1[r], static_cast<unsigned>(n_wt1), g.err, lane)) ok = false;
           for (int i = 0; i < npend; ++i) {
             h_scales(pend_stage[i], pend_kb[i]);
             cp_async_mbar_arrive(&full[pend_stage[i]]);
@@ -440,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
       }
       if (!ready && npend > 0) {
-        if (!wait_count(&sync.g1[r], static_cast<unsigned>(n_wt1), g.err)) ok = false;
+        if (!warp_wait_count(&sync.g1[r], static_cast<unsigned>(n_wt1), g.err, lane)) ok = false;
         for (int i = 0; i < npend; ++i) {
           h_scales(pend_stage[i], pend_kb[i]);
           cp_async_mbar_arrive(&full[pend_stage[i]]);
