@@ -320,7 +320,7 @@ typedef struct {
   int64_t H, I, E, k;  /* shape the entry applies to; 0 matches any value */
   int64_t t_lo, t_hi;  /* token bucket: applies when t_lo <= T <= t_hi */
   int32_t tile;        /* token-tile rows: 32, 128 or 256 (bf16; 256 runs on CTA pairs),
-                          32 or 96 (MXFP4) */
+                          32, 96 or 128 (MXFP4; 128 with one accumulator buffer) */
   int32_t pair;        /* bf16 128-row tiles: GEMMs on CTA pairs (tcgen05 cta_group::2) */
   int32_t g1_256;      /* bf16 pairs: GEMM1 on 256-row token tiles (needs g2_single) */
   int32_t g2_single;   /* bf16 pairs: GEMM2 with one 256-row w2 slice per 256-row tile */

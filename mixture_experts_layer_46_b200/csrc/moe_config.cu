@@ -37,7 +37,7 @@ bool matches(const moe_config_t& c, int64_t T, int64_t H, int64_t I, int64_t E, 
 }
 
 bool tile_ok(int32_t tile, bool mxfp4) {
-  return mxfp4 ? (tile == 32 || tile == 96) : (tile == 32 || tile == 128 || tile == 256);
+  return mxfp4 ? (tile == 32 || tile == 96 || tile == 128) : (tile == 32 || tile == 128 || tile == 256);
 }
 
 bool flag_ok(int32_t v) { return v == 0 || v == 1; }

@@ -469,6 +469,10 @@ cudaError_t launch_gemm_ws_mxfp4(int mode, int tile_max, const CUtensorMap& w0,
   g.err = p.err;
   if (launches) *launches += 1;
   const int64_t max_items = p.max_tiles * p.n_wt;
+  if (tile_max == 128) {  // one accumulator buffer: fewer weight re-reads, epilogue not overlapped
+    if (mode == 0) return launch_mx<0, 128, 4>(w0, w1, x, g, max_items, num_sms, st);
+    return launch_mx<1, 128, 4>(w0, w1, x, g, max_items, num_sms, st);
+  }
   if (tile_max == 96) {
     if (mode == 0) return launch_mx<0, 96, 4>(w0, w1, x, g, max_items, num_sms, st);
     return launch_mx<1, 96, 4>(w0, w1, x, g, max_items, num_sms, st);

@@ -58,7 +58,7 @@ def candidates(T: int, k: int, mxfp4: bool):
     if mxfp4:
         if decode:
             out.append(dict(tile=32, fused=1))
-        for tile in (32, 96):
+        for tile in (32, 96, 128):
             for tiny in tinies:
                 out.append(dict(tile=tile, tiny=tiny, fused=0))
         return out

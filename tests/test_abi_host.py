@@ -184,7 +184,7 @@ def test_config_table_lookup_and_fixed_workspace():
 
 def test_config_table_rejects_malformed_entries():
     bad = [moe.make_config(_abi.MOE_BF16, tile=64),            # no such tile
-           moe.make_config(_abi.MOE_E2M1X2, tile=128),         # MXFP4 tiles are 32 or 96
+           moe.make_config(_abi.MOE_E2M1X2, tile=256),         # MXFP4 tiles are 32, 96 or 128
            moe.make_config(_abi.MOE_BF16, tile=32, pair=2),    # flags are 0 or 1
            moe.make_config(_abi.MOE_BF16, t_lo=10, t_hi=5, tile=32),
            moe.make_config(7, tile=32)]

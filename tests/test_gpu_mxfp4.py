@@ -220,6 +220,25 @@ def test_mxfp4_decode_one_kernel_matches_kernels_and_oracle(T, H, I, E, k, case)
         assert rel_err(outs[1], mx_oracle(cs)) <= MX_TOL
 
 
+@pytest.mark.parametrize("T,H,I,E,k", [
+    (300, 512, 512, 8, 4),     # 150 slots per expert: several tiles of each size, ragged last tiles
+    (77, 256, 256, 6, 3),
+])
+def test_mxfp4_token_tile_configs_agree_and_match_oracle(T, H, I, E, k):
+    # 32- and 96-row tiles (two accumulator buffers) and 128-row tiles (one) are a
+    # performance choice of the block-scaled GEMMs: every one must give the same bits
+    case = make_mx_case(T, H, I, E, k, seed=T + 91)
+    ref = mx_oracle(case)
+    c = cuda_case(case)
+    outs = {}
+    for tile in (32, 96, 128):
+        with moe.config_override((T, H, I, E, k), mxfp4=True, tile=tile):
+            assert moe.get_config(T, H, I, E, k, mxfp4=True)["tile"] == tile
+            outs[tile] = mx_gpu(c)
+        assert rel_err(outs[tile], ref) <= MX_TOL, tile
+    assert torch.equal(outs[32], outs[96]) and torch.equal(outs[96], outs[128])
+
+
 def test_mxfp4_shared_expert_fused_routing():
     # E = 32 routed + 1 shared, top_k = 4 + 1, the 513/11 convention at reduced size
     case = make_mx_case(96, 512, 256, 33, 5, seed=7, shared=True)
