@@ -58,11 +58,14 @@ NCU_TRAFFIC = {
 }
 
 
-def kernel_src_hash() -> str:
+def kernel_src_hash(config: dict) -> str:
+    """Hash of the GEMM kernels' sources and of the configuration the timed forward ran:
+    a recorded traffic figure is reported only while both are unchanged."""
     h = hashlib.sha256()
-    for fn in ("moe_gemm_ws2.cu", "moe_common.cuh", "moe_api.cu"):
+    for fn in ("moe_gemm_ws.cu", "moe_gemm_ws2.cu", "moe_gemm_mxfp4.cu", "moe_common.cuh"):
         with open(os.path.join(ROOT, "mixture_experts_layer_46_b200", "csrc", fn), "rb") as f:
             h.update(f.read())
+    h.update(json.dumps({k: config[k] for k in sorted(config) if k not in ("t_lo", "t_hi")}).encode())
     return h.hexdigest()[:16]
 
 
@@ -462,10 +465,12 @@ def main():
         roof = {"bound": "hbm", "achieved": alg["gemm1_bytes"] / (g1_ms * 1e-3) / 1e9, "peak": hbm,
                 "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    tr = NCU_TRAFFIC.get("gemm1_swiglu")
-    same_case = (args.workload == "qwen3-235b" and w["T"] == 4096 and w["E"] == 128)
-    roof["traffic"] = (tr["bytes_per_launch"] if tr and same_case and tr.get("src") == kernel_src_hash()
+    tr = NCU_TRAFFIC.get(args.workload)
+    cfg_now = moe.get_config(w["T"], w["H"], w["I"], w["E"], w["k"], mxfp4=mx)
+    same_case = tr is not None and tr.get("T") == w["T"] and tr.get("E") == w["E"]
+    roof["traffic"] = (tr["bytes_per_launch"] if same_case and tr.get("src") == kernel_src_hash(cfg_now)
                        else None)
+    roof["traffic_src"] = kernel_src_hash(cfg_now)
     pair = (not mx) and (w["T"] * w["k"] >= 32 * w["E"])
     roof["kernel"] = ("gemm1_swiglu (weight-stationary grouped gate/up GEMM + SwiGLU, tcgen05 "
                       + ("kind::mxf4 block-scaled)" if mx else
