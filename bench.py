@@ -53,8 +53,12 @@ WORKLOADS = {
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed to the hash of the kernel
 # source it was taken on; reported as null once the source has changed.
 NCU_TRAFFIC = {
-    # filled from the ncu launch of GEMM1 on the benchmarked workload (T=4096, E=128),
-    # keyed to the hash of the kernel and host sources it was captured on
+    # GEMM1 on the benchmarked workload (T=4096, E=128, the table's configuration for that
+    # bucket), one-pass ncu capture at the full size: 4.28 GB read + 0.105 GB written per
+    # launch (profiles/launches_qwen3_235b_T4096.md); reported only while the GEMM sources and
+    # the configuration hash to `src`
+    "qwen3-235b": {"T": 4096, "E": 128, "bytes_per_launch": 4.28e9 + 0.10514e9,
+                   "src": "5e161c7fe4099a5d"},
 }
 
 
