@@ -55,8 +55,7 @@ WORKLOADS = {
 NCU_TRAFFIC = {
     # GEMM1 on the benchmarked workload (T=4096, E=128, the table's configuration for that
     # bucket), one-pass ncu capture at the full size: 4.28 GB read + 0.105 GB written per
-    # launch (profiles/launches_qwen3_235b_T4096.md); reported only while the GEMM sources and
-    # the configuration hash to `src`
+    # launch; reported only while the GEMM sources and the configuration hash to `src`
     "qwen3-235b": {"T": 4096, "E": 128, "bytes_per_launch": 4.28e9 + 0.10514e9,
                    "src": "5e161c7fe4099a5d"},
 }
