@@ -313,8 +313,12 @@ moe_status_t moe_profile_read(float* ms, int32_t capacity, int32_t* n);
  * latency": block_m per token bucket).  A forward looks its configuration up
  * in the table installed by moe_set_config_table, then in the table compiled
  * into the library from the committed tuning results, then falls back to a
- * heuristic.  Every configuration gives bit-identical results; only the speed
- * differs.  The workspace size (moe_workspace_bytes) does not depend on it. */
+ * heuristic.  Every configuration with split = 1 gives bit-identical results
+ * (the GEMMs sum each output in the same k order whatever the tiling); a
+ * one-kernel configuration whose GEMM1 is split along K sums the parts' fp32
+ * partials in fixed part order, so it is deterministic but may round
+ * differently.  The workspace size (moe_workspace_bytes) does not depend on
+ * the configuration. */
 typedef struct {
   int32_t wdtype;      /* MOE_BF16 or MOE_E2M1X2 */
   int64_t H, I, E, k;  /* shape the entry applies to; 0 matches any value */
@@ -333,6 +337,11 @@ typedef struct {
                           hand-off, combine by the last CTA of each output tile); bf16
                           needs x with unit inner stride and 16-byte aligned rows; both
                           need H <= 16384; otherwise the kernels above run */
+  int32_t split;       /* one-kernel path: GEMM1 split along K into at most this many parts
+                          (0 = the library's default, 4; 1 = not split).  The kernel takes
+                          as many as put about two GEMM1 units on every SM, with at least
+                          four 64-wide k-blocks per part; the unit that completes a (routed
+                          expert, 128-row) item sums all parts' fp32 partials in part order */
 } moe_config_t;
 
 /* Installs a process-wide configuration table (copied; n = 0 removes it).

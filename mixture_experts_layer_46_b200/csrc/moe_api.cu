@@ -392,6 +392,7 @@ WsLayout make_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, bool
   }
   L.y = take(size_t(p) * H * 2);
   L.w_row = take(mxfp4 ? sizeof(float) * size_t(p) : 0);
+  L.part = take(S <= 32 ? size_t(decode_part_bytes(I)) : 0);
   L.total = off;
   return L;
 }
@@ -478,6 +479,8 @@ moe_status_t forward_mxfp4(const moe_tensor_t* x, const moe_w13_t* w13, const mo
     dp.out = static_cast<__nv_bfloat16*>(out->data);
     dp.os0 = out->strides[0];
     dp.os1 = out->strides[1];
+    dp.part_ws = reinterpret_cast<float*>(w + L.part);
+    dp.max_split = cfg.split;
     dp.err = dev->errors;
     t_prof.n = 0;
     t_prof.have = false;
@@ -692,6 +695,8 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
     dp.out = static_cast<__nv_bfloat16*>(out->data);
     dp.os0 = out->strides[0];
     dp.os1 = out->strides[1];
+    dp.part_ws = reinterpret_cast<float*>(w + L.part);
+    dp.max_split = cfg.split;
     dp.err = dev->errors;
     t_prof.n = 0;
     t_prof.have = false;

@@ -9,9 +9,10 @@
 //   2. the table compiled into the library from the committed tuning results
 //      (configs/b200_tuned.csv, turned into a C array at build time),
 //   3. a heuristic on the average number of routing slots per expert.
-// The first entry whose shape and token bucket match wins.  Every choice gives
-// bit-identical results (the GEMMs sum each output in the same k order whatever
-// the tiling), so the table only affects speed.
+// The first entry whose shape and token bucket match wins.  Every choice with
+// an unsplit GEMM1 gives bit-identical results (the GEMMs sum each output in
+// the same k order whatever the tiling); the one-kernel path's split GEMM1
+// sums its K parts in fixed order (deterministic, rounded differently).
 #include <mutex>
 #include <vector>
 
@@ -47,7 +48,7 @@ bool entry_ok(const moe_config_t& c) {
   if (c.H < 0 || c.I < 0 || c.E < 0 || c.k < 0 || c.t_lo < 0 || c.t_hi < c.t_lo) return false;
   if (!tile_ok(c.tile, c.wdtype == MOE_E2M1X2)) return false;
   return flag_ok(c.pair) && flag_ok(c.g1_256) && flag_ok(c.g2_single) && flag_ok(c.tiny) &&
-         flag_ok(c.prefetch) && flag_ok(c.fused);
+         flag_ok(c.prefetch) && flag_ok(c.fused) && c.split >= 0 && c.split <= kDecodeMaxSplit;
 }
 
 // The measured defaults of the kernels when no table entry matches: 32-row
@@ -98,7 +99,7 @@ moe_config_t select_config(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k
   }
   if (!found) {
     for (int i = 0; i < kNumBuiltinConfigs; ++i)
-      if (matches(kBuiltinConfigs[i], T, H, I, E, k, mxfp4)) {
+      if (entry_ok(kBuiltinConfigs[i]) && matches(kBuiltinConfigs[i], T, H, I, E, k, mxfp4)) {
         c = kBuiltinConfigs[i];
         break;
       }
@@ -115,6 +116,7 @@ moe_config_t select_config(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k
     if (!(c.tile == 32 && S <= 32)) c.prefetch = 0;
   }
   if (S > 32) c.tiny = c.fused = 0;
+  c.split = !c.fused ? 1 : (c.split == 0 ? kDecodeMaxSplit : c.split);
   return c;
 }
 

@@ -33,6 +33,7 @@
 #include <mutex>
 
 #include "../../include/moe.h"
+#include "moe_decode_units.cuh"
 #include "moe_internal.h"
 
 namespace moe {
@@ -74,6 +75,8 @@ struct DecArgs {
   int64_t os0, os1;
   int32_t vec_out;
   int32_t slot;          // counter set of this call
+  float* part_ws;        // GEMM1 split-K partials (layout of decode_part_bytes)
+  int32_t max_split;     // at most this many GEMM1 K parts
   DeviceErrors* err;
 };
 
@@ -216,9 +219,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nd = misc[0];
   const int n_wt1 = static_cast<int>((g.I + kWRows - 1) / kWRows);
   const int n_wt2 = static_cast<int>((g.H + 2 * kWRows - 1) / (2 * kWRows));
-  const int n1 = nd * n_wt1, n_items = n1 + nd * n_wt2;
+  const int n1 = nd * n_wt1;
   const int num_k1 = static_cast<int>((g.H + kBK - 1) / kBK);
   const int num_k2 = static_cast<int>((g.I + kBK - 1) / kBK);
+  const int ks = split_count(n1, num_k1, static_cast<int>(gridDim.x), g.max_split);
+  const int n_items = n1 * ks + nd * n_wt2;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -229,16 +234,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t pol = l2_policy_evict_last();
       bool ok = true;
       for (int u = blockIdx.x; u < n_items && ok; u += gridDim.x) {
-        const bool g1 = u < n1;
-        const int r = g1 ? u / n_wt1 : (u - n1) / n_wt2;
-        const int wt = g1 ? u - r * n_wt1 : (u - n1) - r * n_wt2;
+        const Unit x = unit_of(u, n1, ks, n_wt1, n_wt2, num_k1, num_k2);
+        const bool g1 = x.g1;
+        const int r = x.r, wt = x.wt;
         const int e = d_e[r], cnt = d_cnt[r];
         const unsigned mask = d_mask[r];
         // token rows go in groups of four (one gather each); a group's unused
         // entries repeat its first row, filling tile rows the MMA results skip
         const int n_groups = (cnt + 3) / 4;
         const uint32_t tok_bytes = static_cast<uint32_t>(n_groups) * 4 * kBK * 2;
-        const int num_k = g1 ? num_k1 : num_k2;
         // GEMM2: weights go out at once, the h rows only once the expert's h is complete
         bool ready = g1;
         int pend_stage[kStages], pend_kb[kStages], npend = 0;
@@ -268,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           npend = 0;
           ready = true;
         };
-        for (int kb = 0; kb < num_k && ok; ++kb) {
+        for (int kb = x.kb0; kb < x.kb1 && ok; ++kb) {
           if (!ready && npend == kStages) release_pending();
           if (!mbar_wait(&empty[stage], phase ^ 1u, g.err)) { ok = false; break; }
           uint8_t* sw0 = stages + stage * kStageBytes;
@@ -308,11 +312,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true, issued = false;
       const uint32_t idesc = idesc_bf16_f32(kWRows, kNtok);
       for (int u = blockIdx.x; u < n_items && ok; u += gridDim.x) {
-        const int num_k = u < n1 ? num_k1 : num_k2;
+        const Unit x = unit_of(u, n1, ks, n_wt1, n_wt2, num_k1, num_k2);
         if (!mbar_wait(&tempty[buf], acc_phase ^ 1u, g.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t acc0 = tmem_base + buf * 2 * kNtok, acc1 = acc0 + kNtok;
-        for (int kb = 0; kb < num_k; ++kb) {
+        for (int kb = x.kb0; kb < x.kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, g.err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t w0_addr = smem_u32(stages + stage * kStageBytes);
@@ -321,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
             const uint64_t xd = sw128_kmajor_desc(x_addr + kk * kUmmaK * 2);
-            const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+            const uint32_t acc = (kb > x.kb0 || kk > 0) ? 1u : 0u;
             mma_bf16(acc0, sw128_kmajor_desc(w0_addr + kk * kUmmaK * 2), xd, idesc, acc);
             mma_bf16(acc1, sw128_kmajor_desc(w1_addr + kk * kUmmaK * 2), xd, idesc, acc);
           }
@@ -354,9 +358,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     for (int u = blockIdx.x; u < n_items; u += gridDim.x) {
-      const bool g1 = u < n1;
-      const int r = g1 ? u / n_wt1 : (u - n1) / n_wt2;
-      const int wt = g1 ? u - r * n_wt1 : (u - n1) - r * n_wt2;
+      const Unit x = unit_of(u, n1, ks, n_wt1, n_wt2, num_k1, num_k2);
+      const bool g1 = x.g1;
+      const int r = x.r, wt = x.wt;
       const unsigned mask = d_mask[r];
       const int cnt = d_cnt[r];
       // the token column j of this tile is the slot my_slot (lane j holds it)
@@ -369,6 +373,98 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(&tfull[buf], acc_phase, g.err)) break;
       tc_fence_after();
       const uint32_t lane_base = (static_cast<uint32_t>(quad * 32) << 16) + buf * 2 * kNtok;
+      if (g1 && ks > 1) {
+        // ---- one K part of a GEMM1 item: park the fp32 partials; the unit that
+        // completes the item sums all parts in part order and writes h
+        uint32_t v0[32], v1[32];
+        tmem_ld32(tmem_base + lane_base, v0);
+        tmem_ld32(tmem_base + lane_base + kNtok, v1);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[buf]);
+        if (++buf == 2) { buf = 0; acc_phase ^= 1u; }
+        // this expert's token columns follow those of the routed experts before it
+        int colb = 0;
+        for (int q = 0; q < r; ++q) colb += d_cnt[q];
+        const int row = quad * 32 + lane;
+        const size_t tile_stride = static_cast<size_t>(n_wt1) * kNtok * 2 * kWRows;
+        float* pb = g.part_ws + x.part * tile_stride + (static_cast<size_t>(wt) * kNtok + colb) * 2 * kWRows + row;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          if (j >= cnt) break;
+          pb[j * 2 * kWRows] = __uint_as_float(v0[j]);
+          pb[j * 2 * kWRows + kWRows] = __uint_as_float(v1[j]);
+        }
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(epi_done);
+        if (et == 0) {
+          mbar_wait(epi_done, sync_phase, g.err);
+          __threadfence();
+          const unsigned old = atomicAdd(&sync.g1p[x.item], 1u);
+          misc[2] = (old + 1 == static_cast<unsigned>(ks)) ? 1 : 0;
+          __threadfence();
+          mbar_arrive(epi_last);
+        }
+        mbar_wait(epi_last, sync_phase, g.err);
+        const bool done_item = misc[2] != 0;
+        sync_phase ^= 1u;
+        if (!done_item) continue;
+        __threadfence();
+        float sg[32], su[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) sg[j] = su[j] = 0.0f;
+        for (int p = 0; p < ks; ++p) {
+          if (p == x.part) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              sg[j] += __uint_as_float(v0[j]);
+              su[j] += __uint_as_float(v1[j]);
+            }
+          } else {
+            const float* qb = pb + static_cast<ptrdiff_t>(p - x.part) * static_cast<ptrdiff_t>(tile_stride);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (j >= cnt) break;
+              sg[j] += __ldcg(qb + j * 2 * kWRows);
+              su[j] += __ldcg(qb + j * 2 * kWRows + kWRows);
+            }
+          }
+        }
+        const int64_t col0 = static_cast<int64_t>(wt) * kWRows + quad * 32;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const __nv_bfloat16 hb = __float2bfloat16_rn(silu_mul(sg[j], su[j]));
+          asm volatile("st.shared.b16 [%0], %1;" ::"r"(stg_s + j * 64 + lane * 2),
+                       "h"(*reinterpret_cast<const uint16_t*>(&hb)) : "memory");
+        }
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int idx = q * 32 + lane;
+          const int j = idx >> 2, part = idx & 3;
+          uint4 v;
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                       : "r"(stg_s + j * 64 + part * 16));
+          const int s_j = __shfl_sync(0xffffffffu, my_slot, j);
+          if (s_j >= 0 && col0 < g.I) *reinterpret_cast<uint4*>(g.h_ws + s_j * g.I + col0 + part * 8) = v;
+        }
+        __syncwarp();
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(epi_done);
+        if (et == 0) {
+          mbar_wait(epi_done, sync_phase, g.err);
+          __threadfence();
+          atomicAdd(&sync.g1[r], 1u);
+          mbar_arrive(epi_last);
+        }
+        mbar_wait(epi_last, sync_phase, g.err);
+        sync_phase ^= 1u;
+        continue;
+      }
       const int n_out = g1 ? 1 : 2;
       const int64_t ld = g1 ? g.I : g.H;
       __nv_bfloat16* dst = g1 ? g.h_ws : g.y_ws;
@@ -489,6 +585,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       __threadfence();
       for (int i = 0; i < 32; ++i) sync.g1[i] = 0u;
       for (int i = 0; i < kMaxOutTiles; ++i) sync.g2[i] = 0u;
+      if (ks > 1)
+        for (int i = 0; i < n1; ++i) sync.g1p[i] = 0u;
       __threadfence();
       sync.exit_cnt = 0u;
     }
@@ -544,6 +642,8 @@ cudaError_t launch_decode_fused(const CUtensorMap& gate, const CUtensorMap& up, 
   g.os1 = p.os1;
   g.vec_out = (p.os1 == 1 && (p.os0 * 2) % 16 == 0 && reinterpret_cast<uintptr_t>(p.out) % 16 == 0) ? 1 : 0;
   g.slot = static_cast<int32_t>(next_decode_slot());
+  g.part_ws = p.part_ws;
+  g.max_split = p.max_split;
   g.err = p.err;
   if (launches) *launches += 1;
   return launch_pdl(moe_decode_fused_kernel, dim3(static_cast<unsigned>(num_sms)), dim3(kThreads), kSmem,

@@ -23,6 +23,7 @@
 // 2 scale copies and token quantisation, 3-6 epilogue.  Every wait is bounded;
 // the cross-CTA counters are the decode slots' sets shared with moe_decode.cu.
 #include "../../include/moe.h"
+#include "moe_decode_units.cuh"
 #include "moe_internal.h"
 #include "moe_mx.cuh"
 
@@ -74,6 +75,8 @@ struct MxDecArgs {
   int64_t os0, os1;
   int32_t vec_x, vec_out;
   int32_t slot;
+  float* part_ws;        // GEMM1 split-K partials (layout of decode_part_bytes)
+  int32_t max_split;     // at most this many GEMM1 K parts
   DeviceErrors* err;
 };
 
@@ -221,9 +224,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nd = misc[0];
   const int n_wt1 = static_cast<int>(g.I / kWRows);        // I % 256 == 0 (validated)
   const int n_wt2 = static_cast<int>(g.H / (2 * kWRows));  // H % 256 == 0 (validated)
-  const int n1 = nd * n_wt1, n_items = n1 + nd * n_wt2;
+  const int n1 = nd * n_wt1;
   const int num_k1 = static_cast<int>(g.H / 256);
   const int num_k2 = static_cast<int>(g.I / 256);
+  const int ks = split_count(n1, num_k1, static_cast<int>(gridDim.x), g.max_split);
+  const int n_items = n1 * ks + nd * n_wt2;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -234,14 +239,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t pol = l2_policy_evict_last();
       bool ok = true;
       for (int u = blockIdx.x; u < n_items && ok; u += gridDim.x) {
-        const bool g1 = u < n1;
-        const int r = g1 ? u / n_wt1 : (u - n1) / n_wt2;
-        const int wt = g1 ? u - r * n_wt1 : (u - n1) - r * n_wt2;
+        const Unit x = unit_of(u, n1, ks, n_wt1, n_wt2, num_k1, num_k2);
+        const bool g1 = x.g1;
+        const int r = x.r, wt = x.wt;
         const int e = d_e[r], cnt = d_cnt[r];
         const unsigned mask = d_mask[r];
         const int n_groups = (cnt + 3) / 4;
         const uint32_t tok_bytes = g1 ? 0u : static_cast<uint32_t>(n_groups) * 4 * kRowBytes;
-        const int num_k = g1 ? num_k1 : num_k2;
         bool ready = g1;
         int pend_stage[kStages], pend_kb[kStages], npend = 0;
         auto load_h = [&](int st, int kb) {
@@ -269,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           npend = 0;
           ready = true;
         };
-        for (int kb = 0; kb < num_k && ok; ++kb) {
+        for (int kb = x.kb0; kb < x.kb1 && ok; ++kb) {
           if (!ready && npend == kStages) release_pending();
           if (!mbar_wait(&empty[stage], phase ^ 1u, g.err)) { ok = false; break; }
           uint8_t* sw0 = stages + stage * kStageBytes;
@@ -305,12 +309,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t stage = 0, phase = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_items && ok; u += gridDim.x) {
-      const bool g1 = u < n1;
-      const int r = g1 ? u / n_wt1 : (u - n1) / n_wt2;
-      const int wt = g1 ? u - r * n_wt1 : (u - n1) - r * n_wt2;
+      const Unit x = unit_of(u, n1, ks, n_wt1, n_wt2, num_k1, num_k2);
+      const bool g1 = x.g1;
+      const int r = x.r, wt = x.wt;
       const int e = d_e[r], cnt = d_cnt[r];
       const unsigned mask = d_mask[r];
-      const int num_k = g1 ? num_k1 : num_k2;
       const int64_t w0 = g1 ? wt * kWRows : wt * 2 * kWRows;
       const int64_t w1 = g1 ? w0 : w0 + kWRows;
       const uint8_t* sf0 = g1 ? g.gate_sf : g.w2_sf;
@@ -361,14 +364,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("st.shared.u32 [%0], %1;" ::"r"(sfx + kAtomBytes + 16 * lane), "r"(b) : "memory");
         fence_proxy_async_smem();
       };
-      // GEMM1: quantise the item's token rows once, for all its k-steps
+      // GEMM1: quantise the unit's token rows once, for all its k-steps
       const int64_t rb = g.H / 2, sbytes = g.H / 32;
       const bool use_buf = g1 && cnt * (rb + sbytes) <= kXbufBytes;
       __syncwarp();  // every lane is done with the previous item's buffer
       if (use_buf) {
-        const int nb = static_cast<int>(g.H / 32);
+        const int nb = 8 * (x.kb1 - x.kb0);  // 1x32 blocks of the unit's k-steps, per row
         for (int idx = lane; idx < cnt * nb; idx += 32) {
-          const int q = idx / nb, b = idx - q * nb;
+          const int q = idx / nb, b = idx - q * nb + 8 * x.kb0;
           float v[32];
           load_x_block(q * 8 + (b & 7), b >> 3, v);  // row q, k-step b / 8, block b % 8
           uint32_t wq[4];
@@ -378,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
       }
-      for (int kb = 0; kb < num_k && ok; ++kb) {
+      for (int kb = x.kb0; kb < x.kb1 && ok; ++kb) {
         if (!ready && npend == kStages) {
           if (!warp_wait_count(&sync.g1[r], static_cast<unsigned>(n_wt1), g.err, lane)) ok = false;
           for (int i = 0; i < npend; ++i) {
@@ -469,11 +472,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t stage = 0, phase = 0, buf = 0, acc_phase = 0;
       bool ok = true, issued = false;
       for (int u = blockIdx.x; u < n_items && ok; u += gridDim.x) {
-        const int num_k = u < n1 ? num_k1 : num_k2;
+        const Unit x = unit_of(u, n1, ks, n_wt1, n_wt2, num_k1, num_k2);
         if (!mbar_wait(&tempty[buf], acc_phase ^ 1u, g.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t acc0 = tmem_base + buf * kAccCols, acc1 = acc0 + kNtok;
-        for (int kb = 0; kb < num_k; ++kb) {
+        for (int kb = x.kb0; kb < x.kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, g.err)) { ok = false; break; }
           tc_fence_after();
           fence_proxy_async_smem();  // scales by cp.async and codes by st.shared, read below
@@ -491,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t idesc = idesc_mxf4(kWRows, kNtok, sfid, sfid);
             const uint64_t xd = sw128_kmajor_desc(x_addr + kk * kUmmaKBytes);
             const uint32_t sfx = (sf_t + 16 + 4 * atom) | (sfid << 30);
-            const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+            const uint32_t acc = (kb > x.kb0 || kk > 0) ? 1u : 0u;
             mma_mxf4(acc0, sw128_kmajor_desc(w0_addr + kk * kUmmaKBytes), xd, idesc,
                      (sf_t + 4 * atom) | (sfid << 30), sfx, acc);
             mma_mxf4(acc1, sw128_kmajor_desc(w1_addr + kk * kUmmaKBytes), xd, idesc,
@@ -525,9 +528,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     for (int u = blockIdx.x; u < n_items; u += gridDim.x) {
-      const bool g1 = u < n1;
-      const int r = g1 ? u / n_wt1 : (u - n1) / n_wt2;
-      const int wt = g1 ? u - r * n_wt1 : (u - n1) - r * n_wt2;
+      const Unit x = unit_of(u, n1, ks, n_wt1, n_wt2, num_k1, num_k2);
+      const bool g1 = x.g1;
+      const int r = x.r, wt = x.wt;
       const unsigned mask = d_mask[r];
       const int cnt = d_cnt[r];
       const int my_slot = lane < cnt ? nth_bit(mask, lane) : -1;
@@ -539,6 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(&tfull[buf], acc_phase, g.err)) break;
       tc_fence_after();
       const uint32_t lane_base = (static_cast<uint32_t>(quad * 32) << 16) + buf * kAccCols;
+      bool released = false;  // the accumulator buffer was handed back to the MMA warp
       if (g1) {
         // this warp's 32 rows of I = one 1x32 block for every token: requantise
         const int64_t i0 = static_cast<int64_t>(wt) * kWRows + quad * 32;
@@ -546,6 +550,67 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem_base + lane_base, gv);
         tmem_ld32(tmem_base + lane_base + kNtok, uv);
         tmem_wait_ld();
+        if (ks > 1) {
+          // one K part of the item: park the fp32 partials; the unit that
+          // completes the item sums all parts in part order and requantises
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[buf]);
+          if (++buf == 2) { buf = 0; acc_phase ^= 1u; }
+          released = true;
+          int colb = 0;  // this expert's token columns follow those of the routed experts before it
+          for (int q = 0; q < r; ++q) colb += d_cnt[q];
+          const size_t tile_stride = static_cast<size_t>(n_wt1) * kNtok * 2 * kWRows;
+          float* pb = g.part_ws + x.part * tile_stride +
+                      (static_cast<size_t>(wt) * kNtok + colb) * 2 * kWRows + quad * 32 + lane;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            if (j >= cnt) break;
+            pb[j * 2 * kWRows] = __uint_as_float(gv[j]);
+            pb[j * 2 * kWRows + kWRows] = __uint_as_float(uv[j]);
+          }
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(epi_done);
+          if (et == 0) {
+            mbar_wait(epi_done, sync_phase, g.err);
+            __threadfence();
+            const unsigned old = atomicAdd(&sync.g1p[x.item], 1u);
+            misc[2] = (old + 1 == static_cast<unsigned>(ks)) ? 1 : 0;
+            __threadfence();
+            mbar_arrive(epi_last);
+          }
+          mbar_wait(epi_last, sync_phase, g.err);
+          const bool done_item = misc[2] != 0;
+          sync_phase ^= 1u;
+          if (!done_item) continue;
+          __threadfence();
+          float sg[32], su[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) sg[j] = su[j] = 0.0f;
+          for (int p = 0; p < ks; ++p) {
+            if (p == x.part) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                sg[j] += __uint_as_float(gv[j]);
+                su[j] += __uint_as_float(uv[j]);
+              }
+            } else {
+              const float* qb = pb + static_cast<ptrdiff_t>(p - x.part) * static_cast<ptrdiff_t>(tile_stride);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                if (j >= cnt) break;
+                sg[j] += __ldcg(qb + j * 2 * kWRows);
+                su[j] += __ldcg(qb + j * 2 * kWRows + kWRows);
+              }
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            gv[j] = __float_as_uint(sg[j]);
+            uv[j] = __float_as_uint(su[j]);
+          }
+        }
         uint32_t my_sc = 0;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
@@ -605,10 +670,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[buf]);
-      if (++buf == 2) { buf = 0; acc_phase ^= 1u; }
+      if (!released) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[buf]);
+        if (++buf == 2) { buf = 0; acc_phase ^= 1u; }
+      }
       __threadfence();
       __syncwarp();
       if (lane == 0) mbar_arrive(epi_done);
@@ -674,6 +741,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       __threadfence();
       for (int i = 0; i < 32; ++i) sync.g1[i] = 0u;
       for (int i = 0; i < kMaxOutTiles; ++i) sync.g2[i] = 0u;
+      if (ks > 1)
+        for (int i = 0; i < n1; ++i) sync.g1p[i] = 0u;
       __threadfence();
       sync.exit_cnt = 0u;
     }
@@ -725,6 +794,8 @@ cudaError_t launch_decode_fused_mx(const CUtensorMap& gate, const CUtensorMap& u
   g.vec_x = (p.x.s1 == 1 && (p.x.s0 * 2) % 16 == 0 && reinterpret_cast<uintptr_t>(p.x.data) % 16 == 0) ? 1 : 0;
   g.vec_out = (p.os1 == 1 && (p.os0 * 2) % 16 == 0 && reinterpret_cast<uintptr_t>(p.out) % 16 == 0) ? 1 : 0;
   g.slot = static_cast<int32_t>(next_decode_slot());
+  g.part_ws = p.part_ws;
+  g.max_split = p.max_split;
   g.err = p.err;
   DecodeSyncMx* sets = decode_sync_sets();
   if (!sets) return cudaErrorInvalidDevicePointer;

@@ -36,6 +36,7 @@ struct WsLayout {
   size_t tile_row2, tile_rows2, tile_expert2;
   size_t a1, a1_scale, h, h_scale, y;
   size_t w_row;       // MXFP4: routing weight per grouped row (written by permute)
+  size_t part;        // at most 32 slots: GEMM1 split-K partials of the one-kernel path
   size_t total;
 };
 
@@ -181,6 +182,8 @@ struct DecodeArgs {
   __nv_bfloat16* y_ws;  // [32, H] workspace rows (by slot)
   __nv_bfloat16* out;
   int64_t os0, os1;
+  float* part_ws;     // GEMM1 split-K partials (decode_part_bytes(I))
+  int32_t max_split;  // at most this many GEMM1 K parts (1: not split)
   DeviceErrors* err;
 };
 // maps: gate/up/w2 3-D weight maps ([64 x 128] boxes), x1 = x [T, H] and h1 = h_ws [32, I]
@@ -192,11 +195,20 @@ cudaError_t launch_decode_fused(const CUtensorMap& gate, const CUtensorMap& up, 
 // Cross-CTA counters of the one-kernel decode paths: kDecodeSlots sets in
 // library memory, dealt round-robin to calls; each launch's last CTA resets its set.
 struct DecodeSync {
-  unsigned int g1[32];   // GEMM1 items finished, per routed expert
-  unsigned int g2[64];   // GEMM2 items finished, per 256-column output tile
-  unsigned int exit_cnt; // CTAs finished
+  unsigned int g1[32];    // GEMM1 items finished, per routed expert
+  unsigned int g2[64];    // GEMM2 items finished, per 256-column output tile
+  unsigned int exit_cnt;  // CTAs finished
   unsigned int pad[31];
+  unsigned int g1p[1024]; // K parts of a split GEMM1 item finished, per item
 };
+constexpr int kDecodeMaxSplit = 4;  // GEMM1 K parts of the one-kernel path
+// GEMM1 split-K partial buffer of the decode kernels, fp32
+// [part][128-row tile of I][slot column][gate, up][128 rows]: the routed
+// experts' token columns are packed (at most 32 slots in all), so one column
+// range per (part, row tile) holds every expert's partials
+inline int64_t decode_part_bytes(int64_t I) {
+  return int64_t(kDecodeMaxSplit) * ((I + 127) / 128) * 32 * 2 * 128 * 4;
+}
 constexpr int kDecodeSlots = 16;
 unsigned next_decode_slot();
 DecodeSync* decode_sync_sets();  // device address on the current device (null on error)
@@ -216,6 +228,8 @@ struct DecodeMxArgs {
   __nv_bfloat16* y_ws;
   __nv_bfloat16* out;
   int64_t os0, os1;
+  float* part_ws;    // GEMM1 split-K partials (decode_part_bytes(I))
+  int32_t max_split; // at most this many GEMM1 K parts (1: not split)
   DeviceErrors* err;
 };
 // maps: gate/up/w2 code maps ([128 B x 128] boxes), hc = h codes [32, I/2] bytes with a

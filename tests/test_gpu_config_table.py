@@ -43,8 +43,10 @@ def test_tuned_row_matches_oracle(row, request):
     H, I, E, k = row["H"], row["I"], row["E"], row["k"]
     T = _row_T(row)
     got_cfg = moe.get_config(T, H, I, E, k, mxfp4=mx)
-    for f in ("tile", "pair", "g1_256", "g2_single"):
+    for f in ("tile", "pair", "g1_256", "g2_single", "fused"):
         assert got_cfg[f] == row[f] or (f == "pair" and got_cfg["tile"] != 128), (f, got_cfg, row)
+    if row["fused"]:
+        assert got_cfg["split"] == (row["split"] or 4), (got_cfg, row)
     x = wl.make_x(T, H, seed=2000 + T)
     if mx:
         w = request.getfixturevalue("tp2_weights")

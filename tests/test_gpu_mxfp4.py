@@ -191,7 +191,8 @@ def test_mxfp4_decode_align_permute_one_launch_matches_two(T, k, strided):
 def test_mxfp4_decode_one_kernel_matches_kernels_and_oracle(T, H, I, E, k, case):
     # at most 32 slots: the MXFP4 forward as one kernel (tokens quantised in the
     # kernel with the permute's rule, h requantised by the GEMM1 epilogue's rule)
-    # must give the multi-kernel path's bits and match the oracle
+    # must give the multi-kernel path's bits with GEMM1 unsplit, and match the
+    # oracle with GEMM1 split along K (its fp32 parts summed in part order)
     cs = make_mx_case(T, H, I, E, k, seed=T + k + 307, shared=(case == "shared"))
     if case in ("plain", "strided-x"):
         cs["ids"][0, 1] = E                           # a skipped slot
@@ -205,19 +206,48 @@ def test_mxfp4_decode_one_kernel_matches_kernels_and_oracle(T, H, I, E, k, case)
         c["x"] = cs["x"].t().contiguous().cuda().t()
     moe.device_errors()
     outs, launches = {}, {}
-    for fused in (1, 0):
-        with moe.config_override((T, H, I, E, k), mxfp4=True, fused=fused):
-            outs[fused] = mx_gpu(c)
-            launches[fused] = moe.last_launch_count()
+    variants = {"unsplit": dict(fused=1, split=1), "kernels": dict(fused=0), "split": dict(fused=1)}
+    for name, flags in variants.items():
+        with moe.config_override((T, H, I, E, k), mxfp4=True, **flags):
+            outs[name] = mx_gpu(c)
+            launches[name] = moe.last_launch_count()
+            if name == "split":
+                assert torch.equal(mx_gpu(c), outs[name])  # fixed part order: deterministic
     nbad, nto = moe.device_errors()
     n_skip = int(((cs["ids"] < 0) | (cs["ids"] >= E)).sum().item())
-    assert nbad == 2 * n_skip and nto == 0
-    assert launches[1] == 1 and launches[0] == 4
-    assert torch.equal(outs[1], outs[0])
+    assert nbad == 4 * n_skip and nto == 0
+    assert launches["unsplit"] == 1 and launches["split"] == 1 and launches["kernels"] == 4
+    assert torch.equal(outs["unsplit"], outs["kernels"])
     if case == "no-valid-id":
-        assert bool((outs[1] == 0).all())
+        assert bool((outs["split"] == 0).all()) and bool((outs["unsplit"] == 0).all())
     else:
-        assert rel_err(outs[1], mx_oracle(cs)) <= MX_TOL
+        ref = mx_oracle(cs)
+        assert rel_err(outs["unsplit"], ref) <= MX_TOL
+        assert rel_err(outs["split"], ref) <= MX_TOL
+
+
+@pytest.mark.parametrize("T,E,k", [(1, 16, 4), (2, 24, 10), (3, 40, 8)])
+def test_mxfp4_decode_split_gemm1_each_part_count_matches_oracle(T, E, k):
+    # the MXFP4 one-kernel path with GEMM1 split along K into at most 2, 3 and 4
+    # parts (H = 4096: 16 k-steps of 256 codes, at least four per part; the
+    # cases with few routed experts take the most): each count matches the
+    # oracle and repeats its own bits; unsplit equals the multi-kernel path
+    H, I = 4096, 256
+    cs = make_mx_case(T, H, I, E, k, seed=11 * T + E + k)
+    if T > 1:
+        cs["ids"][T - 1, 0] = cs["ids"][0, 0]          # an expert shared by two tokens
+    c = cuda_case(cs)
+    ref = mx_oracle(cs)
+    outs = {}
+    for split in (1, 2, 3, 4):
+        with moe.config_override((T, H, I, E, k), mxfp4=True, fused=1, split=split):
+            assert moe.get_config(T, H, I, E, k, mxfp4=True)["split"] == split
+            outs[split] = mx_gpu(c)
+            assert moe.last_launch_count() == 1
+            assert torch.equal(mx_gpu(c), outs[split]), split
+        assert rel_err(outs[split], ref) <= MX_TOL, split
+    with moe.config_override((T, H, I, E, k), mxfp4=True, fused=0):
+        assert torch.equal(mx_gpu(c), outs[1])
 
 
 @pytest.mark.parametrize("T,H,I,E,k", [

@@ -423,7 +423,8 @@ def test_decode_align_permute_one_launch_matches_two(T, k, idt, tile, strided):
 def test_decode_one_kernel_matches_kernels_and_oracle(T, H, I, E, k, idt, case):
     # at most 32 slots: the whole forward as one kernel (slots grouped in every CTA,
     # token rows gathered from x, combine by the last CTA of each output tile) must
-    # give the multi-kernel path's bits and match the oracle
+    # give the multi-kernel path's bits with GEMM1 unsplit, and match the oracle
+    # with GEMM1 split along K (these shapes take two parts when few experts are routed)
     cs = make_case(T, H, I, E, k, seed=T + k + 211)
     ids = cs["ids"].to(idt)
     if case in ("plain", "strided-ids", "ragged"):
@@ -441,20 +442,50 @@ def test_decode_one_kernel_matches_kernels_and_oracle(T, H, I, E, k, idt, case):
         c["ids"] = big[:, 1, :]
     moe.device_errors()
     outs, launches = {}, {}
-    for fused in (1, 0):
-        with moe.config_override((T, H, I, E, k), fused=fused):
+    variants = {"unsplit": dict(fused=1, split=1), "kernels": dict(fused=0), "split": dict(fused=1)}
+    for name, flags in variants.items():
+        with moe.config_override((T, H, I, E, k), **flags):
             out = torch.full((T, H), 7.0, dtype=torch.bfloat16, device="cuda")  # stale contents
-            outs[fused] = run_gpu(c, out=out)
-            launches[fused] = moe.last_launch_count()
+            outs[name] = run_gpu(c, out=out)
+            launches[name] = moe.last_launch_count()
+            if name == "split":
+                assert torch.equal(run_gpu(c), outs[name])  # fixed part order: deterministic
     nbad, nto = moe.device_errors()
     n_skip = int(((ids < 0) | (ids >= E)).sum().item())
-    assert nbad == 2 * n_skip and nto == 0
-    assert launches[1] == 1 and launches[0] == 4
-    assert torch.equal(outs[1], outs[0])
+    assert nbad == 4 * n_skip and nto == 0
+    assert launches["unsplit"] == 1 and launches["split"] == 1 and launches["kernels"] == 4
+    assert torch.equal(outs["unsplit"], outs["kernels"])
     if case == "no-valid-id":
-        assert bool((outs[1] == 0).all())
+        assert bool((outs["split"] == 0).all()) and bool((outs["unsplit"] == 0).all())
     else:
-        assert rel_err(outs[1], run_oracle(cs)) <= BF16_TOL
+        ref = run_oracle(cs)
+        assert rel_err(outs["unsplit"], ref) <= BF16_TOL
+        assert rel_err(outs["split"], ref) <= BF16_TOL
+
+
+@pytest.mark.parametrize("T,E,k", [(1, 16, 4), (2, 16, 6), (1, 64, 8), (4, 40, 8)])
+def test_decode_split_gemm1_each_part_count_matches_oracle(T, E, k):
+    # GEMM1 split along K into at most 2, 3 and 4 parts (H = 2048: 32 k-blocks,
+    # so every count keeps at least four per part; the cases with few routed
+    # experts take the most parts; I = 320 leaves a ragged 64-row last item):
+    # each count matches the oracle and repeats its own bits, and the unsplit
+    # one-kernel result equals the multi-kernel path's
+    H, I = 2048, 320
+    cs = make_case(T, H, I, E, k, seed=7 * T + E + k)
+    if T > 1:
+        cs["ids"][T - 1, 0] = cs["ids"][0, 0]          # an expert shared by two tokens
+    c = to_cuda(cs)
+    ref = run_oracle(cs)
+    outs = {}
+    for split in (1, 2, 3, 4):
+        with moe.config_override((T, H, I, E, k), fused=1, split=split):
+            assert moe.get_config(T, H, I, E, k)["split"] == split
+            outs[split] = run_gpu(c)
+            assert moe.last_launch_count() == 1
+            assert torch.equal(run_gpu(c), outs[split]), split
+        assert rel_err(outs[split], ref) <= BF16_TOL, split
+    with moe.config_override((T, H, I, E, k), fused=0):
+        assert torch.equal(run_gpu(c), outs[1])
 
 
 def test_decode_one_kernel_repeated_calls_and_fallback_for_strided_x():
@@ -468,9 +499,12 @@ def test_decode_one_kernel_repeated_calls_and_fallback_for_strided_x():
     assert moe.last_launch_count() == 1
     for _ in range(40):
         assert torch.equal(run_gpu(c), first)
-    xs = cs["x"].t().contiguous().cuda().t()
-    c2 = dict(c, x=xs)
-    got = run_gpu(c2)
-    assert moe.last_launch_count() == 4
-    assert torch.equal(got, first)
-    assert rel_err(first, run_oracle(cs)) <= BF16_TOL
+    with moe.config_override((T, H, I, E, k), split=1):
+        unsplit = run_gpu(c)
+        xs = cs["x"].t().contiguous().cuda().t()
+        c2 = dict(c, x=xs)
+        got = run_gpu(c2)
+        assert moe.last_launch_count() == 4
+    assert torch.equal(got, unsplit)
+    ref = run_oracle(cs)
+    assert rel_err(first, ref) <= BF16_TOL and rel_err(unsplit, ref) <= BF16_TOL

@@ -102,7 +102,7 @@ def test_router_then_forward_on_the_same_stream_decode():
         outs = {}
         for name, flags in (("prefetch", dict(prefetch=1, fused=0)),
                             ("no-prefetch", dict(prefetch=0, fused=0)),
-                            ("one-kernel", dict(fused=1))):
+                            ("one-kernel", dict(fused=1, split=1))):
             with moe.config_override((T, H, I, E, k), **flags):
                 ids.fill_(0)                     # stale routing the prefetch could see
                 moe.router_topk(logits, k, topk_ids=ids, topk_weights=wts)
