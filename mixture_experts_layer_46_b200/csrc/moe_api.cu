@@ -615,7 +615,7 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
 
   // ---- tensor maps (bf16, 128-byte swizzle): weights in [64 x 128] boxes,
   // expert-grouped token rows in one box per CTA and token tile
-  CUtensorMap mA1, mGate, mUp, mH, mW2;
+  CUtensorMap mA1, mGate, mUp, mH, mW2, mGate64, mUp64;
   // the configuration: token-tile rows (32 / 128 on one CTA, 128 / 256 on CTA
   // pairs, which move a sixth fewer shared-memory bytes per FLOP); GEMM2 on
   // pairs with one 256-row w2 slice per 256-row token tile (align's second
@@ -625,12 +625,15 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   const bool pair = cfg.pair != 0;
   const bool g2_single = cfg.g2_single != 0;
   const bool g1_256 = cfg.g1_256 != 0;
+  // GEMM1 with gate and up interleaved in one accumulator: 512-row token tiles
+  // (their own list), 32-row token boxes (a tile's second MMA chunk is often short)
+  const bool g1_512 = cfg.g1_512 != 0;
   const int32_t wpolicy = 0;
   const uint32_t boxw[3] = {64, 128, 1};
   // one TMA box covers a CTA's share of a token tile
   const uint32_t tok_box = pair ? static_cast<uint32_t>(tile / 2) : static_cast<uint32_t>(tile);
   const uint32_t boxt2[2] = {64, g2_single ? 128u : tok_box};
-  const uint32_t boxt1[2] = {64, g1_256 ? 128u : tok_box};
+  const uint32_t boxt1[2] = {64, g1_512 ? 32u : (g1_256 ? 128u : tok_box)};
   {
     const uint64_t d[2] = {uint64_t(pr.H), uint64_t(L.p_max)};
     const uint64_t sb[1] = {uint64_t(pr.H) * 2};
@@ -650,6 +653,15 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
     s = make_map(&mUp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, up->data, d, su, boxw,
                  CU_TENSOR_MAP_SWIZZLE_128B);
     if (s != MOE_OK) return s;
+    if (g1_512) {
+      const uint32_t box64[3] = {64, 64, 1};
+      s = make_map(&mGate64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, gate->data, d, sg, box64,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+      if (s != MOE_OK) return s;
+      s = make_map(&mUp64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, up->data, d, su, box64,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+      if (s != MOE_OK) return s;
+    }
   }
   {
     const uint64_t d[2] = {uint64_t(pr.I), uint64_t(L.p_max)};
@@ -713,7 +725,7 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   // ---- launches
   AlignTiles tiles;
   std::memset(&tiles, 0, sizeof(tiles));
-  tiles.list[0].tile_max = tile;
+  tiles.list[0].tile_max = g1_512 ? 512 : tile;
   tiles.list[0].tile_row = reinterpret_cast<int32_t*>(w + L.tile_row);
   tiles.list[0].tile_rows = reinterpret_cast<int32_t*>(w + L.tile_rows);
   tiles.list[0].tile_expert = reinterpret_cast<int32_t*>(w + L.tile_expert);
@@ -780,8 +792,14 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
     g1.tile_expert = tiles.list[1].tile_expert;
     g1.tok_box = 128;
   }
-  rc = pair ? launch_gemm_ws_pair_bf16(0, g1_256 ? 256 : tile, mGate, mUp, mA1, g1, dev->num_sms, st, &launches)
-            : launch_gemm_ws_bf16(0, tile, mGate, mUp, mA1, g1, dev->num_sms, st, &launches);
+  if (g1_512) {
+    g1.n_wt = (pr.I + 127) / 128;
+    g1.tok_box = 32;
+    rc = launch_gemm_il_pair_bf16(mGate64, mUp64, mA1, g1, dev->num_sms, st, &launches);
+  } else {
+    rc = pair ? launch_gemm_ws_pair_bf16(0, g1_256 ? 256 : tile, mGate, mUp, mA1, g1, dev->num_sms, st, &launches)
+              : launch_gemm_ws_bf16(0, tile, mGate, mUp, mA1, g1, dev->num_sms, st, &launches);
+  }
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm1");
   prof_mark(st);
 

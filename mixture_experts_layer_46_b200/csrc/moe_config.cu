@@ -48,7 +48,8 @@ bool entry_ok(const moe_config_t& c) {
   if (c.H < 0 || c.I < 0 || c.E < 0 || c.k < 0 || c.t_lo < 0 || c.t_hi < c.t_lo) return false;
   if (!tile_ok(c.tile, c.wdtype == MOE_E2M1X2)) return false;
   return flag_ok(c.pair) && flag_ok(c.g1_256) && flag_ok(c.g2_single) && flag_ok(c.tiny) &&
-         flag_ok(c.prefetch) && flag_ok(c.fused) && c.split >= 0 && c.split <= kDecodeMaxSplit;
+         flag_ok(c.prefetch) && flag_ok(c.fused) && c.split >= 0 && c.split <= kDecodeMaxSplit &&
+         flag_ok(c.g1_512);
 }
 
 // The measured defaults of the kernels when no table entry matches: 32-row
@@ -107,8 +108,14 @@ moe_config_t select_config(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k
   // what the kernels can run: flags that do not apply to the chosen tile are cleared
   const int64_t S = T * k;
   if (mxfp4) {
-    c.pair = c.g1_256 = c.g2_single = c.prefetch = 0;
+    c.pair = c.g1_256 = c.g2_single = c.prefetch = c.g1_512 = 0;
   } else {
+    if (c.g1_512) {
+      // GEMM1 on its own 512-row tile list, GEMM2 on the 256-row list
+      c.tile = 128;
+      c.pair = c.g2_single = 1;
+      c.g1_256 = 0;
+    }
     if (c.tile == 256) c.pair = 1;  // 256-row token tiles exist only on CTA pairs
     if (c.tile == 32) c.pair = 0;
     if (!(c.pair && c.tile == 128)) c.g2_single = 0;

@@ -78,8 +78,7 @@ __global__ void __launch_bounds__(128) permute_quant_kernel(View2 x, int64_t T, 
   const int64_t nb = H / 32;  // blocks per row
   {
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-      int32_t pos[kMaxTopK];
-      for (int j = 0; j < k; ++j) pos[j] = inv[t * k + j];
+      const int32_t* pos = inv + t * k;
       // routing weight of each slot at its grouped row, for the down projection's epilogue
       if (threadIdx.x < k && pos[threadIdx.x] >= 0)
         w_row[pos[threadIdx.x]] =
@@ -106,10 +105,11 @@ __global__ void __launch_bounds__(128) permute_quant_kernel(View2 x, int64_t T, 
         uint32_t w[4];
         const uint32_t sc = mx_quant32(v, w);
         for (int j = 0; j < k; ++j) {
-          if (pos[j] < 0) continue;
-          *reinterpret_cast<uint4*>(codes + static_cast<int64_t>(pos[j]) * (H / 2) + b * 16) =
+          const int32_t p = __ldg(pos + j);
+          if (p < 0) continue;
+          *reinterpret_cast<uint4*>(codes + static_cast<int64_t>(p) * (H / 2) + b * 16) =
               make_uint4(w[0], w[1], w[2], w[3]);
-          scales[static_cast<int64_t>(pos[j]) * nb + b] = static_cast<uint8_t>(sc);
+          scales[static_cast<int64_t>(p) * nb + b] = static_cast<uint8_t>(sc);
         }
       }
     }

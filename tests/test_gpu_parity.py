@@ -326,6 +326,7 @@ TILE_VARIANTS = {
     "128/pair-one-slice": dict(tile=128, pair=1, g2_single=1, g1_256=0),
     "128/pair-one-slice-g1-256": dict(tile=128, pair=1, g2_single=1, g1_256=1),
     "256": dict(tile=256),
+    "pair-gate-up-interleaved-512": dict(g1_512=1),
 }
 
 
@@ -333,6 +334,7 @@ TILE_VARIANTS = {
     (300, 512, 384, 4, 2),     # 150 slots per expert: several 32-row granules, partial tiles
     (600, 512, 640, 3, 2),     # 400 slots per expert: >1 token tile of 256 rows, N tail of I
     (77, 288, 96, 6, 3),       # ragged K and output columns
+    (700, 256, 256, 2, 2),     # 700 slots per expert: two 352-row tiles of the 512-row list
 ])
 def test_token_tile_configs_agree_and_match_oracle(T, H, I, E, k):
     # the token-tile size (32 / 128 rows on one CTA, 128 / 256 rows on a CTA pair)
