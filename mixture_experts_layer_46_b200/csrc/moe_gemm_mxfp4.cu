@@ -315,20 +315,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t lane_base = (static_cast<uint32_t>(quad * 32) << 16) + buf * C::kBufCols;
       if (kMode == 0) {
-        // this warp's 32 weight rows = one 1x32 block of I for every token
+        // this warp's 32 weight rows = one 1x32 block of I for every token; the
+        // quadrant's two warps each requantise 16 tokens of every 32-token chunk
         const int64_t i0 = wt * kWRows + quad * 32;
 #pragma unroll 1
-        for (int c = half; c < rows / 32; c += 2) {
-          uint32_t gv[32], uv[32];
-          tmem_ld32(tmem_base + lane_base + c * 32, gv);
-          tmem_ld32(tmem_base + lane_base + kNmax + c * 32, uv);
+        for (int c = 0; c < rows / 32; ++c) {
+          const int j0 = c * 32 + half * 16;
+          uint32_t gv[16], uv[16];
+          tmem_ld16(tmem_base + lane_base + j0, gv);
+          tmem_ld16(tmem_base + lane_base + kNmax + j0, uv);
           tmem_wait_ld();
           uint32_t my_sc = 0;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
+          for (int j = 0; j < 16; ++j) {
             const float h = silu_mul(__uint_as_float(gv[j]), __uint_as_float(uv[j]));
             if (g.h_capture && i0 < g.N)
-              g.h_capture[(row0 + c * 32 + j) * g.N + i0 + lane] = h;
+              g.h_capture[(row0 + j0 + j) * g.N + i0 + lane] = h;
             // |h| as bits orders like its value: one warp reduction gives the block amax
             const float amax = __uint_as_float(
                 __reduce_max_sync(0xffffffffu, __float_as_uint(h) & 0x7fffffffu));
@@ -343,13 +345,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == j) my_sc = static_cast<uint32_t>(sexp + 127);
           }
           __syncwarp();
-          // lane j stores token j's 16 code bytes and its scale
-          uint4 v;
-          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                       : "r"(stg_s + lane * 16));
-          if (i0 < g.N) {
-            const int64_t p = row0 + c * 32 + lane;
+          // lane j < 16 stores token j's 16 code bytes and its scale
+          if (lane < 16 && i0 < g.N) {
+            uint4 v;
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                         : "r"(stg_s + lane * 16));
+            const int64_t p = row0 + j0 + lane;
             *reinterpret_cast<uint4*>(static_cast<uint8_t*>(g.out) + p * g.out_ld + i0 / 2) = v;
             g.out_sf[p * g.out_sf_ld + i0 / 32] = static_cast<uint8_t>(my_sc);
           }
@@ -357,7 +359,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         // both accumulators of a 32-token chunk are loaded together (one wait)
-        // and share the chunk's routing weights
+        // and share the chunk's routing weights (splitting the two w2 slices
+        // between the quadrant's warps instead measured slower: every warp then
+        // broadcasts every chunk's weights)
 #pragma unroll
         for (int c = 0; c < kNmax / 32; ++c) {
           if (c * 32 >= rows) break;
