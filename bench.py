@@ -62,11 +62,14 @@ NCU_TRAFFIC = {
 
 
 def kernel_src_hash(config: dict) -> str:
-    """Hash of the GEMM kernels' sources and of the configuration the timed forward ran:
-    a recorded traffic figure is reported only while both are unchanged."""
+    """Hash of the sources of the GEMM kernels the timed forward's weight type runs, and
+    of its configuration: a recorded traffic figure is reported only while both are
+    unchanged."""
     h = hashlib.sha256()
-    for fn in ("moe_gemm_ws.cu", "moe_gemm_ws2.cu", "moe_gemm_il.cu", "moe_gemm_mxfp4.cu",
-               "moe_common.cuh", "moe_pair.cuh"):
+    mx = config.get("wdtype") == 4
+    files = (("moe_gemm_mxfp4.cu", "moe_mx.cuh") if mx else
+             ("moe_gemm_ws.cu", "moe_gemm_ws2.cu", "moe_gemm_il.cu", "moe_pair.cuh"))
+    for fn in files + ("moe_common.cuh",):
         with open(os.path.join(ROOT, "mixture_experts_layer_46_b200", "csrc", fn), "rb") as f:
             h.update(f.read())
     h.update(json.dumps({k: config[k] for k in sorted(config) if k not in ("t_lo", "t_hi")}).encode())

@@ -42,7 +42,8 @@ constexpr int kSfBytes = 2 * kAtomBytes;       // 8 blocks of 32 per stage
 constexpr int kEpiWarps = 8;                   // two per TMEM lane quadrant, alternating chunks
 constexpr int kSfWarps = 1;                    // scale producer warps
 constexpr int kFirstEpiWarp = 2 + kSfWarps;
-constexpr int kStagingBytes = 32 * 64;
+constexpr int kStagingTile = 32 * 64;                 // a 32 x 32 bf16 tile (or 32 x 32 codes)
+constexpr int kStagingBytes = kStagingTile + 32 * 4;  // + the chunk's 32 routing weights (GEMM2)
 constexpr int kSfColsPerStage = 24;
 constexpr int kTmemCols = 512;
 constexpr int kThreads = 32 * (kFirstEpiWarp + kEpiWarps);
@@ -367,13 +368,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (c * 32 >= rows) break;
           if ((c & 1) != half) continue;
           const int32_t my_slot = slot_r[c];
-          const float my_w = w_r[c];
           uint32_t v0[32], v1[32];
           tmem_ld32(tmem_base + lane_base + c * 32, v0);
           tmem_ld32(tmem_base + lane_base + kNmax + c * 32, v1);
+          // token j's routing weight to every lane: one store per lane, then
+          // eight broadcast 16-byte reads (instead of 32 shuffles)
+          asm volatile("st.shared.f32 [%0], %1;" ::"r"(stg_s + kStagingTile + lane * 4), "f"(w_r[c])
+                       : "memory");
+          __syncwarp();
           float wj[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) wj[j] = __shfl_sync(0xffffffffu, my_w, j);
+          for (int q = 0; q < 8; ++q)
+            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                         : "=f"(wj[4 * q]), "=f"(wj[4 * q + 1]), "=f"(wj[4 * q + 2]), "=f"(wj[4 * q + 3])
+                         : "r"(stg_s + kStagingTile + 16 * q));
           tmem_wait_ld();
 #pragma unroll
           for (int a = 0; a < 2; ++a) {
