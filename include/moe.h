@@ -342,10 +342,11 @@ typedef struct {
                           as many as put about two GEMM1 units on every SM, with at least
                           four 64-wide k-blocks per part; the unit that completes a (routed
                           expert, 128-row) item sums all parts' fp32 partials in part order */
-  int32_t g1_512;      /* bf16: GEMM1 on CTA pairs with gate and up rows interleaved in one
-                          accumulator, token tiles of up to 512 rows (an expert's gate/up
-                          weights are read once per 512 rows instead of once per 256);
-                          implies pair = 1, g2_single = 1, g1_256 = 0 */
+  int32_t g1_il;       /* bf16: 0, or GEMM1 on CTA pairs with gate and up rows interleaved in
+                          one accumulator, on token tiles of up to g1_il rows: 256 (two
+                          accumulator buffers, the epilogue under the next item's MMAs) or
+                          512 (an expert's gate/up weights read once per 512 rows; one
+                          buffer); implies pair = 1, g2_single = 1, g1_256 = 0 */
 } moe_config_t;
 
 /* Installs a process-wide configuration table (copied; n = 0 removes it).

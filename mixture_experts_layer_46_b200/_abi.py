@@ -71,13 +71,13 @@ class MoeConfig(ctypes.Structure):
                 ("t_hi", ctypes.c_int64), ("tile", ctypes.c_int32), ("pair", ctypes.c_int32),
                 ("g1_256", ctypes.c_int32), ("g2_single", ctypes.c_int32), ("tiny", ctypes.c_int32),
                 ("prefetch", ctypes.c_int32), ("fused", ctypes.c_int32), ("split", ctypes.c_int32),
-                ("g1_512", ctypes.c_int32)]
+                ("g1_il", ctypes.c_int32)]
 
     def as_dict(self) -> dict:
         return {name: int(getattr(self, name)) for name, _ in self._fields_}
 
 
-CONFIG_FLAGS = ("tile", "pair", "g1_256", "g2_single", "tiny", "prefetch", "fused", "split", "g1_512")
+CONFIG_FLAGS = ("tile", "pair", "g1_256", "g2_single", "tiny", "prefetch", "fused", "split", "g1_il")
 
 
 _lock = threading.Lock()

@@ -625,15 +625,16 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   const bool pair = cfg.pair != 0;
   const bool g2_single = cfg.g2_single != 0;
   const bool g1_256 = cfg.g1_256 != 0;
-  // GEMM1 with gate and up interleaved in one accumulator: 512-row token tiles
-  // (their own list), 32-row token boxes (a tile's second MMA chunk is often short)
-  const bool g1_512 = cfg.g1_512 != 0;
+  // GEMM1 with gate and up interleaved in one accumulator: 256-row token tiles
+  // (align's second list, as GEMM2's) or 512-row tiles (their own list); 32-row
+  // token boxes (a tile's last MMA chunk is often short)
+  const int32_t g1_il = cfg.g1_il;
   const int32_t wpolicy = 0;
   const uint32_t boxw[3] = {64, 128, 1};
   // one TMA box covers a CTA's share of a token tile
   const uint32_t tok_box = pair ? static_cast<uint32_t>(tile / 2) : static_cast<uint32_t>(tile);
   const uint32_t boxt2[2] = {64, g2_single ? 128u : tok_box};
-  const uint32_t boxt1[2] = {64, g1_512 ? 32u : (g1_256 ? 128u : tok_box)};
+  const uint32_t boxt1[2] = {64, g1_il ? 32u : (g1_256 ? 128u : tok_box)};
   {
     const uint64_t d[2] = {uint64_t(pr.H), uint64_t(L.p_max)};
     const uint64_t sb[1] = {uint64_t(pr.H) * 2};
@@ -653,7 +654,7 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
     s = make_map(&mUp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, up->data, d, su, boxw,
                  CU_TENSOR_MAP_SWIZZLE_128B);
     if (s != MOE_OK) return s;
-    if (g1_512) {
+    if (g1_il) {
       const uint32_t box64[3] = {64, 64, 1};
       s = make_map(&mGate64, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, gate->data, d, sg, box64,
                    CU_TENSOR_MAP_SWIZZLE_128B);
@@ -725,7 +726,7 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   // ---- launches
   AlignTiles tiles;
   std::memset(&tiles, 0, sizeof(tiles));
-  tiles.list[0].tile_max = g1_512 ? 512 : tile;
+  tiles.list[0].tile_max = g1_il == 512 ? 512 : tile;
   tiles.list[0].tile_row = reinterpret_cast<int32_t*>(w + L.tile_row);
   tiles.list[0].tile_rows = reinterpret_cast<int32_t*>(w + L.tile_rows);
   tiles.list[0].tile_expert = reinterpret_cast<int32_t*>(w + L.tile_expert);
@@ -792,10 +793,17 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
     g1.tile_expert = tiles.list[1].tile_expert;
     g1.tok_box = 128;
   }
-  if (g1_512) {
+  if (g1_il) {
+    if (g1_il == 256) {
+      g1.max_tiles = L.t_max2;
+      g1.num_tiles = tiles.list[1].num_tiles;
+      g1.tile_row = tiles.list[1].tile_row;
+      g1.tile_rows = tiles.list[1].tile_rows;
+      g1.tile_expert = tiles.list[1].tile_expert;
+    }
     g1.n_wt = (pr.I + 127) / 128;
     g1.tok_box = 32;
-    rc = launch_gemm_il_pair_bf16(mGate64, mUp64, mA1, g1, dev->num_sms, st, &launches);
+    rc = launch_gemm_il_pair_bf16(g1_il, mGate64, mUp64, mA1, g1, dev->num_sms, st, &launches);
   } else {
     rc = pair ? launch_gemm_ws_pair_bf16(0, g1_256 ? 256 : tile, mGate, mUp, mA1, g1, dev->num_sms, st, &launches)
               : launch_gemm_ws_bf16(0, tile, mGate, mUp, mA1, g1, dev->num_sms, st, &launches);

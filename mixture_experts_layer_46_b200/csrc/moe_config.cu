@@ -49,7 +49,7 @@ bool entry_ok(const moe_config_t& c) {
   if (!tile_ok(c.tile, c.wdtype == MOE_E2M1X2)) return false;
   return flag_ok(c.pair) && flag_ok(c.g1_256) && flag_ok(c.g2_single) && flag_ok(c.tiny) &&
          flag_ok(c.prefetch) && flag_ok(c.fused) && c.split >= 0 && c.split <= kDecodeMaxSplit &&
-         flag_ok(c.g1_512);
+         (c.g1_il == 0 || c.g1_il == 256 || c.g1_il == 512);
 }
 
 // The measured defaults of the kernels when no table entry matches: 32-row
@@ -108,10 +108,10 @@ moe_config_t select_config(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k
   // what the kernels can run: flags that do not apply to the chosen tile are cleared
   const int64_t S = T * k;
   if (mxfp4) {
-    c.pair = c.g1_256 = c.g2_single = c.prefetch = c.g1_512 = 0;
+    c.pair = c.g1_256 = c.g2_single = c.prefetch = c.g1_il = 0;
   } else {
-    if (c.g1_512) {
-      // GEMM1 on its own 512-row tile list, GEMM2 on the 256-row list
+    if (c.g1_il) {
+      // interleaved GEMM1 on the 256-row list (or its own 512-row list), GEMM2 on the 256-row list
       c.tile = 128;
       c.pair = c.g2_single = 1;
       c.g1_256 = 0;

@@ -138,10 +138,11 @@ cudaError_t launch_gemm_ws_pair_bf16(int mode, int tile_max, const CUtensorMap& 
                                      int num_sms, cudaStream_t st, int* launches);
 
 // GEMM1 on CTA pairs with gate and up rows interleaved along M (64 of each per
-// CTA, one accumulator), token tiles of up to 512 rows: gate64 / up64 are the
-// gate and up maps with [64 x 64] boxes, x the expert-grouped token rows with
-// boxes of p.tok_box rows (a divisor of 128); p.n_wt = ceil(I / 128).
-cudaError_t launch_gemm_il_pair_bf16(const CUtensorMap& gate64, const CUtensorMap& up64,
+// CTA, one accumulator), token tiles of up to tile_max = 256 or 512 rows:
+// gate64 / up64 are the gate and up maps with [64 x 64] boxes, x the
+// expert-grouped token rows with boxes of p.tok_box rows (a divisor of 128);
+// p.n_wt = ceil(I / 128).
+cudaError_t launch_gemm_il_pair_bf16(int tile_max, const CUtensorMap& gate64, const CUtensorMap& up64,
                                     const CUtensorMap& x, const WsGemm& p, int num_sms,
                                     cudaStream_t st, int* launches);
 

@@ -69,13 +69,14 @@ def candidates(T: int, k: int, mxfp4: bool):
     out.extend(fused)
     for tiny in tinies:
         for pre in ((1, 0) if decode else (0,)):
-            out.append(dict(tile=32, tiny=tiny, prefetch=pre, fused=0, g1_512=0))
-        out.append(dict(tile=128, pair=0, tiny=tiny, fused=0, g1_512=0))
-        out.append(dict(tile=128, pair=1, g2_single=0, tiny=tiny, fused=0, g1_512=0))
-        out.append(dict(tile=128, pair=1, g2_single=1, g1_256=0, tiny=tiny, fused=0, g1_512=0))
-        out.append(dict(tile=128, pair=1, g2_single=1, g1_256=1, tiny=tiny, fused=0, g1_512=0))
-        out.append(dict(tile=128, pair=1, g2_single=1, g1_512=1, tiny=tiny, fused=0))
-        out.append(dict(tile=256, tiny=tiny, fused=0, g1_512=0))
+            out.append(dict(tile=32, tiny=tiny, prefetch=pre, fused=0, g1_il=0))
+        out.append(dict(tile=128, pair=0, tiny=tiny, fused=0, g1_il=0))
+        out.append(dict(tile=128, pair=1, g2_single=0, tiny=tiny, fused=0, g1_il=0))
+        out.append(dict(tile=128, pair=1, g2_single=1, g1_256=0, tiny=tiny, fused=0, g1_il=0))
+        out.append(dict(tile=128, pair=1, g2_single=1, g1_256=1, tiny=tiny, fused=0, g1_il=0))
+        for il in (256, 512):
+            out.append(dict(tile=128, pair=1, g2_single=1, g1_il=il, tiny=tiny, fused=0))
+        out.append(dict(tile=256, tiny=tiny, fused=0, g1_il=0))
     return out
 
 

@@ -189,20 +189,21 @@ def test_config_normalisation_of_the_split_and_interleaved_flags():
     shape = (4096, 4096, 1536, 128, 8)
     try:
         moe.set_config_table([moe.make_config(_abi.MOE_BF16, t_lo=0, t_hi=10 ** 9, tile=32,
-                                              g1_512=1, g1_256=1, split=3),
+                                              g1_il=512, g1_256=1, split=3),
                               moe.make_config(_abi.MOE_E2M1X2, t_lo=0, t_hi=10 ** 9, tile=96,
-                                              g1_512=1)])
+                                              g1_il=256)])
         got = moe.get_config(*shape)
-        assert (got["g1_512"], got["pair"], got["g2_single"], got["g1_256"], got["tile"]) == (1, 1, 1, 0, 128)
+        assert (got["g1_il"], got["pair"], got["g2_single"], got["g1_256"], got["tile"]) == (512, 1, 1, 0, 128)
         assert got["fused"] == 0 and got["split"] == 1
-        assert moe.get_config(*shape, mxfp4=True)["g1_512"] == 0
+        assert moe.get_config(*shape, mxfp4=True)["g1_il"] == 0
         assert moe.get_config(2, 4096, 1536, 128, 8)["fused"] == 0  # the entry says fused = 0
         moe.set_config_table([moe.make_config(_abi.MOE_BF16, t_lo=0, t_hi=4, tile=32, fused=1)])
         assert moe.get_config(2, 4096, 1536, 128, 8)["split"] == 4
         moe.set_config_table([moe.make_config(_abi.MOE_BF16, t_lo=0, t_hi=4, tile=32, fused=1, split=2)])
         assert moe.get_config(2, 4096, 1536, 128, 8)["split"] == 2
-        with pytest.raises(moe.MoeError):
-            moe.set_config_table([moe.make_config(_abi.MOE_BF16, tile=32, split=5)])
+        for bad in (dict(split=5), dict(g1_il=128), dict(g1_il=1)):
+            with pytest.raises(moe.MoeError):
+                moe.set_config_table([moe.make_config(_abi.MOE_BF16, tile=32, **bad)])
     finally:
         moe.set_config_table([])
 
@@ -228,7 +229,7 @@ def test_builtin_config_table_matches_committed_csv():
         T = r["t_hi"]
         got = moe.get_config(T, r["H"], r["I"], r["E"], r["k"], mxfp4=r["wdtype"] == 4)
         assert got["tile"] == r["tile"], r
-        assert got["g1_512"] == r["g1_512"] and got["fused"] == r["fused"], r
+        assert got["g1_il"] == r["g1_il"] and got["fused"] == r["fused"], r
 
 
 def test_router_argument_errors_before_launch():

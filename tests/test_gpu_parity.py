@@ -326,7 +326,8 @@ TILE_VARIANTS = {
     "128/pair-one-slice": dict(tile=128, pair=1, g2_single=1, g1_256=0),
     "128/pair-one-slice-g1-256": dict(tile=128, pair=1, g2_single=1, g1_256=1),
     "256": dict(tile=256),
-    "pair-gate-up-interleaved-512": dict(g1_512=1),
+    "pair-gate-up-interleaved-256": dict(g1_il=256),
+    "pair-gate-up-interleaved-512": dict(g1_il=512),
 }
 
 
