@@ -54,10 +54,11 @@ WORKLOADS = {
 # source it was taken on; reported as null once the source has changed.
 NCU_TRAFFIC = {
     # GEMM1 on the benchmarked workload (T=4096, E=128, the table's configuration for that
-    # bucket), one-pass ncu capture at the full size: 4.28 GB read + 0.105 GB written per
-    # launch; reported only while the GEMM sources and the configuration hash to `src`
-    "qwen3-235b": {"T": 4096, "E": 128, "bytes_per_launch": 4.28e9 + 0.10514e9,
-                   "src": "5e161c7fe4099a5d"},
+    # bucket: gate/up interleaved on 256-row pair tiles), one-pass ncu capture at the full
+    # size: 3.898 GB read + 0.105 GB written per launch; reported only while the GEMM
+    # sources and the configuration hash to `src` (the hash the capturing run printed)
+    "qwen3-235b": {"T": 4096, "E": 128, "bytes_per_launch": 3.8977e9 + 0.10545e9,
+                   "src": "3f9701359ffc56cc"},
 }
 
 
