@@ -53,6 +53,16 @@ def qwen3_weights():
 
 
 @pytest.fixture(scope="session")
+def glm_weights():
+    """GLM-4.5-Air-shaped expert weights (seed 0) on the GPU and a host copy for the oracle."""
+    from mixture_experts_layer_46_b200 import workloads as wl
+
+    s = wl.GLM45_AIR
+    w13, w2 = wl.make_weights_bf16(s.E, s.I, s.H, seed=0, device="cuda")
+    return {"w13": w13, "w2": w2, "w13_cpu": w13.cpu(), "w2_cpu": w2.cpu()}
+
+
+@pytest.fixture(scope="session")
 def tp2_weights():
     """Qwen3.5-397B TP2 MXFP4 expert weights for E = 513 (seed 0), host and GPU.  The
     weights are drawn expert by expert, so the first 512 are exactly the E = 512 layer's."""

@@ -60,8 +60,9 @@ def test_tuned_row_matches_oracle(row, request):
         kw = {"w2_scale": gw["s2"][:E]}
         tol = 6e-2
     else:
-        assert (H, I, E, k) == (4096, 1536, 128, 8), "only the Qwen3-235B shape is tuned here"
-        w = request.getfixturevalue("qwen3_weights")
+        shapes = {(4096, 1536, 128, 8): "qwen3_weights", (4096, 1408, 128, 8): "glm_weights"}
+        assert (H, I, E, k) in shapes, "only the Qwen3-235B and GLM-4.5-Air shapes are tuned here"
+        w = request.getfixturevalue(shapes[(H, I, E, k)])
         ids, wts = wl.route_softmax_topk(T, E, k, seed=1000 + T)
         args = (x.cuda(), moe.w13_from_packed(w["w13"]), w["w2"], ids.cuda(), wts.cuda())
         kw = {}
