@@ -551,7 +551,47 @@ moe_status_t forward_mxfp4(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   g1.err = dev->errors;
   if (t_capture_h.ptr && t_capture_h.bytes >= sizeof(float) * size_t(L.p_max) * size_t(pr.I))
     g1.h_capture = static_cast<float*>(t_capture_h.ptr);
-  rc = launch_gemm_ws_mxfp4(0, cfg.tile, mGate, mUp, mA1, g1, dev->num_sms, st, &launches);
+  // raw e8m0 scale maps for the GEMMs' TMA scale path, where every view it reads is
+  // 16-byte aligned (base and strides); otherwise the GEMM copies scales with cp.async
+  auto a16 = [](const void* ptr, int64_t s0, int64_t s1) {
+    return reinterpret_cast<uintptr_t>(ptr) % 16 == 0 && s0 % 16 == 0 && s1 % 16 == 0;
+  };
+  CUtensorMap sf1[3], sf2[3];
+  bool sf1_ok = a16(gate->scale, gate->scale_strides[0], gate->scale_strides[1]) &&
+                a16(up->scale, up->scale_strides[0], up->scale_strides[1]) &&
+                a16(w + L.a1_scale, pr.H / 32, 0);
+  bool sf2_ok = a16(w2->scale, w2->scale_strides[0], w2->scale_strides[1]) &&
+                a16(w + L.h_scale, pr.I / 32, 0);
+  {
+    const uint32_t boxw[3] = {16, 128, 1};
+    const uint32_t boxt[2] = {16, static_cast<uint32_t>(cfg.tile)};
+    if (sf1_ok) {
+      const uint64_t d3[3] = {uint64_t(pr.H / 32), uint64_t(pr.I), uint64_t(pr.E)};
+      const uint64_t sg[2] = {uint64_t(gate->scale_strides[1]), uint64_t(gate->scale_strides[0])};
+      const uint64_t su[2] = {uint64_t(up->scale_strides[1]), uint64_t(up->scale_strides[0])};
+      const uint64_t dx[2] = {uint64_t(pr.H / 32), uint64_t(L.p_max)};
+      const uint64_t sx[1] = {uint64_t(pr.H / 32)};
+      s = make_map(&sf1[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, gate->scale, d3, sg, boxw, CU_TENSOR_MAP_SWIZZLE_NONE);
+      if (s == MOE_OK)
+        s = make_map(&sf1[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, up->scale, d3, su, boxw, CU_TENSOR_MAP_SWIZZLE_NONE);
+      if (s == MOE_OK)
+        s = make_map(&sf1[2], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w + L.a1_scale, dx, sx, boxt, CU_TENSOR_MAP_SWIZZLE_NONE);
+      if (s != MOE_OK) return s;
+    }
+    if (sf2_ok) {
+      const uint64_t d3[3] = {uint64_t(pr.I / 32), uint64_t(pr.H), uint64_t(pr.E)};
+      const uint64_t sw[2] = {uint64_t(w2->scale_strides[1]), uint64_t(w2->scale_strides[0])};
+      const uint64_t dh[2] = {uint64_t(pr.I / 32), uint64_t(L.p_max)};
+      const uint64_t sh[1] = {uint64_t(pr.I / 32)};
+      s = make_map(&sf2[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w2->scale, d3, sw, boxw, CU_TENSOR_MAP_SWIZZLE_NONE);
+      if (s == MOE_OK)
+        s = make_map(&sf2[2], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, w + L.h_scale, dh, sh, boxt, CU_TENSOR_MAP_SWIZZLE_NONE);
+      if (s != MOE_OK) return s;
+      sf2[1] = sf2[0];
+    }
+  }
+  rc = launch_gemm_ws_mxfp4(0, cfg.tile, mGate, mUp, mA1, sf1_ok ? sf1 : nullptr, g1, dev->num_sms, st,
+                            &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm1_mxfp4");
   prof_mark(st);
   WsGemmMx g2 = g1;
@@ -573,7 +613,8 @@ moe_status_t forward_mxfp4(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   g2.w1_s1 = g2.w0_s1;
   g2.w_row = reinterpret_cast<const float*>(w + L.w_row);
   g2.h_capture = nullptr;
-  rc = launch_gemm_ws_mxfp4(1, cfg.tile, mW2, mW2, mH, g2, dev->num_sms, st, &launches);
+  rc = launch_gemm_ws_mxfp4(1, cfg.tile, mW2, mW2, mH, sf2_ok ? sf2 : nullptr, g2, dev->num_sms, st,
+                            &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm2_mxfp4");
   prof_mark(st);
   rc = launch_combine(reinterpret_cast<const __nv_bfloat16*>(w + L.y), inv, pr.T, pr.H, pr.k,

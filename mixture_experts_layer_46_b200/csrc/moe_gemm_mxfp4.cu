@@ -18,10 +18,13 @@
 //   warp 1    TMEM allocator, MMA issuer: per stage copies the stage's scales
 //             from shared memory to TMEM (tcgen05.cp 32x128b.warpx4) and issues
 //             2 x 4 x tcgen05.mma.kind::mxf4.block_scale (M=128, N=tile, K=64)
-//   warp 2    scale producer: copies the stage's e8m0 scales through their
-//             strides with 4-byte cp.async straight into the 128-row x 4-block
-//             atom the tensor core reads: byte (row % 32) * 16 + (row / 32) * 4
-//             + block; the stage barrier completes when the copies land
+//   warp 2    scale producer: puts the stage's e8m0 scales into the 128-row x
+//             4-block atom the tensor core reads: byte (row % 32) * 16 +
+//             (row / 32) * 4 + block.  Where the scale views are 16-byte aligned
+//             the TMA producer also loads the raw scale rows of every pair of
+//             k-blocks ([rows x 16 bytes], in the same stream as the codes) and
+//             this warp only moves their words into the atoms; otherwise it
+//             copies them through their strides with 4-byte cp.async.
 //   warps 3-10 epilogue: two warps per 32-lane TMEM quadrant (one weight row
 //             per thread), each taking every other 32-token chunk
 // TMEM: kBufs accumulator buffers of 2 x kNmax columns, then 24 scale columns
@@ -45,8 +48,14 @@ constexpr int kFirstEpiWarp = 2 + kSfWarps;
 constexpr int kStagingTile = 32 * 64;                 // a 32 x 32 bf16 tile (or 32 x 32 codes)
 constexpr int kStagingBytes = kStagingTile + 32 * 4;  // + the chunk's 32 routing weights (GEMM2)
 constexpr int kSfColsPerStage = 24;
+constexpr int kSfRing = 3;                     // raw scale slots (pairs of k-blocks), TMA path
 constexpr int kTmemCols = 512;
 constexpr int kThreads = 32 * (kFirstEpiWarp + kEpiWarps);
+
+__device__ __forceinline__ void st_shared_v4(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w)
+               : "memory");
+}
 
 template <int kNmax, int kStages>
 struct Cfg {
@@ -59,8 +68,13 @@ struct Cfg {
   static constexpr int kBufs = (2 * kBufCols + kStages * kSfColsPerStage <= kTmemCols) ? 2 : 1;
   static constexpr int kSfCol0 = kBufs * kBufCols;
   static_assert(kSfCol0 + kStages * kSfColsPerStage <= kTmemCols, "TMEM budget");
-  static constexpr size_t kSmem = 1024 + size_t(kStages) * kStageBytes +
-                                  kEpiWarps * kStagingBytes + (2 * kStages + 5) * 8 + 16;
+  // raw scale slot (TMA path): 16 bytes (two k-blocks) for each row of W0, W1 and the token tile
+  static constexpr int kSfRawBytes = (2 * kWRows + kNmax) * 16;
+  static constexpr uint32_t kSfRawTx = static_cast<uint32_t>(kSfRawBytes);
+  static constexpr size_t kSmem = 1024 + size_t(kStages) * kStageBytes + kEpiWarps * kStagingBytes +
+                                  size_t(kSfRing) * kSfRawBytes + (2 * kStages + 2 * kSfRing + 5) * 8 + 16;
+  static_assert(kSmem <= 232448, "shared memory per block");
+  static_assert(kSfRawBytes % 128 == 0, "TMA destinations stay 128-byte aligned");
 };
 
 struct MxArgs {
@@ -91,6 +105,9 @@ struct MxArgs {
 struct Smem {
   uint8_t* stages;
   uint8_t* staging;
+  uint8_t* sf_raw;
+  uint64_t* raw_full;
+  uint64_t* raw_empty;
   uint64_t* full;
   uint64_t* empty;
   uint64_t* tfull;
@@ -106,7 +123,11 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
   s.stages = base;
   s.staging = base + kStages * C::kStageBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(s.staging + kEpiWarps * kStagingBytes);
+  s.sf_raw = s.staging + kEpiWarps * kStagingBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s.sf_raw + kSfRing * C::kSfRawBytes);
+  s.raw_full = bars;
+  s.raw_empty = bars + kSfRing;
+  bars += 2 * kSfRing;
   s.full = bars;
   s.empty = bars + kStages;
   s.tfull = bars + 2 * kStages;
@@ -116,11 +137,14 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   return s;
 }
 
-template <int kMode, int kNmax, int kStages>
+template <int kMode, int kNmax, int kStages, bool kTmaSf>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_ws_mxfp4_kernel(const __grid_constant__ CUtensorMap tmW0,
                          const __grid_constant__ CUtensorMap tmW1,
-                         const __grid_constant__ CUtensorMap tmX, const MxArgs g) {
+                         const __grid_constant__ CUtensorMap tmX,
+                         const __grid_constant__ CUtensorMap tmSf0,
+                         const __grid_constant__ CUtensorMap tmSf1,
+                         const __grid_constant__ CUtensorMap tmSfX, const MxArgs g) {
   using C = Cfg<kNmax, kStages>;
   extern __shared__ uint8_t smem_raw[];
   const Smem sm = carve<kNmax, kStages>(smem_raw);
@@ -130,6 +154,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tmW0);
     if (kMode == 0) tma_prefetch_desc(&tmW1);
     tma_prefetch_desc(&tmX);
+    if (kTmaSf) {
+      tma_prefetch_desc(&tmSf0);
+      if (kMode == 0) tma_prefetch_desc(&tmSf1);
+      tma_prefetch_desc(&tmSfX);
+      for (int r = 0; r < kSfRing; ++r) {
+        mbar_init(&sm.raw_full[r], 1);    // the TMA producer (with bytes)
+        mbar_init(&sm.raw_empty[r], 32);  // every lane of the scale producer
+      }
+    }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.full[s], 1 + 32);  // TMA producer (with bytes) + 32 scale-producer lanes
       mbar_init(&sm.empty[s], 1);
@@ -157,9 +190,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (elect_one()) {
-      uint32_t stage = 0, phase = 0;
-      int8_t last_phase[kStages];
+      uint32_t stage = 0, phase = 0, rslot = 0, rphase = 0;
+      int8_t last_phase[kStages], last_rphase[kSfRing];
       for (int s = 0; s < kStages; ++s) last_phase[s] = -1;
+      for (int r = 0; r < kSfRing; ++r) last_rphase[r] = -1;
       const uint64_t pol = l2_policy_evict_last();
       bool ok = true;
       for (int64_t item = blockIdx.x; item < total && ok; item += gridDim.x) {
@@ -174,6 +208,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* sw0 = sm.stages + stage * C::kStageBytes;
           uint8_t* sw1 = sw0 + C::kWBytes;
           uint8_t* sx = sw1 + C::kWBytes;
+          if (kTmaSf && (kb & 1) == 0) {
+            // raw scale rows of k-blocks kb and kb + 1: [W0 128 x 16 B][W1 128 x 16 B][X kNmax x 16 B];
+            // rows past the weight matrix or the token rows read as zeros
+            if (!mbar_wait(&sm.raw_empty[rslot], rphase ^ 1u, g.err)) { ok = false; break; }
+            uint8_t* raw = sm.sf_raw + rslot * C::kSfRawBytes;
+            mbar_arrive_expect_tx(&sm.raw_full[rslot], C::kSfRawTx);
+            tma_load_3d(raw, &tmSf0, &sm.raw_full[rslot], kb * 8, w0, e, pol);
+            tma_load_3d(raw + kWRows * 16, kMode == 0 ? &tmSf1 : &tmSf0, &sm.raw_full[rslot], kb * 8, w1, e, pol);
+            tma_load_2d(raw + 2 * kWRows * 16, &tmSfX, &sm.raw_full[rslot], kb * 8, row0, pol);
+            last_rphase[rslot] = static_cast<int8_t>(rphase);
+            if (++rslot == kSfRing) { rslot = 0; rphase ^= 1u; }
+          }
           mbar_arrive_expect_tx(&sm.full[stage], bytes);
           tma_load_3d(sw0, &tmW0, &sm.full[stage], kb * kRowBytes, w0, e, pol);
           tma_load_3d(sw1, kMode == 0 ? &tmW1 : &tmW0, &sm.full[stage], kb * kRowBytes, w1, e, pol);
@@ -187,6 +233,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) {
         for (int s = 0; s < kStages; ++s)
           if (last_phase[s] >= 0) mbar_wait(&sm.full[s], static_cast<uint32_t>(last_phase[s]), g.err);
+        for (int r = 0; r < kSfRing; ++r)
+          if (last_rphase[r] >= 0) mbar_wait(&sm.raw_full[r], static_cast<uint32_t>(last_rphase[r]), g.err);
+      }
+    }
+  } else if (kTmaSf && warp >= 2 && warp < kFirstEpiWarp) {
+    // ------------------------------------------------------------ scale producer (TMA path)
+    // Lane l moves the words of rows l, l+32, l+64 and l+96: an atom row is the
+    // words of four rows 32 apart, so each atom takes one 16-byte shared store
+    // per lane.  Token rows past the tile get zero scales.
+    uint32_t stage = 0, phase = 0, rslot = 0, rphase = 0;
+    bool ok = true;
+    for (int64_t item = blockIdx.x; item < total && ok; item += gridDim.x) {
+      const int64_t t = item / g.n_wt;
+      const int32_t rows = g.tile_rows[t];
+      for (int kb = 0; kb < num_k; ++kb) {
+        if ((kb & 1) == 0 && !mbar_wait(&sm.raw_full[rslot], rphase, g.err)) { ok = false; break; }
+        if (!mbar_wait(&sm.empty[stage], phase ^ 1u, g.err)) { ok = false; break; }
+        const uint32_t raw = smem_u32(sm.sf_raw + rslot * C::kSfRawBytes) + (kb & 1) * 8;
+        const uint32_t sf = smem_u32(sm.stages + stage * C::kStageBytes + 2 * C::kWBytes + C::kTokBytes);
+#pragma unroll
+        for (int o = 0; o < 3; ++o) {
+          uint32_t lo[4], hi[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int r = lane + 32 * j;
+            lo[j] = 0u;
+            hi[j] = 0u;
+            if (o < 2 || r < rows)
+              asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];"
+                           : "=r"(lo[j]), "=r"(hi[j]) : "r"(raw + (o * kWRows + r) * 16) : "memory");
+          }
+          st_shared_v4(sf + o * kSfBytes + 16 * lane, lo[0], lo[1], lo[2], lo[3]);
+          st_shared_v4(sf + o * kSfBytes + kAtomBytes + 16 * lane, hi[0], hi[1], hi[2], hi[3]);
+        }
+        fence_proxy_async_smem();  // the tensor core's tcgen05.cp reads these bytes
+        mbar_arrive(&sm.full[stage]);
+        if ((kb & 1) == 1 || kb + 1 == num_k) {
+          mbar_arrive(&sm.raw_empty[rslot]);  // this lane's reads of the slot are done
+          if (++rslot == kSfRing) { rslot = 0; rphase ^= 1u; }
+        }
+        if (++stage == kStages) { stage = 0; phase ^= 1u; }
       }
     }
   } else if (warp >= 2 && warp < kFirstEpiWarp) {
@@ -426,16 +513,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int kMode, int kNmax, int kStages>
-cudaError_t launch_mx(const CUtensorMap& w0, const CUtensorMap& w1, const CUtensorMap& x,
-                      const MxArgs& g, int64_t max_items, int num_sms, cudaStream_t st) {
+template <int kMode, int kNmax, int kStages, bool kTmaSf>
+cudaError_t launch_mx_sf(const CUtensorMap& w0, const CUtensorMap& w1, const CUtensorMap& x,
+                         const CUtensorMap& sf0, const CUtensorMap& sf1, const CUtensorMap& sfx,
+                         const MxArgs& g, int64_t max_items, int num_sms, cudaStream_t st) {
   using C = Cfg<kNmax, kStages>;
   static unsigned long long configured = 0;
   int dev = 0;
   cudaError_t rc = cudaGetDevice(&dev);
   if (rc != cudaSuccess) return rc;
   if (dev >= 64 || !(configured & (1ull << dev))) {
-    rc = cudaFuncSetAttribute(gemm_ws_mxfp4_kernel<kMode, kNmax, kStages>,
+    rc = cudaFuncSetAttribute(gemm_ws_mxfp4_kernel<kMode, kNmax, kStages, kTmaSf>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(C::kSmem));
     if (rc != cudaSuccess) return rc;
@@ -443,15 +531,25 @@ cudaError_t launch_mx(const CUtensorMap& w0, const CUtensorMap& w1, const CUtens
   }
   int64_t grid = max_items < num_sms ? max_items : num_sms;
   if (grid < 1) grid = 1;
-  return launch_pdl(gemm_ws_mxfp4_kernel<kMode, kNmax, kStages>, dim3(static_cast<unsigned>(grid)),
-                    dim3(kThreads), C::kSmem, st, w0, w1, x, g);
+  return launch_pdl(gemm_ws_mxfp4_kernel<kMode, kNmax, kStages, kTmaSf>, dim3(static_cast<unsigned>(grid)),
+                    dim3(kThreads), C::kSmem, st, w0, w1, x, sf0, sf1, sfx, g);
+}
+
+template <int kMode, int kNmax, int kStages>
+cudaError_t launch_mx(const CUtensorMap& w0, const CUtensorMap& w1, const CUtensorMap& x,
+                      const CUtensorMap* sf, const MxArgs& g, int64_t max_items, int num_sms,
+                      cudaStream_t st) {
+  if (sf)
+    return launch_mx_sf<kMode, kNmax, kStages, true>(w0, w1, x, sf[0], sf[1], sf[2], g, max_items,
+                                                     num_sms, st);
+  return launch_mx_sf<kMode, kNmax, kStages, false>(w0, w1, x, w0, w1, x, g, max_items, num_sms, st);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm_ws_mxfp4(int mode, int tile_max, const CUtensorMap& w0,
-                                 const CUtensorMap& w1, const CUtensorMap& x, const WsGemmMx& p,
-                                 int num_sms, cudaStream_t st, int* launches) {
+                                 const CUtensorMap& w1, const CUtensorMap& x, const CUtensorMap* sf,
+                                 const WsGemmMx& p, int num_sms, cudaStream_t st, int* launches) {
   MxArgs g;
   g.K = p.K;
   g.N = p.N;
@@ -482,16 +580,16 @@ cudaError_t launch_gemm_ws_mxfp4(int mode, int tile_max, const CUtensorMap& w0,
   if (launches) *launches += 1;
   const int64_t max_items = p.max_tiles * p.n_wt;
   if (tile_max == 128) {  // one accumulator buffer: fewer weight re-reads, epilogue not overlapped
-    if (mode == 0) return launch_mx<0, 128, 4>(w0, w1, x, g, max_items, num_sms, st);
-    return launch_mx<1, 128, 4>(w0, w1, x, g, max_items, num_sms, st);
+    if (mode == 0) return launch_mx<0, 128, 3>(w0, w1, x, sf, g, max_items, num_sms, st);
+    return launch_mx<1, 128, 3>(w0, w1, x, sf, g, max_items, num_sms, st);
   }
   if (tile_max == 96) {
-    if (mode == 0) return launch_mx<0, 96, 4>(w0, w1, x, g, max_items, num_sms, st);
-    return launch_mx<1, 96, 4>(w0, w1, x, g, max_items, num_sms, st);
+    if (mode == 0) return launch_mx<0, 96, 4>(w0, w1, x, sf, g, max_items, num_sms, st);
+    return launch_mx<1, 96, 4>(w0, w1, x, sf, g, max_items, num_sms, st);
   }
   if (tile_max == 32) {
-    if (mode == 0) return launch_mx<0, 32, 5>(w0, w1, x, g, max_items, num_sms, st);
-    return launch_mx<1, 32, 5>(w0, w1, x, g, max_items, num_sms, st);
+    if (mode == 0) return launch_mx<0, 32, 5>(w0, w1, x, sf, g, max_items, num_sms, st);
+    return launch_mx<1, 32, 5>(w0, w1, x, sf, g, max_items, num_sms, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -172,10 +172,12 @@ struct WsGemmMx {
   float* h_capture;       // GEMM1: fp32 h before quantisation, [P, I] (inspection; null: off)
   DeviceErrors* err;
 };
-// tile_max: 96 (4-stage ring) or 32 (5-stage ring)
+// tile_max: 128 (3-stage ring), 96 (4-stage ring) or 32 (5-stage ring).  sf: null, or
+// three maps of the raw e8m0 scales (W0, W1, token rows; uint8, no swizzle, boxes of
+// 16 bytes x 128 weight rows and 16 bytes x tile_max token rows) for the TMA scale path.
 cudaError_t launch_gemm_ws_mxfp4(int mode, int tile_max, const CUtensorMap& w0,
-                                 const CUtensorMap& w1, const CUtensorMap& x, const WsGemmMx& p,
-                                 int num_sms, cudaStream_t st, int* launches);
+                                 const CUtensorMap& w1, const CUtensorMap& x, const CUtensorMap* sf,
+                                 const WsGemmMx& p, int num_sms, cudaStream_t st, int* launches);
 
 // MXFP4 quantiser for rows of a [R, K] bf16/f32 matrix (unit inner stride)
 cudaError_t launch_quantize_rows(const void* src, int32_t src_dtype, int64_t R, int64_t K,

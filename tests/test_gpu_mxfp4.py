@@ -139,6 +139,29 @@ def test_mxfp4_strided_equals_contiguous_and_deterministic():
     assert torch.equal(a, d)
 
 
+@pytest.mark.parametrize("tile", [32, 96, 128])
+def test_mxfp4_scale_load_paths_agree(tile):
+    # The GEMMs load e8m0 scale rows by TMA where every scale view is 16-byte
+    # aligned and by 4-byte cp.async otherwise: scale views whose rows are 24 bytes
+    # apart (8-byte aligned only) take the second path and must give the same bits.
+    T, H, I, E, k = 300, 512, 512, 8, 4
+    case = make_mx_case(T, H, I, E, k, seed=tile + 5)
+    ref = mx_oracle(case)
+    c = cuda_case(case)
+    s13p = torch.zeros(E, 2 * I, H // 32 + 8, dtype=torch.uint8, device="cuda")
+    s13p[:, :, :H // 32] = c["s13"]
+    s2p = torch.zeros(E, H, I // 32 + 8, dtype=torch.uint8, device="cuda")
+    s2p[:, :, :I // 32] = c["s2"]
+    with moe.config_override((T, H, I, E, k), mxfp4=True, tile=tile, fused=0):
+        assert moe.get_config(T, H, I, E, k, mxfp4=True)["tile"] == tile
+        a = mx_gpu(c)
+        v = moe.w13_from_packed(c["c13"], s13p[:, :, :H // 32])
+        b = moe.forward(c["x"], v, c["c2"], c["ids"], c["wts"], w2_scale=s2p[:, :, :I // 32])
+        torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    assert rel_err(a, ref) <= MX_TOL
+
+
 def test_mxfp4_stale_workspace_contents_never_reach_the_output():
     # 0xFF scale bytes are NaN in e8m0: padding rows holding them must not matter
     T, H, I, E, k = 45, 512, 256, 6, 3
