@@ -336,6 +336,7 @@ TILE_VARIANTS = {
     (600, 512, 640, 3, 2),     # 400 slots per expert: >1 token tile of 256 rows, N tail of I
     (77, 288, 96, 6, 3),       # ragged K and output columns
     (700, 256, 256, 2, 2),     # 700 slots per expert: two 352-row tiles of the 512-row list
+    (1000, 256, 256, 8, 2),    # ~250 slots per expert: one or two 256-row tiles (paired work items)
 ])
 def test_token_tile_configs_agree_and_match_oracle(T, H, I, E, k):
     # the token-tile size (32 / 128 rows on one CTA, 128 / 256 rows on a CTA pair)
