@@ -13,8 +13,11 @@ with ``mixture_experts_layer_46_b200`` and never imports it.
 Parity pins: tests/test_oracle_pins.py (brute force against a dense numpy
 formulation, the one-expert special case against a textbook SwiGLU MLP, the
 invariants), tests/test_oracle_mxfp4_pins.py (the MXFP4 worked examples and
-brute-force quantiser) and tests/test_oracle_router_pins.py (the router against
-torch's softmax and sort, brute force, ties and invariants).
+brute-force quantiser), tests/test_oracle_router_pins.py (the router against
+torch's softmax and sort, brute force, ties and invariants) and
+tests/test_oracle_backward_pins.py (the input and routing-weight gradient against
+central finite differences of the oracle forward and against torch autograd of a
+dense fp64 formulation).
 """
 
 from __future__ import annotations
@@ -76,6 +79,9 @@ def _load():
             lib.oracle_moe_forward.argtypes = [P(OracleTensor)] * 6 + [
                 ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
                 ctypes.c_int]
+            lib.oracle_moe_backward_input.restype = ctypes.c_int
+            lib.oracle_moe_backward_input.argtypes = [P(OracleTensor)] * 7 + [
+                ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
             lib.oracle_router_topk.restype = ctypes.c_int
             lib.oracle_router_topk.argtypes = [P(OracleTensor), ctypes.c_int64, ctypes.c_int,
                                                ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
@@ -119,6 +125,27 @@ def e2m1_value(code: int) -> float:
 
 def e8m0_value(code: int) -> float:
     return float(_load().oracle_e8m0_value(code))
+
+
+def moe_backward_input(x, gate, up, w2, ids, weights, dout, *, tokens=None, nthreads=0):
+    """fp64 gradient of the bf16 forward with respect to x and topk_weights (experts
+    frozen), given dout = dL/dout [T, H].  Returns (dx [n, H], dweights [n, k]) float64
+    for the tokens listed (default all)."""
+    d = [_desc(v) for v in (x, gate, up, w2, ids, weights, dout)]
+    T, H = x.shape
+    k = ids.shape[1]
+    if tokens is not None:
+        tokens = tokens.to(torch.int64).contiguous()
+        n_out, tptr = tokens.numel(), tokens.data_ptr()
+    else:
+        n_out, tptr = T, None
+    dx = torch.zeros(n_out, H, dtype=torch.float64)
+    dw = torch.zeros(n_out, k, dtype=torch.float64)
+    rc = _load().oracle_moe_backward_input(*[ctypes.byref(v) for v in d], tptr, n_out,
+                                           dx.data_ptr(), dw.data_ptr(), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_moe_backward_input: shape mismatch")
+    return dx, dw
 
 
 def router_topk(logits: torch.Tensor, k: int, renormalize: bool = True, shared_expert: bool = False):

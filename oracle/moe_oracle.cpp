@@ -291,6 +291,86 @@ int oracle_moe_forward(const oracle_tensor_t* x, const oracle_tensor_t* gate,
   return 0;
 }
 
+// Gradient of the forward with respect to x and topk_weights with the experts
+// frozen (the routing ids are discrete), given dout = dL/dout, in the forward's
+// order: for every token t and column j with e = topk_ids[t, j] in [0, E) and
+// w = topk_weights[t, j]:
+//   g, u, a, y as in the forward;  s_i = 1 / (1 + exp(-g_i))
+//   dweights[t, j] = sum_o dout[t, o] * y_o
+//   da_i = w * sum_o dout[t, o] * w2[e, o, i]
+//   dg_i = da_i * u_i * s_i * (1 + g_i * (1 - s_i))      (the derivative of silu(g) = g s)
+//   du_i = da_i * g_i * s_i
+//   dx[t, h] += sum_i dg_i * gate[e, i, h] + du_i * up[e, i, h]
+// Slots with e outside [0, E) contribute nothing (their dweights is 0).  bf16
+// weights only (the MXFP4 forward's quantisation steps have no gradient).
+//   dout [T, H] bf16/f32 (strided); dx [n_out, H] and dw [n_out, k] fp64, contiguous.
+int oracle_moe_backward_input(const oracle_tensor_t* x, const oracle_tensor_t* gate,
+                              const oracle_tensor_t* up, const oracle_tensor_t* w2,
+                              const oracle_tensor_t* ids, const oracle_tensor_t* weights,
+                              const oracle_tensor_t* dout, const int64_t* tokens, int64_t n_out,
+                              double* dx, double* dw, int nthreads) {
+  const int64_t T = x->sizes[0], H = x->sizes[1];
+  const int64_t E = gate->sizes[0], I = gate->sizes[1];
+  const int64_t k = ids->sizes[1];
+  if (gate->sizes[2] != H || up->sizes[0] != E || up->sizes[1] != I || up->sizes[2] != H ||
+      w2->sizes[0] != E || w2->sizes[1] != H || w2->sizes[2] != I || ids->sizes[0] != T ||
+      weights->sizes[0] != T || weights->sizes[1] != k || dout->sizes[0] != T ||
+      dout->sizes[1] != H || gate->dtype == OR_E2M1X2)
+    return 1;
+  if (!tokens) n_out = T;
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+  for (int64_t r = 0; r < n_out; ++r) {
+    const int64_t t = tokens ? tokens[r] : r;
+    std::vector<double> xt(H), dot(H), g(I), u(I), a(I), dgi(I), dui(I), acc(H, 0.0);
+    for (int64_t h = 0; h < H; ++h) {
+      xt[h] = read_real2(x, t, h);
+      dot[h] = read_real2(dout, t, h);
+    }
+    for (int64_t j = 0; j < k; ++j) {
+      dw[r * k + j] = 0.0;
+      const int64_t e = read_id(ids, t, j);
+      if (e < 0 || e >= E) continue;
+      const double w = read_real2(weights, t, j);
+      for (int64_t i = 0; i < I; ++i) {
+        double gg = 0.0, uu = 0.0;
+        for (int64_t h = 0; h < H; ++h) {
+          gg += xt[h] * read_weight(gate, e, i, h);
+          uu += xt[h] * read_weight(up, e, i, h);
+        }
+        g[i] = gg;
+        u[i] = uu;
+        a[i] = gg / (1.0 + std::exp(-gg)) * uu;
+      }
+      double dwj = 0.0;
+      for (int64_t o = 0; o < H; ++o) {
+        double y = 0.0;
+        for (int64_t i = 0; i < I; ++i) y += a[i] * read_weight(w2, e, o, i);
+        dwj += dot[o] * y;
+      }
+      dw[r * k + j] = dwj;
+      for (int64_t i = 0; i < I; ++i) {
+        double da = 0.0;
+        for (int64_t o = 0; o < H; ++o) da += dot[o] * read_weight(w2, e, o, i);
+        da *= w;
+        const double sg = 1.0 / (1.0 + std::exp(-g[i]));
+        dgi[i] = da * u[i] * sg * (1.0 + g[i] * (1.0 - sg));
+        dui[i] = da * g[i] * sg;
+      }
+      for (int64_t h = 0; h < H; ++h) {
+        double v = 0.0;
+        for (int64_t i = 0; i < I; ++i)
+          v += dgi[i] * read_weight(gate, e, i, h) + dui[i] * read_weight(up, e, i, h);
+        acc[h] += v;
+      }
+    }
+    for (int64_t h = 0; h < H; ++h) dx[r * H + h] = acc[h];
+  }
+  return 0;
+}
+
 // The router that produces the forward's routing inputs, in fp64:
 //   p = softmax(logits[t, :]) over the E experts,
 //   the k experts of largest p, in descending p (a tie goes to the lower expert index),
