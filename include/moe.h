@@ -155,6 +155,37 @@ moe_status_t moe_forward_host(const moe_tensor_t* x_host, const moe_w13_t* w13,
                               const moe_tensor_t* topk_weights_host, moe_tensor_t* out_host,
                               moe_stream_t stream);
 
+/* Gradient path with the experts frozen (bf16 weights): given dout = dL/dout
+ * [T, H] bf16, writes dx = dL/dx [T, H] bf16 and dweights = dL/dtopk_weights
+ * [T, k] f32 (any strides), the routing ids held fixed (they are discrete).
+ * The fused-MoE training path of Liger-Kernel PR #1377 ("Testing Done":
+ * forward and backward CUDA graphs) differentiates this layer; this entry point
+ * covers its input and routing-weight gradients, not the expert weights'.
+ * Per slot (t, j) with e = topk_ids[t, j] in [0, E), w = topk_weights[t, j]:
+ *   dweights[t, j] = dout_t . (w2_e h),  h = silu(gate_e x_t) * (up_e x_t)
+ *   dh = w w2_e^T dout_t;  dg = dh u s (1 + g (1 - s)),  du = dh g s  (s = sigmoid(g))
+ *   dx_t += gate_e^T dg + up_e^T du
+ * Skipped slots (ids outside [0, E)) contribute nothing and get dweights 0.
+ * The GEMMs read the weights K-major, so the caller passes their transposes too:
+ * w13t [E, H, 2I] (the packed w13 [E, 2I, H] transposed: gate^T in columns
+ * [0, I), up^T in [I, 2I)) and w2t [E, I, H]; moe_transpose_experts makes them
+ * (they stay valid while the weights are frozen).  Inner stride 1, 16-byte
+ * aligned strides.  x, w13, w2, topk_ids, topk_weights as for moe_forward_ws;
+ * dx in place of out.  Workspace: moe_backward_workspace_bytes, 256-byte
+ * aligned.  Asynchronous on `stream`, no allocation.  MXFP4 weights:
+ * MOE_ERR_UNSUPPORTED_DTYPE (the forward's quantisation steps have no gradient). */
+size_t moe_backward_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k);
+moe_status_t moe_backward_input_ws(const moe_tensor_t* x, const moe_w13_t* w13, const moe_tensor_t* w2,
+                                   const moe_tensor_t* w13t, const moe_tensor_t* w2t,
+                                   const moe_tensor_t* topk_ids, const moe_tensor_t* topk_weights,
+                                   const moe_tensor_t* dout, moe_tensor_t* dx, moe_tensor_t* dweights,
+                                   void* workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/* dst[e, c, r] = src[e, r, c] for bf16 [E, R, C] -> [E, C, R] (inner stride 1 on
+ * both, other strides free): the K-major weight copies the gradient path reads.
+ * Asynchronous on `stream`. */
+moe_status_t moe_transpose_experts(const moe_tensor_t* src, moe_tensor_t* dst, moe_stream_t stream);
+
 /* Step "align" alone, for inspection and tests: group the T*k slots by expert
  * into block_m-row blocks, block_m being the per-token-bucket block size the
  * aiter kernels tune (ROCm/aiter PR #3859, "Tuned MoE latency": block_m 32, 64

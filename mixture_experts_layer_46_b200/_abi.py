@@ -30,7 +30,8 @@ EXPORTS = ("moe_status_string", "moe_last_cuda_error", "moe_w13_from_packed",
            "moe_profile_enable", "moe_profile_read", "moe_version", "moe_align_noalloc",
            "moe_set_config_table", "moe_get_config", "moe_builtin_config_count",
            "moe_router_topk", "moe_selftest_bounded_wait", "moe_workspace_layout",
-           "moe_debug_capture", "moe_measure_mma_peak")
+           "moe_debug_capture", "moe_measure_mma_peak", "moe_backward_workspace_bytes",
+           "moe_backward_input_ws", "moe_transpose_experts")
 STEP_NAMES = ("align", "permute", "gemm1_swiglu", "gemm2_weighted", "combine")
 
 
@@ -112,6 +113,13 @@ def load() -> ctypes.CDLL:
                                         P(MoeTensor), P(MoeTensor), vp]
             lib.moe_forward_host.restype = ctypes.c_int
             lib.moe_forward_host.argtypes = lib.moe_forward.argtypes
+            lib.moe_backward_workspace_bytes.restype = ctypes.c_size_t
+            lib.moe_backward_workspace_bytes.argtypes = [ctypes.c_int64] * 5
+            lib.moe_backward_input_ws.restype = ctypes.c_int
+            lib.moe_backward_input_ws.argtypes = [P(MoeTensor), P(MoeW13)] + [P(MoeTensor)] * 8 + [
+                vp, ctypes.c_size_t, vp]
+            lib.moe_transpose_experts.restype = ctypes.c_int
+            lib.moe_transpose_experts.argtypes = [P(MoeTensor), P(MoeTensor), vp]
             lib.moe_align.restype = ctypes.c_int
             lib.moe_align.argtypes = [P(MoeTensor), ctypes.c_int64, ctypes.c_int32, vp, vp, vp, vp,
                                       vp, vp, ctypes.c_size_t, vp]
@@ -234,6 +242,41 @@ def forward(x, w13: MoeW13, w2, topk_ids, topk_weights, out=None, *, w2_scale=No
                              ctypes.byref(di), ctypes.byref(dw), ctypes.byref(do), st)
         _check(rc, "moe_forward")
     return out
+
+
+def backward_workspace_bytes(T: int, H: int, I: int, E: int, k: int) -> int:
+    return int(load().moe_backward_workspace_bytes(T, H, I, E, k))
+
+
+def transpose_experts(src: torch.Tensor, dst: torch.Tensor | None = None, *, stream=None) -> torch.Tensor:
+    """dst[e, c, r] = src[e, r, c] (bf16 [E, R, C] -> [E, C, R]) on the GPU."""
+    if dst is None:
+        dst = torch.empty(src.shape[0], src.shape[2], src.shape[1], dtype=src.dtype, device=src.device)
+    ds, dd = desc(src), desc(dst)
+    _check(load().moe_transpose_experts(ctypes.byref(ds), ctypes.byref(dd), _stream_ptr(stream)),
+           "moe_transpose_experts")
+    return dst
+
+
+def backward_input(x, w13: MoeW13, w2, w13t, w2t, topk_ids, topk_weights, dout, dx=None, dweights=None,
+                   *, workspace: torch.Tensor | None = None, stream=None):
+    """(dx, dweights): the forward's gradient with respect to x and the routing
+    weights given dout, experts frozen; w13t [E, H, 2I] and w2t [E, I, H] are the
+    weights' transposes (transpose_experts)."""
+    T, H = x.shape
+    k = topk_ids.shape[1]
+    if dx is None:
+        dx = torch.empty(T, H, dtype=torch.bfloat16, device=x.device)
+    if dweights is None:
+        dweights = torch.empty(T, k, dtype=torch.float32, device=x.device)
+    if workspace is None:
+        n = backward_workspace_bytes(T, H, w2.shape[2], w2.shape[0], k)
+        workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=x.device)
+    d = [desc(v) for v in (x, w2, w13t, w2t, topk_ids, topk_weights, dout, dx, dweights)]
+    rc = load().moe_backward_input_ws(ctypes.byref(d[0]), ctypes.byref(w13), *[ctypes.byref(v) for v in d[1:]],
+                                      workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    _check(rc, "moe_backward_input_ws")
+    return dx, dweights
 
 
 def forward_status(x, w13: MoeW13, w2, topk_ids, topk_weights, out, *, w2_scale=None,

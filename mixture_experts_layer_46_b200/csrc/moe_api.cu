@@ -884,6 +884,180 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
   return MOE_OK;
 }
 
+// ---------------------------------------------------------------- gradient (experts frozen)
+
+// The forward's workspace plus the gradient's own rows: dout gathered into
+// expert-grouped order, dh = dL/dh and [dg | du], each [P_max, .] bf16.
+struct BwdLayout {
+  WsLayout L;
+  size_t d1, dh, dgu, total;
+};
+
+BwdLayout make_bwd_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k) {
+  BwdLayout B;
+  B.L = make_layout(T, H, I, E, k, false, kBm);
+  size_t off = align256(B.L.total);
+  B.d1 = off;
+  off = align256(off + size_t(B.L.p_max) * H * 2);
+  B.dh = off;
+  off = align256(off + size_t(B.L.p_max) * I * 2);
+  B.dgu = off;
+  off = align256(off + size_t(B.L.p_max) * 2 * I * 2);
+  B.total = off;
+  return B;
+}
+
+bool kmajor_bf16(const moe_tensor_t* t, int64_t d0, int64_t d1, int64_t d2) {
+  return t && t->data && t->dtype == MOE_BF16 && t->ndim == 3 && t->sizes[0] == d0 &&
+         t->sizes[1] == d1 && t->sizes[2] == d2 && t->strides[2] == 1 &&
+         (t->strides[1] * 2) % 16 == 0 && (t->strides[0] * 2) % 16 == 0 &&
+         reinterpret_cast<uintptr_t>(t->data) % 16 == 0;
+}
+
+// dx = d out / d x and dweights = d out / d topk_weights contracted with dout,
+// with the routing ids fixed and the experts frozen (see moe.h):
+//   align; x and dout gathered into expert-grouped rows (A1, D1);
+//   dh[p]  = w_slot * w2_e^T dout_t        (GEMM2 kernel on w2^T [E, I, H], K = H)
+//   g, u recomputed from A1 (GEMM1 kernel, mode 3): dg, du -> [dg | du], h
+//   y[p]   = w2_e h[p]                      (GEMM2 kernel, routing weights 1)
+//   dweights[t, j] = dout_t . y[inv(t, j)]  (slot_dot)
+//   da[p]  = [gate_e^T | up_e^T] [dg | du]  (GEMM2 kernel on w13^T [E, H, 2I], K = 2I, weights 1)
+//   dx[t]  = sum_j da[inv(t, j)]            (combine)
+moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe_tensor_t* w2,
+                           const moe_tensor_t* w13t, const moe_tensor_t* w2t,
+                           const moe_tensor_t* ids, const moe_tensor_t* wts,
+                           const moe_tensor_t* dout, moe_tensor_t* dx, moe_tensor_t* dw,
+                           const Problem& pr, void* ws, size_t ws_bytes, cudaStream_t st) {
+  int launches = 0;
+  t_last_launches = 0;
+  if (pr.T == 0) return MOE_OK;
+  const int32_t bm = kBm;
+  const BwdLayout B = make_bwd_layout(pr.T, pr.H, pr.I, pr.E, pr.k);
+  const WsLayout& L = B.L;
+  if (!ws || ws_bytes < B.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return MOE_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  moe_status_t s = device_info(&dev);
+  if (s != MOE_OK) return s;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  int32_t* counts = reinterpret_cast<int32_t*>(w + L.counts);
+  int32_t* offsets = reinterpret_cast<int32_t*>(w + L.offsets);
+  int32_t* num_blocks = reinterpret_cast<int32_t*>(w + L.num_blocks);
+  int32_t* chunk_counts = reinterpret_cast<int32_t*>(w + L.chunk_counts);
+  int32_t* sorted = reinterpret_cast<int32_t*>(w + L.sorted);
+  int32_t* inv = reinterpret_cast<int32_t*>(w + L.inv);
+  int32_t* block_expert = reinterpret_cast<int32_t*>(w + L.block_expert);
+  const moe_tensor_t* gate = &w13->gate;
+  const moe_tensor_t* up = &w13->up;
+
+  // every GEMM on 128-row token tiles, one CTA each (tensor maps: 128-byte swizzle)
+  constexpr int32_t kTile = 128;
+  const uint32_t boxw[3] = {64, 128, 1};
+  const uint32_t boxt[2] = {64, static_cast<uint32_t>(kTile)};
+  CUtensorMap mA1, mD1, mHh, mDGU, mGate, mUp, mW2, mW2T, mW13T;
+  auto rows_map = [&](CUtensorMap* m, uint8_t* base, int64_t K) {
+    const uint64_t d[2] = {uint64_t(K), uint64_t(L.p_max)};
+    const uint64_t sb[1] = {uint64_t(K) * 2};
+    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, d, sb, boxt, CU_TENSOR_MAP_SWIZZLE_128B);
+  };
+  auto weight_map = [&](CUtensorMap* m, const moe_tensor_t* t, int64_t K, int64_t N) {
+    const uint64_t d[3] = {uint64_t(K), uint64_t(N), uint64_t(pr.E)};
+    const uint64_t sb[2] = {uint64_t(t->strides[1]) * 2, uint64_t(t->strides[0]) * 2};
+    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, t->data, d, sb, boxw, CU_TENSOR_MAP_SWIZZLE_128B);
+  };
+  if ((s = rows_map(&mA1, w + L.a1, pr.H)) != MOE_OK) return s;
+  if ((s = rows_map(&mD1, w + B.d1, pr.H)) != MOE_OK) return s;
+  if ((s = rows_map(&mHh, w + L.h, pr.I)) != MOE_OK) return s;
+  if ((s = rows_map(&mDGU, w + B.dgu, 2 * pr.I)) != MOE_OK) return s;
+  if ((s = weight_map(&mGate, gate, pr.H, pr.I)) != MOE_OK) return s;
+  if ((s = weight_map(&mUp, up, pr.H, pr.I)) != MOE_OK) return s;
+  if ((s = weight_map(&mW2, w2, pr.I, pr.H)) != MOE_OK) return s;
+  if ((s = weight_map(&mW2T, w2t, pr.H, pr.I)) != MOE_OK) return s;
+  if ((s = weight_map(&mW13T, w13t, 2 * pr.I, pr.H)) != MOE_OK) return s;
+
+  AlignTiles tiles;
+  std::memset(&tiles, 0, sizeof(tiles));
+  tiles.list[0].tile_max = kTile;
+  tiles.list[0].tile_row = reinterpret_cast<int32_t*>(w + L.tile_row);
+  tiles.list[0].tile_rows = reinterpret_cast<int32_t*>(w + L.tile_rows);
+  tiles.list[0].tile_expert = reinterpret_cast<int32_t*>(w + L.tile_expert);
+  tiles.list[0].num_tiles = num_blocks + 1;
+  cudaError_t rc = launch_align(view2(ids), pr.T, pr.k, pr.E, bm, counts, offsets, sorted, inv,
+                                block_expert, num_blocks, chunk_counts, L.n_chunks, dev->errors, st,
+                                &launches, &tiles);
+  if (rc != cudaSuccess) return cuda_fail(rc, "align");
+  rc = launch_permute_bf16(view2(x), pr.T, pr.H, pr.k, inv, reinterpret_cast<__nv_bfloat16*>(w + L.a1),
+                           st, &launches);
+  if (rc != cudaSuccess) return cuda_fail(rc, "permute x");
+  rc = launch_permute_bf16(view2(dout), pr.T, pr.H, pr.k, inv,
+                           reinterpret_cast<__nv_bfloat16*>(w + B.d1), st, &launches);
+  if (rc != cudaSuccess) return cuda_fail(rc, "permute dout");
+
+  WsGemm gb;
+  std::memset(&gb, 0, sizeof(gb));
+  gb.max_tiles = L.t_max;
+  gb.num_tiles = tiles.list[0].num_tiles;
+  gb.tile_row = tiles.list[0].tile_row;
+  gb.tile_rows = tiles.list[0].tile_rows;
+  gb.tile_expert = tiles.list[0].tile_expert;
+  gb.sorted = sorted;
+  gb.S = L.S;
+  gb.k = pr.k;
+  gb.err = dev->errors;
+  gb.tok_box = kTile;
+  gb.topk_w = view2(wts);
+
+  WsGemm g = gb;  // dh = w * w2^T dout
+  g.K = pr.H;
+  g.N = pr.I;
+  g.n_wt = (pr.I + 255) / 256;
+  g.out = w + B.dh;
+  g.out_ld = pr.I;
+  rc = launch_gemm_ws_bf16(1, kTile, mW2T, mW2T, mD1, g, dev->num_sms, st, &launches);
+  if (rc != cudaSuccess) return cuda_fail(rc, "gemm dh");
+
+  g = gb;  // g, u recomputed: [dg | du] and h
+  g.K = pr.H;
+  g.N = pr.I;
+  g.n_wt = (pr.I + 127) / 128;
+  g.out = w + B.dgu;
+  g.out_ld = 2 * pr.I;
+  g.dh = w + B.dh;
+  g.dh_ld = pr.I;
+  g.h_out = w + L.h;
+  g.h_ld = pr.I;
+  rc = launch_gemm_ws_bf16(3, kTile, mGate, mUp, mA1, g, dev->num_sms, st, &launches);
+  if (rc != cudaSuccess) return cuda_fail(rc, "gemm dg du");
+
+  g = gb;  // y = w2 h, unweighted
+  g.K = pr.I;
+  g.N = pr.H;
+  g.n_wt = (pr.H + 255) / 256;
+  g.out = w + L.y;
+  g.out_ld = pr.H;
+  g.unit_w = 1;
+  rc = launch_gemm_ws_bf16(1, kTile, mW2, mW2, mHh, g, dev->num_sms, st, &launches);
+  if (rc != cudaSuccess) return cuda_fail(rc, "gemm y");
+  rc = launch_slot_dot(view2(dout), reinterpret_cast<const __nv_bfloat16*>(w + L.y), inv, pr.T, pr.H,
+                       pr.k, view2(dw), st, &launches);
+  if (rc != cudaSuccess) return cuda_fail(rc, "slot_dot");
+
+  g = gb;  // da = [gate^T | up^T] [dg | du]
+  g.K = 2 * pr.I;
+  g.N = pr.H;
+  g.n_wt = (pr.H + 255) / 256;
+  g.out = w + L.y;
+  g.out_ld = pr.H;
+  g.unit_w = 1;
+  rc = launch_gemm_ws_bf16(1, kTile, mW13T, mW13T, mDGU, g, dev->num_sms, st, &launches);
+  if (rc != cudaSuccess) return cuda_fail(rc, "gemm da");
+  rc = launch_combine(reinterpret_cast<const __nv_bfloat16*>(w + L.y), inv, pr.T, pr.H, pr.k,
+                      dx->data, dx->strides[0], dx->strides[1], st, &launches);
+  if (rc != cudaSuccess) return cuda_fail(rc, "combine dx");
+  t_last_launches = launches;
+  return MOE_OK;
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -981,6 +1155,47 @@ moe_status_t moe_forward(const moe_tensor_t* x, const moe_w13_t* w13, const moe_
   if (s != MOE_OK) return s;
   return forward_impl(x, w13, w2, topk_ids, topk_weights, out, pr, ws, need,
                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t moe_backward_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k) {
+  if (T < 0 || H <= 0 || I <= 0 || E <= 0 || k <= 0) return 0;
+  return make_bwd_layout(T, H, I, E, k).total;
+}
+
+moe_status_t moe_backward_input_ws(const moe_tensor_t* x, const moe_w13_t* w13, const moe_tensor_t* w2,
+                                   const moe_tensor_t* w13t, const moe_tensor_t* w2t,
+                                   const moe_tensor_t* topk_ids, const moe_tensor_t* topk_weights,
+                                   const moe_tensor_t* dout, moe_tensor_t* dx, moe_tensor_t* dweights,
+                                   void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+  t_last_launches = 0;
+  Problem pr;
+  moe_status_t s = validate(x, w13, w2, topk_ids, topk_weights, dx, false, &pr);
+  if (s != MOE_OK) return s;
+  if (pr.mxfp4) return MOE_ERR_UNSUPPORTED_DTYPE;
+  if (!w13t || !w2t || !dout || !dweights) return MOE_ERR_INVALID_ARG;
+  if (!kmajor_bf16(w13t, pr.E, pr.H, 2 * pr.I) || !kmajor_bf16(w2t, pr.E, pr.I, pr.H))
+    return MOE_ERR_UNSUPPORTED_LAYOUT;
+  if (!sizes_ok(dout, 2) || dout->sizes[0] != pr.T || dout->sizes[1] != pr.H) return MOE_ERR_SHAPE_MISMATCH;
+  if (dout->dtype != MOE_BF16 || dweights->dtype != MOE_F32) return MOE_ERR_UNSUPPORTED_DTYPE;
+  if (!sizes_ok(dweights, 2) || dweights->sizes[0] != pr.T || dweights->sizes[1] != pr.k)
+    return MOE_ERR_SHAPE_MISMATCH;
+  if (!dout->data || !dweights->data) return MOE_ERR_INVALID_ARG;
+  return backward_impl(x, w13, w2, w13t, w2t, topk_ids, topk_weights, dout, dx, dweights, pr, workspace,
+                       workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_transpose_experts(const moe_tensor_t* src, moe_tensor_t* dst, moe_stream_t stream) {
+  if (!src || !dst || !src->data || !dst->data) return MOE_ERR_INVALID_ARG;
+  if (src->dtype != MOE_BF16 || dst->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED_DTYPE;
+  if (src->ndim != 3 || dst->ndim != 3) return MOE_ERR_SHAPE_MISMATCH;
+  const int64_t E = src->sizes[0], R = src->sizes[1], C = src->sizes[2];
+  if (E < 0 || R < 0 || C < 0 || dst->sizes[0] != E || dst->sizes[1] != C || dst->sizes[2] != R)
+    return MOE_ERR_SHAPE_MISMATCH;
+  if (src->strides[2] != 1 || dst->strides[2] != 1) return MOE_ERR_UNSUPPORTED_LAYOUT;
+  const cudaError_t rc = launch_transpose_experts(src->data, src->strides[0], src->strides[1], dst->data,
+                                                  dst->strides[0], dst->strides[1], E, R, C,
+                                                  reinterpret_cast<cudaStream_t>(stream));
+  return rc == cudaSuccess ? MOE_OK : cuda_fail(rc, "transpose");
 }
 
 moe_status_t moe_forward_host(const moe_tensor_t* x_host, const moe_w13_t* w13,

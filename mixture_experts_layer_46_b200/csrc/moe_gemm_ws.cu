@@ -71,6 +71,11 @@ struct WsArgs {
   View2 pre_ids;     // GEMM1, at most 32 slots: routing ids (pre_S = 0: not used)
   int32_t pre_E, pre_S;
   DeviceErrors* err;
+  int32_t unit_w;    // GEMM2: weight 1 for every routed slot
+  const __nv_bfloat16* dh;  // mode 3: gradient of h [P, N], row stride dh_ld
+  int64_t dh_ld;
+  __nv_bfloat16* h_out;     // mode 3: recomputed h [P, N], row stride h_ld
+  int64_t h_ld;
 };
 
 // Decode batches (at most 32 routing slots on 32-row tiles) have one tile per
@@ -136,6 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemm_ws_bf16_kernel(const __grid_constant__ CUtensorMap tmW0,
                         const __grid_constant__ CUtensorMap tmW1,
                         const __grid_constant__ CUtensorMap tmX, const WsArgs g) {
+  constexpr bool kG1 = kMode == 0 || kMode == 3;  // gate and up tiles (GEMM1 forms)
   using C = Cfg<kNmax, kStages>;
   extern __shared__ uint8_t smem_raw[];
   const Smem<kStages> sm = carve<kNmax, kStages>(smem_raw);
@@ -143,7 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmW0);
-    if (kMode == 0) tma_prefetch_desc(&tmW1);
+    if (kG1) tma_prefetch_desc(&tmW1);
     tma_prefetch_desc(&tmX);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.full[s], 1);
@@ -208,8 +214,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int64_t item = blockIdx.x; item < total && ok; item += gridDim.x) {
         const int64_t t = item / g.n_wt, wt = item - t * g.n_wt;
         const int32_t e = g.tile_expert[t], row0 = g.tile_row[t], rows = g.tile_rows[t];
-        const int32_t w0 = static_cast<int32_t>(kMode == 0 ? wt * kWRows : wt * 2 * kWRows);
-        const int32_t w1 = kMode == 0 ? w0 : w0 + kWRows;
+        const int32_t w0 = static_cast<int32_t>(kG1 ? wt * kWRows : wt * 2 * kWRows);
+        const int32_t w1 = kG1 ? w0 : w0 + kWRows;
         // whole boxes: a box may run past the tile (rows the MMA's N excludes)
         const int nbox = (rows + g.tok_box - 1) / g.tok_box;
         const uint32_t tok_bytes = nbox * g.tok_box * kBK * 2;
@@ -232,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             mbar_arrive_expect_tx(&sm.full[stage], bytes);
             tma_load_3d(sw0, &tmW0, &sm.full[stage], kb * kBK, w0, e, wpol);
-            tma_load_3d(sw1, kMode == 0 ? &tmW1 : &tmW0, &sm.full[stage], kb * kBK, w1, e, wpol);
+            tma_load_3d(sw1, kG1 ? &tmW1 : &tmW0, &sm.full[stage], kb * kBK, w1, e, wpol);
           }
           for (int b = 0; b < nbox; ++b)
             tma_load_2d(sx + b * g.tok_box * kBK * 2, &tmX, &sm.full[stage], kb * kBK,
@@ -318,19 +324,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           w_r[c] = 0.0f;
           if (slot_r[c] < g.S) {
             const int64_t tt = slot_r[c] / g.k, jj = slot_r[c] - tt * g.k;
-            w_r[c] = static_cast<const float*>(g.topk_w.data)[tt * g.topk_w.s0 + jj * g.topk_w.s1];
+            w_r[c] = g.unit_w ? 1.0f
+                              : static_cast<const float*>(g.topk_w.data)[tt * g.topk_w.s0 + jj * g.topk_w.s1];
           }
         }
       }
       if (!mbar_wait(&sm.tfull[buf], acc_phase, g.err)) break;
       tc_fence_after();
       const uint32_t lane_base = (static_cast<uint32_t>(quad * 32) << 16) + buf * C::kBufCols;
-      constexpr int kAccs = (kMode == 0) ? 1 : 2;  // GEMM1 combines both into one output
+      constexpr int kAccs = kG1 ? 1 : 2;  // GEMM1 combines both into one output
 #pragma unroll 1
       for (int a = 0; a < kAccs; ++a) {
         // output column (weight row) block of this warp
-        const int64_t col0 = (kMode == 0) ? wt * kWRows + quad * 32
-                                          : wt * 2 * kWRows + a * kWRows + quad * 32;
+        const int64_t col0 = kG1 ? wt * kWRows + quad * 32 : wt * 2 * kWRows + a * kWRows + quad * 32;
         const bool col_ok = col0 < g.N;
 #pragma unroll
         for (int c = 0; c < kNmax / 32; ++c) {
@@ -339,6 +345,48 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float my_w = (kMode == 1) ? w_r[c] : 0.0f;
           uint32_t v0[32];
           tmem_ld32(tmem_base + lane_base + a * kNmax + c * 32, v0);
+          if (kMode == 3) {
+            // gradient of h = silu(g) u for this warp's 32 rows of I and the chunk's
+            // 32 token rows: dg, du and h go out through the staging tile in turn
+            uint32_t v1[32];
+            tmem_ld32(tmem_base + lane_base + kNmax + c * 32, v1);
+            float dhv[32];
+            const __nv_bfloat16* dsrc = g.dh + (row0 + c * 32) * g.dh_ld + col0 + lane;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) dhv[j] = col_ok ? __bfloat162float(dsrc[j * g.dh_ld]) : 0.0f;
+            tmem_wait_ld();
+#pragma unroll 1
+            for (int o = 0; o < 3; ++o) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const float gg = __uint_as_float(v0[j]), uu = __uint_as_float(v1[j]);
+                const float sg = __fdividef(1.0f, 1.0f + __expf(-gg));
+                const float v = o == 0 ? dhv[j] * uu * sg * (1.0f + gg * (1.0f - sg))
+                              : o == 1 ? dhv[j] * gg * sg
+                                       : gg * sg * uu;
+                const __nv_bfloat16 vb = __float2bfloat16_rn(v);
+                asm volatile("st.shared.b16 [%0], %1;" ::"r"(stg_s + j * 64 + lane * 2),
+                             "h"(*reinterpret_cast<const uint16_t*>(&vb)) : "memory");
+              }
+              __syncwarp();
+              __nv_bfloat16* dst = o == 2 ? g.h_out : static_cast<__nv_bfloat16*>(g.out);
+              const int64_t ld = o == 2 ? g.h_ld : g.out_ld;
+              const int64_t cbase = col0 + (o == 1 ? g.N : 0);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int idx = q * 32 + lane;
+                const int j = idx >> 2, part = idx & 3;
+                uint4 v;
+                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                             : "r"(stg_s + j * 64 + part * 16));
+                if (col_ok)
+                  *reinterpret_cast<uint4*>(dst + (row0 + c * 32 + j) * ld + cbase + part * 8) = v;
+              }
+              __syncwarp();
+            }
+            continue;
+          }
           if (kMode == 0) {
             uint32_t v1[32];
             tmem_ld32(tmem_base + lane_base + kNmax + c * 32, v1);
@@ -444,10 +492,17 @@ cudaError_t launch_gemm_ws_bf16(int mode, int tile_max, const CUtensorMap& w0,
   g.pre_ids = p.pre_ids;
   g.pre_E = p.pre_E;
   g.pre_S = (mode == 0 && tile_max == 32 && p.pre_S <= 32) ? p.pre_S : 0;
+  g.unit_w = p.unit_w;
+  g.dh = static_cast<const __nv_bfloat16*>(p.dh);
+  g.dh_ld = p.dh_ld;
+  g.h_out = static_cast<__nv_bfloat16*>(p.h_out);
+  g.h_ld = p.h_ld;
+  if (mode == 3 && (!p.dh || !p.h_out)) return cudaErrorInvalidValue;
   if (launches) *launches += 1;
   const int64_t max_items = p.max_tiles * p.n_wt;
   if (tile_max == 128) {
     if (mode == 0) return launch_ws<0, 128, 4>(w0, w1, x, g, max_items, num_sms, st);
+    if (mode == 3) return launch_ws<3, 128, 4>(w0, w1, x, g, max_items, num_sms, st);
     return launch_ws<1, 128, 4>(w0, w1, x, g, max_items, num_sms, st);
   }
   if (tile_max == 32) {

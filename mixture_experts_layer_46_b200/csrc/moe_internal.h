@@ -99,6 +99,16 @@ cudaError_t launch_permute_quant(const View2& x, int64_t T, int64_t H, int64_t k
                                  const View2& topk_w, float* w_row, cudaStream_t st,
                                  int* launches);
 
+// routing-weight gradient: dw[t, j] = sum_o dout[t, o] * y[inv[t*k + j], o] (fp32;
+// 0 for a skipped slot); dout [T, H] bf16 strided, dw [T, k] f32 strided
+cudaError_t launch_slot_dot(const View2& dout, const __nv_bfloat16* y, const int32_t* inv,
+                            int64_t T, int64_t H, int64_t k, const View2& dw, cudaStream_t st,
+                            int* launches);
+
+// dst[e, c, r] = src[e, r, c] for bf16 [E, R, C] (element strides; inner stride 1 both)
+cudaError_t launch_transpose_experts(const void* src, int64_t s0, int64_t s1, void* dst, int64_t d0,
+                                     int64_t d1, int64_t E, int64_t R, int64_t C, cudaStream_t st);
+
 // combine: out[t, :] = sum_j y[inv[t*k + j], :] over valid slots (fixed j order)
 cudaError_t launch_combine(const __nv_bfloat16* y, const int32_t* inv, int64_t T, int64_t H,
                            int64_t k, void* out, int64_t os0, int64_t os1, cudaStream_t st,
@@ -124,8 +134,18 @@ struct WsGemm {
   View2 pre_ids;
   int32_t pre_E, pre_S;
   DeviceErrors* err;
+  // mode 1: every routed slot gets weight 1 instead of its routing weight
+  int32_t unit_w;
+  // mode 3 (gradient of GEMM1 + SwiGLU): dh [P, N] in, h [P, N] out (row strides in elements)
+  const void* dh;
+  int64_t dh_ld;
+  void* h_out;
+  int64_t h_ld;
 };
-// mode 0: GEMM1 (gate/up + SwiGLU -> h), mode 1: GEMM2 (down + routing weight -> y)
+// mode 0: GEMM1 (gate/up + SwiGLU -> h), mode 1: GEMM2 (down + routing weight -> y),
+// mode 3: GEMM1 recomputed for the gradient: with g, u the two accumulators and dh
+// read from p.dh, out[p, i] = dh s u (1 + g (1 - s)), out[p, N + i] = dh g s
+// (s = sigmoid(g)) and h_out[p, i] = g s u, for every row of the token tiles.
 // tile_max: 128 (4-stage ring) or 32 (6-stage ring)
 cudaError_t launch_gemm_ws_bf16(int mode, int tile_max, const CUtensorMap& w0,
                                 const CUtensorMap& w1, const CUtensorMap& x, const WsGemm& p,

@@ -1,0 +1,123 @@
+"""GPU parity of the gradient path (moe_backward_input_ws, moe_transpose_experts)
+against the fp64 oracle gradient (oracle.moe_backward_input).
+
+Tolerance: the CUDA path rounds to bf16 where the oracle keeps fp64: dh, dg and du,
+the recomputed h, the per-slot expert output y (for the routing-weight gradient)
+and the per-slot da rows (for dx), then dx itself.  Each rounding is at most
+2^-9 relative per element and the sums after it run in fp32, so the error
+relative to the largest element stays a few times 2^-9 (~0.2 %) per step; 2e-2
+relative to the largest |dx| (|dweights|) leaves room for four such steps and the
+fp32 accumulation order, while a wrong term, sign or index (the oracle pins'
+failure modes) moves results by O(1).
+"""
+
+import pytest
+import torch
+
+import mixture_experts_layer_46_b200 as moe
+from mixture_experts_layer_46_b200 import workloads as wl
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+BWD_TOL = 2e-2
+
+
+def rel_err(got, ref):
+    got, ref = got.double().cpu(), ref.double().cpu()
+    return (got - ref).abs().max().item() / ref.abs().max().item()
+
+
+def make_case(T, H, I, E, k, seed):
+    x = wl.make_x(T, H, seed=seed + 1)
+    w13, w2 = wl.make_weights_bf16(E, I, H, seed=seed)
+    ids, wts = wl.route_softmax_topk(T, E, k, seed=seed + 2)
+    dout = wl.make_x(T, H, seed=seed + 3)
+    return {"x": x, "w13": w13, "w2": w2, "ids": ids, "wts": wts, "dout": dout}
+
+
+def gpu_backward(c, dout=None, dx=None, dw=None):
+    w13, w2 = c["w13"], c["w2"]
+    gate, up = wl.gate_up_views(w13)
+    v = moe.w13_from_packed(w13)
+    w13t = moe.transpose_experts(w13)
+    w2t = moe.transpose_experts(w2)
+    dxo, dwo = moe.backward_input(c["x"], v, w2, w13t, w2t, c["ids"], c["wts"],
+                                  c["dout"] if dout is None else dout, dx, dw)
+    torch.cuda.synchronize()
+    return dxo, dwo
+
+
+def oracle_backward(c, tokens=None):
+    gate, up = wl.gate_up_views(c["w13"])
+    return oracle.moe_backward_input(c["x"], gate, up, c["w2"], c["ids"], c["wts"], c["dout"],
+                                     tokens=tokens)
+
+
+def test_transpose_experts_is_exact_for_strided_views():
+    w13, _ = wl.make_weights_bf16(3, 96, 160, seed=4, device="cuda")
+    got = moe.transpose_experts(w13)
+    assert torch.equal(got, w13.transpose(1, 2))
+    gate, _ = wl.gate_up_views(w13)  # a strided view: rows [0, I) of each expert
+    got = moe.transpose_experts(gate)
+    assert torch.equal(got, gate.transpose(1, 2))
+
+
+@pytest.mark.parametrize("T,H,I,E,k", [
+    (64, 256, 256, 8, 2),
+    (200, 512, 384, 16, 4),    # several 128-row token tiles, N tail of I in the dh GEMM
+    (1, 256, 256, 4, 2),
+    (77, 288, 96, 6, 3),       # ragged K (H = 4.5 k-blocks) and output columns
+])
+def test_backward_matches_oracle(T, H, I, E, k):
+    case = make_case(T, H, I, E, k, seed=T + 17)
+    ref_dx, ref_dw = oracle_backward(case)
+    c = {n: v.cuda() for n, v in case.items()}
+    dx, dw = gpu_backward(c)
+    assert rel_err(dx, ref_dx) <= BWD_TOL
+    assert rel_err(dw, ref_dw) <= BWD_TOL
+
+
+def test_backward_is_deterministic_and_reads_strided_views():
+    case = make_case(150, 512, 256, 8, 4, seed=29)
+    c = {n: v.cuda() for n, v in case.items()}
+    a = gpu_backward(c)
+    b = gpu_backward(c)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    # dout and both outputs as strided views of wider buffers
+    wide = torch.zeros(150, 2 * 512, dtype=torch.bfloat16, device="cuda")
+    wide[:, ::2] = c["dout"]
+    dxw = torch.zeros(150, 3 * 512, dtype=torch.bfloat16, device="cuda")
+    dww = torch.zeros(150, 3 * 4, dtype=torch.float32, device="cuda")
+    s = gpu_backward(c, dout=wide[:, ::2], dx=dxw[:, ::3], dw=dww[:, ::3])
+    assert torch.equal(s[0], a[0]) and torch.equal(s[1], a[1])
+
+
+def test_skipped_ids_get_zero_weight_gradient():
+    case = make_case(40, 256, 256, 8, 2, seed=3)
+    case["ids"][5, 1] = 99
+    case["ids"][7, 0] = -1
+    ref_dx, ref_dw = oracle_backward(case)
+    c = {n: v.cuda() for n, v in case.items()}
+    dx, dw = gpu_backward(c)
+    assert dw[5, 1].item() == 0.0 and dw[7, 0].item() == 0.0
+    assert rel_err(dx, ref_dx) <= BWD_TOL
+    assert rel_err(dw, ref_dw) <= BWD_TOL
+
+
+@pytest.mark.slow
+def test_qwen3_235b_shape_sampled_tokens(qwen3_weights):
+    s = wl.QWEN3_235B
+    T = 512
+    x = wl.make_x(T, s.H, seed=71)
+    ids, wts = wl.route_softmax_topk(T, s.E, s.k, seed=72)
+    dout = wl.make_x(T, s.H, seed=73)
+    c = {"x": x.cuda(), "w13": qwen3_weights["w13"], "w2": qwen3_weights["w2"], "ids": ids.cuda(),
+         "wts": wts.cuda(), "dout": dout.cuda()}
+    dx, dw = gpu_backward(c)
+    toks = torch.tensor([0, 1, 255, 510, 511])
+    host = {"x": x, "w13": qwen3_weights["w13_cpu"], "w2": qwen3_weights["w2_cpu"], "ids": ids,
+            "wts": wts, "dout": dout}
+    ref_dx, ref_dw = oracle_backward(host, tokens=toks)
+    assert rel_err(dx.cpu()[toks], ref_dx) <= BWD_TOL
+    assert rel_err(dw.cpu()[toks], ref_dw) <= BWD_TOL
