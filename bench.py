@@ -352,6 +352,9 @@ def main():
     ap.add_argument("--E", type=int, default=None, help="override the expert count (profiling)")
     ap.add_argument("--sweep", default=None, help="write a token-sweep JSONL here (extra lines)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--grad", action="store_true",
+                    help="time the gradient path (dx and the routing-weight gradient, experts frozen) "
+                         "instead of the forward; prints its own JSON line")
     ap.add_argument("--config", default=None,
                     help="override configuration flags of the timed forward, e.g. fused=1,tile=32 "
                          "(installed with moe_set_config_table for this problem only)")
@@ -395,6 +398,12 @@ def main():
     def step():
         moe.forward(inp["x"], v13, inp["w2"], inp["ids"], inp["wts"], out=out, workspace=ws,
                     stream=stream, w2_scale=s2)
+
+    if args.grad:
+        if mx:
+            raise SystemExit("--grad: the gradient path takes bf16 weights")
+        run_grad(args, w, moe, wl, inp, v13, dev, stream, flush)
+        return
 
     if args.config:
         flags = {kv.split("=")[0]: int(kv.split("=")[1]) for kv in args.config.split(",")}
@@ -527,6 +536,60 @@ def main():
     if pg:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
+
+
+def run_grad(args, w, moe, wl, inp, v13, dev, stream, flush):
+    """The gradient path (moe_backward_input_ws) on the forward's workload, timed like
+    the forward: L2 flushed clean before every step, CUDA events, clocks sampled.
+    Roofline: 12 H I FLOPs per slot (twice the forward: dh, the gate/up recompute, the
+    unweighted down projection and da) against the slower of the bf16 burst peak and
+    the HBM time of the activated experts' weights read twice (w2^T, gate/up, w2,
+    w13^T) plus x, dout and dx."""
+    hbm, tf_burst, _, _ = peaks()
+    T, H = w["T"], w["H"]
+    w13t = moe.transpose_experts(inp["w13"])
+    w2t = moe.transpose_experts(inp["w2"])
+    dout = wl.make_x(T, H, seed=3, device=dev)
+    dx = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    dwt = torch.empty(T, w["k"], dtype=torch.float32, device=dev)
+    gws = torch.empty(moe.backward_workspace_bytes(T, H, w["I"], w["E"], w["k"]), dtype=torch.uint8,
+                      device=dev)
+
+    def gstep():
+        moe.backward_input(inp["x"], v13, inp["w2"], w13t, w2t, inp["ids"], inp["wts"], dout, dx, dwt,
+                           workspace=gws, stream=stream)
+
+    for _ in range(args.warmup):
+        gstep()
+    launches = moe.last_launch_count()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for i in range(args.steps):
+        wl.flush_l2(flush, i)
+        evs[i][0].record(stream)
+        gstep()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    per = sorted(a.elapsed_time(b) for a, b in evs)
+    ms = sum(per) / len(per)
+    alg = algorithmic(w, inp["ids"])
+    flops = 2.0 * alg["flops"]
+    gbytes = 2.0 * 3.0 * w["I"] * H * 2.0 * alg["active_experts"] + 3.0 * T * H * 2
+    t_roof = max(flops / (tf_burst * 1e12), gbytes / (hbm * 1e9))
+    print(json.dumps({
+        "metric": "fused-MoE layer gradient (dx, routing weights; experts frozen) tokens/s on 1 B200",
+        "value": T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": args.steps,
+        "warmup": args.warmup, "higher_is_better": True, "dtype": "bf16",
+        "config": {"workload": workload_name(w) + " gradient", "tokens_per_gpu": T,
+                   "us_per_call_p10": per[len(per) // 10] * 1e3,
+                   "us_per_call_p90": per[(9 * len(per)) // 10] * 1e3},
+        "roofline": {"t_roof_us": t_roof * 1e6, "frac": t_roof / (ms * 1e-3), "flops": flops,
+                     "bytes": gbytes, "bound": "tensor" if flops / (tf_burst * 1e12) > gbytes / (hbm * 1e9) else "hbm"},
+        "gpu_launches": launches * args.steps, "clocks": clocks}), flush=True)
 
 
 def sweep(args, w, moe, wl, dev, stream, flush):
