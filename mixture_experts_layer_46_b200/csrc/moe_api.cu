@@ -982,6 +982,16 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   tiles.list[0].tile_rows = reinterpret_cast<int32_t*>(w + L.tile_rows);
   tiles.list[0].tile_expert = reinterpret_cast<int32_t*>(w + L.tile_expert);
   tiles.list[0].num_tiles = num_blocks + 1;
+  // the down-projection-form GEMMs (dh, y, da) on CTA pairs with one 256-row weight slice
+  // per 256-row token tile wherever the forward's table picks that form for GEMM2
+  const bool pair2 = select_config(pr.T, pr.H, pr.I, pr.E, pr.k, false).g2_single != 0;
+  if (pair2) {
+    tiles.list[1].tile_max = 256;
+    tiles.list[1].tile_row = reinterpret_cast<int32_t*>(w + L.tile_row2);
+    tiles.list[1].tile_rows = reinterpret_cast<int32_t*>(w + L.tile_rows2);
+    tiles.list[1].tile_expert = reinterpret_cast<int32_t*>(w + L.tile_expert2);
+    tiles.list[1].num_tiles = num_blocks + 2;
+  }
   cudaError_t rc = launch_align(view2(ids), pr.T, pr.k, pr.E, bm, counts, offsets, sorted, inv,
                                 block_expert, num_blocks, chunk_counts, L.n_chunks, dev->errors, st,
                                 &launches, &tiles);
@@ -1006,14 +1016,26 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   gb.err = dev->errors;
   gb.tok_box = kTile;
   gb.topk_w = view2(wts);
+  WsGemm gp = gb;  // the same on align's 256-row tiles (CTA pairs: 128 token rows per CTA)
+  if (pair2) {
+    gp.max_tiles = L.t_max2;
+    gp.num_tiles = tiles.list[1].num_tiles;
+    gp.tile_row = tiles.list[1].tile_row;
+    gp.tile_rows = tiles.list[1].tile_rows;
+    gp.tile_expert = tiles.list[1].tile_expert;
+  }
+  auto down_form = [&](const WsGemm& p, const CUtensorMap& wm, const CUtensorMap& xm) {
+    return pair2 ? launch_gemm_ws_pair_bf16(2, 256, wm, wm, xm, p, dev->num_sms, st, &launches)
+                 : launch_gemm_ws_bf16(1, kTile, wm, wm, xm, p, dev->num_sms, st, &launches);
+  };
 
-  WsGemm g = gb;  // dh = w * w2^T dout
+  WsGemm g = gp;  // dh = w * w2^T dout
   g.K = pr.H;
   g.N = pr.I;
   g.n_wt = (pr.I + 255) / 256;
   g.out = w + B.dh;
   g.out_ld = pr.I;
-  rc = launch_gemm_ws_bf16(1, kTile, mW2T, mW2T, mD1, g, dev->num_sms, st, &launches);
+  rc = down_form(g, mW2T, mD1);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm dh");
 
   g = gb;  // g, u recomputed: [dg | du] and h
@@ -1029,27 +1051,27 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   rc = launch_gemm_ws_bf16(3, kTile, mGate, mUp, mA1, g, dev->num_sms, st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm dg du");
 
-  g = gb;  // y = w2 h, unweighted
+  g = gp;  // y = w2 h, unweighted
   g.K = pr.I;
   g.N = pr.H;
   g.n_wt = (pr.H + 255) / 256;
   g.out = w + L.y;
   g.out_ld = pr.H;
   g.unit_w = 1;
-  rc = launch_gemm_ws_bf16(1, kTile, mW2, mW2, mHh, g, dev->num_sms, st, &launches);
+  rc = down_form(g, mW2, mHh);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm y");
   rc = launch_slot_dot(view2(dout), reinterpret_cast<const __nv_bfloat16*>(w + L.y), inv, pr.T, pr.H,
                        pr.k, view2(dw), st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "slot_dot");
 
-  g = gb;  // da = [gate^T | up^T] [dg | du]
+  g = gp;  // da = [gate^T | up^T] [dg | du]
   g.K = 2 * pr.I;
   g.N = pr.H;
   g.n_wt = (pr.H + 255) / 256;
   g.out = w + L.y;
   g.out_ld = pr.H;
   g.unit_w = 1;
-  rc = launch_gemm_ws_bf16(1, kTile, mW13T, mW13T, mDGU, g, dev->num_sms, st, &launches);
+  rc = down_form(g, mW13T, mDGU);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm da");
   rc = launch_combine(reinterpret_cast<const __nv_bfloat16*>(w + L.y), inv, pr.T, pr.H, pr.k,
                       dx->data, dx->strides[0], dx->strides[1], st, &launches);

@@ -74,6 +74,7 @@ struct Args {
   int64_t k;
   int32_t weights_evict_first;
   int32_t tok_box;  // token rows per TMA box (the map's box height)
+  int32_t unit_w;   // modes 1/2: weight 1 for every routed slot
   DeviceErrors* err;
 };
 
@@ -239,7 +240,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           w_r[i] = 0.0f;
           if (slot_r[i] < g.S) {
             const int64_t tt = slot_r[i] / g.k, jj = slot_r[i] - tt * g.k;
-            w_r[i] = static_cast<const float*>(g.topk_w.data)[tt * g.topk_w.s0 + jj * g.topk_w.s1];
+            w_r[i] = g.unit_w ? 1.0f
+                              : static_cast<const float*>(g.topk_w.data)[tt * g.topk_w.s0 + jj * g.topk_w.s1];
           }
         }
       }
@@ -366,6 +368,7 @@ cudaError_t launch_gemm_ws_pair_bf16(int mode, int tile_max, const CUtensorMap& 
   g.err = p.err;
   g.weights_evict_first = p.weights_evict_first;
   g.tok_box = p.tok_box;
+  g.unit_w = p.unit_w;
   if (launches) *launches += 1;
   const int64_t max_items = p.max_tiles * p.n_wt;
   if (tile_max == 256) {

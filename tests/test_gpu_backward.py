@@ -78,6 +78,26 @@ def test_backward_matches_oracle(T, H, I, E, k):
     assert rel_err(dw, ref_dw) <= BWD_TOL
 
 
+@pytest.mark.parametrize("T,H,I,E,k", [
+    (600, 512, 384, 3, 2),     # 400 slots per expert: two 256-row tiles, N tail of I (dh)
+    (300, 288, 96, 2, 2),      # ragged K and output columns on CTA pairs
+])
+def test_backward_pair_route_matches_one_cta_route(T, H, I, E, k):
+    # dh, y and da run on CTA pairs (one 256-row weight slice per 256-row token tile)
+    # where the configuration picks that GEMM2 form, on one CTA otherwise: same bits
+    case = make_case(T, H, I, E, k, seed=T + 41)
+    ref_dx, ref_dw = oracle_backward(case)
+    c = {n: v.cuda() for n, v in case.items()}
+    with moe.config_override((T, H, I, E, k), tile=128, pair=0, g2_single=0):
+        one = gpu_backward(c)
+    with moe.config_override((T, H, I, E, k), tile=128, pair=1, g2_single=1):
+        assert moe.get_config(T, H, I, E, k)["g2_single"] == 1
+        pair = gpu_backward(c)
+    assert torch.equal(one[0], pair[0]) and torch.equal(one[1], pair[1])
+    assert rel_err(pair[0], ref_dx) <= BWD_TOL
+    assert rel_err(pair[1], ref_dw) <= BWD_TOL
+
+
 def test_backward_is_deterministic_and_reads_strided_views():
     case = make_case(150, 512, 256, 8, 4, seed=29)
     c = {n: v.cuda() for n, v in case.items()}
