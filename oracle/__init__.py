@@ -82,6 +82,8 @@ def _load():
             lib.oracle_moe_backward_input.restype = ctypes.c_int
             lib.oracle_moe_backward_input.argtypes = [P(OracleTensor)] * 7 + [
                 ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+            lib.oracle_moe_backward_weights.restype = ctypes.c_int
+            lib.oracle_moe_backward_weights.argtypes = [P(OracleTensor)] * 7 + [ctypes.c_void_p] * 3
             lib.oracle_router_topk.restype = ctypes.c_int
             lib.oracle_router_topk.argtypes = [P(OracleTensor), ctypes.c_int64, ctypes.c_int,
                                                ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
@@ -146,6 +148,21 @@ def moe_backward_input(x, gate, up, w2, ids, weights, dout, *, tokens=None, nthr
     if rc != 0:
         raise ValueError("oracle_moe_backward_input: shape mismatch")
     return dx, dw
+
+
+def moe_backward_weights(x, gate, up, w2, ids, weights, dout):
+    """fp64 gradient of the bf16 forward with respect to the expert weights given
+    dout [T, H]: (dgate [E, I, H], dup [E, I, H], dw2 [E, H, I]) float64."""
+    d = [_desc(v) for v in (x, gate, up, w2, ids, weights, dout)]
+    E, I, H = gate.shape
+    dg = torch.zeros(E, I, H, dtype=torch.float64)
+    du = torch.zeros(E, I, H, dtype=torch.float64)
+    dw2 = torch.zeros(E, H, I, dtype=torch.float64)
+    rc = _load().oracle_moe_backward_weights(*[ctypes.byref(v) for v in d], dg.data_ptr(),
+                                             du.data_ptr(), dw2.data_ptr())
+    if rc != 0:
+        raise ValueError("oracle_moe_backward_weights: shape mismatch")
+    return dg, du, dw2
 
 
 def router_topk(logits: torch.Tensor, k: int, renormalize: bool = True, shared_expert: bool = False):

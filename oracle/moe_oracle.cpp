@@ -371,6 +371,71 @@ int oracle_moe_backward_input(const oracle_tensor_t* x, const oracle_tensor_t* g
   return 0;
 }
 
+// Gradient of the forward with respect to the expert weights, given dout, the
+// routing fixed: for every token t and column j with e = topk_ids[t, j] in
+// [0, E) and w = topk_weights[t, j], with g, u, a = silu(g) u, s, dg, du as in
+// oracle_moe_backward_input:
+//   dw2[e, o, i]   += w * dout[t, o] * a_i
+//   dgate[e, i, h] += dg_i * x[t, h]
+//   dup[e, i, h]   += du_i * x[t, h]
+// (tokens in ascending order, columns in order).  bf16 weights only.
+//   dgate, dup [E, I, H] and dw2 [E, H, I] fp64, contiguous, overwritten.
+int oracle_moe_backward_weights(const oracle_tensor_t* x, const oracle_tensor_t* gate,
+                                const oracle_tensor_t* up, const oracle_tensor_t* w2,
+                                const oracle_tensor_t* ids, const oracle_tensor_t* weights,
+                                const oracle_tensor_t* dout, double* dgate, double* dup,
+                                double* dw2) {
+  const int64_t T = x->sizes[0], H = x->sizes[1];
+  const int64_t E = gate->sizes[0], I = gate->sizes[1];
+  const int64_t k = ids->sizes[1];
+  if (gate->sizes[2] != H || up->sizes[0] != E || up->sizes[1] != I || up->sizes[2] != H ||
+      w2->sizes[0] != E || w2->sizes[1] != H || w2->sizes[2] != I || ids->sizes[0] != T ||
+      weights->sizes[0] != T || weights->sizes[1] != k || dout->sizes[0] != T ||
+      dout->sizes[1] != H || gate->dtype == OR_E2M1X2)
+    return 1;
+  std::fill(dgate, dgate + E * I * H, 0.0);
+  std::fill(dup, dup + E * I * H, 0.0);
+  std::fill(dw2, dw2 + E * H * I, 0.0);
+  std::vector<double> xt(H), dot(H), g(I), u(I), a(I), dg(I), du(I);
+  for (int64_t t = 0; t < T; ++t) {
+    for (int64_t h = 0; h < H; ++h) {
+      xt[h] = read_real2(x, t, h);
+      dot[h] = read_real2(dout, t, h);
+    }
+    for (int64_t j = 0; j < k; ++j) {
+      const int64_t e = read_id(ids, t, j);
+      if (e < 0 || e >= E) continue;
+      const double w = read_real2(weights, t, j);
+      for (int64_t i = 0; i < I; ++i) {
+        double gg = 0.0, uu = 0.0;
+        for (int64_t h = 0; h < H; ++h) {
+          gg += xt[h] * read_weight(gate, e, i, h);
+          uu += xt[h] * read_weight(up, e, i, h);
+        }
+        g[i] = gg;
+        u[i] = uu;
+        a[i] = gg / (1.0 + std::exp(-gg)) * uu;
+      }
+      for (int64_t o = 0; o < H; ++o)
+        for (int64_t i = 0; i < I; ++i) dw2[(e * H + o) * I + i] += w * dot[o] * a[i];
+      for (int64_t i = 0; i < I; ++i) {
+        double da = 0.0;
+        for (int64_t o = 0; o < H; ++o) da += dot[o] * read_weight(w2, e, o, i);
+        da *= w;
+        const double sg = 1.0 / (1.0 + std::exp(-g[i]));
+        dg[i] = da * u[i] * sg * (1.0 + g[i] * (1.0 - sg));
+        du[i] = da * g[i] * sg;
+      }
+      for (int64_t i = 0; i < I; ++i)
+        for (int64_t h = 0; h < H; ++h) {
+          dgate[(e * I + i) * H + h] += dg[i] * xt[h];
+          dup[(e * I + i) * H + h] += du[i] * xt[h];
+        }
+    }
+  }
+  return 0;
+}
+
 // The router that produces the forward's routing inputs, in fp64:
 //   p = softmax(logits[t, :]) over the E experts,
 //   the k experts of largest p, in descending p (a tie goes to the lower expert index),

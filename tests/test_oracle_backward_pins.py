@@ -1,4 +1,5 @@
-"""Pins for the oracle's input and routing-weight gradient (experts frozen).
+"""Pins for the oracle's gradients: with respect to the inputs and routing weights
+(experts frozen) and with respect to the expert weights.
 
 * central finite differences of the oracle forward (itself pinned by
   tests/test_oracle_pins.py): L = sum_t,o out[t, o] * dout[t, o], each element of x
@@ -105,3 +106,50 @@ def test_token_subset_rows_match_full_run():
     toks = torch.tensor([4, 1])
     part = oracle.moe_backward_input(x, gate, up, w2, ids, wts, dout, tokens=toks)
     assert torch.equal(part[0], full[0][toks]) and torch.equal(part[1], full[1][toks])
+
+
+def test_weight_gradient_matches_central_finite_differences():
+    x, gate, up, w2, ids, wts, dout = _case(T=3, H=8, I=4, E=2, k=2, seed=12)
+    dg, du, dw2 = oracle.moe_backward_weights(x, gate, up, w2, ids, wts, dout)
+    d = 1e-3
+    for name, tensor, grad in (("gate", gate, dg), ("up", up, du), ("w2", w2, dw2)):
+        num = torch.zeros_like(grad)
+        for idx in range(tensor.numel()):
+            p, m = tensor.clone(), tensor.clone()
+            p.view(-1)[idx] += d
+            m.view(-1)[idx] -= d
+            step = float(p.view(-1)[idx].double() - m.view(-1)[idx].double())
+            args = dict(gate=gate, up=up, w2=w2)
+            lp = _loss(x, **{**args, name: p}, ids=ids, wts=wts, dout=dout)
+            lm = _loss(x, **{**args, name: m}, ids=ids, wts=wts, dout=dout)
+            num.view(-1)[idx] = (lp - lm) / step
+        assert (grad - num).abs().max() <= 1e-5 * grad.abs().max(), name
+
+
+def test_weight_gradient_matches_autograd_of_dense_formulation():
+    x, gate, up, w2, ids, wts, dout = _case(T=5, H=24, I=12, E=4, k=3, seed=19)
+    g_ = gate.double().requires_grad_(True)
+    u_ = up.double().requires_grad_(True)
+    d_ = w2.double().requires_grad_(True)
+    xd = x.double()
+    E = gate.shape[0]
+    R = torch.zeros(x.shape[0], E, dtype=torch.float64).index_put(
+        (torch.arange(x.shape[0]).repeat_interleave(ids.shape[1]), ids.long().reshape(-1)),
+        wts.double().reshape(-1), accumulate=True)
+    out = torch.zeros(x.shape[0], x.shape[1], dtype=torch.float64)
+    for e in range(E):
+        hmid = torch.nn.functional.silu(xd @ g_[e].T) * (xd @ u_[e].T)
+        out = out + R[:, e:e + 1] * (hmid @ d_[e].T)
+    out.backward(dout.double())
+    dg, du, dw2 = oracle.moe_backward_weights(x, gate, up, w2, ids, wts, dout)
+    assert torch.allclose(dg, g_.grad, rtol=1e-10, atol=1e-12)
+    assert torch.allclose(du, u_.grad, rtol=1e-10, atol=1e-12)
+    assert torch.allclose(dw2, d_.grad, rtol=1e-10, atol=1e-12)
+
+
+def test_unrouted_expert_gets_zero_weight_gradient():
+    x, gate, up, w2, ids, wts, dout = _case(T=4, H=16, I=8, E=4, k=1, seed=2)
+    ids = torch.zeros_like(ids)  # every token on expert 0
+    dg, du, dw2 = oracle.moe_backward_weights(x, gate, up, w2, ids, wts, dout)
+    assert dg[1:].abs().max() == 0 and du[1:].abs().max() == 0 and dw2[1:].abs().max() == 0
+    assert dg[0].abs().max() > 0
