@@ -155,12 +155,13 @@ moe_status_t moe_forward_host(const moe_tensor_t* x_host, const moe_w13_t* w13,
                               const moe_tensor_t* topk_weights_host, moe_tensor_t* out_host,
                               moe_stream_t stream);
 
-/* Gradient path with the experts frozen (bf16 weights): given dout = dL/dout
+/* Gradient path (bf16 weights): given dout = dL/dout
  * [T, H] bf16, writes dx = dL/dx [T, H] bf16 and dweights = dL/dtopk_weights
  * [T, k] f32 (any strides), the routing ids held fixed (they are discrete).
  * The fused-MoE training path of Liger-Kernel PR #1377 ("Testing Done":
  * forward and backward CUDA graphs) differentiates this layer; this entry point
- * covers its input and routing-weight gradients, not the expert weights'.
+ * gives its input and routing-weight gradients (moe_backward_ws adds the expert
+ * weights').
  * Per slot (t, j) with e = topk_ids[t, j] in [0, E), w = topk_weights[t, j]:
  *   dweights[t, j] = dout_t . (w2_e h),  h = silu(gate_e x_t) * (up_e x_t)
  *   dh = w w2_e^T dout_t;  dg = dh u s (1 + g (1 - s)),  du = dh g s  (s = sigmoid(g))
@@ -175,6 +176,21 @@ moe_status_t moe_forward_host(const moe_tensor_t* x_host, const moe_w13_t* w13,
  * aligned.  Asynchronous on `stream`, no allocation.  MXFP4 weights:
  * MOE_ERR_UNSUPPORTED_DTYPE (the forward's quantisation steps have no gradient). */
 size_t moe_backward_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k);
+
+/* The same plus the expert-weight gradients (either may be NULL): dw13 = dL/dw13
+ * f32 [E, 2I, H] packed like w13 (dgate rows [0, I), dup rows [I, 2I)) and dw2 =
+ * dL/dw2 f32 [E, H, I], overwritten (zero for an expert no slot routes to), inner
+ * stride 1 and the other strides multiples of 4 elements, 16-byte aligned; H and I
+ * multiples of 32.  With the routing fixed:
+ *   dw2[e]   = sum over e's slots (t, j) of w (dout_t) a^T,   a = silu(g) * u
+ *   dgate[e] = sum of dg x_t^T,  dup[e] = sum of du x_t^T
+ * each a GEMM that contracts over the expert's slots (fp32 accumulation). */
+moe_status_t moe_backward_ws(const moe_tensor_t* x, const moe_w13_t* w13, const moe_tensor_t* w2,
+                             const moe_tensor_t* w13t, const moe_tensor_t* w2t,
+                             const moe_tensor_t* topk_ids, const moe_tensor_t* topk_weights,
+                             const moe_tensor_t* dout, moe_tensor_t* dx, moe_tensor_t* dweights,
+                             moe_tensor_t* dw13, moe_tensor_t* dw2, void* workspace, size_t workspace_bytes,
+                             moe_stream_t stream);
 moe_status_t moe_backward_input_ws(const moe_tensor_t* x, const moe_w13_t* w13, const moe_tensor_t* w2,
                                    const moe_tensor_t* w13t, const moe_tensor_t* w2t,
                                    const moe_tensor_t* topk_ids, const moe_tensor_t* topk_weights,

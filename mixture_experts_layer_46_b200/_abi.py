@@ -31,7 +31,7 @@ EXPORTS = ("moe_status_string", "moe_last_cuda_error", "moe_w13_from_packed",
            "moe_set_config_table", "moe_get_config", "moe_builtin_config_count",
            "moe_router_topk", "moe_selftest_bounded_wait", "moe_workspace_layout",
            "moe_debug_capture", "moe_measure_mma_peak", "moe_backward_workspace_bytes",
-           "moe_backward_input_ws", "moe_transpose_experts")
+           "moe_backward_input_ws", "moe_backward_ws", "moe_transpose_experts")
 STEP_NAMES = ("align", "permute", "gemm1_swiglu", "gemm2_weighted", "combine")
 
 
@@ -117,6 +117,9 @@ def load() -> ctypes.CDLL:
             lib.moe_backward_workspace_bytes.argtypes = [ctypes.c_int64] * 5
             lib.moe_backward_input_ws.restype = ctypes.c_int
             lib.moe_backward_input_ws.argtypes = [P(MoeTensor), P(MoeW13)] + [P(MoeTensor)] * 8 + [
+                vp, ctypes.c_size_t, vp]
+            lib.moe_backward_ws.restype = ctypes.c_int
+            lib.moe_backward_ws.argtypes = [P(MoeTensor), P(MoeW13)] + [P(MoeTensor)] * 10 + [
                 vp, ctypes.c_size_t, vp]
             lib.moe_transpose_experts.restype = ctypes.c_int
             lib.moe_transpose_experts.argtypes = [P(MoeTensor), P(MoeTensor), vp]
@@ -256,6 +259,34 @@ def transpose_experts(src: torch.Tensor, dst: torch.Tensor | None = None, *, str
     _check(load().moe_transpose_experts(ctypes.byref(ds), ctypes.byref(dd), _stream_ptr(stream)),
            "moe_transpose_experts")
     return dst
+
+
+def backward(x, w13: MoeW13, w2, w13t, w2t, topk_ids, topk_weights, dout, dx=None, dweights=None,
+             dw13=None, dw2=None, *, weights=True, workspace: torch.Tensor | None = None, stream=None):
+    """(dx, dweights, dw13, dw2): the forward's gradients given dout; dw13 f32 [E, 2I, H]
+    (packed like w13) and dw2 f32 [E, H, I] are computed when `weights` (else None)."""
+    T, H = x.shape
+    k = topk_ids.shape[1]
+    E, _, I = w2.shape
+    dev = x.device
+    if dx is None:
+        dx = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    if dweights is None:
+        dweights = torch.empty(T, k, dtype=torch.float32, device=dev)
+    if weights and dw13 is None:
+        dw13 = torch.empty(E, 2 * I, H, dtype=torch.float32, device=dev)
+    if weights and dw2 is None:
+        dw2 = torch.empty(E, H, I, dtype=torch.float32, device=dev)
+    if workspace is None:
+        n = backward_workspace_bytes(T, H, I, E, k)
+        workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=dev)
+    d = [desc(v) for v in (x, w2, w13t, w2t, topk_ids, topk_weights, dout, dx, dweights)]
+    g13 = ctypes.byref(desc(dw13)) if dw13 is not None else None
+    g2 = ctypes.byref(desc(dw2)) if dw2 is not None else None
+    rc = load().moe_backward_ws(ctypes.byref(d[0]), ctypes.byref(w13), *[ctypes.byref(v) for v in d[1:]],
+                                g13, g2, workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    _check(rc, "moe_backward_ws")
+    return dx, dweights, dw13, dw2
 
 
 def backward_input(x, w13: MoeW13, w2, w13t, w2t, topk_ids, topk_weights, dout, dx=None, dweights=None,

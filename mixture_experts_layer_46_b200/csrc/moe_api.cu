@@ -888,21 +888,35 @@ moe_status_t forward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe
 
 // The forward's workspace plus the gradient's own rows: dout gathered into
 // expert-grouped order, dh = dL/dh and [dg | du], each [P_max, .] bf16.
+// The weight-gradient GEMMs contract over each expert's grouped rows in 64-row
+// k-blocks, so the gradient path groups slots in 64-row granules.
+constexpr int32_t kBwdBm = 64;
+
 struct BwdLayout {
   WsLayout L;
-  size_t d1, dh, dgu, total;
+  size_t d1, dh, dgu, dyT, hT, dguT, a1T, total;
 };
 
+// The forward's workspace plus the gradient's own rows: dout gathered into
+// expert-grouped order, dh and [dg | du] ([P, .] bf16), and the four transposed
+// grouped matrices of the weight gradients ([., P] bf16).
 BwdLayout make_bwd_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k) {
   BwdLayout B;
-  B.L = make_layout(T, H, I, E, k, false, kBm);
+  B.L = make_layout(T, H, I, E, k, false, kBwdBm);
+  const size_t P = size_t(B.L.p_max);
   size_t off = align256(B.L.total);
-  B.d1 = off;
-  off = align256(off + size_t(B.L.p_max) * H * 2);
-  B.dh = off;
-  off = align256(off + size_t(B.L.p_max) * I * 2);
-  B.dgu = off;
-  off = align256(off + size_t(B.L.p_max) * 2 * I * 2);
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  B.d1 = take(P * H * 2);
+  B.dh = take(P * I * 2);
+  B.dgu = take(P * 2 * I * 2);
+  B.dyT = take(P * H * 2);
+  B.hT = take(P * I * 2);
+  B.dguT = take(P * 2 * I * 2);
+  B.a1T = take(P * H * 2);
   B.total = off;
   return B;
 }
@@ -927,11 +941,17 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
                            const moe_tensor_t* w13t, const moe_tensor_t* w2t,
                            const moe_tensor_t* ids, const moe_tensor_t* wts,
                            const moe_tensor_t* dout, moe_tensor_t* dx, moe_tensor_t* dw,
-                           const Problem& pr, void* ws, size_t ws_bytes, cudaStream_t st) {
+                           moe_tensor_t* dw13, moe_tensor_t* dw2, const Problem& pr, void* ws,
+                           size_t ws_bytes, cudaStream_t st) {
   int launches = 0;
   t_last_launches = 0;
-  if (pr.T == 0) return MOE_OK;
-  const int32_t bm = kBm;
+  if (pr.T == 0) {
+    // no tokens: the weight gradients are zero
+    if (dw13) MOE_CUDA(cudaMemsetAsync(dw13->data, 0, size_t(pr.E) * dw13->strides[0] * 4, st));
+    if (dw2) MOE_CUDA(cudaMemsetAsync(dw2->data, 0, size_t(pr.E) * dw2->strides[0] * 4, st));
+    return MOE_OK;
+  }
+  const int32_t bm = kBwdBm;
   const BwdLayout B = make_bwd_layout(pr.T, pr.H, pr.I, pr.E, pr.k);
   const WsLayout& L = B.L;
   if (!ws || ws_bytes < B.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
@@ -1076,6 +1096,55 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   rc = launch_combine(reinterpret_cast<const __nv_bfloat16*>(w + L.y), inv, pr.T, pr.H, pr.k,
                       dx->data, dx->strides[0], dx->strides[1], st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "combine dx");
+
+  if (dw13 || dw2) {
+    // expert-weight gradients: the grouped rows transposed (padding rows zero), then
+    // GEMMs contracting over each expert's rows
+    const int64_t P = L.p_max;
+    View2 none;
+    std::memset(&none, 0, sizeof(none));
+    View2 dgu_rows;
+    dgu_rows.data = w + B.dgu;
+    dgu_rows.s0 = 2 * pr.I;
+    dgu_rows.s1 = 1;
+    dgu_rows.dtype = MOE_BF16;
+    CUtensorMap mA, mB;
+    const uint32_t box[2] = {64, 128};
+    auto tmap = [&](CUtensorMap* m, uint8_t* base, int64_t rows) {
+      const uint64_t d[2] = {uint64_t(P), uint64_t(rows)};
+      const uint64_t sb[1] = {uint64_t(P) * 2};
+      return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, d, sb, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    };
+    if (dw2) {
+      View2 h_rows;
+      h_rows.data = w + L.h;
+      h_rows.s0 = pr.I;
+      h_rows.s1 = 1;
+      h_rows.dtype = MOE_BF16;
+      rc = launch_gather_transpose(view2(dout), 1, sorted, L.S, pr.k, view2(wts), 1, w + B.dyT, P, pr.H, st,
+                                   &launches);
+      if (rc == cudaSuccess)
+        rc = launch_gather_transpose(h_rows, 0, sorted, L.S, pr.k, none, 0, w + B.hT, P, pr.I, st, &launches);
+      if (rc != cudaSuccess) return cuda_fail(rc, "transpose dy h");
+      if ((s = tmap(&mA, w + B.dyT, pr.H)) != MOE_OK) return s;
+      if ((s = tmap(&mB, w + B.hT, pr.I)) != MOE_OK) return s;
+      rc = launch_gemm_kgroup(mA, mB, pr.H, pr.I, pr.E, offsets, static_cast<float*>(dw2->data),
+                              dw2->strides[0], dw2->strides[1], dev->errors, dev->num_sms, st, &launches);
+      if (rc != cudaSuccess) return cuda_fail(rc, "gemm dw2");
+    }
+    if (dw13) {
+      rc = launch_gather_transpose(dgu_rows, 0, sorted, L.S, pr.k, none, 0, w + B.dguT, P, 2 * pr.I, st,
+                                   &launches);
+      if (rc == cudaSuccess)
+        rc = launch_gather_transpose(view2(x), 1, sorted, L.S, pr.k, none, 0, w + B.a1T, P, pr.H, st, &launches);
+      if (rc != cudaSuccess) return cuda_fail(rc, "transpose dgu x");
+      if ((s = tmap(&mA, w + B.dguT, 2 * pr.I)) != MOE_OK) return s;
+      if ((s = tmap(&mB, w + B.a1T, pr.H)) != MOE_OK) return s;
+      rc = launch_gemm_kgroup(mA, mB, 2 * pr.I, pr.H, pr.E, offsets, static_cast<float*>(dw13->data),
+                              dw13->strides[0], dw13->strides[1], dev->errors, dev->num_sms, st, &launches);
+      if (rc != cudaSuccess) return cuda_fail(rc, "gemm dw13");
+    }
+  }
   t_last_launches = launches;
   return MOE_OK;
 }
@@ -1184,11 +1253,12 @@ size_t moe_backward_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, 
   return make_bwd_layout(T, H, I, E, k).total;
 }
 
-moe_status_t moe_backward_input_ws(const moe_tensor_t* x, const moe_w13_t* w13, const moe_tensor_t* w2,
-                                   const moe_tensor_t* w13t, const moe_tensor_t* w2t,
-                                   const moe_tensor_t* topk_ids, const moe_tensor_t* topk_weights,
-                                   const moe_tensor_t* dout, moe_tensor_t* dx, moe_tensor_t* dweights,
-                                   void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+moe_status_t moe_backward_ws(const moe_tensor_t* x, const moe_w13_t* w13, const moe_tensor_t* w2,
+                             const moe_tensor_t* w13t, const moe_tensor_t* w2t,
+                             const moe_tensor_t* topk_ids, const moe_tensor_t* topk_weights,
+                             const moe_tensor_t* dout, moe_tensor_t* dx, moe_tensor_t* dweights,
+                             moe_tensor_t* dw13, moe_tensor_t* dw2, void* workspace, size_t workspace_bytes,
+                             moe_stream_t stream) {
   t_last_launches = 0;
   Problem pr;
   moe_status_t s = validate(x, w13, w2, topk_ids, topk_weights, dx, false, &pr);
@@ -1202,8 +1272,26 @@ moe_status_t moe_backward_input_ws(const moe_tensor_t* x, const moe_w13_t* w13, 
   if (!sizes_ok(dweights, 2) || dweights->sizes[0] != pr.T || dweights->sizes[1] != pr.k)
     return MOE_ERR_SHAPE_MISMATCH;
   if (!dout->data || !dweights->data) return MOE_ERR_INVALID_ARG;
-  return backward_impl(x, w13, w2, w13t, w2t, topk_ids, topk_weights, dout, dx, dweights, pr, workspace,
-                       workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+  // fp32 weight gradients [E, 2I, H] (packed like w13) and [E, H, I]: rows 16-byte aligned
+  auto grad_ok = [&](const moe_tensor_t* t, int64_t R, int64_t C) {
+    return t->data && t->dtype == MOE_F32 && t->ndim == 3 && t->sizes[0] == pr.E && t->sizes[1] == R &&
+           t->sizes[2] == C && t->strides[2] == 1 && t->strides[1] % 4 == 0 && t->strides[0] % 4 == 0 &&
+           t->strides[0] >= R * t->strides[1] && reinterpret_cast<uintptr_t>(t->data) % 16 == 0;
+  };
+  if ((dw13 && !grad_ok(dw13, 2 * pr.I, pr.H)) || (dw2 && !grad_ok(dw2, pr.H, pr.I)))
+    return MOE_ERR_UNSUPPORTED_LAYOUT;
+  if ((dw13 || dw2) && (pr.H % 32 != 0 || pr.I % 32 != 0)) return MOE_ERR_UNSUPPORTED_LAYOUT;
+  return backward_impl(x, w13, w2, w13t, w2t, topk_ids, topk_weights, dout, dx, dweights, dw13, dw2, pr,
+                       workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_backward_input_ws(const moe_tensor_t* x, const moe_w13_t* w13, const moe_tensor_t* w2,
+                                   const moe_tensor_t* w13t, const moe_tensor_t* w2t,
+                                   const moe_tensor_t* topk_ids, const moe_tensor_t* topk_weights,
+                                   const moe_tensor_t* dout, moe_tensor_t* dx, moe_tensor_t* dweights,
+                                   void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+  return moe_backward_ws(x, w13, w2, w13t, w2t, topk_ids, topk_weights, dout, dx, dweights, nullptr, nullptr,
+                         workspace, workspace_bytes, stream);
 }
 
 moe_status_t moe_transpose_experts(const moe_tensor_t* src, moe_tensor_t* dst, moe_stream_t stream) {

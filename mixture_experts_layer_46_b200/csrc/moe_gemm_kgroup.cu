@@ -1,0 +1,276 @@
+// Expert-weight gradients: GEMMs grouped along K (tcgen05, sm_100a).
+//
+//   C[e, m, n] = sum over the expert's grouped rows p of A[m, p] * B[n, p]
+//
+// A [M, P] and B [N, P] are row-major bf16 (the grouped activations transposed,
+// so the contraction over an expert's rows is contiguous and both operands are
+// K-major like every other GEMM here); expert e owns rows [offsets[e],
+// offsets[e + 1]), a multiple of 64 (the align granule of the gradient path), and
+// its padding rows hold zeros in A and B.  C is fp32 [E, M, N]:
+//   dw2[e]          = (w dout)^T_e h_e        A = (w dout)^T [H, P], B = h^T [I, P]
+//   [dgate; dup][e] = [dg | du]^T_e x_e       A = [dg | du]^T [2I, P], B = x^T [H, P]
+// (the gradients of out = sum_j w y with respect to w2, gate and up).
+//
+// Kernel shape: one persistent CTA per SM, 6 warps: warp 0 TMA producer (one
+// [64 x 128] box of A and of B per k-block, 128-byte swizzle), warp 1 TMEM
+// allocator and MMA issuer (M = 128, N = 128, fp32 accumulators, two buffers),
+// warps 2-5 epilogue (one row m per thread, 32 columns per TMEM load, 128 bytes
+// of fp32 per row and chunk).  Work item = (expert, 128-row tile of M, 128-column
+// tile of N), expert-major; an expert with no rows gets zeros.
+#include "../../include/moe.h"
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kTM = 128, kTN = 128, kBK = 64, kUmmaK = 16;
+constexpr int kStages = 6;
+constexpr int kEpiWarps = 4;
+constexpr int kThreads = 32 * (2 + kEpiWarps);
+constexpr int kTmemCols = 2 * kTN;
+constexpr int kABytes = kTM * kBK * 2;  // 16 KiB
+constexpr int kBBytes = kTN * kBK * 2;  // 16 KiB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr size_t kSmem = 1024 + size_t(kStages) * kStageBytes + (2 * kStages + 4 + 1) * 8 + 16;
+
+struct KgArgs {
+  int64_t M, N, E;
+  int64_t n_mt, n_nt;
+  const int32_t* offsets;  // [E + 1] grouped-row offsets, multiples of 64
+  float* out;              // C[e, m, n] at out[e * o0 + m * o1 + n]
+  int64_t o0, o1;
+  DeviceErrors* err;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kgroup_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                       const KgArgs g) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stages = base;
+  uint64_t* full = reinterpret_cast<uint64_t*>(stages + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  pdl_wait();
+  const int64_t per_e = g.n_mt * g.n_nt;
+  const int64_t total = g.E * per_e;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      uint32_t stage = 0, phase = 0;
+      int8_t last_phase[kStages];
+      for (int s = 0; s < kStages; ++s) last_phase[s] = -1;
+      const uint64_t pol = l2_policy_evict_last();
+      bool ok = true;
+      for (int64_t item = blockIdx.x; item < total && ok; item += gridDim.x) {
+        const int64_t e = item / per_e, r = item - e * per_e;
+        const int32_t m0 = static_cast<int32_t>((r / g.n_nt) * kTM);
+        const int32_t n0 = static_cast<int32_t>((r % g.n_nt) * kTN);
+        const int k0 = g.offsets[e] / kBK, k1 = g.offsets[e + 1] / kBK;
+        for (int kb = k0; kb < k1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, g.err)) { ok = false; break; }
+          uint8_t* sa = stages + stage * kStageBytes;
+          mbar_arrive_expect_tx(&full[stage], kStageBytes);
+          tma_load_2d(sa, &tmA, &full[stage], kb * kBK, m0, pol);
+          tma_load_2d(sa + kABytes, &tmB, &full[stage], kb * kBK, n0, pol);
+          last_phase[stage] = static_cast<int8_t>(phase);
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        for (int s = 0; s < kStages; ++s)
+          if (last_phase[s] >= 0) mbar_wait(&full[s], static_cast<uint32_t>(last_phase[s]), g.err);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      uint32_t stage = 0, phase = 0, buf = 0, acc_phase = 0;
+      bool ok = true, issued = false;
+      const uint32_t idesc = idesc_bf16_f32(kTM, kTN);
+      for (int64_t item = blockIdx.x; item < total && ok; item += gridDim.x) {
+        const int64_t e = item / per_e;
+        const int k0 = g.offsets[e] / kBK, k1 = g.offsets[e + 1] / kBK;
+        if (!mbar_wait(&tempty[buf], acc_phase ^ 1u, g.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t acc = tmem_base + buf * kTN;
+        for (int kb = k0; kb < k1; ++kb) {
+          if (!mbar_wait(&full[stage], phase, g.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(stages + stage * kStageBytes);
+          const uint32_t b_addr = a_addr + kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / kUmmaK; ++kk)
+            mma_bf16(acc, sw128_kmajor_desc(a_addr + kk * kUmmaK * 2), sw128_kmajor_desc(b_addr + kk * kUmmaK * 2),
+                     idesc, (kb > k0 || kk > 0) ? 1u : 0u);
+          issued = true;
+          mma_commit(&empty[stage]);
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit(&tfull[buf]);  // with no k-block it completes at once (the epilogue writes zeros)
+        if (++buf == 2) { buf = 0; acc_phase ^= 1u; }
+      }
+      if (!ok && issued) {
+        mma_commit(drain);
+        mbar_wait(drain, 0, g.err);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quad = warp & 3;  // TMEM lanes [32 quad, 32 quad + 32) = rows m of this warp
+    uint32_t buf = 0, acc_phase = 0;
+    for (int64_t item = blockIdx.x; item < total; item += gridDim.x) {
+      const int64_t e = item / per_e, r = item - e * per_e;
+      const int64_t m = (r / g.n_nt) * kTM + quad * 32 + lane;
+      const int64_t n0 = (r % g.n_nt) * kTN;
+      const bool empty_e = g.offsets[e + 1] == g.offsets[e];
+      if (!mbar_wait(&tfull[buf], acc_phase, g.err)) break;
+      tc_fence_after();
+      const uint32_t lane_base = (static_cast<uint32_t>(quad * 32) << 16) + buf * kTN;
+      float* row = g.out + e * g.o0 + m * g.o1;
+#pragma unroll 1
+      for (int c = 0; c < kTN / 32; ++c) {
+        uint32_t v[32];
+        if (!empty_e) {
+          tmem_ld32(tmem_base + lane_base + c * 32, v);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = 0u;
+        }
+        const int64_t n = n0 + c * 32;
+        if (m < g.M && n < g.N) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<uint4*>(row + n + 4 * q) = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
+      if (++buf == 2) { buf = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  pdl_launch_dependents();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// dst[c, p] = 0 for a padding row p (sorted[p] >= S), else scale(p) * src_row(p)[c],
+// where src_row(p) is row sorted[p] / k of a token-major tensor (gather) or row p
+// of a grouped [P, C] matrix, and scale(p) is the slot's routing weight or 1;
+// 32 x 32 tiles through shared memory.
+__global__ void __launch_bounds__(32 * 8) gather_transpose_kernel(View2 src, int gather, const int32_t* sorted,
+                                                                 int64_t S, int64_t k, View2 wts, int scale,
+                                                                 uint16_t* dst, int64_t P, int64_t C) {
+  __shared__ uint16_t tile[32][33];
+  pdl_wait();
+  const int64_t p0 = static_cast<int64_t>(blockIdx.x) * 32, c0 = static_cast<int64_t>(blockIdx.y) * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int i = ty; i < 32; i += 8) {
+    const int64_t p = p0 + i, c = c0 + tx;
+    uint16_t v = 0;
+    if (p < P && c < C) {
+      const int32_t s = sorted[p];
+      if (s >= 0 && s < S) {
+        const int64_t t = s / k, j = s - t * k;
+        const int64_t rowi = gather ? t : p;
+        const uint16_t raw = static_cast<const uint16_t*>(src.data)[rowi * src.s0 + c * src.s1];
+        if (scale) {
+          const float w = static_cast<const float*>(wts.data)[t * wts.s0 + j * wts.s1];
+          const __nv_bfloat16 b = __float2bfloat16_rn(w * __uint_as_float(static_cast<uint32_t>(raw) << 16));
+          v = __bfloat16_as_ushort(b);
+        } else {
+          v = raw;
+        }
+      }
+    }
+    tile[i][tx] = v;
+  }
+  __syncthreads();
+  for (int i = ty; i < 32; i += 8) {
+    const int64_t c = c0 + i, p = p0 + tx;
+    if (c < C && p < P) dst[c * P + p] = tile[tx][i];
+  }
+  pdl_launch_dependents();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_kgroup(const CUtensorMap& a, const CUtensorMap& b, int64_t M, int64_t N, int64_t E,
+                               const int32_t* offsets, float* out, int64_t o0, int64_t o1, DeviceErrors* err,
+                               int num_sms, cudaStream_t st, int* launches) {
+  static unsigned long long configured = 0;
+  int dev = 0;
+  cudaError_t rc = cudaGetDevice(&dev);
+  if (rc != cudaSuccess) return rc;
+  if (dev >= 64 || !(configured & (1ull << dev))) {
+    rc = cudaFuncSetAttribute(gemm_kgroup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(kSmem));
+    if (rc != cudaSuccess) return rc;
+    if (dev < 64) configured |= 1ull << dev;
+  }
+  KgArgs g;
+  g.M = M;
+  g.N = N;
+  g.E = E;
+  g.n_mt = (M + kTM - 1) / kTM;
+  g.n_nt = (N + kTN - 1) / kTN;
+  g.offsets = offsets;
+  g.out = out;
+  g.o0 = o0;
+  g.o1 = o1;
+  g.err = err;
+  const int64_t total = E * g.n_mt * g.n_nt;
+  int64_t grid = total < num_sms ? total : num_sms;
+  if (grid < 1) grid = 1;
+  if (launches) *launches += 1;
+  return launch_pdl(gemm_kgroup_kernel, dim3(static_cast<unsigned>(grid)), dim3(kThreads), kSmem, st, a, b, g);
+}
+
+cudaError_t launch_gather_transpose(const View2& src, int gather, const int32_t* sorted, int64_t S, int64_t k,
+                                    const View2& wts, int scale, void* dst, int64_t P, int64_t C,
+                                    cudaStream_t st, int* launches) {
+  if (P == 0 || C == 0) return cudaSuccess;
+  if ((C + 31) / 32 > 65535) return cudaErrorInvalidValue;
+  if (launches) *launches += 1;
+  const dim3 grid(static_cast<unsigned>((P + 31) / 32), static_cast<unsigned>((C + 31) / 32));
+  return launch_pdl(gather_transpose_kernel, grid, dim3(32 * 8), 0, st, src, gather, sorted, S, k, wts, scale,
+                    static_cast<uint16_t*>(dst), P, C);
+}
+
+}  // namespace moe

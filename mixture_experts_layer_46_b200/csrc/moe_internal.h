@@ -105,6 +105,20 @@ cudaError_t launch_slot_dot(const View2& dout, const __nv_bfloat16* y, const int
                             int64_t T, int64_t H, int64_t k, const View2& dw, cudaStream_t st,
                             int* launches);
 
+// Expert-weight gradient GEMM grouped along K: C[e, m, n] = sum over expert e's
+// grouped rows p of A[m, p] B[n, p]; a / b map A [M, P] and B [N, P] bf16 ([64 x 128]
+// boxes, 128-byte swizzle); offsets [E + 1] multiples of 64; C fp32 at
+// out[e * o0 + m * o1 + n] (N % 32 == 0, 16-byte aligned rows)
+cudaError_t launch_gemm_kgroup(const CUtensorMap& a, const CUtensorMap& b, int64_t M, int64_t N, int64_t E,
+                               const int32_t* offsets, float* out, int64_t o0, int64_t o1, DeviceErrors* err,
+                               int num_sms, cudaStream_t st, int* launches);
+// dst [C, P] (row-major) = the grouped rows transposed, padding rows as zeros:
+// dst[c, p] = scale(p) * src_row(p)[c], src_row(p) = row sorted[p] / k of src
+// (gather = 1) or row p of src, scale(p) = routing weight of slot sorted[p] (scale = 1) or 1
+cudaError_t launch_gather_transpose(const View2& src, int gather, const int32_t* sorted, int64_t S, int64_t k,
+                                    const View2& wts, int scale, void* dst, int64_t P, int64_t C,
+                                    cudaStream_t st, int* launches);
+
 // dst[e, c, r] = src[e, r, c] for bf16 [E, R, C] (element strides; inner stride 1 both)
 cudaError_t launch_transpose_experts(const void* src, int64_t s0, int64_t s1, void* dst, int64_t d0,
                                      int64_t d1, int64_t E, int64_t R, int64_t C, cudaStream_t st);

@@ -1,5 +1,6 @@
-"""GPU parity of the gradient path (moe_backward_input_ws, moe_transpose_experts)
-against the fp64 oracle gradient (oracle.moe_backward_input).
+"""GPU parity of the gradient path (moe_backward_ws, moe_backward_input_ws,
+moe_transpose_experts) against the fp64 oracle gradients (oracle.moe_backward_input,
+oracle.moe_backward_weights).
 
 Tolerance: the CUDA path rounds to bf16 where the oracle keeps fp64: dh, dg and du,
 the recomputed h, the per-slot expert output y (for the routing-weight gradient)
@@ -8,7 +9,9 @@ and the per-slot da rows (for dx), then dx itself.  Each rounding is at most
 relative to the largest element stays a few times 2^-9 (~0.2 %) per step; 2e-2
 relative to the largest |dx| (|dweights|) leaves room for four such steps and the
 fp32 accumulation order, while a wrong term, sign or index (the oracle pins'
-failure modes) moves results by O(1).
+failure modes) moves results by O(1).  The weight gradients sum bf16 products of
+the same rounded operands (w dout, h, dg, du, x) in fp32 over an expert's slots,
+relative to the largest element of each gradient tensor: the same bound.
 """
 
 import pytest
@@ -141,3 +144,53 @@ def test_qwen3_235b_shape_sampled_tokens(qwen3_weights):
     ref_dx, ref_dw = oracle_backward(host, tokens=toks)
     assert rel_err(dx.cpu()[toks], ref_dx) <= BWD_TOL
     assert rel_err(dw.cpu()[toks], ref_dw) <= BWD_TOL
+
+
+def gpu_backward_weights(c, **kw):
+    v = moe.w13_from_packed(c["w13"])
+    w13t = moe.transpose_experts(c["w13"])
+    w2t = moe.transpose_experts(c["w2"])
+    res = moe.backward(c["x"], v, c["w2"], w13t, w2t, c["ids"], c["wts"], c["dout"], **kw)
+    torch.cuda.synchronize()
+    return res
+
+
+@pytest.mark.parametrize("T,H,I,E,k", [
+    (64, 256, 256, 8, 2),
+    (200, 512, 384, 16, 4),    # several 128-row tiles of M and N, N tail of I (dw2)
+    (77, 288, 96, 6, 3),       # ragged K of the recompute, M and N not multiples of 128
+    (4, 256, 128, 32, 2),      # most experts get no slot: their gradients are zero
+])
+def test_weight_gradients_match_oracle(T, H, I, E, k):
+    case = make_case(T, H, I, E, k, seed=T + 53)
+    gate, up = wl.gate_up_views(case["w13"])
+    ref_dg, ref_du, ref_dw2 = oracle.moe_backward_weights(case["x"], gate, up, case["w2"], case["ids"],
+                                                          case["wts"], case["dout"])
+    ref_dx, ref_dw = oracle_backward(case)
+    c = {n: v.cuda() for n, v in case.items()}
+    dx, dw, dw13, dw2 = gpu_backward_weights(c)
+    assert rel_err(dx, ref_dx) <= BWD_TOL
+    assert rel_err(dw, ref_dw) <= BWD_TOL
+    assert rel_err(dw13[:, :I], ref_dg) <= BWD_TOL
+    assert rel_err(dw13[:, I:], ref_du) <= BWD_TOL
+    assert rel_err(dw2, ref_dw2) <= BWD_TOL
+    unrouted = sorted(set(range(E)) - set(case["ids"].reshape(-1).tolist()))
+    for e in unrouted:
+        assert dw13[e].abs().max().item() == 0.0 and dw2[e].abs().max().item() == 0.0
+    # the input gradients do not depend on whether the weight gradients are asked for
+    dx2, dw_2, _, _ = gpu_backward_weights(c, weights=False)
+    assert torch.equal(dx2, dx) and torch.equal(dw_2, dw)
+
+
+def test_weight_gradients_into_strided_outputs_are_deterministic():
+    case = make_case(150, 256, 128, 8, 4, seed=61)
+    c = {n: v.cuda() for n, v in case.items()}
+    _, _, a13, a2 = gpu_backward_weights(c)
+    _, _, b13, b2 = gpu_backward_weights(c)
+    assert torch.equal(a13, b13) and torch.equal(a2, b2)
+    big13 = torch.full((8, 2 * 128 + 4, 256 + 8), 7.0, device="cuda")
+    big2 = torch.full((8, 256, 128 + 12), 7.0, device="cuda")
+    _, _, s13, s2 = gpu_backward_weights(c, dw13=big13[:, 2:2 + 2 * 128, 4:4 + 256],
+                                         dw2=big2[:, :, 8:8 + 128])
+    assert torch.equal(s13, a13) and torch.equal(s2, a2)
+    assert (big2[:, :, :8] == 7.0).all() and (big13[:, :2] == 7.0).all()  # nothing written outside
