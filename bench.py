@@ -353,7 +353,7 @@ def main():
     ap.add_argument("--sweep", default=None, help="write a token-sweep JSONL here (extra lines)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--grad", action="store_true",
-                    help="time the gradient path (dx and the routing-weight gradient, experts frozen) "
+                    help="time the gradient (dx, the routing-weight and the expert-weight gradients) "
                          "instead of the forward; prints its own JSON line")
     ap.add_argument("--config", default=None,
                     help="override configuration flags of the timed forward, e.g. fused=1,tile=32 "
@@ -539,12 +539,13 @@ def main():
 
 
 def run_grad(args, w, moe, wl, inp, v13, dev, stream, flush):
-    """The gradient path (moe_backward_input_ws) on the forward's workload, timed like
-    the forward: L2 flushed clean before every step, CUDA events, clocks sampled.
-    Roofline: 12 H I FLOPs per slot (twice the forward: dh, the gate/up recompute, the
-    unweighted down projection and da) against the slower of the bf16 burst peak and
+    """The full gradient (moe_backward_ws: dx, the routing-weight gradient and the
+    expert-weight gradients) on the forward's workload, timed like the forward: L2
+    flushed clean before every step, CUDA events, clocks sampled.  Roofline: 18 H I
+    FLOPs per slot (three times the forward: dh, the gate/up recompute, the unweighted
+    down projection, da, dw2 and dw13) against the slower of the bf16 burst peak and
     the HBM time of the activated experts' weights read twice (w2^T, gate/up, w2,
-    w13^T) plus x, dout and dx."""
+    w13^T), the fp32 weight gradients written, and x, dout and dx."""
     hbm, tf_burst, _, _ = peaks()
     T, H = w["T"], w["H"]
     w13t = moe.transpose_experts(inp["w13"])
@@ -554,10 +555,12 @@ def run_grad(args, w, moe, wl, inp, v13, dev, stream, flush):
     dwt = torch.empty(T, w["k"], dtype=torch.float32, device=dev)
     gws = torch.empty(moe.backward_workspace_bytes(T, H, w["I"], w["E"], w["k"]), dtype=torch.uint8,
                       device=dev)
+    dw13 = torch.empty(w["E"], 2 * w["I"], H, dtype=torch.float32, device=dev)
+    dw2 = torch.empty(w["E"], H, w["I"], dtype=torch.float32, device=dev)
 
     def gstep():
-        moe.backward_input(inp["x"], v13, inp["w2"], w13t, w2t, inp["ids"], inp["wts"], dout, dx, dwt,
-                           workspace=gws, stream=stream)
+        moe.backward(inp["x"], v13, inp["w2"], w13t, w2t, inp["ids"], inp["wts"], dout, dx, dwt, dw13, dw2,
+                     workspace=gws, stream=stream)
 
     for _ in range(args.warmup):
         gstep()
@@ -577,11 +580,12 @@ def run_grad(args, w, moe, wl, inp, v13, dev, stream, flush):
     per = sorted(a.elapsed_time(b) for a, b in evs)
     ms = sum(per) / len(per)
     alg = algorithmic(w, inp["ids"])
-    flops = 2.0 * alg["flops"]
-    gbytes = 2.0 * 3.0 * w["I"] * H * 2.0 * alg["active_experts"] + 3.0 * T * H * 2
+    flops = 3.0 * alg["flops"]
+    gbytes = (2.0 * 3.0 * w["I"] * H * 2.0 * alg["active_experts"] + 3.0 * w["I"] * H * 4.0 * w["E"] +
+              3.0 * T * H * 2)
     t_roof = max(flops / (tf_burst * 1e12), gbytes / (hbm * 1e9))
     print(json.dumps({
-        "metric": "fused-MoE layer gradient (dx, routing weights; experts frozen) tokens/s on 1 B200",
+        "metric": "fused-MoE layer gradient (dx, routing weights, expert weights) tokens/s on 1 B200",
         "value": T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": args.steps,
         "warmup": args.warmup, "higher_is_better": True, "dtype": "bf16",
         "config": {"workload": workload_name(w) + " gradient", "tokens_per_gpu": T,

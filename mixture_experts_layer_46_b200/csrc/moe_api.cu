@@ -1108,8 +1108,15 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
     dgu_rows.s0 = 2 * pr.I;
     dgu_rows.s1 = 1;
     dgu_rows.dtype = MOE_BF16;
-    CUtensorMap mA, mB;
+    CUtensorMap mA, mB, mC;
     const uint32_t box[2] = {64, 128};
+    // fp32 gradient [E, M, N] stored by TMA in [32 x 32] tiles
+    auto cmap = [&](CUtensorMap* m, const moe_tensor_t* t, int64_t M, int64_t N) {
+      const uint64_t d[3] = {uint64_t(N), uint64_t(M), uint64_t(pr.E)};
+      const uint64_t sb[2] = {uint64_t(t->strides[1]) * 4, uint64_t(t->strides[0]) * 4};
+      const uint32_t cbox[3] = {32, 32, 1};
+      return make_map(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, t->data, d, sb, cbox, CU_TENSOR_MAP_SWIZZLE_128B);
+    };
     auto tmap = [&](CUtensorMap* m, uint8_t* base, int64_t rows) {
       const uint64_t d[2] = {uint64_t(P), uint64_t(rows)};
       const uint64_t sb[1] = {uint64_t(P) * 2};
@@ -1128,8 +1135,8 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
       if (rc != cudaSuccess) return cuda_fail(rc, "transpose dy h");
       if ((s = tmap(&mA, w + B.dyT, pr.H)) != MOE_OK) return s;
       if ((s = tmap(&mB, w + B.hT, pr.I)) != MOE_OK) return s;
-      rc = launch_gemm_kgroup(mA, mB, pr.H, pr.I, pr.E, offsets, static_cast<float*>(dw2->data),
-                              dw2->strides[0], dw2->strides[1], dev->errors, dev->num_sms, st, &launches);
+      if ((s = cmap(&mC, dw2, pr.H, pr.I)) != MOE_OK) return s;
+      rc = launch_gemm_kgroup(mA, mB, mC, pr.H, pr.I, pr.E, offsets, dev->errors, dev->num_sms, st, &launches);
       if (rc != cudaSuccess) return cuda_fail(rc, "gemm dw2");
     }
     if (dw13) {
@@ -1140,8 +1147,9 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
       if (rc != cudaSuccess) return cuda_fail(rc, "transpose dgu x");
       if ((s = tmap(&mA, w + B.dguT, 2 * pr.I)) != MOE_OK) return s;
       if ((s = tmap(&mB, w + B.a1T, pr.H)) != MOE_OK) return s;
-      rc = launch_gemm_kgroup(mA, mB, 2 * pr.I, pr.H, pr.E, offsets, static_cast<float*>(dw13->data),
-                              dw13->strides[0], dw13->strides[1], dev->errors, dev->num_sms, st, &launches);
+      if ((s = cmap(&mC, dw13, 2 * pr.I, pr.H)) != MOE_OK) return s;
+      rc = launch_gemm_kgroup(mA, mB, mC, 2 * pr.I, pr.H, pr.E, offsets, dev->errors, dev->num_sms, st,
+                              &launches);
       if (rc != cudaSuccess) return cuda_fail(rc, "gemm dw13");
     }
   }

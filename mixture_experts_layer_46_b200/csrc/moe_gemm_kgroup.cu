@@ -14,9 +14,11 @@
 // Kernel shape: one persistent CTA per SM, 6 warps: warp 0 TMA producer (one
 // [64 x 128] box of A and of B per k-block, 128-byte swizzle), warp 1 TMEM
 // allocator and MMA issuer (M = 128, N = 128, fp32 accumulators, two buffers),
-// warps 2-5 epilogue (one row m per thread, 32 columns per TMEM load, 128 bytes
-// of fp32 per row and chunk).  Work item = (expert, 128-row tile of M, 128-column
-// tile of N), expert-major; an expert with no rows gets zeros.
+// warps 2-5 epilogue (one row m per thread, 32 columns per TMEM load: the warp's
+// 32 x 32 fp32 tile goes to shared memory in the 128-byte swizzled layout and out
+// with one TMA store, which also clips the M and N tails).  Work item = (expert,
+// 128-row tile of M, 128-column tile of N), expert-major; an expert with no rows
+// gets zeros.
 #include "../../include/moe.h"
 #include "moe_internal.h"
 
@@ -31,24 +33,39 @@ constexpr int kTmemCols = 2 * kTN;
 constexpr int kABytes = kTM * kBK * 2;  // 16 KiB
 constexpr int kBBytes = kTN * kBK * 2;  // 16 KiB
 constexpr int kStageBytes = kABytes + kBBytes;
-constexpr size_t kSmem = 1024 + size_t(kStages) * kStageBytes + (2 * kStages + 4 + 1) * 8 + 16;
+constexpr int kStgBytes = 32 * 128;  // per epilogue warp: 32 rows x 32 fp32
+constexpr size_t kSmem = 1024 + size_t(kStages) * kStageBytes + kEpiWarps * kStgBytes +
+                         (2 * kStages + 4 + 1) * 8 + 16;
 
 struct KgArgs {
   int64_t M, N, E;
   int64_t n_mt, n_nt;
   const int32_t* offsets;  // [E + 1] grouped-row offsets, multiples of 64
-  float* out;              // C[e, m, n] at out[e * o0 + m * o1 + n]
-  int64_t o0, o1;
   DeviceErrors* err;
 };
 
+// shared -> global tile store (bulk group of the issuing thread)
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int32_t c0, int32_t c1,
+                                             int32_t c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kgroup_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                       const KgArgs g) {
+                       const __grid_constant__ CUtensorMap tmC, const KgArgs g) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = base;
-  uint64_t* full = reinterpret_cast<uint64_t*>(stages + kStages * kStageBytes);
+  uint8_t* staging = stages + kStages * kStageBytes;  // 1024-byte aligned: the swizzle atom
+  uint64_t* full = reinterpret_cast<uint64_t*>(staging + kEpiWarps * kStgBytes);
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
@@ -59,6 +76,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmC);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -148,16 +166,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int quad = warp & 3;  // TMEM lanes [32 quad, 32 quad + 32) = rows m of this warp
+    const uint32_t stg = smem_u32(staging + (warp - 2) * kStgBytes);
     uint32_t buf = 0, acc_phase = 0;
     for (int64_t item = blockIdx.x; item < total; item += gridDim.x) {
       const int64_t e = item / per_e, r = item - e * per_e;
-      const int64_t m = (r / g.n_nt) * kTM + quad * 32 + lane;
-      const int64_t n0 = (r % g.n_nt) * kTN;
+      const int32_t m0 = static_cast<int32_t>((r / g.n_nt) * kTM + quad * 32);
+      const int32_t n0 = static_cast<int32_t>((r % g.n_nt) * kTN);
       const bool empty_e = g.offsets[e + 1] == g.offsets[e];
       if (!mbar_wait(&tfull[buf], acc_phase, g.err)) break;
       tc_fence_after();
       const uint32_t lane_base = (static_cast<uint32_t>(quad * 32) << 16) + buf * kTN;
-      float* row = g.out + e * g.o0 + m * g.o1;
 #pragma unroll 1
       for (int c = 0; c < kTN / 32; ++c) {
         uint32_t v[32];
@@ -168,11 +186,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = 0u;
         }
-        const int64_t n = n0 + c * 32;
-        if (m < g.M && n < g.N) {
+        if (m0 < g.M && n0 + c * 32 < g.N) {
+          if (lane == 0) bulk_wait_read_all();  // the previous tile store has read the staging
+          __syncwarp();
+          // row `lane` of the tile: 16-byte chunk q at position q ^ (row % 8) (128-byte swizzle)
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            *reinterpret_cast<uint4*>(row + n + 4 * q) = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stg + lane * 128 + ((q ^ (lane & 7)) * 16)),
+                         "r"(v[4 * q]), "r"(v[4 * q + 1]), "r"(v[4 * q + 2]), "r"(v[4 * q + 3])
+                         : "memory");
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&tmC, stg, n0 + c * 32, m0, static_cast<int32_t>(e));
+            bulk_commit();
+          }
         }
       }
       tc_fence_before();
@@ -180,6 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&tempty[buf]);
       if (++buf == 2) { buf = 0; acc_phase ^= 1u; }
     }
+    if (lane == 0) bulk_wait_all();  // C is written before the kernel ends
   }
 
   pdl_launch_dependents();
@@ -192,48 +221,58 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // dst[c, p] = 0 for a padding row p (sorted[p] >= S), else scale(p) * src_row(p)[c],
 // where src_row(p) is row sorted[p] / k of a token-major tensor (gather) or row p
-// of a grouped [P, C] matrix, and scale(p) is the slot's routing weight or 1;
-// 32 x 32 tiles through shared memory.
-__global__ void __launch_bounds__(32 * 8) gather_transpose_kernel(View2 src, int gather, const int32_t* sorted,
-                                                                 int64_t S, int64_t k, View2 wts, int scale,
-                                                                 uint16_t* dst, int64_t P, int64_t C) {
-  __shared__ uint16_t tile[32][33];
+// of a grouped [P, C] matrix, and scale(p) is the slot's routing weight or 1.
+// 64 x 64 tiles through shared memory, 256 threads: a warp reads two consecutive
+// columns per lane (128 bytes of a source row) and writes two consecutive rows p per
+// lane (128 bytes of a destination row).  P is even (a multiple of the 64-row granule).
+__device__ __forceinline__ uint16_t gt_elem(const View2& src, int64_t rowi, int64_t c, int64_t C, int scale,
+                                            float w) {
+  if (c >= C) return 0;
+  const uint16_t raw = static_cast<const uint16_t*>(src.data)[rowi * src.s0 + c * src.s1];
+  if (!scale) return raw;
+  return __bfloat16_as_ushort(__float2bfloat16_rn(w * __uint_as_float(static_cast<uint32_t>(raw) << 16)));
+}
+
+__global__ void __launch_bounds__(256) gather_transpose_kernel(View2 src, int gather, const int32_t* sorted,
+                                                               int64_t S, int64_t k, View2 wts, int scale,
+                                                               uint32_t* dst, int64_t P, int64_t C) {
+  __shared__ uint32_t tile[64][33];  // [row p][column pair], one padding word per row
   pdl_wait();
-  const int64_t p0 = static_cast<int64_t>(blockIdx.x) * 32, c0 = static_cast<int64_t>(blockIdx.y) * 32;
+  const int64_t p0 = static_cast<int64_t>(blockIdx.x) * 64, c0 = static_cast<int64_t>(blockIdx.y) * 64;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  for (int i = ty; i < 32; i += 8) {
-    const int64_t p = p0 + i, c = c0 + tx;
-    uint16_t v = 0;
-    if (p < P && c < C) {
+  for (int i = ty; i < 64; i += 8) {
+    const int64_t p = p0 + i, c = c0 + 2 * tx;
+    uint32_t v = 0;
+    if (p < P) {
       const int32_t s = sorted[p];
       if (s >= 0 && s < S) {
         const int64_t t = s / k, j = s - t * k;
         const int64_t rowi = gather ? t : p;
-        const uint16_t raw = static_cast<const uint16_t*>(src.data)[rowi * src.s0 + c * src.s1];
-        if (scale) {
-          const float w = static_cast<const float*>(wts.data)[t * wts.s0 + j * wts.s1];
-          const __nv_bfloat16 b = __float2bfloat16_rn(w * __uint_as_float(static_cast<uint32_t>(raw) << 16));
-          v = __bfloat16_as_ushort(b);
-        } else {
-          v = raw;
-        }
+        const float w = scale ? static_cast<const float*>(wts.data)[t * wts.s0 + j * wts.s1] : 1.0f;
+        v = static_cast<uint32_t>(gt_elem(src, rowi, c, C, scale, w)) |
+            (static_cast<uint32_t>(gt_elem(src, rowi, c + 1, C, scale, w)) << 16);
       }
     }
     tile[i][tx] = v;
   }
   __syncthreads();
-  for (int i = ty; i < 32; i += 8) {
-    const int64_t c = c0 + i, p = p0 + tx;
-    if (c < C && p < P) dst[c * P + p] = tile[tx][i];
+  for (int i = ty; i < 64; i += 8) {
+    const int64_t c = c0 + i, p = p0 + 2 * tx;
+    if (c < C && p < P) {
+      const uint32_t sh = (i & 1) * 16;
+      const uint32_t lo = (tile[2 * tx][i >> 1] >> sh) & 0xffffu;
+      const uint32_t hi = (tile[2 * tx + 1][i >> 1] >> sh) & 0xffffu;
+      dst[(c * P + p) >> 1] = lo | (hi << 16);
+    }
   }
   pdl_launch_dependents();
 }
 
 }  // namespace
 
-cudaError_t launch_gemm_kgroup(const CUtensorMap& a, const CUtensorMap& b, int64_t M, int64_t N, int64_t E,
-                               const int32_t* offsets, float* out, int64_t o0, int64_t o1, DeviceErrors* err,
-                               int num_sms, cudaStream_t st, int* launches) {
+cudaError_t launch_gemm_kgroup(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c, int64_t M,
+                               int64_t N, int64_t E, const int32_t* offsets, DeviceErrors* err, int num_sms,
+                               cudaStream_t st, int* launches) {
   static unsigned long long configured = 0;
   int dev = 0;
   cudaError_t rc = cudaGetDevice(&dev);
@@ -251,26 +290,24 @@ cudaError_t launch_gemm_kgroup(const CUtensorMap& a, const CUtensorMap& b, int64
   g.n_mt = (M + kTM - 1) / kTM;
   g.n_nt = (N + kTN - 1) / kTN;
   g.offsets = offsets;
-  g.out = out;
-  g.o0 = o0;
-  g.o1 = o1;
   g.err = err;
   const int64_t total = E * g.n_mt * g.n_nt;
   int64_t grid = total < num_sms ? total : num_sms;
   if (grid < 1) grid = 1;
   if (launches) *launches += 1;
-  return launch_pdl(gemm_kgroup_kernel, dim3(static_cast<unsigned>(grid)), dim3(kThreads), kSmem, st, a, b, g);
+  return launch_pdl(gemm_kgroup_kernel, dim3(static_cast<unsigned>(grid)), dim3(kThreads), kSmem, st, a, b, c, g);
 }
 
 cudaError_t launch_gather_transpose(const View2& src, int gather, const int32_t* sorted, int64_t S, int64_t k,
                                     const View2& wts, int scale, void* dst, int64_t P, int64_t C,
                                     cudaStream_t st, int* launches) {
   if (P == 0 || C == 0) return cudaSuccess;
-  if ((C + 31) / 32 > 65535) return cudaErrorInvalidValue;
+  if ((C + 63) / 64 > 65535 || P % 2 != 0 || reinterpret_cast<uintptr_t>(dst) % 4 != 0)
+    return cudaErrorInvalidValue;
   if (launches) *launches += 1;
-  const dim3 grid(static_cast<unsigned>((P + 31) / 32), static_cast<unsigned>((C + 31) / 32));
-  return launch_pdl(gather_transpose_kernel, grid, dim3(32 * 8), 0, st, src, gather, sorted, S, k, wts, scale,
-                    static_cast<uint16_t*>(dst), P, C);
+  const dim3 grid(static_cast<unsigned>((P + 63) / 64), static_cast<unsigned>((C + 63) / 64));
+  return launch_pdl(gather_transpose_kernel, grid, dim3(256), 0, st, src, gather, sorted, S, k, wts, scale,
+                    static_cast<uint32_t*>(dst), P, C);
 }
 
 }  // namespace moe
