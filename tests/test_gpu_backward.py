@@ -194,3 +194,19 @@ def test_weight_gradients_into_strided_outputs_are_deterministic():
                                          dw2=big2[:, :, 8:8 + 128])
     assert torch.equal(s13, a13) and torch.equal(s2, a2)
     assert (big2[:, :, :8] == 7.0).all() and (big13[:, :2] == 7.0).all()  # nothing written outside
+
+
+@pytest.mark.slow
+def test_weight_gradients_at_qwen3_expert_dimensions():
+    # the Qwen3-235B expert shape (H=4096, I=1536) with 8 experts, so the fp64 oracle's
+    # dense gradients stay small: full-size M and N tiling of the grouped GEMMs
+    T, H, I, E, k = 48, 4096, 1536, 8, 4
+    case = make_case(T, H, I, E, k, seed=83)
+    gate, up = wl.gate_up_views(case["w13"])
+    ref_dg, ref_du, ref_dw2 = oracle.moe_backward_weights(case["x"], gate, up, case["w2"], case["ids"],
+                                                          case["wts"], case["dout"])
+    c = {n: v.cuda() for n, v in case.items()}
+    _, _, dw13, dw2 = gpu_backward_weights(c)
+    assert rel_err(dw13[:, :I], ref_dg) <= BWD_TOL
+    assert rel_err(dw13[:, I:], ref_du) <= BWD_TOL
+    assert rel_err(dw2, ref_dw2) <= BWD_TOL
