@@ -545,7 +545,7 @@ def run_grad(args, w, moe, wl, inp, v13, dev, stream, flush):
     FLOPs per slot (three times the forward: dh, the gate/up recompute, the unweighted
     down projection, da, dw2 and dw13) against the slower of the bf16 burst peak and
     the HBM time of the activated experts' weights read twice (w2^T, gate/up, w2,
-    w13^T), the fp32 weight gradients written, and x, dout and dx."""
+    w13^T), the bf16 weight gradients written, and x, dout and dx."""
     hbm, tf_burst, _, _ = peaks()
     T, H = w["T"], w["H"]
     w13t = moe.transpose_experts(inp["w13"])
@@ -555,8 +555,9 @@ def run_grad(args, w, moe, wl, inp, v13, dev, stream, flush):
     dwt = torch.empty(T, w["k"], dtype=torch.float32, device=dev)
     gws = torch.empty(moe.backward_workspace_bytes(T, H, w["I"], w["E"], w["k"]), dtype=torch.uint8,
                       device=dev)
-    dw13 = torch.empty(w["E"], 2 * w["I"], H, dtype=torch.float32, device=dev)
-    dw2 = torch.empty(w["E"], H, w["I"], dtype=torch.float32, device=dev)
+    # weight gradients in the weights' own dtype (bf16), as an autograd framework keeps them
+    dw13 = torch.empty(w["E"], 2 * w["I"], H, dtype=torch.bfloat16, device=dev)
+    dw2 = torch.empty(w["E"], H, w["I"], dtype=torch.bfloat16, device=dev)
 
     def gstep():
         moe.backward(inp["x"], v13, inp["w2"], w13t, w2t, inp["ids"], inp["wts"], dout, dx, dwt, dw13, dw2,
@@ -581,7 +582,7 @@ def run_grad(args, w, moe, wl, inp, v13, dev, stream, flush):
     ms = sum(per) / len(per)
     alg = algorithmic(w, inp["ids"])
     flops = 3.0 * alg["flops"]
-    gbytes = (2.0 * 3.0 * w["I"] * H * 2.0 * alg["active_experts"] + 3.0 * w["I"] * H * 4.0 * w["E"] +
+    gbytes = (2.0 * 3.0 * w["I"] * H * 2.0 * alg["active_experts"] + 3.0 * w["I"] * H * 2.0 * w["E"] +
               3.0 * T * H * 2)
     t_roof = max(flops / (tf_burst * 1e12), gbytes / (hbm * 1e9))
     print(json.dumps({

@@ -178,10 +178,11 @@ moe_status_t moe_forward_host(const moe_tensor_t* x_host, const moe_w13_t* w13,
 size_t moe_backward_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k);
 
 /* The same plus the expert-weight gradients (either may be NULL): dw13 = dL/dw13
- * f32 [E, 2I, H] packed like w13 (dgate rows [0, I), dup rows [I, 2I)) and dw2 =
- * dL/dw2 f32 [E, H, I], overwritten (zero for an expert no slot routes to), inner
- * stride 1 and the other strides multiples of 4 elements, 16-byte aligned; H and I
- * multiples of 32.  With the routing fixed:
+ * [E, 2I, H] packed like w13 (dgate rows [0, I), dup rows [I, 2I)) and dw2 = dL/dw2
+ * [E, H, I], f32 or bf16 (fp32 sums rounded once), overwritten (zero for an expert no
+ * slot routes to); inner stride 1, the other strides multiples of 16 bytes, 16-byte
+ * aligned, the last dimension a multiple of 32 (f32) or 64 (bf16) elements.  With the
+ * routing fixed:
  *   dw2[e]   = sum over e's slots (t, j) of w (dout_t) a^T,   a = silu(g) * u
  *   dgate[e] = sum of dg x_t^T,  dup[e] = sum of du x_t^T
  * each a GEMM that contracts over the expert's slots (fp32 accumulation). */

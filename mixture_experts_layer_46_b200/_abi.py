@@ -262,9 +262,11 @@ def transpose_experts(src: torch.Tensor, dst: torch.Tensor | None = None, *, str
 
 
 def backward(x, w13: MoeW13, w2, w13t, w2t, topk_ids, topk_weights, dout, dx=None, dweights=None,
-             dw13=None, dw2=None, *, weights=True, workspace: torch.Tensor | None = None, stream=None):
-    """(dx, dweights, dw13, dw2): the forward's gradients given dout; dw13 f32 [E, 2I, H]
-    (packed like w13) and dw2 f32 [E, H, I] are computed when `weights` (else None)."""
+             dw13=None, dw2=None, *, weights=True, grad_dtype=torch.float32,
+             workspace: torch.Tensor | None = None, stream=None):
+    """(dx, dweights, dw13, dw2): the forward's gradients given dout; dw13 [E, 2I, H]
+    (packed like w13) and dw2 [E, H, I] in grad_dtype (float32 or bfloat16) are
+    computed when `weights` (else None)."""
     T, H = x.shape
     k = topk_ids.shape[1]
     E, _, I = w2.shape
@@ -274,9 +276,9 @@ def backward(x, w13: MoeW13, w2, w13t, w2t, topk_ids, topk_weights, dout, dx=Non
     if dweights is None:
         dweights = torch.empty(T, k, dtype=torch.float32, device=dev)
     if weights and dw13 is None:
-        dw13 = torch.empty(E, 2 * I, H, dtype=torch.float32, device=dev)
+        dw13 = torch.empty(E, 2 * I, H, dtype=grad_dtype, device=dev)
     if weights and dw2 is None:
-        dw2 = torch.empty(E, H, I, dtype=torch.float32, device=dev)
+        dw2 = torch.empty(E, H, I, dtype=grad_dtype, device=dev)
     if workspace is None:
         n = backward_workspace_bytes(T, H, I, E, k)
         workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=dev)

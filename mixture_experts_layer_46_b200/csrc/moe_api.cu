@@ -947,8 +947,8 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   t_last_launches = 0;
   if (pr.T == 0) {
     // no tokens: the weight gradients are zero
-    if (dw13) MOE_CUDA(cudaMemsetAsync(dw13->data, 0, size_t(pr.E) * dw13->strides[0] * 4, st));
-    if (dw2) MOE_CUDA(cudaMemsetAsync(dw2->data, 0, size_t(pr.E) * dw2->strides[0] * 4, st));
+    if (dw13) MOE_CUDA(cudaMemsetAsync(dw13->data, 0, size_t(pr.E) * dw13->strides[0] * dtype_size(dw13->dtype), st));
+    if (dw2) MOE_CUDA(cudaMemsetAsync(dw2->data, 0, size_t(pr.E) * dw2->strides[0] * dtype_size(dw2->dtype), st));
     return MOE_OK;
   }
   const int32_t bm = kBwdBm;
@@ -1110,12 +1110,15 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
     dgu_rows.dtype = MOE_BF16;
     CUtensorMap mA, mB, mC;
     const uint32_t box[2] = {64, 128};
-    // fp32 gradient [E, M, N] stored by TMA in [32 x 32] tiles
+    // gradient [E, M, N] stored by TMA in 32-row tiles of 128-byte rows (fp32 or bf16)
     auto cmap = [&](CUtensorMap* m, const moe_tensor_t* t, int64_t M, int64_t N) {
+      const bool b16 = t->dtype == MOE_BF16;
+      const uint64_t es = b16 ? 2 : 4;
       const uint64_t d[3] = {uint64_t(N), uint64_t(M), uint64_t(pr.E)};
-      const uint64_t sb[2] = {uint64_t(t->strides[1]) * 4, uint64_t(t->strides[0]) * 4};
-      const uint32_t cbox[3] = {32, 32, 1};
-      return make_map(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, t->data, d, sb, cbox, CU_TENSOR_MAP_SWIZZLE_128B);
+      const uint64_t sb[2] = {uint64_t(t->strides[1]) * es, uint64_t(t->strides[0]) * es};
+      const uint32_t cbox[3] = {b16 ? 64u : 32u, 32, 1};
+      return make_map(m, b16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, t->data, d,
+                      sb, cbox, CU_TENSOR_MAP_SWIZZLE_128B);
     };
     auto tmap = [&](CUtensorMap* m, uint8_t* base, int64_t rows) {
       const uint64_t d[2] = {uint64_t(P), uint64_t(rows)};
@@ -1136,7 +1139,8 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
       if ((s = tmap(&mA, w + B.dyT, pr.H)) != MOE_OK) return s;
       if ((s = tmap(&mB, w + B.hT, pr.I)) != MOE_OK) return s;
       if ((s = cmap(&mC, dw2, pr.H, pr.I)) != MOE_OK) return s;
-      rc = launch_gemm_kgroup(mA, mB, mC, pr.H, pr.I, pr.E, offsets, dev->errors, dev->num_sms, st, &launches);
+      rc = launch_gemm_kgroup(mA, mB, mC, dw2->dtype == MOE_BF16, pr.H, pr.I, pr.E, offsets, dev->errors,
+                              dev->num_sms, st, &launches);
       if (rc != cudaSuccess) return cuda_fail(rc, "gemm dw2");
     }
     if (dw13) {
@@ -1148,8 +1152,8 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
       if ((s = tmap(&mA, w + B.dguT, 2 * pr.I)) != MOE_OK) return s;
       if ((s = tmap(&mB, w + B.a1T, pr.H)) != MOE_OK) return s;
       if ((s = cmap(&mC, dw13, 2 * pr.I, pr.H)) != MOE_OK) return s;
-      rc = launch_gemm_kgroup(mA, mB, mC, 2 * pr.I, pr.H, pr.E, offsets, dev->errors, dev->num_sms, st,
-                              &launches);
+      rc = launch_gemm_kgroup(mA, mB, mC, dw13->dtype == MOE_BF16, 2 * pr.I, pr.H, pr.E, offsets, dev->errors,
+                              dev->num_sms, st, &launches);
       if (rc != cudaSuccess) return cuda_fail(rc, "gemm dw13");
     }
   }
@@ -1280,15 +1284,17 @@ moe_status_t moe_backward_ws(const moe_tensor_t* x, const moe_w13_t* w13, const 
   if (!sizes_ok(dweights, 2) || dweights->sizes[0] != pr.T || dweights->sizes[1] != pr.k)
     return MOE_ERR_SHAPE_MISMATCH;
   if (!dout->data || !dweights->data) return MOE_ERR_INVALID_ARG;
-  // fp32 weight gradients [E, 2I, H] (packed like w13) and [E, H, I]: rows 16-byte aligned
+  // weight gradients [E, 2I, H] (packed like w13) and [E, H, I], fp32 or bf16: 16-byte
+  // aligned rows; the columns a multiple of one 128-byte tile row (32 fp32, 64 bf16)
   auto grad_ok = [&](const moe_tensor_t* t, int64_t R, int64_t C) {
-    return t->data && t->dtype == MOE_F32 && t->ndim == 3 && t->sizes[0] == pr.E && t->sizes[1] == R &&
-           t->sizes[2] == C && t->strides[2] == 1 && t->strides[1] % 4 == 0 && t->strides[0] % 4 == 0 &&
+    if (t->dtype != MOE_F32 && t->dtype != MOE_BF16) return false;
+    const int64_t v = 16 / dtype_size(t->dtype), cols = 128 / dtype_size(t->dtype);
+    return t->data && t->ndim == 3 && t->sizes[0] == pr.E && t->sizes[1] == R && t->sizes[2] == C &&
+           t->strides[2] == 1 && t->strides[1] % v == 0 && t->strides[0] % v == 0 && C % cols == 0 &&
            t->strides[0] >= R * t->strides[1] && reinterpret_cast<uintptr_t>(t->data) % 16 == 0;
   };
   if ((dw13 && !grad_ok(dw13, 2 * pr.I, pr.H)) || (dw2 && !grad_ok(dw2, pr.H, pr.I)))
     return MOE_ERR_UNSUPPORTED_LAYOUT;
-  if ((dw13 || dw2) && (pr.H % 32 != 0 || pr.I % 32 != 0)) return MOE_ERR_UNSUPPORTED_LAYOUT;
   return backward_impl(x, w13, w2, w13t, w2t, topk_ids, topk_weights, dout, dx, dweights, dw13, dw2, pr,
                        workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }

@@ -6,7 +6,7 @@
 // so the contraction over an expert's rows is contiguous and both operands are
 // K-major like every other GEMM here); expert e owns rows [offsets[e],
 // offsets[e + 1]), a multiple of 64 (the align granule of the gradient path), and
-// its padding rows hold zeros in A and B.  C is fp32 [E, M, N]:
+// its padding rows hold zeros in A and B.  C is [E, M, N], fp32 or bf16 (fp32 sums):
 //   dw2[e]          = (w dout)^T_e h_e        A = (w dout)^T [H, P], B = h^T [I, P]
 //   [dgate; dup][e] = [dg | du]^T_e x_e       A = [dg | du]^T [2I, P], B = x^T [H, P]
 // (the gradients of out = sum_j w y with respect to w2, gate and up).
@@ -14,9 +14,9 @@
 // Kernel shape: one persistent CTA per SM, 6 warps: warp 0 TMA producer (one
 // [64 x 128] box of A and of B per k-block, 128-byte swizzle), warp 1 TMEM
 // allocator and MMA issuer (M = 128, N = 128, fp32 accumulators, two buffers),
-// warps 2-5 epilogue (one row m per thread, 32 columns per TMEM load: the warp's
-// 32 x 32 fp32 tile goes to shared memory in the 128-byte swizzled layout and out
-// with one TMA store, which also clips the M and N tails).  Work item = (expert,
+// warps 2-5 epilogue (one row m per thread: the warp's 32-row tile of 32 fp32 or
+// 64 bf16 columns, 128 bytes a row, goes to shared memory in the 128-byte swizzled
+// layout and out with one TMA store, which also clips the M and N tails).  Work item = (expert,
 // 128-row tile of M, 128-column tile of N), expert-major; an expert with no rows
 // gets zeros.
 #include "../../include/moe.h"
@@ -58,6 +58,7 @@ __device__ __forceinline__ void bulk_wait_read_all() {
 }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+template <bool kBf16Out>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kgroup_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const __grid_constant__ CUtensorMap tmC, const KgArgs g) {
@@ -176,17 +177,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(&tfull[buf], acc_phase, g.err)) break;
       tc_fence_after();
       const uint32_t lane_base = (static_cast<uint32_t>(quad * 32) << 16) + buf * kTN;
+      // one staged tile row is 128 bytes: 32 fp32 or 64 bf16 columns
+      constexpr int kCols = kBf16Out ? 64 : 32;
 #pragma unroll 1
-      for (int c = 0; c < kTN / 32; ++c) {
+      for (int c = 0; c < kTN / kCols; ++c) {
         uint32_t v[32];
-        if (!empty_e) {
-          tmem_ld32(tmem_base + lane_base + c * 32, v);
-          tmem_wait_ld();
-        } else {
+        if (empty_e) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = 0u;
+        } else if (kBf16Out) {
+          uint32_t a[32], b[32];
+          tmem_ld32(tmem_base + lane_base + c * 64, a);
+          tmem_ld32(tmem_base + lane_base + c * 64 + 32, b);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            v[j] = pack_bf16x2(__uint_as_float(a[2 * j]), __uint_as_float(a[2 * j + 1]));
+            v[16 + j] = pack_bf16x2(__uint_as_float(b[2 * j]), __uint_as_float(b[2 * j + 1]));
+          }
+        } else {
+          tmem_ld32(tmem_base + lane_base + c * 32, v);
+          tmem_wait_ld();
         }
-        if (m0 < g.M && n0 + c * 32 < g.N) {
+        if (m0 < g.M && n0 + c * kCols < g.N) {
           if (lane == 0) bulk_wait_read_all();  // the previous tile store has read the staging
           __syncwarp();
           // row `lane` of the tile: 16-byte chunk q at position q ^ (row % 8) (128-byte swizzle)
@@ -198,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_3d(&tmC, stg, n0 + c * 32, m0, static_cast<int32_t>(e));
+            tma_store_3d(&tmC, stg, n0 + c * kCols, m0, static_cast<int32_t>(e));
             bulk_commit();
           }
         }
@@ -270,18 +283,19 @@ __global__ void __launch_bounds__(256) gather_transpose_kernel(View2 src, int ga
 
 }  // namespace
 
-cudaError_t launch_gemm_kgroup(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c, int64_t M,
-                               int64_t N, int64_t E, const int32_t* offsets, DeviceErrors* err, int num_sms,
-                               cudaStream_t st, int* launches) {
-  static unsigned long long configured = 0;
+cudaError_t launch_gemm_kgroup(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c, int bf16_out,
+                               int64_t M, int64_t N, int64_t E, const int32_t* offsets, DeviceErrors* err,
+                               int num_sms, cudaStream_t st, int* launches) {
+  static unsigned long long configured[2] = {0, 0};
   int dev = 0;
   cudaError_t rc = cudaGetDevice(&dev);
   if (rc != cudaSuccess) return rc;
-  if (dev >= 64 || !(configured & (1ull << dev))) {
-    rc = cudaFuncSetAttribute(gemm_kgroup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(kSmem));
+  const int bi = bf16_out ? 1 : 0;
+  if (dev >= 64 || !(configured[bi] & (1ull << dev))) {
+    rc = cudaFuncSetAttribute(bf16_out ? gemm_kgroup_kernel<true> : gemm_kgroup_kernel<false>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem));
     if (rc != cudaSuccess) return rc;
-    if (dev < 64) configured |= 1ull << dev;
+    if (dev < 64) configured[bi] |= 1ull << dev;
   }
   KgArgs g;
   g.M = M;
@@ -295,7 +309,11 @@ cudaError_t launch_gemm_kgroup(const CUtensorMap& a, const CUtensorMap& b, const
   int64_t grid = total < num_sms ? total : num_sms;
   if (grid < 1) grid = 1;
   if (launches) *launches += 1;
-  return launch_pdl(gemm_kgroup_kernel, dim3(static_cast<unsigned>(grid)), dim3(kThreads), kSmem, st, a, b, c, g);
+  if (bf16_out)
+    return launch_pdl(gemm_kgroup_kernel<true>, dim3(static_cast<unsigned>(grid)), dim3(kThreads), kSmem, st, a, b,
+                      c, g);
+  return launch_pdl(gemm_kgroup_kernel<false>, dim3(static_cast<unsigned>(grid)), dim3(kThreads), kSmem, st, a, b,
+                    c, g);
 }
 
 cudaError_t launch_gather_transpose(const View2& src, int gather, const int32_t* sorted, int64_t S, int64_t k,

@@ -107,11 +107,12 @@ cudaError_t launch_slot_dot(const View2& dout, const __nv_bfloat16* y, const int
 
 // Expert-weight gradient GEMM grouped along K: C[e, m, n] = sum over expert e's
 // grouped rows p of A[m, p] B[n, p]; a / b map A [M, P] and B [N, P] bf16 ([64 x 128]
-// boxes, 128-byte swizzle); offsets [E + 1] multiples of 64; c maps C fp32 [E, M, N]
-// (dims {N, M, E}, [32 x 32 x 1] boxes, 128-byte swizzle; N % 32 == 0)
-cudaError_t launch_gemm_kgroup(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c, int64_t M,
-                               int64_t N, int64_t E, const int32_t* offsets, DeviceErrors* err, int num_sms,
-                               cudaStream_t st, int* launches);
+// boxes, 128-byte swizzle); offsets [E + 1] multiples of 64; c maps C [E, M, N] (dims
+// {N, M, E}, 128-byte swizzle): fp32 in [32 x 32 x 1] boxes (N % 32 == 0) or, with
+// bf16_out, bf16 in [64 x 32 x 1] boxes (N % 64 == 0)
+cudaError_t launch_gemm_kgroup(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c, int bf16_out,
+                               int64_t M, int64_t N, int64_t E, const int32_t* offsets, DeviceErrors* err,
+                               int num_sms, cudaStream_t st, int* launches);
 // dst [C, P] (row-major) = the grouped rows transposed, padding rows as zeros:
 // dst[c, p] = scale(p) * src_row(p)[c], src_row(p) = row sorted[p] / k of src
 // (gather = 1) or row p of src, scale(p) = routing weight of slot sorted[p] (scale = 1) or 1
