@@ -235,47 +235,64 @@ __global__ void __launch_bounds__(kThreads, 1)
 // dst[c, p] = 0 for a padding row p (sorted[p] >= S), else scale(p) * src_row(p)[c],
 // where src_row(p) is row sorted[p] / k of a token-major tensor (gather) or row p
 // of a grouped [P, C] matrix, and scale(p) is the slot's routing weight or 1.
-// 64 x 64 tiles through shared memory, 256 threads: a warp reads two consecutive
-// columns per lane (128 bytes of a source row) and writes two consecutive rows p per
-// lane (128 bytes of a destination row).  P is even (a multiple of the 64-row granule).
-__device__ __forceinline__ uint16_t gt_elem(const View2& src, int64_t rowi, int64_t c, int64_t C, int scale,
-                                            float w) {
-  if (c >= C) return 0;
-  const uint16_t raw = static_cast<const uint16_t*>(src.data)[rowi * src.s0 + c * src.s1];
-  if (!scale) return raw;
+// 64 x 64 tiles through shared memory, 256 threads: each thread reads 8 consecutive
+// columns of a source row (16 bytes; element loads where the rows are not 16-byte
+// aligned) and writes 8 consecutive rows p of a destination row (16 bytes).  P is a
+// multiple of 64 (the granule), dst 16-byte aligned.
+__device__ __forceinline__ uint16_t gt_scale(uint16_t raw, float w) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(w * __uint_as_float(static_cast<uint32_t>(raw) << 16)));
 }
 
-__global__ void __launch_bounds__(256) gather_transpose_kernel(View2 src, int gather, const int32_t* sorted,
+__global__ void __launch_bounds__(256) gather_transpose_kernel(View2 src, int gather, int vec, const int32_t* sorted,
                                                                int64_t S, int64_t k, View2 wts, int scale,
-                                                               uint32_t* dst, int64_t P, int64_t C) {
-  __shared__ uint32_t tile[64][33];  // [row p][column pair], one padding word per row
+                                                               uint16_t* dst, int64_t P, int64_t C) {
+  __shared__ uint16_t tile[64][64 + 8];  // [row p][column c]; 16 bytes of padding per row
   pdl_wait();
   const int64_t p0 = static_cast<int64_t>(blockIdx.x) * 64, c0 = static_cast<int64_t>(blockIdx.y) * 64;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  for (int i = ty; i < 64; i += 8) {
-    const int64_t p = p0 + i, c = c0 + 2 * tx;
-    uint32_t v = 0;
+  const int tid = threadIdx.x;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int i = (tid >> 3) + 32 * h, q = tid & 7;  // row i of the tile, 8-column chunk q
+    const int64_t p = p0 + i, c = c0 + 8 * q;
+    uint16_t v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (p < P) {
       const int32_t s = sorted[p];
       if (s >= 0 && s < S) {
         const int64_t t = s / k, j = s - t * k;
-        const int64_t rowi = gather ? t : p;
-        const float w = scale ? static_cast<const float*>(wts.data)[t * wts.s0 + j * wts.s1] : 1.0f;
-        v = static_cast<uint32_t>(gt_elem(src, rowi, c, C, scale, w)) |
-            (static_cast<uint32_t>(gt_elem(src, rowi, c + 1, C, scale, w)) << 16);
+        const uint16_t* row = static_cast<const uint16_t*>(src.data) + (gather ? t : p) * src.s0;
+        if (vec && c + 8 <= C) {
+          const uint4 u = *reinterpret_cast<const uint4*>(row + c);
+          const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            v[2 * r] = static_cast<uint16_t>(w4[r] & 0xffffu);
+            v[2 * r + 1] = static_cast<uint16_t>(w4[r] >> 16);
+          }
+        } else {
+#pragma unroll
+          for (int r = 0; r < 8; ++r) v[r] = c + r < C ? row[(c + r) * src.s1] : uint16_t(0);
+        }
+        if (scale) {
+          const float w = static_cast<const float*>(wts.data)[t * wts.s0 + j * wts.s1];
+#pragma unroll
+          for (int r = 0; r < 8; ++r) v[r] = gt_scale(v[r], w);
+        }
       }
     }
-    tile[i][tx] = v;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) tile[i][8 * q + r] = v[r];
   }
   __syncthreads();
-  for (int i = ty; i < 64; i += 8) {
-    const int64_t c = c0 + i, p = p0 + 2 * tx;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int ci = (tid >> 3) + 32 * h, q = tid & 7;  // destination row c0 + ci, rows p 8q .. 8q + 7
+    const int64_t c = c0 + ci, p = p0 + 8 * q;
     if (c < C && p < P) {
-      const uint32_t sh = (i & 1) * 16;
-      const uint32_t lo = (tile[2 * tx][i >> 1] >> sh) & 0xffffu;
-      const uint32_t hi = (tile[2 * tx + 1][i >> 1] >> sh) & 0xffffu;
-      dst[(c * P + p) >> 1] = lo | (hi << 16);
+      uint32_t w4[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+        w4[r] = static_cast<uint32_t>(tile[8 * q + 2 * r][ci]) | (static_cast<uint32_t>(tile[8 * q + 2 * r + 1][ci]) << 16);
+      *reinterpret_cast<uint4*>(dst + c * P + p) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
     }
   }
   pdl_launch_dependents();
@@ -320,12 +337,13 @@ cudaError_t launch_gather_transpose(const View2& src, int gather, const int32_t*
                                     const View2& wts, int scale, void* dst, int64_t P, int64_t C,
                                     cudaStream_t st, int* launches) {
   if (P == 0 || C == 0) return cudaSuccess;
-  if ((C + 63) / 64 > 65535 || P % 2 != 0 || reinterpret_cast<uintptr_t>(dst) % 4 != 0)
+  if ((C + 63) / 64 > 65535 || P % 64 != 0 || reinterpret_cast<uintptr_t>(dst) % 16 != 0)
     return cudaErrorInvalidValue;
+  const int vec = src.s1 == 1 && (src.s0 * 2) % 16 == 0 && reinterpret_cast<uintptr_t>(src.data) % 16 == 0;
   if (launches) *launches += 1;
-  const dim3 grid(static_cast<unsigned>((P + 63) / 64), static_cast<unsigned>((C + 63) / 64));
-  return launch_pdl(gather_transpose_kernel, grid, dim3(256), 0, st, src, gather, sorted, S, k, wts, scale,
-                    static_cast<uint32_t*>(dst), P, C);
+  const dim3 grid(static_cast<unsigned>(P / 64), static_cast<unsigned>((C + 63) / 64));
+  return launch_pdl(gather_transpose_kernel, grid, dim3(256), 0, st, src, gather, vec, sorted, S, k, wts, scale,
+                    static_cast<uint16_t*>(dst), P, C);
 }
 
 }  // namespace moe
