@@ -55,10 +55,10 @@ WORKLOADS = {
 NCU_TRAFFIC = {
     # GEMM1 on the benchmarked workload (T=4096, E=128, the table's configuration for that
     # bucket: gate/up interleaved on 256-row pair tiles), one-pass ncu capture at the full
-    # size: 3.898 GB read + 0.105 GB written per launch; reported only while the GEMM
+    # size: 3.786 GB read + 0.105 GB written per launch; reported only while the GEMM
     # sources and the configuration hash to `src` (the hash the capturing run printed)
-    "qwen3-235b": {"T": 4096, "E": 128, "bytes_per_launch": 3.8977e9 + 0.10545e9,
-                   "src": "3f9701359ffc56cc"},
+    "qwen3-235b": {"T": 4096, "E": 128, "bytes_per_launch": 3.7860e9 + 0.10480e9,
+                   "src": "55e3e3b55bb96a1a"},
 }
 
 

@@ -1002,8 +1002,9 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   tiles.list[0].tile_rows = reinterpret_cast<int32_t*>(w + L.tile_rows);
   tiles.list[0].tile_expert = reinterpret_cast<int32_t*>(w + L.tile_expert);
   tiles.list[0].num_tiles = num_blocks + 1;
-  // the down-projection-form GEMMs (dh, y, da) on CTA pairs with one 256-row weight slice
-  // per 256-row token tile wherever the forward's table picks that form for GEMM2
+  // the GEMMs on CTA pairs over 256-row token tiles wherever the forward's table picks
+  // that form for GEMM2: dh, y and da with one 256-row weight slice per item, the gate/up
+  // recompute with 256 rows of I per item
   const bool pair2 = select_config(pr.T, pr.H, pr.I, pr.E, pr.k, false).g2_single != 0;
   if (pair2) {
     tiles.list[1].tile_max = 256;
@@ -1058,17 +1059,18 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   rc = down_form(g, mW2T, mD1);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm dh");
 
-  g = gb;  // g, u recomputed: [dg | du] and h
+  g = pair2 ? gp : gb;  // g, u recomputed: [dg | du] and h (CTA pairs: 256 rows of I per item)
   g.K = pr.H;
   g.N = pr.I;
-  g.n_wt = (pr.I + 127) / 128;
+  g.n_wt = pair2 ? (pr.I + 255) / 256 : (pr.I + 127) / 128;
   g.out = w + B.dgu;
   g.out_ld = 2 * pr.I;
   g.dh = w + B.dh;
   g.dh_ld = pr.I;
   g.h_out = w + L.h;
   g.h_ld = pr.I;
-  rc = launch_gemm_ws_bf16(3, kTile, mGate, mUp, mA1, g, dev->num_sms, st, &launches);
+  rc = pair2 ? launch_gemm_ws_pair_bf16(3, 256, mGate, mUp, mA1, g, dev->num_sms, st, &launches)
+             : launch_gemm_ws_bf16(3, kTile, mGate, mUp, mA1, g, dev->num_sms, st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm dg du");
 
   g = gp;  // y = w2 h, unweighted

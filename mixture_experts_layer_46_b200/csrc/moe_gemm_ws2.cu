@@ -75,6 +75,10 @@ struct Args {
   int32_t weights_evict_first;
   int32_t tok_box;  // token rows per TMA box (the map's box height)
   int32_t unit_w;   // modes 1/2: weight 1 for every routed slot
+  const __nv_bfloat16* dh;  // mode 3: gradient of h [P, N], row stride dh_ld
+  int64_t dh_ld;
+  __nv_bfloat16* h_out;     // mode 3: recomputed h [P, N], row stride h_ld
+  int64_t h_ld;
   DeviceErrors* err;
 };
 
@@ -103,7 +107,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmW0);
-    if (kMode == 0) tma_prefetch_desc(&tmW1);
+    if (kMode == 0 || kMode == 3) tma_prefetch_desc(&tmW1);
     tma_prefetch_desc(&tmX);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -162,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
           tma_load_3d_pair(sw0, &tmW0, fb, kb * kBK, w0, e, wpol);
           if (C::kTiles == 2)
-            tma_load_3d_pair(sw1, kMode == 0 ? &tmW1 : &tmW0, fb, kb * kBK, w1, e, wpol);
+            tma_load_3d_pair(sw1, (kMode == 0 || kMode == 3) ? &tmW1 : &tmW0, fb, kb * kBK, w1, e, wpol);
           for (int b = 0; b < nbox; ++b)
             tma_load_2d_pair(sx + b * g.tok_box * kBK * 2, &tmX, fb, kb * kBK, my_row0 + b * g.tok_box, pol);
           last_phase[stage] = static_cast<int8_t>(phase);
@@ -229,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // and routing weights while the accumulator is being built
       int32_t slot_r[kNmax / 64];
       float w_r[kNmax / 64];
-      if (kMode >= 1) {
+      if (kMode == 1 || kMode == 2) {
 #pragma unroll
         for (int i = 0; i < kNmax / 64; ++i) {
           const int c = half + 2 * i;
@@ -256,9 +260,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem_base + lane_base + c * 32, v0);
         if (C::kTiles == 2) tmem_ld32(tmem_base + lane_base + kNmax + c * 32, v1);
         float wj[32];
-        if (kMode >= 1) {
+        if (kMode == 1 || kMode == 2) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) wj[j] = __shfl_sync(0xffffffffu, w_r[i], j);
+        }
+        if (kMode == 3) {
+          // gradient of h = silu(g) u for this warp's 32 rows of I and the chunk's 32
+          // token rows: dg, du and h go out through the staging tile in turn
+          const int64_t col0 = wt * 2 * kWRows + rank * kWRows + quad * 32;
+          const bool col_ok = col0 < g.N;
+          float dhv[32];
+          const __nv_bfloat16* dsrc = g.dh + (row0 + c * 32) * g.dh_ld + col0 + lane;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) dhv[j] = col_ok ? __bfloat162float(dsrc[j * g.dh_ld]) : 0.0f;
+          tmem_wait_ld();
+#pragma unroll 1
+          for (int o = 0; o < 3; ++o) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float gg = __uint_as_float(v0[j]), uu = __uint_as_float(v1[j]);
+              const float sg = __fdividef(1.0f, 1.0f + __expf(-gg));
+              const float v = o == 0 ? dhv[j] * uu * sg * (1.0f + gg * (1.0f - sg))
+                            : o == 1 ? dhv[j] * gg * sg
+                                     : gg * sg * uu;
+              const __nv_bfloat16 vb = __float2bfloat16_rn(v);
+              asm volatile("st.shared.b16 [%0], %1;" ::"r"(stg_s + j * 64 + lane * 2),
+                           "h"(*reinterpret_cast<const uint16_t*>(&vb)) : "memory");
+            }
+            __syncwarp();
+            __nv_bfloat16* dst = o == 2 ? g.h_out : static_cast<__nv_bfloat16*>(g.out);
+            const int64_t ld = o == 2 ? g.h_ld : g.out_ld;
+            const int64_t cbase = col0 + (o == 1 ? g.N : 0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int idx = q * 32 + lane;
+              const int j = idx >> 2, part = idx & 3;
+              uint4 v;
+              asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                           : "r"(stg_s + j * 64 + part * 16));
+              if (col_ok)
+                *reinterpret_cast<uint4*>(dst + (row0 + c * 32 + j) * ld + cbase + part * 8) = v;
+            }
+            __syncwarp();
+          }
+          continue;
         }
         tmem_wait_ld();
         constexpr int kOuts = (kMode == 1) ? 2 : 1;
@@ -288,9 +334,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                          : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                          : "r"(stg_s + j * 64 + part * 16));
-            const int32_t s_j = (kMode >= 1) ? __shfl_sync(0xffffffffu, slot_r[i], j) : 0;
+            const int32_t s_j = (kMode == 1 || kMode == 2) ? __shfl_sync(0xffffffffu, slot_r[i], j) : 0;
             if (!col_ok) continue;
-            if (kMode >= 1 && s_j >= g.S) continue;
+            if ((kMode == 1 || kMode == 2) && s_j >= g.S) continue;
             const int64_t p = row0 + c * 32 + j;
             *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + p * g.out_ld + col0 + part * 8) = v;
           }
@@ -369,10 +415,16 @@ cudaError_t launch_gemm_ws_pair_bf16(int mode, int tile_max, const CUtensorMap& 
   g.weights_evict_first = p.weights_evict_first;
   g.tok_box = p.tok_box;
   g.unit_w = p.unit_w;
+  g.dh = static_cast<const __nv_bfloat16*>(p.dh);
+  g.dh_ld = p.dh_ld;
+  g.h_out = static_cast<__nv_bfloat16*>(p.h_out);
+  g.h_ld = p.h_ld;
+  if (mode == 3 && (!p.dh || !p.h_out)) return cudaErrorInvalidValue;
   if (launches) *launches += 1;
   const int64_t max_items = p.max_tiles * p.n_wt;
   if (tile_max == 256) {
     if (mode == 0) return launch_pair<0, 256>(w0, w1, x, g, max_items, num_sms, st);
+    if (mode == 3) return launch_pair<3, 256>(w0, w1, x, g, max_items, num_sms, st);
     if (mode == 2) return launch_pair<2, 256>(w0, w1, x, g, max_items, num_sms, st);
     return launch_pair<1, 256>(w0, w1, x, g, max_items, num_sms, st);
   }

@@ -167,7 +167,9 @@ cudaError_t launch_gemm_ws_bf16(int mode, int tile_max, const CUtensorMap& w0,
                                 int num_sms, cudaStream_t st, int* launches);
 
 // The same GEMMs on CTA pairs (cluster of 2, tcgen05 cta_group::2): M = 256
-// weight rows split over the pair, token tiles of up to 256 rows (tile_max 256).
+// weight rows split over the pair, token tiles of up to 256 rows (tile_max 256);
+// modes 0, 1, 3 as above (mode 3 at tile_max 256 only), mode 2: one 256-row weight
+// slice per item (GEMM2).
 cudaError_t launch_gemm_ws_pair_bf16(int mode, int tile_max, const CUtensorMap& w0,
                                      const CUtensorMap& w1, const CUtensorMap& x, const WsGemm& p,
                                      int num_sms, cudaStream_t st, int* launches);
