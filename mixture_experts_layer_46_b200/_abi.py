@@ -291,6 +291,19 @@ def backward(x, w13: MoeW13, w2, w13t, w2t, topk_ids, topk_weights, dout, dx=Non
     return dx, dweights, dw13, dw2
 
 
+def backward_status(x, w13: MoeW13, w2, w13t, w2t, topk_ids, topk_weights, dout, dx, dweights, dw13=None,
+                    dw2=None, *, workspace=None, stream=None) -> int:
+    """Like backward() but returns the raw moe_status_t (for error-path tests)."""
+    d = [desc(v) for v in (x, w2, w13t, w2t, topk_ids, topk_weights, dout, dx, dweights)]
+    g13 = ctypes.byref(desc(dw13)) if dw13 is not None else None
+    g2 = ctypes.byref(desc(dw2)) if dw2 is not None else None
+    st = _stream_ptr(stream) if torch.cuda.is_available() else None
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_n = workspace.numel() if workspace is not None else 0
+    return int(load().moe_backward_ws(ctypes.byref(d[0]), ctypes.byref(w13), *[ctypes.byref(v) for v in d[1:]],
+                                      g13, g2, ws_ptr, ws_n, st))
+
+
 def backward_input(x, w13: MoeW13, w2, w13t, w2t, topk_ids, topk_weights, dout, dx=None, dweights=None,
                    *, workspace: torch.Tensor | None = None, stream=None):
     """(dx, dweights): the forward's gradient with respect to x and the routing

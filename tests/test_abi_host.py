@@ -130,6 +130,40 @@ def test_validation_errors():
     assert _status(x, v, w2, ids, wts, out, ws) == 5
 
 
+def test_backward_validation_errors():
+    # the gradient entry point rejects bad arguments on the host, before any device work
+    x, w13, w2, ids, wts, dx = _cpu_problem(T=8, H=64, I=32, E=4, k=2)
+    v = moe.w13_from_packed(w13)
+    w13t = torch.zeros(4, 64, 64, dtype=torch.bfloat16)
+    w2t = torch.zeros(4, 32, 64, dtype=torch.bfloat16)
+    dout = torch.zeros(8, 64, dtype=torch.bfloat16)
+    dw = torch.zeros(8, 2, dtype=torch.float32)
+    ws = torch.zeros(16, dtype=torch.uint8)
+
+    def st(**kw):
+        a = dict(x=x, w13=v, w2=w2, w13t=w13t, w2t=w2t, topk_ids=ids, topk_weights=wts, dout=dout, dx=dx,
+                 dweights=dw, workspace=ws)
+        a.update(kw)
+        return moe.backward_status(**a)
+
+    assert st() == 5                                                       # workspace too small
+    assert st(w13t=torch.zeros(4, 64, 32, dtype=torch.bfloat16)) == 4     # w13t must be [E, H, 2I]
+    assert st(w2t=torch.zeros(4, 64, 32, dtype=torch.bfloat16)) == 4      # w2t must be [E, I, H]
+    assert st(w2t=torch.zeros(4, 64, 32, dtype=torch.bfloat16).transpose(1, 2)) == 4  # inner stride
+    assert st(dout=torch.zeros(8, 32, dtype=torch.bfloat16)) == 2         # dout [T, H]
+    assert st(dout=torch.zeros(8, 64, dtype=torch.float32)) == 3          # dout bf16
+    assert st(dweights=torch.zeros(8, 2, dtype=torch.bfloat16)) == 3      # dweights f32
+    assert st(dweights=torch.zeros(8, 3, dtype=torch.float32)) == 2       # dweights [T, k]
+    assert st(dx=torch.zeros(8, 64, dtype=torch.float32)) == 3            # dx bf16, like out
+    g13 = torch.zeros(4, 64, 64, dtype=torch.float32)
+    g2 = torch.zeros(4, 64, 32, dtype=torch.float32)
+    assert st(dw13=g13, dw2=g2) == 5                                       # valid weight gradients
+    assert st(dw13=g13.int(), dw2=g2) == 4                                 # f32 or bf16 only
+    assert st(dw13=g13, dw2=g2.to(torch.bfloat16)) == 4                    # bf16 rows: 64-column tiles
+    assert st(dw13=torch.zeros(4, 32, 64), dw2=g2) == 4                    # [E, 2I, H]
+    assert moe.last_launch_count() == 0
+
+
 def test_zero_tokens_is_a_noop():
     x, w13, w2, ids, wts, out = _cpu_problem(T=0)
     assert _status(x, moe.w13_from_packed(w13), w2, ids, wts, out) == 0
