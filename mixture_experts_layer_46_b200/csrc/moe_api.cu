@@ -931,12 +931,15 @@ bool kmajor_bf16(const moe_tensor_t* t, int64_t d0, int64_t d1, int64_t d2) {
 // dx = d out / d x and dweights = d out / d topk_weights contracted with dout,
 // with the routing ids fixed and the experts frozen (see moe.h):
 //   align; x and dout gathered into expert-grouped rows (A1, D1);
-//   dh[p]  = w_slot * w2_e^T dout_t        (GEMM2 kernel on w2^T [E, I, H], K = H)
-//   g, u recomputed from A1 (GEMM1 kernel, mode 3): dg, du -> [dg | du], h
-//   y[p]   = w2_e h[p]                      (GEMM2 kernel, routing weights 1)
-//   dweights[t, j] = dout_t . y[inv(t, j)]  (slot_dot)
-//   da[p]  = [gate_e^T | up_e^T] [dg | du]  (GEMM2 kernel on w13^T [E, H, 2I], K = 2I, weights 1)
+//   dh'[p] = w2_e^T dout_t                  (GEMM2 kernel on w2^T [E, I, H], K = H, weights 1)
+//   g, u recomputed from A1 (GEMM1 kernel, mode 3) with dh': dg', du' -> [dg' | du'], h
+//   dweights[t, j] = dh'[p] . h[p], p = inv(t, j)   (slot_dot on grouped rows)
+//   da[p]  = w_slot [gate_e^T | up_e^T] [dg' | du'] (GEMM2 kernel on w13^T [E, H, 2I], K = 2I)
 //   dx[t]  = sum_j da[inv(t, j)]            (combine)
+// The routing weight w_slot scales dh = w_slot dh', and dg, du are linear in dh, so it is
+// applied once, in da's epilogue (and to [dg' | du'] where the weight gradients transpose
+// them); the routing-weight gradient dout_t . (w2_e h) is the same bilinear form as
+// (w2_e^T dout_t) . h, so no separate y = w2_e h GEMM is run.
 moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const moe_tensor_t* w2,
                            const moe_tensor_t* w13t, const moe_tensor_t* w2t,
                            const moe_tensor_t* ids, const moe_tensor_t* wts,
@@ -974,7 +977,7 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   constexpr int32_t kTile = 128;
   const uint32_t boxw[3] = {64, 128, 1};
   const uint32_t boxt[2] = {64, static_cast<uint32_t>(kTile)};
-  CUtensorMap mA1, mD1, mHh, mDGU, mGate, mUp, mW2, mW2T, mW13T;
+  CUtensorMap mA1, mD1, mDGU, mGate, mUp, mW2T, mW13T;
   auto rows_map = [&](CUtensorMap* m, uint8_t* base, int64_t K) {
     const uint64_t d[2] = {uint64_t(K), uint64_t(L.p_max)};
     const uint64_t sb[1] = {uint64_t(K) * 2};
@@ -987,11 +990,9 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   };
   if ((s = rows_map(&mA1, w + L.a1, pr.H)) != MOE_OK) return s;
   if ((s = rows_map(&mD1, w + B.d1, pr.H)) != MOE_OK) return s;
-  if ((s = rows_map(&mHh, w + L.h, pr.I)) != MOE_OK) return s;
   if ((s = rows_map(&mDGU, w + B.dgu, 2 * pr.I)) != MOE_OK) return s;
   if ((s = weight_map(&mGate, gate, pr.H, pr.I)) != MOE_OK) return s;
   if ((s = weight_map(&mUp, up, pr.H, pr.I)) != MOE_OK) return s;
-  if ((s = weight_map(&mW2, w2, pr.I, pr.H)) != MOE_OK) return s;
   if ((s = weight_map(&mW2T, w2t, pr.H, pr.I)) != MOE_OK) return s;
   if ((s = weight_map(&mW13T, w13t, 2 * pr.I, pr.H)) != MOE_OK) return s;
 
@@ -1050,12 +1051,13 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
                  : launch_gemm_ws_bf16(1, kTile, wm, wm, xm, p, dev->num_sms, st, &launches);
   };
 
-  WsGemm g = gp;  // dh = w * w2^T dout
+  WsGemm g = gp;  // dh' = w2^T dout, unweighted
   g.K = pr.H;
   g.N = pr.I;
   g.n_wt = (pr.I + 255) / 256;
   g.out = w + B.dh;
   g.out_ld = pr.I;
+  g.unit_w = 1;
   rc = down_form(g, mW2T, mD1);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm dh");
 
@@ -1073,26 +1075,22 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
              : launch_gemm_ws_bf16(3, kTile, mGate, mUp, mA1, g, dev->num_sms, st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm dg du");
 
-  g = gp;  // y = w2 h, unweighted
-  g.K = pr.I;
-  g.N = pr.H;
-  g.n_wt = (pr.H + 255) / 256;
-  g.out = w + L.y;
-  g.out_ld = pr.H;
-  g.unit_w = 1;
-  rc = down_form(g, mW2, mHh);
-  if (rc != cudaSuccess) return cuda_fail(rc, "gemm y");
-  rc = launch_slot_dot(view2(dout), reinterpret_cast<const __nv_bfloat16*>(w + L.y), inv, pr.T, pr.H,
-                       pr.k, view2(dw), st, &launches);
+  View2 dh_rows;  // dh' in grouped rows [P, I]
+  dh_rows.data = w + B.dh;
+  dh_rows.s0 = pr.I;
+  dh_rows.s1 = 1;
+  dh_rows.dtype = MOE_BF16;
+  rc = launch_slot_dot(dh_rows, 1, reinterpret_cast<const __nv_bfloat16*>(w + L.h), inv, pr.T, pr.I, pr.k,
+                       view2(dw), st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "slot_dot");
 
-  g = gp;  // da = [gate^T | up^T] [dg | du]
+  g = gp;  // da = w [gate^T | up^T] [dg' | du']
   g.K = 2 * pr.I;
   g.N = pr.H;
   g.n_wt = (pr.H + 255) / 256;
   g.out = w + L.y;
   g.out_ld = pr.H;
-  g.unit_w = 1;
+  g.unit_w = 0;
   rc = down_form(g, mW13T, mDGU);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm da");
   rc = launch_combine(reinterpret_cast<const __nv_bfloat16*>(w + L.y), inv, pr.T, pr.H, pr.k,
@@ -1111,7 +1109,7 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
     dgu_rows.s1 = 1;
     dgu_rows.dtype = MOE_BF16;
     CUtensorMap mA, mB, mC;
-    const uint32_t box[2] = {64, 128};
+
     // gradient [E, M, N] stored by TMA in 32-row tiles of 128-byte rows (fp32 or bf16)
     auto cmap = [&](CUtensorMap* m, const moe_tensor_t* t, int64_t M, int64_t N) {
       const bool b16 = t->dtype == MOE_BF16;
@@ -1122,9 +1120,10 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
       return make_map(m, b16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, t->data, d,
                       sb, cbox, CU_TENSOR_MAP_SWIZZLE_128B);
     };
-    auto tmap = [&](CUtensorMap* m, uint8_t* base, int64_t rows) {
+    auto tmap = [&](CUtensorMap* m, uint8_t* base, int64_t rows, uint32_t box_rows) {
       const uint64_t d[2] = {uint64_t(P), uint64_t(rows)};
       const uint64_t sb[1] = {uint64_t(P) * 2};
+      const uint32_t box[2] = {64, box_rows};
       return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, d, sb, box, CU_TENSOR_MAP_SWIZZLE_128B);
     };
     if (dw2) {
@@ -1138,21 +1137,21 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
       if (rc == cudaSuccess)
         rc = launch_gather_transpose(h_rows, 0, sorted, L.S, pr.k, none, 0, w + B.hT, P, pr.I, st, &launches);
       if (rc != cudaSuccess) return cuda_fail(rc, "transpose dy h");
-      if ((s = tmap(&mA, w + B.dyT, pr.H)) != MOE_OK) return s;
-      if ((s = tmap(&mB, w + B.hT, pr.I)) != MOE_OK) return s;
+      if ((s = tmap(&mA, w + B.dyT, pr.H, kKgroupTileM)) != MOE_OK) return s;
+      if ((s = tmap(&mB, w + B.hT, pr.I, kKgroupTileN)) != MOE_OK) return s;
       if ((s = cmap(&mC, dw2, pr.H, pr.I)) != MOE_OK) return s;
       rc = launch_gemm_kgroup(mA, mB, mC, dw2->dtype == MOE_BF16, pr.H, pr.I, pr.E, offsets, dev->errors,
                               dev->num_sms, st, &launches);
       if (rc != cudaSuccess) return cuda_fail(rc, "gemm dw2");
     }
     if (dw13) {
-      rc = launch_gather_transpose(dgu_rows, 0, sorted, L.S, pr.k, none, 0, w + B.dguT, P, 2 * pr.I, st,
+      rc = launch_gather_transpose(dgu_rows, 0, sorted, L.S, pr.k, view2(wts), 1, w + B.dguT, P, 2 * pr.I, st,
                                    &launches);
       if (rc == cudaSuccess)
         rc = launch_gather_transpose(view2(x), 1, sorted, L.S, pr.k, none, 0, w + B.a1T, P, pr.H, st, &launches);
       if (rc != cudaSuccess) return cuda_fail(rc, "transpose dgu x");
-      if ((s = tmap(&mA, w + B.dguT, 2 * pr.I)) != MOE_OK) return s;
-      if ((s = tmap(&mB, w + B.a1T, pr.H)) != MOE_OK) return s;
+      if ((s = tmap(&mA, w + B.dguT, 2 * pr.I, kKgroupTileM)) != MOE_OK) return s;
+      if ((s = tmap(&mB, w + B.a1T, pr.H, kKgroupTileN)) != MOE_OK) return s;
       if ((s = cmap(&mC, dw13, 2 * pr.I, pr.H)) != MOE_OK) return s;
       rc = launch_gemm_kgroup(mA, mB, mC, dw13->dtype == MOE_BF16, 2 * pr.I, pr.H, pr.E, offsets, dev->errors,
                               dev->num_sms, st, &launches);

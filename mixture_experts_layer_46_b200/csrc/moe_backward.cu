@@ -3,9 +3,11 @@
 // The gradient of the forward with respect to x and the routing weights, the
 // experts frozen (the routing ids are discrete), is computed by the GEMM kernels
 // run on transposed weights plus these two steps:
-//   slot_dot:  dweights[t, j] = sum_o dout[t, o] * y[inv[t*k + j], o], where y is
-//              GEMM2 run with every routing weight 1 (the expert's output before
-//              its routing weight scales it);
+//   slot_dot:  dweights[t, j] = sum_o a[o] * y[inv[t*k + j], o], a = row t of a
+//              token-major tensor or row inv[t*k + j] of a grouped one; the gradient
+//              path takes a = dh' = w2_e^T dout_t and y = h (grouped rows, length I),
+//              the same value as dout_t . (w2_e h), the expert's output before its
+//              routing weight scales it;
 //   transpose: the expert weights with the contraction axis swapped, so that the
 //              gradient GEMMs read them K-major like the forward does: w2 [E, H, I]
 //              -> [E, I, H] (dh = w * w2^T dout) and the packed w13 [E, 2I, H] ->
@@ -20,8 +22,9 @@ constexpr int kDotWarps = 8;
 
 // one warp per routing slot: lane l sums elements [8 l + 256 m, 8 l + 256 m + 8) for m =
 // 0, 1, ... in order (16-byte loads of both rows where they are aligned), then the
-// warp adds its lanes in a fixed tree
-__global__ void __launch_bounds__(kDotWarps * 32) slot_dot_kernel(View2 dout, const __nv_bfloat16* y,
+// warp adds its lanes in a fixed tree; `grouped` picks row inv[s] of dout instead of row t
+__global__ void __launch_bounds__(kDotWarps * 32) slot_dot_kernel(View2 dout, int grouped,
+                                                                 const __nv_bfloat16* y,
                                                                  const int32_t* inv, int64_t T,
                                                                  int64_t H, int64_t k, View2 dw,
                                                                  int vec) {
@@ -33,7 +36,7 @@ __global__ void __launch_bounds__(kDotWarps * 32) slot_dot_kernel(View2 dout, co
     const int32_t row = inv[s];
     float acc = 0.0f;
     if (row >= 0) {
-      const uint16_t* d = static_cast<const uint16_t*>(dout.data) + t * dout.s0;
+      const uint16_t* d = static_cast<const uint16_t*>(dout.data) + (grouped ? row : t) * dout.s0;
       const uint16_t* yr = reinterpret_cast<const uint16_t*>(y) + static_cast<int64_t>(row) * H;
       if (vec) {
         for (int64_t o = lane * 8; o < H; o += 256) {
@@ -83,7 +86,7 @@ __global__ void __launch_bounds__(32 * 8) transpose_kernel(const uint16_t* src, 
 
 }  // namespace
 
-cudaError_t launch_slot_dot(const View2& dout, const __nv_bfloat16* y, const int32_t* inv,
+cudaError_t launch_slot_dot(const View2& dout, int grouped, const __nv_bfloat16* y, const int32_t* inv,
                             int64_t T, int64_t H, int64_t k, const View2& dw, cudaStream_t st,
                             int* launches) {
   const int64_t S = T * k;
@@ -93,7 +96,8 @@ cudaError_t launch_slot_dot(const View2& dout, const __nv_bfloat16* y, const int
                   reinterpret_cast<uintptr_t>(y) % 16 == 0;
   if (launches) *launches += 1;
   const dim3 grid(static_cast<unsigned>((S + kDotWarps - 1) / kDotWarps));
-  return launch_pdl(slot_dot_kernel, grid, dim3(kDotWarps * 32), 0, st, dout, y, inv, T, H, k, dw, vec);
+  return launch_pdl(slot_dot_kernel, grid, dim3(kDotWarps * 32), 0, st, dout, grouped, y, inv, T, H, k, dw,
+                    vec);
 }
 
 cudaError_t launch_transpose_experts(const void* src, int64_t s0, int64_t s1, void* dst, int64_t d0,

@@ -11,31 +11,38 @@
 //   [dgate; dup][e] = [dg | du]^T_e x_e       A = [dg | du]^T [2I, P], B = x^T [H, P]
 // (the gradients of out = sum_j w y with respect to w2, gate and up).
 //
-// Kernel shape: one persistent CTA per SM, 6 warps: warp 0 TMA producer (one
-// [64 x 128] box of A and of B per k-block, 128-byte swizzle), warp 1 TMEM
-// allocator and MMA issuer (M = 128, N = 128, fp32 accumulators, two buffers),
-// warps 2-5 epilogue (one row m per thread: the warp's 32-row tile of 32 fp32 or
-// 64 bf16 columns, 128 bytes a row, goes to shared memory in the 128-byte swizzled
-// layout and out with one TMA store, which also clips the M and N tails).  Work item = (expert,
-// 128-row tile of M, 128-column tile of N), expert-major; an expert with no rows
-// gets zeros.
+// Kernel shape: one persistent CTA per SM, 10 warps: warp 0 TMA producer (one
+// [64 x 128] box of A and one [64 x 256] box of B per k-block, 128-byte swizzle),
+// warp 1 TMEM allocator and MMA issuer (M = 128, N = 256, fp32 accumulators, two
+// buffers: all 512 TMEM columns), warps 2-9 epilogue, two per TMEM lane quadrant,
+// each on 128 of the tile's 256 columns (one row m per thread: the warp's 32-row
+// tile of 32 fp32 or 64 bf16 columns, 128 bytes a row, goes to shared memory in the
+// 128-byte swizzled layout and out with one TMA store, which also clips the M and N
+// tails).  With K an expert's few hundred rows, an item's MMAs take about as long as
+// draining its accumulator, so the drain is split across eight warps.  Work item = (expert,
+// 128-row tile of M, 256-column tile of N), expert-major; an expert with no rows
+// gets zeros.  The operand tiles come from L2 once per work item (each A tile is read
+// N / 256 times, each B tile M / 128 times), so the 256-column tile moves a quarter
+// fewer operand bytes per FLOP than a square 128 x 128 one.
 #include "../../include/moe.h"
 #include "moe_internal.h"
 
 namespace moe {
 namespace {
 
-constexpr int kTM = 128, kTN = 128, kBK = 64, kUmmaK = 16;
-constexpr int kStages = 6;
-constexpr int kEpiWarps = 4;
+constexpr int kTM = kKgroupTileM, kTN = kKgroupTileN, kBK = 64, kUmmaK = 16;
+constexpr int kStages = 4;
+constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant, each on half the columns
 constexpr int kThreads = 32 * (2 + kEpiWarps);
 constexpr int kTmemCols = 2 * kTN;
 constexpr int kABytes = kTM * kBK * 2;  // 16 KiB
-constexpr int kBBytes = kTN * kBK * 2;  // 16 KiB
+constexpr int kBBytes = kTN * kBK * 2;  // 32 KiB
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kStgBytes = 32 * 128;  // per epilogue warp: 32 rows x 32 fp32
 constexpr size_t kSmem = 1024 + size_t(kStages) * kStageBytes + kEpiWarps * kStgBytes +
                          (2 * kStages + 4 + 1) * 8 + 16;
+static_assert(kSmem <= 227 * 1024, "K-grouped GEMM shared memory");
+static_assert(kTmemCols <= 512, "two accumulator buffers fit the 512 TMEM columns");
 
 struct KgArgs {
   int64_t M, N, E;
@@ -166,21 +173,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quad = warp & 3;  // TMEM lanes [32 quad, 32 quad + 32) = rows m of this warp
+    const int quad = warp & 3;              // TMEM lanes [32 quad, 32 quad + 32) = rows m of this warp
+    const int half = (warp - 2) / 4;        // columns [half kTN / 2, (half + 1) kTN / 2) of the tile
     const uint32_t stg = smem_u32(staging + (warp - 2) * kStgBytes);
     uint32_t buf = 0, acc_phase = 0;
     for (int64_t item = blockIdx.x; item < total; item += gridDim.x) {
       const int64_t e = item / per_e, r = item - e * per_e;
       const int32_t m0 = static_cast<int32_t>((r / g.n_nt) * kTM + quad * 32);
-      const int32_t n0 = static_cast<int32_t>((r % g.n_nt) * kTN);
+      const int32_t n0 = static_cast<int32_t>((r % g.n_nt) * kTN + half * (kTN / 2));
       const bool empty_e = g.offsets[e + 1] == g.offsets[e];
       if (!mbar_wait(&tfull[buf], acc_phase, g.err)) break;
       tc_fence_after();
-      const uint32_t lane_base = (static_cast<uint32_t>(quad * 32) << 16) + buf * kTN;
+      const uint32_t lane_base = (static_cast<uint32_t>(quad * 32) << 16) + buf * kTN + half * (kTN / 2);
       // one staged tile row is 128 bytes: 32 fp32 or 64 bf16 columns
       constexpr int kCols = kBf16Out ? 64 : 32;
 #pragma unroll 1
-      for (int c = 0; c < kTN / kCols; ++c) {
+      for (int c = 0; c < kTN / 2 / kCols; ++c) {
         uint32_t v[32];
         if (empty_e) {
 #pragma unroll
@@ -235,64 +243,97 @@ __global__ void __launch_bounds__(kThreads, 1)
 // dst[c, p] = 0 for a padding row p (sorted[p] >= S), else scale(p) * src_row(p)[c],
 // where src_row(p) is row sorted[p] / k of a token-major tensor (gather) or row p
 // of a grouped [P, C] matrix, and scale(p) is the slot's routing weight or 1.
-// 64 x 64 tiles through shared memory, 256 threads: each thread reads 8 consecutive
-// columns of a source row (16 bytes; element loads where the rows are not 16-byte
-// aligned) and writes 8 consecutive rows p of a destination row (16 bytes).  P is a
-// multiple of 64 (the granule), dst 16-byte aligned.
+// A block moves 64 rows p by kGtTiles 64-column tiles through unpadded [p][c]
+// shared tiles, 256 threads.  Load phase: a thread resolves its two rows once, then
+// issues all its source reads (8 consecutive columns, 16 bytes, per row and tile;
+// element loads where the rows are not 16-byte aligned) before it stores any, so
+// each thread keeps 2 x kGtTiles loads in flight; a warp fills 512 contiguous bytes
+// of a tile.  Store phase: a thread owns one column c and 16 rows p of a tile; a
+// warp's 32 columns of one tile row are 16 consecutive 4-byte words (no bank
+// conflict), and each thread writes 32 contiguous bytes (one sector) of dst row c.
+// P is a multiple of 64 (the granule), dst 16-byte aligned.
+constexpr int kGtTiles = 4;
+
 __device__ __forceinline__ uint16_t gt_scale(uint16_t raw, float w) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(w * __uint_as_float(static_cast<uint32_t>(raw) << 16)));
+}
+__device__ __forceinline__ uint32_t gt_scale2(uint32_t pair, float w) {
+  return static_cast<uint32_t>(gt_scale(static_cast<uint16_t>(pair & 0xffffu), w)) |
+         (static_cast<uint32_t>(gt_scale(static_cast<uint16_t>(pair >> 16), w)) << 16);
 }
 
 __global__ void __launch_bounds__(256) gather_transpose_kernel(View2 src, int gather, int vec, const int32_t* sorted,
                                                                int64_t S, int64_t k, View2 wts, int scale,
                                                                uint16_t* dst, int64_t P, int64_t C) {
-  __shared__ uint16_t tile[64][64 + 8];  // [row p][column c]; 16 bytes of padding per row
+  __shared__ __align__(16) uint16_t tile[kGtTiles][64][64];  // [column tile][row p][column c]
   pdl_wait();
-  const int64_t p0 = static_cast<int64_t>(blockIdx.x) * 64, c0 = static_cast<int64_t>(blockIdx.y) * 64;
-  const int tid = threadIdx.x;
+  const int64_t p0 = static_cast<int64_t>(blockIdx.x) * 64, cb = static_cast<int64_t>(blockIdx.y) * (64 * kGtTiles);
+  const int tid = threadIdx.x, q = tid & 7;
+  const uint16_t* row[2];
+  float wr[2];
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const int i = (tid >> 3) + 32 * h, q = tid & 7;  // row i of the tile, 8-column chunk q
-    const int64_t p = p0 + i, c = c0 + 8 * q;
-    uint16_t v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    if (p < P) {
-      const int32_t s = sorted[p];
-      if (s >= 0 && s < S) {
-        const int64_t t = s / k, j = s - t * k;
-        const uint16_t* row = static_cast<const uint16_t*>(src.data) + (gather ? t : p) * src.s0;
+    const int64_t p = p0 + (tid >> 3) + 32 * h;
+    row[h] = nullptr;
+    wr[h] = 1.0f;
+    const int32_t s = p < P ? sorted[p] : -1;
+    if (s >= 0 && s < S) {
+      const int64_t t = s / k, j = s - t * k;
+      row[h] = static_cast<const uint16_t*>(src.data) + (gather ? t : p) * src.s0;
+      if (scale) wr[h] = static_cast<const float*>(wts.data)[t * wts.s0 + j * wts.s1];
+    }
+  }
+  uint4 u[2][kGtTiles];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+#pragma unroll
+    for (int ct = 0; ct < kGtTiles; ++ct) {
+      const int64_t c = cb + 64 * ct + 8 * q;
+      u[h][ct] = make_uint4(0u, 0u, 0u, 0u);
+      if (row[h] != nullptr && c < C) {
         if (vec && c + 8 <= C) {
-          const uint4 u = *reinterpret_cast<const uint4*>(row + c);
-          const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+          u[h][ct] = *reinterpret_cast<const uint4*>(row[h] + c);
+        } else {
+          uint32_t e4[4];
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
-            v[2 * r] = static_cast<uint16_t>(w4[r] & 0xffffu);
-            v[2 * r + 1] = static_cast<uint16_t>(w4[r] >> 16);
+            const uint32_t lo = c + 2 * r < C ? row[h][(c + 2 * r) * src.s1] : 0u;
+            const uint32_t hi = c + 2 * r + 1 < C ? row[h][(c + 2 * r + 1) * src.s1] : 0u;
+            e4[r] = lo | (hi << 16);
           }
-        } else {
-#pragma unroll
-          for (int r = 0; r < 8; ++r) v[r] = c + r < C ? row[(c + r) * src.s1] : uint16_t(0);
-        }
-        if (scale) {
-          const float w = static_cast<const float*>(wts.data)[t * wts.s0 + j * wts.s1];
-#pragma unroll
-          for (int r = 0; r < 8; ++r) v[r] = gt_scale(v[r], w);
+          u[h][ct] = make_uint4(e4[0], e4[1], e4[2], e4[3]);
         }
       }
     }
-#pragma unroll
-    for (int r = 0; r < 8; ++r) tile[i][8 * q + r] = v[r];
   }
-  __syncthreads();
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const int ci = (tid >> 3) + 32 * h, q = tid & 7;  // destination row c0 + ci, rows p 8q .. 8q + 7
-    const int64_t c = c0 + ci, p = p0 + 8 * q;
-    if (c < C && p < P) {
-      uint32_t w4[4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
-        w4[r] = static_cast<uint32_t>(tile[8 * q + 2 * r][ci]) | (static_cast<uint32_t>(tile[8 * q + 2 * r + 1][ci]) << 16);
-      *reinterpret_cast<uint4*>(dst + c * P + p) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    for (int ct = 0; ct < kGtTiles; ++ct) {
+      uint4 v = u[h][ct];
+      if (scale) {
+        v.x = gt_scale2(v.x, wr[h]);
+        v.y = gt_scale2(v.y, wr[h]);
+        v.z = gt_scale2(v.z, wr[h]);
+        v.w = gt_scale2(v.w, wr[h]);
+      }
+      *reinterpret_cast<uint4*>(&tile[ct][(tid >> 3) + 32 * h][8 * q]) = v;
+    }
+  }
+  __syncthreads();
+  const int ci = tid & 63, g = tid >> 6;  // destination rows cb + 64 ct + ci, rows p 16g .. 16g + 15
+#pragma unroll
+  for (int ct = 0; ct < kGtTiles; ++ct) {
+    const int64_t c = cb + 64 * ct + ci;
+    if (c < C) {
+      uint32_t w8[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        w8[r] = static_cast<uint32_t>(tile[ct][16 * g + 2 * r][ci]) |
+                (static_cast<uint32_t>(tile[ct][16 * g + 2 * r + 1][ci]) << 16);
+      uint4* d = reinterpret_cast<uint4*>(dst + c * P + p0 + 16 * g);
+      d[0] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+      d[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
     }
   }
   pdl_launch_dependents();
@@ -337,11 +378,12 @@ cudaError_t launch_gather_transpose(const View2& src, int gather, const int32_t*
                                     const View2& wts, int scale, void* dst, int64_t P, int64_t C,
                                     cudaStream_t st, int* launches) {
   if (P == 0 || C == 0) return cudaSuccess;
-  if ((C + 63) / 64 > 65535 || P % 64 != 0 || reinterpret_cast<uintptr_t>(dst) % 16 != 0)
+  constexpr int64_t kCols = 64 * kGtTiles;
+  if ((C + kCols - 1) / kCols > 65535 || P % 64 != 0 || reinterpret_cast<uintptr_t>(dst) % 16 != 0)
     return cudaErrorInvalidValue;
   const int vec = src.s1 == 1 && (src.s0 * 2) % 16 == 0 && reinterpret_cast<uintptr_t>(src.data) % 16 == 0;
   if (launches) *launches += 1;
-  const dim3 grid(static_cast<unsigned>(P / 64), static_cast<unsigned>((C + 63) / 64));
+  const dim3 grid(static_cast<unsigned>(P / 64), static_cast<unsigned>((C + kCols - 1) / kCols));
   return launch_pdl(gather_transpose_kernel, grid, dim3(256), 0, st, src, gather, vec, sorted, S, k, wts, scale,
                     static_cast<uint16_t*>(dst), P, C);
 }

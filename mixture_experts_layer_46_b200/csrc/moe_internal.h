@@ -99,15 +99,17 @@ cudaError_t launch_permute_quant(const View2& x, int64_t T, int64_t H, int64_t k
                                  const View2& topk_w, float* w_row, cudaStream_t st,
                                  int* launches);
 
-// routing-weight gradient: dw[t, j] = sum_o dout[t, o] * y[inv[t*k + j], o] (fp32;
-// 0 for a skipped slot); dout [T, H] bf16 strided, dw [T, k] f32 strided
-cudaError_t launch_slot_dot(const View2& dout, const __nv_bfloat16* y, const int32_t* inv,
+// routing-weight gradient: dw[t, j] = sum_o a[o] * y[inv[t*k + j], o] (fp32; 0 for a
+// skipped slot), a = row t of dout [T, H] (grouped = 0) or row inv[t*k + j] of dout
+// (grouped = 1: grouped rows [P, H]); bf16 strided rows, y [P, H] contiguous, dw [T, k] f32 strided
+cudaError_t launch_slot_dot(const View2& dout, int grouped, const __nv_bfloat16* y, const int32_t* inv,
                             int64_t T, int64_t H, int64_t k, const View2& dw, cudaStream_t st,
                             int* launches);
 
+constexpr int kKgroupTileM = 128, kKgroupTileN = 256;  // the GEMM's output tile
 // Expert-weight gradient GEMM grouped along K: C[e, m, n] = sum over expert e's
-// grouped rows p of A[m, p] B[n, p]; a / b map A [M, P] and B [N, P] bf16 ([64 x 128]
-// boxes, 128-byte swizzle); offsets [E + 1] multiples of 64; c maps C [E, M, N] (dims
+// grouped rows p of A[m, p] B[n, p]; a / b map A [M, P] and B [N, P] bf16 ([64 x
+// kKgroupTileM] and [64 x kKgroupTileN] boxes, 128-byte swizzle); offsets [E + 1] multiples of 64; c maps C [E, M, N] (dims
 // {N, M, E}, 128-byte swizzle): fp32 in [32 x 32 x 1] boxes (N % 32 == 0) or, with
 // bf16_out, bf16 in [64 x 32 x 1] boxes (N % 64 == 0)
 cudaError_t launch_gemm_kgroup(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c, int bf16_out,
