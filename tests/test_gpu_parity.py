@@ -379,6 +379,41 @@ def test_decode_weight_prefetch_matches_oracle_and_unprefetched(T, k, idt):
     assert rel_err(outs[1], ref) <= BF16_TOL
 
 
+@pytest.mark.parametrize("T,k", [(1, 8), (4, 8)])
+def test_decode_prefetch_with_ids_from_the_router_just_before(T, k):
+    # the router kernel writes the ids and weights on the same stream right before
+    # each forward; it releases its dependents at its start, so GEMM1 can issue its
+    # early weight requests while the router is still writing: the prefetch must be
+    # checked against align's tile list, and every call must match its own routing
+    H, I, E = 512, 384, 16
+    case = make_case(T, H, I, E, k, seed=T + 151)
+    gen = torch.Generator().manual_seed(T + 7)
+    logits = [torch.randn(T, E, generator=gen) for _ in range(2)]
+    refs = []
+    for lg in logits:
+        ids, wts = oracle.router_topk(lg, k)
+        refs.append(run_oracle(dict(case, ids=ids, wts=wts.float())))
+    c = to_cuda(case)
+    lg_dev = [lg.cuda() for lg in logits]
+    ids_buf = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    wts_buf = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    v = moe.w13_from_packed(c["w13"])
+    ws = torch.empty(moe.workspace_bytes(T, H, I, E, k), dtype=torch.uint8, device="cuda")
+    moe.device_errors()
+    outs = []
+    with moe.config_override((T, H, I, E, k), prefetch=1, fused=0):
+        assert moe.get_config(T, H, I, E, k)["prefetch"] == 1
+        for it in range(24):
+            moe.router_topk(lg_dev[it % 2], k, topk_ids=ids_buf, topk_weights=wts_buf)
+            outs.append(moe.forward(c["x"], v, c["w2"], ids_buf, wts_buf, workspace=ws))
+        torch.cuda.synchronize()
+    nbad, nto = moe.device_errors()
+    assert nbad == 0 and nto == 0
+    for it, o in enumerate(outs):
+        assert rel_err(o, refs[it % 2]) <= BF16_TOL, it
+        assert torch.equal(o, outs[it % 2]), it
+
+
 @pytest.mark.parametrize("T,k,idt,tile,strided", [
     (1, 8, torch.int32, None, False),      # decode
     (4, 8, torch.int64, None, False),      # 32 slots, the largest one-launch batch
