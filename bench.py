@@ -355,6 +355,9 @@ def main():
     ap.add_argument("--grad", action="store_true",
                     help="time the gradient (dx, the routing-weight and the expert-weight gradients) "
                          "instead of the forward; prints its own JSON line")
+    ap.add_argument("--grad-weights", default="bf16", choices=["bf16", "fp32", "none"],
+                    help="with --grad: the expert-weight gradients' dtype, or none for dx and the "
+                         "routing-weight gradient alone (moe_backward_input_ws)")
     ap.add_argument("--config", default=None,
                     help="override configuration flags of the timed forward, e.g. fused=1,tile=32 "
                          "(installed with moe_set_config_table for this problem only)")
@@ -541,11 +544,12 @@ def main():
 def run_grad(args, w, moe, wl, inp, v13, dev, stream, flush):
     """The full gradient (moe_backward_ws: dx, the routing-weight gradient and the
     expert-weight gradients) on the forward's workload, timed like the forward: L2
-    flushed clean before every step, CUDA events, clocks sampled.  Roofline: 18 H I
-    FLOPs per slot (three times the forward: dh, the gate/up recompute, the unweighted
-    down projection, da, dw2 and dw13) against the slower of the bf16 burst peak and
-    the HBM time of the activated experts' weights read twice (w2^T, gate/up, w2,
-    w13^T), the bf16 weight gradients written, and x, dout and dx."""
+    flushed clean before every step, CUDA events, clocks sampled.  Roofline: 16 H I
+    FLOPs per slot (dh' = w2^T dout 2, the gate/up recompute 4, da 4, dw2 2, dw13 4;
+    10 without the weight gradients) at the bf16 burst peak against the HBM time of the
+    activated experts' weights read twice (the contraction needs w2 and w13 once each
+    transposed and the gate/up recompute reads w13 again; two passes is the floor),
+    the weight gradients of all E experts written, and x, dout and dx."""
     hbm, tf_burst, _, _ = peaks()
     T, H = w["T"], w["H"]
     w13t = moe.transpose_experts(inp["w13"])
@@ -555,13 +559,16 @@ def run_grad(args, w, moe, wl, inp, v13, dev, stream, flush):
     dwt = torch.empty(T, w["k"], dtype=torch.float32, device=dev)
     gws = torch.empty(moe.backward_workspace_bytes(T, H, w["I"], w["E"], w["k"]), dtype=torch.uint8,
                       device=dev)
-    # weight gradients in the weights' own dtype (bf16), as an autograd framework keeps them
-    dw13 = torch.empty(w["E"], 2 * w["I"], H, dtype=torch.bfloat16, device=dev)
-    dw2 = torch.empty(w["E"], H, w["I"], dtype=torch.bfloat16, device=dev)
+    # weight gradients by default in the weights' own dtype (bf16), as an autograd framework
+    # keeps them; fp32, or none (dx and the routing-weight gradient alone), on request
+    gw = args.grad_weights
+    gdt = torch.float32 if gw == "fp32" else torch.bfloat16
+    dw13 = torch.empty(w["E"], 2 * w["I"], H, dtype=gdt, device=dev) if gw != "none" else None
+    dw2 = torch.empty(w["E"], H, w["I"], dtype=gdt, device=dev) if gw != "none" else None
 
     def gstep():
         moe.backward(inp["x"], v13, inp["w2"], w13t, w2t, inp["ids"], inp["wts"], dout, dx, dwt, dw13, dw2,
-                     workspace=gws, stream=stream)
+                     weights=gw != "none", workspace=gws, stream=stream)
 
     for _ in range(args.warmup):
         gstep()
@@ -581,15 +588,20 @@ def run_grad(args, w, moe, wl, inp, v13, dev, stream, flush):
     per = sorted(a.elapsed_time(b) for a, b in evs)
     ms = sum(per) / len(per)
     alg = algorithmic(w, inp["ids"])
-    flops = 3.0 * alg["flops"]
-    gbytes = (2.0 * 3.0 * w["I"] * H * 2.0 * alg["active_experts"] + 3.0 * w["I"] * H * 2.0 * w["E"] +
-              3.0 * T * H * 2)
+    flops = alg["flops"] * 16.0 / 6.0  # the forward's 6 H I per slot
+    if gw == "none":
+        flops = alg["flops"] * 10.0 / 6.0
+        gbytes = 2.0 * 3.0 * w["I"] * H * 2.0 * alg["active_experts"] + 3.0 * T * H * 2
+    else:
+        gbytes = (2.0 * 3.0 * w["I"] * H * 2.0 * alg["active_experts"] +
+                  3.0 * w["I"] * H * gdt.itemsize * w["E"] + 3.0 * T * H * 2)
     t_roof = max(flops / (tf_burst * 1e12), gbytes / (hbm * 1e9))
     print(json.dumps({
         "metric": "fused-MoE layer gradient (dx, routing weights, expert weights) tokens/s on 1 B200",
         "value": T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": args.steps,
         "warmup": args.warmup, "higher_is_better": True, "dtype": "bf16",
         "config": {"workload": workload_name(w) + " gradient", "tokens_per_gpu": T,
+                   "weight_gradients": gw,
                    "us_per_call_p10": per[len(per) // 10] * 1e3,
                    "us_per_call_p90": per[(9 * len(per)) // 10] * 1e3},
         "roofline": {"t_roof_us": t_roof * 1e6, "frac": t_roof / (ms * 1e-3), "flops": flops,

@@ -977,20 +977,22 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   constexpr int32_t kTile = 128;
   const uint32_t boxw[3] = {64, 128, 1};
   const uint32_t boxt[2] = {64, static_cast<uint32_t>(kTile)};
-  CUtensorMap mA1, mD1, mDGU, mGate, mUp, mW2T, mW13T;
-  auto rows_map = [&](CUtensorMap* m, uint8_t* base, int64_t K) {
+  const uint32_t boxt64[2] = {64, 64};  // half of a 128-row tile: one CTA of a pair
+  CUtensorMap mA1, mA1h, mD1, mDGU, mGate, mUp, mW2T, mW13T;
+  auto rows_map = [&](CUtensorMap* m, uint8_t* base, int64_t K, const uint32_t* box) {
     const uint64_t d[2] = {uint64_t(K), uint64_t(L.p_max)};
     const uint64_t sb[1] = {uint64_t(K) * 2};
-    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, d, sb, boxt, CU_TENSOR_MAP_SWIZZLE_128B);
+    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, d, sb, box, CU_TENSOR_MAP_SWIZZLE_128B);
   };
   auto weight_map = [&](CUtensorMap* m, const moe_tensor_t* t, int64_t K, int64_t N) {
     const uint64_t d[3] = {uint64_t(K), uint64_t(N), uint64_t(pr.E)};
     const uint64_t sb[2] = {uint64_t(t->strides[1]) * 2, uint64_t(t->strides[0]) * 2};
     return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, t->data, d, sb, boxw, CU_TENSOR_MAP_SWIZZLE_128B);
   };
-  if ((s = rows_map(&mA1, w + L.a1, pr.H)) != MOE_OK) return s;
-  if ((s = rows_map(&mD1, w + B.d1, pr.H)) != MOE_OK) return s;
-  if ((s = rows_map(&mDGU, w + B.dgu, 2 * pr.I)) != MOE_OK) return s;
+  if ((s = rows_map(&mA1, w + L.a1, pr.H, boxt)) != MOE_OK) return s;
+  if ((s = rows_map(&mA1h, w + L.a1, pr.H, boxt64)) != MOE_OK) return s;
+  if ((s = rows_map(&mD1, w + B.d1, pr.H, boxt)) != MOE_OK) return s;
+  if ((s = rows_map(&mDGU, w + B.dgu, 2 * pr.I, boxt)) != MOE_OK) return s;
   if ((s = weight_map(&mGate, gate, pr.H, pr.I)) != MOE_OK) return s;
   if ((s = weight_map(&mUp, up, pr.H, pr.I)) != MOE_OK) return s;
   if ((s = weight_map(&mW2T, w2t, pr.H, pr.I)) != MOE_OK) return s;
@@ -1061,7 +1063,11 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   rc = down_form(g, mW2T, mD1);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm dh");
 
-  g = pair2 ? gp : gb;  // g, u recomputed: [dg | du] and h (CTA pairs: 256 rows of I per item)
+  // g, u recomputed: [dg' | du'] and h.  CTA pairs take align's 128-row tiles (64 token rows
+  // per CTA) and 256 rows of I per item: gate and up accumulators of 128 columns each leave
+  // room for a second TMEM buffer, so the SwiGLU-gradient epilogue overlaps the next item
+  g = gb;
+  if (pair2) g.tok_box = 64;
   g.K = pr.H;
   g.N = pr.I;
   g.n_wt = pair2 ? (pr.I + 255) / 256 : (pr.I + 127) / 128;
@@ -1071,7 +1077,7 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   g.dh_ld = pr.I;
   g.h_out = w + L.h;
   g.h_ld = pr.I;
-  rc = pair2 ? launch_gemm_ws_pair_bf16(3, 256, mGate, mUp, mA1, g, dev->num_sms, st, &launches)
+  rc = pair2 ? launch_gemm_ws_pair_bf16(3, 128, mGate, mUp, mA1h, g, dev->num_sms, st, &launches)
              : launch_gemm_ws_bf16(3, kTile, mGate, mUp, mA1, g, dev->num_sms, st, &launches);
   if (rc != cudaSuccess) return cuda_fail(rc, "gemm dg du");
 

@@ -424,12 +424,12 @@ cudaError_t launch_gemm_ws_pair_bf16(int mode, int tile_max, const CUtensorMap& 
   const int64_t max_items = p.max_tiles * p.n_wt;
   if (tile_max == 256) {
     if (mode == 0) return launch_pair<0, 256>(w0, w1, x, g, max_items, num_sms, st);
-    if (mode == 3) return launch_pair<3, 256>(w0, w1, x, g, max_items, num_sms, st);
     if (mode == 2) return launch_pair<2, 256>(w0, w1, x, g, max_items, num_sms, st);
     return launch_pair<1, 256>(w0, w1, x, g, max_items, num_sms, st);
   }
   if (tile_max == 128) {
     if (mode == 0) return launch_pair<0, 128>(w0, w1, x, g, max_items, num_sms, st);
+    if (mode == 3) return launch_pair<3, 128>(w0, w1, x, g, max_items, num_sms, st);
     if (mode == 2) return launch_pair<2, 128>(w0, w1, x, g, max_items, num_sms, st);
     return launch_pair<1, 128>(w0, w1, x, g, max_items, num_sms, st);
   }

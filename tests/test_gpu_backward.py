@@ -86,19 +86,31 @@ def test_backward_matches_oracle(T, H, I, E, k):
     (300, 288, 96, 2, 2),      # ragged K and output columns on CTA pairs
 ])
 def test_backward_pair_route_matches_one_cta_route(T, H, I, E, k):
-    # dh, y and da run on CTA pairs (one 256-row weight slice per 256-row token tile)
+    # dh' and da run on CTA pairs (one 256-row weight slice per 256-row token tile)
     # where the configuration picks that GEMM2 form, on one CTA otherwise: same bits
     case = make_case(T, H, I, E, k, seed=T + 41)
     ref_dx, ref_dw = oracle_backward(case)
     c = {n: v.cuda() for n, v in case.items()}
     with moe.config_override((T, H, I, E, k), tile=128, pair=0, g2_single=0):
         one = gpu_backward(c)
+        one_w = gpu_backward_weights(c)
     with moe.config_override((T, H, I, E, k), tile=128, pair=1, g2_single=1):
         assert moe.get_config(T, H, I, E, k)["g2_single"] == 1
         pair = gpu_backward(c)
+        pair_w = gpu_backward_weights(c)
     assert torch.equal(one[0], pair[0]) and torch.equal(one[1], pair[1])
     assert rel_err(pair[0], ref_dx) <= BWD_TOL
     assert rel_err(pair[1], ref_dw) <= BWD_TOL
+    # the weight gradients take h and [dg' | du'] from the route's recompute: the same
+    # bits either way
+    for a, b in zip(one_w, pair_w):
+        assert torch.equal(a, b)
+    gate, up = wl.gate_up_views(case["w13"])
+    ref_dg, ref_du, ref_dw2 = oracle.moe_backward_weights(case["x"], gate, up, case["w2"], case["ids"],
+                                                          case["wts"], case["dout"])
+    assert rel_err(pair_w[2][:, :I], ref_dg) <= BWD_TOL
+    assert rel_err(pair_w[2][:, I:], ref_du) <= BWD_TOL
+    assert rel_err(pair_w[3], ref_dw2) <= BWD_TOL
 
 
 def test_backward_is_deterministic_and_reads_strided_views():
