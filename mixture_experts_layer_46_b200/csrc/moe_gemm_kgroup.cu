@@ -11,15 +11,14 @@
 //   [dgate; dup][e] = [dg | du]^T_e x_e       A = [dg | du]^T [2I, P], B = x^T [H, P]
 // (the gradients of out = sum_j w y with respect to w2, gate and up).
 //
-// Kernel shape: one persistent CTA per SM, 10 warps: warp 0 TMA producer (one
+// Kernel shape: one persistent CTA per SM, 6 warps: warp 0 TMA producer (one
 // [64 x 128] box of A and one [64 x 256] box of B per k-block, 128-byte swizzle),
 // warp 1 TMEM allocator and MMA issuer (M = 128, N = 256, fp32 accumulators, two
-// buffers: all 512 TMEM columns), warps 2-9 epilogue, two per TMEM lane quadrant,
-// each on 128 of the tile's 256 columns (one row m per thread: the warp's 32-row
-// tile of 32 fp32 or 64 bf16 columns, 128 bytes a row, goes to shared memory in the
-// 128-byte swizzled layout and out with one TMA store, which also clips the M and N
-// tails).  With K an expert's few hundred rows, an item's MMAs take about as long as
-// draining its accumulator, so the drain is split across eight warps.  Work item = (expert,
+// buffers: all 512 TMEM columns), warps 2-5 epilogue, one per TMEM lane quadrant
+// (one row m per thread: the warp's 32-row tile of 32 fp32 or 64 bf16 columns, 128
+// bytes a row, goes to shared memory in the 128-byte swizzled layout and out with one
+// TMA store, which also clips the M and N tails; two staging tiles per warp, so a
+// tile is filled while the previous one's store is still reading).  Work item = (expert,
 // 128-row tile of M, 256-column tile of N), expert-major; an expert with no rows
 // gets zeros.  The operand tiles come from L2 once per work item (each A tile is read
 // N / 256 times, each B tile M / 128 times), so the 256-column tile moves a quarter
@@ -32,14 +31,14 @@ namespace {
 
 constexpr int kTM = kKgroupTileM, kTN = kKgroupTileN, kBK = 64, kUmmaK = 16;
 constexpr int kStages = 4;
-constexpr int kEpiWarps = 8;  // two per TMEM lane quadrant, each on half the columns
+constexpr int kEpiWarps = 4;  // one per TMEM lane quadrant
 constexpr int kThreads = 32 * (2 + kEpiWarps);
 constexpr int kTmemCols = 2 * kTN;
 constexpr int kABytes = kTM * kBK * 2;  // 16 KiB
 constexpr int kBBytes = kTN * kBK * 2;  // 32 KiB
 constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kStgBytes = 32 * 128;  // per epilogue warp: 32 rows x 32 fp32
-constexpr size_t kSmem = 1024 + size_t(kStages) * kStageBytes + kEpiWarps * kStgBytes +
+constexpr int kStgBytes = 32 * 128;  // one staging tile: 32 rows x 32 fp32 (two per epilogue warp)
+constexpr size_t kSmem = 1024 + size_t(kStages) * kStageBytes + 2 * kEpiWarps * kStgBytes +
                          (2 * kStages + 4 + 1) * 8 + 16;
 static_assert(kSmem <= 227 * 1024, "K-grouped GEMM shared memory");
 static_assert(kTmemCols <= 512, "two accumulator buffers fit the 512 TMEM columns");
@@ -60,8 +59,8 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t sr
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read_all() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+__device__ __forceinline__ void bulk_wait_read_1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
@@ -73,7 +72,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = base;
   uint8_t* staging = stages + kStages * kStageBytes;  // 1024-byte aligned: the swizzle atom
-  uint64_t* full = reinterpret_cast<uint64_t*>(staging + kEpiWarps * kStgBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(staging + 2 * kEpiWarps * kStgBytes);
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
@@ -173,22 +172,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quad = warp & 3;              // TMEM lanes [32 quad, 32 quad + 32) = rows m of this warp
-    const int half = (warp - 2) / 4;        // columns [half kTN / 2, (half + 1) kTN / 2) of the tile
-    const uint32_t stg = smem_u32(staging + (warp - 2) * kStgBytes);
-    uint32_t buf = 0, acc_phase = 0;
+    const int quad = warp & 3;  // TMEM lanes [32 quad, 32 quad + 32) = rows m of this warp
+    const uint32_t stg = smem_u32(staging + (warp - 2) * 2 * kStgBytes);
+    uint32_t buf = 0, acc_phase = 0, nstore = 0;
     for (int64_t item = blockIdx.x; item < total; item += gridDim.x) {
       const int64_t e = item / per_e, r = item - e * per_e;
       const int32_t m0 = static_cast<int32_t>((r / g.n_nt) * kTM + quad * 32);
-      const int32_t n0 = static_cast<int32_t>((r % g.n_nt) * kTN + half * (kTN / 2));
+      const int32_t n0 = static_cast<int32_t>((r % g.n_nt) * kTN);
       const bool empty_e = g.offsets[e + 1] == g.offsets[e];
       if (!mbar_wait(&tfull[buf], acc_phase, g.err)) break;
       tc_fence_after();
-      const uint32_t lane_base = (static_cast<uint32_t>(quad * 32) << 16) + buf * kTN + half * (kTN / 2);
+      const uint32_t lane_base = (static_cast<uint32_t>(quad * 32) << 16) + buf * kTN;
       // one staged tile row is 128 bytes: 32 fp32 or 64 bf16 columns
       constexpr int kCols = kBf16Out ? 64 : 32;
 #pragma unroll 1
-      for (int c = 0; c < kTN / 2 / kCols; ++c) {
+      for (int c = 0; c < kTN / kCols; ++c) {
         uint32_t v[32];
         if (empty_e) {
 #pragma unroll
@@ -208,18 +206,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
         }
         if (m0 < g.M && n0 + c * kCols < g.N) {
-          if (lane == 0) bulk_wait_read_all();  // the previous tile store has read the staging
+          // two staging tiles in turn: the store issued two tiles ago (the last one to use
+          // this tile) has read it, while the previous one may still be in flight
+          const uint32_t sb = stg + (nstore & 1u) * kStgBytes;
+          ++nstore;
+          if (lane == 0) bulk_wait_read_1();
           __syncwarp();
           // row `lane` of the tile: 16-byte chunk q at position q ^ (row % 8) (128-byte swizzle)
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(stg + lane * 128 + ((q ^ (lane & 7)) * 16)),
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sb + lane * 128 + ((q ^ (lane & 7)) * 16)),
                          "r"(v[4 * q]), "r"(v[4 * q + 1]), "r"(v[4 * q + 2]), "r"(v[4 * q + 3])
                          : "memory");
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_3d(&tmC, stg, n0 + c * kCols, m0, static_cast<int32_t>(e));
+            tma_store_3d(&tmC, sb, n0 + c * kCols, m0, static_cast<int32_t>(e));
             bulk_commit();
           }
         }
