@@ -55,10 +55,10 @@ WORKLOADS = {
 NCU_TRAFFIC = {
     # GEMM1 on the benchmarked workload (T=4096, E=128, the table's configuration for that
     # bucket: gate/up interleaved on 256-row pair tiles), one-pass ncu capture at the full
-    # size: 3.786 GB read + 0.105 GB written per launch; reported only while the GEMM
+    # size: 3.805 GB read + 0.107 GB written per launch; reported only while the GEMM
     # sources and the configuration hash to `src` (the hash the capturing run printed)
-    "qwen3-235b": {"T": 4096, "E": 128, "bytes_per_launch": 3.7860e9 + 0.10480e9,
-                   "src": "55e3e3b55bb96a1a"},
+    "qwen3-235b": {"T": 4096, "E": 128, "bytes_per_launch": 3.8048e9 + 0.10703e9,
+                   "src": "dc8721d8a820bb53"},
 }
 
 
@@ -547,9 +547,9 @@ def run_grad(args, w, moe, wl, inp, v13, dev, stream, flush):
     flushed clean before every step, CUDA events, clocks sampled.  Roofline: 16 H I
     FLOPs per slot (dh' = w2^T dout 2, the gate/up recompute 4, da 4, dw2 2, dw13 4;
     10 without the weight gradients) at the bf16 burst peak against the HBM time of the
-    activated experts' weights read twice (the contraction needs w2 and w13 once each
-    transposed and the gate/up recompute reads w13 again; two passes is the floor),
-    the weight gradients of all E experts written, and x, dout and dx."""
+    activated experts' weights as the path must read them (w2 once, for dh'; w13 twice,
+    for the gate/up recompute and for da: 5 I H bf16 values per expert, five thirds of
+    the weights), the weight gradients of all E experts written, and x, dout and dx."""
     hbm, tf_burst, _, _ = peaks()
     T, H = w["T"], w["H"]
     w13t = moe.transpose_experts(inp["w13"])
@@ -589,12 +589,12 @@ def run_grad(args, w, moe, wl, inp, v13, dev, stream, flush):
     ms = sum(per) / len(per)
     alg = algorithmic(w, inp["ids"])
     flops = alg["flops"] * 16.0 / 6.0  # the forward's 6 H I per slot
+    wread = 5.0 * w["I"] * H * 2.0 * alg["active_experts"]
     if gw == "none":
         flops = alg["flops"] * 10.0 / 6.0
-        gbytes = 2.0 * 3.0 * w["I"] * H * 2.0 * alg["active_experts"] + 3.0 * T * H * 2
+        gbytes = wread + 3.0 * T * H * 2
     else:
-        gbytes = (2.0 * 3.0 * w["I"] * H * 2.0 * alg["active_experts"] +
-                  3.0 * w["I"] * H * gdt.itemsize * w["E"] + 3.0 * T * H * 2)
+        gbytes = wread + 3.0 * w["I"] * H * gdt.itemsize * w["E"] + 3.0 * T * H * 2
     t_roof = max(flops / (tf_burst * 1e12), gbytes / (hbm * 1e9))
     print(json.dumps({
         "metric": "fused-MoE layer gradient (dx, routing weights, expert weights) tokens/s on 1 B200",
