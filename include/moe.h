@@ -166,6 +166,8 @@ moe_status_t moe_forward_host(const moe_tensor_t* x_host, const moe_w13_t* w13,
  *   dweights[t, j] = dout_t . (w2_e h),  h = silu(gate_e x_t) * (up_e x_t)
  *   dh = w w2_e^T dout_t;  dg = dh u s (1 + g (1 - s)),  du = dh g s  (s = sigmoid(g))
  *   dx_t += gate_e^T dg + up_e^T du
+ * (computed as dh' = w2_e^T dout_t once: dweights = dh' . h, the routing weight w
+ * applied where da = w [gate_e^T | up_e^T] [dg' | du'] leaves its GEMM).
  * Skipped slots (ids outside [0, E)) contribute nothing and get dweights 0.
  * The GEMMs read the weights K-major, so the caller passes their transposes too:
  * w13t [E, H, 2I] (the packed w13 [E, 2I, H] transposed: gate^T in columns
