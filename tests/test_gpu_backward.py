@@ -215,6 +215,24 @@ def test_weight_gradients_into_strided_outputs_are_deterministic():
     assert (big2[:, :, :8] == 7.0).all() and (big13[:, :2] == 7.0).all()  # nothing written outside
 
 
+def test_weight_gradients_read_strided_x_and_dout():
+    # x column-major and dout every other column of a wider buffer: the gather-transposes
+    # take their element-load path for both, and every result keeps the contiguous bits
+    T, H, I, E, k = 150, 256, 128, 8, 4
+    case = make_case(T, H, I, E, k, seed=67)
+    c = {n: v.cuda() for n, v in case.items()}
+    ref = gpu_backward_weights(c, grad_dtype=torch.bfloat16)
+    s = dict(c)
+    s["x"] = case["x"].t().contiguous().cuda().t()
+    assert s["x"].stride() == (1, T)
+    wide = torch.zeros(T, 2 * H, dtype=torch.bfloat16, device="cuda")
+    wide[:, ::2] = c["dout"]
+    s["dout"] = wide[:, ::2]
+    got = gpu_backward_weights(s, grad_dtype=torch.bfloat16)
+    for a, b in zip(ref, got):
+        assert torch.equal(a, b)
+
+
 @pytest.mark.slow
 def test_weight_gradients_at_qwen3_expert_dimensions():
     # the Qwen3-235B expert shape (H=4096, I=1536) with 8 experts, so the fp64 oracle's
