@@ -155,6 +155,28 @@ moe_status_t moe_forward_host(const moe_tensor_t* x_host, const moe_w13_t* w13,
                               const moe_tensor_t* topk_weights_host, moe_tensor_t* out_host,
                               moe_stream_t stream);
 
+/* Device bytes moe_forward_host_ws needs for (T, H, I, E, k, weight dtype): the
+ * forward's workspace plus staging for x, the ids (room for int64), the routing
+ * weights and out.  Returns 0 for invalid arguments. */
+size_t moe_host_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, int32_t wdtype);
+
+/* moe_forward_host without the wait: enqueues on `stream` the copies of x, topk_ids and
+ * topk_weights (HOST tensors, inner stride 1) into `workspace` (device, at least
+ * moe_host_workspace_bytes(...), 256-byte aligned), the forward, and the copy of the
+ * result into out_host, then returns.  out_host holds the result once `stream` has
+ * reached that point (synchronise the stream or an event recorded after the call), and
+ * the host inputs must stay unchanged until then.  With pinned host memory the copies
+ * are asynchronous, so calls on different streams with different workspaces can be in
+ * flight together and one call's copies overlap another call's kernels.  Two calls of
+ * at most 32 routing slots each should not overlap: the configuration table may pick
+ * the one-kernel decode for them, whose thread blocks wait on one another and need the
+ * GPU to themselves.  No allocation, no synchronisation.  Errors as for moe_forward_ws;
+ * a workspace below the size is MOE_ERR_WORKSPACE_TOO_SMALL. */
+moe_status_t moe_forward_host_ws(const moe_tensor_t* x_host, const moe_w13_t* w13, const moe_tensor_t* w2,
+                                 const moe_tensor_t* topk_ids_host, const moe_tensor_t* topk_weights_host,
+                                 moe_tensor_t* out_host, void* workspace, size_t workspace_bytes,
+                                 moe_stream_t stream);
+
 /* Gradient path (bf16 weights): given dout = dL/dout
  * [T, H] bf16, writes dx = dL/dx [T, H] bf16 and dweights = dL/dtopk_weights
  * [T, k] f32 (any strides), the routing ids held fixed (they are discrete).

@@ -12,4 +12,4 @@ from ._abi import (MoeConfig, MoeError, MoeTensor, MoeW13, align, builtin_config
                    quantize_mxfp4, router_status, router_topk, set_config_table, version, w13_from_packed, w13_from_views,
                    workspace_bytes, workspace_layout, debug_capture, MOE_CAPTURE_H_PREQUANT,
                    measure_mma_peak, backward, backward_input, backward_status, backward_workspace_bytes,
-                   transpose_experts)
+                   transpose_experts, host_workspace_bytes)

@@ -31,7 +31,8 @@ EXPORTS = ("moe_status_string", "moe_last_cuda_error", "moe_w13_from_packed",
            "moe_set_config_table", "moe_get_config", "moe_builtin_config_count",
            "moe_router_topk", "moe_selftest_bounded_wait", "moe_workspace_layout",
            "moe_debug_capture", "moe_measure_mma_peak", "moe_backward_workspace_bytes",
-           "moe_backward_input_ws", "moe_backward_ws", "moe_transpose_experts")
+           "moe_backward_input_ws", "moe_backward_ws", "moe_transpose_experts",
+           "moe_host_workspace_bytes", "moe_forward_host_ws")
 STEP_NAMES = ("align", "permute", "gemm1_swiglu", "gemm2_weighted", "combine")
 
 
@@ -113,6 +114,10 @@ def load() -> ctypes.CDLL:
                                         P(MoeTensor), P(MoeTensor), vp]
             lib.moe_forward_host.restype = ctypes.c_int
             lib.moe_forward_host.argtypes = lib.moe_forward.argtypes
+            lib.moe_host_workspace_bytes.restype = ctypes.c_size_t
+            lib.moe_host_workspace_bytes.argtypes = [ctypes.c_int64] * 5 + [ctypes.c_int32]
+            lib.moe_forward_host_ws.restype = ctypes.c_int
+            lib.moe_forward_host_ws.argtypes = lib.moe_forward_ws.argtypes
             lib.moe_backward_workspace_bytes.restype = ctypes.c_size_t
             lib.moe_backward_workspace_bytes.argtypes = [ctypes.c_int64] * 5
             lib.moe_backward_input_ws.restype = ctypes.c_int
@@ -338,15 +343,28 @@ def forward_status(x, w13: MoeW13, w2, topk_ids, topk_weights, out, *, w2_scale=
                                   ws_n, st))
 
 
+def host_workspace_bytes(T: int, H: int, I: int, E: int, k: int, mxfp4: bool = False) -> int:
+    return int(load().moe_host_workspace_bytes(T, H, I, E, k, MOE_E2M1X2 if mxfp4 else MOE_BF16))
+
+
 def forward_host(x_host, w13: MoeW13, w2, ids_host, weights_host, out_host, *, w2_scale=None,
-                 stream=None) -> torch.Tensor:
-    """Host activations in, host result out (copies and a stream sync inside)."""
+                 workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Host activations in, host result out.  Without `workspace`: moe_forward_host
+    (library staging, the stream synchronised before it returns).  With a device
+    `workspace` of host_workspace_bytes(...): moe_forward_host_ws, which only enqueues
+    the copies and the forward on `stream`; out_host is ready once the stream is."""
     dx, dw2, di, dw, do = (desc(x_host), desc(w2, w2_scale), desc(ids_host), desc(weights_host),
                            desc(out_host))
-    rc = load().moe_forward_host(ctypes.byref(dx), ctypes.byref(w13), ctypes.byref(dw2),
-                                 ctypes.byref(di), ctypes.byref(dw), ctypes.byref(do),
-                                 _stream_ptr(stream))
-    _check(rc, "moe_forward_host")
+    if workspace is None:
+        rc = load().moe_forward_host(ctypes.byref(dx), ctypes.byref(w13), ctypes.byref(dw2),
+                                     ctypes.byref(di), ctypes.byref(dw), ctypes.byref(do),
+                                     _stream_ptr(stream))
+        _check(rc, "moe_forward_host")
+        return out_host
+    rc = load().moe_forward_host_ws(ctypes.byref(dx), ctypes.byref(w13), ctypes.byref(dw2),
+                                    ctypes.byref(di), ctypes.byref(dw), ctypes.byref(do),
+                                    workspace.data_ptr(), workspace.numel(), _stream_ptr(stream))
+    _check(rc, "moe_forward_host_ws")
     return out_host
 
 

@@ -1168,6 +1168,57 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
   return MOE_OK;
 }
 
+// device staging of the host-buffer forms: the forward's own workspace, then x, the ids
+// (8 bytes per id, so int32 and int64 ids share one layout), the routing weights and out
+struct HostLayout {
+  size_t core, x_off, ids_off, w_off, o_off, total;
+};
+HostLayout host_layout(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, int32_t wdtype) {
+  HostLayout hl;
+  hl.core = moe_workspace_bytes(T, H, I, E, k, wdtype);
+  hl.x_off = align256(hl.core);
+  hl.ids_off = align256(hl.x_off + size_t(T) * H * 2);
+  hl.w_off = align256(hl.ids_off + size_t(T) * k * 8);
+  hl.o_off = align256(hl.w_off + size_t(T) * k * 4);
+  hl.total = align256(hl.o_off + size_t(T) * H * 2);
+  return hl;
+}
+
+// H2D copies of x, ids and weights, the forward on the staged copies, D2H of out: all
+// enqueued on `st`, nothing waited for
+moe_status_t forward_host_enqueue(const moe_tensor_t* x_host, const moe_w13_t* w13, const moe_tensor_t* w2,
+                                  const moe_tensor_t* topk_ids_host, const moe_tensor_t* topk_weights_host,
+                                  moe_tensor_t* out_host, const Problem& pr, const HostLayout& hl, uint8_t* w,
+                                  cudaStream_t st) {
+  const int64_t idsz = dtype_size(topk_ids_host->dtype);
+  MOE_CUDA(cudaMemcpy2DAsync(w + hl.x_off, pr.H * 2, x_host->data, x_host->strides[0] * 2, pr.H * 2,
+                             pr.T, cudaMemcpyHostToDevice, st));
+  MOE_CUDA(cudaMemcpy2DAsync(w + hl.ids_off, pr.k * idsz, topk_ids_host->data,
+                             topk_ids_host->strides[0] * idsz, pr.k * idsz, pr.T,
+                             cudaMemcpyHostToDevice, st));
+  MOE_CUDA(cudaMemcpy2DAsync(w + hl.w_off, pr.k * 4, topk_weights_host->data,
+                             topk_weights_host->strides[0] * 4, pr.k * 4, pr.T,
+                             cudaMemcpyHostToDevice, st));
+  moe_tensor_t xd = *x_host, idd = *topk_ids_host, wd = *topk_weights_host, od = *out_host;
+  xd.data = w + hl.x_off;
+  xd.strides[0] = pr.H;
+  xd.strides[1] = 1;
+  idd.data = w + hl.ids_off;
+  idd.strides[0] = pr.k;
+  idd.strides[1] = 1;
+  wd.data = w + hl.w_off;
+  wd.strides[0] = pr.k;
+  wd.strides[1] = 1;
+  od.data = w + hl.o_off;
+  od.strides[0] = pr.H;
+  od.strides[1] = 1;
+  moe_status_t s = forward_impl(&xd, w13, w2, &idd, &wd, &od, pr, w, hl.core, st);
+  if (s != MOE_OK) return s;
+  MOE_CUDA(cudaMemcpy2DAsync(out_host->data, out_host->strides[0] * 2, w + hl.o_off, pr.H * 2,
+                             pr.H * 2, pr.T, cudaMemcpyDeviceToHost, st));
+  return MOE_OK;
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -1340,47 +1391,39 @@ moe_status_t moe_forward_host(const moe_tensor_t* x_host, const moe_w13_t* w13,
   if (s != MOE_OK) return s;
   if (pr.T == 0) return MOE_OK;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  // device staging for the activations after the forward's own workspace
-  const size_t core = moe_workspace_bytes(pr.T, pr.H, pr.I, pr.E, pr.k, w13->gate.dtype);
-  const int64_t idsz = dtype_size(topk_ids_host->dtype);
-  const size_t x_off = align256(core);
-  const size_t ids_off = align256(x_off + size_t(pr.T) * pr.H * 2);
-  const size_t w_off = align256(ids_off + size_t(pr.T) * pr.k * idsz);
-  const size_t o_off = align256(w_off + size_t(pr.T) * pr.k * 4);
-  const size_t need = align256(o_off + size_t(pr.T) * pr.H * 2);
+  const HostLayout hl = host_layout(pr.T, pr.H, pr.I, pr.E, pr.k, w13->gate.dtype);
   void* ws = nullptr;
-  s = cached_workspace(need, &ws);
+  s = cached_workspace(hl.total, &ws);
   if (s != MOE_OK) return s;
-  uint8_t* w = static_cast<uint8_t*>(ws);
-  MOE_CUDA(cudaMemcpy2DAsync(w + x_off, pr.H * 2, x_host->data, x_host->strides[0] * 2, pr.H * 2,
-                             pr.T, cudaMemcpyHostToDevice, st));
-  MOE_CUDA(cudaMemcpy2DAsync(w + ids_off, pr.k * idsz, topk_ids_host->data,
-                             topk_ids_host->strides[0] * idsz, pr.k * idsz, pr.T,
-                             cudaMemcpyHostToDevice, st));
-  MOE_CUDA(cudaMemcpy2DAsync(w + w_off, pr.k * 4, topk_weights_host->data,
-                             topk_weights_host->strides[0] * 4, pr.k * 4, pr.T,
-                             cudaMemcpyHostToDevice, st));
-  moe_tensor_t xd = *x_host, idd = *topk_ids_host, wd = *topk_weights_host, od = *out_host;
-  xd.data = w + x_off;
-  xd.strides[0] = pr.H;
-  xd.strides[1] = 1;
-  idd.data = w + ids_off;
-  idd.strides[0] = pr.k;
-  idd.strides[1] = 1;
-  wd.data = w + w_off;
-  wd.strides[0] = pr.k;
-  wd.strides[1] = 1;
-  od.data = w + o_off;
-  od.strides[0] = pr.H;
-  od.strides[1] = 1;
-  s = forward_impl(&xd, w13, w2, &idd, &wd, &od, pr, ws, core, st);
+  s = forward_host_enqueue(x_host, w13, w2, topk_ids_host, topk_weights_host, out_host, pr, hl,
+                           static_cast<uint8_t*>(ws), st);
   if (s != MOE_OK) return s;
   const int32_t fwd_launches = t_last_launches;
-  MOE_CUDA(cudaMemcpy2DAsync(out_host->data, out_host->strides[0] * 2, w + o_off, pr.H * 2,
-                             pr.H * 2, pr.T, cudaMemcpyDeviceToHost, st));
   MOE_CUDA(cudaStreamSynchronize(st));
   t_last_launches = fwd_launches;
   return MOE_OK;
+}
+
+size_t moe_host_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, int32_t wdtype) {
+  if (moe_workspace_bytes(T, H, I, E, k, wdtype) == 0) return 0;
+  return host_layout(T, H, I, E, k, wdtype).total;
+}
+
+moe_status_t moe_forward_host_ws(const moe_tensor_t* x_host, const moe_w13_t* w13, const moe_tensor_t* w2,
+                                 const moe_tensor_t* topk_ids_host, const moe_tensor_t* topk_weights_host,
+                                 moe_tensor_t* out_host, void* workspace, size_t workspace_bytes,
+                                 moe_stream_t stream) {
+  t_last_launches = 0;
+  Problem pr;
+  moe_status_t s =
+      validate(x_host, w13, w2, topk_ids_host, topk_weights_host, out_host, true, &pr);
+  if (s != MOE_OK) return s;
+  if (pr.T == 0) return MOE_OK;
+  const HostLayout hl = host_layout(pr.T, pr.H, pr.I, pr.E, pr.k, w13->gate.dtype);
+  if (!workspace || workspace_bytes < hl.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return MOE_ERR_INVALID_ARG;
+  return forward_host_enqueue(x_host, w13, w2, topk_ids_host, topk_weights_host, out_host, pr, hl,
+                              static_cast<uint8_t*>(workspace), reinterpret_cast<cudaStream_t>(stream));
 }
 
 moe_status_t moe_align(const moe_tensor_t* topk_ids, int64_t E, int32_t block_m, int32_t* counts,

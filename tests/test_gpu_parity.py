@@ -217,6 +217,36 @@ def test_forward_host_matches_device():
     assert torch.equal(out_h, dev.cpu())
 
 
+def test_forward_host_ws_two_calls_in_flight_on_two_streams():
+    # the asynchronous host form: two calls with their own workspaces, host inputs and
+    # outputs, enqueued on two streams before either is waited for, each equal to the
+    # device forward of its own inputs
+    T, H, I, E, k = 300, 512, 384, 8, 4
+    cases = [make_case(T, H, I, E, k, seed=s) for s in (71, 72)]
+    w13, w2 = cases[0]["w13"].cuda(), cases[0]["w2"].cuda()  # shared weights
+    v = moe.w13_from_packed(w13)
+    devs = [run_gpu(dict(to_cuda(cs), w13=w13, w2=w2)) for cs in cases]
+    nbytes = moe.host_workspace_bytes(T, H, I, E, k)
+    assert nbytes >= moe.workspace_bytes(T, H, I, E, k) + 2 * T * H * 2
+    streams = [torch.cuda.Stream() for _ in cases]
+    wss = [torch.empty(nbytes, dtype=torch.uint8, device="cuda") for _ in cases]
+    hosts = [{n: cs[n].contiguous().pin_memory() for n in ("x", "ids", "wts")} for cs in cases]
+    outs = [torch.empty(T, H, dtype=torch.bfloat16).pin_memory() for _ in cases]
+    torch.cuda.synchronize()
+    for i in range(2):
+        h = hosts[i]
+        moe.forward_host(h["x"], v, w2, h["ids"], h["wts"], outs[i], workspace=wss[i], stream=streams[i])
+    for st in streams:
+        st.synchronize()
+    for i in range(2):
+        assert torch.equal(outs[i], devs[i].cpu())
+    small = torch.empty(nbytes - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(moe.MoeError) as err:
+        h = hosts[0]
+        moe.forward_host(h["x"], v, w2, h["ids"], h["wts"], outs[0], workspace=small)
+    assert err.value.status == 5  # MOE_ERR_WORKSPACE_TOO_SMALL
+
+
 @pytest.mark.parametrize("T,H,I,E,k", [
     (37, 288, 96, 6, 3),       # one-CTA kernels, padded 32-row granules
     (300, 512, 384, 4, 2),     # CTA pairs
