@@ -160,7 +160,8 @@ moe_status_t moe_forward_host(const moe_tensor_t* x_host, const moe_w13_t* w13,
  * weights and out.  Returns 0 for invalid arguments. */
 size_t moe_host_workspace_bytes(int64_t T, int64_t H, int64_t I, int64_t E, int64_t k, int32_t wdtype);
 
-/* moe_forward_host without the wait: enqueues on `stream` the copies of x, topk_ids and
+/* moe_forward_host without the wait (the operation of moe_forward, Liger-Kernel PR #1377,
+ * "Problems", with host activations): enqueues on `stream` the copies of x, topk_ids and
  * topk_weights (HOST tensors, inner stride 1) into `workspace` (device, at least
  * moe_host_workspace_bytes(...), 256-byte aligned), the forward, and the copy of the
  * result into out_host, then returns.  out_host holds the result once `stream` has

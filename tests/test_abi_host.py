@@ -84,6 +84,31 @@ def test_workspace_independent_of_weight_size_and_layout():
     assert moe.load().moe_workspace_bytes(4, 64, 64, 4, 2, 9) == 0
 
 
+def test_host_workspace_holds_the_forward_workspace_and_the_staging():
+    # the asynchronous host form stages x, the ids (room for int64), the weights and out
+    # after the forward's own workspace, each region 256-byte aligned
+    T, H, I, E, k = 4096, 4096, 1536, 128, 8
+    for mx in (False, True):
+        core = moe.workspace_bytes(T, H, I, E, k, mxfp4=mx)
+        got = moe.host_workspace_bytes(T, H, I, E, k, mxfp4=mx)
+        staging = T * H * 2 + T * k * 8 + T * k * 4 + T * H * 2
+        assert core + staging <= got <= core + staging + 5 * 256
+        assert got % 256 == 0
+    assert moe.load().moe_host_workspace_bytes(4, 64, 64, 4, 2, 9) == 0
+    assert moe.load().moe_host_workspace_bytes(4, 0, 64, 4, 2, 0) == 0
+
+
+def test_host_forward_rejects_a_small_workspace_before_any_copy():
+    x, w13, w2, ids, wts, out = _cpu_problem()
+    v = moe.w13_from_packed(w13)
+    need = moe.host_workspace_bytes(8, 64, 32, 4, 2)
+    ws = torch.zeros(need - 256, dtype=torch.uint8)  # never touched: the size is checked first
+    with pytest.raises(moe.MoeError) as err:
+        moe.forward_host(x, v, w2, ids, wts, out, workspace=ws, stream=0)
+    assert err.value.status == 5
+    assert moe.last_launch_count() == 0
+
+
 def _cpu_problem(T=8, H=64, I=32, E=4, k=2):
     x = torch.zeros(T, H, dtype=torch.bfloat16)
     w13 = torch.zeros(E, 2 * I, H, dtype=torch.bfloat16)
