@@ -10,7 +10,7 @@
 //              routing weight scales it;
 //   transpose: the expert weights with the contraction axis swapped, so that the
 //              gradient GEMMs read them K-major like the forward does: w2 [E, H, I]
-//              -> [E, I, H] (dh = w * w2^T dout) and the packed w13 [E, 2I, H] ->
+//              -> [E, I, H] (dh' = w2^T dout) and the packed w13 [E, 2I, H] ->
 //              [E, H, 2I] (dx = gate^T dg + up^T du in one contraction over 2I).
 #include "../../include/moe.h"
 #include "moe_internal.h"

@@ -2,15 +2,15 @@
 moe_transpose_experts) against the fp64 oracle gradients (oracle.moe_backward_input,
 oracle.moe_backward_weights).
 
-Tolerance: the CUDA path rounds to bf16 where the oracle keeps fp64: dh, dg and du,
-the recomputed h, the per-slot expert output y (for the routing-weight gradient)
-and the per-slot da rows (for dx), then dx itself.  Each rounding is at most
+Tolerance: the CUDA path rounds to bf16 where the oracle keeps fp64: dh' (w2^T dout,
+before the routing weight), dg' and du', the recomputed h (dh' . h is the routing-weight
+gradient) and the per-slot da rows (for dx), then dx itself.  Each rounding is at most
 2^-9 relative per element and the sums after it run in fp32, so the error
 relative to the largest element stays a few times 2^-9 (~0.2 %) per step; 2e-2
 relative to the largest |dx| (|dweights|) leaves room for four such steps and the
 fp32 accumulation order, while a wrong term, sign or index (the oracle pins'
 failure modes) moves results by O(1).  The weight gradients sum bf16 products of
-the same rounded operands (w dout, h, dg, du, x) in fp32 over an expert's slots,
+the same rounded operands (w dout, h, w dg', w du', x) in fp32 over an expert's slots,
 relative to the largest element of each gradient tensor: the same bound.
 """
 
