@@ -1115,7 +1115,6 @@ moe_status_t backward_impl(const moe_tensor_t* x, const moe_w13_t* w13, const mo
     dgu_rows.s1 = 1;
     dgu_rows.dtype = MOE_BF16;
     CUtensorMap mA, mB, mC;
-
     // gradient [E, M, N] stored by TMA in 32-row tiles of 128-byte rows (fp32 or bf16)
     auto cmap = [&](CUtensorMap* m, const moe_tensor_t* t, int64_t M, int64_t N) {
       const bool b16 = t->dtype == MOE_BF16;
